@@ -1,0 +1,86 @@
+/*
+ * kld_oracle.h -- plain fp64 CPU oracle for the logit KL-divergence statistic.
+ *
+ * TEST INFRASTRUCTURE ONLY. Nothing in the product library includes, links or
+ * calls this file; only the tests, the smoke check and the benchmark's CPU
+ * baseline leg do. It shares no header, constant or helper with the CUDA path.
+ *
+ * What it computes (per row i of two [N, V] logit tensors, base b and quant q):
+ *   - log-softmax of both rows over the full vocabulary,
+ *   - KL(P_base || P_quant) in nats,
+ *   - argmax of each row, lowest index on ties ("Same Top P"),
+ *   - optionally NLL_i = -log P_quant(tok_i),
+ * and over all rows: mean / median / p90 / p99 / max KLD, top-1 agreement
+ * count and percentage, mean NLL and PPL = exp(mean NLL).
+ *
+ * Sources:
+ *   "Qwen3.6 27B Quantization Benchmark" (huy.rocks), sections "Measurement
+ *     method", "Understand KLD and Same Top P" and the "Raw benchmark data"
+ *     table (columns Mean PPL(Q), Mean KLD, Same top p).
+ *   "Mistral-Small-4-119B-2603 GSQ-RCO IQ3_S GGUF" model card, "Quality" and
+ *     "How it was made" steps 5 and 7: the direction is KL(BF16 || quantized)
+ *     over the full vocabulary.
+ *   Percentiles (median/p90/p99) are not printed on any page; they follow the
+ *   linear-interpolation ("type 7") order-statistic rule stated below.
+ */
+#ifndef KLD_ORACLE_H
+#define KLD_ORACLE_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Element type of the logit tensors. */
+enum { ORACLE_F32 = 0, ORACLE_BF16 = 1, ORACLE_F16 = 2 };
+
+/* Per-row flag bits (same meaning and values as the product library states). */
+enum {
+  ORACLE_ROW_NONFINITE = 1u << 0, /* a NaN or +inf in either row: row excluded */
+  ORACLE_ROW_EMPTY     = 1u << 1, /* every entry of a row is -inf: row excluded */
+  ORACLE_ROW_INF_KL    = 1u << 2, /* b_j finite where q_j = -inf: KL = +inf   */
+  ORACLE_ROW_BAD_TOKEN = 1u << 3, /* token id outside [0, V): no NLL for row  */
+  ORACLE_ROW_INF_NLL   = 1u << 4  /* q[tok] = -inf: NLL = +inf                 */
+};
+
+typedef struct {
+  int64_t n_rows;     /* rows given                                         */
+  int64_t n_valid;    /* rows without NONFINITE / EMPTY                     */
+  double mean_kld;    /* left-to-right sum over valid rows / n_valid        */
+  double median_kld;  /* type-7 percentiles of the valid KL values          */
+  double p90_kld;
+  double p99_kld;
+  double max_kld;
+  int64_t top1_agree; /* valid rows with argmax_base == argmax_quant        */
+  double top1_agree_pct;
+  int32_t has_nll;
+  int32_t _pad;
+  int64_t n_nll;      /* valid rows with an in-range token id               */
+  double mean_nll;
+  double ppl;
+  int64_t n_flagged;  /* rows with any flag set                             */
+  uint32_t flags_or;  /* OR of all row flags                                */
+  uint32_t _pad2;
+} oracle_result_t;
+
+/* Per-row statistics of rows [0, N). `tok` may be NULL (no NLL). Rows are
+ * independent; nthreads > 1 spreads whole rows over std::threads, which
+ * leaves every per-row value bit-identical. Returns 0, or -1 on bad args. */
+int oracle_rows(const void* base, const void* quant, const int32_t* tok,
+                int64_t N, int64_t V, int dtype, double* kld, double* nll,
+                int32_t* amax_b, int32_t* amax_q, uint32_t* flags,
+                int nthreads);
+
+/* Reduction of per-row values to the summary statistics. */
+int oracle_reduce(const double* kld, const double* nll, const int32_t* amax_b,
+                  const int32_t* amax_q, const uint32_t* flags, int64_t N,
+                  int has_nll, oracle_result_t* out);
+
+/* Type-7 percentile of an ascending array x[0..n): pos = p*(n-1). */
+double oracle_percentile_sorted(const double* x, int64_t n, double p);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* KLD_ORACLE_H */

@@ -1,0 +1,75 @@
+"""The oracle's pins must catch plausible mistakes.
+
+Each case compiles a copy of the oracle with one planted mistake (on the CPU,
+into a temporary directory) and runs the pin suite against it through
+``KLD_ORACLE_LIB``; the suite has to fail for every mutant.
+"""
+import os
+import subprocess
+import sys
+import tempfile
+
+import pytest
+
+import oracle
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+SRC = os.path.join(ROOT, "oracle", "kld_oracle.cpp")
+
+MUTANTS = {
+    "kl_direction_swapped": ("kl += std::exp(logp) * (logp - logr);",
+                             "kl += std::exp(logr) * (logr - logp);"),
+    "kl_sign_flipped": ("kl += std::exp(logp) * (logp - logr);",
+                        "kl += std::exp(logp) * (logr - logp);"),
+    "log_softmax_drops_normaliser": ("const double logp = b[j] - lse_b;",
+                                     "const double logp = b[j] - m_b;"),
+    "quant_normaliser_from_base": ("const double logr = q[j] - lse_q;",
+                                   "const double logr = q[j] - lse_b;"),
+    "last_vocab_entry_dropped": ("for (int64_t j = 0; j < V; ++j) s_b += std::exp(b[j] - m_b);",
+                                 "for (int64_t j = 0; j + 1 < V; ++j) s_b += std::exp(b[j] - m_b);"),
+    "argmax_ties_to_highest": ("if (amax_b < 0 && b[j] == m_b) amax_b = (int32_t)j;",
+                               "if (b[j] == m_b) amax_b = (int32_t)j;"),
+    "percentile_position_off": ("const double pos = p * (double)(n - 1);",
+                                "const double pos = p * (double)n;"),
+    "nll_sign_flipped": ("*nll = lse_q - q[tok];", "*nll = q[tok] - lse_q;"),
+    "nll_under_base_row": ("*nll = lse_q - q[tok];", "*nll = lse_b - b[tok];"),
+    "excluded_rows_enter_mean": ("if (f & (ORACLE_ROW_NONFINITE | ORACLE_ROW_EMPTY)) continue;",
+                                 "if (f & ORACLE_ROW_NONFINITE) continue;"),
+    "masked_quant_entry_ignored": ("      inf_kl = true;\n      continue;", "      continue;"),
+    "bf16_widening_wrong": ("uint32_t u = (uint32_t)h << 16;", "uint32_t u = (uint32_t)h << 15;"),
+    "agreement_counts_all_rows": ("if (amax_b[i] == amax_q[i]) ++agree;", "++agree;"),
+}
+
+
+@pytest.fixture(scope="module")
+def mutant_dir():
+    with tempfile.TemporaryDirectory() as d:
+        yield d
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_pins_reject_mutant(name, mutant_dir):
+    old, new = MUTANTS[name]
+    src = open(SRC).read()
+    assert src.count(old) == 1, f"mutation site not unique/present: {name}"
+    msrc = os.path.join(mutant_dir, f"{name}.cpp")
+    with open(msrc, "w") as f:
+        f.write(src.replace(old, new))
+    lib = os.path.join(mutant_dir, f"{name}.so")
+    subprocess.run(["g++", "-O2", "-std=c++17", "-fPIC", "-shared", "-pthread",
+                    "-I", os.path.join(ROOT, "oracle"), "-o", lib, msrc], check=True)
+    env = dict(os.environ, KLD_ORACLE_LIB=lib)
+    proc = subprocess.run(
+        [sys.executable, "-m", "pytest", "-q", "-x", "-p", "no:cacheprovider",
+         os.path.join(ROOT, "tests", "test_oracle_pins.py")],
+        cwd=ROOT, env=env, capture_output=True, text=True, timeout=300)
+    assert proc.returncode != 0, f"pins did not catch mutant {name}:\n{proc.stdout[-2000:]}"
+
+
+def test_unmutated_oracle_passes_the_same_way():
+    oracle.build()
+    proc = subprocess.run(
+        [sys.executable, "-m", "pytest", "-q", "-x", "-p", "no:cacheprovider",
+         os.path.join(ROOT, "tests", "test_oracle_pins.py")],
+        cwd=ROOT, capture_output=True, text=True, timeout=300)
+    assert proc.returncode == 0, proc.stdout[-2000:]

@@ -1,0 +1,392 @@
+"""Pins of the fp64 CPU oracle against facts that do not come from the oracle.
+
+Each check uses something independent of the oracle's code path: a closed
+form, an invariant of KL divergence, a brute-force evaluation of the textbook
+formula sum p*log(p/r) in Python (no max subtraction, no log-softmax), the
+worked example printed in "Qwen3.6 27B Quantization Benchmark" (section
+"Understand KLD and Same Top P"), or a library routine (numpy argmax,
+numpy.percentile, math.fsum, numpy's float16 widening).
+"""
+import json
+import math
+import os
+from decimal import Decimal, getcontext
+
+import numpy as np
+import pytest
+
+import oracle
+
+RNG = np.random.default_rng(12345)
+NEG_INF = np.float32(-np.inf)
+
+
+def _run(b, q, tok=None, dtype=oracle.F32, nthreads=1):
+    return oracle.run(b, q, tok, dtype, nthreads)
+
+
+def _brute_kl(b_row, q_row):
+    """sum_j p_j log(p_j / r_j) with p, r from exp(x) / sum exp(x) directly."""
+    eb = [math.exp(float(x)) for x in b_row]
+    eq = [math.exp(float(x)) for x in q_row]
+    sb, sq = math.fsum(eb), math.fsum(eq)
+    terms = []
+    for x, y in zip(eb, eq):
+        p, r = x / sb, y / sq
+        if p > 0:
+            terms.append(p * math.log(p / r))
+    return math.fsum(terms)
+
+
+# ---------------------------------------------------------------- KL basics
+
+@pytest.mark.parametrize("V", [1, 2, 7, 33, 1000, 32000])
+def test_kl_of_identical_rows_is_exactly_zero(V):
+    b = RNG.normal(0, 2.5, size=(6, V)).astype(np.float32)
+    r, res = _run(b, b.copy())
+    assert np.all(r["kld"] == 0.0)
+    assert np.array_equal(r["amax_b"], r["amax_q"])
+    assert res["top1_agree"] == 6 and res["top1_agree_pct"] == 100.0
+    assert res["mean_kld"] == 0.0 and res["max_kld"] == 0.0
+
+
+def test_kl_is_nonnegative():
+    b = RNG.normal(0, 2.5, size=(200, 257)).astype(np.float32)
+    q = (b + RNG.normal(0, 0.5, size=b.shape)).astype(np.float32)
+    r, _ = _run(b, q)
+    assert np.all(r["kld"] >= 0.0)
+    assert np.all(r["kld"] > 0.0)  # noise makes every row differ
+
+
+@pytest.mark.parametrize("shift_b,shift_q", [(4.0, 0.0), (0.0, -8.0), (2.0, 512.0)])
+def test_kl_invariant_to_adding_a_constant(shift_b, shift_q):
+    # values on a 2^-10 grid with |x| < 2^12: adding these constants is exact
+    b = (np.round(RNG.normal(0, 2.5, size=(8, 513)) * 1024) / 1024).astype(np.float32)
+    q = (np.round((b + RNG.normal(0, 0.3, size=b.shape)) * 1024) / 1024).astype(np.float32)
+    b2 = (b + np.float32(shift_b)).astype(np.float32)
+    q2 = (q + np.float32(shift_q)).astype(np.float32)
+    assert np.array_equal(b2.astype(np.float64) - shift_b, b.astype(np.float64))
+    r1, _ = _run(b, q)
+    r2, _ = _run(b2, q2)
+    np.testing.assert_allclose(r2["kld"], r1["kld"], rtol=1e-11, atol=1e-13)
+    assert np.array_equal(r1["amax_b"], r2["amax_b"])
+    assert np.array_equal(r1["amax_q"], r2["amax_q"])
+
+
+def test_kl_invariant_to_common_vocab_permutation():
+    b = RNG.normal(0, 2.5, size=(10, 999)).astype(np.float32)
+    q = (b + RNG.normal(0, 0.4, size=b.shape)).astype(np.float32)
+    perm = RNG.permutation(999)
+    r1, _ = _run(b, q)
+    r2, _ = _run(np.ascontiguousarray(b[:, perm]), np.ascontiguousarray(q[:, perm]))
+    np.testing.assert_allclose(r2["kld"], r1["kld"], rtol=1e-11, atol=1e-14)
+    # argmax moves with the permutation (random data: no ties)
+    assert np.array_equal(perm[r2["amax_b"]], r1["amax_b"])
+    assert np.array_equal(perm[r2["amax_q"]], r1["amax_q"])
+
+
+def test_kl_direction_is_base_first():
+    # P = base, R = quant; swapping the operands changes the value
+    b = np.array([[0.0, -1.0, -3.0]], np.float32)
+    q = np.array([[-2.0, 0.5, 0.0]], np.float32)
+    r_bq, _ = _run(b, q)
+    r_qb, _ = _run(q, b)
+    assert abs(r_bq["kld"][0] - _brute_kl(b[0], q[0])) < 1e-14
+    assert abs(r_qb["kld"][0] - _brute_kl(q[0], b[0])) < 1e-14
+    assert abs(r_bq["kld"][0] - r_qb["kld"][0]) > 1e-3
+
+
+# ---------------------------------------------------------------- closed forms
+
+@pytest.mark.parametrize("V", [1, 2, 5, 32000, 151936])
+def test_one_hot_base_against_uniform_quant_is_log_V(V):
+    hot = V // 3
+    b = np.full((1, V), NEG_INF, np.float32)
+    b[0, hot] = 1.25
+    q = np.zeros((1, V), np.float32)
+    r, _ = _run(b, q)
+    assert abs(r["kld"][0] - math.log(V)) <= 1e-12 * max(1.0, math.log(V))
+    assert r["amax_b"][0] == hot
+    assert r["amax_q"][0] == 0  # all equal: lowest index wins
+    assert r["flags"][0] == 0
+
+
+def test_uniform_base_against_one_hot_quant_is_infinite():
+    V = 16
+    b = np.zeros((1, V), np.float32)
+    q = np.full((1, V), NEG_INF, np.float32)
+    q[0, 3] = 0.0
+    r, res = _run(b, q)
+    assert r["kld"][0] == math.inf
+    assert r["flags"][0] == oracle.ROW_INF_KL
+    assert res["n_valid"] == 1 and res["mean_kld"] == math.inf
+
+
+@pytest.mark.parametrize("b0,b1,q0,q1", [
+    (0.0, 0.0, 0.0, 1.0), (0.3, -1.7, 2.0, 0.5), (-4.0, 4.0, 1.0, -1.0),
+    (10.0, 9.5, 10.0, 10.5), (100.0, 101.0, -50.0, -49.0),
+])
+def test_two_token_rows_match_bernoulli_closed_form(b0, b1, q0, q1):
+    b = np.array([[b0, b1]], np.float32)
+    q = np.array([[q0, q1]], np.float32)
+    x0, x1, y0, y1 = (float(v) for v in (b[0, 0], b[0, 1], q[0, 0], q[0, 1]))
+    p = 1.0 / (1.0 + math.exp(x0 - x1))  # sigmoid(b1 - b0) = P_base(token 1)
+    s = 1.0 / (1.0 + math.exp(y0 - y1))
+    want = p * math.log(p / s) + (1 - p) * math.log((1 - p) / (1 - s))
+    r, _ = _run(b, q)
+    assert abs(r["kld"][0] - want) <= 1e-12 * max(1.0, abs(want))
+
+
+def test_small_vocab_brute_force():
+    for V in range(1, 9):
+        b = RNG.normal(0, 2.0, size=(40, V)).astype(np.float32)
+        q = (b + RNG.normal(0, 1.0, size=b.shape)).astype(np.float32)
+        r, _ = _run(b, q)
+        for i in range(40):
+            want = _brute_kl(b[i], q[i])
+            assert abs(r["kld"][i] - want) <= 1e-13 + 1e-11 * want, (V, i)
+            assert r["amax_b"][i] == int(np.argmax(b[i]))
+            assert r["amax_q"][i] == int(np.argmax(q[i]))
+
+
+def test_second_order_expansion_for_small_perturbations():
+    # KL(softmax(b) || softmax(b + e)) = Var_p(e) / 2 + O(|e|^3)
+    V = 20000
+    b = RNG.normal(0, 2.0, size=(4, V)).astype(np.float32)
+    q = (b + RNG.normal(0, 2e-3, size=b.shape)).astype(np.float32)
+    r, _ = _run(b, q)
+    for i in range(4):
+        x = b[i].astype(np.float64)
+        e = q[i].astype(np.float64) - x  # exact perturbation of the stored values
+        p = np.exp(x - x.max())
+        p /= p.sum()
+        mean_e = np.dot(p, e)
+        half_var = 0.5 * np.dot(p, (e - mean_e) ** 2)
+        assert abs(r["kld"][i] - half_var) <= 2e-2 * half_var
+
+
+# ---------------------------------------------------------------- worked example
+
+def _homework_case(golden_dir, key):
+    with open(os.path.join(golden_dir, "worked_example_homework.json")) as f:
+        case = json.load(f)[key]
+    return case
+
+
+def test_page_worked_example_renormalised(golden_dir):
+    case = _homework_case(golden_dir, "renormalised")
+    pb = [Decimal(x) / Decimal(100) for x in case["base_percent"]]
+    pq = [Decimal(x) / Decimal(100) for x in case["quant_percent"]]
+    getcontext().prec = 50
+    zb, zq = sum(pb), sum(pq)
+    want = sum((x / zb) * ((x / zb) / (y / zq)).ln() for x, y in zip(pb, pq))
+    b = np.array([[math.log(float(x)) for x in pb]], np.float32)
+    q = np.array([[math.log(float(y)) for y in pq]], np.float32)
+    # the logits are fp32-rounded logs, so compare with the stored values too
+    r, res = _run(b, q)
+    assert abs(r["kld"][0] - _brute_kl(b[0], q[0])) < 1e-14
+    assert abs(r["kld"][0] - float(want)) < 1e-6  # fp32 rounding of the logs
+    # by hand: p = (.9375, .052083, .010417), r = (.5, .3, .2);
+    # .9375 ln 1.875 + .052083 ln .17361 + .010417 ln .052083
+    # = .589321 - .091195 - .030780 = .467346
+    assert abs(float(want) - 0.467346) < 2e-6
+    assert r["amax_b"][0] == case["top_index"] == r["amax_q"][0]
+    assert res["top1_agree_pct"] == 100.0
+
+
+def test_page_worked_example_with_residual_mass(golden_dir):
+    case = _homework_case(golden_dir, "residual")
+    b = np.array([[math.log(x / 100) if x > 0 else -np.inf
+                   for x in case["base_percent"]]], np.float32)
+    q = np.array([[math.log(x / 100) if x > 0 else -np.inf
+                   for x in case["quant_percent"]]], np.float32)
+    r, _ = _run(b, q)
+    assert r["kld"][0] == math.inf
+    assert r["flags"][0] & oracle.ROW_INF_KL
+    assert r["amax_b"][0] == r["amax_q"][0] == case["top_index"]
+
+
+# ---------------------------------------------------------------- NLL / PPL
+
+@pytest.mark.parametrize("V", [3, 1000, 151936])
+def test_uniform_quant_gives_nll_log_V_and_ppl_V(V):
+    b = RNG.normal(0, 1, size=(5, V)).astype(np.float32)
+    q = np.full((5, V), -3.5, np.float32)
+    tok = RNG.integers(0, V, size=5).astype(np.int32)
+    r, res = _run(b, q, tok)
+    np.testing.assert_allclose(r["nll"], math.log(V), rtol=1e-13)
+    assert abs(res["ppl"] - V) <= 1e-10 * V
+
+
+def test_one_hot_quant_nll():
+    V = 64
+    b = RNG.normal(0, 1, size=(2, V)).astype(np.float32)
+    q = np.full((2, V), NEG_INF, np.float32)
+    q[:, 9] = 2.0
+    tok = np.array([9, 10], np.int32)
+    r, res = _run(b, q, tok)
+    assert r["nll"][0] == 0.0
+    assert r["nll"][1] == math.inf and r["flags"][1] & oracle.ROW_INF_NLL
+    assert res["ppl"] == math.inf
+
+
+def test_nll_matches_brute_force_log_prob():
+    V = 7
+    b = RNG.normal(0, 1, size=(30, V)).astype(np.float32)
+    q = RNG.normal(0, 2, size=(30, V)).astype(np.float32)
+    tok = RNG.integers(0, V, size=30).astype(np.int32)
+    r, res = _run(b, q, tok)
+    want = []
+    for i in range(30):
+        e = [math.exp(float(x)) for x in q[i]]
+        want.append(-math.log(e[tok[i]] / math.fsum(e)))
+    np.testing.assert_allclose(r["nll"], want, rtol=1e-13)
+    assert abs(res["mean_nll"] - math.fsum(want) / 30) < 1e-13
+    assert abs(res["ppl"] - math.exp(math.fsum(want) / 30)) < 1e-12 * res["ppl"]
+
+
+def test_bad_token_ids_are_flagged_and_excluded_from_ppl():
+    V = 10
+    b = RNG.normal(0, 1, size=(4, V)).astype(np.float32)
+    q = RNG.normal(0, 1, size=(4, V)).astype(np.float32)
+    tok = np.array([0, -1, V, 3], np.int32)
+    r, res = _run(b, q, tok)
+    assert list(r["flags"] & oracle.ROW_BAD_TOKEN) == [0, oracle.ROW_BAD_TOKEN,
+                                                       oracle.ROW_BAD_TOKEN, 0]
+    assert res["n_nll"] == 2 and res["n_valid"] == 4
+    assert abs(res["mean_nll"] - (r["nll"][0] + r["nll"][3]) / 2) < 1e-15
+
+
+# ---------------------------------------------------------------- argmax / ties
+
+def test_argmax_ties_go_to_lowest_index():
+    V = 50
+    b = RNG.normal(0, 1, size=(20, V)).astype(np.float32)
+    q = b.copy()
+    for i in range(20):
+        idx = np.sort(RNG.choice(V, size=2 + i % 7, replace=False))
+        b[i, idx] = 9.0
+        q[i, idx[::-1][: max(2, len(idx) - 1)]] = 9.5
+    r, _ = _run(b, q)
+    for i in range(20):
+        assert r["amax_b"][i] == int(np.argmax(b[i]))  # numpy: first occurrence
+        assert r["amax_q"][i] == int(np.argmax(q[i]))
+
+
+def test_same_top_p_counts_index_agreement():
+    b = np.array([[0, 5, 5], [1, 0, 0], [0, 0, 2]], np.float32)
+    q = np.array([[0, 5, 5], [0, 1, 0], [0, 0, 3]], np.float32)
+    r, res = _run(b, q)
+    assert list(r["amax_b"]) == [1, 0, 2] and list(r["amax_q"]) == [1, 1, 2]
+    assert res["top1_agree"] == 2
+    assert abs(res["top1_agree_pct"] - 200.0 / 3) < 1e-12
+
+
+# ---------------------------------------------------------------- reductions
+
+def test_percentiles_hand_values():
+    x = np.array([1.0, 2.0, 3.0, 4.0, 5.0])
+    assert oracle.percentile_sorted(x, 0.5) == 3.0
+    assert abs(oracle.percentile_sorted(x, 0.9) - 4.6) < 1e-15
+    assert abs(oracle.percentile_sorted(x, 0.99) - 4.96) < 1e-15
+    assert oracle.percentile_sorted(np.array([1.0, 2.0]), 0.5) == 1.5
+    assert oracle.percentile_sorted(np.array([7.0]), 0.99) == 7.0
+
+
+@pytest.mark.parametrize("n", [1, 2, 3, 10, 101, 4096, 32768])
+def test_percentiles_match_numpy_linear(n):
+    x = np.sort(RNG.gamma(0.5, 0.1, size=n))
+    for p in (0.5, 0.9, 0.99):
+        want = np.percentile(x, 100 * p, method="linear")
+        got = oracle.percentile_sorted(x, p)
+        assert abs(got - want) <= 1e-15 * max(1.0, abs(want)) + 1e-300
+
+
+def test_reduction_against_library_sums():
+    b = RNG.normal(0, 2.5, size=(301, 211)).astype(np.float32)
+    q = (b + RNG.normal(0, 0.3, size=b.shape)).astype(np.float32)
+    tok = RNG.integers(0, 211, size=301).astype(np.int32)
+    r, res = _run(b, q, tok)
+    assert abs(res["mean_kld"] - math.fsum(r["kld"]) / 301) <= 1e-13 * res["mean_kld"]
+    want_nll = math.fsum(r["nll"]) / 301
+    assert abs(res["mean_nll"] - want_nll) <= 1e-13 * want_nll
+    srt = np.sort(r["kld"])
+    assert res["median_kld"] == np.percentile(srt, 50, method="linear")
+    assert abs(res["p99_kld"] - np.percentile(srt, 99, method="linear")) <= 1e-15
+    assert res["max_kld"] == srt[-1]
+    assert res["top1_agree"] == int(np.sum(r["amax_b"] == r["amax_q"]))
+
+
+# ---------------------------------------------------------------- flags
+
+def test_nonfinite_and_empty_rows_are_flagged_and_excluded():
+    V = 12
+    b = RNG.normal(0, 1, size=(6, V)).astype(np.float32)
+    q = (b + 0.1).astype(np.float32)
+    b[1, 3] = np.nan
+    q[2, 5] = np.inf
+    b[3, :] = -np.inf
+    q[4, :] = -np.inf
+    r, res = _run(b, q)
+    fl = list(r["flags"])
+    assert fl[0] == 0 and fl[5] == 0
+    assert fl[1] == oracle.ROW_NONFINITE and fl[2] == oracle.ROW_NONFINITE
+    assert fl[3] == oracle.ROW_EMPTY and fl[4] == oracle.ROW_EMPTY
+    for i in (1, 2, 3, 4):
+        assert math.isnan(r["kld"][i]) and r["amax_b"][i] == -1 and r["amax_q"][i] == -1
+    assert res["n_valid"] == 2 and res["n_flagged"] == 4
+    assert abs(res["mean_kld"] - (r["kld"][0] + r["kld"][5]) / 2) < 1e-15
+
+
+def test_masked_vocab_entries_contribute_nothing():
+    # -inf in both rows on the same entries == dropping those entries
+    V = 300
+    b = RNG.normal(0, 2, size=(5, V)).astype(np.float32)
+    q = (b + RNG.normal(0, 0.3, size=b.shape)).astype(np.float32)
+    bm, qm = b.copy(), q.copy()
+    bm[:, -37:] = -np.inf
+    qm[:, -37:] = -np.inf
+    r1, _ = _run(bm, qm)
+    r2, _ = _run(np.ascontiguousarray(b[:, :-37]), np.ascontiguousarray(q[:, :-37]))
+    np.testing.assert_allclose(r1["kld"], r2["kld"], rtol=1e-14, atol=0)
+    assert np.all(r1["flags"] == 0)
+
+
+# ---------------------------------------------------------------- dtypes, threads
+
+def test_bf16_input_equals_widened_fp32_input():
+    b32 = RNG.normal(0, 2.5, size=(9, 515)).astype(np.float32)
+    q32 = (b32 + RNG.normal(0, 0.2, size=b32.shape)).astype(np.float32)
+    # round to bf16 by keeping the top 16 bits with round-to-nearest-even
+    def to_bf16_bits(x):
+        u = x.view(np.uint32).astype(np.uint64)
+        u = (u + 0x7FFF + ((u >> 16) & 1)) >> 16
+        return u.astype(np.uint16)
+    bb, qb = to_bf16_bits(b32), to_bf16_bits(q32)
+    bw = (bb.astype(np.uint32) << 16).view(np.float32)
+    qw = (qb.astype(np.uint32) << 16).view(np.float32)
+    r16, s16 = _run(bb, qb, dtype=oracle.BF16)
+    r32, s32 = _run(bw, qw, dtype=oracle.F32)
+    for k in ("kld", "amax_b", "amax_q", "flags"):
+        assert np.array_equal(r16[k], r32[k])
+
+
+def test_f16_input_equals_numpy_widening():
+    x = RNG.normal(0, 3, size=(7, 333)).astype(np.float16)
+    x[0, :20] = np.array([6e-8, -6e-8, 1e-5, 65504, -65504] * 4, np.float16)
+    y = (x.astype(np.float32) + RNG.normal(0, 0.5, size=x.shape)).astype(np.float16)
+    r16, _ = _run(x.view(np.uint16), y.view(np.uint16), dtype=oracle.F16)
+    r32, _ = _run(x.astype(np.float32), y.astype(np.float32), dtype=oracle.F32)
+    for k in ("kld", "amax_b", "amax_q", "flags"):
+        assert np.array_equal(r16[k], r32[k])
+
+
+def test_threaded_rows_are_bit_identical():
+    b = RNG.normal(0, 2.5, size=(37, 1001)).astype(np.float32)
+    q = (b + RNG.normal(0, 0.3, size=b.shape)).astype(np.float32)
+    tok = RNG.integers(0, 1001, size=37).astype(np.int32)
+    r1, s1 = _run(b, q, tok, nthreads=1)
+    r4, s4 = _run(b, q, tok, nthreads=4)
+    for k in r1:
+        assert np.array_equal(r1[k], r4[k])
+    assert s1 == s4
