@@ -1,0 +1,373 @@
+"""Benchmark of the KLD statistic on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+A step is one pass of the whole statistic over one batch: the fused row pass
+(log-softmax of both rows, KL, argmaxes, NLL) over every row, then the
+fixed-order reduction and exact percentile selection, then the result copied
+to the host. The batch is one 8192-token context at a vocabulary of 151936
+(fp32 logits, 2 x 4.98 GB per GPU), generated on the device by the seeded
+generator; it is far larger than L2, so no L2 flush is needed between steps.
+
+With N GPUs (torchrun, one rank per GPU) every rank scores its own context
+(weak scaling); the per-row records are all-gathered over NCCL and every
+rank reduces the full set, since exact percentiles need all rows.
+
+Prints one JSON line (rank 0).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import shutil
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "logit rows/s and HBM GB/s (fraction of B200 peak) for KLD+top-1 at V=151936"
+WORKLOAD = "ctx8192_v151936_f32"
+VARIANT = "ctx8192_v151936_bf16"
+FALLBACK_HBM_GBS = 6650.0
+RESULT_BYTES = 120  # sizeof(kld_result_t)
+ROW_RECORD_BYTES = 32
+
+
+def _env_int(name, default):
+    try:
+        return int(os.environ.get(name, default))
+    except ValueError:
+        return default
+
+
+def measured_peak():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for name in ("kld_rows.cu", "kld_internal.h"):
+        with open(os.path.join(ROOT, "logit_kl_divergence_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken
+    on the current row-kernel source; else None."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        e = d.get(workload)
+        if e and e.get("kernel_source_hash") == kernel_source_hash():
+            return float(e["dram_bytes_per_launch"])
+    except Exception:
+        pass
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.proc = None
+        self.gpu = gpu_index
+        exe = shutil.which("nvidia-smi")
+        if exe:
+            self.proc = subprocess.Popen(
+                [exe, f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "100",
+                 "-i", str(gpu_index)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def cpu_baseline(name: str, budget_s: float = 12.0, max_rows: int = 4096):
+    """The oracle, as it stands, single-threaded, on a bounded sample of rows
+    of the same workload recipe (generated on the host)."""
+    import oracle
+    from logit_kl_divergence_b200 import synth
+
+    odt = {synth.F32: oracle.F32, synth.BF16: oracle.BF16, synth.F16: oracle.F16}
+    probe = synth.make(name, n=8)
+    t0 = time.perf_counter()
+    oracle.rows(probe.base, probe.quant, probe.token_ids, odt[probe.dtype], 1)
+    per_row = (time.perf_counter() - t0) / 8
+    rows = int(max(8, min(max_rows, budget_s / max(per_row, 1e-6))))
+    w = synth.make(name, n=rows, seed=synth.WORKLOADS[name][4] + 1000)
+    t0 = time.perf_counter()
+    r = oracle.rows(w.base, w.quant, w.token_ids, odt[w.dtype], 1)
+    oracle.reduce(r, True)
+    dt = time.perf_counter() - t0
+    return {"value": rows / dt, "unit": "rows/s", "cores": 1, "kind": "oracle",
+            "sample": f"{rows} rows of {name} (same recipe, host-generated), "
+                      f"fp64 two-pass oracle, single thread, {dt:.1f} s"}
+
+
+def run_reference(args, rank: int):
+    if rank != 0:
+        return
+    from logit_kl_divergence_b200 import synth
+
+    import oracle
+
+    odt = {synth.F32: oracle.F32, synth.BF16: oracle.BF16, synth.F16: oracle.F16}
+    rows = 64
+    samples = [synth.make(WORKLOAD, n=rows, seed=100 + i) for i in range(min(args.steps, 4))]
+    for i in range(args.warmup):
+        w = samples[i % len(samples)]
+        oracle.reduce(oracle.rows(w.base, w.quant, w.token_ids, odt[w.dtype], 1), True)
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        w = samples[i % len(samples)]
+        oracle.reduce(oracle.rows(w.base, w.quant, w.token_ids, odt[w.dtype], 1), True)
+    dt = time.perf_counter() - t0
+    value = rows * args.steps / dt
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "rows/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1000 * dt / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "rows_per_step": rows, "vocab": 151936,
+                   "logit_dtype": "f32", "sample": "64-row sample of the workload per step"},
+        "cpu_baseline": {"value": value, "unit": "rows/s", "cores": 1, "kind": "oracle",
+                         "sample": f"{rows} rows per step of {WORKLOAD}, single-threaded fp64 oracle"},
+        "e2e": {"value": value, "unit": "rows/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-variants", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)
+
+    rank = _env_int("RANK", 0)
+    world = _env_int("WORLD_SIZE", 1)
+    local = _env_int("LOCAL_RANK", 0)
+
+    if args.impl == "reference":
+        run_reference(args, rank)
+        return
+
+    import torch
+    import torch.distributed as dist
+
+    from logit_kl_divergence_b200 import KLDStats, synth
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+
+        dist.init_process_group("nccl", device_id=dev, timeout=datetime.timedelta(seconds=120))
+
+    name = WORKLOAD
+    w = synth.make(name, device=dev, seed=synth.WORKLOADS[name][4] + 7919 * rank)
+    N, V = w.base.shape
+    eb = w.bytes_per_elem
+    in_bytes = 2 * N * V * eb
+    stream = torch.cuda.current_stream(dev)
+
+    st = KLDStats(max_rows=N * world, device=dev)
+    st.set_timing(world == 1)
+    records = None
+    gathered = None
+    if world > 1:
+        records = torch.empty((N, ROW_RECORD_BYTES), dtype=torch.uint8, device=dev)
+        gathered = torch.empty((N * world, ROW_RECORD_BYTES), dtype=torch.uint8, device=dev)
+
+    row_ms = []
+
+    def step(timed: bool):
+        if world == 1:
+            st.run(w.base, w.quant, w.token_ids)
+            res = st.result()
+            if timed:
+                row_ms.append(st.timing()[0])
+        else:
+            st.run_rows(w.base, w.quant, w.token_ids, out=records)
+            dist.all_gather_into_tensor(gathered, records)
+            st.reduce(gathered, N * world, True)
+            res = st.result()
+        return res
+
+    for _ in range(args.warmup):
+        res = step(False)
+
+    # Row-kernel time on its own stream for multi-GPU too (events bracket the
+    # row pass only; used for the roofline).
+    if world > 1:
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+    sampler = ClockSampler(local)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for _ in range(args.steps):
+        if world == 1:
+            res = step(True)
+        else:
+            e0.record(stream)
+            st.run_rows(w.base, w.quant, w.token_ids, out=records)
+            e1.record(stream)
+            dist.all_gather_into_tensor(gathered, records)
+            st.reduce(gathered, N * world, True)
+            res = st.result()
+            row_ms.append(e0.elapsed_time(e1))
+    end.record(stream)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop()
+    ms = start.elapsed_time(end)
+    if world > 1:
+        t = torch.tensor([ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    ms_per_step = ms / args.steps
+    total_rows = N * world
+    value = total_rows / (ms_per_step / 1000.0)
+
+    peak, peak_kind = measured_peak()
+    avg_row_ms = sum(row_ms) / len(row_ms)
+    achieved = in_bytes / (avg_row_ms / 1000.0) / 1e9
+    traffic = recorded_traffic(name)
+    roofline = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                "frac": achieved / peak, "traffic": traffic,
+                "peak_source": f"{peak_kind} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)",
+                "frac_of_8TBs_nominal": achieved / 8000.0,
+                "kernel": "kld_rows_kernel<f32>", "row_pass_ms": avg_row_ms,
+                "algorithmic_bytes_per_launch": in_bytes}
+
+    # bf16 variant of the same context (the target names both dtypes).
+    variants = {}
+    if world == 1 and not args.no_variants:
+        del w
+        torch.cuda.empty_cache()
+        wb = synth.make(VARIANT, device=dev)
+        for _ in range(3):
+            st.run(wb.base, wb.quant, wb.token_ids)
+            st.result()
+        torch.cuda.synchronize(dev)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        rms = []
+        a.record(stream)
+        for _ in range(args.steps):
+            st.run(wb.base, wb.quant, wb.token_ids)
+            st.result()
+            rms.append(st.timing()[0])
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        vb_bytes = 2 * wb.base.numel() * wb.bytes_per_elem
+        vms = a.elapsed_time(b) / args.steps
+        rrow = sum(rms) / len(rms)
+        variants[VARIANT] = {"value": wb.n / (vms / 1000.0), "unit": "rows/s", "ms_per_step": vms,
+                             "row_pass_ms": rrow, "achieved_gbs": vb_bytes / (rrow / 1000.0) / 1e9,
+                             "frac": vb_bytes / (rrow / 1000.0) / 1e9 / peak}
+        del wb
+        torch.cuda.empty_cache()
+        w = synth.make(name, device=dev, seed=synth.WORKLOADS[name][4])
+
+    # End to end through the public host-memory entry point: pinned host
+    # buffers in, the result struct out, copies inside the timed region.
+    e2e = None
+    if world == 1 and args.e2e_steps > 0:
+        hb = w.base.cpu().pin_memory()
+        hq = w.quant.cpu().pin_memory()
+        ht = w.token_ids.cpu().pin_memory()
+        st.run_host(hb, hq, ht)
+        st.result()
+        torch.cuda.synchronize(dev)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(args.e2e_steps):
+            st.run_host(hb, hq, ht)
+            st.result()
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        ems = a.elapsed_time(b) / args.e2e_steps
+        e2e = {"value": N / (ems / 1000.0), "unit": "rows/s",
+               "h2d_bytes_per_step": in_bytes + 4 * N, "d2h_bytes_per_step": RESULT_BYTES,
+               "ms_per_step": ems, "path": "kld_stats_run_host (pinned host buffers)"}
+        del hb, hq, ht
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(name)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "rows/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": name, "rows_per_gpu": N, "vocab": V, "logit_dtype": "f32",
+                       "global_rows": total_rows,
+                       "parallelism": f"rows sharded over {world} GPU(s), records all-gathered",
+                       "l2": "inputs (9.96 GB per step per GPU) exceed the 126 MB L2; no flush"},
+            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": 2 * args.steps, "clocks": clocks,
+            "gbs": in_bytes * world / (ms_per_step / 1000.0) / 1e9,
+            "mean_kld": res["mean_kld"], "top1_agree_pct": res["top1_agree_pct"], "ppl": res["ppl"],
+            "variants": variants,
+        }
+        print(json.dumps(line), flush=True)
+
+    st.close()
+    if world > 1:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

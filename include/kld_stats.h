@@ -1,0 +1,230 @@
+/*
+ * kld_stats.h -- C ABI of the B200 (sm_100a) logit KL-divergence statistics
+ * library (libkld_stats.so).
+ *
+ * The statistic is the one `llama-perplexity --kl-divergence` prints when a
+ * quantized model is scored against its BF16 base ("Qwen3.6 27B Quantization
+ * Benchmark", sections "Measurement method" and "Understand KLD and Same Top
+ * P", and the "Raw benchmark data" table). For each of N token positions the
+ * library takes a base logit row b and a quantized logit row q over a
+ * vocabulary of V entries and computes, in one pass over HBM:
+ *
+ *   KL_i   = sum_j P_j (log P_j - log R_j),  P = softmax(b), R = softmax(q),
+ *            natural log, over the full vocabulary, base first
+ *            ("Mistral-Small-4-119B-2603 GSQ-RCO IQ3_S GGUF", "How it was
+ *            made", step 5: KL(BF16 || quantized) over the full vocabulary);
+ *   amax_i = argmax_j b_j and argmax_j q_j, lowest index on ties
+ *            ("Same Top P": how often both models pick the same token);
+ *   NLL_i  = -log R_{tok_i} when next-token ids are given (the table's
+ *            "Mean PPL(Q)" column is exp(mean NLL));
+ *
+ * and reduces them over the rows to mean / median / p90 / p99 / max KLD,
+ * the top-1 agreement count and percentage, mean NLL and PPL. Percentiles
+ * interpolate linearly between order statistics at pos = p*(n-1).
+ *
+ * Conventions shared by every call:
+ *   - Logit tensors are row-major [N, V], contiguous, in device memory
+ *     (except kld_stats_run_host), element type kld_dtype_t. Row i of base
+ *     and row i of quant are paired. Both pointers must be aligned to their
+ *     element size and have the same address modulo 16 (true for any two
+ *     tensors from cudaMalloc or the PyTorch allocator).
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream). Work is enqueued asynchronously; inputs must stay valid and
+ *     unchanged until kld_stats_result() returns.
+ *   - Memory passed in is owned by the caller; memory a handle allocates is
+ *     owned by the handle and released by kld_stats_destroy().
+ *   - Errors are reported by return codes only: nothing on the device traps
+ *     or aborts. Arguments are checked before anything is enqueued; errors
+ *     that arise on the device (a bounded wait giving up, rows that must be
+ *     excluded) surface in kld_stats_result().
+ *   - A handle is bound to one device and is not thread-safe; use one handle
+ *     per concurrent stream.
+ *
+ * Row policy (the pages are silent; both this library and its test oracle
+ * follow it):
+ *   - a row holding NaN or +inf in b or q: flag NONFINITE, KL/NLL = NaN,
+ *     argmaxes -1, excluded from every statistic;
+ *   - a row whose b or q entries are all -inf: flag EMPTY, treated the same;
+ *   - entries with b_j = -inf have P_j = 0 and add nothing (padding masks);
+ *     b_j finite with q_j = -inf gives KL = +inf (flag INF_KL, row kept);
+ *   - token id outside [0, V): flag BAD_TOKEN, row left out of NLL/PPL;
+ *     q[tok] = -inf gives NLL = +inf (flag INF_NLL, row kept).
+ */
+#ifndef KLD_STATS_H
+#define KLD_STATS_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define KLD_ABI_VERSION 1
+
+typedef enum {
+  KLD_OK = 0,
+  KLD_ERR_INVALID_ARG = 1, /* null/unaligned pointer, N or V out of range  */
+  KLD_ERR_DTYPE = 2,       /* unknown element type                         */
+  KLD_ERR_OOM = 3,         /* a device or pinned allocation failed          */
+  KLD_ERR_CUDA = 4,        /* a CUDA call failed; see kld_last_cuda_error() */
+  KLD_ERR_NONFINITE = 5,   /* some rows were NONFINITE or EMPTY (excluded);
+                              the statistics of the other rows are valid     */
+  KLD_ERR_BAD_TOKEN = 6,   /* some token ids were outside [0, V); PPL uses
+                              the other rows                                 */
+  KLD_ERR_TIMEOUT = 7,     /* a bounded device-side wait gave up            */
+  KLD_ERR_NO_DEVICE = 8,   /* no usable sm_100 device                       */
+  KLD_ERR_NOT_READY = 9    /* kld_stats_result() before any run             */
+} kld_status_t;
+
+typedef enum { KLD_F32 = 0, KLD_BF16 = 1, KLD_F16 = 2 } kld_dtype_t;
+
+/* Per-row flag bits (kld_row_t.flags). */
+#define KLD_ROW_NONFINITE (1u << 0)
+#define KLD_ROW_EMPTY     (1u << 1)
+#define KLD_ROW_INF_KL    (1u << 2)
+#define KLD_ROW_BAD_TOKEN (1u << 3)
+#define KLD_ROW_INF_NLL   (1u << 4)
+
+/* One 32-byte record per row, written by the row pass. */
+typedef struct {
+  double kld;            /* KL(P_base || P_quant) in nats (NaN if excluded) */
+  double nll;            /* -log P_quant(tok) (NaN if no/bad token)        */
+  int32_t argmax_base;   /* lowest index of the row maximum, -1 if excluded */
+  int32_t argmax_quant;
+  uint32_t flags;        /* KLD_ROW_* bits                                  */
+  uint32_t reserved;
+} kld_row_t;
+
+/* Summary statistics (caller-owned plain struct). */
+typedef struct {
+  int64_t n_rows;        /* rows reduced                                      */
+  int64_t n_valid;       /* rows that are neither NONFINITE nor EMPTY         */
+  double mean_kld;       /* statistics over the valid rows (NaN if none)      */
+  double median_kld;
+  double p90_kld;
+  double p99_kld;
+  double max_kld;
+  int64_t top1_agree;    /* valid rows whose two argmaxes are equal           */
+  double top1_agree_pct; /* 100 * top1_agree / n_valid                        */
+  int32_t has_nll;       /* token ids were given                              */
+  int32_t reserved0;
+  int64_t n_nll;         /* valid rows with an in-range token id              */
+  double mean_nll;
+  double ppl;            /* exp(mean_nll)                                     */
+  int64_t n_flagged;     /* rows with any flag                                */
+  uint32_t flags_or;     /* OR of all row flags                               */
+  uint32_t device_error; /* nonzero if a bounded device wait gave up          */
+} kld_result_t;
+
+typedef struct kld_stats_s* kld_stats_t;
+
+/* ABI version this library was built with (KLD_ABI_VERSION). */
+int kld_abi_version(void);
+
+/* Static description of a status code. Never NULL. */
+const char* kld_status_string(kld_status_t status);
+
+/* Text of the last CUDA error seen by this thread's calls ("" if none). */
+const char* kld_last_cuda_error(void);
+
+/*
+ * Create a handle on `device` for runs of up to `max_rows` rows.
+ * Allocates a device workspace of max_rows records (32 bytes each) plus a few
+ * KB, and a pinned host copy of the result. Returns KLD_ERR_NO_DEVICE if the
+ * device is not a compute-capability 10.0 (B200-class) GPU.
+ */
+kld_status_t kld_stats_create(kld_stats_t* out, int64_t max_rows, int device);
+
+/* Release everything the handle owns. Waits for its pending work. NULL ok. */
+void kld_stats_destroy(kld_stats_t h);
+
+/*
+ * The whole statistic for rows [0, N): the fused row pass, then the
+ * fixed-order reduction and exact percentile selection, then an async copy
+ * of the result to pinned host memory. token_ids (device, int32[N]) may be
+ * NULL: no NLL/PPL. 1 <= N <= max_rows, 1 <= V <= 2^31-1. Asynchronous.
+ */
+kld_status_t kld_stats_run(kld_stats_t h, const void* base, const void* quant,
+                           const int32_t* token_ids, int64_t N, int64_t V,
+                           kld_dtype_t dtype, void* stream);
+
+/*
+ * Wait for the last run/reduce of this handle and copy its statistics to
+ * *out. Returns KLD_OK, or KLD_ERR_NONFINITE / KLD_ERR_BAD_TOKEN (statistics
+ * of the remaining rows still filled in), KLD_ERR_TIMEOUT, KLD_ERR_CUDA.
+ */
+kld_status_t kld_stats_result(kld_stats_t h, kld_result_t* out);
+
+/*
+ * Device pointer to the per-row records of the last kld_stats_run (N of
+ * them, stream-ordered after that run). Valid until the next run or destroy.
+ */
+kld_status_t kld_stats_rows(kld_stats_t h, const kld_row_t** rows_dev,
+                            int64_t* n_rows);
+
+/*
+ * The row pass alone: per-row records for rows [0, N) written to rows_out
+ * (device, N records, caller-owned; NULL = the handle's workspace). This is
+ * the unit a row-sharded multi-GPU run executes on each GPU before the
+ * records are gathered and reduced. Asynchronous.
+ */
+kld_status_t kld_stats_run_rows(kld_stats_t h, const void* base,
+                                const void* quant, const int32_t* token_ids,
+                                int64_t N, int64_t V, kld_dtype_t dtype,
+                                kld_row_t* rows_out, void* stream);
+
+/*
+ * Reduction and percentile selection over N records in device memory
+ * (rows_dev; NULL = the handle's workspace), e.g. the records of all GPUs
+ * after a gather. has_nll: whether token ids were given to the row pass.
+ * N may exceed max_rows. Result through kld_stats_result(). Asynchronous.
+ */
+kld_status_t kld_stats_reduce(kld_stats_t h, const kld_row_t* rows_dev,
+                              int64_t N, int has_nll, void* stream);
+
+/*
+ * kld_stats_run for logits in HOST memory (e.g. logits saved by a base-model
+ * run): rows are copied to the device in chunks on an internal copy stream,
+ * overlapped with the row pass of the previous chunk, then reduced as in
+ * kld_stats_run. Pinned host memory gives full PCIe bandwidth; pageable
+ * memory works but is slower. token_ids is a host pointer or NULL. The first
+ * call allocates two device staging buffers (kept until destroy).
+ */
+kld_status_t kld_stats_run_host(kld_stats_t h, const void* base_host,
+                                const void* quant_host,
+                                const int32_t* token_ids_host, int64_t N,
+                                int64_t V, kld_dtype_t dtype, void* stream);
+
+/*
+ * Kernel timing of the next runs: when enabled, kld_stats_run records CUDA
+ * events around its row pass and its reduction; kld_stats_timing() returns
+ * the last run's durations in milliseconds (waits for that run).
+ */
+kld_status_t kld_stats_set_timing(kld_stats_t h, int enable);
+kld_status_t kld_stats_timing(kld_stats_t h, float* row_pass_ms,
+                              float* reduce_ms);
+
+/*
+ * Launch plan the row pass would use for (N, V, dtype) on this handle's
+ * device: kernel variant (0 = one CTA per row, 1 = split row over a thread-
+ * block cluster), grid size, CTAs per row, threads per CTA, dynamic shared
+ * memory bytes. Pure host logic; enqueues nothing.
+ */
+typedef struct {
+  int32_t variant;
+  int32_t grid;
+  int32_t ctas_per_row;
+  int32_t threads;
+  int32_t smem_bytes;
+  int32_t stage_bytes;
+  int32_t stages;
+  int32_t reserved;
+} kld_plan_t;
+
+kld_status_t kld_plan(int64_t N, int64_t V, kld_dtype_t dtype, int sm_count,
+                      kld_plan_t* out);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* KLD_STATS_H */

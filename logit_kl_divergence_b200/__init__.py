@@ -1,0 +1,204 @@
+"""KL-divergence statistics of quantized vs. base logits on B200 (sm_100a).
+
+Thin Python binding over the C ABI of ``libkld_stats.so`` (``include/
+kld_stats.h``). PyTorch supplies device memory and streams; all arithmetic
+runs in the library's CUDA kernels.
+
+    >>> from logit_kl_divergence_b200 import KLDStats
+    >>> st = KLDStats(max_rows=8192)
+    >>> st.run(base_logits, quant_logits, next_token_ids)   # async on the stream
+    >>> res = st.result()    # mean/median/p90/p99/max KLD, top-1 agreement, PPL
+"""
+from __future__ import annotations
+
+import ctypes
+
+import torch
+
+from . import _lib
+from ._lib import (KLD_BF16, KLD_F16, KLD_F32, ROW_BAD_TOKEN, ROW_EMPTY,  # noqa: F401
+                   ROW_INF_KL, ROW_INF_NLL, ROW_NONFINITE, KLDError)
+
+__all__ = ["KLDStats", "kld_stats", "dtype_code", "ROW_RECORD_BYTES"]
+
+ROW_RECORD_BYTES = 32
+
+_DTYPES = {torch.float32: KLD_F32, torch.bfloat16: KLD_BF16, torch.float16: KLD_F16}
+
+# statuses that still come with valid statistics of the remaining rows
+_SOFT = (_lib.KLD_OK, _lib.KLD_ERR_NONFINITE, _lib.KLD_ERR_BAD_TOKEN)
+
+
+def dtype_code(t: torch.Tensor) -> int:
+    try:
+        return _DTYPES[t.dtype]
+    except KeyError:
+        raise TypeError(f"unsupported logit dtype {t.dtype}") from None
+
+
+def _stream_ptr(stream, device) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    return int(stream.cuda_stream)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _check_pair(base: torch.Tensor, quant: torch.Tensor, token_ids, on_device: bool):
+    if base.dim() != 2 or base.shape != quant.shape:
+        raise ValueError("base and quant must be [N, V] tensors of the same shape")
+    if base.dtype != quant.dtype:
+        raise TypeError("base and quant must share a dtype")
+    if not (base.is_contiguous() and quant.is_contiguous()):
+        raise ValueError("base and quant must be contiguous")
+    if on_device and not (base.is_cuda and quant.is_cuda):
+        raise ValueError("base and quant must be CUDA tensors")
+    if token_ids is not None:
+        if token_ids.dtype != torch.int32 or token_ids.dim() != 1 or token_ids.shape[0] != base.shape[0]:
+            raise ValueError("token_ids must be an int32 [N] tensor")
+        if not token_ids.is_contiguous():
+            raise ValueError("token_ids must be contiguous")
+        if on_device and token_ids.device != base.device:
+            raise ValueError("token_ids must be on the logits' device")
+
+
+def rows_view(records: torch.Tensor) -> dict:
+    """Field views of a [N, 32] uint8 tensor of row records."""
+    r = records.view(torch.uint8).reshape(-1, ROW_RECORD_BYTES)
+    f64 = r[:, :16].contiguous().view(torch.float64)
+    i32 = r[:, 16:28].contiguous().view(torch.int32)
+    return {"kld": f64[:, 0], "nll": f64[:, 1], "amax_b": i32[:, 0], "amax_q": i32[:, 1],
+            "flags": i32[:, 2]}
+
+
+class KLDStats:
+    """One handle of the library: workspace for up to ``max_rows`` rows on one
+    device. Not thread-safe; use one per concurrent stream."""
+
+    def __init__(self, max_rows: int, device=None):
+        self._lib = _lib.load()
+        if device is None:
+            device = torch.cuda.current_device()
+        self.device = torch.device("cuda", torch.device(device).index if not isinstance(device, int) else device)
+        self.max_rows = int(max_rows)
+        h = ctypes.c_void_p()
+        _lib.check(self._lib.kld_stats_create(ctypes.byref(h), self.max_rows, self.device.index),
+                   "kld_stats_create")
+        self._h = h
+        self._has_nll = False
+
+    def close(self):
+        if getattr(self, "_h", None):
+            self._lib.kld_stats_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *exc):
+        self.close()
+
+    # ------------------------------------------------------------ calls
+    def run(self, base: torch.Tensor, quant: torch.Tensor, token_ids: torch.Tensor | None = None,
+            stream=None) -> None:
+        _check_pair(base, quant, token_ids, True)
+        st = self._lib.kld_stats_run(self._h, _ptr(base), _ptr(quant), _ptr(token_ids),
+                                     base.shape[0], base.shape[1], dtype_code(base),
+                                     ctypes.c_void_p(_stream_ptr(stream, base.device)))
+        _lib.check(st, "kld_stats_run")
+
+    def run_host(self, base: torch.Tensor, quant: torch.Tensor, token_ids: torch.Tensor | None = None,
+                 stream=None) -> None:
+        """Same as :meth:`run` for host (preferably pinned) CPU tensors."""
+        _check_pair(base, quant, token_ids, False)
+        if base.is_cuda:
+            raise ValueError("run_host takes CPU tensors")
+        st = self._lib.kld_stats_run_host(self._h, _ptr(base), _ptr(quant), _ptr(token_ids),
+                                          base.shape[0], base.shape[1], dtype_code(base),
+                                          ctypes.c_void_p(_stream_ptr(stream, self.device)))
+        _lib.check(st, "kld_stats_run_host")
+
+    def run_rows(self, base, quant, token_ids=None, out: torch.Tensor | None = None, stream=None):
+        """Row pass only; records go to ``out`` ([N, 32] uint8 on the device)
+        or to the handle's workspace."""
+        _check_pair(base, quant, token_ids, True)
+        if out is not None and (out.dtype != torch.uint8 or out.numel() < base.shape[0] * ROW_RECORD_BYTES):
+            raise ValueError("out must be a uint8 tensor of N*32 bytes")
+        st = self._lib.kld_stats_run_rows(self._h, _ptr(base), _ptr(quant), _ptr(token_ids),
+                                          base.shape[0], base.shape[1], dtype_code(base), _ptr(out),
+                                          ctypes.c_void_p(_stream_ptr(stream, base.device)))
+        _lib.check(st, "kld_stats_run_rows")
+        return out
+
+    def reduce(self, records: torch.Tensor | None, n_rows: int, has_nll: bool, stream=None) -> None:
+        """Reduction over ``n_rows`` records (a device uint8 tensor, or None for
+        the handle's workspace)."""
+        st = self._lib.kld_stats_reduce(self._h, _ptr(records), int(n_rows), int(bool(has_nll)),
+                                        ctypes.c_void_p(_stream_ptr(stream, self.device)))
+        _lib.check(st, "kld_stats_reduce")
+
+    def result(self, raise_on_soft: bool = False) -> dict:
+        """Wait for the last run and return its statistics as a dict. Rows that
+        were excluded (``status`` != 0) do not raise unless asked to."""
+        res = _lib.Result()
+        st = self._lib.kld_stats_result(self._h, ctypes.byref(res))
+        if st not in _SOFT or (raise_on_soft and st != _lib.KLD_OK):
+            _lib.check(st, "kld_stats_result")
+        out = {name: getattr(res, name) for name, _ in _lib.Result._fields_
+               if not name.startswith("reserved")}
+        out["status"] = st
+        return out
+
+    def rows(self) -> torch.Tensor:
+        """Copy of the last run's per-row records as a [N, 32] uint8 CUDA
+        tensor (see :func:`rows_view`), ordered after the run on the current
+        stream."""
+        p = ctypes.c_void_p()
+        n = ctypes.c_int64()
+        _lib.check(self._lib.kld_stats_rows(self._h, ctypes.byref(p), ctypes.byref(n)), "kld_stats_rows")
+        nbytes = n.value * ROW_RECORD_BYTES
+        if nbytes == 0:
+            return torch.empty((0, ROW_RECORD_BYTES), dtype=torch.uint8, device=self.device)
+        view = torch.as_tensor(_DeviceBytes(p.value, nbytes), device=self.device)
+        return view.view(n.value, ROW_RECORD_BYTES).clone()
+
+    def set_timing(self, enable: bool) -> None:
+        _lib.check(self._lib.kld_stats_set_timing(self._h, int(bool(enable))), "kld_stats_set_timing")
+
+    def timing(self) -> tuple[float, float]:
+        a, b = ctypes.c_float(), ctypes.c_float()
+        _lib.check(self._lib.kld_stats_timing(self._h, ctypes.byref(a), ctypes.byref(b)), "kld_stats_timing")
+        return a.value, b.value
+
+    def plan(self, n_rows: int, vocab: int, dtype: int) -> dict:
+        return plan(n_rows, vocab, dtype, torch.cuda.get_device_properties(self.device).multi_processor_count)
+
+
+def plan(n_rows: int, vocab: int, dtype: int, sm_count: int) -> dict:
+    lib = _lib.load()
+    p = _lib.Plan()
+    _lib.check(lib.kld_plan(int(n_rows), int(vocab), int(dtype), int(sm_count), ctypes.byref(p)), "kld_plan")
+    return {name: getattr(p, name) for name, _ in _lib.Plan._fields_ if name != "reserved"}
+
+
+class _DeviceBytes:
+    """Zero-copy view of library-owned device memory for torch.as_tensor."""
+
+    def __init__(self, ptr: int, nbytes: int):
+        self.__cuda_array_interface__ = {"shape": (nbytes,), "typestr": "|u1",
+                                         "data": (ptr, True), "version": 3}
+
+
+def kld_stats(base: torch.Tensor, quant: torch.Tensor, token_ids: torch.Tensor | None = None) -> dict:
+    """One-shot convenience: statistics of one [N, V] pair on the current stream."""
+    with KLDStats(base.shape[0], base.device) as st:
+        st.run(base, quant, token_ids)
+        return st.result()

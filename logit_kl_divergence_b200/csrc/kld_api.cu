@@ -1,0 +1,387 @@
+// kld_api.cu -- host side of the C ABI declared in include/kld_stats.h.
+//
+// Owns the per-handle device workspace (one 32-byte record per row, the
+// device result, an error word), the pinned host copy of the result and the
+// staging buffers of the host-memory path; validates arguments before
+// anything is enqueued and maps CUDA failures to status codes. Every step of
+// the statistic runs in the kernels of kld_rows.cu and kld_reduce.cu.
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <cstring>
+#include <string>
+
+#include "kld_internal.h"
+
+namespace {
+
+thread_local std::string g_last_cuda_error;
+
+kld_status_t cuda_fail(cudaError_t e, const char* what) {
+  g_last_cuda_error = std::string(what) + ": " + cudaGetErrorString(e);
+  if (e == cudaErrorMemoryAllocation) return KLD_ERR_OOM;
+  if (e == cudaErrorNoDevice || e == cudaErrorInsufficientDriver ||
+      e == cudaErrorNoKernelImageForDevice)
+    return KLD_ERR_NO_DEVICE;
+  return KLD_ERR_CUDA;
+}
+
+#define KLD_CUDA(call)                                 \
+  do {                                                 \
+    cudaError_t _e = (call);                           \
+    if (_e != cudaSuccess) return cuda_fail(_e, #call); \
+  } while (0)
+
+// Makes the handle's device current for the duration of a call.
+class DeviceGuard {
+ public:
+  explicit DeviceGuard(int dev) {
+    ok_ = cudaGetDevice(&prev_) == cudaSuccess;
+    if (ok_ && prev_ != dev) ok_ = cudaSetDevice(dev) == cudaSuccess;
+    switched_ = ok_ && prev_ != dev;
+  }
+  ~DeviceGuard() {
+    if (switched_) cudaSetDevice(prev_);
+  }
+  bool ok() const { return ok_; }
+
+ private:
+  int prev_ = 0;
+  bool ok_ = false;
+  bool switched_ = false;
+};
+
+// Host-path staging: two buffers, each holding a chunk of base rows, quant
+// rows and token ids.
+constexpr size_t kStageTargetBytes = 128ull << 20;  // per operand per buffer
+
+}  // namespace
+
+struct kld_stats_s {
+  int device = 0;
+  int sm_count = 0;
+  int64_t max_rows = 0;
+  kld_row_t* rows = nullptr;
+  kld_result_t* dres = nullptr;
+  uint32_t* derr = nullptr;
+  kld_result_t* hres = nullptr;
+  cudaEvent_t done = nullptr;
+  bool has_result = false;
+  int64_t last_rows = 0;
+  bool timing = false;
+  bool timing_valid = false;
+  cudaEvent_t tev[3] = {nullptr, nullptr, nullptr};
+  // host path
+  cudaStream_t copy_stream = nullptr;
+  cudaEvent_t copied[2] = {nullptr, nullptr};
+  cudaEvent_t freed[2] = {nullptr, nullptr};
+  void* stage[2] = {nullptr, nullptr};
+  size_t stage_bytes = 0;  // per buffer
+};
+
+namespace {
+
+bool valid_dtype(kld_dtype_t dt) { return dt == KLD_F32 || dt == KLD_BF16 || dt == KLD_F16; }
+
+kld_status_t check_inputs(const void* base, const void* quant, const int32_t* tok, int64_t N,
+                          int64_t V, kld_dtype_t dtype, bool device_ptrs) {
+  if (!valid_dtype(dtype)) return KLD_ERR_DTYPE;
+  if (!base || !quant) return KLD_ERR_INVALID_ARG;
+  if (N < 1 || V < 1 || V > INT32_MAX) return KLD_ERR_INVALID_ARG;
+  const uintptr_t eb = static_cast<uintptr_t>(kld::elem_bytes(dtype));
+  const uintptr_t ab = reinterpret_cast<uintptr_t>(base);
+  const uintptr_t aq = reinterpret_cast<uintptr_t>(quant);
+  if (ab % eb || aq % eb) return KLD_ERR_INVALID_ARG;
+  if (device_ptrs && ((ab - aq) & 15u)) return KLD_ERR_INVALID_ARG;
+  if (tok && (reinterpret_cast<uintptr_t>(tok) & 3u)) return KLD_ERR_INVALID_ARG;
+  return KLD_OK;
+}
+
+int row_grid(const kld_stats_s* h, int64_t N) {
+  const int64_t g = N < h->sm_count ? N : h->sm_count;
+  return static_cast<int>(g < 1 ? 1 : g);
+}
+
+kld_status_t enqueue_reduce(kld_stats_t h, const kld_row_t* rows, int64_t N, int has_nll,
+                            cudaStream_t s) {
+  KLD_CUDA(kld::launch_reduce(rows, N, has_nll, h->derr, h->dres, s));
+  if (h->timing && h->timing_valid) KLD_CUDA(cudaEventRecord(h->tev[2], s));
+  KLD_CUDA(cudaMemcpyAsync(h->hres, h->dres, sizeof(kld_result_t), cudaMemcpyDeviceToHost, s));
+  KLD_CUDA(cudaEventRecord(h->done, s));
+  h->has_result = true;
+  return KLD_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int kld_abi_version(void) { return KLD_ABI_VERSION; }
+
+const char* kld_status_string(kld_status_t s) {
+  switch (s) {
+    case KLD_OK: return "ok";
+    case KLD_ERR_INVALID_ARG: return "invalid argument";
+    case KLD_ERR_DTYPE: return "unknown element type";
+    case KLD_ERR_OOM: return "out of memory";
+    case KLD_ERR_CUDA: return "CUDA error";
+    case KLD_ERR_NONFINITE: return "rows with NaN/+inf or all -inf were excluded";
+    case KLD_ERR_BAD_TOKEN: return "token ids outside [0, V) were excluded from PPL";
+    case KLD_ERR_TIMEOUT: return "a bounded device wait gave up";
+    case KLD_ERR_NO_DEVICE: return "no usable sm_100 device";
+    case KLD_ERR_NOT_READY: return "no run to report";
+  }
+  return "unknown status";
+}
+
+const char* kld_last_cuda_error(void) { return g_last_cuda_error.c_str(); }
+
+kld_status_t kld_plan(int64_t N, int64_t V, kld_dtype_t dtype, int sm_count, kld_plan_t* out) {
+  if (!out) return KLD_ERR_INVALID_ARG;
+  if (!valid_dtype(dtype)) return KLD_ERR_DTYPE;
+  if (N < 1 || V < 1 || V > INT32_MAX || sm_count < 1) return KLD_ERR_INVALID_ARG;
+  std::memset(out, 0, sizeof(*out));
+  out->variant = 0;
+  out->grid = static_cast<int32_t>(N < sm_count ? N : sm_count);
+  out->ctas_per_row = 1;
+  out->threads = kld::kRowThreads;
+  out->smem_bytes = kld::kRowSmemBytes;
+  out->stage_bytes = kld::kStageBytes;
+  out->stages = kld::kStages;
+  return KLD_OK;
+}
+
+kld_status_t kld_stats_create(kld_stats_t* out, int64_t max_rows, int device) {
+  if (!out) return KLD_ERR_INVALID_ARG;
+  *out = nullptr;
+  if (max_rows < 1 || device < 0) return KLD_ERR_INVALID_ARG;
+  int ndev = 0;
+  cudaError_t e = cudaGetDeviceCount(&ndev);
+  if (e != cudaSuccess || ndev == 0) {
+    g_last_cuda_error = e != cudaSuccess ? cudaGetErrorString(e) : "no CUDA device";
+    return KLD_ERR_NO_DEVICE;
+  }
+  if (device >= ndev) return KLD_ERR_INVALID_ARG;
+  int major = 0, minor = 0, sms = 0;
+  KLD_CUDA(cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, device));
+  KLD_CUDA(cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, device));
+  KLD_CUDA(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, device));
+  if (major != 10 || minor != 0) {
+    g_last_cuda_error = "device is not compute capability 10.0";
+    return KLD_ERR_NO_DEVICE;
+  }
+  DeviceGuard guard(device);
+  if (!guard.ok()) return cuda_fail(cudaGetLastError(), "cudaSetDevice");
+  KLD_CUDA(kld::prepare_rows_kernels());
+
+  kld_stats_s* h = new kld_stats_s();
+  h->device = device;
+  h->sm_count = sms;
+  h->max_rows = max_rows;
+  kld_status_t st = KLD_OK;
+  do {
+    cudaError_t err;
+    if ((err = cudaMalloc(&h->rows, sizeof(kld_row_t) * static_cast<size_t>(max_rows))) !=
+        cudaSuccess) { st = cuda_fail(err, "cudaMalloc(rows)"); break; }
+    if ((err = cudaMalloc(&h->dres, sizeof(kld_result_t))) != cudaSuccess) {
+      st = cuda_fail(err, "cudaMalloc(result)"); break; }
+    if ((err = cudaMalloc(&h->derr, sizeof(uint32_t))) != cudaSuccess) {
+      st = cuda_fail(err, "cudaMalloc(error word)"); break; }
+    if ((err = cudaMemset(h->derr, 0, sizeof(uint32_t))) != cudaSuccess) {
+      st = cuda_fail(err, "cudaMemset"); break; }
+    if ((err = cudaMallocHost(&h->hres, sizeof(kld_result_t))) != cudaSuccess) {
+      st = cuda_fail(err, "cudaMallocHost"); break; }
+    if ((err = cudaEventCreateWithFlags(&h->done, cudaEventDisableTiming)) != cudaSuccess) {
+      st = cuda_fail(err, "cudaEventCreate"); break; }
+    for (int i = 0; i < 3 && st == KLD_OK; ++i)
+      if ((err = cudaEventCreate(&h->tev[i])) != cudaSuccess) st = cuda_fail(err, "cudaEventCreate");
+  } while (0);
+  if (st != KLD_OK) {
+    kld_stats_destroy(h);
+    return st;
+  }
+  *out = h;
+  return KLD_OK;
+}
+
+void kld_stats_destroy(kld_stats_t h) {
+  if (!h) return;
+  DeviceGuard guard(h->device);
+  if (h->copy_stream) cudaStreamSynchronize(h->copy_stream);
+  if (h->done && h->has_result) cudaEventSynchronize(h->done);
+  for (int i = 0; i < 2; ++i) {
+    if (h->freed[i]) cudaEventSynchronize(h->freed[i]);
+    if (h->stage[i]) cudaFree(h->stage[i]);
+    if (h->copied[i]) cudaEventDestroy(h->copied[i]);
+    if (h->freed[i]) cudaEventDestroy(h->freed[i]);
+  }
+  if (h->copy_stream) cudaStreamDestroy(h->copy_stream);
+  for (int i = 0; i < 3; ++i)
+    if (h->tev[i]) cudaEventDestroy(h->tev[i]);
+  if (h->done) cudaEventDestroy(h->done);
+  if (h->hres) cudaFreeHost(h->hres);
+  if (h->derr) cudaFree(h->derr);
+  if (h->dres) cudaFree(h->dres);
+  if (h->rows) cudaFree(h->rows);
+  delete h;
+}
+
+kld_status_t kld_stats_run_rows(kld_stats_t h, const void* base, const void* quant,
+                                const int32_t* token_ids, int64_t N, int64_t V,
+                                kld_dtype_t dtype, kld_row_t* rows_out, void* stream) {
+  if (!h) return KLD_ERR_INVALID_ARG;
+  kld_status_t st = check_inputs(base, quant, token_ids, N, V, dtype, true);
+  if (st != KLD_OK) return st;
+  if (!rows_out && N > h->max_rows) return KLD_ERR_INVALID_ARG;
+  if (rows_out && (reinterpret_cast<uintptr_t>(rows_out) & 7u)) return KLD_ERR_INVALID_ARG;
+  DeviceGuard guard(h->device);
+  if (!guard.ok()) return cuda_fail(cudaGetLastError(), "cudaSetDevice");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  KLD_CUDA(kld::launch_rows(base, quant, token_ids, N, V, dtype, rows_out ? rows_out : h->rows,
+                            h->derr, row_grid(h, N), s));
+  if (!rows_out) h->last_rows = N;
+  h->timing_valid = false;
+  return KLD_OK;
+}
+
+kld_status_t kld_stats_reduce(kld_stats_t h, const kld_row_t* rows_dev, int64_t N, int has_nll,
+                              void* stream) {
+  if (!h) return KLD_ERR_INVALID_ARG;
+  if (N < 1) return KLD_ERR_INVALID_ARG;
+  if (!rows_dev && N > h->max_rows) return KLD_ERR_INVALID_ARG;
+  if (rows_dev && (reinterpret_cast<uintptr_t>(rows_dev) & 7u)) return KLD_ERR_INVALID_ARG;
+  DeviceGuard guard(h->device);
+  if (!guard.ok()) return cuda_fail(cudaGetLastError(), "cudaSetDevice");
+  h->timing_valid = false;
+  return enqueue_reduce(h, rows_dev ? rows_dev : h->rows, N, has_nll ? 1 : 0,
+                        static_cast<cudaStream_t>(stream));
+}
+
+kld_status_t kld_stats_run(kld_stats_t h, const void* base, const void* quant,
+                           const int32_t* token_ids, int64_t N, int64_t V, kld_dtype_t dtype,
+                           void* stream) {
+  if (!h) return KLD_ERR_INVALID_ARG;
+  kld_status_t st = check_inputs(base, quant, token_ids, N, V, dtype, true);
+  if (st != KLD_OK) return st;
+  if (N > h->max_rows) return KLD_ERR_INVALID_ARG;
+  DeviceGuard guard(h->device);
+  if (!guard.ok()) return cuda_fail(cudaGetLastError(), "cudaSetDevice");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  h->timing_valid = h->timing;
+  if (h->timing) KLD_CUDA(cudaEventRecord(h->tev[0], s));
+  KLD_CUDA(kld::launch_rows(base, quant, token_ids, N, V, dtype, h->rows, h->derr,
+                            row_grid(h, N), s));
+  if (h->timing) KLD_CUDA(cudaEventRecord(h->tev[1], s));
+  h->last_rows = N;
+  return enqueue_reduce(h, h->rows, N, token_ids != nullptr, s);
+}
+
+kld_status_t kld_stats_result(kld_stats_t h, kld_result_t* out) {
+  if (!h || !out) return KLD_ERR_INVALID_ARG;
+  if (!h->has_result) return KLD_ERR_NOT_READY;
+  DeviceGuard guard(h->device);
+  if (!guard.ok()) return cuda_fail(cudaGetLastError(), "cudaSetDevice");
+  KLD_CUDA(cudaEventSynchronize(h->done));
+  *out = *h->hres;
+  if (out->device_error) return KLD_ERR_TIMEOUT;
+  if (out->flags_or & (KLD_ROW_NONFINITE | KLD_ROW_EMPTY)) return KLD_ERR_NONFINITE;
+  if (out->flags_or & KLD_ROW_BAD_TOKEN) return KLD_ERR_BAD_TOKEN;
+  return KLD_OK;
+}
+
+kld_status_t kld_stats_rows(kld_stats_t h, const kld_row_t** rows_dev, int64_t* n_rows) {
+  if (!h || !rows_dev || !n_rows) return KLD_ERR_INVALID_ARG;
+  *rows_dev = h->rows;
+  *n_rows = h->last_rows;
+  return KLD_OK;
+}
+
+kld_status_t kld_stats_set_timing(kld_stats_t h, int enable) {
+  if (!h) return KLD_ERR_INVALID_ARG;
+  h->timing = enable != 0;
+  h->timing_valid = false;
+  return KLD_OK;
+}
+
+kld_status_t kld_stats_timing(kld_stats_t h, float* row_pass_ms, float* reduce_ms) {
+  if (!h || !row_pass_ms || !reduce_ms) return KLD_ERR_INVALID_ARG;
+  if (!h->timing_valid || !h->has_result) return KLD_ERR_NOT_READY;
+  DeviceGuard guard(h->device);
+  if (!guard.ok()) return cuda_fail(cudaGetLastError(), "cudaSetDevice");
+  KLD_CUDA(cudaEventSynchronize(h->done));
+  KLD_CUDA(cudaEventElapsedTime(row_pass_ms, h->tev[0], h->tev[1]));
+  KLD_CUDA(cudaEventElapsedTime(reduce_ms, h->tev[1], h->tev[2]));
+  return KLD_OK;
+}
+
+kld_status_t kld_stats_run_host(kld_stats_t h, const void* base_host, const void* quant_host,
+                                const int32_t* token_ids_host, int64_t N, int64_t V,
+                                kld_dtype_t dtype, void* stream) {
+  if (!h) return KLD_ERR_INVALID_ARG;
+  kld_status_t st = check_inputs(base_host, quant_host, token_ids_host, N, V, dtype, false);
+  if (st != KLD_OK) return st;
+  if (N > h->max_rows) return KLD_ERR_INVALID_ARG;
+  DeviceGuard guard(h->device);
+  if (!guard.ok()) return cuda_fail(cudaGetLastError(), "cudaSetDevice");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+
+  const size_t row_bytes = static_cast<size_t>(V) * static_cast<size_t>(kld::elem_bytes(dtype));
+  int64_t chunk = static_cast<int64_t>(kStageTargetBytes / row_bytes);
+  if (chunk < 1) chunk = 1;
+  if (chunk > N) chunk = N;
+  // Each buffer: [chunk rows of base][chunk rows of quant][chunk token ids],
+  // every part starting on a 256-byte boundary.
+  const size_t part = ((static_cast<size_t>(chunk) * row_bytes) + 255) & ~static_cast<size_t>(255);
+  const size_t need = 2 * part + ((static_cast<size_t>(chunk) * 4 + 255) & ~static_cast<size_t>(255));
+  if (!h->copy_stream) {
+    KLD_CUDA(cudaStreamCreateWithFlags(&h->copy_stream, cudaStreamNonBlocking));
+    for (int i = 0; i < 2; ++i) {
+      KLD_CUDA(cudaEventCreateWithFlags(&h->copied[i], cudaEventDisableTiming));
+      KLD_CUDA(cudaEventCreateWithFlags(&h->freed[i], cudaEventDisableTiming));
+    }
+  }
+  if (need > h->stage_bytes) {
+    for (int i = 0; i < 2; ++i) {
+      KLD_CUDA(cudaEventSynchronize(h->freed[i]));
+      if (h->stage[i]) cudaFree(h->stage[i]);
+      h->stage[i] = nullptr;
+    }
+    h->stage_bytes = 0;
+    for (int i = 0; i < 2; ++i) KLD_CUDA(cudaMalloc(&h->stage[i], need));
+    h->stage_bytes = need;
+  }
+  // Earlier work of `stream` may still read the staging buffers.
+  for (int i = 0; i < 2; ++i) KLD_CUDA(cudaEventRecord(h->freed[i], s));
+
+  h->timing_valid = false;
+  const char* hb = static_cast<const char*>(base_host);
+  const char* hq = static_cast<const char*>(quant_host);
+  const int64_t nchunks = (N + chunk - 1) / chunk;
+  for (int64_t c = 0; c < nchunks; ++c) {
+    const int b = static_cast<int>(c & 1);
+    const int64_t r0 = c * chunk;
+    const int64_t n = (N - r0) < chunk ? (N - r0) : chunk;
+    char* sb = static_cast<char*>(h->stage[b]);
+    char* sq = sb + part;
+    int32_t* stok = reinterpret_cast<int32_t*>(sb + 2 * part);
+    KLD_CUDA(cudaStreamWaitEvent(h->copy_stream, h->freed[b], 0));
+    KLD_CUDA(cudaMemcpyAsync(sb, hb + static_cast<size_t>(r0) * row_bytes,
+                             static_cast<size_t>(n) * row_bytes, cudaMemcpyHostToDevice,
+                             h->copy_stream));
+    KLD_CUDA(cudaMemcpyAsync(sq, hq + static_cast<size_t>(r0) * row_bytes,
+                             static_cast<size_t>(n) * row_bytes, cudaMemcpyHostToDevice,
+                             h->copy_stream));
+    if (token_ids_host)
+      KLD_CUDA(cudaMemcpyAsync(stok, token_ids_host + r0, static_cast<size_t>(n) * 4,
+                               cudaMemcpyHostToDevice, h->copy_stream));
+    KLD_CUDA(cudaEventRecord(h->copied[b], h->copy_stream));
+    KLD_CUDA(cudaStreamWaitEvent(s, h->copied[b], 0));
+    KLD_CUDA(kld::launch_rows(sb, sq, token_ids_host ? stok : nullptr, n, V, dtype,
+                              h->rows + r0, h->derr, row_grid(h, n), s));
+    KLD_CUDA(cudaEventRecord(h->freed[b], s));
+  }
+  h->last_rows = N;
+  return enqueue_reduce(h, h->rows, N, token_ids_host != nullptr, s);
+}
+
+}  // extern "C"

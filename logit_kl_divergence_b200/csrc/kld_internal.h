@@ -1,0 +1,45 @@
+// kld_internal.h -- declarations shared by the library's translation units
+// (row pass, reduction, host API). Not part of the public ABI.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "kld_stats.h"
+
+namespace kld {
+
+// Device error word bits (kld_result_t.device_error).
+constexpr uint32_t kErrWaitTimeout = 1u << 0;  // a bounded mbarrier wait gave up
+
+// Row-pass tile geometry: a producer warp streams both rows through a ring of
+// shared-memory stages with bulk copies; kConsumerWarps warps consume them.
+constexpr int kConsumerWarps = 8;
+constexpr int kRowThreads = (kConsumerWarps + 1) * 32;
+constexpr int kStageBytes = 32 * 1024;  // per operand per stage
+constexpr int kStages = 3;
+constexpr int kChunkElems = 1024;       // elements per warp-chunk (32 per lane)
+
+// Dynamic shared memory of the row kernel: stages for both operands, then a
+// small control block (mbarriers, per-warp partials, argmax slots).
+constexpr int kRowCtrlBytes = 1024;
+constexpr int kRowSmemBytes = kStages * 2 * kStageBytes + kRowCtrlBytes;
+
+// Reduction kernel geometry.
+constexpr int kReduceThreads = 1024;
+
+inline int elem_bytes(kld_dtype_t dt) { return dt == KLD_F32 ? 4 : 2; }
+
+// Launchers (defined in the .cu files). They enqueue on `stream` and return
+// the launch error.
+cudaError_t launch_rows(const void* base, const void* quant,
+                        const int32_t* token_ids, int64_t N, int64_t V,
+                        kld_dtype_t dtype, kld_row_t* rows, uint32_t* derr,
+                        int grid, cudaStream_t stream);
+cudaError_t prepare_rows_kernels();  // per-device attribute setup
+
+cudaError_t launch_reduce(const kld_row_t* rows, int64_t N, int has_nll,
+                          uint32_t* derr, kld_result_t* out,
+                          cudaStream_t stream);
+
+}  // namespace kld

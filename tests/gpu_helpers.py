@@ -1,0 +1,111 @@
+"""Shared helpers of the GPU parity tests: run the CUDA path through the C ABI
+and compare with the fp64 oracle at the stated tolerances.
+
+Tolerances: argmax indices, flags and agreement counts bit-exact; per-row KL
+and NLL |gpu - ref| <= 1e-6 + 1e-4 * |ref|; mean KLD, percentiles, mean NLL
+and PPL within 1e-5 relative (absolute floor 1e-12 for values near zero).
+"""
+from __future__ import annotations
+
+import math
+import os
+
+import numpy as np
+import torch
+
+import oracle
+from logit_kl_divergence_b200 import KLDStats, rows_view, synth
+
+ODT = {synth.F32: oracle.F32, synth.BF16: oracle.BF16, synth.F16: oracle.F16}
+EXCLUDED = oracle.ROW_NONFINITE | oracle.ROW_EMPTY
+ROW_ATOL, ROW_RTOL = 1e-6, 1e-4
+STAT_RTOL, STAT_ATOL = 1e-5, 1e-12
+CORES = max(1, os.cpu_count() or 1)
+
+
+def gpu_run(base, quant, tok=None, use_rows_api=False):
+    """The whole statistic on the GPU; returns (per-row numpy dict, result)."""
+    st = KLDStats(max_rows=base.shape[0], device=base.device)
+    try:
+        if use_rows_api:
+            out = torch.empty((base.shape[0], 32), dtype=torch.uint8, device=base.device)
+            st.run_rows(base, quant, tok, out=out)
+            st.reduce(out, base.shape[0], tok is not None)
+            res = st.result()
+            rec = rows_view(out)
+        else:
+            st.run(base, quant, tok)
+            res = st.result()
+            rec = rows_view(st.rows())
+        rows = {k: v.cpu().numpy() for k, v in rec.items()}
+        rows["flags"] = rows["flags"].astype(np.uint32)
+        return rows, res
+    finally:
+        st.close()
+
+
+def _close_rows(g, o, what, idx):
+    g = np.asarray(g, np.float64)
+    o = np.asarray(o, np.float64)
+    both_nan = np.isnan(g) & np.isnan(o)
+    both_inf = np.isinf(g) & np.isinf(o) & (np.sign(g) == np.sign(o))
+    ok = both_nan | both_inf | (np.abs(g - o) <= ROW_ATOL + ROW_RTOL * np.abs(o))
+    if not ok.all():
+        bad = np.nonzero(~ok)[0][:8]
+        raise AssertionError(f"{what} mismatch at rows {idx[bad]}: gpu={g[bad]} ref={o[bad]}")
+
+
+def assert_rows_match(g: dict, o: dict, idx=None):
+    n = len(o["kld"])
+    idx = np.arange(n) if idx is None else np.asarray(idx)
+    assert np.array_equal(g["flags"], o["flags"]), (
+        f"flags differ at rows {idx[np.nonzero(g['flags'] != o['flags'])[0][:8]]}")
+    assert np.array_equal(g["amax_b"], o["amax_b"]), (
+        f"argmax_base differs at rows {idx[np.nonzero(g['amax_b'] != o['amax_b'])[0][:8]]}")
+    assert np.array_equal(g["amax_q"], o["amax_q"]), (
+        f"argmax_quant differs at rows {idx[np.nonzero(g['amax_q'] != o['amax_q'])[0][:8]]}")
+    _close_rows(g["kld"], o["kld"], "kld", idx)
+    _close_rows(g["nll"], o["nll"], "nll", idx)
+
+
+def stat_close(a, b):
+    if (isinstance(a, float) and math.isnan(a)) or (isinstance(b, float) and math.isnan(b)):
+        return math.isnan(a) and math.isnan(b)
+    if math.isinf(a) or math.isinf(b):
+        return a == b
+    return abs(a - b) <= STAT_ATOL + STAT_RTOL * abs(b)
+
+
+def assert_stats_match(gres: dict, ores: dict):
+    for k in ("n_rows", "n_valid", "top1_agree", "n_nll", "n_flagged", "flags_or", "has_nll"):
+        assert int(gres[k]) == int(ores[k]), (k, gres[k], ores[k])
+    for k in ("mean_kld", "median_kld", "p90_kld", "p99_kld", "max_kld", "top1_agree_pct",
+              "mean_nll", "ppl"):
+        assert stat_close(gres[k], ores[k]), (k, gres[k], ores[k])
+    assert gres["device_error"] == 0
+
+
+def assert_select_exact(g_rows: dict, gres: dict, has_nll: bool):
+    """The GPU's percentiles are the exact order statistics of its own per-row
+    array (the oracle's std::sort + interpolation applied to the same values)."""
+    ref = oracle.reduce(g_rows, has_nll)
+    for k in ("median_kld", "p90_kld", "p99_kld", "max_kld"):
+        a, b = gres[k], ref[k]
+        assert (a == b) or (math.isnan(a) and math.isnan(b)), (k, a, b)
+    for k in ("n_valid", "top1_agree", "n_nll", "n_flagged", "flags_or"):
+        assert int(gres[k]) == int(ref[k]), k
+
+
+def oracle_rows_chunked(w, nthreads=CORES, chunk_rows=1024):
+    """Oracle per-row values of a device workload, computed on host chunks."""
+    n = w.base.shape[0]
+    out = {k: [] for k in ("kld", "nll", "amax_b", "amax_q", "flags")}
+    for r0 in range(0, n, chunk_rows):
+        r1 = min(n, r0 + chunk_rows)
+        b = w.base[r0:r1].cpu()
+        q = w.quant[r0:r1].cpu()
+        t = w.token_ids[r0:r1].cpu() if w.token_ids is not None else None
+        r = oracle.rows(b, q, t, ODT[w.dtype], nthreads)
+        for k in out:
+            out[k].append(r[k])
+    return {k: np.concatenate(v) for k, v in out.items()}

@@ -1,0 +1,116 @@
+"""The reduction + exact percentile kernel on synthetic per-row records.
+
+Record arrays are built directly (no row pass) so the radix select meets
+distributions the row pass rarely produces: heavy duplicates, all-equal
+values, tiny negative KL from rounding, +inf, excluded rows, and sizes from a
+single row to well past the gather threshold (several radix passes)."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from logit_kl_divergence_b200 import KLDStats
+
+pytestmark = pytest.mark.gpu
+DEV = torch.device("cuda", 0)
+
+REC = np.dtype([("kld", "<f8"), ("nll", "<f8"), ("amax_b", "<i4"), ("amax_q", "<i4"),
+                ("flags", "<u4"), ("reserved", "<u4")])
+
+
+def make_records(kld, rng, flags=None, nll=True):
+    n = len(kld)
+    r = np.zeros(n, REC)
+    r["kld"] = kld
+    r["nll"] = rng.gamma(2.0, 1.0, n) if nll else np.nan
+    r["amax_b"] = rng.integers(0, 5, n)
+    r["amax_q"] = rng.integers(0, 5, n)
+    if flags is not None:
+        r["flags"] = flags
+        excl = (flags & (oracle.ROW_NONFINITE | oracle.ROW_EMPTY)) != 0
+        r["kld"][excl] = np.nan
+        r["amax_b"][excl] = -1
+        r["amax_q"][excl] = -1
+    return r
+
+
+def run_reduce(rec, has_nll=True):
+    t = torch.from_numpy(rec.view(np.uint8).copy()).to(DEV)
+    st = KLDStats(max_rows=1, device=DEV)
+    st.reduce(t, len(rec), has_nll)
+    res = st.result()
+    st.close()
+    return res
+
+
+def check(rec, has_nll=True):
+    g = run_reduce(rec, has_nll)
+    d = {"kld": rec["kld"], "nll": rec["nll"], "amax_b": rec["amax_b"],
+         "amax_q": rec["amax_q"], "flags": rec["flags"]}
+    o = oracle.reduce(d, has_nll)
+    for k in ("median_kld", "p90_kld", "p99_kld", "max_kld"):
+        assert g[k] == o[k] or (math.isnan(g[k]) and math.isnan(o[k])), (k, g[k], o[k])
+    for k in ("n_rows", "n_valid", "top1_agree", "n_nll", "n_flagged", "flags_or"):
+        assert int(g[k]) == int(o[k]), k
+    for k in ("mean_kld", "mean_nll", "ppl", "top1_agree_pct"):
+        a, b = g[k], o[k]
+        if math.isnan(b) or math.isinf(b):
+            assert (math.isnan(a) and math.isnan(b)) or a == b, (k, a, b)
+        else:
+            assert abs(a - b) <= 1e-12 * abs(b) + 1e-300, (k, a, b)
+    return g
+
+
+@pytest.mark.parametrize("n", [1, 2, 3, 4, 5, 100, 4095, 4096, 4097, 8192, 32768, 100003, 1 << 20])
+def test_continuous_values(n):
+    rng = np.random.default_rng(n)
+    check(make_records(rng.gamma(0.6, 0.08, n), rng))
+
+
+@pytest.mark.parametrize("n", [10, 5000, 70000])
+def test_heavy_duplicates(n):
+    rng = np.random.default_rng(7)
+    vals = rng.choice(np.array([0.0, 1e-3, 0.05, 0.05000000000000001, 2.0]), size=n)
+    check(make_records(vals, rng))
+
+
+@pytest.mark.parametrize("n", [1, 4097, 50000])
+def test_all_equal(n):
+    rng = np.random.default_rng(3)
+    check(make_records(np.full(n, 0.0123), rng))
+
+
+def test_tiny_negatives_zeros_and_infinities():
+    rng = np.random.default_rng(11)
+    n = 60000
+    v = rng.gamma(0.6, 0.08, n)
+    v[rng.integers(0, n, 500)] = -1e-13
+    v[rng.integers(0, n, 500)] = -0.0
+    v[rng.integers(0, n, 500)] = 0.0
+    v[rng.integers(0, n, 50)] = np.inf
+    check(make_records(v, rng))
+
+
+def test_excluded_rows_and_bad_tokens():
+    rng = np.random.default_rng(5)
+    n = 20000
+    flags = np.zeros(n, np.uint32)
+    flags[rng.integers(0, n, 300)] |= oracle.ROW_NONFINITE
+    flags[rng.integers(0, n, 300)] |= oracle.ROW_EMPTY
+    flags[rng.integers(0, n, 300)] |= oracle.ROW_BAD_TOKEN
+    check(make_records(rng.gamma(0.6, 0.08, n), rng, flags))
+
+
+def test_all_rows_excluded():
+    rng = np.random.default_rng(2)
+    flags = np.full(10, oracle.ROW_EMPTY, np.uint32)
+    g = check(make_records(np.zeros(10), rng, flags))
+    assert g["n_valid"] == 0 and math.isnan(g["mean_kld"]) and math.isnan(g["median_kld"])
+
+
+def test_without_nll():
+    rng = np.random.default_rng(9)
+    g = check(make_records(rng.gamma(0.6, 0.08, 999), rng, nll=False), has_nll=False)
+    assert math.isnan(g["ppl"]) and g["has_nll"] == 0
