@@ -194,7 +194,7 @@ class _DeviceBytes:
 
     def __init__(self, ptr: int, nbytes: int):
         self.__cuda_array_interface__ = {"shape": (nbytes,), "typestr": "|u1",
-                                         "data": (ptr, True), "version": 3}
+                                         "data": (ptr, False), "version": 3}
 
 
 def kld_stats(base: torch.Tensor, quant: torch.Tensor, token_ids: torch.Tensor | None = None) -> dict:
