@@ -9,16 +9,17 @@
 // was made", step 5).
 //
 // Streaming form of the statistic. With L = log2(e) rounded to fp32 and a
-// reference exponent c (in log2 units) per row operand,
-//   u_j = b_j*L - c_b,  v_j = q_j*L - c_q       (one FMA each, no rounding of
-//                                                the product)
+// reference c per row operand (the running maximum),
+//   u_j = (b_j - c_b) * L,  v_j = (q_j - c_q) * L
 //   S_b = sum 2^u_j,  S_q = sum 2^v_j,  T = sum 2^u_j * (u_j - v_j)
 //   KL  = ln2 * T / S_b + ln(S_q / S_b)
-// The references cancel exactly, so c may be any value near the running max;
-// all terms stay max-relative and a constant shift of a whole row (e.g.
-// quant = base + 1000) does not cancel catastrophically. Changing c_b by d
-// scales S_b and T by 2^-d and subtracts d*S_b from T; changing c_q by d adds
-// d*S_b to T and scales S_q by 2^-d.
+// The references cancel exactly in KL; they only keep every term max-
+// relative, so a constant shift of a whole row (e.g. quant = base + 1000)
+// does not cancel catastrophically, the maximum contributes exactly 2^0 = 1,
+// and an exact shift gives bit-identical u and v (KL exactly 0). Raising c_b
+// by D rescales S_b and T by 2^-(D*L) and subtracts D*L*S_b from T; raising
+// c_q by D adds D*L*S_b to T and rescales S_q by 2^-(D*L). (Since L is fp32,
+// exponentials are of (1 + 1.4e-8) * x; KL and NLL change by that factor.)
 //
 // Structure (one CTA per row at a time, persistent over rows):
 //   - warp 8 (producer): one lane streams the row's 16-byte-aligned body in
@@ -48,6 +49,7 @@ namespace kld {
 namespace {
 
 constexpr float kLog2e = 1.4426950408889634f;  // log2(e) rounded to fp32
+constexpr double kLog2eD = static_cast<double>(kLog2e);  // the same value
 constexpr double kLn2 = 0.6931471805599453;    // ln(2)
 constexpr float kNegBig = -1.0e30f;
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
@@ -191,7 +193,7 @@ struct Elem<KLD_F16> {
 // Warp-uniform reference of one row operand pair.
 struct WarpRef {
   float Mb, Mq;  // running maxima seen by this warp (-inf before any)
-  float cb, cq;  // reference exponents fl(M * L); 0 before any finite max
+  float cb, cq;  // references: the running maxima once finite, 0 before
 };
 
 // Per-lane accumulators and argmax memory.
@@ -219,23 +221,21 @@ struct Ctrl {
 static_assert(sizeof(Ctrl) <= kRowCtrlBytes, "control block too large");
 
 __device__ __forceinline__ void raise_base(float wmax, WarpRef& r, LaneAcc& a) {
-  const float cn = wmax * kLog2e;
   if (r.Mb != -INFINITY) {  // accumulators are exactly 0 before any finite max
-    const double d = static_cast<double>(cn) - static_cast<double>(r.cb);
+    const double d = (static_cast<double>(wmax) - static_cast<double>(r.cb)) * kLog2eD;
     const double sc = exp2(-d);
     a.T = (a.T - d * a.Sb) * sc;
     a.Sb *= sc;
   }
-  r.cb = cn;
+  r.cb = wmax;
   r.Mb = wmax;
 }
 
 __device__ __forceinline__ void raise_quant(float wmax, WarpRef& r, LaneAcc& a) {
-  const float cn = wmax * kLog2e;
-  const double d = static_cast<double>(cn) - static_cast<double>(r.cq);
+  const double d = (static_cast<double>(wmax) - static_cast<double>(r.cq)) * kLog2eD;
   a.T += d * a.Sb;
   if (r.Mq != -INFINITY) a.Sq *= exp2(-d);
-  r.cq = cn;
+  r.cq = wmax;
   r.Mq = wmax;
 }
 
@@ -248,14 +248,14 @@ __device__ __forceinline__ void accumulate32(const float* xb, const float* xq,
   const float wmq = warp_max(mq);
   if (wmb > ref.Mb) raise_base(wmb, ref, acc);
   if (wmq > ref.Mq) raise_quant(wmq, ref, acc);
-  const float nb = -ref.cb, nq = -ref.cq;
+  const float cb = ref.cb, cq = ref.cq;
   float sb0 = 0.f, sb1 = 0.f, sq0 = 0.f, sq1 = 0.f, t0 = 0.f, t1 = 0.f;
 #pragma unroll
   for (int i = 0; i < 32; i += 2) {
-    const float u0 = fmaf(xb[i], kLog2e, nb);
-    const float v0 = fmaf(xq[i], kLog2e, nq);
-    const float u1 = fmaf(xb[i + 1], kLog2e, nb);
-    const float v1 = fmaf(xq[i + 1], kLog2e, nq);
+    const float u0 = __fmul_rn(__fsub_rn(xb[i], cb), kLog2e);
+    const float v0 = __fmul_rn(__fsub_rn(xq[i], cq), kLog2e);
+    const float u1 = __fmul_rn(__fsub_rn(xb[i + 1], cb), kLog2e);
+    const float v1 = __fmul_rn(__fsub_rn(xq[i + 1], cq), kLog2e);
     const float e0 = ex2(u0), f0 = ex2(v0);
     const float e1 = ex2(u1), f1 = ex2(v1);
     sb0 += e0;
@@ -522,8 +522,8 @@ __global__ void __launch_bounds__(kRowThreads, 1)
       const float wmq = warp_max(xe_q);
       if (wmb > ref.Mb) raise_base(wmb, ref, acc);
       if (wmq > ref.Mq) raise_quant(wmq, ref, acc);
-      const float u = fmaf(xe_b, kLog2e, -ref.cb);
-      const float v = fmaf(xe_q, kLog2e, -ref.cq);
+      const float u = __fmul_rn(__fsub_rn(xe_b, ref.cb), kLog2e);
+      const float v = __fmul_rn(__fsub_rn(xe_q, ref.cq), kLog2e);
       const float e = ex2(u);
       acc.Sb += static_cast<double>(e);
       acc.Sq += static_cast<double>(ex2(v));
@@ -598,9 +598,9 @@ __global__ void __launch_bounds__(kRowThreads, 1)
         bool inf_kl = false;
         for (int w = 0; w < kConsumerWarps; ++w) {
           const WarpPart& p = ctrl->part[pb][w];
-          const double dq = static_cast<double>(Cq) - static_cast<double>(p.cq);
+          const double dq = (static_cast<double>(Cq) - static_cast<double>(p.cq)) * kLog2eD;
           if (p.Mb > -INFINITY) {
-            const double db = static_cast<double>(Cb) - static_cast<double>(p.cb);
+            const double db = (static_cast<double>(Cb) - static_cast<double>(p.cb)) * kLog2eD;
             const double sc = exp2(-db);
             sb += p.Sb * sc;
             if (!isfinite(p.T)) {
@@ -622,8 +622,8 @@ __global__ void __launch_bounds__(kRowThreads, 1)
             nll = INFINITY;
             flags |= KLD_ROW_INF_NLL;
           } else {
-            nll = log(sq) + kLn2 * (static_cast<double>(Cq) -
-                                    static_cast<double>(q_tok) * static_cast<double>(kLog2e));
+            nll = log(sq) +
+                  kLn2 * ((static_cast<double>(Cq) - static_cast<double>(q_tok)) * kLog2eD);
           }
         }
         ab = ctrl->amax[pb][0];
