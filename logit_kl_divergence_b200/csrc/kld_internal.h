@@ -12,17 +12,21 @@ namespace kld {
 // Device error word bits (kld_result_t.device_error).
 constexpr uint32_t kErrWaitTimeout = 1u << 0;  // a bounded mbarrier wait gave up
 
-// Row-pass tile geometry: a producer warp streams both rows through a ring of
-// shared-memory stages with bulk copies; kConsumerWarps warps consume them.
-constexpr int kConsumerWarps = 8;
-constexpr int kRowThreads = (kConsumerWarps + 1) * 32;
+// Row-pass geometry: a producer warp streams both rows through a ring of
+// shared-memory stages with bulk copies; kConsumerWarps warps consume them in
+// chunks of kLaneElems elements per lane; one epilogue warp combines each
+// row's partials (published through a ring of kSlots slots).
+constexpr int kConsumerWarps = 16;
+constexpr int kRowThreads = (kConsumerWarps + 2) * 32;
 constexpr int kStageBytes = 32 * 1024;  // per operand per stage
 constexpr int kStages = 3;
-constexpr int kChunkElems = 1024;       // elements per warp-chunk (32 per lane)
+constexpr int kLaneElems = 16;
+constexpr int kChunkElems = kLaneElems * 32;  // elements per warp-chunk
+constexpr int kSlots = 4;
 
-// Dynamic shared memory of the row kernel: stages for both operands, then a
-// small control block (mbarriers, per-warp partials, argmax slots).
-constexpr int kRowCtrlBytes = 1024;
+// Dynamic shared memory of the row kernel: stages for both operands, then the
+// control block (mbarriers and the partial slots).
+constexpr int kRowCtrlBytes = 24 * 1024;
 constexpr int kRowSmemBytes = kStages * 2 * kStageBytes + kRowCtrlBytes;
 
 // Reduction kernel geometry.

@@ -8,36 +8,46 @@
 // full vocabulary from "Mistral-Small-4-119B-2603 GSQ-RCO IQ3_S GGUF", "How it
 // was made", step 5).
 //
-// Streaming form of the statistic. With L = log2(e) rounded to fp32 and a
-// reference c per row operand (the running maximum),
-//   u_j = (b_j - c_b) * L,  v_j = (q_j - c_q) * L
-//   S_b = sum 2^u_j,  S_q = sum 2^v_j,  T = sum 2^u_j * (u_j - v_j)
-//   KL  = ln2 * T / S_b + ln(S_q / S_b)
-// The references cancel exactly in KL; they only keep every term max-
-// relative, so a constant shift of a whole row (e.g. quant = base + 1000)
-// does not cancel catastrophically, the maximum contributes exactly 2^0 = 1,
-// and an exact shift gives bit-identical u and v (KL exactly 0). Raising c_b
-// by D rescales S_b and T by 2^-(D*L) and subtracts D*L*S_b from T; raising
-// c_q by D adds D*L*S_b to T and rescales S_q by 2^-(D*L). (Since L is fp32,
-// exponentials are of (1 + 1.4e-8) * x; KL and NLL change by that factor.)
+// Streaming form of the statistic. With p = softmax(b), r = softmax(q) and
+// the exact per-element log-ratio x_j = (q_j - b_j) + K (K: any constant),
+//   KL = sum_j p_j (log p_j - log r_j) = -E_p[x] + ln E_p[e^x]
+//      = -A/S + log1p(B/S),   S = sum e_j,  A = sum e_j x_j,
+//                             B = sum e_j (e^x_j - 1) = sum (h_j - e_j),
+// where e_j = 2^(b_j*L - R_b) are base weights in a frame R_b near the row
+// maximum and h_j = e_j e^x_j the matching quant weights. When the two rows
+// are close, A/S and log1p(B/S) are both O(sigma) and cancel to O(sigma^2),
+// so B is split as B = A + C with C = sum e_j phi(x_j), phi(y) = e^y - 1 - y
+// evaluated by a fitted polynomial (see phi_poly_fit.py): every term keeps
+// ~1e-7 relative accuracy and rounding errors of the exponentials enter only
+// at second order. Chunks where some |x| > 1.25 (or x is not finite: masked
+// or infinite entries) take a direct path that sums h_j = 2^(q_j*L - R_q)
+// with its own exponential instead. K follows (b - q) at the running maximum
+// of b (per warp), so x is ~0 where the base mass sits and the split keeps
+// its accuracy for peaked rows; moving K by d is an exact rebase in fp64:
+// A += d*S, C -> e^{ld} C + (e^{ld} - 1) l A + (e^{ld} - 1 - l d) S. L = log2(e)
+// rounded to fp32; all exponentials are of lambda*y with lambda = L*ln2
+// = 1 + 1.4e-8, i.e. the statistic of softmax(lambda*b) and softmax(lambda*q),
+// within 3e-8 relative of the exact one.
 //
-// Structure (one CTA per row at a time, persistent over rows):
-//   - warp 8 (producer): one lane streams the row's 16-byte-aligned body in
-//     32 KB tiles per operand into a 3-stage shared-memory ring with
-//     cp.async.bulk (no multicast), completing on mbarriers; it runs ahead
-//     across row boundaries.
-//   - warps 0..7 (consumers): each takes 1024-element chunks of a tile (32
-//     elements per lane, conflict-free 16-byte shared loads). Per chunk: lane
-//     max, warp max (redux.sync), a warp-uniform reference raise when the
-//     max grew, then 2 exp2 + a few FMA per element pair in fp32, folded
-//     into per-lane fp64 accumulators once per chunk.
-//   - argmax: each lane remembers the first chunk in which its own maximum
-//     appeared (strict >, increasing index order); at the end of the row
-//     only lanes whose maximum equals the row maximum re-read that chunk's
-//     32 elements to find the lowest matching index.
-//   - the unaligned head/tail (< 16 bytes each) is read directly by warp 0.
-//   - all intra-CTA waits are mbarrier waits bounded by wall time; a wait
-//     that gives up sets an error bit the reduction reports.
+// Structure (one CTA per SM, persistent over rows r = blockIdx.x + k*grid):
+//   - warp 16 (producer): one lane streams the 16-byte-aligned body of each
+//     row pair in 32 KB tiles per operand into a 3-stage shared-memory ring
+//     with cp.async.bulk (no multicast) completing on mbarriers, running
+//     ahead across row boundaries.
+//   - warps 0..15 (consumers): 512-element chunks (16 elements per lane,
+//     conflict-free 16-byte shared loads): lane and warp maxima (redux.sync),
+//     a warp-uniform frame raise when the maximum grew, then the fp32 terms
+//     of the chunk folded into per-lane fp64 accumulators. Each lane also
+//     remembers the first chunk in which its own maxima appeared. At the end
+//     of a row each warp reduces its accumulators and publishes them in a
+//     4-slot shared ring, then goes on with the next row.
+//   - warp 17 (epilogue): per row, the unaligned head/tail (< 16 bytes each)
+//     and the token gather, the exact lowest-index argmax (re-reading only
+//     the chunks of lanes whose maximum equals the row maximum), the fp64
+//     combine of the 17 partials and the 32-byte record.
+//   All waits are mbarrier waits bounded by wall time; a wait that gives up
+//   sets an error bit that the reduction reports, and the CTA leaves only
+//   after its bulk copies have landed.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -49,10 +59,31 @@ namespace kld {
 namespace {
 
 constexpr float kLog2e = 1.4426950408889634f;  // log2(e) rounded to fp32
-constexpr double kLog2eD = static_cast<double>(kLog2e);  // the same value
-constexpr double kLn2 = 0.6931471805599453;    // ln(2)
-constexpr float kNegBig = -1.0e30f;
+constexpr double kLog2eD = static_cast<double>(kLog2e);
+constexpr double kLn2 = 0.6931471805599453;  // ln(2)
+constexpr double kLambda = kLog2eD * kLn2;   // 1 + 1.4e-8
+constexpr float kBig = 1.0e30f;
+constexpr float kTau = 2.5f;                 // |x| bound of the polynomial path
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
+
+// phi(y) = y^2 * P(y), P of degree 8 fitted on [-2.5, 2.5]
+// (phi_poly_fit.py, max relative error of phi in fp32 9e-7); the kernel
+// evaluates phi(lambda*x) = x^2 * Q(x), Q_k = P_k * lambda^(k+2).
+constexpr double kP0 = 0.4999997655, kP1 = 0.1666656346, kP2 = 0.0416678794,
+                 kP3 = 0.008335872564, kP4 = 0.00138800956, kP5 = 0.0001968192101,
+                 kP6 = 2.495779646e-05, kP7 = 3.111933302e-06, kP8 = 2.814820757e-07;
+constexpr double lam_pow(int n) { return n == 0 ? 1.0 : kLambda * lam_pow(n - 1); }
+constexpr float kQ0 = static_cast<float>(kP0 * lam_pow(2));
+constexpr float kQ1 = static_cast<float>(kP1 * lam_pow(3));
+constexpr float kQ2 = static_cast<float>(kP2 * lam_pow(4));
+constexpr float kQ3 = static_cast<float>(kP3 * lam_pow(5));
+constexpr float kQ4 = static_cast<float>(kP4 * lam_pow(6));
+constexpr float kQ5 = static_cast<float>(kP5 * lam_pow(7));
+constexpr float kQ6 = static_cast<float>(kP6 * lam_pow(8));
+constexpr float kQ7 = static_cast<float>(kP7 * lam_pow(9));
+constexpr float kQ8 = static_cast<float>(kP8 * lam_pow(10));
+
+constexpr int kProducerWarp = kConsumerWarps;
 
 // ------------------------------------------------------------- PTX helpers
 
@@ -88,8 +119,7 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 }
 // Wait for the phase of `parity` to complete; gives up after kWaitLimitNs or
 // as soon as another thread of the CTA has raised *abort.
-__device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity,
-                                       volatile int* abort) {
+__device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer();
   for (uint32_t i = 1;; ++i) {
@@ -105,9 +135,8 @@ __device__ __forceinline__ uint64_t evict_first_policy() {
   asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
   return pol;
 }
-__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src,
-                                          uint32_t bytes, uint32_t bar,
-                                          uint64_t policy) {
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes,
+                                          uint32_t bar, uint64_t policy) {
   asm volatile(
       "cp.async.bulk.shared::cta.global.mbarrier::complete_tx::bytes.L2::cache_hint"
       " [%0], [%1], %2, [%3], %4;" ::"r"(dst),
@@ -128,6 +157,68 @@ __device__ __forceinline__ float max3(float a, float b, float c) {
   float y;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(y) : "f"(a), "f"(b), "f"(c));
   return y;
+}
+// Packed pairs of fp32 (sm_100 f32x2 arithmetic: one issue slot for two
+// lanes of FMA-pipe work).
+struct f2 {
+  unsigned long long v;
+};
+__device__ __forceinline__ f2 pk(float a, float b) {
+  f2 r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r.v) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ void upk(f2 x, float& a, float& b) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(x.v));
+}
+__device__ __forceinline__ f2 add2(f2 a, f2 b) {
+  f2 r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r.v) : "l"(a.v), "l"(b.v));
+  return r;
+}
+__device__ __forceinline__ f2 sub2(f2 a, f2 b) {
+  f2 r;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r.v) : "l"(a.v), "l"(b.v));
+  return r;
+}
+__device__ __forceinline__ f2 mul2(f2 a, f2 b) {
+  f2 r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r.v) : "l"(a.v), "l"(b.v));
+  return r;
+}
+__device__ __forceinline__ f2 fma2(f2 a, f2 b, f2 c) {
+  f2 r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r.v) : "l"(a.v), "l"(b.v), "l"(c.v));
+  return r;
+}
+__device__ __forceinline__ f2 splat(float a) { return pk(a, a); }
+
+// phi(lambda*x) / x^2 by Horner (scalar and packed).
+__device__ __forceinline__ float phi_q(float x) {
+  float q = fmaf(kQ8, x, kQ7);
+  q = fmaf(q, x, kQ6);
+  q = fmaf(q, x, kQ5);
+  q = fmaf(q, x, kQ4);
+  q = fmaf(q, x, kQ3);
+  q = fmaf(q, x, kQ2);
+  q = fmaf(q, x, kQ1);
+  return fmaf(q, x, kQ0);
+}
+__device__ __forceinline__ f2 phi_q2(f2 x) {
+  f2 q = fma2(splat(kQ8), x, splat(kQ7));
+  q = fma2(q, x, splat(kQ6));
+  q = fma2(q, x, splat(kQ5));
+  q = fma2(q, x, splat(kQ4));
+  q = fma2(q, x, splat(kQ3));
+  q = fma2(q, x, splat(kQ2));
+  q = fma2(q, x, splat(kQ1));
+  return fma2(q, x, splat(kQ0));
+}
+
+__device__ __forceinline__ double warp_sum(double x) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+  return x;
 }
 
 // ------------------------------------------------------------ element types
@@ -190,106 +281,217 @@ struct Elem<KLD_F16> {
 
 // ------------------------------------------------------------- per-row state
 
-// Warp-uniform reference of one row operand pair.
-struct WarpRef {
+// Warp-uniform frames of one row operand pair.
+struct Ref {
   float Mb, Mq;  // running maxima seen by this warp (-inf before any)
-  float cb, cq;  // references: the running maxima once finite, 0 before
+  float Rb, Rq;  // integer frames floor(M*L) once M is finite, 0 before
+  float K;       // log-ratio centre: (b - q) at the running maximum of b
 };
 
-// Per-lane accumulators and argmax memory.
-struct LaneAcc {
-  double Sb, Sq, T;
-  float best_b, best_q;  // lane maximum over its chunks so far
-  int loc_b, loc_q;      // chunk in which it first appeared
+// Per-lane fp64 accumulators (see the file comment): S_b over all chunks;
+// Ap = sum e*x and C = sum e*phi over polynomial-path chunks; Ad = sum e*x,
+// Se = sum e and Sh = sum h over direct-path chunks. A = Ap + Ad.
+struct Acc {
+  double Sb, Ap, C, Ad, Se, Sh;
 };
 
-// Per-warp partial handed to the row combine.
+struct Best {
+  float b, q;  // lane maxima so far
+  int lb, lq;  // chunk in which each first appeared
+};
+
+// Per-warp partial handed to the epilogue warp.
 struct WarpPart {
-  float Mb, Mq, cb, cq;
-  double Sb, Sq, T;
+  float Mb, Mq, Rb, Rq, K;
+  int pad;
+  double Sb, Ap, C, Ad, Se, Sh;
+  unsigned cand_b, cand_q;  // lanes whose own maximum equals the warp maximum
+};
+
+struct Slot {
+  WarpPart part[kConsumerWarps];
+  int loc_b[kConsumerWarps][32];
+  int loc_q[kConsumerWarps][32];
 };
 
 struct Ctrl {
   unsigned long long full[kStages];
   unsigned long long empty[kStages];
-  unsigned long long part_bar;
-  unsigned long long cand_bar;
-  WarpPart part[2][kConsumerWarps];
-  int amax[2][2];
+  unsigned long long slot_full[kSlots];
+  unsigned long long slot_empty[kSlots];
   int abort;
+  int pad;
+  Slot slot[kSlots];
 };
 static_assert(sizeof(Ctrl) <= kRowCtrlBytes, "control block too large");
 
-__device__ __forceinline__ void raise_base(float wmax, WarpRef& r, LaneAcc& a) {
-  if (r.Mb != -INFINITY) {  // accumulators are exactly 0 before any finite max
-    const double d = (static_cast<double>(wmax) - static_cast<double>(r.cb)) * kLog2eD;
-    const double sc = exp2(-d);
-    a.T = (a.T - d * a.Sb) * sc;
-    a.Sb *= sc;
+// Exact 2^k for an integer-valued difference of frames (0 on underflow).
+__device__ __forceinline__ double pow2i(float k) {
+  return ldexp(1.0, static_cast<int>(fmaxf(k, -2000.f)));
+}
+
+// One step of PE element pairs per lane (a 16-element consumer chunk, or the
+// head/tail elements one per lane). Elements whose bit in `valid` is clear
+// are absent (b = q = -inf, x = 0: they contribute nothing).
+template <int PE>
+__device__ __forceinline__ void chunk_step(const float* b, const float* q, unsigned valid,
+                                           Ref& r, Acc& a, Best& best, int chunk_id) {
+  float mb = b[0], mq = q[0];
+#pragma unroll
+  for (int i = 1; i + 1 < PE; i += 2) {
+    mb = max3(mb, b[i], b[i + 1]);
+    mq = max3(mq, q[i], q[i + 1]);
   }
-  r.cb = wmax;
-  r.Mb = wmax;
-}
-
-__device__ __forceinline__ void raise_quant(float wmax, WarpRef& r, LaneAcc& a) {
-  const double d = (static_cast<double>(wmax) - static_cast<double>(r.cq)) * kLog2eD;
-  a.T += d * a.Sb;
-  if (r.Mq != -INFINITY) a.Sq *= exp2(-d);
-  r.cq = wmax;
-  r.Mq = wmax;
-}
-
-// Accumulate 32 element pairs per lane (already widened to fp32) whose warp
-// maxima are wmb / wmq and lane maxima mb / mq.
-__device__ __forceinline__ void accumulate32(const float* xb, const float* xq,
-                                             float mb, float mq, WarpRef& ref,
-                                             LaneAcc& acc, int chunk_id) {
+  if (PE % 2 == 0) {
+    mb = fmaxf(mb, b[PE - 1]);
+    mq = fmaxf(mq, q[PE - 1]);
+  }
   const float wmb = warp_max(mb);
   const float wmq = warp_max(mq);
-  if (wmb > ref.Mb) raise_base(wmb, ref, acc);
-  if (wmq > ref.Mq) raise_quant(wmq, ref, acc);
-  const float cb = ref.cb, cq = ref.cq;
-  float sb0 = 0.f, sb1 = 0.f, sq0 = 0.f, sq1 = 0.f, t0 = 0.f, t1 = 0.f;
+  if (wmb > r.Mb) {  // raise the base frame and move the centre (warp-uniform)
+    // New centre: (b - q) at the lowest lane's first element holding wmb.
+    float dl = 0.f;
+    bool has = false;
 #pragma unroll
-  for (int i = 0; i < 32; i += 2) {
-    const float u0 = __fmul_rn(__fsub_rn(xb[i], cb), kLog2e);
-    const float v0 = __fmul_rn(__fsub_rn(xq[i], cq), kLog2e);
-    const float u1 = __fmul_rn(__fsub_rn(xb[i + 1], cb), kLog2e);
-    const float v1 = __fmul_rn(__fsub_rn(xq[i + 1], cq), kLog2e);
-    const float e0 = ex2(u0), f0 = ex2(v0);
-    const float e1 = ex2(u1), f1 = ex2(v1);
-    sb0 += e0;
-    sq0 += f0;
-    sb1 += e1;
-    sq1 += f1;
-    // d < -1e30 only where 2^u underflows to 0; the clamp turns the
-    // (-inf) - (-inf) of masked entries into a harmless finite value.
-    t0 = fmaf(e0, fmaxf(u0 - v0, kNegBig), t0);
-    t1 = fmaf(e1, fmaxf(u1 - v1, kNegBig), t1);
+    for (int i = 0; i < PE; ++i) {
+      if (!has && b[i] == wmb) {
+        dl = b[i] - q[i];
+        has = true;
+      }
+    }
+    const unsigned who = __ballot_sync(0xffffffffu, has);
+    const float Kn = __shfl_sync(0xffffffffu, dl, __ffs(who) - 1);
+    const float nR = floorf(wmb * kLog2e);
+    if (isfinite(Kn)) {
+      const double d = static_cast<double>(Kn) - static_cast<double>(r.K);
+      if (r.Mb != -INFINITY) {
+        // e^{ld} - 1 = l d + phi(l d); phi from the same polynomial when
+        // |d| is in its range, so the (e^{ld} - 1 - l d) term stays exact.
+        double ph;
+        if (fabs(d) <= static_cast<double>(kTau)) {
+          const float df = static_cast<float>(d);
+          ph = static_cast<double>(df * df * phi_q(df));
+        } else {
+          ph = expm1(kLambda * d) - kLambda * d;
+        }
+        const double em = kLambda * d + ph;
+        if (isfinite(em)) {
+          const double Sp = a.Sb - a.Se;
+          a.C = (em + 1.0) * a.C + em * kLambda * a.Ap + ph * Sp;
+          a.Ap += d * Sp;
+          a.Ad += d * a.Se;
+          r.K = Kn;
+        }
+      } else {
+        // First finite maximum: only direct-path terms of masked base
+        // entries (e = 0) can have been accumulated.
+        a.Ad += d * a.Se;
+        r.K = Kn;
+      }
+    }
+    if (r.Mb != -INFINITY) {
+      const double sc = pow2i(r.Rb - nR);  // exact power of two
+      a.Sb *= sc;
+      a.Ap *= sc;
+      a.C *= sc;
+      a.Ad *= sc;
+      a.Se *= sc;
+    }
+    r.Rb = nR;
+    r.Mb = wmb;
   }
-  acc.Sb += static_cast<double>(sb0 + sb1);
-  acc.Sq += static_cast<double>(sq0 + sq1);
-  acc.T += static_cast<double>(t0 + t1);
-  if (mb > acc.best_b) {
-    acc.best_b = mb;
-    acc.loc_b = chunk_id;
+  if (wmq > r.Mq) {  // raise the quant frame (direct-path sums only)
+    const float nR = floorf(wmq * kLog2e);
+    if (r.Mq != -INFINITY) a.Sh *= pow2i(r.Rq - nR);
+    r.Rq = nR;
+    r.Mq = wmq;
   }
-  if (mq > acc.best_q) {
-    acc.best_q = mq;
-    acc.loc_q = chunk_id;
+
+  // Log-ratios x = (q - b) + K, in packed pairs.
+  constexpr int NP = (PE + 1) / 2;
+  f2 X[NP];
+  bool ok = true;
+  const f2 K2 = splat(r.K);
+#pragma unroll
+  for (int j = 0; j < NP; ++j) {
+    const int i0 = 2 * j, i1 = (2 * j + 1 < PE) ? 2 * j + 1 : 2 * j;
+    X[j] = add2(sub2(pk(q[i0], q[i1]), pk(b[i0], b[i1])), K2);
+    float x0, x1;
+    upk(X[j], x0, x1);
+    if (((valid >> i0) & 1u) == 0u) x0 = 0.f;
+    if (((valid >> i1) & 1u) == 0u || i1 == i0) x1 = 0.f;
+    X[j] = pk(x0, x1);
+    ok &= fabsf(x0) <= kTau;  // false for NaN
+    ok &= fabsf(x1) <= kTau;
+  }
+  if (__all_sync(0xffffffffu, ok)) {
+    // Polynomial path: every pair finite with |x| <= 2.5.
+    const f2 L2 = splat(kLog2e), nR2 = splat(-r.Rb);
+    f2 SB = splat(0.f), SA = splat(0.f), SC = splat(0.f);
+#pragma unroll
+    for (int j = 0; j < NP; ++j) {
+      const int i0 = 2 * j, i1 = (2 * j + 1 < PE) ? 2 * j + 1 : 2 * j;
+      float u0, u1;
+      upk(fma2(pk(b[i0], b[i1]), L2, nR2), u0, u1);
+      const f2 E = pk(ex2(u0), i1 == i0 ? 0.f : ex2(u1));
+      const f2 T = mul2(E, X[j]);
+      SB = add2(SB, E);
+      SA = add2(SA, T);
+      SC = fma2(mul2(T, X[j]), phi_q2(X[j]), SC);
+    }
+    float sb0, sb1, sa0, sa1, sc0, sc1;
+    upk(SB, sb0, sb1);
+    upk(SA, sa0, sa1);
+    upk(SC, sc0, sc1);
+    a.Sb += static_cast<double>(sb0) + static_cast<double>(sb1);
+    a.Ap += static_cast<double>(sa0) + static_cast<double>(sa1);
+    a.C += static_cast<double>(sc0) + static_cast<double>(sc1);
+  } else {
+    // Direct path: quant weights in their own frame. x -> +BIG keeps 0*x = 0
+    // for masked base entries; x = -inf (quant masked, base finite) makes A
+    // -inf, i.e. KL = +inf.
+    const float nRb = -r.Rb, nRq = -r.Rq;
+    float sb = 0.f, sa = 0.f, sh = 0.f;
+#pragma unroll
+    for (int j = 0; j < NP; ++j) {
+      float x0, x1;
+      upk(X[j], x0, x1);
+      const float xs[2] = {x0, x1};
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int i = 2 * j + h;
+        if (i < PE) {
+          const float e = ex2(fmaf(b[i], kLog2e, nRb));
+          sb += e;
+          sa = fmaf(e, fminf(xs[h], kBig), sa);
+          sh += ex2(fmaf(q[i], kLog2e, nRq));
+        }
+      }
+    }
+    a.Sb += static_cast<double>(sb);
+    a.Se += static_cast<double>(sb);
+    a.Ad += static_cast<double>(sa);
+    a.Sh += static_cast<double>(sh);
+  }
+  if (mb > best.b) {
+    best.b = mb;
+    best.lb = chunk_id;
+  }
+  if (mq > best.q) {
+    best.q = mq;
+    best.lq = chunk_id;
   }
 }
 
-// One 1024-element chunk of the current tile. `valid_vecs` < 32*VPC marks a
-// ragged last chunk whose vectors beyond it are treated as -inf.
+// One 512-element chunk of the current tile (16 elements per lane).
 template <int DT, bool kMasked>
-__device__ __forceinline__ void process_chunk(const uint4* cb, const uint4* cq,
-                                              int lane, int valid_vecs,
-                                              WarpRef& ref, LaneAcc& acc,
+__device__ __forceinline__ void process_chunk(const uint4* cb, const uint4* cq, int lane,
+                                              int valid_vecs, Ref& r, Acc& a, Best& best,
                                               int chunk_id) {
   constexpr int E = Elem<DT>::kPerVec;
-  constexpr int VPC = 32 / E;
-  float xb[32], xq[32];
+  constexpr int VPC = kLaneElems / E;
+  float xb[kLaneElems], xq[kLaneElems];
+  unsigned valid = (1u << kLaneElems) - 1u;
 #pragma unroll
   for (int k = 0; k < VPC; ++k) {
     const int vi = k * 32 + lane;
@@ -298,6 +500,7 @@ __device__ __forceinline__ void process_chunk(const uint4* cb, const uint4* cq,
     Elem<DT>::unpack(vb, &xb[k * E]);
     Elem<DT>::unpack(vq, &xq[k * E]);
     if (kMasked && vi >= valid_vecs) {
+      valid &= ~(((1u << E) - 1u) << (k * E));
 #pragma unroll
       for (int i = 0; i < E; ++i) {
         xb[k * E + i] = -INFINITY;
@@ -305,40 +508,7 @@ __device__ __forceinline__ void process_chunk(const uint4* cb, const uint4* cq,
       }
     }
   }
-  float mb = max3(xb[0], xb[1], xb[2]);
-  float mq = max3(xq[0], xq[1], xq[2]);
-#pragma unroll
-  for (int i = 3; i < 31; i += 2) {
-    mb = max3(mb, xb[i], xb[i + 1]);
-    mq = max3(mq, xq[i], xq[i + 1]);
-  }
-  mb = fmaxf(mb, xb[31]);
-  mq = fmaxf(mq, xq[31]);
-  accumulate32(xb, xq, mb, mq, ref, acc, chunk_id);
-}
-
-// Lowest index in a lane's chunk whose value equals m (INT_MAX if none).
-template <int DT>
-__device__ int rescan_chunk(const void* row, int64_t body_start, int64_t body_len,
-                            int chunk_id, int lane, float m) {
-  constexpr int E = Elem<DT>::kPerVec;
-  constexpr int VPC = 32 / E;
-  const int64_t c0 = static_cast<int64_t>(chunk_id) * kChunkElems;
-  for (int k = 0; k < VPC; ++k) {
-    for (int i = 0; i < E; ++i) {
-      const int64_t off = c0 + static_cast<int64_t>(k * 32 + lane) * E + i;
-      if (off >= body_len) return INT_MAX;
-      if (Elem<DT>::load(row, body_start + off) == m)
-        return static_cast<int>(body_start + off);
-    }
-  }
-  return INT_MAX;
-}
-
-__device__ __forceinline__ double warp_sum(double x) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
-  return x;
+  chunk_step<kLaneElems>(xb, xq, valid, r, a, best, chunk_id);
 }
 
 __device__ __forceinline__ void fail(Ctrl* ctrl, uint32_t* derr) {
@@ -367,6 +537,36 @@ __device__ __forceinline__ RowGeom row_geom(const void* rowb, int64_t V) {
   return g;
 }
 
+// Offset (within the body) of element i of lane `lane` in chunk `chunk_id`.
+template <int DT>
+__device__ __forceinline__ int64_t chunk_elem_offset(int chunk_id, int lane, int i) {
+  constexpr int E = Elem<DT>::kPerVec;
+  return static_cast<int64_t>(chunk_id) * kChunkElems +
+         static_cast<int64_t>((i / E) * 32 + lane) * E + (i % E);
+}
+
+// Lowest index holding `m` among the candidate lanes (mask) of one warp's
+// published partial; lanes 0..15 of the calling warp each test one element.
+template <int DT>
+__device__ int rescan_candidates(const void* row, const RowGeom& g, unsigned mask,
+                                 const int* locs, float m, int lane) {
+  int best = INT_MAX;
+  while (mask) {
+    const int cl = __ffs(mask) - 1;
+    mask &= mask - 1u;
+    const int loc = locs[cl];
+    int idx = INT_MAX;
+    if (lane < kLaneElems && loc >= 0) {
+      const int64_t off = chunk_elem_offset<DT>(loc, cl, lane);
+      if (off < g.body_len && Elem<DT>::load(row, g.head + off) == m)
+        idx = static_cast<int>(g.head + off);
+    }
+    idx = __reduce_min_sync(0xffffffffu, idx);
+    if (idx < best) best = idx;
+  }
+  return best;
+}
+
 template <int DT>
 __global__ void __launch_bounds__(kRowThreads, 1)
     kld_rows_kernel(const void* __restrict__ base, const void* __restrict__ quant,
@@ -391,10 +591,10 @@ __global__ void __launch_bounds__(kRowThreads, 1)
       mbar_init(smem_u32(&ctrl->full[s]), 1);
       mbar_init(smem_u32(&ctrl->empty[s]), kConsumerWarps);
     }
-    mbar_init(smem_u32(&ctrl->part_bar), kConsumerWarps);
-    mbar_init(smem_u32(&ctrl->cand_bar), kConsumerWarps);
-    ctrl->amax[0][0] = ctrl->amax[0][1] = INT_MAX;
-    ctrl->amax[1][0] = ctrl->amax[1][1] = INT_MAX;
+    for (int s = 0; s < kSlots; ++s) {
+      mbar_init(smem_u32(&ctrl->slot_full[s]), kConsumerWarps);
+      mbar_init(smem_u32(&ctrl->slot_empty[s]), 1);
+    }
     ctrl->abort = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -403,7 +603,7 @@ __global__ void __launch_bounds__(kRowThreads, 1)
   const char* B = static_cast<const char*>(base);
   const char* Q = static_cast<const char*>(quant);
 
-  if (warp == kConsumerWarps) {
+  if (warp == kProducerWarp) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       const uint64_t pol = evict_first_policy();
@@ -453,182 +653,237 @@ __global__ void __launch_bounds__(kRowThreads, 1)
     return;
   }
 
-  // ---------------------------------------------------------------- consumers
-  uint32_t it = 0;
+  if (warp < kConsumerWarps) {
+    // ----------------------------------------------------------- consumers
+    uint32_t it = 0;
+    int rowk = 0;
+    for (int64_t r = blockIdx.x; r < N; r += gridDim.x, ++rowk) {
+      const char* rb = B + r * V * EB;
+      const RowGeom g = row_geom<DT>(rb, V);
+      Ref ref{-INFINITY, -INFINITY, 0.f, 0.f, 0.f};
+      Acc acc{0.0, 0.0, 0.0, 0.0, 0.0, 0.0};
+      Best best{-INFINITY, -INFINITY, -1, -1};
+      for (int64_t t = 0; t < g.ntiles; ++t, ++it) {
+        const int s = static_cast<int>(it % kStages);
+        const uint32_t ph = (it / kStages) & 1u;
+        if (!mbar_wait(smem_u32(&ctrl->full[s]), ph, abort)) {
+          fail(ctrl, derr);
+          return;
+        }
+        int64_t len = g.body_len - t * kStageElems;
+        if (len > kStageElems) len = kStageElems;
+        const uint4* tb = reinterpret_cast<const uint4*>(stage_b + s * kStageBytes);
+        const uint4* tq = reinterpret_cast<const uint4*>(stage_q + s * kStageBytes);
+#pragma unroll 1
+        for (int c = warp; c < kChunksPerTile; c += kConsumerWarps) {
+          const int cstart = c * kChunkElems;
+          if (cstart >= len) break;
+          const int gid = static_cast<int>(t) * kChunksPerTile + c;
+          const uint4* cb = tb + cstart / E;
+          const uint4* cq = tq + cstart / E;
+          if (cstart + kChunkElems <= len) {
+            process_chunk<DT, false>(cb, cq, lane, 0, ref, acc, best, gid);
+          } else {
+            process_chunk<DT, true>(cb, cq, lane, static_cast<int>((len - cstart) / E), ref, acc,
+                                    best, gid);
+          }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&ctrl->empty[s]));
+      }
+
+      // Publish the warp partial into the slot ring.
+      const int slot = rowk % kSlots;
+      const uint32_t sph = (rowk / kSlots) & 1u;
+      const double Sb = warp_sum(acc.Sb), Ap = warp_sum(acc.Ap), C = warp_sum(acc.C);
+      const double Ad = warp_sum(acc.Ad), Se = warp_sum(acc.Se), Sh = warp_sum(acc.Sh);
+      const unsigned cb_mask = __ballot_sync(0xffffffffu, ref.Mb > -INFINITY && best.b == ref.Mb);
+      const unsigned cq_mask = __ballot_sync(0xffffffffu, ref.Mq > -INFINITY && best.q == ref.Mq);
+      if (!mbar_wait(smem_u32(&ctrl->slot_empty[slot]), sph ^ 1u, abort)) {
+        fail(ctrl, derr);
+        return;
+      }
+      Slot& sl = ctrl->slot[slot];
+      if ((cb_mask >> lane) & 1u) sl.loc_b[warp][lane] = best.lb;
+      if ((cq_mask >> lane) & 1u) sl.loc_q[warp][lane] = best.lq;
+      if (lane == 0) {
+        WarpPart p;
+        p.Mb = ref.Mb;
+        p.Mq = ref.Mq;
+        p.Rb = ref.Rb;
+        p.Rq = ref.Rq;
+        p.K = ref.K;
+        p.pad = 0;
+        p.Sb = Sb;
+        p.Ap = Ap;
+        p.C = C;
+        p.Ad = Ad;
+        p.Se = Se;
+        p.Sh = Sh;
+        p.cand_b = cb_mask;
+        p.cand_q = cq_mask;
+        sl.part[warp] = p;
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&ctrl->slot_full[slot]));
+    }
+    return;
+  }
+
+  // ------------------------------------------------------------------ epilogue
   int rowk = 0;
   for (int64_t r = blockIdx.x; r < N; r += gridDim.x, ++rowk) {
     const char* rb = B + r * V * EB;
     const char* rq = Q + r * V * EB;
     const RowGeom g = row_geom<DT>(rb, V);
-    const int pb = rowk & 1;
 
-    WarpRef ref{-INFINITY, -INFINITY, 0.f, 0.f};
-    LaneAcc acc{0.0, 0.0, 0.0, -INFINITY, -INFINITY, -1, -1};
-
-    // Head/tail elements (warp 0), loaded now and used at the row end.
+    // Head/tail elements (one per lane) and the next-token gather, issued
+    // before waiting for the consumers' partials.
+    const int n_extra = static_cast<int>(g.head + g.tail);
     float xe_b = -INFINITY, xe_q = -INFINITY;
     int idx_e = INT_MAX;
-    const int n_extra = static_cast<int>(g.head + g.tail);
-    if (warp == 0 && lane < n_extra) {
+    if (lane < n_extra) {
       const int64_t j = lane < g.head ? lane : g.head + g.body_len + (lane - g.head);
       idx_e = static_cast<int>(j);
       xe_b = Elem<DT>::load(rb, j);
       xe_q = Elem<DT>::load(rq, j);
     }
-    // Next-token gather (thread 0), also issued early.
     int32_t tk = 0;
     bool tok_ok = false;
     float q_tok = 0.f;
-    if (threadIdx.x == 0 && tok != nullptr) {
+    if (tok != nullptr) {
       tk = __ldg(tok + r);
       tok_ok = tk >= 0 && static_cast<int64_t>(tk) < V;
-      if (tok_ok) q_tok = Elem<DT>::load(rq, tk);
+      if (tok_ok && lane == 0) q_tok = Elem<DT>::load(rq, tk);
     }
 
-    bool ok = true;
-    for (int64_t t = 0; t < g.ntiles; ++t, ++it) {
-      const int s = static_cast<int>(it % kStages);
-      const uint32_t ph = (it / kStages) & 1u;
-      if (!mbar_wait(smem_u32(&ctrl->full[s]), ph, abort)) {
-        fail(ctrl, derr);
-        ok = false;
-        break;
-      }
-      int64_t len = g.body_len - t * kStageElems;
-      if (len > kStageElems) len = kStageElems;
-      const uint4* tb = reinterpret_cast<const uint4*>(stage_b + s * kStageBytes);
-      const uint4* tq = reinterpret_cast<const uint4*>(stage_q + s * kStageBytes);
-      for (int c = warp; c < kChunksPerTile; c += kConsumerWarps) {
-        const int cstart = c * kChunkElems;
-        if (cstart >= len) break;
-        const int gid = static_cast<int>(t) * kChunksPerTile + c;
-        const uint4* cb = tb + cstart / E;
-        const uint4* cq = tq + cstart / E;
-        if (cstart + kChunkElems <= len) {
-          process_chunk<DT, false>(cb, cq, lane, 0, ref, acc, gid);
-        } else {
-          process_chunk<DT, true>(cb, cq, lane, static_cast<int>((len - cstart) / E),
-                                  ref, acc, gid);
-        }
-      }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&ctrl->empty[s]));
+    // The head/tail as one more partial of the same form.
+    Ref eref{-INFINITY, -INFINITY, 0.f, 0.f, 0.f};
+    Acc eacc{0.0, 0.0, 0.0, 0.0, 0.0, 0.0};
+    Best ebest{-INFINITY, -INFINITY, -1, -1};
+    if (n_extra > 0) {
+      chunk_step<1>(&xe_b, &xe_q, lane < n_extra ? 1u : 0u, eref, eacc, ebest, 0);
     }
-    if (!ok) return;
+    const double eSb = warp_sum(eacc.Sb), eAp = warp_sum(eacc.Ap), eC = warp_sum(eacc.C);
+    const double eAd = warp_sum(eacc.Ad), eSe = warp_sum(eacc.Se), eSh = warp_sum(eacc.Sh);
 
-    // Head/tail as one more (sparse) step of warp 0: one element per lane.
-    if (warp == 0 && n_extra > 0) {
-      const float wmb = warp_max(xe_b);
-      const float wmq = warp_max(xe_q);
-      if (wmb > ref.Mb) raise_base(wmb, ref, acc);
-      if (wmq > ref.Mq) raise_quant(wmq, ref, acc);
-      const float u = __fmul_rn(__fsub_rn(xe_b, ref.cb), kLog2e);
-      const float v = __fmul_rn(__fsub_rn(xe_q, ref.cq), kLog2e);
-      const float e = ex2(u);
-      acc.Sb += static_cast<double>(e);
-      acc.Sq += static_cast<double>(ex2(v));
-      acc.T += static_cast<double>(e * fmaxf(u - v, kNegBig));
-    }
-
-    // Warp partial -> shared memory.
-    const double Sb = warp_sum(acc.Sb);
-    const double Sq = warp_sum(acc.Sq);
-    const double T = warp_sum(acc.T);
-    if (lane == 0) ctrl->part[pb][warp] = WarpPart{ref.Mb, ref.Mq, ref.cb, ref.cq, Sb, Sq, T};
-    __syncwarp();
-    if (lane == 0) mbar_arrive(smem_u32(&ctrl->part_bar));
-    if (!mbar_wait(smem_u32(&ctrl->part_bar), rowk & 1, abort)) {
+    const int slot = rowk % kSlots;
+    const uint32_t sph = (rowk / kSlots) & 1u;
+    if (!mbar_wait(smem_u32(&ctrl->slot_full[slot]), sph, abort)) {
       fail(ctrl, derr);
       return;
     }
+    const Slot& sl = ctrl->slot[slot];
 
-    // Row maxima, then the lowest index holding each.
-    float Mb = -INFINITY, Mq = -INFINITY;
-#pragma unroll
-    for (int w = 0; w < kConsumerWarps; ++w) {
-      Mb = fmaxf(Mb, ctrl->part[pb][w].Mb);
-      Mq = fmaxf(Mq, ctrl->part[pb][w].Mq);
-    }
-    const bool finite_max = Mb > -INFINITY && Mb < INFINITY && Mq > -INFINITY && Mq < INFINITY;
-    if (finite_max) {
-      int cb_idx = INT_MAX, cq_idx = INT_MAX;
-      if (acc.best_b == Mb) cb_idx = rescan_chunk<DT>(rb, g.head, g.body_len, acc.loc_b, lane, Mb);
-      if (acc.best_q == Mq) cq_idx = rescan_chunk<DT>(rq, g.head, g.body_len, acc.loc_q, lane, Mq);
-      if (warp == 0 && xe_b == Mb && idx_e < cb_idx) cb_idx = idx_e;
-      if (warp == 0 && xe_q == Mq && idx_e < cq_idx) cq_idx = idx_e;
-      cb_idx = __reduce_min_sync(0xffffffffu, cb_idx);
-      cq_idx = __reduce_min_sync(0xffffffffu, cq_idx);
-      if (lane == 0) {
-        if (cb_idx != INT_MAX) atomicMin(&ctrl->amax[pb][0], cb_idx);
-        if (cq_idx != INT_MAX) atomicMin(&ctrl->amax[pb][1], cq_idx);
+    // Lane w < 16 takes warp w's partial, lane 16 the head/tail partial.
+    WarpPart p;
+    if (lane < kConsumerWarps) {
+      p = sl.part[lane];
+    } else {
+      p.Mb = p.Mq = -INFINITY;
+      p.Rb = p.Rq = p.K = 0.f;
+      p.pad = 0;
+      p.Sb = p.Ap = p.C = p.Ad = p.Se = p.Sh = 0.0;
+      p.cand_b = p.cand_q = 0u;
+      if (lane == kConsumerWarps) {
+        p.Mb = eref.Mb;
+        p.Mq = eref.Mq;
+        p.Rb = eref.Rb;
+        p.Rq = eref.Rq;
+        p.K = eref.K;
+        p.Sb = eSb;
+        p.Ap = eAp;
+        p.C = eC;
+        p.Ad = eAd;
+        p.Se = eSe;
+        p.Sh = eSh;
       }
+    }
+    const float Mb = warp_max(p.Mb);
+    const float Mq = warp_max(p.Mq);
+    const bool nan_part = isnan(p.Sb) || isnan(p.Sh) || isnan(p.C);
+    const bool nonfinite = __any_sync(0xffffffffu, nan_part) || !(Mb < INFINITY) ||
+                           !(Mq < INFINITY);
+    const bool empty = Mb == -INFINITY || Mq == -INFINITY;
+
+    uint32_t flags = 0;
+    if (tok != nullptr && !tok_ok) flags |= KLD_ROW_BAD_TOKEN;
+    double kl = __longlong_as_double(0x7ff8000000000000ll);  // NaN
+    double nll = kl;
+    int ab = -1, aq = -1;
+    if (nonfinite) {
+      flags |= KLD_ROW_NONFINITE;
+    } else if (empty) {
+      flags |= KLD_ROW_EMPTY;
+    } else {
+      // Common frames and centre.
+      const float Cb = warp_max(p.Mb > -INFINITY ? p.Rb : -INFINITY);
+      // Centre of the part that holds the row maximum of b.
+      const unsigned kmask = __ballot_sync(0xffffffffu, p.Mb == Mb);
+      const float Kref = __shfl_sync(0xffffffffu, p.K, __ffs(kmask) - 1);
+      // Only direct-path sums can be infinite: b_j finite where q_j = -inf.
+      const bool inf_kl = __any_sync(0xffffffffu, !isfinite(p.Ad));
+      const double dK = static_cast<double>(Kref) - static_cast<double>(p.K);
+      const double fb = p.Mb > -INFINITY ? pow2i(p.Rb - Cb) : 0.0;
+      // Polynomial-path part of B in the warp's own centre, moved to Kref:
+      // e^{l(x+d)} - 1 = e^{l d}(e^{l x} - 1) + (e^{l d} - 1).
+      const double Bp = kLambda * p.Ap + p.C;
+      const double Sp = p.Sb - p.Se;
+      const double em = expm1(kLambda * dK);
+      const double BpK = Bp + em * (Bp + Sp);
+      // Direct-path quant weights, from their own frame to Cb - Kref*L.
+      const double Bh = p.Mq > -INFINITY
+                            ? p.Sh * exp2(static_cast<double>(p.Rq) - static_cast<double>(Cb) +
+                                          static_cast<double>(Kref) * kLog2eD)
+                            : 0.0;
+      const double sb = warp_sum(p.Sb * fb);
+      const double sbB = warp_sum(BpK * fb + Bh - p.Se * fb);
+      const double sa = warp_sum(inf_kl ? 0.0 : (p.Ap + p.Ad + dK * p.Sb) * fb);
+      if (inf_kl) {
+        kl = INFINITY;
+        flags |= KLD_ROW_INF_KL;
+      } else {
+        kl = -kLambda * (sa / sb) + log1p(sbB / sb);
+      }
+      if (tok_ok) {
+        const float qt = __shfl_sync(0xffffffffu, q_tok, 0);
+        if (qt == -INFINITY) {
+          nll = INFINITY;
+          flags |= KLD_ROW_INF_NLL;
+        } else {
+          // B + S is the sum of all quant weights in frame Cb - Kref*L.
+          nll = log(sbB + sb) +
+                kLn2 * (static_cast<double>(Cb) -
+                        (static_cast<double>(Kref) + static_cast<double>(qt)) * kLog2eD);
+        }
+      }
+      // Lowest index of each row maximum.
+      int amb = (xe_b == Mb) ? idx_e : INT_MAX;
+      int amq = (xe_q == Mq) ? idx_e : INT_MAX;
+      amb = __reduce_min_sync(0xffffffffu, amb);
+      amq = __reduce_min_sync(0xffffffffu, amq);
+      unsigned wb = __ballot_sync(0xffffffffu, lane < kConsumerWarps && p.Mb == Mb);
+      unsigned wq = __ballot_sync(0xffffffffu, lane < kConsumerWarps && p.Mq == Mq);
+      while (wb) {
+        const int w = __ffs(wb) - 1;
+        wb &= wb - 1u;
+        const unsigned cm = __shfl_sync(0xffffffffu, p.cand_b, w);
+        const int i = rescan_candidates<DT>(rb, g, cm, sl.loc_b[w], Mb, lane);
+        if (i < amb) amb = i;
+      }
+      while (wq) {
+        const int w = __ffs(wq) - 1;
+        wq &= wq - 1u;
+        const unsigned cm = __shfl_sync(0xffffffffu, p.cand_q, w);
+        const int i = rescan_candidates<DT>(rq, g, cm, sl.loc_q[w], Mq, lane);
+        if (i < amq) amq = i;
+      }
+      ab = amb;
+      aq = amq;
     }
     __syncwarp();
-    if (lane == 0) mbar_arrive(smem_u32(&ctrl->cand_bar));
-
-    if (threadIdx.x == 0) {
-      if (!mbar_wait(smem_u32(&ctrl->cand_bar), rowk & 1, abort)) {
-        fail(ctrl, derr);
-        return;
-      }
-      uint32_t flags = 0;
-      if (tok != nullptr && !tok_ok) flags |= KLD_ROW_BAD_TOKEN;
-      bool nonfinite = !(Mb < INFINITY) || !(Mq < INFINITY);
-      for (int w = 0; w < kConsumerWarps; ++w) {
-        const WarpPart& p = ctrl->part[pb][w];
-        if (isnan(p.Sb) || isnan(p.Sq)) nonfinite = true;
-      }
-      double kl = __longlong_as_double(0x7ff8000000000000ll);  // NaN
-      double nll = kl;
-      int ab = -1, aq = -1;
-      if (nonfinite) {
-        flags |= KLD_ROW_NONFINITE;
-      } else if (Mb == -INFINITY || Mq == -INFINITY) {
-        flags |= KLD_ROW_EMPTY;
-      } else {
-        // Common references: the largest per-warp reference of warps that
-        // saw a finite maximum.
-        float Cb = -INFINITY, Cq = -INFINITY;
-        for (int w = 0; w < kConsumerWarps; ++w) {
-          const WarpPart& p = ctrl->part[pb][w];
-          if (p.Mb > -INFINITY) Cb = fmaxf(Cb, p.cb);
-          if (p.Mq > -INFINITY) Cq = fmaxf(Cq, p.cq);
-        }
-        double sb = 0.0, sq = 0.0, tt = 0.0;
-        bool inf_kl = false;
-        for (int w = 0; w < kConsumerWarps; ++w) {
-          const WarpPart& p = ctrl->part[pb][w];
-          const double dq = (static_cast<double>(Cq) - static_cast<double>(p.cq)) * kLog2eD;
-          if (p.Mb > -INFINITY) {
-            const double db = (static_cast<double>(Cb) - static_cast<double>(p.cb)) * kLog2eD;
-            const double sc = exp2(-db);
-            sb += p.Sb * sc;
-            if (!isfinite(p.T)) {
-              inf_kl = true;
-            } else {
-              tt += sc * (p.T - (db - dq) * p.Sb);
-            }
-          }
-          if (p.Mq > -INFINITY) sq += p.Sq * exp2(-dq);
-        }
-        if (inf_kl) {
-          kl = INFINITY;
-          flags |= KLD_ROW_INF_KL;
-        } else {
-          kl = kLn2 * (tt / sb) + log(sq / sb);
-        }
-        if (tok_ok) {
-          if (q_tok == -INFINITY) {
-            nll = INFINITY;
-            flags |= KLD_ROW_INF_NLL;
-          } else {
-            nll = log(sq) +
-                  kLn2 * ((static_cast<double>(Cq) - static_cast<double>(q_tok)) * kLog2eD);
-          }
-        }
-        ab = ctrl->amax[pb][0];
-        aq = ctrl->amax[pb][1];
-      }
+    if (lane == 0) {
+      mbar_arrive(smem_u32(&ctrl->slot_empty[slot]));
       kld_row_t rec;
       rec.kld = kl;
       rec.nll = nll;
@@ -637,8 +892,6 @@ __global__ void __launch_bounds__(kRowThreads, 1)
       rec.flags = flags;
       rec.reserved = 0u;
       rows[r] = rec;
-      ctrl->amax[pb][0] = INT_MAX;
-      ctrl->amax[pb][1] = INT_MAX;
     }
   }
 }
@@ -647,32 +900,32 @@ __global__ void __launch_bounds__(kRowThreads, 1)
 
 cudaError_t prepare_rows_kernels() {
   cudaError_t e;
-  e = cudaFuncSetAttribute(kld_rows_kernel<KLD_F32>,
-                           cudaFuncAttributeMaxDynamicSharedMemorySize, kRowSmemBytes);
+  e = cudaFuncSetAttribute(kld_rows_kernel<KLD_F32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           kRowSmemBytes);
   if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(kld_rows_kernel<KLD_BF16>,
-                           cudaFuncAttributeMaxDynamicSharedMemorySize, kRowSmemBytes);
+  e = cudaFuncSetAttribute(kld_rows_kernel<KLD_BF16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           kRowSmemBytes);
   if (e != cudaSuccess) return e;
   return cudaFuncSetAttribute(kld_rows_kernel<KLD_F16>,
                               cudaFuncAttributeMaxDynamicSharedMemorySize, kRowSmemBytes);
 }
 
-cudaError_t launch_rows(const void* base, const void* quant, const int32_t* token_ids,
-                        int64_t N, int64_t V, kld_dtype_t dtype, kld_row_t* rows,
-                        uint32_t* derr, int grid, cudaStream_t stream) {
+cudaError_t launch_rows(const void* base, const void* quant, const int32_t* token_ids, int64_t N,
+                        int64_t V, kld_dtype_t dtype, kld_row_t* rows, uint32_t* derr, int grid,
+                        cudaStream_t stream) {
   const dim3 g(static_cast<unsigned>(grid)), b(kRowThreads);
   switch (dtype) {
     case KLD_F32:
-      kld_rows_kernel<KLD_F32><<<g, b, kRowSmemBytes, stream>>>(base, quant, token_ids, N, V,
-                                                                 rows, derr);
+      kld_rows_kernel<KLD_F32><<<g, b, kRowSmemBytes, stream>>>(base, quant, token_ids, N, V, rows,
+                                                                 derr);
       break;
     case KLD_BF16:
       kld_rows_kernel<KLD_BF16><<<g, b, kRowSmemBytes, stream>>>(base, quant, token_ids, N, V,
                                                                   rows, derr);
       break;
     case KLD_F16:
-      kld_rows_kernel<KLD_F16><<<g, b, kRowSmemBytes, stream>>>(base, quant, token_ids, N, V,
-                                                                 rows, derr);
+      kld_rows_kernel<KLD_F16><<<g, b, kRowSmemBytes, stream>>>(base, quant, token_ids, N, V, rows,
+                                                                 derr);
       break;
     default:
       return cudaErrorInvalidValue;

@@ -3,7 +3,9 @@ and compare with the fp64 oracle at the stated tolerances.
 
 Tolerances: argmax indices, flags and agreement counts bit-exact; per-row KL
 and NLL |gpu - ref| <= 1e-6 + 1e-4 * |ref|; mean KLD, percentiles, mean NLL
-and PPL within 1e-5 relative (absolute floor 1e-12 for values near zero).
+and PPL within 1e-5 relative, with an absolute floor where the reference is
+~0 (1e-9 nats for KL statistics, 1e-7 nats for mean NLL, i.e. 1e-7 relative
+for PPL): fp32 inputs do not resolve a log-probability better than that.
 """
 from __future__ import annotations
 
@@ -19,7 +21,9 @@ from logit_kl_divergence_b200 import KLDStats, rows_view, synth
 ODT = {synth.F32: oracle.F32, synth.BF16: oracle.BF16, synth.F16: oracle.F16}
 EXCLUDED = oracle.ROW_NONFINITE | oracle.ROW_EMPTY
 ROW_ATOL, ROW_RTOL = 1e-6, 1e-4
-STAT_RTOL, STAT_ATOL = 1e-5, 1e-12
+STAT_RTOL = 1e-5
+STAT_ATOL = {"mean_kld": 1e-9, "median_kld": 1e-9, "p90_kld": 1e-9, "p99_kld": 1e-9,
+             "max_kld": 1e-9, "mean_nll": 1e-7, "top1_agree_pct": 0.0}
 CORES = max(1, os.cpu_count() or 1)
 
 
@@ -68,12 +72,14 @@ def assert_rows_match(g: dict, o: dict, idx=None):
     _close_rows(g["nll"], o["nll"], "nll", idx)
 
 
-def stat_close(a, b):
+def stat_close(a, b, key):
     if (isinstance(a, float) and math.isnan(a)) or (isinstance(b, float) and math.isnan(b)):
         return math.isnan(a) and math.isnan(b)
     if math.isinf(a) or math.isinf(b):
         return a == b
-    return abs(a - b) <= STAT_ATOL + STAT_RTOL * abs(b)
+    if key == "ppl":
+        return abs(a - b) <= (STAT_RTOL + 1e-7) * abs(b)
+    return abs(a - b) <= STAT_ATOL[key] + STAT_RTOL * abs(b)
 
 
 def assert_stats_match(gres: dict, ores: dict):
@@ -81,7 +87,7 @@ def assert_stats_match(gres: dict, ores: dict):
         assert int(gres[k]) == int(ores[k]), (k, gres[k], ores[k])
     for k in ("mean_kld", "median_kld", "p90_kld", "p99_kld", "max_kld", "top1_agree_pct",
               "mean_nll", "ppl"):
-        assert stat_close(gres[k], ores[k]), (k, gres[k], ores[k])
+        assert stat_close(gres[k], ores[k], k), (k, gres[k], ores[k])
     assert gres["device_error"] == 0
 
 
