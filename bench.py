@@ -80,48 +80,76 @@ def recorded_traffic(workload: str):
 
 
 class ClockSampler:
-    """nvidia-smi clock / throttle-reason samples during the timed region."""
+    """SM clock and throttle reasons sampled during the timed region: NVML
+    polled from a thread every ~2 ms (the region lasts tens of ms), with
+    nvidia-smi as the fallback."""
 
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = {  # NVML clocks-event reason bits
+        "hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
+        "hw_power_brake_slowdown": 0x80, "sw_power_cap": 0x4,
+    }
 
     def __init__(self, gpu_index: int):
-        self.proc = None
-        self.gpu = gpu_index
-        exe = shutil.which("nvidia-smi")
-        if exe:
-            self.proc = subprocess.Popen(
-                [exe, f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "100",
-                 "-i", str(gpu_index)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        import threading
+
+        self.samples, self.maxes, self.reasons = [], [], set()
+        self._stop = threading.Event()
+        self._thread = None
+        self._proc = None
+        try:
+            import pynvml
+
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(gpu_index)
+            self._thread = threading.Thread(target=self._poll, daemon=True)
+            self._thread.start()
+        except Exception:
+            self._nv = None
+            exe = shutil.which("nvidia-smi")
+            if exe:
+                self._proc = subprocess.Popen(
+                    [exe, "--query-gpu=clocks.sm,clocks.max.sm,clocks_event_reasons.active",
+                     "--format=csv,noheader,nounits", "-lms", "100", "-i", str(gpu_index)],
+                    stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+
+    def _poll(self):
+        nv, h = self._nv, self._h
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM))
+                self.maxes.append(nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM))
+                bits = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+                for name, bit in self.REASONS.items():
+                    if bits & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            self._stop.wait(0.002)
 
     def stop(self):
-        if self.proc is None:
-            return None
-        self.proc.terminate()
-        try:
-            out, _ = self.proc.communicate(timeout=5)
-        except subprocess.TimeoutExpired:
-            self.proc.kill()
-            out, _ = self.proc.communicate()
-        sm, mx, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in out.strip().splitlines():
-            parts = [p.strip() for p in line.split(",")]
-            if len(parts) < 9:
-                continue
+        if self._thread is not None:
+            self._stop.set()
+            self._thread.join(timeout=5)
+        elif self._proc is not None:
+            self._proc.terminate()
             try:
-                sm.append(float(parts[1]))
-                mx.append(float(parts[2]))
-            except ValueError:
-                continue
-            for n, v in zip(names, parts[5:9]):
-                if v.lower() == "active":
-                    reasons.add(n)
-        if not sm:
+                out, _ = self._proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self._proc.kill()
+                out, _ = self._proc.communicate()
+            for line in out.strip().splitlines():
+                parts = [x.strip() for x in line.split(",")]
+                try:
+                    self.samples.append(float(parts[0]))
+                    self.maxes.append(float(parts[1]))
+                except (ValueError, IndexError):
+                    continue
+        if not self.samples:
             return None
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
-                "samples": len(sm)}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": max(self.maxes),
+                "reasons": sorted(self.reasons), "samples": len(self.samples),
+                "source": "nvml" if self._thread is not None else "nvidia-smi"}
 
 
 def cpu_baseline(name: str, budget_s: float = 12.0, max_rows: int = 4096):
@@ -188,6 +216,10 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-variants", action="store_true")
+    ap.add_argument("--rows", type=int, default=None,
+                    help="profiling only: fewer rows of the same recipe (not a bench line)")
+    ap.add_argument("--dtype", choices=["f32", "bf16"], default="f32",
+                    help="profiling only: logit dtype of the workload")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
 
@@ -212,7 +244,9 @@ def main():
         dist.init_process_group("nccl", device_id=dev, timeout=datetime.timedelta(seconds=120))
 
     name = WORKLOAD
-    w = synth.make(name, device=dev, seed=synth.WORKLOADS[name][4] + 7919 * rank)
+    dt = synth.F32 if args.dtype == "f32" else synth.BF16
+    w = synth.make(name, device=dev, seed=synth.WORKLOADS[name][4] + 7919 * rank, n=args.rows,
+                   dtype=dt)
     N, V = w.base.shape
     eb = w.bytes_per_elem
     in_bytes = 2 * N * V * eb
@@ -362,6 +396,9 @@ def main():
             "mean_kld": res["mean_kld"], "top1_agree_pct": res["top1_agree_pct"], "ppl": res["ppl"],
             "variants": variants,
         }
+        if args.rows is not None or args.dtype != "f32":
+            line["config"]["override"] = {"rows": N, "dtype": args.dtype,
+                                          "note": "profiling run, not the benchmark workload"}
         print(json.dumps(line), flush=True)
 
     st.close()
