@@ -73,7 +73,8 @@ typedef enum {
                               the other rows                                 */
   KLD_ERR_TIMEOUT = 7,     /* a bounded device-side wait gave up            */
   KLD_ERR_NO_DEVICE = 8,   /* no usable sm_100 device                       */
-  KLD_ERR_NOT_READY = 9    /* kld_stats_result() before any run             */
+  KLD_ERR_NOT_READY = 9,   /* kld_stats_result() before any run             */
+  KLD_ERR_CAPACITY = 10    /* more rows than kld_stats_run_static can hold  */
 } kld_status_t;
 
 typedef enum { KLD_F32 = 0, KLD_BF16 = 1, KLD_F16 = 2 } kld_dtype_t;
@@ -223,6 +224,37 @@ typedef struct {
 
 kld_status_t kld_plan(int64_t N, int64_t V, kld_dtype_t dtype, int sm_count,
                       kld_plan_t* out);
+
+/*
+ * Allocation-free kld_stats_run (no counterpart on the source pages: it is a
+ * deployment convenience of this library).
+ *
+ * For callers that cannot allocate device memory when they need the
+ * statistic -- e.g. a server that reserves almost all HBM for its own pool at
+ * start-up, or a loop that cannot afford the device synchronisation
+ * cudaMalloc/cudaFree may cause. It takes no handle and allocates nothing:
+ * per-row records and the error word live in one fixed array compiled into
+ * the library (KLD_STATIC_MAX_ROWS records, about 2 MiB), which every GPU
+ * that loads the library keeps until the process exits.
+ *
+ * Runs on the calling thread's current device and enqueues the row pass and
+ * the reduction on `stream`; inputs as for kld_stats_run (device pointers).
+ * result_dev: caller-owned DEVICE memory for one kld_result_t (8-byte
+ * aligned), written asynchronously; its flags_or / device_error fields carry
+ * what kld_stats_result() would report as status. 1 <= N <=
+ * KLD_STATIC_MAX_ROWS, else KLD_ERR_CAPACITY (nothing enqueued).
+ *
+ * The first call on a device (with it current) looks up the array's device
+ * address and sets kernel attributes; make that first call before any stream
+ * capture. All calls share the one array and each overwrites the previous
+ * call's records, so calls whose GPU work overlaps (other streams or threads)
+ * race: order them.
+ */
+#define KLD_STATIC_MAX_ROWS 65536
+kld_status_t kld_stats_run_static(const void* base, const void* quant,
+                                  const int32_t* token_ids, int64_t N,
+                                  int64_t V, kld_dtype_t dtype,
+                                  kld_result_t* result_dev, void* stream);
 
 #ifdef __cplusplus
 }

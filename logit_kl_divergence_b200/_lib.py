@@ -22,6 +22,8 @@ KLD_ERR_BAD_TOKEN = 6
 KLD_ERR_TIMEOUT = 7
 KLD_ERR_NO_DEVICE = 8
 KLD_ERR_NOT_READY = 9
+KLD_ERR_CAPACITY = 10
+KLD_STATIC_MAX_ROWS = 65536
 
 KLD_F32, KLD_BF16, KLD_F16 = 0, 1, 2
 
@@ -100,6 +102,7 @@ SIGNATURES = {
     "kld_stats_set_timing": (_ST, [_P, _I32]),
     "kld_stats_timing": (_ST, [_P, ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ctypes.c_float)]),
     "kld_plan": (_ST, [_I64, _I64, _I32, _I32, ctypes.POINTER(Plan)]),
+    "kld_stats_run_static": (_ST, [_P, _P, _P, _I64, _I64, _I32, _P, _P]),
 }
 
 _lock = threading.Lock()

@@ -130,6 +130,7 @@ const char* kld_status_string(kld_status_t s) {
     case KLD_ERR_TIMEOUT: return "a bounded device wait gave up";
     case KLD_ERR_NO_DEVICE: return "no usable sm_100 device";
     case KLD_ERR_NOT_READY: return "no run to report";
+    case KLD_ERR_CAPACITY: return "more rows than the fixed scratch of kld_stats_run_static";
   }
   return "unknown status";
 }
