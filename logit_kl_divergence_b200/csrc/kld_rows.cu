@@ -119,8 +119,7 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 }
 // Wait for the phase of `parity` to complete; gives up after kWaitLimitNs or
 // as soon as another thread of the CTA has raised *abort.
-__device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort) {
-  if (mbar_try_wait(bar, parity)) return true;
+__device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, volatile int* abort) {
   const uint64_t t0 = globaltimer();
   for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
@@ -129,6 +128,9 @@ __device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile i
       if (globaltimer() - t0 > kWaitLimitNs) return false;
     }
   }
+}
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort) {
+  return mbar_try_wait(bar, parity) || mbar_wait_slow(bar, parity, abort);
 }
 __device__ __forceinline__ uint64_t evict_first_policy() {
   uint64_t pol;
@@ -204,17 +206,32 @@ __device__ __forceinline__ float phi_q(float x) {
   q = fmaf(q, x, kQ1);
   return fmaf(q, x, kQ0);
 }
+// The coefficients as (c, c) pairs in constant memory: packed FMAs take no
+// immediates, and constant-bank operands cost no registers.
+__constant__ __align__(8) float kQpair[18] = {kQ0, kQ0, kQ1, kQ1, kQ2, kQ2, kQ3, kQ3, kQ4,
+                                              kQ4, kQ5, kQ5, kQ6, kQ6, kQ7, kQ7, kQ8, kQ8};
+__device__ __forceinline__ f2 qc(int k) {
+  f2 r;
+  r.v = reinterpret_cast<const unsigned long long*>(kQpair)[k];
+  return r;
+}
 __device__ __forceinline__ f2 phi_q2(f2 x) {
-  f2 q = fma2(splat(kQ8), x, splat(kQ7));
-  q = fma2(q, x, splat(kQ6));
-  q = fma2(q, x, splat(kQ5));
-  q = fma2(q, x, splat(kQ4));
-  q = fma2(q, x, splat(kQ3));
-  q = fma2(q, x, splat(kQ2));
-  q = fma2(q, x, splat(kQ1));
-  return fma2(q, x, splat(kQ0));
+  f2 q = fma2(qc(8), x, qc(7));
+  q = fma2(q, x, qc(6));
+  q = fma2(q, x, qc(5));
+  q = fma2(q, x, qc(4));
+  q = fma2(q, x, qc(3));
+  q = fma2(q, x, qc(2));
+  q = fma2(q, x, qc(1));
+  return fma2(q, x, qc(0));
 }
 
+// Maximum that propagates NaN (so a NaN anywhere fails a "<= bound" test).
+__device__ __forceinline__ float max3_nan(float a, float b, float c) {
+  float y;
+  asm("max.NaN.f32 %0, %1, %2, %3;" : "=f"(y) : "f"(a), "f"(b), "f"(c));
+  return y;
+}
 __device__ __forceinline__ double warp_sum(double x) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
@@ -410,7 +427,7 @@ __device__ __forceinline__ void chunk_step(const float* b, const float* q, unsig
   // Log-ratios x = (q - b) + K, in packed pairs.
   constexpr int NP = (PE + 1) / 2;
   f2 X[NP];
-  bool ok = true;
+  float ax0 = 0.f, ax1 = 0.f;  // max |x| of the lane (two chains), NaN if any x is NaN
   const f2 K2 = splat(r.K);
 #pragma unroll
   for (int j = 0; j < NP; ++j) {
@@ -421,10 +438,12 @@ __device__ __forceinline__ void chunk_step(const float* b, const float* q, unsig
     if (((valid >> i0) & 1u) == 0u) x0 = 0.f;
     if (((valid >> i1) & 1u) == 0u || i1 == i0) x1 = 0.f;
     X[j] = pk(x0, x1);
-    ok &= fabsf(x0) <= kTau;  // false for NaN
-    ok &= fabsf(x1) <= kTau;
+    if (j & 1)
+      ax1 = max3_nan(ax1, fabsf(x0), fabsf(x1));
+    else
+      ax0 = max3_nan(ax0, fabsf(x0), fabsf(x1));
   }
-  if (__all_sync(0xffffffffu, ok)) {
+  if (__all_sync(0xffffffffu, ax0 <= kTau && ax1 <= kTau)) {  // false for NaN
     // Polynomial path: every pair finite with |x| <= 2.5.
     const f2 L2 = splat(kLog2e), nR2 = splat(-r.Rb);
     f2 SB = splat(0.f), SA = splat(0.f), SC = splat(0.f);
@@ -443,9 +462,9 @@ __device__ __forceinline__ void chunk_step(const float* b, const float* q, unsig
     upk(SB, sb0, sb1);
     upk(SA, sa0, sa1);
     upk(SC, sc0, sc1);
-    a.Sb += static_cast<double>(sb0) + static_cast<double>(sb1);
-    a.Ap += static_cast<double>(sa0) + static_cast<double>(sa1);
-    a.C += static_cast<double>(sc0) + static_cast<double>(sc1);
+    a.Sb += static_cast<double>(sb0 + sb1);
+    a.Ap += static_cast<double>(sa0 + sa1);
+    a.C += static_cast<double>(sc0 + sc1);
   } else {
     // Direct path: quant weights in their own frame. x -> +BIG keeps 0*x = 0
     // for masked base entries; x = -inf (quant masked, base finite) makes A
@@ -655,7 +674,10 @@ __global__ void __launch_bounds__(kRowThreads, 1)
 
   if (warp < kConsumerWarps) {
     // ----------------------------------------------------------- consumers
-    uint32_t it = 0;
+    constexpr int kChunksPerWarp = kChunksPerTile / kConsumerWarps;
+    static_assert(kChunksPerTile % kConsumerWarps == 0, "chunks must split evenly");
+    int s = 0;         // stage of the next tile
+    uint32_t ph = 0u;  // its phase parity
     int rowk = 0;
     for (int64_t r = blockIdx.x; r < N; r += gridDim.x, ++rowk) {
       const char* rb = B + r * V * EB;
@@ -663,33 +685,40 @@ __global__ void __launch_bounds__(kRowThreads, 1)
       Ref ref{-INFINITY, -INFINITY, 0.f, 0.f, 0.f};
       Acc acc{0.0, 0.0, 0.0, 0.0, 0.0, 0.0};
       Best best{-INFINITY, -INFINITY, -1, -1};
-      for (int64_t t = 0; t < g.ntiles; ++t, ++it) {
-        const int s = static_cast<int>(it % kStages);
-        const uint32_t ph = (it / kStages) & 1u;
+      const int ntiles = static_cast<int>(g.ntiles);
+      for (int t = 0; t < ntiles; ++t) {
         if (!mbar_wait(smem_u32(&ctrl->full[s]), ph, abort)) {
           fail(ctrl, derr);
           return;
         }
-        int64_t len = g.body_len - t * kStageElems;
-        if (len > kStageElems) len = kStageElems;
         const uint4* tb = reinterpret_cast<const uint4*>(stage_b + s * kStageBytes);
         const uint4* tq = reinterpret_cast<const uint4*>(stage_q + s * kStageBytes);
+        const int64_t rem = g.body_len - static_cast<int64_t>(t) * kStageElems;
+        if (rem >= kStageElems) {
+          // Full tile: this warp's chunks, no masking.
+#pragma unroll
+          for (int k = 0; k < kChunksPerWarp; ++k) {
+            const int c = warp + k * kConsumerWarps;
+            process_chunk<DT, false>(tb + c * (kChunkElems / E), tq + c * (kChunkElems / E), lane,
+                                     0, ref, acc, best, t * kChunksPerTile + c);
+          }
+        } else {
+          const int len = static_cast<int>(rem);
 #pragma unroll 1
-        for (int c = warp; c < kChunksPerTile; c += kConsumerWarps) {
-          const int cstart = c * kChunkElems;
-          if (cstart >= len) break;
-          const int gid = static_cast<int>(t) * kChunksPerTile + c;
-          const uint4* cb = tb + cstart / E;
-          const uint4* cq = tq + cstart / E;
-          if (cstart + kChunkElems <= len) {
-            process_chunk<DT, false>(cb, cq, lane, 0, ref, acc, best, gid);
-          } else {
-            process_chunk<DT, true>(cb, cq, lane, static_cast<int>((len - cstart) / E), ref, acc,
-                                    best, gid);
+          for (int k = 0; k < kChunksPerWarp; ++k) {
+            const int c = warp + k * kConsumerWarps;
+            const int cstart = c * kChunkElems;
+            if (cstart >= len) break;
+            process_chunk<DT, true>(tb + cstart / E, tq + cstart / E, lane, (len - cstart) / E,
+                                    ref, acc, best, t * kChunksPerTile + c);
           }
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_u32(&ctrl->empty[s]));
+        if (++s == kStages) {
+          s = 0;
+          ph ^= 1u;
+        }
       }
 
       // Publish the warp partial into the slot ring.
