@@ -69,6 +69,14 @@ constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
 // phi(y) = y^2 * P(y), P of degree 8 fitted on [-2.5, 2.5]
 // (phi_poly_fit.py, max relative error of phi in fp32 9e-7); the kernel
 // evaluates phi(lambda*x) = x^2 * Q(x), Q_k = P_k * lambda^(k+2).
+// Narrower ranges need fewer terms; each chunk takes the cheapest
+// polynomial whose range holds all of its |x| (same accuracy, ~5e-7):
+// degree 5 on [-0.75, 0.75], degree 6 on [-1.25, 1.25], degree 8 on [-2.5, 2.5].
+constexpr float kTauA = 0.75f, kTauB = 1.25f;
+constexpr double kPA[6] = {0.5000001341, 0.1666664912, 0.0416622865,
+                           0.00833420901, 0.001409831012, 0.0001987944535};
+constexpr double kPB[7] = {0.5000000702, 0.1666677589, 0.04166594746, 0.008327533423,
+                           0.001389740978, 0.0002059674399, 2.494043224e-05};
 constexpr double kP0 = 0.4999997655, kP1 = 0.1666656346, kP2 = 0.0416678794,
                  kP3 = 0.008335872564, kP4 = 0.00138800956, kP5 = 0.0001968192101,
                  kP6 = 2.495779646e-05, kP7 = 3.111933302e-06, kP8 = 2.814820757e-07;
@@ -206,24 +214,29 @@ __device__ __forceinline__ float phi_q(float x) {
   q = fmaf(q, x, kQ1);
   return fmaf(q, x, kQ0);
 }
-// The coefficients as (c, c) pairs in constant memory: packed FMAs take no
-// immediates, and constant-bank operands cost no registers.
-__constant__ __align__(8) float kQpair[18] = {kQ0, kQ0, kQ1, kQ1, kQ2, kQ2, kQ3, kQ3, kQ4,
-                                              kQ4, kQ5, kQ5, kQ6, kQ6, kQ7, kQ7, kQ8, kQ8};
+// The coefficients, scaled by lambda^(k+2), as (c, c) pairs in constant
+// memory (packed FMAs take no immediates): 6 for tier A, 7 for tier B, 9 for
+// tier C.
+constexpr float qa(int k) { return static_cast<float>(kPA[k] * lam_pow(k + 2)); }
+constexpr float qb(int k) { return static_cast<float>(kPB[k] * lam_pow(k + 2)); }
+__constant__ __align__(8) float kQpair[44] = {
+    qa(0), qa(0), qa(1), qa(1), qa(2), qa(2), qa(3), qa(3), qa(4), qa(4), qa(5), qa(5),
+    qb(0), qb(0), qb(1), qb(1), qb(2), qb(2), qb(3), qb(3), qb(4), qb(4), qb(5), qb(5),
+    qb(6), qb(6),
+    kQ0, kQ0, kQ1, kQ1, kQ2, kQ2, kQ3, kQ3, kQ4, kQ4, kQ5, kQ5, kQ6, kQ6, kQ7, kQ7, kQ8, kQ8};
 __device__ __forceinline__ f2 qc(int k) {
   f2 r;
   r.v = reinterpret_cast<const unsigned long long*>(kQpair)[k];
   return r;
 }
+// Horner for tier T (0, 1, 2) with NC coefficients.
+template <int T, int NC>
 __device__ __forceinline__ f2 phi_q2(f2 x) {
-  f2 q = fma2(qc(8), x, qc(7));
-  q = fma2(q, x, qc(6));
-  q = fma2(q, x, qc(5));
-  q = fma2(q, x, qc(4));
-  q = fma2(q, x, qc(3));
-  q = fma2(q, x, qc(2));
-  q = fma2(q, x, qc(1));
-  return fma2(q, x, qc(0));
+  constexpr int o = T == 0 ? 0 : (T == 1 ? 6 : 13);
+  f2 q = fma2(qc(o + NC - 1), x, qc(o + NC - 2));
+#pragma unroll
+  for (int k = NC - 3; k >= 0; --k) q = fma2(q, x, qc(o + k));
+  return q;
 }
 
 // Maximum that propagates NaN (so a NaN anywhere fails a "<= bound" test).
@@ -300,7 +313,8 @@ struct Elem<KLD_F16> {
 
 // Warp-uniform frames of one row operand pair.
 struct Ref {
-  float Mb, Mq;  // running maxima seen by this warp (-inf before any)
+  float Mb;   // running maximum of b seen by this warp (-inf before any)
+  float Mqf;  // maximum of q over this warp's direct-path chunks (-inf before)
   float Rb, Rq;  // integer frames floor(M*L) once M is finite, 0 before
   float K;       // log-ratio centre: (b - q) at the running maximum of b
 };
@@ -347,6 +361,36 @@ __device__ __forceinline__ double pow2i(float k) {
   return ldexp(1.0, static_cast<int>(fmaxf(k, -2000.f)));
 }
 
+// Polynomial path of one step: every x finite with |x| within tier T's range.
+// S += e, Ap += e*x, C += e*x^2*Q_T(x), e = 2^(b*L - R_b).
+template <int PE, int T, int NC>
+__device__ __forceinline__ void poly_accumulate(const float* b, const f2* X, const Ref& r,
+                                                Acc& a) {
+  constexpr int NP = (PE + 1) / 2;
+  const f2 L2 = splat(kLog2e), nR2 = splat(-r.Rb);
+  // Two accumulator sets (even / odd pairs) halve the dependent-add chains.
+  f2 SB[2] = {splat(0.f), splat(0.f)}, SA[2] = {splat(0.f), splat(0.f)};
+  f2 SC[2] = {splat(0.f), splat(0.f)};
+#pragma unroll
+  for (int j = 0; j < NP; ++j) {
+    const int i0 = 2 * j, i1 = (2 * j + 1 < PE) ? 2 * j + 1 : 2 * j;
+    float u0, u1;
+    upk(fma2(pk(b[i0], b[i1]), L2, nR2), u0, u1);
+    const f2 E = pk(ex2(u0), i1 == i0 ? 0.f : ex2(u1));
+    const f2 T2 = mul2(E, X[j]);
+    SB[j & 1] = add2(SB[j & 1], E);
+    SA[j & 1] = add2(SA[j & 1], T2);
+    SC[j & 1] = fma2(mul2(T2, X[j]), phi_q2<T, NC>(X[j]), SC[j & 1]);
+  }
+  float sb0, sb1, sa0, sa1, sc0, sc1;
+  upk(add2(SB[0], SB[1]), sb0, sb1);
+  upk(add2(SA[0], SA[1]), sa0, sa1);
+  upk(add2(SC[0], SC[1]), sc0, sc1);
+  a.Sb += static_cast<double>(sb0 + sb1);
+  a.Ap += static_cast<double>(sa0 + sa1);
+  a.C += static_cast<double>(sc0 + sc1);
+}
+
 // One step of PE element pairs per lane (a 16-element consumer chunk, or the
 // head/tail elements one per lane). Elements whose bit in `valid` is clear
 // are absent (b = q = -inf, x = 0: they contribute nothing).
@@ -364,7 +408,6 @@ __device__ __forceinline__ void chunk_step(const float* b, const float* q, unsig
     mq = fmaxf(mq, q[PE - 1]);
   }
   const float wmb = warp_max(mb);
-  const float wmq = warp_max(mq);
   if (wmb > r.Mb) {  // raise the base frame and move the centre (warp-uniform)
     // New centre: (b - q) at the lowest lane's first element holding wmb.
     float dl = 0.f;
@@ -417,12 +460,6 @@ __device__ __forceinline__ void chunk_step(const float* b, const float* q, unsig
     r.Rb = nR;
     r.Mb = wmb;
   }
-  if (wmq > r.Mq) {  // raise the quant frame (direct-path sums only)
-    const float nR = floorf(wmq * kLog2e);
-    if (r.Mq != -INFINITY) a.Sh *= pow2i(r.Rq - nR);
-    r.Rq = nR;
-    r.Mq = wmq;
-  }
 
   // Log-ratios x = (q - b) + K, in packed pairs.
   constexpr int NP = (PE + 1) / 2;
@@ -443,32 +480,22 @@ __device__ __forceinline__ void chunk_step(const float* b, const float* q, unsig
     else
       ax0 = max3_nan(ax0, fabsf(x0), fabsf(x1));
   }
-  if (__all_sync(0xffffffffu, ax0 <= kTau && ax1 <= kTau)) {  // false for NaN
-    // Polynomial path: every pair finite with |x| <= 2.5.
-    const f2 L2 = splat(kLog2e), nR2 = splat(-r.Rb);
-    f2 SB = splat(0.f), SA = splat(0.f), SC = splat(0.f);
-#pragma unroll
-    for (int j = 0; j < NP; ++j) {
-      const int i0 = 2 * j, i1 = (2 * j + 1 < PE) ? 2 * j + 1 : 2 * j;
-      float u0, u1;
-      upk(fma2(pk(b[i0], b[i1]), L2, nR2), u0, u1);
-      const f2 E = pk(ex2(u0), i1 == i0 ? 0.f : ex2(u1));
-      const f2 T = mul2(E, X[j]);
-      SB = add2(SB, E);
-      SA = add2(SA, T);
-      SC = fma2(mul2(T, X[j]), phi_q2(X[j]), SC);
-    }
-    float sb0, sb1, sa0, sa1, sc0, sc1;
-    upk(SB, sb0, sb1);
-    upk(SA, sa0, sa1);
-    upk(SC, sc0, sc1);
-    a.Sb += static_cast<double>(sb0 + sb1);
-    a.Ap += static_cast<double>(sa0 + sa1);
-    a.C += static_cast<double>(sc0 + sc1);
+  // Warp max of |x| (NaN if any x is NaN: every comparison below fails).
+  float wax;
+  asm volatile("redux.sync.max.NaN.f32 %0, %1, 0xffffffff;" : "=f"(wax) : "f"(max3_nan(ax0, ax1, 0.f)));
+  if (wax <= kTau) {
+    poly_accumulate<PE, 2, 9>(b, X, r, a);
   } else {
     // Direct path: quant weights in their own frame. x -> +BIG keeps 0*x = 0
     // for masked base entries; x = -inf (quant masked, base finite) makes A
     // -inf, i.e. KL = +inf.
+    const float wmq = warp_max(mq);
+    if (wmq > r.Mqf) {  // raise the quant frame (direct-path sums only)
+      const float nR = floorf(wmq * kLog2e);
+      if (r.Mqf != -INFINITY) a.Sh *= pow2i(r.Rq - nR);
+      r.Rq = nR;
+      r.Mqf = wmq;
+    }
     const float nRb = -r.Rb, nRq = -r.Rq;
     float sb = 0.f, sa = 0.f, sh = 0.f;
 #pragma unroll
@@ -726,8 +753,9 @@ __global__ void __launch_bounds__(kRowThreads, 1)
       const uint32_t sph = (rowk / kSlots) & 1u;
       const double Sb = warp_sum(acc.Sb), Ap = warp_sum(acc.Ap), C = warp_sum(acc.C);
       const double Ad = warp_sum(acc.Ad), Se = warp_sum(acc.Se), Sh = warp_sum(acc.Sh);
+      const float wq = warp_max(best.q);  // the warp's maximum of q
       const unsigned cb_mask = __ballot_sync(0xffffffffu, ref.Mb > -INFINITY && best.b == ref.Mb);
-      const unsigned cq_mask = __ballot_sync(0xffffffffu, ref.Mq > -INFINITY && best.q == ref.Mq);
+      const unsigned cq_mask = __ballot_sync(0xffffffffu, wq > -INFINITY && best.q == wq);
       if (!mbar_wait(smem_u32(&ctrl->slot_empty[slot]), sph ^ 1u, abort)) {
         fail(ctrl, derr);
         return;
@@ -738,7 +766,7 @@ __global__ void __launch_bounds__(kRowThreads, 1)
       if (lane == 0) {
         WarpPart p;
         p.Mb = ref.Mb;
-        p.Mq = ref.Mq;
+        p.Mq = wq;
         p.Rb = ref.Rb;
         p.Rq = ref.Rq;
         p.K = ref.K;
@@ -793,6 +821,7 @@ __global__ void __launch_bounds__(kRowThreads, 1)
     if (n_extra > 0) {
       chunk_step<1>(&xe_b, &xe_q, lane < n_extra ? 1u : 0u, eref, eacc, ebest, 0);
     }
+    const float eMq = warp_max(xe_q);
     const double eSb = warp_sum(eacc.Sb), eAp = warp_sum(eacc.Ap), eC = warp_sum(eacc.C);
     const double eAd = warp_sum(eacc.Ad), eSe = warp_sum(eacc.Se), eSh = warp_sum(eacc.Sh);
 
@@ -816,7 +845,7 @@ __global__ void __launch_bounds__(kRowThreads, 1)
       p.cand_b = p.cand_q = 0u;
       if (lane == kConsumerWarps) {
         p.Mb = eref.Mb;
-        p.Mq = eref.Mq;
+        p.Mq = eMq;
         p.Rb = eref.Rb;
         p.Rq = eref.Rq;
         p.K = eref.K;
@@ -861,7 +890,7 @@ __global__ void __launch_bounds__(kRowThreads, 1)
       const double em = expm1(kLambda * dK);
       const double BpK = Bp + em * (Bp + Sp);
       // Direct-path quant weights, from their own frame to Cb - Kref*L.
-      const double Bh = p.Mq > -INFINITY
+      const double Bh = p.Sh != 0.0
                             ? p.Sh * exp2(static_cast<double>(p.Rq) - static_cast<double>(Cb) +
                                           static_cast<double>(Kref) * kLog2eD)
                             : 0.0;
