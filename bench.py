@@ -207,6 +207,96 @@ def run_reference(args, rank: int):
     print(json.dumps(line), flush=True)
 
 
+SPLIT_ROWS = (1, 4, 16, 32)
+SPLIT_CALLS = 1000
+SPLIT_COLD_BYTES = 256 << 20  # inputs rotated per call cycle: twice the 126 MB L2
+
+
+def split_row_latency(dev, stream):
+    """Few-row, large-vocabulary launches (N in SPLIT_ROWS, V = 262144 fp32):
+    SPLIT_CALLS back-to-back calls of the whole statistic on one stream,
+    plainly and as CUDA-graph replays, with the whole-row launch shape
+    (kld_stats_run_static) beside them. Each call reads its own copy of the
+    inputs from a ring larger than L2, so every call streams from HBM."""
+    import torch
+
+    from logit_kl_divergence_b200 import KLDStats, run_static, synth
+
+    out = {"workload": "splitrow{1,4,16,32}_v262144_f32", "min_calls": SPLIT_CALLS,
+           "l2": f"inputs rotated over copies totalling >= {SPLIT_COLD_BYTES >> 20} MB per cycle",
+           "per_rows": {}}
+    ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+    for n in SPLIT_ROWS:
+        w = synth.make(f"splitrow{n}_v262144_f32", device=dev)
+        V = w.base.shape[1]
+        call_bytes = 2 * n * V * w.bytes_per_elem
+        k = max(1, -(-SPLIT_COLD_BYTES // call_bytes))
+        bs = w.base.unsqueeze(0).repeat(k, 1, 1)
+        qs = w.quant.unsqueeze(0).repeat(k, 1, 1)
+        tok = w.token_ids
+        st = KLDStats(max_rows=n, device=dev)
+        res_buf = torch.zeros(256, dtype=torch.uint8, device=dev)
+        calls = -(-SPLIT_CALLS // k) * k
+
+        def timed(fn, reps):
+            for i in range(min(k, 8)):
+                fn(i)
+            torch.cuda.synchronize(dev)
+            a, b = ev(), ev()
+            a.record(stream)
+            for i in range(reps):
+                fn(i % k)
+            b.record(stream)
+            torch.cuda.synchronize(dev)
+            return a.elapsed_time(b) * 1000.0 / reps
+
+        us_stream = timed(lambda i: st.run(bs[i], qs[i], tok), calls)
+        us_whole = timed(lambda i: run_static(bs[i], qs[i], tok, res_buf), calls)
+        # one graph holding one call per copy, replayed
+        g = torch.cuda.CUDAGraph()
+        side = torch.cuda.Stream(dev)
+        side.wait_stream(stream)
+        with torch.cuda.stream(side):
+            for i in range(k):
+                st.run(bs[i], qs[i], tok)
+        stream.wait_stream(side)
+        torch.cuda.synchronize(dev)
+        with torch.cuda.graph(g):
+            for i in range(k):
+                st.run(bs[i], qs[i], tok)
+        reps = calls // k
+        g.replay()
+        torch.cuda.synchronize(dev)
+        a, b = ev(), ev()
+        a.record(stream)
+        for _ in range(reps):
+            g.replay()
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        us_graph = a.elapsed_time(b) * 1000.0 / (reps * k)
+        # kernel-only time of the row pass (events around it, cold inputs)
+        st.set_timing(True)
+        rp = []
+        for i in range(min(k, 50)):
+            st.run(bs[i], qs[i], tok)
+            st.result()
+            rp.append(st.timing()[0] * 1000.0)
+        st.set_timing(False)
+        res = st.result()
+        out["per_rows"][str(n)] = {
+            "plan": st.plan(n, V, 0),
+            "us_per_call_stream": us_stream, "us_per_call_graph": us_graph,
+            "us_per_call_whole_row_launch": us_whole,
+            "row_pass_us_median": statistics.median(rp),
+            "gbs_stream": call_bytes / (us_stream * 1e3), "gbs_graph": call_bytes / (us_graph * 1e3),
+            "gbs_row_pass": call_bytes / (statistics.median(rp) * 1e3),
+            "calls": calls, "input_copies": k, "mean_kld": res["mean_kld"]}
+        del g, bs, qs, w, st
+        torch.cuda.synchronize(dev)
+        torch.cuda.empty_cache()
+    return out
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -216,6 +306,7 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-variants", action="store_true")
+    ap.add_argument("--no-split-row", action="store_true")
     ap.add_argument("--rows", type=int, default=None,
                     help="profiling only: fewer rows of the same recipe (not a bench line)")
     ap.add_argument("--dtype", choices=["f32", "bf16"], default="f32",
@@ -377,6 +468,12 @@ def main():
                "ms_per_step": ems, "path": "kld_stats_run_host (pinned host buffers)"}
         del hb, hq, ht
 
+    split_row = None
+    if world == 1 and not args.no_split_row and args.rows is None:
+        del w
+        torch.cuda.empty_cache()
+        split_row = split_row_latency(dev, stream)
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(name)
@@ -394,7 +491,7 @@ def main():
             "gpu_launches": 2 * args.steps, "clocks": clocks,
             "gbs": in_bytes * world / (ms_per_step / 1000.0) / 1e9,
             "mean_kld": res["mean_kld"], "top1_agree_pct": res["top1_agree_pct"], "ppl": res["ppl"],
-            "variants": variants,
+            "variants": variants, "split_row": split_row,
         }
         if args.rows is not None or args.dtype != "f32":
             line["config"]["override"] = {"rows": N, "dtype": args.dtype,

@@ -206,10 +206,18 @@ kld_status_t kld_stats_timing(kld_stats_t h, float* row_pass_ms,
                               float* reduce_ms);
 
 /*
- * Launch plan the row pass would use for (N, V, dtype) on this handle's
- * device: kernel variant (0 = one CTA per row, 1 = split row over a thread-
- * block cluster), grid size, CTAs per row, threads per CTA, dynamic shared
- * memory bytes. Pure host logic; enqueues nothing.
+ * Launch plan of the row pass for (N, V, dtype) on a device with sm_count
+ * SMs: variant 0 = whole rows (one persistent CTA per SM, each taking rows
+ * r, r + grid, ...); variant 1 = split rows, used when N <= sm_count / 2 so
+ * that few rows still occupy the GPU: each row's 512-element chunks are
+ * divided among ctas_per_row CTAs, grouped in thread-block clusters of
+ * cluster_ctas CTAs (a power of two <= 8) whose partial sums meet in the
+ * cluster leader's shared memory; the row's clusters then meet through a
+ * small global scratch and an arrival counter. Also: threads per CTA,
+ * dynamic shared memory bytes, stage bytes per operand, stages. Pure host
+ * logic; enqueues nothing. The launch itself may lower ctas_per_row when the
+ * device can hold fewer clusters at once than sm_count / cluster_ctas (the
+ * count comes from cudaOccupancyMaxActiveClusters).
  */
 typedef struct {
   int32_t variant;
@@ -219,7 +227,7 @@ typedef struct {
   int32_t smem_bytes;
   int32_t stage_bytes;
   int32_t stages;
-  int32_t reserved;
+  int32_t cluster_ctas;
 } kld_plan_t;
 
 kld_status_t kld_plan(int64_t N, int64_t V, kld_dtype_t dtype, int sm_count,

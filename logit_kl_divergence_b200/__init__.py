@@ -19,7 +19,8 @@ from . import _lib
 from ._lib import (KLD_BF16, KLD_F16, KLD_F32, ROW_BAD_TOKEN, ROW_EMPTY,  # noqa: F401
                    ROW_INF_KL, ROW_INF_NLL, ROW_NONFINITE, KLDError)
 
-__all__ = ["KLDStats", "kld_stats", "dtype_code", "ROW_RECORD_BYTES"]
+__all__ = ["KLDStats", "kld_stats", "run_static", "result_from_bytes", "plan", "dtype_code",
+           "ROW_RECORD_BYTES"]
 
 ROW_RECORD_BYTES = 32
 
@@ -182,11 +183,33 @@ class KLDStats:
         return plan(n_rows, vocab, dtype, torch.cuda.get_device_properties(self.device).multi_processor_count)
 
 
+def run_static(base: torch.Tensor, quant: torch.Tensor, token_ids: torch.Tensor | None,
+               result_out: torch.Tensor, stream=None) -> None:
+    """kld_stats_run_static: the whole statistic with no allocation, written
+    asynchronously into ``result_out`` (a device uint8 tensor of at least
+    ``sizeof(kld_result_t)`` bytes, 8-byte aligned; decode with
+    :func:`result_from_bytes`)."""
+    _check_pair(base, quant, token_ids, True)
+    if result_out.dtype != torch.uint8 or result_out.numel() < ctypes.sizeof(_lib.Result) or not result_out.is_cuda:
+        raise ValueError("result_out must be a CUDA uint8 tensor of sizeof(kld_result_t) bytes")
+    lib = _lib.load()
+    st = lib.kld_stats_run_static(_ptr(base), _ptr(quant), _ptr(token_ids), base.shape[0], base.shape[1],
+                                  dtype_code(base), _ptr(result_out),
+                                  ctypes.c_void_p(_stream_ptr(stream, base.device)))
+    _lib.check(st, "kld_stats_run_static")
+
+
+def result_from_bytes(buf: torch.Tensor) -> dict:
+    """Statistics from a kld_result_t held in a uint8 tensor (copied to host)."""
+    res = _lib.Result.from_buffer_copy(bytes(buf[:ctypes.sizeof(_lib.Result)].cpu().numpy()))
+    return {name: getattr(res, name) for name, _ in _lib.Result._fields_ if not name.startswith("reserved")}
+
+
 def plan(n_rows: int, vocab: int, dtype: int, sm_count: int) -> dict:
     lib = _lib.load()
     p = _lib.Plan()
     _lib.check(lib.kld_plan(int(n_rows), int(vocab), int(dtype), int(sm_count), ctypes.byref(p)), "kld_plan")
-    return {name: getattr(p, name) for name, _ in _lib.Plan._fields_ if name != "reserved"}
+    return {name: getattr(p, name) for name, _ in _lib.Plan._fields_}
 
 
 class _DeviceBytes:

@@ -76,7 +76,7 @@ class Plan(ctypes.Structure):
         ("smem_bytes", ctypes.c_int32),
         ("stage_bytes", ctypes.c_int32),
         ("stages", ctypes.c_int32),
-        ("reserved", ctypes.c_int32),
+        ("cluster_ctas", ctypes.c_int32),
     ]
 
 

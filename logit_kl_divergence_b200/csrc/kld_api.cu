@@ -62,6 +62,8 @@ struct kld_stats_s {
   int sm_count = 0;
   int64_t max_rows = 0;
   kld_row_t* rows = nullptr;
+  void* split_mem = nullptr;  // split-row scratch: partials, then tickets
+  kld::SplitScratch split = {nullptr, nullptr, 0};
   kld_result_t* dres = nullptr;
   uint32_t* derr = nullptr;
   kld_result_t* hres = nullptr;
@@ -97,9 +99,9 @@ kld_status_t check_inputs(const void* base, const void* quant, const int32_t* to
   return KLD_OK;
 }
 
-int row_grid(const kld_stats_s* h, int64_t N) {
-  const int64_t g = N < h->sm_count ? N : h->sm_count;
-  return static_cast<int>(g < 1 ? 1 : g);
+cudaError_t launch_rows(kld_stats_s* h, const void* base, const void* quant, const int32_t* tok,
+                        int64_t N, int64_t V, kld_dtype_t dtype, kld_row_t* rows, cudaStream_t s) {
+  return kld::launch_rows(base, quant, tok, N, V, dtype, rows, h->derr, h->sm_count, &h->split, s);
 }
 
 kld_status_t enqueue_reduce(kld_stats_t h, const kld_row_t* rows, int64_t N, int has_nll,
@@ -142,9 +144,11 @@ kld_status_t kld_plan(int64_t N, int64_t V, kld_dtype_t dtype, int sm_count, kld
   if (!valid_dtype(dtype)) return KLD_ERR_DTYPE;
   if (N < 1 || V < 1 || V > INT32_MAX || sm_count < 1) return KLD_ERR_INVALID_ARG;
   std::memset(out, 0, sizeof(*out));
-  out->variant = 0;
-  out->grid = static_cast<int32_t>(N < sm_count ? N : sm_count);
-  out->ctas_per_row = 1;
+  const kld::RowPlan pl = kld::plan_rows(N, sm_count, 0, true);
+  out->variant = pl.parts_per_row > 1 ? 1 : 0;
+  out->grid = pl.grid;
+  out->ctas_per_row = pl.parts_per_row;
+  out->cluster_ctas = pl.cluster_ctas;
   out->threads = kld::kRowThreads;
   out->smem_bytes = kld::kRowSmemBytes;
   out->stage_bytes = kld::kStageBytes;
@@ -190,6 +194,20 @@ kld_status_t kld_stats_create(kld_stats_t* out, int64_t max_rows, int device) {
       st = cuda_fail(err, "cudaMalloc(error word)"); break; }
     if ((err = cudaMemset(h->derr, 0, sizeof(uint32_t))) != cudaSuccess) {
       st = cuda_fail(err, "cudaMemset"); break; }
+    {
+      // Split rows: at most one partial per SM-sized cluster slot and one
+      // arrival counter per row (rows <= SMs / 2), counters zeroed once;
+      // each row's last arriver puts its counter back to zero.
+      const size_t pbytes = static_cast<size_t>(sms) * kld::kSplitPartBytes;
+      const size_t tbytes = static_cast<size_t>(sms) * sizeof(unsigned);
+      if ((err = cudaMalloc(&h->split_mem, pbytes + tbytes)) != cudaSuccess) {
+        st = cuda_fail(err, "cudaMalloc(split scratch)"); break; }
+      if ((err = cudaMemset(h->split_mem, 0, pbytes + tbytes)) != cudaSuccess) {
+        st = cuda_fail(err, "cudaMemset"); break; }
+      h->split.parts = h->split_mem;
+      h->split.tickets = reinterpret_cast<unsigned*>(static_cast<char*>(h->split_mem) + pbytes);
+      h->split.capacity = sms;
+    }
     if ((err = cudaMallocHost(&h->hres, sizeof(kld_result_t))) != cudaSuccess) {
       st = cuda_fail(err, "cudaMallocHost"); break; }
     if ((err = cudaEventCreateWithFlags(&h->done, cudaEventDisableTiming)) != cudaSuccess) {
@@ -224,6 +242,7 @@ void kld_stats_destroy(kld_stats_t h) {
   if (h->derr) cudaFree(h->derr);
   if (h->dres) cudaFree(h->dres);
   if (h->rows) cudaFree(h->rows);
+  if (h->split_mem) cudaFree(h->split_mem);
   delete h;
 }
 
@@ -238,8 +257,7 @@ kld_status_t kld_stats_run_rows(kld_stats_t h, const void* base, const void* qua
   DeviceGuard guard(h->device);
   if (!guard.ok()) return cuda_fail(cudaGetLastError(), "cudaSetDevice");
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  KLD_CUDA(kld::launch_rows(base, quant, token_ids, N, V, dtype, rows_out ? rows_out : h->rows,
-                            h->derr, row_grid(h, N), s));
+  KLD_CUDA(launch_rows(h, base, quant, token_ids, N, V, dtype, rows_out ? rows_out : h->rows, s));
   if (!rows_out) h->last_rows = N;
   h->timing_valid = false;
   return KLD_OK;
@@ -270,8 +288,7 @@ kld_status_t kld_stats_run(kld_stats_t h, const void* base, const void* quant,
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   h->timing_valid = h->timing;
   if (h->timing) KLD_CUDA(cudaEventRecord(h->tev[0], s));
-  KLD_CUDA(kld::launch_rows(base, quant, token_ids, N, V, dtype, h->rows, h->derr,
-                            row_grid(h, N), s));
+  KLD_CUDA(launch_rows(h, base, quant, token_ids, N, V, dtype, h->rows, s));
   if (h->timing) KLD_CUDA(cudaEventRecord(h->tev[1], s));
   h->last_rows = N;
   return enqueue_reduce(h, h->rows, N, token_ids != nullptr, s);
@@ -377,8 +394,7 @@ kld_status_t kld_stats_run_host(kld_stats_t h, const void* base_host, const void
                                cudaMemcpyHostToDevice, h->copy_stream));
     KLD_CUDA(cudaEventRecord(h->copied[b], h->copy_stream));
     KLD_CUDA(cudaStreamWaitEvent(s, h->copied[b], 0));
-    KLD_CUDA(kld::launch_rows(sb, sq, token_ids_host ? stok : nullptr, n, V, dtype,
-                              h->rows + r0, h->derr, row_grid(h, n), s));
+    KLD_CUDA(launch_rows(h, sb, sq, token_ids_host ? stok : nullptr, n, V, dtype, h->rows + r0, s));
     KLD_CUDA(cudaEventRecord(h->freed[b], s));
   }
   h->last_rows = N;

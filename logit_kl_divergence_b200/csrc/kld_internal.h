@@ -24,6 +24,21 @@ constexpr int kLaneElems = 16;
 constexpr int kChunkElems = kLaneElems * 32;  // elements per warp-chunk
 constexpr int kSlots = 4;
 
+// Split-row mode: up to kMaxClusterCtas CTAs per thread-block cluster share
+// one row; their partials meet in the cluster leader's shared memory.
+constexpr int kMaxClusterCtas = 8;
+
+// Per-launch global scratch of split-row mode: one merged partial per
+// cluster (kSplitPartBytes) and one arrival ticket per row; `parts` holds
+// `capacity` partials and `tickets` at least as many counters as rows. Tickets start at zero and are reset by
+// the last arriver.
+constexpr int kSplitPartBytes = 64;
+struct SplitScratch {
+  void* parts;
+  unsigned* tickets;
+  int capacity;
+};
+
 // Dynamic shared memory of the row kernel: stages for both operands, then the
 // control block (mbarriers and the partial slots).
 constexpr int kRowCtrlBytes = 24 * 1024;
@@ -36,10 +51,20 @@ inline int elem_bytes(kld_dtype_t dt) { return dt == KLD_F32 ? 4 : 2; }
 
 // Launchers (defined in the .cu files). They enqueue on `stream` and return
 // the launch error.
+// Row pass. With split == nullptr every CTA handles whole rows; otherwise
+// few-row launches spread each row over clusters of CTAs (see RowPlan).
 cudaError_t launch_rows(const void* base, const void* quant,
                         const int32_t* token_ids, int64_t N, int64_t V,
                         kld_dtype_t dtype, kld_row_t* rows, uint32_t* derr,
-                        int grid, cudaStream_t stream);
+                        int sm_count, const SplitScratch* split, cudaStream_t stream);
+
+// Launch shape of the row pass: parts_per_row = 1 (whole rows, persistent
+// grid) or > 1 (split rows: grid = N * parts_per_row, clusters of
+// cluster_ctas CTAs, parts_per_row / cluster_ctas clusters per row).
+struct RowPlan {
+  int grid, parts_per_row, cluster_ctas;
+};
+RowPlan plan_rows(int64_t N, int sm_count, int max_active_clusters_for_8, bool split_allowed);
 cudaError_t prepare_rows_kernels();  // per-device attribute setup
 
 cudaError_t launch_reduce(const kld_row_t* rows, int64_t N, int has_nll,

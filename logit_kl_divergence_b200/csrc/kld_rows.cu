@@ -51,6 +51,7 @@
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
+#include <atomic>
 #include <climits>
 
 #include "kld_internal.h"
@@ -69,14 +70,6 @@ constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
 // phi(y) = y^2 * P(y), P of degree 8 fitted on [-2.5, 2.5]
 // (phi_poly_fit.py, max relative error of phi in fp32 9e-7); the kernel
 // evaluates phi(lambda*x) = x^2 * Q(x), Q_k = P_k * lambda^(k+2).
-// Narrower ranges need fewer terms; each chunk takes the cheapest
-// polynomial whose range holds all of its |x| (same accuracy, ~5e-7):
-// degree 5 on [-0.75, 0.75], degree 6 on [-1.25, 1.25], degree 8 on [-2.5, 2.5].
-constexpr float kTauA = 0.75f, kTauB = 1.25f;
-constexpr double kPA[6] = {0.5000001341, 0.1666664912, 0.0416622865,
-                           0.00833420901, 0.001409831012, 0.0001987944535};
-constexpr double kPB[7] = {0.5000000702, 0.1666677589, 0.04166594746, 0.008327533423,
-                           0.001389740978, 0.0002059674399, 2.494043224e-05};
 constexpr double kP0 = 0.4999997655, kP1 = 0.1666656346, kP2 = 0.0416678794,
                  kP3 = 0.008335872564, kP4 = 0.00138800956, kP5 = 0.0001968192101,
                  kP6 = 2.495779646e-05, kP7 = 3.111933302e-06, kP8 = 2.814820757e-07;
@@ -214,28 +207,20 @@ __device__ __forceinline__ float phi_q(float x) {
   q = fmaf(q, x, kQ1);
   return fmaf(q, x, kQ0);
 }
-// The coefficients, scaled by lambda^(k+2), as (c, c) pairs in constant
-// memory (packed FMAs take no immediates): 6 for tier A, 7 for tier B, 9 for
-// tier C.
-constexpr float qa(int k) { return static_cast<float>(kPA[k] * lam_pow(k + 2)); }
-constexpr float qb(int k) { return static_cast<float>(kPB[k] * lam_pow(k + 2)); }
-__constant__ __align__(8) float kQpair[44] = {
-    qa(0), qa(0), qa(1), qa(1), qa(2), qa(2), qa(3), qa(3), qa(4), qa(4), qa(5), qa(5),
-    qb(0), qb(0), qb(1), qb(1), qb(2), qb(2), qb(3), qb(3), qb(4), qb(4), qb(5), qb(5),
-    qb(6), qb(6),
-    kQ0, kQ0, kQ1, kQ1, kQ2, kQ2, kQ3, kQ3, kQ4, kQ4, kQ5, kQ5, kQ6, kQ6, kQ7, kQ7, kQ8, kQ8};
+// The coefficients Q_k as (c, c) pairs in constant memory (packed FMAs take
+// no immediates).
+__constant__ __align__(8) float kQpair[18] = {kQ0, kQ0, kQ1, kQ1, kQ2, kQ2, kQ3, kQ3, kQ4,
+                                              kQ4, kQ5, kQ5, kQ6, kQ6, kQ7, kQ7, kQ8, kQ8};
 __device__ __forceinline__ f2 qc(int k) {
   f2 r;
   r.v = reinterpret_cast<const unsigned long long*>(kQpair)[k];
   return r;
 }
-// Horner for tier T (0, 1, 2) with NC coefficients.
-template <int T, int NC>
+// Horner for Q on a packed pair.
 __device__ __forceinline__ f2 phi_q2(f2 x) {
-  constexpr int o = T == 0 ? 0 : (T == 1 ? 6 : 13);
-  f2 q = fma2(qc(o + NC - 1), x, qc(o + NC - 2));
+  f2 q = fma2(qc(8), x, qc(7));
 #pragma unroll
-  for (int k = NC - 3; k >= 0; --k) q = fma2(q, x, qc(o + k));
+  for (int k = 6; k >= 0; --k) q = fma2(q, x, qc(k));
   return q;
 }
 
@@ -345,13 +330,30 @@ struct Slot {
   int loc_q[kConsumerWarps][32];
 };
 
+// Merged partial of a contiguous part of a row (a warp, a CTA, a cluster):
+// maxima, base frame Cb (integer log2), centre K, and in that frame / centre
+// S = sum e, A = sum e x, B = sum e (e^{lx} - 1); exact lowest argmax indices
+// of the part (INT_MAX if none); flags (kPartNonfinite, kPartInfKl).
+struct __align__(16) MPart {
+  float Mb, Mq, Cb, K;
+  double Sb, A, B;
+  int amax_b, amax_q;
+  unsigned flags, pad;
+  unsigned long long pad2;  // 64 bytes: four 16-byte words
+};
+constexpr unsigned kPartNonfinite = 1u, kPartInfKl = 2u;
+constexpr unsigned kPartFailed = 4u;  // a bounded wait gave up on this part
+static_assert(sizeof(MPart) == kSplitPartBytes, "MPart layout");
+
 struct Ctrl {
   unsigned long long full[kStages];
   unsigned long long empty[kStages];
   unsigned long long slot_full[kSlots];
   unsigned long long slot_empty[kSlots];
+  unsigned long long cl_full;  // split mode: cluster peers' partials arrived (leader)
   int abort;
   int pad;
+  MPart cl_part[kMaxClusterCtas];  // split mode: partials pushed by the cluster peers
   Slot slot[kSlots];
 };
 static_assert(sizeof(Ctrl) <= kRowCtrlBytes, "control block too large");
@@ -361,9 +363,9 @@ __device__ __forceinline__ double pow2i(float k) {
   return ldexp(1.0, static_cast<int>(fmaxf(k, -2000.f)));
 }
 
-// Polynomial path of one step: every x finite with |x| within tier T's range.
-// S += e, Ap += e*x, C += e*x^2*Q_T(x), e = 2^(b*L - R_b).
-template <int PE, int T, int NC>
+// Polynomial path of one step: every x finite with |x| <= kTau.
+// S += e, Ap += e*x, C += e*x^2*Q(x), e = 2^(b*L - R_b).
+template <int PE>
 __device__ __forceinline__ void poly_accumulate(const float* b, const f2* X, const Ref& r,
                                                 Acc& a) {
   constexpr int NP = (PE + 1) / 2;
@@ -380,7 +382,7 @@ __device__ __forceinline__ void poly_accumulate(const float* b, const f2* X, con
     const f2 T2 = mul2(E, X[j]);
     SB[j & 1] = add2(SB[j & 1], E);
     SA[j & 1] = add2(SA[j & 1], T2);
-    SC[j & 1] = fma2(mul2(T2, X[j]), phi_q2<T, NC>(X[j]), SC[j & 1]);
+    SC[j & 1] = fma2(mul2(T2, X[j]), phi_q2(X[j]), SC[j & 1]);
   }
   float sb0, sb1, sa0, sa1, sc0, sc1;
   upk(add2(SB[0], SB[1]), sb0, sb1);
@@ -484,7 +486,7 @@ __device__ __forceinline__ void chunk_step(const float* b, const float* q, unsig
   float wax;
   asm volatile("redux.sync.max.NaN.f32 %0, %1, 0xffffffff;" : "=f"(wax) : "f"(max3_nan(ax0, ax1, 0.f)));
   if (wax <= kTau) {
-    poly_accumulate<PE, 2, 9>(b, X, r, a);
+    poly_accumulate<PE>(b, X, r, a);
   } else {
     // Direct path: quant weights in their own frame. x -> +BIG keeps 0*x = 0
     // for masked base entries; x = -inf (quant masked, base finite) makes A
@@ -565,21 +567,20 @@ __device__ __forceinline__ void fail(Ctrl* ctrl, uint32_t* derr) {
 // Row geometry: the unaligned head and tail (< 16 bytes each) are read
 // directly; the 16-byte-aligned body is streamed in tiles.
 struct RowGeom {
-  int64_t head, body_len, tail, ntiles;
+  int64_t head, body_len, tail, nch;  // nch: 512-element chunks of the body
 };
 
 template <int DT>
 __device__ __forceinline__ RowGeom row_geom(const void* rowb, int64_t V) {
   constexpr int EB = Elem<DT>::kBytes;
   constexpr int E = Elem<DT>::kPerVec;
-  constexpr int64_t kStageElems = kStageBytes / EB;
   RowGeom g;
   const uint32_t mis = static_cast<uint32_t>(reinterpret_cast<uintptr_t>(rowb) & 15u);
   g.head = static_cast<int64_t>(((16u - mis) & 15u) / EB);
   if (g.head > V) g.head = V;
   g.body_len = ((V - g.head) / E) * E;
   g.tail = V - g.head - g.body_len;
-  g.ntiles = (g.body_len + kStageElems - 1) / kStageElems;
+  g.nch = (g.body_len + kChunkElems - 1) / kChunkElems;
   return g;
 }
 
@@ -592,9 +593,10 @@ __device__ __forceinline__ int64_t chunk_elem_offset(int chunk_id, int lane, int
 }
 
 // Lowest index holding `m` among the candidate lanes (mask) of one warp's
-// published partial; lanes 0..15 of the calling warp each test one element.
+// published partial (chunk ids counted from body element s0); lanes 0..15 of
+// the calling warp each test one element.
 template <int DT>
-__device__ int rescan_candidates(const void* row, const RowGeom& g, unsigned mask,
+__device__ int rescan_candidates(const void* row, const RowGeom& g, int64_t s0, unsigned mask,
                                  const int* locs, float m, int lane) {
   int best = INT_MAX;
   while (mask) {
@@ -603,7 +605,7 @@ __device__ int rescan_candidates(const void* row, const RowGeom& g, unsigned mas
     const int loc = locs[cl];
     int idx = INT_MAX;
     if (lane < kLaneElems && loc >= 0) {
-      const int64_t off = chunk_elem_offset<DT>(loc, cl, lane);
+      const int64_t off = s0 + chunk_elem_offset<DT>(loc, cl, lane);
       if (off < g.body_len && Elem<DT>::load(row, g.head + off) == m)
         idx = static_cast<int>(g.head + off);
     }
@@ -613,11 +615,189 @@ __device__ int rescan_candidates(const void* row, const RowGeom& g, unsigned mas
   return best;
 }
 
+// One work item: body elements [s0, s1) of row r; part k of parts_per_row.
+struct Item {
+  int64_t r, s0, s1;
+  int k;
+};
+
+template <int DT>
+__device__ __forceinline__ bool item_at(int j, int P, const char* B, int64_t N, int64_t V,
+                                        Item& it, RowGeom& g) {
+  constexpr int EB = Elem<DT>::kBytes;
+  if (P == 1) {
+    it.r = blockIdx.x + static_cast<int64_t>(j) * gridDim.x;
+    if (it.r >= N) return false;
+    g = row_geom<DT>(B + it.r * V * EB, V);
+    it.s0 = 0;
+    it.s1 = g.body_len;
+    it.k = 0;
+    return true;
+  }
+  if (j > 0) return false;
+  it.r = blockIdx.x / P;
+  it.k = static_cast<int>(blockIdx.x % P);
+  g = row_geom<DT>(B + it.r * V * EB, V);
+  const int64_t c0 = g.nch * it.k / P, c1 = g.nch * (it.k + 1) / P;
+  it.s0 = c0 * kChunkElems;
+  it.s1 = c1 * kChunkElems < g.body_len ? c1 * kChunkElems : g.body_len;
+  if (it.s1 < it.s0) it.s1 = it.s0;
+  return true;
+}
+
+// MPart as eight 64-bit words and back (explicit, so no copy goes through
+// local memory).
+__device__ __forceinline__ unsigned long long pack2(float lo, float hi) {
+  return static_cast<unsigned long long>(__float_as_uint(lo)) |
+         (static_cast<unsigned long long>(__float_as_uint(hi)) << 32);
+}
+__device__ __forceinline__ unsigned long long pack2(unsigned lo, unsigned hi) {
+  return static_cast<unsigned long long>(lo) | (static_cast<unsigned long long>(hi) << 32);
+}
+__device__ __forceinline__ void part_words(const MPart& m, unsigned long long (&w)[8]) {
+  w[0] = pack2(m.Mb, m.Mq);
+  w[1] = pack2(m.Cb, m.K);
+  w[2] = static_cast<unsigned long long>(__double_as_longlong(m.Sb));
+  w[3] = static_cast<unsigned long long>(__double_as_longlong(m.A));
+  w[4] = static_cast<unsigned long long>(__double_as_longlong(m.B));
+  w[5] = pack2(static_cast<unsigned>(m.amax_b), static_cast<unsigned>(m.amax_q));
+  w[6] = pack2(m.flags, 0u);
+  w[7] = 0ull;
+}
+__device__ __forceinline__ MPart part_from_words(const unsigned long long (&w)[8]) {
+  MPart m;
+  m.Mb = __uint_as_float(static_cast<unsigned>(w[0]));
+  m.Mq = __uint_as_float(static_cast<unsigned>(w[0] >> 32));
+  m.Cb = __uint_as_float(static_cast<unsigned>(w[1]));
+  m.K = __uint_as_float(static_cast<unsigned>(w[1] >> 32));
+  m.Sb = __longlong_as_double(static_cast<long long>(w[2]));
+  m.A = __longlong_as_double(static_cast<long long>(w[3]));
+  m.B = __longlong_as_double(static_cast<long long>(w[4]));
+  m.amax_b = static_cast<int>(static_cast<unsigned>(w[5]));
+  m.amax_q = static_cast<int>(static_cast<unsigned>(w[5] >> 32));
+  m.flags = static_cast<unsigned>(w[6]);
+  m.pad = 0u;
+  m.pad2 = 0ull;
+  return m;
+}
+
+__device__ __forceinline__ MPart empty_part() {
+  MPart m;
+  m.Mb = m.Mq = -INFINITY;
+  m.Cb = m.K = 0.f;
+  m.Sb = m.A = m.B = 0.0;
+  m.amax_b = m.amax_q = INT_MAX;
+  m.flags = m.pad = 0u;
+  m.pad2 = 0ull;
+  return m;
+}
+
+// Warp-collective merge of the partials held by the lanes. Every lane gets
+// the merged partial: its frame is the largest base frame among parts with
+// base mass, its centre that of the part holding the maximum of b. Moving a
+// part by dK = K' - K and fb = 2^(Cb - Cb'): S' = S fb, A' = (A + dK S) fb,
+// B' = (B + (e^{l dK} - 1)(B + S)) fb. A part without base mass (every b is
+// -inf) carries only quant weight B, moved by one power of two.
+__device__ MPart warp_merge(const MPart& p) {
+  const bool has_b = p.Sb != 0.0;
+  const bool used = has_b || p.B != 0.0;
+  MPart m;
+  m.Mb = warp_max(p.Mb);
+  m.Mq = warp_max(p.Mq);
+  m.flags = __reduce_or_sync(0xffffffffu, p.flags);
+  m.amax_b = __reduce_min_sync(0xffffffffu, p.Mb == m.Mb ? p.amax_b : INT_MAX);
+  m.amax_q = __reduce_min_sync(0xffffffffu, p.Mq == m.Mq ? p.amax_q : INT_MAX);
+  m.pad = 0u;
+  m.pad2 = 0ull;
+  if (__any_sync(0xffffffffu, has_b)) {
+    m.Cb = warp_max(has_b ? p.Cb : -INFINITY);
+    const unsigned kmask = __ballot_sync(0xffffffffu, has_b && p.Mb == m.Mb);
+    m.K = __shfl_sync(0xffffffffu, p.K, kmask ? __ffs(kmask) - 1 : 0);
+  } else {
+    m.Cb = __any_sync(0xffffffffu, used) ? warp_max(used ? p.Cb : -INFINITY) : 0.f;
+    m.K = 0.f;
+  }
+  double sb = 0.0, sa = 0.0, sB = 0.0;
+  const double dK = static_cast<double>(m.K) - static_cast<double>(p.K);
+  if (has_b) {
+    const double fb = pow2i(p.Cb - m.Cb);
+    const double em = expm1(kLambda * dK);
+    sb = p.Sb * fb;
+    sa = (m.flags & kPartInfKl) ? 0.0 : (p.A + dK * p.Sb) * fb;
+    sB = (p.B + em * (p.B + p.Sb)) * fb;
+  } else if (used) {
+    sB = p.B * exp2(static_cast<double>(p.Cb) - static_cast<double>(m.Cb) + dK * kLog2eD);
+  }
+  m.Sb = warp_sum(sb);
+  m.A = warp_sum(sa);
+  m.B = warp_sum(sB);
+  return m;
+}
+
+// The record of a whole row from its merged partial.
+__device__ kld_row_t finalize_row(const MPart& m, bool has_tok, bool tok_ok, float q_tok) {
+  kld_row_t rec;
+  uint32_t flags = 0;
+  if (has_tok && !tok_ok) flags |= KLD_ROW_BAD_TOKEN;
+  const double nan = __longlong_as_double(0x7ff8000000000000ll);
+  rec.kld = nan;
+  rec.nll = nan;
+  rec.argmax_base = -1;
+  rec.argmax_quant = -1;
+  const bool nonfinite = (m.flags & (kPartNonfinite | kPartFailed)) || isnan(m.Sb) || isnan(m.B) ||
+                         !(m.Mb < INFINITY) || !(m.Mq < INFINITY);
+  if (nonfinite) {
+    flags |= KLD_ROW_NONFINITE;
+  } else if (m.Mb == -INFINITY || m.Mq == -INFINITY) {
+    flags |= KLD_ROW_EMPTY;
+  } else {
+    if (m.flags & kPartInfKl) {
+      rec.kld = INFINITY;
+      flags |= KLD_ROW_INF_KL;
+    } else {
+      rec.kld = -kLambda * (m.A / m.Sb) + log1p(m.B / m.Sb);
+    }
+    if (tok_ok) {
+      if (q_tok == -INFINITY) {
+        rec.nll = INFINITY;
+        flags |= KLD_ROW_INF_NLL;
+      } else {
+        // B + S is the sum of all quant weights in frame Cb - K*L.
+        rec.nll = log(m.B + m.Sb) +
+                  kLn2 * (static_cast<double>(m.Cb) -
+                          (static_cast<double>(m.K) + static_cast<double>(q_tok)) * kLog2eD);
+      }
+    }
+    rec.argmax_base = m.amax_b;
+    rec.argmax_quant = m.amax_q;
+  }
+  rec.flags = flags;
+  rec.reserved = 0u;
+  return rec;
+}
+
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ uint32_t cluster_nctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ uint32_t map_to_rank(uint32_t local, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local), "r"(rank));
+  return r;
+}
+
 template <int DT>
 __global__ void __launch_bounds__(kRowThreads, 1)
     kld_rows_kernel(const void* __restrict__ base, const void* __restrict__ quant,
                     const int32_t* __restrict__ tok, int64_t N, int64_t V,
-                    kld_row_t* __restrict__ rows, uint32_t* __restrict__ derr) {
+                    kld_row_t* __restrict__ rows, uint32_t* __restrict__ derr, int P,
+                    MPart* __restrict__ gparts, unsigned* __restrict__ tickets) {
   constexpr int EB = Elem<DT>::kBytes;
   constexpr int E = Elem<DT>::kPerVec;
   constexpr int kStageElems = kStageBytes / EB;
@@ -631,6 +811,7 @@ __global__ void __launch_bounds__(kRowThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  const uint32_t G = P > 1 ? cluster_nctarank() : 1u;  // CTAs per cluster
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -641,10 +822,15 @@ __global__ void __launch_bounds__(kRowThreads, 1)
       mbar_init(smem_u32(&ctrl->slot_full[s]), kConsumerWarps);
       mbar_init(smem_u32(&ctrl->slot_empty[s]), 1);
     }
+    mbar_init(smem_u32(&ctrl->cl_full), G > 1 ? G - 1 : 1);
     ctrl->abort = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   __syncthreads();
+  if (G > 1) {
+    // Peers push into this CTA's barrier and slots only after it initialised them.
+    asm volatile("barrier.cluster.arrive.release;\n\tbarrier.cluster.wait.acquire;" ::: "memory");
+  }
 
   const char* B = static_cast<const char*>(base);
   const char* Q = static_cast<const char*>(quant);
@@ -653,37 +839,46 @@ __global__ void __launch_bounds__(kRowThreads, 1)
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       const uint64_t pol = evict_first_policy();
-      uint32_t it = 0;
+      int s = 0;
+      uint32_t ph = 0u;
+      uint32_t issued = 0;
       bool ok = true;
-      for (int64_t r = blockIdx.x; r < N && ok; r += gridDim.x) {
-        const char* rb = B + r * V * EB;
-        const char* rq = Q + r * V * EB;
-        const RowGeom g = row_geom<DT>(rb, V);
-        for (int64_t t = 0; t < g.ntiles; ++t, ++it) {
-          const int s = static_cast<int>(it % kStages);
-          const uint32_t ph = (it / kStages) & 1u;
+      Item it;
+      RowGeom g;
+      for (int j = 0; ok && item_at<DT>(j, P, B, N, V, it, g); ++j) {
+        const char* rb = B + it.r * V * EB;
+        const char* rq = Q + it.r * V * EB;
+        const int64_t n = it.s1 - it.s0;
+        const int64_t ntiles = (n + kStageElems - 1) / kStageElems;
+        for (int64_t t = 0; t < ntiles; ++t) {
           if (!mbar_wait(smem_u32(&ctrl->empty[s]), ph ^ 1u, abort)) {
             fail(ctrl, derr);
             ok = false;
             break;
           }
-          const int64_t off = g.head + t * kStageElems;
-          int64_t len = g.body_len - t * kStageElems;
+          const int64_t off = g.head + it.s0 + t * kStageElems;
+          int64_t len = n - t * kStageElems;
           if (len > kStageElems) len = kStageElems;
           const uint32_t bytes = static_cast<uint32_t>(len * EB);
           const uint32_t fb = smem_u32(&ctrl->full[s]);
           mbar_arrive_expect_tx(fb, 2u * bytes);
           bulk_load(smem_u32(stage_b + s * kStageBytes), rb + off * EB, bytes, fb, pol);
           bulk_load(smem_u32(stage_q + s * kStageBytes), rq + off * EB, bytes, fb, pol);
+          ++issued;
+          if (++s == kStages) {
+            s = 0;
+            ph ^= 1u;
+          }
         }
       }
       // Never leave with copies in flight: wait (bounded) for the last
       // stages issued. In a normal run they have long completed.
-      const uint32_t last = it < kStages ? it : kStages;
+      const uint32_t last = issued < kStages ? issued : kStages;
       for (uint32_t k = 0; k < last; ++k) {
-        const uint32_t j = it - 1u - k;
-        const int s = static_cast<int>(j % kStages);
-        const uint32_t ph = (j / kStages) & 1u;
+        if (--s < 0) {
+          s = kStages - 1;
+          ph ^= 1u;
+        }
         const uint32_t fb = smem_u32(&ctrl->full[s]);
         if (!mbar_try_wait(fb, ph)) {
           const uint64_t t0 = globaltimer();
@@ -696,31 +891,29 @@ __global__ void __launch_bounds__(kRowThreads, 1)
         }
       }
     }
-    return;
-  }
-
-  if (warp < kConsumerWarps) {
+  } else if (warp < kConsumerWarps) {
     // ----------------------------------------------------------- consumers
     constexpr int kChunksPerWarp = kChunksPerTile / kConsumerWarps;
     static_assert(kChunksPerTile % kConsumerWarps == 0, "chunks must split evenly");
     int s = 0;         // stage of the next tile
     uint32_t ph = 0u;  // its phase parity
-    int rowk = 0;
-    for (int64_t r = blockIdx.x; r < N; r += gridDim.x, ++rowk) {
-      const char* rb = B + r * V * EB;
-      const RowGeom g = row_geom<DT>(rb, V);
+    // One item of n body elements (chunk ids count from its start): stream
+    // its tiles, then publish the warp partial in slot j % kSlots. The
+    // whole-row and split-row loops below each inline their own copy, so
+    // the split bookkeeping costs the whole-row loop no registers.
+    auto consume = [&](int n, int j) -> bool {
       Ref ref{-INFINITY, -INFINITY, 0.f, 0.f, 0.f};
       Acc acc{0.0, 0.0, 0.0, 0.0, 0.0, 0.0};
       Best best{-INFINITY, -INFINITY, -1, -1};
-      const int ntiles = static_cast<int>(g.ntiles);
+      const int ntiles = (n + kStageElems - 1) / kStageElems;
       for (int t = 0; t < ntiles; ++t) {
         if (!mbar_wait(smem_u32(&ctrl->full[s]), ph, abort)) {
           fail(ctrl, derr);
-          return;
+          return false;
         }
         const uint4* tb = reinterpret_cast<const uint4*>(stage_b + s * kStageBytes);
         const uint4* tq = reinterpret_cast<const uint4*>(stage_q + s * kStageBytes);
-        const int64_t rem = g.body_len - static_cast<int64_t>(t) * kStageElems;
+        const int rem = n - t * kStageElems;
         if (rem >= kStageElems) {
           // Full tile: this warp's chunks, no masking.
 #pragma unroll
@@ -730,7 +923,7 @@ __global__ void __launch_bounds__(kRowThreads, 1)
                                      0, ref, acc, best, t * kChunksPerTile + c);
           }
         } else {
-          const int len = static_cast<int>(rem);
+          const int len = rem;
 #pragma unroll 1
           for (int k = 0; k < kChunksPerWarp; ++k) {
             const int c = warp + k * kConsumerWarps;
@@ -749,8 +942,8 @@ __global__ void __launch_bounds__(kRowThreads, 1)
       }
 
       // Publish the warp partial into the slot ring.
-      const int slot = rowk % kSlots;
-      const uint32_t sph = (rowk / kSlots) & 1u;
+      const int slot = j % kSlots;
+      const uint32_t sph = (j / kSlots) & 1u;
       const double Sb = warp_sum(acc.Sb), Ap = warp_sum(acc.Ap), C = warp_sum(acc.C);
       const double Ad = warp_sum(acc.Ad), Se = warp_sum(acc.Se), Sh = warp_sum(acc.Sh);
       const float wq = warp_max(best.q);  // the warp's maximum of q
@@ -758,7 +951,7 @@ __global__ void __launch_bounds__(kRowThreads, 1)
       const unsigned cq_mask = __ballot_sync(0xffffffffu, wq > -INFINITY && best.q == wq);
       if (!mbar_wait(smem_u32(&ctrl->slot_empty[slot]), sph ^ 1u, abort)) {
         fail(ctrl, derr);
-        return;
+        return false;
       }
       Slot& sl = ctrl->slot[slot];
       if ((cb_mask >> lane) & 1u) sl.loc_b[warp][lane] = best.lb;
@@ -783,175 +976,309 @@ __global__ void __launch_bounds__(kRowThreads, 1)
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&ctrl->slot_full[slot]));
-    }
-    return;
-  }
-
-  // ------------------------------------------------------------------ epilogue
-  int rowk = 0;
-  for (int64_t r = blockIdx.x; r < N; r += gridDim.x, ++rowk) {
-    const char* rb = B + r * V * EB;
-    const char* rq = Q + r * V * EB;
-    const RowGeom g = row_geom<DT>(rb, V);
-
-    // Head/tail elements (one per lane) and the next-token gather, issued
-    // before waiting for the consumers' partials.
-    const int n_extra = static_cast<int>(g.head + g.tail);
-    float xe_b = -INFINITY, xe_q = -INFINITY;
-    int idx_e = INT_MAX;
-    if (lane < n_extra) {
-      const int64_t j = lane < g.head ? lane : g.head + g.body_len + (lane - g.head);
-      idx_e = static_cast<int>(j);
-      xe_b = Elem<DT>::load(rb, j);
-      xe_q = Elem<DT>::load(rq, j);
-    }
-    int32_t tk = 0;
-    bool tok_ok = false;
-    float q_tok = 0.f;
-    if (tok != nullptr) {
-      tk = __ldg(tok + r);
-      tok_ok = tk >= 0 && static_cast<int64_t>(tk) < V;
-      if (tok_ok && lane == 0) q_tok = Elem<DT>::load(rq, tk);
-    }
-
-    // The head/tail as one more partial of the same form.
-    Ref eref{-INFINITY, -INFINITY, 0.f, 0.f, 0.f};
-    Acc eacc{0.0, 0.0, 0.0, 0.0, 0.0, 0.0};
-    Best ebest{-INFINITY, -INFINITY, -1, -1};
-    if (n_extra > 0) {
-      chunk_step<1>(&xe_b, &xe_q, lane < n_extra ? 1u : 0u, eref, eacc, ebest, 0);
-    }
-    const float eMq = warp_max(xe_q);
-    const double eSb = warp_sum(eacc.Sb), eAp = warp_sum(eacc.Ap), eC = warp_sum(eacc.C);
-    const double eAd = warp_sum(eacc.Ad), eSe = warp_sum(eacc.Se), eSh = warp_sum(eacc.Sh);
-
-    const int slot = rowk % kSlots;
-    const uint32_t sph = (rowk / kSlots) & 1u;
-    if (!mbar_wait(smem_u32(&ctrl->slot_full[slot]), sph, abort)) {
-      fail(ctrl, derr);
-      return;
-    }
-    const Slot& sl = ctrl->slot[slot];
-
-    // Lane w < 16 takes warp w's partial, lane 16 the head/tail partial.
-    WarpPart p;
-    if (lane < kConsumerWarps) {
-      p = sl.part[lane];
-    } else {
-      p.Mb = p.Mq = -INFINITY;
-      p.Rb = p.Rq = p.K = 0.f;
-      p.pad = 0;
-      p.Sb = p.Ap = p.C = p.Ad = p.Se = p.Sh = 0.0;
-      p.cand_b = p.cand_q = 0u;
-      if (lane == kConsumerWarps) {
-        p.Mb = eref.Mb;
-        p.Mq = eMq;
-        p.Rb = eref.Rb;
-        p.Rq = eref.Rq;
-        p.K = eref.K;
-        p.Sb = eSb;
-        p.Ap = eAp;
-        p.C = eC;
-        p.Ad = eAd;
-        p.Se = eSe;
-        p.Sh = eSh;
+      return true;
+    };
+    if (P == 1) {
+      for (int j = 0;; ++j) {
+        const int64_t r = blockIdx.x + static_cast<int64_t>(j) * gridDim.x;
+        if (r >= N) break;
+        const RowGeom g = row_geom<DT>(B + r * V * EB, V);
+        if (!consume(static_cast<int>(g.body_len), j)) break;
       }
-    }
-    const float Mb = warp_max(p.Mb);
-    const float Mq = warp_max(p.Mq);
-    const bool nan_part = isnan(p.Sb) || isnan(p.Sh) || isnan(p.C);
-    const bool nonfinite = __any_sync(0xffffffffu, nan_part) || !(Mb < INFINITY) ||
-                           !(Mq < INFINITY);
-    const bool empty = Mb == -INFINITY || Mq == -INFINITY;
-
-    uint32_t flags = 0;
-    if (tok != nullptr && !tok_ok) flags |= KLD_ROW_BAD_TOKEN;
-    double kl = __longlong_as_double(0x7ff8000000000000ll);  // NaN
-    double nll = kl;
-    int ab = -1, aq = -1;
-    if (nonfinite) {
-      flags |= KLD_ROW_NONFINITE;
-    } else if (empty) {
-      flags |= KLD_ROW_EMPTY;
     } else {
-      // Common frames and centre.
-      const float Cb = warp_max(p.Mb > -INFINITY ? p.Rb : -INFINITY);
-      // Centre of the part that holds the row maximum of b.
-      const unsigned kmask = __ballot_sync(0xffffffffu, p.Mb == Mb);
-      const float Kref = __shfl_sync(0xffffffffu, p.K, __ffs(kmask) - 1);
-      // Only direct-path sums can be infinite: b_j finite where q_j = -inf.
-      const bool inf_kl = __any_sync(0xffffffffu, !isfinite(p.Ad));
-      const double dK = static_cast<double>(Kref) - static_cast<double>(p.K);
-      const double fb = p.Mb > -INFINITY ? pow2i(p.Rb - Cb) : 0.0;
-      // Polynomial-path part of B in the warp's own centre, moved to Kref:
-      // e^{l(x+d)} - 1 = e^{l d}(e^{l x} - 1) + (e^{l d} - 1).
-      const double Bp = kLambda * p.Ap + p.C;
-      const double Sp = p.Sb - p.Se;
-      const double em = expm1(kLambda * dK);
-      const double BpK = Bp + em * (Bp + Sp);
-      // Direct-path quant weights, from their own frame to Cb - Kref*L.
-      const double Bh = p.Sh != 0.0
-                            ? p.Sh * exp2(static_cast<double>(p.Rq) - static_cast<double>(Cb) +
-                                          static_cast<double>(Kref) * kLog2eD)
-                            : 0.0;
-      const double sb = warp_sum(p.Sb * fb);
-      const double sbB = warp_sum(BpK * fb + Bh - p.Se * fb);
-      const double sa = warp_sum(inf_kl ? 0.0 : (p.Ap + p.Ad + dK * p.Sb) * fb);
-      if (inf_kl) {
-        kl = INFINITY;
-        flags |= KLD_ROW_INF_KL;
+      Item it;
+      RowGeom g;
+      item_at<DT>(0, P, B, N, V, it, g);
+      consume(static_cast<int>(it.s1 - it.s0), 0);
+    }
+  } else {
+    // ---------------------------------------------------------------- epilogue
+    Item it;
+    RowGeom g;
+    for (int j = 0; item_at<DT>(j, P, B, N, V, it, g); ++j) {
+      const int64_t r = it.r;
+      const char* rb = B + r * V * EB;
+      const char* rq = Q + r * V * EB;
+      // Head/tail elements (one per lane; part 0 of a row only), issued
+      // before waiting for the consumers' partials.
+      const int n_extra = it.k == 0 ? static_cast<int>(g.head + g.tail) : 0;
+      float xe_b = -INFINITY, xe_q = -INFINITY;
+      int idx_e = INT_MAX;
+      if (lane < n_extra) {
+        const int64_t jj = lane < g.head ? lane : g.head + g.body_len + (lane - g.head);
+        idx_e = static_cast<int>(jj);
+        xe_b = Elem<DT>::load(rb, jj);
+        xe_q = Elem<DT>::load(rq, jj);
+      }
+      Ref eref{-INFINITY, -INFINITY, 0.f, 0.f, 0.f};
+      Acc eacc{0.0, 0.0, 0.0, 0.0, 0.0, 0.0};
+      Best ebest{-INFINITY, -INFINITY, -1, -1};
+      if (n_extra > 0) chunk_step<1>(&xe_b, &xe_q, lane < n_extra ? 1u : 0u, eref, eacc, ebest, 0);
+      const float eMq = warp_max(xe_q);
+      const double eSb = warp_sum(eacc.Sb), eAp = warp_sum(eacc.Ap), eC = warp_sum(eacc.C);
+      const double eAd = warp_sum(eacc.Ad), eSe = warp_sum(eacc.Se), eSh = warp_sum(eacc.Sh);
+
+      const int slot = j % kSlots;
+      const uint32_t sph = (j / kSlots) & 1u;
+      const bool got = mbar_wait(smem_u32(&ctrl->slot_full[slot]), sph, abort);
+      MPart m = empty_part();
+      if (!got) {
+        // Whole rows: nothing is written for this or later rows. Split rows:
+        // the part still travels, flagged, so the row's combine completes.
+        fail(ctrl, derr);
+        if (P == 1) break;
+        m.flags = kPartFailed;
       } else {
-        kl = -kLambda * (sa / sb) + log1p(sbB / sb);
-      }
-      if (tok_ok) {
-        const float qt = __shfl_sync(0xffffffffu, q_tok, 0);
-        if (qt == -INFINITY) {
-          nll = INFINITY;
-          flags |= KLD_ROW_INF_NLL;
+      const Slot& sl = ctrl->slot[slot];
+
+      // Lane w < 16 holds warp w's partial, lane 16 the head/tail partial,
+      // each as a merged partial in its own frame and centre.
+      MPart mp = empty_part();
+      unsigned cand_b = 0u, cand_q = 0u;
+      if (lane <= kConsumerWarps) {
+        WarpPart p;
+        if (lane < kConsumerWarps) {
+          p = sl.part[lane];
+          cand_b = p.cand_b;
+          cand_q = p.cand_q;
         } else {
-          // B + S is the sum of all quant weights in frame Cb - Kref*L.
-          nll = log(sbB + sb) +
-                kLn2 * (static_cast<double>(Cb) -
-                        (static_cast<double>(Kref) + static_cast<double>(qt)) * kLog2eD);
+          p.Mb = eref.Mb;
+          p.Mq = eMq;
+          p.Rb = eref.Rb;
+          p.Rq = eref.Rq;
+          p.K = eref.K;
+          p.Sb = eSb;
+          p.Ap = eAp;
+          p.C = eC;
+          p.Ad = eAd;
+          p.Se = eSe;
+          p.Sh = eSh;
         }
+        mp.Mb = p.Mb;
+        mp.Mq = p.Mq;
+        if (p.Mb > -INFINITY) {
+          mp.Cb = p.Rb;
+          mp.K = p.K;
+          mp.Sb = p.Sb;
+          mp.A = p.Ap + p.Ad;
+          // direct-path quant weights from their own frame to Rb - K*L
+          const double Bh = p.Sh != 0.0 ? p.Sh * exp2(static_cast<double>(p.Rq) -
+                                                       static_cast<double>(p.Rb) +
+                                                       static_cast<double>(p.K) * kLog2eD)
+                                        : 0.0;
+          mp.B = kLambda * p.Ap + p.C + Bh - p.Se;
+        } else {
+          // no finite b: only quant weights, in their own frame (K = 0)
+          mp.Cb = p.Rq;
+          mp.B = p.Sh;
+        }
+        if (isnan(p.Sb) || isnan(p.Sh) || isnan(p.C)) mp.flags |= kPartNonfinite;
+        if (!isfinite(p.Ad)) mp.flags |= kPartInfKl;
       }
-      // Lowest index of each row maximum.
-      int amb = (xe_b == Mb) ? idx_e : INT_MAX;
-      int amq = (xe_q == Mq) ? idx_e : INT_MAX;
-      amb = __reduce_min_sync(0xffffffffu, amb);
-      amq = __reduce_min_sync(0xffffffffu, amq);
-      unsigned wb = __ballot_sync(0xffffffffu, lane < kConsumerWarps && p.Mb == Mb);
-      unsigned wq = __ballot_sync(0xffffffffu, lane < kConsumerWarps && p.Mq == Mq);
-      while (wb) {
-        const int w = __ffs(wb) - 1;
-        wb &= wb - 1u;
-        const unsigned cm = __shfl_sync(0xffffffffu, p.cand_b, w);
-        const int i = rescan_candidates<DT>(rb, g, cm, sl.loc_b[w], Mb, lane);
-        if (i < amb) amb = i;
+      m = warp_merge(mp);
+
+      // Exact lowest index of this part's maxima: re-read only the chunks
+      // of lanes whose maximum equals it.
+      if (!(m.flags & kPartNonfinite)) {
+        const bool fin_b = m.Mb > -INFINITY && m.Mb < INFINITY;
+        const bool fin_q = m.Mq > -INFINITY && m.Mq < INFINITY;
+        int amb = (fin_b && xe_b == m.Mb) ? idx_e : INT_MAX;
+        int amq = (fin_q && xe_q == m.Mq) ? idx_e : INT_MAX;
+        amb = __reduce_min_sync(0xffffffffu, amb);
+        amq = __reduce_min_sync(0xffffffffu, amq);
+        unsigned wb = __ballot_sync(0xffffffffu, fin_b && lane < kConsumerWarps && mp.Mb == m.Mb);
+        unsigned wq = __ballot_sync(0xffffffffu, fin_q && lane < kConsumerWarps && mp.Mq == m.Mq);
+        while (wb) {
+          const int w = __ffs(wb) - 1;
+          wb &= wb - 1u;
+          const unsigned cm = __shfl_sync(0xffffffffu, cand_b, w);
+          const int i = rescan_candidates<DT>(rb, g, it.s0, cm, sl.loc_b[w], m.Mb, lane);
+          if (i < amb) amb = i;
+        }
+        while (wq) {
+          const int w = __ffs(wq) - 1;
+          wq &= wq - 1u;
+          const unsigned cm = __shfl_sync(0xffffffffu, cand_q, w);
+          const int i = rescan_candidates<DT>(rq, g, it.s0, cm, sl.loc_q[w], m.Mq, lane);
+          if (i < amq) amq = i;
+        }
+        m.amax_b = amb;
+        m.amax_q = amq;
       }
-      while (wq) {
-        const int w = __ffs(wq) - 1;
-        wq &= wq - 1u;
-        const unsigned cm = __shfl_sync(0xffffffffu, p.cand_q, w);
-        const int i = rescan_candidates<DT>(rq, g, cm, sl.loc_q[w], Mq, lane);
-        if (i < amq) amq = i;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&ctrl->slot_empty[slot]));
       }
-      ab = amb;
-      aq = amq;
-    }
-    __syncwarp();
-    if (lane == 0) {
-      mbar_arrive(smem_u32(&ctrl->slot_empty[slot]));
-      kld_row_t rec;
-      rec.kld = kl;
-      rec.nll = nll;
-      rec.argmax_base = ab;
-      rec.argmax_quant = aq;
-      rec.flags = flags;
-      rec.reserved = 0u;
-      rows[r] = rec;
+
+      // Next-token gather (only the CTA that finalises the row needs it).
+      int32_t tk = 0;
+      bool tok_ok = false;
+      float q_tok = 0.f;
+      auto gather_token = [&]() {
+        if (tok != nullptr) {
+          tk = __ldg(tok + r);
+          tok_ok = tk >= 0 && static_cast<int64_t>(tk) < V;
+          if (tok_ok) q_tok = Elem<DT>::load(rq, tk);
+        }
+      };
+
+      if (P == 1) {
+        gather_token();
+        const kld_row_t rec = finalize_row(m, tok != nullptr, tok_ok, q_tok);
+        if (lane == 0) rows[r] = rec;
+        continue;
+      }
+
+      // ---------------- split row: cluster combine through DSMEM, then across
+      // the row's clusters through global memory and a ticket.
+      const uint32_t rank = G > 1 ? cluster_ctarank() : 0u;
+      if (G > 1 && rank != 0) {
+        // Push this CTA's partial into the leader's shared memory, then
+        // arrive on the leader's barrier (release at cluster scope).
+        if (lane == 0) {
+          const uint32_t dst = map_to_rank(smem_u32(&ctrl->cl_part[rank]), 0u);
+          unsigned long long wds[8];
+          part_words(m, wds);
+#pragma unroll
+          for (int w = 0; w < 8; ++w)
+            asm volatile("st.shared::cluster.u64 [%0], %1;" ::"r"(dst + 8 * w), "l"(wds[w])
+                         : "memory");
+          const uint32_t bar = map_to_rank(smem_u32(&ctrl->cl_full), 0u);
+          asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar)
+                       : "memory");
+        }
+        continue;
+      }
+      MPart cm = m;
+      if (G > 1) {
+        // Wait (bounded) for the peers' partials; every lane acquires them.
+        const uint32_t bar = smem_u32(&ctrl->cl_full);
+        uint32_t okw = 0;
+        const uint64_t t0 = globaltimer();
+        for (uint32_t i = 0;; ++i) {
+          asm volatile(
+              "{\n\t.reg .pred p;\n\t"
+              "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], 0;\n\t"
+              "selp.u32 %0, 1, 0, p;\n\t}"
+              : "=r"(okw)
+              : "r"(bar)
+              : "memory");
+          if (okw) break;
+          if ((i & 63u) == 63u && globaltimer() - t0 > kWaitLimitNs) break;
+        }
+        MPart q = empty_part();
+        if (__all_sync(0xffffffffu, okw != 0)) {
+          if (lane == 0) q = m;
+          if (lane >= 1 && lane < static_cast<int>(G)) {
+            const ulonglong2* src = reinterpret_cast<const ulonglong2*>(&ctrl->cl_part[lane]);
+            unsigned long long wds[8];
+#pragma unroll
+            for (int w = 0; w < 4; ++w) {
+              const ulonglong2 v = src[w];
+              wds[2 * w] = v.x;
+              wds[2 * w + 1] = v.y;
+            }
+            q = part_from_words(wds);
+          }
+        } else {
+          fail(ctrl, derr);
+          if (lane == 0) {
+            q = m;
+            q.flags |= kPartFailed;
+          }
+        }
+        cm = warp_merge(q);
+      }
+      const int C = P / static_cast<int>(G);  // clusters per row
+      if (C == 1) {
+        gather_token();
+        const kld_row_t rec = finalize_row(cm, tok != nullptr, tok_ok, q_tok);
+        if (lane == 0) rows[r] = rec;
+        continue;
+      }
+      const int cid = it.k / static_cast<int>(G);
+      unsigned ticket = 0u;
+      if (lane == 0) {
+        unsigned long long wds[8];
+        part_words(cm, wds);
+        ulonglong2* dst = reinterpret_cast<ulonglong2*>(&gparts[r * C + cid]);
+#pragma unroll
+        for (int w = 0; w < 4; ++w) dst[w] = make_ulonglong2(wds[2 * w], wds[2 * w + 1]);
+        __threadfence();
+        ticket = atomicAdd(&tickets[r], 1u);
+      }
+      ticket = __shfl_sync(0xffffffffu, ticket, 0);
+      if (ticket != static_cast<unsigned>(C - 1)) continue;  // not the last cluster
+      __threadfence();
+      MPart q = empty_part();
+      if (lane < C) {
+        const ulonglong2* src = reinterpret_cast<const ulonglong2*>(&gparts[r * C + lane]);
+        unsigned long long wds[8];
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+          const ulonglong2 v = __ldcg(src + w);
+          wds[2 * w] = v.x;
+          wds[2 * w + 1] = v.y;
+        }
+        q = part_from_words(wds);
+      }
+      const MPart fm = warp_merge(q);
+      gather_token();
+      const kld_row_t rec = finalize_row(fm, tok != nullptr, tok_ok, q_tok);
+      if (lane == 0) {
+        rows[r] = rec;
+        tickets[r] = 0u;  // ready for the next launch
+      }
     }
   }
+
+  if (G > 1) {
+    // No CTA leaves while a peer may still store into its shared memory.
+    __syncwarp();
+    asm volatile("barrier.cluster.arrive.release;\n\tbarrier.cluster.wait.acquire;" ::: "memory");
+  }
+}
+
+template <int DT>
+int max_active_clusters(int cluster_ctas) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(cluster_ctas * 32));
+  cfg.blockDim = dim3(kRowThreads);
+  cfg.dynamicSmemBytes = kRowSmemBytes;
+  cudaLaunchAttribute attr;
+  attr.id = cudaLaunchAttributeClusterDimension;
+  attr.val.clusterDim.x = static_cast<unsigned>(cluster_ctas);
+  attr.val.clusterDim.y = 1;
+  attr.val.clusterDim.z = 1;
+  cfg.attrs = &attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, kld_rows_kernel<DT>, &cfg) != cudaSuccess) {
+    cudaGetLastError();
+    return 0;
+  }
+  return n;
+}
+
+template <int DT>
+cudaError_t launch_typed(const void* base, const void* quant, const int32_t* tok, int64_t N,
+                         int64_t V, kld_row_t* rows, uint32_t* derr, const RowPlan& pl,
+                         const SplitScratch* split, cudaStream_t stream) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(pl.grid));
+  cfg.blockDim = dim3(kRowThreads);
+  cfg.dynamicSmemBytes = kRowSmemBytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr;
+  attr.id = cudaLaunchAttributeClusterDimension;
+  attr.val.clusterDim.x = static_cast<unsigned>(pl.cluster_ctas);
+  attr.val.clusterDim.y = 1;
+  attr.val.clusterDim.z = 1;
+  cfg.attrs = &attr;
+  cfg.numAttrs = pl.parts_per_row > 1 ? 1 : 0;
+  MPart* gp = split ? static_cast<MPart*>(split->parts) : nullptr;
+  unsigned* tk = split ? split->tickets : nullptr;
+  return cudaLaunchKernelEx(&cfg, kld_rows_kernel<DT>, base, quant, tok, N, V, rows, derr,
+                            pl.parts_per_row, gp, tk);
 }
 
 }  // namespace
@@ -968,27 +1295,70 @@ cudaError_t prepare_rows_kernels() {
                               cudaFuncAttributeMaxDynamicSharedMemorySize, kRowSmemBytes);
 }
 
+RowPlan plan_rows(int64_t N, int sm_count, int max_active_clusters_for_8, bool split_allowed) {
+  RowPlan pl;
+  pl.parts_per_row = 1;
+  pl.cluster_ctas = 1;
+  pl.grid = static_cast<int>(N < sm_count ? N : sm_count);
+  if (pl.grid < 1) pl.grid = 1;
+  if (!split_allowed || N * 2 > sm_count) return pl;
+  // Largest cluster (power of two, <= 8) with one cluster per row in one wave.
+  int G = kMaxClusterCtas;
+  while (G > 1 && N * G > sm_count) G >>= 1;
+  if (G < 2) return pl;
+  // Clusters of 8 that fit at once, scaled to the chosen size.
+  int fit = max_active_clusters_for_8 * (kMaxClusterCtas / G);
+  if (fit < 1) fit = sm_count / G;
+  int C = static_cast<int>(fit / N);
+  if (C < 1) C = 1;
+  if (C > 32) C = 32;  // a row's clusters are merged by one warp
+  pl.cluster_ctas = G;
+  pl.parts_per_row = G * C;
+  pl.grid = static_cast<int>(N) * pl.parts_per_row;
+  return pl;
+}
+
+// Clusters of kMaxClusterCtas CTAs the current device holds at once, asked
+// once per device and element type (0 if the query fails).
+int max_active_clusters8(kld_dtype_t dtype) {
+  constexpr int kMaxDevices = 64;
+  static std::atomic<int> cache[kMaxDevices][3];  // 0: not asked yet; else count + 1
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 0;
+  const int t = dtype == KLD_F32 ? 0 : (dtype == KLD_BF16 ? 1 : 2);
+  const int c = cache[dev][t].load(std::memory_order_relaxed);
+  if (c > 0) return c - 1;
+  int n = 0;
+  switch (dtype) {
+    case KLD_F32: n = max_active_clusters<KLD_F32>(kMaxClusterCtas); break;
+    case KLD_BF16: n = max_active_clusters<KLD_BF16>(kMaxClusterCtas); break;
+    case KLD_F16: n = max_active_clusters<KLD_F16>(kMaxClusterCtas); break;
+  }
+  cache[dev][t].store(n + 1, std::memory_order_relaxed);
+  return n;
+}
+
 cudaError_t launch_rows(const void* base, const void* quant, const int32_t* token_ids, int64_t N,
-                        int64_t V, kld_dtype_t dtype, kld_row_t* rows, uint32_t* derr, int grid,
-                        cudaStream_t stream) {
-  const dim3 g(static_cast<unsigned>(grid)), b(kRowThreads);
+                        int64_t V, kld_dtype_t dtype, kld_row_t* rows, uint32_t* derr,
+                        int sm_count, const SplitScratch* split, cudaStream_t stream) {
+  RowPlan pl = plan_rows(N, sm_count, 0, false);
+  if (split != nullptr && N * 2 <= sm_count) {
+    // No split when the device reports no room for a cluster of 8 at once.
+    const int mac = max_active_clusters8(dtype);
+    if (mac > 0) pl = plan_rows(N, sm_count, mac, true);
+    if (static_cast<int64_t>(pl.grid) / pl.cluster_ctas > split->capacity || N > split->capacity) {
+      pl = plan_rows(N, sm_count, 0, false);
+    }
+  }
   switch (dtype) {
     case KLD_F32:
-      kld_rows_kernel<KLD_F32><<<g, b, kRowSmemBytes, stream>>>(base, quant, token_ids, N, V, rows,
-                                                                 derr);
-      break;
+      return launch_typed<KLD_F32>(base, quant, token_ids, N, V, rows, derr, pl, split, stream);
     case KLD_BF16:
-      kld_rows_kernel<KLD_BF16><<<g, b, kRowSmemBytes, stream>>>(base, quant, token_ids, N, V,
-                                                                  rows, derr);
-      break;
+      return launch_typed<KLD_BF16>(base, quant, token_ids, N, V, rows, derr, pl, split, stream);
     case KLD_F16:
-      kld_rows_kernel<KLD_F16><<<g, b, kRowSmemBytes, stream>>>(base, quant, token_ids, N, V, rows,
-                                                                 derr);
-      break;
-    default:
-      return cudaErrorInvalidValue;
+      return launch_typed<KLD_F16>(base, quant, token_ids, N, V, rows, derr, pl, split, stream);
   }
-  return cudaGetLastError();
+  return cudaErrorInvalidValue;
 }
 
 }  // namespace kld

@@ -107,13 +107,13 @@ extern "C" kld_status_t kld_stats_run_static(const void* base, const void* quant
   kld_row_t* rows = reinterpret_cast<kld_row_t*>(scratch);
   uint32_t* derr = reinterpret_cast<uint32_t*>(scratch + kRowsBytes);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const int grid = static_cast<int>(N < dev.sm_count ? N : dev.sm_count);
 
   // The array keeps the previous call's contents: the error word must start
   // at zero (the records are rewritten for every row before they are read).
   cudaError_t e = cudaMemsetAsync(derr, 0, sizeof(uint32_t), s);
   if (e != cudaSuccess) return fail_cuda(e);
-  e = kld::launch_rows(base, quant, token_ids, N, V, dtype, rows, derr, grid, s);
+  // Whole-row mode only: split rows would need scratch beyond the fixed array.
+  e = kld::launch_rows(base, quant, token_ids, N, V, dtype, rows, derr, dev.sm_count, nullptr, s);
   if (e != cudaSuccess) return fail_cuda(e);
   e = kld::launch_reduce(rows, N, token_ids != nullptr, derr, result_dev, s);
   if (e != cudaSuccess) return fail_cuda(e);

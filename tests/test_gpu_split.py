@@ -1,0 +1,133 @@
+"""Split-row launches (few rows: each row's chunks spread over thread-block
+clusters of CTAs whose partial sums merge in shared memory, then across
+clusters through global memory) against the fp64 CPU oracle.
+
+Rows <= SMs / 2 take this path; the largest cluster is 8 CTAs, and a row may
+span several clusters. The cases put maxima, ties, NaN, masks and the
+target token in parts other than the first, leave parts with no chunk at
+small vocabularies, and reuse one handle so that the per-row arrival
+counters must come back to zero after every launch.
+"""
+import ctypes
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from logit_kl_divergence_b200 import KLDStats, _lib, dtype_code, synth
+
+from gpu_helpers import ODT, assert_rows_match, assert_select_exact, assert_stats_match, gpu_run
+
+pytestmark = pytest.mark.gpu
+DEV = torch.device("cuda", 0)
+V_FULL = 151936
+
+
+def _sm_count():
+    return torch.cuda.get_device_properties(DEV).multi_processor_count
+
+
+def _parity(base, quant, tok, odt):
+    g_rows, gres = gpu_run(base.to(DEV), quant.to(DEV), None if tok is None else tok.to(DEV))
+    o_rows, ores = oracle.run(base, quant, tok, odt)
+    assert_rows_match(g_rows, o_rows)
+    assert_stats_match(gres, ores)
+    assert_select_exact(g_rows, gres, tok is not None)
+    return g_rows, gres
+
+
+@pytest.mark.parametrize("dtype", [synth.F32, synth.BF16])
+@pytest.mark.parametrize("n", [1, 2, 3, 4, 7, 9, 16, 20, 37, 38, 64, 74])
+def test_split_rows_full_vocabulary(n, dtype):
+    st = KLDStats(max_rows=n, device=DEV)
+    p = st.plan(n, V_FULL, _lib.KLD_F32 if dtype == synth.F32 else _lib.KLD_BF16)
+    st.close()
+    if 2 * n <= _sm_count():
+        assert p["variant"] == 1 and p["ctas_per_row"] >= 2
+    w = synth.make_recipe("ctx", n=n, v=V_FULL, dtype=dtype, seed=100 + n)
+    _parity(w.base, w.quant, w.token_ids, ODT[dtype])
+
+
+@pytest.mark.parametrize("v", [1, 7, 512, 513, 1024, 4097, 16385, 100003])
+def test_split_rows_small_vocabularies_leave_parts_empty(v):
+    w = synth.make_recipe("ctx", n=2, v=v, dtype=synth.F16, seed=v)
+    _parity(w.base, w.quant, w.token_ids, oracle.F16)
+
+
+def test_split_rows_ties_across_parts_lowest_index_wins():
+    n, v = 3, V_FULL
+    g = torch.Generator().manual_seed(11)
+    b = torch.randn((n, v), generator=g)
+    q = b + 0.1 * torch.randn((n, v), generator=g)
+    b[0, [150000, 70001, 70000, 151935]] = 30.0      # lowest tie in a middle part
+    q[0, [151935, 99999]] = 40.0
+    b[1, [151935, 1]] = 30.0                          # head element vs last element
+    q[1, [0, 151935]] = 40.0
+    b[2, [151000, 150999]] = 30.0                     # both in the last part
+    q[2, [2047, 2048, 4095]] = 40.0
+    g_rows, _ = _parity(b.contiguous(), q.contiguous(), None, oracle.F32)
+    assert list(g_rows["amax_b"]) == [70000, 1, 150999]
+    assert list(g_rows["amax_q"]) == [99999, 0, 2047]
+
+
+def test_split_rows_special_values_in_later_parts():
+    n, v = 6, V_FULL
+    g = torch.Generator().manual_seed(12)
+    b = torch.randn((n, v), generator=g)
+    q = b + 0.3 * torch.randn((n, v), generator=g)
+    b[0, :100000] = -math.inf                         # parts with quant weight only
+    q[0, :100000] += 2.0
+    b[1] -= 1000.0                                    # deep frames, same masks
+    q[1] -= 1000.0
+    b[1, :100000] = -math.inf
+    b[2, 150000] = math.nan                           # NaN in the last part
+    q[3, 140000] = -math.inf                          # KL = +inf from a late part
+    b[4, :] = -math.inf                               # one finite base entry, late
+    b[4, 151000] = 3.0
+    q[5, 120000:] = -math.inf                         # quant mask over the last parts
+    b[5, 120000:] = -math.inf
+    tok = torch.tensor([5, 50000, 7, 140000, 151000, 130000], dtype=torch.int32)
+    g_rows, gres = _parity(b.contiguous(), q.contiguous(), tok, oracle.F32)
+    assert g_rows["amax_b"][4] == 151000
+    assert math.isinf(g_rows["kld"][3]) and math.isinf(g_rows["nll"][3])
+    assert math.isinf(g_rows["nll"][5])
+
+
+def test_split_rows_repeat_launches_on_one_handle():
+    st = KLDStats(max_rows=8, device=DEV)
+    try:
+        for n, v, dt, seed in [(1, V_FULL, synth.F32, 1), (5, 70001, synth.BF16, 2),
+                               (1, V_FULL, synth.F32, 3), (8, 4097, synth.F16, 4),
+                               (2, V_FULL, synth.BF16, 5)]:
+            w = synth.make_recipe("ctx", n=n, v=v, dtype=dt, seed=seed)
+            st.run(w.base.to(DEV), w.quant.to(DEV), w.token_ids.to(DEV))
+            gres = st.result()
+            _, ores = oracle.run(w.base, w.quant, w.token_ids, ODT[dt])
+            assert_stats_match(dict(gres), ores)
+    finally:
+        st.close()
+
+
+def test_split_rows_agree_with_whole_row_launch():
+    # kld_stats_run_static keeps whole rows at any N: the same rows through
+    # both launch shapes must agree with the oracle.
+    w = synth.make_recipe("ctx", n=6, v=V_FULL, dtype=synth.BF16, seed=13)
+    b, q, t = w.base.to(DEV), w.quant.to(DEV), w.token_ids.to(DEV)
+    lib = _lib.load()
+    out = torch.zeros(ctypes.sizeof(_lib.Result), dtype=torch.uint8, device=DEV)
+    stream = torch.cuda.current_stream(DEV)
+    st = lib.kld_stats_run_static(ctypes.c_void_p(b.data_ptr()), ctypes.c_void_p(q.data_ptr()),
+                                  ctypes.c_void_p(t.data_ptr()), 6, V_FULL, dtype_code(b),
+                                  ctypes.c_void_p(out.data_ptr()), ctypes.c_void_p(stream.cuda_stream))
+    assert st == _lib.KLD_OK
+    stream.synchronize()
+    res = _lib.Result.from_buffer_copy(bytes(out.cpu().numpy()))
+    whole = {name: getattr(res, name) for name, _ in _lib.Result._fields_ if not name.startswith("reserved")}
+    _, split = gpu_run(b, q, t)
+    _, ores = oracle.run(w.base, w.quant, w.token_ids, oracle.BF16)
+    for r in (whole, split):
+        assert int(r["top1_agree"]) == int(ores["top1_agree"])
+        for k in ("mean_kld", "median_kld", "max_kld", "mean_nll"):
+            assert math.isclose(r[k], ores[k], rel_tol=1e-5, abs_tol=1e-9), (k, r[k], ores[k])
