@@ -197,6 +197,22 @@ kld_status_t kld_stats_run_host(kld_stats_t h, const void* base_host,
                                 int64_t V, kld_dtype_t dtype, void* stream);
 
 /*
+ * Launch shape of the row pass for few rows (N <= SMs / 2), where whole-row
+ * launches would leave most SMs idle and each row is split into parts
+ * instead (see kld_plan):
+ *   -1: never split (one CTA per row at any N);
+ *    0: the library default (currently 1);
+ *    1: split over independent CTAs, merged through global memory;
+ *    2, 4, 8: split over thread-block clusters of up to that many CTAs,
+ *       merged first through distributed shared memory, then across the
+ *       row's clusters through global memory.
+ * Results agree within rounding whatever the shape. Measured on B200 with
+ * V = 262144 fp32 rows, plain CTAs were as fast as or up to ~10% faster than
+ * clusters, hence the default. Other values: KLD_ERR_INVALID_ARG.
+ */
+kld_status_t kld_stats_set_split(kld_stats_t h, int cluster_ctas);
+
+/*
  * Kernel timing of the next runs: when enabled, kld_stats_run records CUDA
  * events around its row pass and its reduction; kld_stats_timing() returns
  * the last run's durations in milliseconds (waits for that run).
@@ -207,16 +223,17 @@ kld_status_t kld_stats_timing(kld_stats_t h, float* row_pass_ms,
 
 /*
  * Launch plan of the row pass for (N, V, dtype) on a device with sm_count
- * SMs: variant 0 = whole rows (one persistent CTA per SM, each taking rows
- * r, r + grid, ...); variant 1 = split rows, used when N <= sm_count / 2 so
- * that few rows still occupy the GPU: each row's 512-element chunks are
- * divided among ctas_per_row CTAs, grouped in thread-block clusters of
- * cluster_ctas CTAs (a power of two <= 8) whose partial sums meet in the
- * cluster leader's shared memory; the row's clusters then meet through a
- * small global scratch and an arrival counter. Also: threads per CTA,
- * dynamic shared memory bytes, stage bytes per operand, stages. Pure host
- * logic; enqueues nothing. The launch itself may lower ctas_per_row when the
- * device can hold fewer clusters at once than sm_count / cluster_ctas (the
+ * SMs, for the default split setting (kld_stats_set_split): variant 0 =
+ * whole rows (one persistent CTA per SM, each taking rows r, r + grid, ...);
+ * variant 1 = split rows, used when N <= sm_count / 2 so that few rows still
+ * occupy the GPU: each row's 512-element chunks are divided among
+ * ctas_per_row CTAs, in groups (thread-block clusters when cluster_ctas > 1,
+ * whose partial sums meet in the cluster leader's shared memory) that meet
+ * through a small global scratch and a per-row arrival counter; all of a
+ * launch's CTAs fit on the device at once. Also: threads per CTA, dynamic
+ * shared memory bytes, stage bytes per operand, stages. Pure host logic;
+ * enqueues nothing. With clusters the launch may use fewer CTAs per row when
+ * the device holds fewer clusters at once than sm_count / cluster_ctas (the
  * count comes from cudaOccupancyMaxActiveClusters).
  */
 typedef struct {

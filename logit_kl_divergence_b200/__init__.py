@@ -171,6 +171,11 @@ class KLDStats:
         view = torch.as_tensor(_DeviceBytes(p.value, nbytes), device=self.device)
         return view.view(n.value, ROW_RECORD_BYTES).clone()
 
+    def set_split(self, cluster_ctas: int) -> None:
+        """Few-row launch shape: -1 never split rows, 0 default, 1 plain
+        CTAs, 2/4/8 thread-block clusters of up to that many CTAs."""
+        _lib.check(self._lib.kld_stats_set_split(self._h, int(cluster_ctas)), "kld_stats_set_split")
+
     def set_timing(self, enable: bool) -> None:
         _lib.check(self._lib.kld_stats_set_timing(self._h, int(bool(enable))), "kld_stats_set_timing")
 

@@ -63,7 +63,7 @@ struct kld_stats_s {
   int64_t max_rows = 0;
   kld_row_t* rows = nullptr;
   void* split_mem = nullptr;  // split-row scratch: partials, then tickets
-  kld::SplitScratch split = {nullptr, nullptr, 0};
+  kld::SplitScratch split = {nullptr, nullptr, 0, kld::kDefaultClusterCtas};
   kld_result_t* dres = nullptr;
   uint32_t* derr = nullptr;
   kld_result_t* hres = nullptr;
@@ -144,7 +144,7 @@ kld_status_t kld_plan(int64_t N, int64_t V, kld_dtype_t dtype, int sm_count, kld
   if (!valid_dtype(dtype)) return KLD_ERR_DTYPE;
   if (N < 1 || V < 1 || V > INT32_MAX || sm_count < 1) return KLD_ERR_INVALID_ARG;
   std::memset(out, 0, sizeof(*out));
-  const kld::RowPlan pl = kld::plan_rows(N, sm_count, 0, true);
+  const kld::RowPlan pl = kld::plan_rows(N, sm_count, nullptr, kld::kDefaultClusterCtas);
   out->variant = pl.parts_per_row > 1 ? 1 : 0;
   out->grid = pl.grid;
   out->ctas_per_row = pl.parts_per_row;
@@ -312,6 +312,16 @@ kld_status_t kld_stats_rows(kld_stats_t h, const kld_row_t** rows_dev, int64_t* 
   *rows_dev = h->rows;
   *n_rows = h->last_rows;
   return KLD_OK;
+}
+
+kld_status_t kld_stats_set_split(kld_stats_t h, int cluster_ctas) {
+  if (!h) return KLD_ERR_INVALID_ARG;
+  switch (cluster_ctas) {
+    case -1: h->split.max_cluster_ctas = 0; return KLD_OK;
+    case 0: h->split.max_cluster_ctas = kld::kDefaultClusterCtas; return KLD_OK;
+    case 1: case 2: case 4: case 8: h->split.max_cluster_ctas = cluster_ctas; return KLD_OK;
+    default: return KLD_ERR_INVALID_ARG;
+  }
 }
 
 kld_status_t kld_stats_set_timing(kld_stats_t h, int enable) {

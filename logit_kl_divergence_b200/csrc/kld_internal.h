@@ -37,7 +37,10 @@ struct SplitScratch {
   void* parts;
   unsigned* tickets;
   int capacity;
+  int max_cluster_ctas;  // largest cluster the plan may use (1: plain CTAs)
 };
+// Cluster size split rows use unless the caller asks otherwise.
+constexpr int kDefaultClusterCtas = 1;
 
 // Dynamic shared memory of the row kernel: stages for both operands, then the
 // control block (mbarriers and the partial slots).
@@ -64,7 +67,12 @@ cudaError_t launch_rows(const void* base, const void* quant,
 struct RowPlan {
   int grid, parts_per_row, cluster_ctas;
 };
-RowPlan plan_rows(int64_t N, int sm_count, int max_active_clusters_for_8, bool split_allowed);
+// fit[i]: clusters of 2^i CTAs the device holds at once (i = 0..3; <= 0:
+// unknown, estimated as sm_count >> i). Split rows only when N <= sm_count/2
+// and max_cluster_ctas >= 1: the cluster is the largest power of two <=
+// max_cluster_ctas that leaves one cluster per row in one wave, and each row
+// takes as many clusters (<= 32) as still fit in that wave.
+RowPlan plan_rows(int64_t N, int sm_count, const int fit[4], int max_cluster_ctas);
 cudaError_t prepare_rows_kernels();  // per-device attribute setup
 
 cudaError_t launch_reduce(const kld_row_t* rows, int64_t N, int has_nll,

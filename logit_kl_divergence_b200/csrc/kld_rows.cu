@@ -827,10 +827,11 @@ __global__ void __launch_bounds__(kRowThreads, 1)
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   __syncthreads();
-  if (G > 1) {
-    // Peers push into this CTA's barrier and slots only after it initialised them.
-    asm volatile("barrier.cluster.arrive.release;\n\tbarrier.cluster.wait.acquire;" ::: "memory");
-  }
+  // Cluster barrier, first phase: every thread arrives now (the barrier
+  // initialisation above is released with it) and waits only where it next
+  // touches a peer's shared memory, so no CTA stalls here at start-up.
+  bool cl_waited = false;
+  if (G > 1) asm volatile("barrier.cluster.arrive.release;" ::: "memory");
 
   const char* B = static_cast<const char*>(base);
   const char* Q = static_cast<const char*>(quant);
@@ -1132,8 +1133,11 @@ __global__ void __launch_bounds__(kRowThreads, 1)
       // the row's clusters through global memory and a ticket.
       const uint32_t rank = G > 1 ? cluster_ctarank() : 0u;
       if (G > 1 && rank != 0) {
-        // Push this CTA's partial into the leader's shared memory, then
-        // arrive on the leader's barrier (release at cluster scope).
+        // Push this CTA's partial into the leader's shared memory (its
+        // barrier is initialised once the first cluster phase completes),
+        // then arrive on the leader's barrier (release at cluster scope).
+        asm volatile("barrier.cluster.wait.acquire;" ::: "memory");
+        cl_waited = true;
         if (lane == 0) {
           const uint32_t dst = map_to_rank(smem_u32(&ctrl->cl_part[rank]), 0u);
           unsigned long long wds[8];
@@ -1232,8 +1236,9 @@ __global__ void __launch_bounds__(kRowThreads, 1)
   }
 
   if (G > 1) {
-    // No CTA leaves while a peer may still store into its shared memory.
-    __syncwarp();
+    // Second phase: no CTA leaves while a peer may still store into its
+    // shared memory.
+    if (!cl_waited) asm volatile("barrier.cluster.wait.acquire;" ::: "memory");
     asm volatile("barrier.cluster.arrive.release;\n\tbarrier.cluster.wait.acquire;" ::: "memory");
   }
 }
@@ -1274,7 +1279,7 @@ cudaError_t launch_typed(const void* base, const void* quant, const int32_t* tok
   attr.val.clusterDim.y = 1;
   attr.val.clusterDim.z = 1;
   cfg.attrs = &attr;
-  cfg.numAttrs = pl.parts_per_row > 1 ? 1 : 0;
+  cfg.numAttrs = pl.cluster_ctas > 1 ? 1 : 0;
   MPart* gp = split ? static_cast<MPart*>(split->parts) : nullptr;
   unsigned* tk = split ? split->tickets : nullptr;
   return cudaLaunchKernelEx(&cfg, kld_rows_kernel<DT>, base, quant, tok, N, V, rows, derr,
@@ -1295,60 +1300,61 @@ cudaError_t prepare_rows_kernels() {
                               cudaFuncAttributeMaxDynamicSharedMemorySize, kRowSmemBytes);
 }
 
-RowPlan plan_rows(int64_t N, int sm_count, int max_active_clusters_for_8, bool split_allowed) {
+RowPlan plan_rows(int64_t N, int sm_count, const int fit[4], int max_cluster_ctas) {
   RowPlan pl;
   pl.parts_per_row = 1;
   pl.cluster_ctas = 1;
   pl.grid = static_cast<int>(N < sm_count ? N : sm_count);
   if (pl.grid < 1) pl.grid = 1;
-  if (!split_allowed || N * 2 > sm_count) return pl;
-  // Largest cluster (power of two, <= 8) with one cluster per row in one wave.
-  int G = kMaxClusterCtas;
-  while (G > 1 && N * G > sm_count) G >>= 1;
-  if (G < 2) return pl;
-  // Clusters of 8 that fit at once, scaled to the chosen size.
-  int fit = max_active_clusters_for_8 * (kMaxClusterCtas / G);
-  if (fit < 1) fit = sm_count / G;
-  int C = static_cast<int>(fit / N);
-  if (C < 1) C = 1;
-  if (C > 32) C = 32;  // a row's clusters are merged by one warp
-  pl.cluster_ctas = G;
-  pl.parts_per_row = G * C;
-  pl.grid = static_cast<int>(N) * pl.parts_per_row;
+  if (max_cluster_ctas < 1 || N * 2 > sm_count) return pl;
+  int lg = 0;
+  while (lg < 3 && (2 << lg) <= max_cluster_ctas) ++lg;
+  for (; lg >= 0; --lg) {
+    const int G = 1 << lg;
+    const int f = fit != nullptr && fit[lg] > 0 ? fit[lg] : sm_count / G;
+    if (f < N) continue;  // not one cluster per row in one wave
+    int C = static_cast<int>(f / N);
+    if (C > 32) C = 32;  // a row's clusters are merged by one warp
+    if (G * C < 2) continue;
+    pl.cluster_ctas = G;
+    pl.parts_per_row = G * C;
+    pl.grid = static_cast<int>(N) * pl.parts_per_row;
+    return pl;
+  }
   return pl;
 }
 
-// Clusters of kMaxClusterCtas CTAs the current device holds at once, asked
-// once per device and element type (0 if the query fails).
-int max_active_clusters8(kld_dtype_t dtype) {
+// Clusters of 2^lg CTAs the current device holds at once, asked once per
+// device, element type and size (0 if the query fails).
+int active_clusters(kld_dtype_t dtype, int lg) {
   constexpr int kMaxDevices = 64;
-  static std::atomic<int> cache[kMaxDevices][3];  // 0: not asked yet; else count + 1
+  static std::atomic<int> cache[kMaxDevices][3][4];  // 0: not asked yet; else count + 1
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 0;
   const int t = dtype == KLD_F32 ? 0 : (dtype == KLD_BF16 ? 1 : 2);
-  const int c = cache[dev][t].load(std::memory_order_relaxed);
+  const int c = cache[dev][t][lg].load(std::memory_order_relaxed);
   if (c > 0) return c - 1;
   int n = 0;
   switch (dtype) {
-    case KLD_F32: n = max_active_clusters<KLD_F32>(kMaxClusterCtas); break;
-    case KLD_BF16: n = max_active_clusters<KLD_BF16>(kMaxClusterCtas); break;
-    case KLD_F16: n = max_active_clusters<KLD_F16>(kMaxClusterCtas); break;
+    case KLD_F32: n = max_active_clusters<KLD_F32>(1 << lg); break;
+    case KLD_BF16: n = max_active_clusters<KLD_BF16>(1 << lg); break;
+    case KLD_F16: n = max_active_clusters<KLD_F16>(1 << lg); break;
   }
-  cache[dev][t].store(n + 1, std::memory_order_relaxed);
+  cache[dev][t][lg].store(n + 1, std::memory_order_relaxed);
   return n;
 }
 
 cudaError_t launch_rows(const void* base, const void* quant, const int32_t* token_ids, int64_t N,
                         int64_t V, kld_dtype_t dtype, kld_row_t* rows, uint32_t* derr,
                         int sm_count, const SplitScratch* split, cudaStream_t stream) {
-  RowPlan pl = plan_rows(N, sm_count, 0, false);
-  if (split != nullptr && N * 2 <= sm_count) {
-    // No split when the device reports no room for a cluster of 8 at once.
-    const int mac = max_active_clusters8(dtype);
-    if (mac > 0) pl = plan_rows(N, sm_count, mac, true);
-    if (static_cast<int64_t>(pl.grid) / pl.cluster_ctas > split->capacity || N > split->capacity) {
-      pl = plan_rows(N, sm_count, 0, false);
-    }
+  RowPlan pl = plan_rows(N, sm_count, nullptr, 0);
+  if (split != nullptr && N * 2 <= sm_count && split->max_cluster_ctas >= 1) {
+    int fit[4] = {0, 0, 0, 0};
+    for (int lg = 0; lg < 4 && (1 << lg) <= split->max_cluster_ctas; ++lg)
+      fit[lg] = active_clusters(dtype, lg);
+    pl = plan_rows(N, sm_count, fit, split->max_cluster_ctas);
+    if (static_cast<int64_t>(pl.grid) / pl.cluster_ctas > split->capacity || N > split->capacity)
+      pl = plan_rows(N, sm_count, nullptr, 0);
   }
   switch (dtype) {
     case KLD_F32:

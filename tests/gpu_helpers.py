@@ -27,9 +27,12 @@ STAT_ATOL = {"mean_kld": 1e-9, "median_kld": 1e-9, "p90_kld": 1e-9, "p99_kld": 1
 CORES = max(1, os.cpu_count() or 1)
 
 
-def gpu_run(base, quant, tok=None, use_rows_api=False):
-    """The whole statistic on the GPU; returns (per-row numpy dict, result)."""
+def gpu_run(base, quant, tok=None, use_rows_api=False, split=None):
+    """The whole statistic on the GPU; returns (per-row numpy dict, result).
+    ``split``: the handle's few-row launch shape (kld_stats_set_split)."""
     st = KLDStats(max_rows=base.shape[0], device=base.device)
+    if split is not None:
+        st.set_split(split)
     try:
         if use_rows_api:
             out = torch.empty((base.shape[0], 32), dtype=torch.uint8, device=base.device)

@@ -2,11 +2,13 @@
 clusters of CTAs whose partial sums merge in shared memory, then across
 clusters through global memory) against the fp64 CPU oracle.
 
-Rows <= SMs / 2 take this path; the largest cluster is 8 CTAs, and a row may
-span several clusters. The cases put maxima, ties, NaN, masks and the
-target token in parts other than the first, leave parts with no chunk at
-small vocabularies, and reuse one handle so that the per-row arrival
-counters must come back to zero after every launch.
+Rows <= SMs / 2 take this path. By default a row is split over plain CTAs
+(kld_stats_set_split(1)); the cluster shapes (2, 4, 8 CTAs, combined through
+distributed shared memory) and whole-row launches (-1) are selected
+explicitly here. The cases put maxima, ties, NaN, masks and the target token
+in parts other than the first, leave parts with no chunk at small
+vocabularies, and reuse one handle so that the per-row arrival counters must
+come back to zero after every launch.
 """
 import ctypes
 import math
@@ -29,8 +31,12 @@ def _sm_count():
     return torch.cuda.get_device_properties(DEV).multi_processor_count
 
 
-def _parity(base, quant, tok, odt):
-    g_rows, gres = gpu_run(base.to(DEV), quant.to(DEV), None if tok is None else tok.to(DEV))
+SHAPES = [1, 2, 4, 8]  # split over plain CTAs, then clusters of up to 2, 4, 8 CTAs
+
+
+def _parity(base, quant, tok, odt, split=None):
+    g_rows, gres = gpu_run(base.to(DEV), quant.to(DEV), None if tok is None else tok.to(DEV),
+                           split=split)
     o_rows, ores = oracle.run(base, quant, tok, odt)
     assert_rows_match(g_rows, o_rows)
     assert_stats_match(gres, ores)
@@ -50,13 +56,22 @@ def test_split_rows_full_vocabulary(n, dtype):
     _parity(w.base, w.quant, w.token_ids, ODT[dtype])
 
 
+@pytest.mark.parametrize("split", SHAPES + [-1])
+@pytest.mark.parametrize("n", [1, 3, 9, 20, 38, 74])
+def test_every_launch_shape_full_vocabulary(n, split):
+    w = synth.make_recipe("ctx", n=n, v=V_FULL, dtype=synth.F32, seed=200 + n)
+    _parity(w.base, w.quant, w.token_ids, oracle.F32, split=split)
+
+
+@pytest.mark.parametrize("split", [1, 8])
 @pytest.mark.parametrize("v", [1, 7, 512, 513, 1024, 4097, 16385, 100003])
-def test_split_rows_small_vocabularies_leave_parts_empty(v):
+def test_split_rows_small_vocabularies_leave_parts_empty(v, split):
     w = synth.make_recipe("ctx", n=2, v=v, dtype=synth.F16, seed=v)
-    _parity(w.base, w.quant, w.token_ids, oracle.F16)
+    _parity(w.base, w.quant, w.token_ids, oracle.F16, split=split)
 
 
-def test_split_rows_ties_across_parts_lowest_index_wins():
+@pytest.mark.parametrize("split", SHAPES)
+def test_split_rows_ties_across_parts_lowest_index_wins(split):
     n, v = 3, V_FULL
     g = torch.Generator().manual_seed(11)
     b = torch.randn((n, v), generator=g)
@@ -67,12 +82,13 @@ def test_split_rows_ties_across_parts_lowest_index_wins():
     q[1, [0, 151935]] = 40.0
     b[2, [151000, 150999]] = 30.0                     # both in the last part
     q[2, [2047, 2048, 4095]] = 40.0
-    g_rows, _ = _parity(b.contiguous(), q.contiguous(), None, oracle.F32)
+    g_rows, _ = _parity(b.contiguous(), q.contiguous(), None, oracle.F32, split=split)
     assert list(g_rows["amax_b"]) == [70000, 1, 150999]
     assert list(g_rows["amax_q"]) == [99999, 0, 2047]
 
 
-def test_split_rows_special_values_in_later_parts():
+@pytest.mark.parametrize("split", SHAPES)
+def test_split_rows_special_values_in_later_parts(split):
     n, v = 6, V_FULL
     g = torch.Generator().manual_seed(12)
     b = torch.randn((n, v), generator=g)
@@ -89,7 +105,7 @@ def test_split_rows_special_values_in_later_parts():
     q[5, 120000:] = -math.inf                         # quant mask over the last parts
     b[5, 120000:] = -math.inf
     tok = torch.tensor([5, 50000, 7, 140000, 151000, 130000], dtype=torch.int32)
-    g_rows, gres = _parity(b.contiguous(), q.contiguous(), tok, oracle.F32)
+    g_rows, gres = _parity(b.contiguous(), q.contiguous(), tok, oracle.F32, split=split)
     assert g_rows["amax_b"][4] == 151000
     assert math.isinf(g_rows["kld"][3]) and math.isinf(g_rows["nll"][3])
     assert math.isinf(g_rows["nll"][5])
@@ -98,9 +114,11 @@ def test_split_rows_special_values_in_later_parts():
 def test_split_rows_repeat_launches_on_one_handle():
     st = KLDStats(max_rows=8, device=DEV)
     try:
-        for n, v, dt, seed in [(1, V_FULL, synth.F32, 1), (5, 70001, synth.BF16, 2),
-                               (1, V_FULL, synth.F32, 3), (8, 4097, synth.F16, 4),
-                               (2, V_FULL, synth.BF16, 5)]:
+        for n, v, dt, seed, split in [(1, V_FULL, synth.F32, 1, 0), (5, 70001, synth.BF16, 2, 8),
+                                      (1, V_FULL, synth.F32, 3, 4), (8, 4097, synth.F16, 4, 1),
+                                      (2, V_FULL, synth.BF16, 5, 2), (3, V_FULL, synth.F32, 6, -1),
+                                      (1, V_FULL, synth.F32, 7, 0)]:
+            st.set_split(split)
             w = synth.make_recipe("ctx", n=n, v=v, dtype=dt, seed=seed)
             st.run(w.base.to(DEV), w.quant.to(DEV), w.token_ids.to(DEV))
             gres = st.result()
@@ -131,3 +149,15 @@ def test_split_rows_agree_with_whole_row_launch():
         assert int(r["top1_agree"]) == int(ores["top1_agree"])
         for k in ("mean_kld", "median_kld", "max_kld", "mean_nll"):
             assert math.isclose(r[k], ores[k], rel_tol=1e-5, abs_tol=1e-9), (k, r[k], ores[k])
+
+
+def test_set_split_rejects_unknown_shapes():
+    st = KLDStats(max_rows=4, device=DEV)
+    try:
+        for bad in (-2, 3, 5, 16):
+            with pytest.raises(_lib.KLDError):
+                st.set_split(bad)
+        for ok in (-1, 0, 1, 2, 4, 8):
+            st.set_split(ok)
+    finally:
+        st.close()
