@@ -1,10 +1,11 @@
 // kld_api.cu -- host side of the C ABI declared in include/kld_stats.h.
 //
-// Owns the per-handle device workspace (one 32-byte record per row, the
-// device result, an error word), the pinned host copy of the result and the
-// staging buffers of the host-memory path; validates arguments before
-// anything is enqueued and maps CUDA failures to status codes. Every step of
-// the statistic runs in the kernels of kld_rows.cu and kld_reduce.cu.
+// Owns the per-handle device workspace (one 32-byte record per row, an
+// error word, the split-row scratch), the mapped pinned host result that the
+// reduction kernel writes directly, and the staging buffers of the
+// host-memory path; validates arguments before anything is enqueued and maps
+// CUDA failures to status codes. Every step of the statistic runs in the
+// kernels of kld_rows.cu and kld_reduce.cu.
 #include <cuda_runtime.h>
 
 #include <cstdint>
@@ -64,9 +65,9 @@ struct kld_stats_s {
   kld_row_t* rows = nullptr;
   void* split_mem = nullptr;  // split-row scratch: partials, then tickets
   kld::SplitScratch split = {nullptr, nullptr, 0, kld::kDefaultClusterCtas};
-  kld_result_t* dres = nullptr;
   uint32_t* derr = nullptr;
-  kld_result_t* hres = nullptr;
+  kld_result_t* hres = nullptr;      // pinned, mapped host memory
+  kld_result_t* hres_dev = nullptr;  // its device-side pointer
   cudaEvent_t done = nullptr;
   bool has_result = false;
   int64_t last_rows = 0;
@@ -106,9 +107,10 @@ cudaError_t launch_rows(kld_stats_s* h, const void* base, const void* quant, con
 
 kld_status_t enqueue_reduce(kld_stats_t h, const kld_row_t* rows, int64_t N, int has_nll,
                             cudaStream_t s) {
-  KLD_CUDA(kld::launch_reduce(rows, N, has_nll, h->derr, h->dres, s));
+  // The reduction writes the result straight into the handle's mapped
+  // pinned host buffer: no separate device-to-host copy.
+  KLD_CUDA(kld::launch_reduce(rows, N, has_nll, h->derr, h->hres_dev, s));
   if (h->timing && h->timing_valid) KLD_CUDA(cudaEventRecord(h->tev[2], s));
-  KLD_CUDA(cudaMemcpyAsync(h->hres, h->dres, sizeof(kld_result_t), cudaMemcpyDeviceToHost, s));
   KLD_CUDA(cudaEventRecord(h->done, s));
   h->has_result = true;
   return KLD_OK;
@@ -188,8 +190,6 @@ kld_status_t kld_stats_create(kld_stats_t* out, int64_t max_rows, int device) {
     cudaError_t err;
     if ((err = cudaMalloc(&h->rows, sizeof(kld_row_t) * static_cast<size_t>(max_rows))) !=
         cudaSuccess) { st = cuda_fail(err, "cudaMalloc(rows)"); break; }
-    if ((err = cudaMalloc(&h->dres, sizeof(kld_result_t))) != cudaSuccess) {
-      st = cuda_fail(err, "cudaMalloc(result)"); break; }
     if ((err = cudaMalloc(&h->derr, sizeof(uint32_t))) != cudaSuccess) {
       st = cuda_fail(err, "cudaMalloc(error word)"); break; }
     if ((err = cudaMemset(h->derr, 0, sizeof(uint32_t))) != cudaSuccess) {
@@ -208,8 +208,12 @@ kld_status_t kld_stats_create(kld_stats_t* out, int64_t max_rows, int device) {
       h->split.tickets = reinterpret_cast<unsigned*>(static_cast<char*>(h->split_mem) + pbytes);
       h->split.capacity = sms;
     }
-    if ((err = cudaMallocHost(&h->hres, sizeof(kld_result_t))) != cudaSuccess) {
-      st = cuda_fail(err, "cudaMallocHost"); break; }
+    if ((err = cudaHostAlloc(reinterpret_cast<void**>(&h->hres), sizeof(kld_result_t),
+                             cudaHostAllocMapped | cudaHostAllocPortable)) != cudaSuccess) {
+      st = cuda_fail(err, "cudaHostAlloc"); break; }
+    std::memset(h->hres, 0, sizeof(kld_result_t));
+    if ((err = cudaHostGetDevicePointer(reinterpret_cast<void**>(&h->hres_dev), h->hres, 0)) !=
+        cudaSuccess) { st = cuda_fail(err, "cudaHostGetDevicePointer"); break; }
     if ((err = cudaEventCreateWithFlags(&h->done, cudaEventDisableTiming)) != cudaSuccess) {
       st = cuda_fail(err, "cudaEventCreate"); break; }
     for (int i = 0; i < 3 && st == KLD_OK; ++i)
@@ -240,7 +244,6 @@ void kld_stats_destroy(kld_stats_t h) {
   if (h->done) cudaEventDestroy(h->done);
   if (h->hres) cudaFreeHost(h->hres);
   if (h->derr) cudaFree(h->derr);
-  if (h->dres) cudaFree(h->dres);
   if (h->rows) cudaFree(h->rows);
   if (h->split_mem) cudaFree(h->split_mem);
   delete h;

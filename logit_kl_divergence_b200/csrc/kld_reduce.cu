@@ -11,9 +11,11 @@
 //   percentile = x_(k) + (pos - k) * (x_(k+1) - x_(k)),  pos = p*(n-1),
 //                k = floor(pos), over the sorted valid KL values; max = x_(n-1).
 //
-// One CTA of 1024 threads:
-//   1. thread t sums records t, t+1024, ... in order; the 1024 partials are
-//      combined by a fixed shuffle tree, so the fp64 sums are deterministic.
+// One CTA of T threads (T = 1024, or N rounded up to a warp multiple between
+// 128 and 1024 when N is smaller, so small inputs pay for few threads):
+//   1. thread t sums records t, t+T, ... in order; the T partials are
+//      combined by a fixed shuffle tree, so the fp64 sums are deterministic
+//      for a given N.
 //   2. the up to seven ranks the percentiles need are selected exactly with
 //      an MSB-first radix select on order-preserving 64-bit keys of the
 //      doubles (8 bits per pass, one shared histogram per distinct prefix,
@@ -73,12 +75,16 @@ __global__ void __launch_bounds__(kReduceThreads, 1)
   __shared__ ReduceShared sh;
   const int tid = threadIdx.x;
   const int lane = tid & 31, warp = tid >> 5;
+  const int nt = static_cast<int>(blockDim.x);
+  // Launched as a programmatic dependent of the row pass: its launch may
+  // overlap the row pass, the records are read only after it completed.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
 
   // ---------------------------------------------------------------- sums
   double s_kl = 0.0, s_nll = 0.0;
   long long n_valid = 0, agree = 0, n_nll = 0, n_flag = 0;
   unsigned int f_or = 0;
-  for (int64_t i = tid; i < N; i += kReduceThreads) {
+  for (int64_t i = tid; i < N; i += nt) {
     const kld_row_t rec = rows[i];
     f_or |= rec.flags;
     if (rec.flags) ++n_flag;
@@ -112,13 +118,14 @@ __global__ void __launch_bounds__(kReduceThreads, 1)
   }
   __syncthreads();
   if (warp == 0) {
-    s_kl = sh.dsum[lane][0];
-    s_nll = sh.dsum[lane][1];
-    n_valid = sh.isum[lane][0];
-    agree = sh.isum[lane][1];
-    n_nll = sh.isum[lane][2];
-    n_flag = sh.isum[lane][3];
-    f_or = sh.flags_or[lane];
+    const bool has = lane < (nt >> 5);
+    s_kl = has ? sh.dsum[lane][0] : 0.0;
+    s_nll = has ? sh.dsum[lane][1] : 0.0;
+    n_valid = has ? sh.isum[lane][0] : 0;
+    agree = has ? sh.isum[lane][1] : 0;
+    n_nll = has ? sh.isum[lane][2] : 0;
+    n_flag = has ? sh.isum[lane][3] : 0;
+    f_or = has ? sh.flags_or[lane] : 0u;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
       s_kl += __shfl_down_sync(0xffffffffu, s_kl, o);
@@ -174,10 +181,10 @@ __global__ void __launch_bounds__(kReduceThreads, 1)
       if (total <= static_cast<unsigned long long>(kGatherCap)) break;
 
       const int ng = sh.ngroups;
-      for (int i = tid; i < ng * 256; i += kReduceThreads) (&sh.hist[0][0])[i] = 0u;
+      for (int i = tid; i < ng * 256; i += nt) (&sh.hist[0][0])[i] = 0u;
       __syncthreads();
       const uint64_t himask = decided == 0 ? 0ull : (~0ull << (64 - decided));
-      for (int64_t base_i = 0; base_i < N; base_i += kReduceThreads) {
+      for (int64_t base_i = 0; base_i < N; base_i += nt) {
         const int64_t i = base_i + tid;
         int slot = -1;
         if (i < N) {
@@ -241,7 +248,7 @@ __global__ void __launch_bounds__(kReduceThreads, 1)
       __syncthreads();
       const uint64_t himask = decided == 0 ? 0ull : (~0ull << (64 - decided));
       const int ng = sh.ngroups;
-      for (int64_t i = tid; i < N; i += kReduceThreads) {
+      for (int64_t i = tid; i < N; i += nt) {
         const kld_row_t rec = rows[i];
         if (rec.flags & kExcluded) continue;
         const uint64_t key = order_key(rec.kld);
@@ -258,11 +265,11 @@ __global__ void __launch_bounds__(kReduceThreads, 1)
       if (n > kGatherCap) n = kGatherCap;  // unreachable: counts bound it
       int p2 = 1;
       while (p2 < n) p2 <<= 1;
-      for (int i = n + tid; i < p2; i += kReduceThreads) sh.cand[i] = ~0ull;
+      for (int i = n + tid; i < p2; i += nt) sh.cand[i] = ~0ull;
       __syncthreads();
       for (int k = 2; k <= p2; k <<= 1) {
         for (int j = k >> 1; j > 0; j >>= 1) {
-          for (int i = tid; i < p2; i += kReduceThreads) {
+          for (int i = tid; i < p2; i += nt) {
             const int ixj = i ^ j;
             if (ixj > i) {
               const unsigned long long a = sh.cand[i], b = sh.cand[ixj];
@@ -332,8 +339,21 @@ __global__ void __launch_bounds__(kReduceThreads, 1)
 
 cudaError_t launch_reduce(const kld_row_t* rows, int64_t N, int has_nll, uint32_t* derr,
                           kld_result_t* out, cudaStream_t stream) {
-  kld_reduce_kernel<<<1, kReduceThreads, 0, stream>>>(rows, N, has_nll, derr, out);
-  return cudaGetLastError();
+  int threads = kReduceThreads;
+  if (N < kReduceThreads) {
+    threads = static_cast<int>((N + 31) / 32 * 32);
+    if (threads < 128) threads = 128;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(1);
+  cfg.blockDim = dim3(static_cast<unsigned>(threads));
+  cfg.stream = stream;
+  cudaLaunchAttribute attr;
+  attr.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr.val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = &attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kld_reduce_kernel, rows, N, has_nll, derr, out);
 }
 
 }  // namespace kld

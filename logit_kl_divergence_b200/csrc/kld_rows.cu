@@ -832,6 +832,9 @@ __global__ void __launch_bounds__(kRowThreads, 1)
   // touches a peer's shared memory, so no CTA stalls here at start-up.
   bool cl_waited = false;
   if (G > 1) asm volatile("barrier.cluster.arrive.release;" ::: "memory");
+  // The reduction launched after this pass may be scheduled now; it waits
+  // for this grid's completion before reading anything.
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
   const char* B = static_cast<const char*>(base);
   const char* Q = static_cast<const char*>(quant);
