@@ -19,28 +19,35 @@
 // so B is split as B = A + C with C = sum e_j phi(x_j), phi(y) = e^y - 1 - y
 // evaluated by a fitted polynomial (see phi_poly_fit.py): every term keeps
 // ~1e-7 relative accuracy and rounding errors of the exponentials enter only
-// at second order. Chunks where some |x| > 1.25 (or x is not finite: masked
-// or infinite entries) take a direct path that sums h_j = 2^(q_j*L - R_q)
-// with its own exponential instead. K follows (b - q) at the running maximum
-// of b (per warp), so x is ~0 where the base mass sits and the split keeps
-// its accuracy for peaked rows; moving K by d is an exact rebase in fp64:
+// at second order; each chunk uses the cheapest of three polynomial tiers
+// whose range holds all its |x|. Chunks where some |x| > 2.5 (or x is not
+// finite: masked or infinite entries) take a direct path that sums
+// h_j = 2^(q_j*L - R_q) with its own exponential instead. K follows (b - q)
+// at the element that last moved the frame (per warp: the frame moves when a
+// chunk's maximum of b passes the previous one by more than one nat), so x
+// is ~0 where the base mass sits and the split keeps its accuracy for peaked
+// rows; moving K by d is an exact rebase in fp64:
 // A += d*S, C -> e^{ld} C + (e^{ld} - 1) l A + (e^{ld} - 1 - l d) S. L = log2(e)
 // rounded to fp32; all exponentials are of lambda*y with lambda = L*ln2
 // = 1 + 1.4e-8, i.e. the statistic of softmax(lambda*b) and softmax(lambda*q),
 // within 3e-8 relative of the exact one.
 //
-// Structure (one CTA per SM, persistent over rows r = blockIdx.x + k*grid):
+// Structure (whole rows: one CTA per SM, persistent over rows
+// r = blockIdx.x + k*grid; split rows, for few rows: CTA k of a row's P
+// parts takes a contiguous run of its 512-element chunks, and the parts
+// merge in shared memory of a cluster and / or through global memory):
 //   - warp 16 (producer): one lane streams the 16-byte-aligned body of each
 //     row pair in 32 KB tiles per operand into a 3-stage shared-memory ring
 //     with cp.async.bulk (no multicast) completing on mbarriers, running
 //     ahead across row boundaries.
 //   - warps 0..15 (consumers): 512-element chunks (16 elements per lane,
-//     conflict-free 16-byte shared loads): lane and warp maxima (redux.sync),
-//     a warp-uniform frame raise when the maximum grew, then the fp32 terms
-//     of the chunk folded into per-lane fp64 accumulators. Each lane also
-//     remembers the first chunk in which its own maxima appeared. At the end
-//     of a row each warp reduces its accumulators and publishes them in a
-//     4-slot shared ring, then goes on with the next row.
+//     conflict-free 16-byte shared loads): lane maxima, a vote on whether
+//     the frame must move (then the warp maximum and a warp-uniform rebase),
+//     then the fp32 terms of the chunk folded into per-lane fp64
+//     accumulators. Each lane also remembers the first chunk in which its
+//     own maxima appeared. At the end of a row each warp reduces its
+//     accumulators and exact maxima and publishes them in a 4-slot shared
+//     ring, then goes on with the next row.
 //   - warp 17 (epilogue): per row, the unaligned head/tail (< 16 bytes each)
 //     and the token gather, the exact lowest-index argmax (re-reading only
 //     the chunks of lanes whose maximum equals the row maximum), the fp64
@@ -67,9 +74,18 @@ constexpr float kBig = 1.0e30f;
 constexpr float kTau = 2.5f;                 // |x| bound of the polynomial path
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
 
-// phi(y) = y^2 * P(y), P of degree 8 fitted on [-2.5, 2.5]
-// (phi_poly_fit.py, max relative error of phi in fp32 9e-7); the kernel
-// evaluates phi(lambda*x) = x^2 * Q(x), Q_k = P_k * lambda^(k+2).
+// phi(y) = y^2 * P(y), P fitted by phi_poly_fit.py in three tiers, the
+// cheapest whose range holds every |x| of a chunk being used (max relative
+// error of phi in fp32 evaluation):
+//   tier A: degree 5 on [-1, 1]     (1.7e-6)
+//   tier B: degree 6 on [-1.5, 1.5] (1.6e-6)
+//   tier C: degree 8 on [-2.5, 2.5] (9.0e-7)
+// The kernel evaluates phi(lambda*x) = x^2 * Q(x), Q_k = P_k * lambda^(k+2).
+constexpr float kTauA = 1.0f, kTauB = 1.5f;
+constexpr double kPA[6] = {0.5000007367, 0.1666656843, 0.0416529078,
+                           0.008336109943, 0.001426139768, 0.0001990834212};
+constexpr double kPB[7] = {0.5000002972, 0.1666698525, 0.0416645243, 0.008321388792,
+                           0.001390665576, 0.0002093027501, 2.499857965e-05};
 constexpr double kP0 = 0.4999997655, kP1 = 0.1666656346, kP2 = 0.0416678794,
                  kP3 = 0.008335872564, kP4 = 0.00138800956, kP5 = 0.0001968192101,
                  kP6 = 2.495779646e-05, kP7 = 3.111933302e-06, kP8 = 2.814820757e-07;
@@ -132,6 +148,30 @@ __device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, volat
 }
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort) {
   return mbar_try_wait(bar, parity) || mbar_wait_slow(bar, parity, abort);
+}
+// For the producer and epilogue warps, which spend most of their time
+// waiting: each probe suspends the thread for up to kIdleSuspendNs (it wakes
+// as soon as the phase completes), so the waiting warp does not take issue
+// slots from the consumer warps on its scheduler.
+constexpr uint32_t kIdleSuspendNs = 2000;
+__device__ __forceinline__ bool mbar_try_wait_idle(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity), "r"(kIdleSuspendNs)
+      : "memory");
+  return ok != 0;
+}
+__device__ __noinline__ bool mbar_wait_idle(uint32_t bar, uint32_t parity, volatile int* abort) {
+  const uint64_t t0 = globaltimer();
+  for (;;) {
+    if (mbar_try_wait_idle(bar, parity)) return true;
+    if (*abort) return false;
+    if (globaltimer() - t0 > kWaitLimitNs) return false;
+  }
 }
 __device__ __forceinline__ uint64_t evict_first_policy() {
   uint64_t pol;
@@ -208,19 +248,27 @@ __device__ __forceinline__ float phi_q(float x) {
   return fmaf(q, x, kQ0);
 }
 // The coefficients Q_k as (c, c) pairs in constant memory (packed FMAs take
-// no immediates).
-__constant__ __align__(8) float kQpair[18] = {kQ0, kQ0, kQ1, kQ1, kQ2, kQ2, kQ3, kQ3, kQ4,
-                                              kQ4, kQ5, kQ5, kQ6, kQ6, kQ7, kQ7, kQ8, kQ8};
+// no immediates): 6 for tier A, 7 for tier B, 9 for tier C.
+constexpr float qa(int k) { return static_cast<float>(kPA[k] * lam_pow(k + 2)); }
+constexpr float qb(int k) { return static_cast<float>(kPB[k] * lam_pow(k + 2)); }
+__constant__ __align__(8) float kQpair[44] = {
+    qa(0), qa(0), qa(1), qa(1), qa(2), qa(2), qa(3), qa(3), qa(4), qa(4), qa(5), qa(5),
+    qb(0), qb(0), qb(1), qb(1), qb(2), qb(2), qb(3), qb(3), qb(4), qb(4), qb(5), qb(5),
+    qb(6), qb(6),
+    kQ0, kQ0, kQ1, kQ1, kQ2, kQ2, kQ3, kQ3, kQ4, kQ4, kQ5, kQ5, kQ6, kQ6, kQ7, kQ7, kQ8, kQ8};
 __device__ __forceinline__ f2 qc(int k) {
   f2 r;
   r.v = reinterpret_cast<const unsigned long long*>(kQpair)[k];
   return r;
 }
-// Horner for Q on a packed pair.
+// Horner for tier T (0: A, 1: B, 2: C) on a packed pair.
+template <int T>
 __device__ __forceinline__ f2 phi_q2(f2 x) {
-  f2 q = fma2(qc(8), x, qc(7));
+  constexpr int o = T == 0 ? 0 : (T == 1 ? 6 : 13);
+  constexpr int nc = T == 0 ? 6 : (T == 1 ? 7 : 9);
+  f2 q = fma2(qc(o + nc - 1), x, qc(o + nc - 2));
 #pragma unroll
-  for (int k = 6; k >= 0; --k) q = fma2(q, x, qc(k));
+  for (int k = nc - 3; k >= 0; --k) q = fma2(q, x, qc(o + k));
   return q;
 }
 
@@ -297,11 +345,17 @@ struct Elem<KLD_F16> {
 // ------------------------------------------------------------- per-row state
 
 // Warp-uniform frames of one row operand pair.
+// The base frame and centre move only when a chunk's maximum exceeds the
+// one they were set at by more than kRaiseMargin (about half as many moves
+// per row); the exact maximum of b is tracked per lane in Best and reduced
+// when the warp publishes its partial.
+constexpr float kRaiseMargin = 1.0f;
 struct Ref {
-  float Mb;   // running maximum of b seen by this warp (-inf before any)
+  float Mb;   // maximum of b when the frame was last set (-inf before any)
   float Mqf;  // maximum of q over this warp's direct-path chunks (-inf before)
   float Rb, Rq;  // integer frames floor(M*L) once M is finite, 0 before
-  float K;       // log-ratio centre: (b - q) at the running maximum of b
+  float K;       // log-ratio centre: (b - q) at the element that set Mb
+  float T;       // Mb + kRaiseMargin: a chunk maximum above it moves the frame
 };
 
 // Per-lane fp64 accumulators (see the file comment): S_b over all chunks;
@@ -363,9 +417,9 @@ __device__ __forceinline__ double pow2i(float k) {
   return ldexp(1.0, static_cast<int>(fmaxf(k, -2000.f)));
 }
 
-// Polynomial path of one step: every x finite with |x| <= kTau.
-// S += e, Ap += e*x, C += e*x^2*Q(x), e = 2^(b*L - R_b).
-template <int PE>
+// Polynomial path of one step: every x finite with |x| within tier T's range.
+// S += e, Ap += e*x, C += e*x^2*Q_T(x), e = 2^(b*L - R_b).
+template <int PE, int T>
 __device__ __forceinline__ void poly_accumulate(const float* b, const f2* X, const Ref& r,
                                                 Acc& a) {
   constexpr int NP = (PE + 1) / 2;
@@ -382,7 +436,7 @@ __device__ __forceinline__ void poly_accumulate(const float* b, const f2* X, con
     const f2 T2 = mul2(E, X[j]);
     SB[j & 1] = add2(SB[j & 1], E);
     SA[j & 1] = add2(SA[j & 1], T2);
-    SC[j & 1] = fma2(mul2(T2, X[j]), phi_q2(X[j]), SC[j & 1]);
+    SC[j & 1] = fma2(mul2(T2, X[j]), phi_q2<T>(X[j]), SC[j & 1]);
   }
   float sb0, sb1, sa0, sa1, sc0, sc1;
   upk(add2(SB[0], SB[1]), sb0, sb1);
@@ -409,8 +463,11 @@ __device__ __forceinline__ void chunk_step(const float* b, const float* q, unsig
     mb = fmaxf(mb, b[PE - 1]);
     mq = fmaxf(mq, q[PE - 1]);
   }
-  const float wmb = warp_max(mb);
-  if (wmb > r.Mb) {  // raise the base frame and move the centre (warp-uniform)
+  // The warp maximum is needed only when some lane's maximum passes the
+  // threshold (a few chunks per row): a vote first, then the shuffle tree.
+  if (__any_sync(0xffffffffu, mb > r.T)) {
+    // raise the base frame and move the centre (warp-uniform)
+    const float wmb = warp_max(mb);
     // New centre: (b - q) at the lowest lane's first element holding wmb.
     float dl = 0.f;
     bool has = false;
@@ -461,6 +518,7 @@ __device__ __forceinline__ void chunk_step(const float* b, const float* q, unsig
     }
     r.Rb = nR;
     r.Mb = wmb;
+    r.T = wmb + kRaiseMargin;
   }
 
   // Log-ratios x = (q - b) + K, in packed pairs.
@@ -482,11 +540,15 @@ __device__ __forceinline__ void chunk_step(const float* b, const float* q, unsig
     else
       ax0 = max3_nan(ax0, fabsf(x0), fabsf(x1));
   }
-  // Warp max of |x| (NaN if any x is NaN: every comparison below fails).
-  float wax;
-  asm volatile("redux.sync.max.NaN.f32 %0, %1, 0xffffffff;" : "=f"(wax) : "f"(max3_nan(ax0, ax1, 0.f)));
-  if (wax <= kTau) {
-    poly_accumulate<PE>(b, X, r, a);
+  // The cheapest polynomial tier whose range holds every |x| of the warp's
+  // step (a NaN fails every test and takes the direct path).
+  const float axl = max3_nan(ax0, ax1, 0.f);
+  if (__all_sync(0xffffffffu, axl <= kTauA)) {
+    poly_accumulate<PE, 0>(b, X, r, a);
+  } else if (__all_sync(0xffffffffu, axl <= kTauB)) {
+    poly_accumulate<PE, 1>(b, X, r, a);
+  } else if (__all_sync(0xffffffffu, axl <= kTau)) {
+    poly_accumulate<PE, 2>(b, X, r, a);
   } else {
     // Direct path: quant weights in their own frame. x -> +BIG keeps 0*x = 0
     // for masked base entries; x = -inf (quant masked, base finite) makes A
@@ -855,7 +917,8 @@ __global__ void __launch_bounds__(kRowThreads, 1)
         const int64_t n = it.s1 - it.s0;
         const int64_t ntiles = (n + kStageElems - 1) / kStageElems;
         for (int64_t t = 0; t < ntiles; ++t) {
-          if (!mbar_wait(smem_u32(&ctrl->empty[s]), ph ^ 1u, abort)) {
+          if (!mbar_try_wait(smem_u32(&ctrl->empty[s]), ph ^ 1u) &&
+              !mbar_wait_idle(smem_u32(&ctrl->empty[s]), ph ^ 1u, abort)) {
             fail(ctrl, derr);
             ok = false;
             break;
@@ -906,7 +969,7 @@ __global__ void __launch_bounds__(kRowThreads, 1)
     // whole-row and split-row loops below each inline their own copy, so
     // the split bookkeeping costs the whole-row loop no registers.
     auto consume = [&](int n, int j) -> bool {
-      Ref ref{-INFINITY, -INFINITY, 0.f, 0.f, 0.f};
+      Ref ref{-INFINITY, -INFINITY, 0.f, 0.f, 0.f, -INFINITY};
       Acc acc{0.0, 0.0, 0.0, 0.0, 0.0, 0.0};
       Best best{-INFINITY, -INFINITY, -1, -1};
       const int ntiles = (n + kStageElems - 1) / kStageElems;
@@ -950,8 +1013,9 @@ __global__ void __launch_bounds__(kRowThreads, 1)
       const uint32_t sph = (j / kSlots) & 1u;
       const double Sb = warp_sum(acc.Sb), Ap = warp_sum(acc.Ap), C = warp_sum(acc.C);
       const double Ad = warp_sum(acc.Ad), Se = warp_sum(acc.Se), Sh = warp_sum(acc.Sh);
-      const float wq = warp_max(best.q);  // the warp's maximum of q
-      const unsigned cb_mask = __ballot_sync(0xffffffffu, ref.Mb > -INFINITY && best.b == ref.Mb);
+      const float wb = warp_max(best.b);  // the warp's exact maxima of b and q
+      const float wq = warp_max(best.q);
+      const unsigned cb_mask = __ballot_sync(0xffffffffu, wb > -INFINITY && best.b == wb);
       const unsigned cq_mask = __ballot_sync(0xffffffffu, wq > -INFINITY && best.q == wq);
       if (!mbar_wait(smem_u32(&ctrl->slot_empty[slot]), sph ^ 1u, abort)) {
         fail(ctrl, derr);
@@ -962,7 +1026,7 @@ __global__ void __launch_bounds__(kRowThreads, 1)
       if ((cq_mask >> lane) & 1u) sl.loc_q[warp][lane] = best.lq;
       if (lane == 0) {
         WarpPart p;
-        p.Mb = ref.Mb;
+        p.Mb = wb;
         p.Mq = wq;
         p.Rb = ref.Rb;
         p.Rq = ref.Rq;
@@ -1014,17 +1078,18 @@ __global__ void __launch_bounds__(kRowThreads, 1)
         xe_b = Elem<DT>::load(rb, jj);
         xe_q = Elem<DT>::load(rq, jj);
       }
-      Ref eref{-INFINITY, -INFINITY, 0.f, 0.f, 0.f};
+      Ref eref{-INFINITY, -INFINITY, 0.f, 0.f, 0.f, -INFINITY};
       Acc eacc{0.0, 0.0, 0.0, 0.0, 0.0, 0.0};
       Best ebest{-INFINITY, -INFINITY, -1, -1};
       if (n_extra > 0) chunk_step<1>(&xe_b, &xe_q, lane < n_extra ? 1u : 0u, eref, eacc, ebest, 0);
-      const float eMq = warp_max(xe_q);
+      const float eMb = warp_max(xe_b), eMq = warp_max(xe_q);
       const double eSb = warp_sum(eacc.Sb), eAp = warp_sum(eacc.Ap), eC = warp_sum(eacc.C);
       const double eAd = warp_sum(eacc.Ad), eSe = warp_sum(eacc.Se), eSh = warp_sum(eacc.Sh);
 
       const int slot = j % kSlots;
       const uint32_t sph = (j / kSlots) & 1u;
-      const bool got = mbar_wait(smem_u32(&ctrl->slot_full[slot]), sph, abort);
+      const bool got = mbar_try_wait(smem_u32(&ctrl->slot_full[slot]), sph) ||
+                       mbar_wait_idle(smem_u32(&ctrl->slot_full[slot]), sph, abort);
       MPart m = empty_part();
       if (!got) {
         // Whole rows: nothing is written for this or later rows. Split rows:
@@ -1046,7 +1111,7 @@ __global__ void __launch_bounds__(kRowThreads, 1)
           cand_b = p.cand_b;
           cand_q = p.cand_q;
         } else {
-          p.Mb = eref.Mb;
+          p.Mb = eMb;
           p.Mq = eMq;
           p.Rb = eref.Rb;
           p.Rq = eref.Rq;

@@ -1,12 +1,14 @@
-"""Derivation of the polynomial the row kernel uses for phi(y) = e^y - 1 - y.
+"""Derivation of the polynomials the row kernel uses for phi(y) = e^y - 1 - y.
 
 The kernel needs phi(y) to about 1e-6 relative accuracy for |y| <= 2.5 (it
 is the second-order part of the quant/base normaliser ratio, the same order
-as the KL itself). It evaluates phi(y) = y^2 * P(y) with P of degree 8 in
-fp32 Horner form. P is fitted here by weighted least squares (relative error)
-at 400 Chebyshev nodes of [-2.5, 2.5] against phi(y)/y^2 evaluated in
-40-digit arithmetic; the script prints the coefficients and the worst
-relative error of the fp32 evaluation on a dense grid (about 9e-7).
+as the KL itself). It evaluates phi(y) = y^2 * P(y) in fp32 Horner form,
+with the cheapest of three tiers whose range holds a whole chunk: degree 5
+on [-1, 1], degree 6 on [-1.5, 1.5], degree 8 on [-2.5, 2.5]. Each P is
+fitted here by weighted least squares (relative error) at 400 Chebyshev
+nodes of its range against phi(y)/y^2 evaluated in 40-digit arithmetic; the
+script prints the coefficients and the worst relative error of the fp32
+evaluation on a dense grid (1.7e-6, 1.6e-6, 9.0e-7).
 
     python logit_kl_divergence_b200/csrc/phi_poly_fit.py
 
@@ -49,7 +51,10 @@ def fp32_rel_error(c, tau=TAU):
     return float(np.max(np.abs(phi32[keep] - ref[keep]) / np.abs(ref[keep])))
 
 
+TIERS = ((1.0, 5), (1.5, 6), (TAU, DEG))
+
 if __name__ == "__main__":
-    c = fit()
-    print("coefficients (y^0 .. y^5):", ", ".join(f"{v:.9g}" for v in c))
-    print("max relative error of phi in fp32:", fp32_rel_error(c))
+    for tau, deg in TIERS:
+        c = fit(tau, deg)
+        print(f"[-{tau}, {tau}] degree {deg}:", ", ".join(f"{v:.10g}" for v in c))
+        print("  max relative error of phi in fp32:", fp32_rel_error(c, tau))
