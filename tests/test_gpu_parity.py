@@ -85,6 +85,35 @@ def test_constant_shift_rows_are_near_zero():
     assert_rows_match(g_rows, o_rows)
 
 
+@pytest.mark.parametrize("split", [None, -1])
+@pytest.mark.parametrize("dtype", [synth.F32, synth.BF16])
+def test_dominant_element_at_every_gap_above_the_rest(dtype, split):
+    # One element far enough above the rest to hold most of the mass, placed
+    # late in its row (after the running maximum has settled), at gaps from
+    # a fraction of a nat to well past the frame's move threshold; small
+    # quant noise so that the KL is tiny and any centring error would show.
+    gaps = [0.25, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 5.0, 6.0, 8.0, 10.0, 12.0, 16.0, 24.0]
+    v = 32768
+    g = torch.Generator().manual_seed(21)
+    rows_b, rows_q = [], []
+    for gap in gaps:
+        for sigma in (0.003, 0.03):
+            b = torch.randn(v, generator=g)
+            b[-700] = b.max() + gap
+            rows_b.append(b)
+            rows_q.append(b + sigma * torch.randn(v, generator=g))
+    b = torch.stack(rows_b)
+    q = torch.stack(rows_q)
+    if dtype == synth.BF16:
+        b, q = b.to(torch.bfloat16), q.to(torch.bfloat16)
+    tok = torch.randint(0, v, (b.shape[0],), generator=g, dtype=torch.int32)
+    g_rows, gres = gpu_run(b.contiguous().to(DEV), q.contiguous().to(DEV), tok.to(DEV),
+                           split=split)
+    o_rows, ores = oracle.run(b.contiguous(), q.contiguous(), tok, ODT[dtype])
+    assert_rows_match(g_rows, o_rows)
+    assert_stats_match(gres, ores)
+
+
 def test_planted_ties_lowest_index_wins():
     n, v = 64, 9000
     g = torch.Generator().manual_seed(4)
