@@ -1016,7 +1016,14 @@ __global__ void __launch_bounds__(kRowThreads, 1)
       const int slot = j % kSlots;
       const uint32_t sph = (j / kSlots) & 1u;
       const double Sb = warp_sum(acc.Sb), Ap = warp_sum(acc.Ap), C = warp_sum(acc.C);
-      const double Ad = warp_sum(acc.Ad), Se = warp_sum(acc.Se), Sh = warp_sum(acc.Sh);
+      // Direct-path sums are zero unless some chunk of the row took that path
+      // (a NaN compares unequal to zero and keeps them).
+      double Ad = 0.0, Se = 0.0, Sh = 0.0;
+      if (__any_sync(0xffffffffu, acc.Ad != 0.0 || acc.Se != 0.0 || acc.Sh != 0.0)) {
+        Ad = warp_sum(acc.Ad);
+        Se = warp_sum(acc.Se);
+        Sh = warp_sum(acc.Sh);
+      }
       const float wb = warp_max(best.b);  // the warp's exact maxima of b and q
       const float wq = warp_max(best.q);
       const unsigned cb_mask = __ballot_sync(0xffffffffu, wb > -INFINITY && best.b == wb);
