@@ -212,7 +212,7 @@ SPLIT_CALLS = 1000
 SPLIT_COLD_BYTES = 256 << 20  # inputs rotated per call cycle: twice the 126 MB L2
 
 
-def split_row_latency(dev, stream):
+def split_row_latency(dev, stream, min_calls: int = SPLIT_CALLS):
     """Few-row, large-vocabulary launches (N in SPLIT_ROWS, V = 262144 fp32):
     SPLIT_CALLS back-to-back calls of the whole statistic on one stream,
     plainly and as CUDA-graph replays, with the whole-row launch shape
@@ -222,7 +222,7 @@ def split_row_latency(dev, stream):
 
     from logit_kl_divergence_b200 import KLDStats, run_static, synth
 
-    out = {"workload": "splitrow{1,4,16,32}_v262144_f32", "min_calls": SPLIT_CALLS,
+    out = {"workload": "splitrow{1,4,16,32}_v262144_f32", "min_calls": min_calls,
            "l2": f"inputs rotated over copies totalling >= {SPLIT_COLD_BYTES >> 20} MB per cycle",
            "per_rows": {}}
     ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
@@ -236,7 +236,7 @@ def split_row_latency(dev, stream):
         tok = w.token_ids
         st = KLDStats(max_rows=n, device=dev)
         res_buf = torch.zeros(256, dtype=torch.uint8, device=dev)
-        calls = -(-SPLIT_CALLS // k) * k
+        calls = -(-min_calls // k) * k
 
         def timed(fn, reps):
             for i in range(min(k, 8)):
@@ -307,6 +307,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-variants", action="store_true")
     ap.add_argument("--no-split-row", action="store_true")
+    ap.add_argument("--split-calls", type=int, default=SPLIT_CALLS,
+                    help="profiling only: fewer calls per size in the split-row section")
     ap.add_argument("--rows", type=int, default=None,
                     help="profiling only: fewer rows of the same recipe (not a bench line)")
     ap.add_argument("--dtype", choices=["f32", "bf16"], default="f32",
@@ -440,7 +442,9 @@ def main():
         rrow = sum(rms) / len(rms)
         variants[VARIANT] = {"value": wb.n / (vms / 1000.0), "unit": "rows/s", "ms_per_step": vms,
                              "row_pass_ms": rrow, "achieved_gbs": vb_bytes / (rrow / 1000.0) / 1e9,
-                             "frac": vb_bytes / (rrow / 1000.0) / 1e9 / peak}
+                             "frac": vb_bytes / (rrow / 1000.0) / 1e9 / peak,
+                             "traffic": recorded_traffic(VARIANT),
+                             "algorithmic_bytes_per_launch": vb_bytes}
         del wb
         torch.cuda.empty_cache()
         w = synth.make(name, device=dev, seed=synth.WORKLOADS[name][4])
@@ -472,7 +476,7 @@ def main():
     if world == 1 and not args.no_split_row and args.rows is None:
         del w
         torch.cuda.empty_cache()
-        split_row = split_row_latency(dev, stream)
+        split_row = split_row_latency(dev, stream, max(1, args.split_calls))
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -493,8 +497,9 @@ def main():
             "mean_kld": res["mean_kld"], "top1_agree_pct": res["top1_agree_pct"], "ppl": res["ppl"],
             "variants": variants, "split_row": split_row,
         }
-        if args.rows is not None or args.dtype != "f32":
+        if args.rows is not None or args.dtype != "f32" or args.split_calls != SPLIT_CALLS:
             line["config"]["override"] = {"rows": N, "dtype": args.dtype,
+                                          "split_calls": args.split_calls,
                                           "note": "profiling run, not the benchmark workload"}
         print(json.dumps(line), flush=True)
 
