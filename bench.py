@@ -328,6 +328,7 @@ def main():
     import torch.distributed as dist
 
     from logit_kl_divergence_b200 import KLDStats, synth
+    from logit_kl_divergence_b200.sharded import gather_records
 
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
@@ -348,10 +349,8 @@ def main():
     st = KLDStats(max_rows=N * world, device=dev)
     st.set_timing(world == 1)
     records = None
-    gathered = None
     if world > 1:
         records = torch.empty((N, ROW_RECORD_BYTES), dtype=torch.uint8, device=dev)
-        gathered = torch.empty((N * world, ROW_RECORD_BYTES), dtype=torch.uint8, device=dev)
 
     row_ms = []
 
@@ -363,7 +362,7 @@ def main():
                 row_ms.append(st.timing()[0])
         else:
             st.run_rows(w.base, w.quant, w.token_ids, out=records)
-            dist.all_gather_into_tensor(gathered, records)
+            gathered = gather_records(records, counts=[N] * world)
             st.reduce(gathered, N * world, True)
             res = st.result()
         return res
@@ -389,7 +388,7 @@ def main():
             e0.record(stream)
             st.run_rows(w.base, w.quant, w.token_ids, out=records)
             e1.record(stream)
-            dist.all_gather_into_tensor(gathered, records)
+            gathered = gather_records(records, counts=[N] * world)
             st.reduce(gathered, N * world, True)
             res = st.result()
             row_ms.append(e0.elapsed_time(e1))

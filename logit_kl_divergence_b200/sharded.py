@@ -1,0 +1,99 @@
+"""Row-sharded statistics over several processes, one GPU each.
+
+Rows are independent, so N rows split across ranks with no exchange in the
+row pass. The one real exchange is for the order statistics: every rank
+all-gathers the 32-byte per-row records in rank order (NCCL over NVLink on
+GPUs; any torch.distributed backend carries the gather) and reduces the full
+set, so the percentiles stay exact and every rank holds the same result.
+
+    >>> sk = ShardedKLDStats(max_rows_per_rank=8192, device=dev)   # after init_process_group
+    >>> res = sk.run(base_shard, quant_shard, token_shard)          # same dict on every rank
+"""
+from __future__ import annotations
+
+import torch
+import torch.distributed as dist
+
+ROW_RECORD_BYTES = 32
+
+
+def shard_bounds(n_rows: int, world: int, rank: int) -> tuple[int, int]:
+    """Contiguous [start, stop) rows of `rank` when n_rows are split over
+    `world` ranks; the first n_rows % world ranks take one row more."""
+    if world < 1 or not 0 <= rank < world or n_rows < 0:
+        raise ValueError("need world >= 1, 0 <= rank < world, n_rows >= 0")
+    base, extra = divmod(n_rows, world)
+    start = rank * base + min(rank, extra)
+    return start, start + base + (1 if rank < extra else 0)
+
+
+def gather_records(records: torch.Tensor, group=None, counts: list[int] | None = None) -> torch.Tensor:
+    """All-gather every rank's [n_r, 32] uint8 records, concatenated in rank
+    order (ranks may hold different row counts). Collective: every rank of
+    `group` calls it with its own records, in the same order of calls.
+    `counts`: every rank's row count when the caller knows them (skips one
+    small all-gather)."""
+    if records.dtype != torch.uint8 or records.dim() != 2 or records.shape[1] != ROW_RECORD_BYTES:
+        raise ValueError("records must be a [n, 32] uint8 tensor")
+    world = dist.get_world_size(group)
+    if counts is None:
+        n = torch.tensor([records.shape[0]], dtype=torch.int64, device=records.device)
+        sizes = [torch.zeros_like(n) for _ in range(world)]
+        dist.all_gather(sizes, n, group=group)
+        counts = [int(c.item()) for c in sizes]
+    elif len(counts) != world or counts[dist.get_rank(group)] != records.shape[0]:
+        raise ValueError("counts must list every rank's row count")
+    m = max(counts)
+    padded = records
+    if records.shape[0] != m:
+        padded = records.new_zeros((m, ROW_RECORD_BYTES))
+        padded[:records.shape[0]] = records
+    padded = padded.contiguous()
+    if dist.get_backend(group) == "nccl":
+        out = records.new_empty((m * world, ROW_RECORD_BYTES))
+        dist.all_gather_into_tensor(out, padded, group=group)
+        parts = list(out.view(world, m, ROW_RECORD_BYTES))
+    else:
+        parts = [torch.empty_like(padded) for _ in range(world)]
+        dist.all_gather(parts, padded, group=group)
+    if all(c == m for c in counts):
+        return torch.cat(parts) if len(parts) > 1 else parts[0]
+    return torch.cat([p[:c] for p, c in zip(parts, counts)])
+
+
+class ShardedKLDStats:
+    """The statistic over rows sharded across the ranks of `group`: each rank
+    runs the row pass on its own rows, the records are gathered, and each rank
+    runs the reduction on all of them. `stats` is the per-rank handle (a
+    :class:`KLDStats` on this rank's GPU by default)."""
+
+    def __init__(self, max_rows_per_rank: int, device=None, group=None, stats=None):
+        if stats is None:
+            from . import KLDStats
+
+            stats = KLDStats(max_rows=max_rows_per_rank, device=device)
+        self.stats = stats
+        self.group = group
+        self.max_rows_per_rank = int(max_rows_per_rank)
+        self._records = None
+
+    def run(self, base: torch.Tensor, quant: torch.Tensor, token_ids: torch.Tensor | None = None) -> dict:
+        """Collective. Every rank passes its own [n_r, V] rows (same V, dtype
+        and token-id presence on every rank); returns the statistics of all
+        ranks' rows."""
+        n = base.shape[0]
+        if n > self.max_rows_per_rank:
+            raise ValueError("more rows than max_rows_per_rank")
+        if self._records is None or self._records.device != base.device:
+            self._records = torch.empty((self.max_rows_per_rank, ROW_RECORD_BYTES), dtype=torch.uint8,
+                                        device=base.device)
+        records = self._records[:n]
+        self.stats.run_rows(base, quant, token_ids, out=records)
+        gathered = gather_records(records, self.group)
+        self.stats.reduce(gathered, gathered.shape[0], token_ids is not None)
+        return self.stats.result()
+
+    def close(self):
+        close = getattr(self.stats, "close", None)
+        if close is not None:
+            close()

@@ -1,0 +1,121 @@
+"""Row sharding across processes (the multi-GPU path's host logic), run as
+gloo ranks on the CPU: shard bounds, the rank-ordered all-gather of 32-byte
+records (equal and unequal row counts), and the orchestration of
+ShardedKLDStats with the per-rank row pass and reduction supplied by the
+oracle, so the statistics of the gathered shards must equal the oracle's
+statistics of all rows exactly."""
+import math
+import os
+import socket
+
+import numpy as np
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+import oracle
+from logit_kl_divergence_b200 import rows_view, synth
+from logit_kl_divergence_b200.sharded import ShardedKLDStats, gather_records, shard_bounds
+
+RECORD = np.dtype([("kld", "<f8"), ("nll", "<f8"), ("amax_b", "<i4"), ("amax_q", "<i4"),
+                   ("flags", "<u4"), ("reserved", "<u4")])
+assert RECORD.itemsize == 32
+
+
+def _pack(r: dict) -> np.ndarray:
+    a = np.zeros(r["kld"].shape[0], dtype=RECORD)
+    for k in ("kld", "nll", "amax_b", "amax_q", "flags"):
+        a[k] = r[k]
+    return a.view(np.uint8).reshape(-1, 32)
+
+
+class OracleStats:
+    """Per-rank stand-in for the GPU handle: the oracle's row pass writes
+    records in the library's layout, its reduction reads them back."""
+
+    def __init__(self, dtype):
+        self.dtype = dtype
+        self.res = None
+
+    def run_rows(self, base, quant, token_ids=None, out=None):
+        r = oracle.rows(base, quant, token_ids, self.dtype)
+        out.copy_(torch.from_numpy(_pack(r)))
+        return out
+
+    def reduce(self, records, n_rows, has_nll):
+        v = rows_view(records[:n_rows])
+        r = {k: t.numpy().copy() for k, t in v.items()}
+        r["flags"] = r["flags"].astype(np.uint32)
+        self.res = oracle.reduce(r, has_nll)
+
+    def result(self):
+        return self.res
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _same(a, b):
+    assert a.keys() == b.keys()
+    for k in a:
+        x, y = a[k], b[k]
+        if isinstance(x, float) and math.isnan(x):
+            assert isinstance(y, float) and math.isnan(y), k
+        else:
+            assert x == y, (k, x, y)
+
+
+def _worker(rank, world, port, n_rows, with_tokens, errq):
+    try:
+        dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank,
+                                world_size=world)
+        w = synth.make_recipe("edge", n=n_rows, v=3001, dtype=synth.F32, seed=7)
+        tok = w.token_ids if with_tokens else None
+        lo, hi = shard_bounds(n_rows, world, rank)
+        # rank-ordered gather of raw records
+        mine = torch.full((hi - lo, 32), rank, dtype=torch.uint8)
+        got = gather_records(mine)
+        expect = torch.cat([torch.full((b - a, 32), r, dtype=torch.uint8)
+                            for r, (a, b) in enumerate(shard_bounds(n_rows, world, q) for q in range(world))])
+        assert torch.equal(got, expect)
+        # the whole orchestration, oracle-backed
+        sk = ShardedKLDStats(max_rows_per_rank=hi - lo + 1, stats=OracleStats(oracle.F32))
+        res = sk.run(w.base[lo:hi].contiguous(), w.quant[lo:hi].contiguous(),
+                     None if tok is None else tok[lo:hi].contiguous())
+        _, full = oracle.run(w.base, w.quant, tok, oracle.F32)
+        _same(res, full)
+        assert res["n_rows"] == n_rows
+        dist.barrier()
+        dist.destroy_process_group()
+    except BaseException as e:  # reported to the parent
+        errq.put(f"rank {rank}: {type(e).__name__}: {e}")
+        raise
+
+
+def _spawn(world, n_rows, with_tokens):
+    ctx = mp.get_context("spawn")
+    errq = ctx.SimpleQueue()
+    mp.start_processes(_worker, args=(world, _free_port(), n_rows, with_tokens, errq), nprocs=world,
+                       join=True, start_method="spawn")
+    assert errq.empty(), errq.get()
+
+
+def test_shard_bounds_cover_all_rows_in_order():
+    for n in (0, 1, 7, 8, 37, 8192):
+        for world in (1, 2, 3, 8):
+            b = [shard_bounds(n, world, r) for r in range(world)]
+            assert b[0][0] == 0 and b[-1][1] == n
+            assert all(b[i][1] == b[i + 1][0] for i in range(world - 1))
+            sizes = [hi - lo for lo, hi in b]
+            assert max(sizes) - min(sizes) <= 1 and sizes == sorted(sizes, reverse=True)
+    with pytest.raises(ValueError):
+        shard_bounds(4, 2, 2)
+
+
+@pytest.mark.parametrize("world,n_rows,with_tokens", [(2, 64, True), (2, 37, False), (3, 37, True)])
+def test_sharded_statistics_equal_single_process_oracle(world, n_rows, with_tokens):
+    _spawn(world, n_rows, with_tokens)
