@@ -10,7 +10,8 @@ marshals numpy arrays through ctypes. Sources for each step are cited in the
 C++ file: "Qwen3.6 27B Quantization Benchmark" (sections "Understand KLD and
 Same Top P" and "Raw benchmark data") and the "Mistral-Small-4-119B-2603
 GSQ-RCO IQ3_S GGUF" card ("How it was made", step 5: KL(BF16 || quantized)
-over the full vocabulary).
+over the full vocabulary; "Quality": the perplexity ratio and the points of
+probability given to the correct token).
 
 Parity of every function here is pinned by ``tests/test_oracle_pins.py``
 against closed forms, invariants, brute force and library routines.
@@ -36,6 +37,7 @@ ROW_EMPTY = 1 << 1
 ROW_INF_KL = 1 << 2
 ROW_BAD_TOKEN = 1 << 3
 ROW_INF_NLL = 1 << 4
+ROW_INF_NLLB = 1 << 5
 
 
 class _Result(ctypes.Structure):
@@ -57,6 +59,11 @@ class _Result(ctypes.Structure):
         ("n_flagged", ctypes.c_int64),
         ("flags_or", ctypes.c_uint32),
         ("_pad2", ctypes.c_uint32),
+        ("mean_nll_base", ctypes.c_double),
+        ("ppl_base", ctypes.c_double),
+        ("ln_ppl_ratio", ctypes.c_double),
+        ("mean_dp", ctypes.c_double),
+        ("rms_dp", ctypes.c_double),
     ]
 
 
@@ -95,13 +102,13 @@ def _load():
                 ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
                 ctypes.c_int64, ctypes.c_int64, ctypes.c_int,
                 ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
-                ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int,
+                ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int,
             ]
             lib.oracle_reduce.restype = ctypes.c_int
             lib.oracle_reduce.argtypes = [
                 ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
-                ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64,
-                ctypes.c_int, ctypes.POINTER(_Result),
+                ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                ctypes.c_int64, ctypes.c_int, ctypes.POINTER(_Result),
             ]
             lib.oracle_percentile_sorted.restype = ctypes.c_double
             lib.oracle_percentile_sorted.argtypes = [
@@ -134,7 +141,8 @@ def _as_logits(x, dtype: int) -> np.ndarray:
 
 
 def rows(base, quant, token_ids=None, dtype: int = F32, nthreads: int = 1) -> dict:
-    """Per-row KL, NLL, argmaxes and flags (numpy arrays of length N)."""
+    """Per-row KL, NLL under quant and base, argmaxes and flags (numpy arrays
+    of length N)."""
     lib = _load()
     b = _as_logits(base, dtype)
     q = _as_logits(quant, dtype)
@@ -151,6 +159,7 @@ def rows(base, quant, token_ids=None, dtype: int = F32, nthreads: int = 1) -> di
     out = {
         "kld": np.empty(N, np.float64),
         "nll": np.empty(N, np.float64),
+        "nll_base": np.empty(N, np.float64),
         "amax_b": np.empty(N, np.int32),
         "amax_q": np.empty(N, np.int32),
         "flags": np.empty(N, np.uint32),
@@ -158,7 +167,7 @@ def rows(base, quant, token_ids=None, dtype: int = F32, nthreads: int = 1) -> di
     rc = lib.oracle_rows(
         b.ctypes.data, q.ctypes.data, None if tok is None else tok.ctypes.data,
         N, V, dtype,
-        out["kld"].ctypes.data, out["nll"].ctypes.data,
+        out["kld"].ctypes.data, out["nll"].ctypes.data, out["nll_base"].ctypes.data,
         out["amax_b"].ctypes.data, out["amax_q"].ctypes.data,
         out["flags"].ctypes.data, int(nthreads),
     )
@@ -173,11 +182,12 @@ def reduce(r: dict, has_nll: bool) -> dict:
     N = r["kld"].shape[0]
     kld = np.ascontiguousarray(r["kld"], np.float64)
     nll = np.ascontiguousarray(r["nll"], np.float64)
+    nllb = np.ascontiguousarray(r.get("nll_base", np.full(N, np.nan)), np.float64)
     ab = np.ascontiguousarray(r["amax_b"], np.int32)
     aq = np.ascontiguousarray(r["amax_q"], np.int32)
     fl = np.ascontiguousarray(r["flags"], np.uint32)
     res = _Result()
-    rc = lib.oracle_reduce(kld.ctypes.data, nll.ctypes.data, ab.ctypes.data,
+    rc = lib.oracle_reduce(kld.ctypes.data, nll.ctypes.data, nllb.ctypes.data, ab.ctypes.data,
                            aq.ctypes.data, fl.ctypes.data, N, int(bool(has_nll)),
                            ctypes.byref(res))
     if rc != 0:

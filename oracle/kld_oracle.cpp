@@ -25,7 +25,13 @@
  *     b_j finite with q_j = -inf makes the KL +inf (flag INF_KL, kept);
  *   - percentiles use linear interpolation between order statistics,
  *     pos = p*(n-1) (the "type 7" rule); max is the largest order statistic;
- *   - means run over the valid rows; PPL = exp(mean NLL).
+ *   - means run over the valid rows; PPL = exp(mean NLL);
+ *   - the base model's NLL of the same token (NLLB) gives PPL(base) and the
+ *     perplexity ratio ("Mistral-Small-4-119B-2603 GSQ-RCO IQ3_S GGUF",
+ *     "Quality"); dp = P_quant(tok) - P_base(tok), averaged and as a root
+ *     mean square over the rows with a token (the Qwen3.6 table's "RMS dp
+ *     (%)" column, the same card's points of probability); b[tok] = -inf
+ *     makes NLLB +inf (flag INF_NLLB) and P_base(tok) = 0.
  */
 #include "kld_oracle.h"
 
@@ -82,11 +88,12 @@ const double kInf = std::numeric_limits<double>::infinity();
 
 /* Statistics of one row pair, by the definitions, two passes per row. */
 void one_row(const double* b, const double* q, int64_t V, int has_tok,
-             int32_t tok, double* kld, double* nll, int32_t* ab, int32_t* aq,
-             uint32_t* flags) {
+             int32_t tok, double* kld, double* nll, double* nllb, int32_t* ab,
+             int32_t* aq, uint32_t* flags) {
   uint32_t f = 0;
   *kld = kNaN;
   *nll = kNaN;
+  *nllb = kNaN;
   *ab = -1;
   *aq = -1;
 
@@ -149,15 +156,24 @@ void one_row(const double* b, const double* q, int64_t V, int has_tok,
     f |= ORACLE_ROW_INF_KL;
   }
 
-  /* Step 6: NLL of the given next token under the quantized row. */
+  /* Step 6: NLL of the given next token under the quantized row, and under
+   * the base row. */
   if (has_tok) {
     if (tok < 0 || (int64_t)tok >= V) {
       f |= ORACLE_ROW_BAD_TOKEN;
-    } else if (q[tok] == -kInf) {
-      *nll = kInf;
-      f |= ORACLE_ROW_INF_NLL;
     } else {
-      *nll = lse_q - q[tok];
+      if (q[tok] == -kInf) {
+        *nll = kInf;
+        f |= ORACLE_ROW_INF_NLL;
+      } else {
+        *nll = lse_q - q[tok];
+      }
+      if (b[tok] == -kInf) {
+        *nllb = kInf;
+        f |= ORACLE_ROW_INF_NLLB;
+      } else {
+        *nllb = lse_b - b[tok];
+      }
     }
   }
 
@@ -169,13 +185,14 @@ void one_row(const double* b, const double* q, int64_t V, int has_tok,
 
 void rows_range(const void* base, const void* quant, const int32_t* tok,
                 int64_t r0, int64_t r1, int64_t V, int dtype, double* kld,
-                double* nll, int32_t* ab, int32_t* aq, uint32_t* flags) {
+                double* nll, double* nllb, int32_t* ab, int32_t* aq,
+                uint32_t* flags) {
   std::vector<double> b((size_t)V), q((size_t)V);
   for (int64_t r = r0; r < r1; ++r) {
     load_row(base, dtype, r, V, b.data());
     load_row(quant, dtype, r, V, q.data());
     one_row(b.data(), q.data(), V, tok != nullptr, tok ? tok[r] : 0, &kld[r],
-            &nll[r], &ab[r], &aq[r], &flags[r]);
+            &nll[r], &nllb[r], &ab[r], &aq[r], &flags[r]);
   }
 }
 
@@ -183,16 +200,18 @@ void rows_range(const void* base, const void* quant, const int32_t* tok,
 
 extern "C" int oracle_rows(const void* base, const void* quant,
                            const int32_t* tok, int64_t N, int64_t V, int dtype,
-                           double* kld, double* nll, int32_t* amax_b,
-                           int32_t* amax_q, uint32_t* flags, int nthreads) {
-  if (!base || !quant || !kld || !nll || !amax_b || !amax_q || !flags)
+                           double* kld, double* nll, double* nll_base,
+                           int32_t* amax_b, int32_t* amax_q, uint32_t* flags,
+                           int nthreads) {
+  if (!base || !quant || !kld || !nll || !nll_base || !amax_b || !amax_q ||
+      !flags)
     return -1;
   if (N < 0 || V < 1 || V > 0x7fffffffLL) return -1;
   if (dtype != ORACLE_F32 && dtype != ORACLE_BF16 && dtype != ORACLE_F16)
     return -1;
   if (nthreads <= 1 || N < 2) {
-    rows_range(base, quant, tok, 0, N, V, dtype, kld, nll, amax_b, amax_q,
-               flags);
+    rows_range(base, quant, tok, 0, N, V, dtype, kld, nll, nll_base, amax_b,
+               amax_q, flags);
     return 0;
   }
   /* Whole rows per thread: every row is computed by the same code in the same
@@ -202,7 +221,7 @@ extern "C" int oracle_rows(const void* base, const void* quant,
   for (int64_t t = 0; t < T; ++t) {
     int64_t r0 = N * t / T, r1 = N * (t + 1) / T;
     pool.emplace_back(rows_range, base, quant, tok, r0, r1, V, dtype, kld, nll,
-                      amax_b, amax_q, flags);
+                      nll_base, amax_b, amax_q, flags);
   }
   for (auto& th : pool) th.join();
   return 0;
@@ -222,18 +241,18 @@ extern "C" double oracle_percentile_sorted(const double* x, int64_t n,
 }
 
 extern "C" int oracle_reduce(const double* kld, const double* nll,
-                             const int32_t* amax_b, const int32_t* amax_q,
-                             const uint32_t* flags, int64_t N, int has_nll,
-                             oracle_result_t* out) {
+                             const double* nll_base, const int32_t* amax_b,
+                             const int32_t* amax_q, const uint32_t* flags,
+                             int64_t N, int has_nll, oracle_result_t* out) {
   if (!kld || !amax_b || !amax_q || !flags || !out || N < 0) return -1;
-  if (has_nll && !nll) return -1;
+  if (has_nll && (!nll || !nll_base)) return -1;
   std::memset(out, 0, sizeof(*out));
   out->n_rows = N;
   out->has_nll = has_nll ? 1 : 0;
 
   std::vector<double> valid;
   valid.reserve((size_t)N);
-  double sum_kl = 0.0, sum_nll = 0.0;
+  double sum_kl = 0.0, sum_nll = 0.0, sum_nllb = 0.0, sum_dp = 0.0, sum_dp2 = 0.0;
   int64_t agree = 0, n_nll = 0, n_flagged = 0;
   uint32_t f_or = 0;
   for (int64_t i = 0; i < N; ++i) {
@@ -246,6 +265,11 @@ extern "C" int oracle_reduce(const double* kld, const double* nll,
     if (amax_b[i] == amax_q[i]) ++agree;
     if (has_nll && !(f & ORACLE_ROW_BAD_TOKEN)) {
       sum_nll += nll[i];
+      sum_nllb += nll_base[i];
+      /* P(tok) = exp(-NLL) for each model; exp(-inf) = 0. */
+      const double dp = std::exp(-nll[i]) - std::exp(-nll_base[i]);
+      sum_dp += dp;
+      sum_dp2 += dp * dp;
       ++n_nll;
     }
   }
@@ -270,8 +294,15 @@ extern "C" int oracle_reduce(const double* kld, const double* nll,
   if (has_nll && n_nll > 0) {
     out->mean_nll = sum_nll / (double)n_nll;
     out->ppl = std::exp(out->mean_nll);
+    out->mean_nll_base = sum_nllb / (double)n_nll;
+    out->ppl_base = std::exp(out->mean_nll_base);
+    out->ln_ppl_ratio = out->mean_nll - out->mean_nll_base;
+    out->mean_dp = sum_dp / (double)n_nll;
+    out->rms_dp = std::sqrt(sum_dp2 / (double)n_nll);
   } else {
     out->mean_nll = out->ppl = kNaN;
+    out->mean_nll_base = out->ppl_base = out->ln_ppl_ratio = kNaN;
+    out->mean_dp = out->rms_dp = kNaN;
   }
   return 0;
 }

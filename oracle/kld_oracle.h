@@ -9,9 +9,12 @@
  *   - log-softmax of both rows over the full vocabulary,
  *   - KL(P_base || P_quant) in nats,
  *   - argmax of each row, lowest index on ties ("Same Top P"),
- *   - optionally NLL_i = -log P_quant(tok_i),
+ *   - optionally NLL_i = -log P_quant(tok_i) and NLLB_i = -log P_base(tok_i),
  * and over all rows: mean / median / p90 / p99 / max KLD, top-1 agreement
- * count and percentage, mean NLL and PPL = exp(mean NLL).
+ * count and percentage, mean NLL and PPL = exp(mean NLL), the same for the
+ * base row (PPL(base)), ln(PPL(Q)/PPL(base)) = mean NLL - mean NLLB, and the
+ * token-probability shift dp_i = P_quant(tok_i) - P_base(tok_i): its mean
+ * and its root mean square ("RMS dp").
  *
  * Sources:
  *   "Qwen3.6 27B Quantization Benchmark" (huy.rocks), sections "Measurement
@@ -19,7 +22,10 @@
  *     table (columns Mean PPL(Q), Mean KLD, Same top p).
  *   "Mistral-Small-4-119B-2603 GSQ-RCO IQ3_S GGUF" model card, "Quality" and
  *     "How it was made" steps 5 and 7: the direction is KL(BF16 || quantized)
- *     over the full vocabulary.
+ *     over the full vocabulary. Its "Quality" section also reads the
+ *     perplexity ratio and how many points of probability the quantized
+ *     model gives the correct token less than BF16 on average (mean dp);
+ *     the Qwen3.6 page's table has the "RMS dp (%)" column.
  *   Percentiles (median/p90/p99) are not printed on any page; they follow the
  *   linear-interpolation ("type 7") order-statistic rule stated below.
  */
@@ -41,7 +47,8 @@ enum {
   ORACLE_ROW_EMPTY     = 1u << 1, /* every entry of a row is -inf: row excluded */
   ORACLE_ROW_INF_KL    = 1u << 2, /* b_j finite where q_j = -inf: KL = +inf   */
   ORACLE_ROW_BAD_TOKEN = 1u << 3, /* token id outside [0, V): no NLL for row  */
-  ORACLE_ROW_INF_NLL   = 1u << 4  /* q[tok] = -inf: NLL = +inf                 */
+  ORACLE_ROW_INF_NLL   = 1u << 4, /* q[tok] = -inf: NLL = +inf                 */
+  ORACLE_ROW_INF_NLLB  = 1u << 5  /* b[tok] = -inf: NLLB = +inf                */
 };
 
 typedef struct {
@@ -62,6 +69,12 @@ typedef struct {
   int64_t n_flagged;  /* rows with any flag set                             */
   uint32_t flags_or;  /* OR of all row flags                                */
   uint32_t _pad2;
+  /* over the same rows as mean_nll (NaN without token ids): */
+  double mean_nll_base; /* mean of NLLB                                     */
+  double ppl_base;      /* exp(mean_nll_base)                               */
+  double ln_ppl_ratio;  /* mean_nll - mean_nll_base = ln(PPL(Q)/PPL(base))  */
+  double mean_dp;       /* mean of dp = exp(-NLL) - exp(-NLLB)              */
+  double rms_dp;        /* sqrt(mean of dp^2)                               */
 } oracle_result_t;
 
 /* Per-row statistics of rows [0, N). `tok` may be NULL (no NLL). Rows are
@@ -69,13 +82,14 @@ typedef struct {
  * leaves every per-row value bit-identical. Returns 0, or -1 on bad args. */
 int oracle_rows(const void* base, const void* quant, const int32_t* tok,
                 int64_t N, int64_t V, int dtype, double* kld, double* nll,
-                int32_t* amax_b, int32_t* amax_q, uint32_t* flags,
-                int nthreads);
+                double* nll_base, int32_t* amax_b, int32_t* amax_q,
+                uint32_t* flags, int nthreads);
 
 /* Reduction of per-row values to the summary statistics. */
-int oracle_reduce(const double* kld, const double* nll, const int32_t* amax_b,
-                  const int32_t* amax_q, const uint32_t* flags, int64_t N,
-                  int has_nll, oracle_result_t* out);
+int oracle_reduce(const double* kld, const double* nll, const double* nll_base,
+                  const int32_t* amax_b, const int32_t* amax_q,
+                  const uint32_t* flags, int64_t N, int has_nll,
+                  oracle_result_t* out);
 
 /* Type-7 percentile of an ascending array x[0..n): pos = p*(n-1). */
 double oracle_percentile_sorted(const double* x, int64_t n, double p);

@@ -38,6 +38,14 @@ MUTANTS = {
     "masked_quant_entry_ignored": ("      inf_kl = true;\n      continue;", "      continue;"),
     "bf16_widening_wrong": ("uint32_t u = (uint32_t)h << 16;", "uint32_t u = (uint32_t)h << 15;"),
     "agreement_counts_all_rows": ("if (amax_b[i] == amax_q[i]) ++agree;", "++agree;"),
+    "base_nll_under_quant_row": ("*nllb = lse_b - b[tok];", "*nllb = lse_q - q[tok];"),
+    "base_nll_without_normaliser": ("*nllb = lse_b - b[tok];", "*nllb = m_b - b[tok];"),
+    "dp_sign_flipped": ("const double dp = std::exp(-nll[i]) - std::exp(-nll_base[i]);",
+                        "const double dp = std::exp(-nll_base[i]) - std::exp(-nll[i]);"),
+    "rms_dp_without_root": ("out->rms_dp = std::sqrt(sum_dp2 / (double)n_nll);",
+                            "out->rms_dp = sum_dp2 / (double)n_nll;"),
+    "ppl_ratio_inverted": ("out->ln_ppl_ratio = out->mean_nll - out->mean_nll_base;",
+                           "out->ln_ppl_ratio = out->mean_nll_base - out->mean_nll;"),
 }
 
 

@@ -257,6 +257,87 @@ def test_bad_token_ids_are_flagged_and_excluded_from_ppl():
     assert abs(res["mean_nll"] - (r["nll"][0] + r["nll"][3]) / 2) < 1e-15
 
 
+# ------------------------------------------- base NLL, PPL(base), ratio, dp
+
+def test_base_nll_matches_brute_force_and_dp_statistics():
+    V, n = 9, 40
+    b = RNG.normal(0, 1.5, size=(n, V)).astype(np.float32)
+    q = RNG.normal(0, 2, size=(n, V)).astype(np.float32)
+    tok = RNG.integers(0, V, size=n).astype(np.int32)
+    r, res = _run(b, q, tok)
+    pb, pq = [], []
+    for i in range(n):
+        eb = [math.exp(float(x)) for x in b[i]]
+        eq = [math.exp(float(x)) for x in q[i]]
+        pb.append(eb[tok[i]] / math.fsum(eb))
+        pq.append(eq[tok[i]] / math.fsum(eq))
+    np.testing.assert_allclose(r["nll_base"], [-math.log(x) for x in pb], rtol=1e-13)
+    dp = [x - y for x, y in zip(pq, pb)]  # P_quant(tok) - P_base(tok)
+    assert abs(res["mean_dp"] - math.fsum(dp) / n) < 1e-14
+    assert abs(res["rms_dp"] - math.sqrt(math.fsum(d * d for d in dp) / n)) < 1e-14
+    want_b = math.fsum(-math.log(x) for x in pb) / n
+    assert abs(res["mean_nll_base"] - want_b) < 1e-13
+    assert abs(res["ppl_base"] - math.exp(want_b)) < 1e-12 * res["ppl_base"]
+    assert abs(res["ln_ppl_ratio"] - (res["mean_nll"] - want_b)) < 1e-13
+    assert abs(math.exp(res["ln_ppl_ratio"]) - res["ppl"] / res["ppl_base"]) < 1e-12
+
+
+def test_uniform_base_against_one_hot_quant_at_the_token():
+    # P_base(tok) = 1/V, P_quant(tok) = 1: dp = 1 - 1/V on every row, so the
+    # mean and the root mean square both equal it (a dropped square root or a
+    # flipped sign shows); NLLB = log V, NLL = 0, ln(PPL(Q)/PPL(base)) = -log V.
+    V = 50
+    b = np.zeros((6, V), np.float32)
+    q = np.full((6, V), NEG_INF, np.float32)
+    tok = np.arange(6, dtype=np.int32) * 7
+    q[np.arange(6), tok] = 3.0
+    r, res = _run(b, q, tok)
+    np.testing.assert_allclose(r["nll_base"], math.log(V), rtol=1e-14)
+    assert np.all(r["nll"] == 0.0)
+    assert abs(res["mean_dp"] - (1 - 1 / V)) < 1e-15
+    assert abs(res["rms_dp"] - (1 - 1 / V)) < 1e-15
+    assert abs(res["ln_ppl_ratio"] + math.log(V)) < 1e-14
+    assert abs(res["ppl_base"] - V) < 1e-11
+
+
+def test_identical_rows_have_zero_dp_and_unit_ppl_ratio():
+    b = RNG.normal(0, 2, size=(25, 3000)).astype(np.float32)
+    tok = RNG.integers(0, 3000, size=25).astype(np.int32)
+    r, res = _run(b, b.copy(), tok)
+    assert np.array_equal(r["nll"], r["nll_base"])
+    assert res["mean_dp"] == 0.0 and res["rms_dp"] == 0.0 and res["ln_ppl_ratio"] == 0.0
+    assert res["ppl"] == res["ppl_base"]
+
+
+def test_base_nll_invariant_to_adding_a_constant_and_masked_token():
+    V = 300
+    # logits on a 2^-10 grid, so that adding 64 is exact in fp32
+    b = (np.round(RNG.normal(0, 1, size=(3, V)) * 1024) / 1024).astype(np.float32)
+    q = RNG.normal(0, 1, size=(3, V)).astype(np.float32)
+    tok = np.array([5, 17, 200], np.int32)
+    r0, _ = _run(b, q, tok)
+    assert np.array_equal((b + np.float32(64.0)).astype(np.float64) - 64.0, b.astype(np.float64))
+    r1, _ = _run(b + np.float32(64.0), q, tok)
+    np.testing.assert_allclose(r1["nll_base"], r0["nll_base"], rtol=1e-13)
+    b2 = b.copy()
+    b2[2, 200] = NEG_INF   # the base gives the token no probability
+    r2, res2 = _run(b2, q, tok)
+    assert r2["nll_base"][2] == math.inf and r2["flags"][2] & oracle.ROW_INF_NLLB
+    assert res2["ppl_base"] == math.inf
+    # P_base(tok) = 0 there, so that row's dp is P_quant(tok), still finite
+    pq = math.exp(-r2["nll"][2])
+    dp = [math.exp(-r2["nll"][i]) - math.exp(-r2["nll_base"][i]) for i in range(3)]
+    assert abs(dp[2] - pq) < 1e-16 and abs(res2["mean_dp"] - math.fsum(dp) / 3) < 1e-15
+
+
+def test_without_tokens_base_statistics_are_nan():
+    b = RNG.normal(0, 1, size=(4, 50)).astype(np.float32)
+    r, res = _run(b, b + np.float32(0.1))
+    assert np.all(np.isnan(r["nll_base"]))
+    for k in ("mean_nll_base", "ppl_base", "ln_ppl_ratio", "mean_dp", "rms_dp"):
+        assert math.isnan(res[k]), k
+
+
 # ---------------------------------------------------------------- argmax / ties
 
 def test_argmax_ties_go_to_lowest_index():
