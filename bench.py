@@ -35,8 +35,8 @@ METRIC = "logit rows/s and HBM GB/s (fraction of B200 peak) for KLD+top-1 at V=1
 WORKLOAD = "ctx8192_v151936_f32"
 VARIANT = "ctx8192_v151936_bf16"
 FALLBACK_HBM_GBS = 6650.0
-RESULT_BYTES = 120  # sizeof(kld_result_t)
-ROW_RECORD_BYTES = 32
+RESULT_BYTES = 160  # sizeof(kld_result_t)
+ROW_RECORD_BYTES = 40  # sizeof(kld_row_t)
 
 
 def _env_int(name, default):
@@ -494,6 +494,7 @@ def main():
             "gpu_launches": 2 * args.steps, "clocks": clocks,
             "gbs": in_bytes * world / (ms_per_step / 1000.0) / 1e9,
             "mean_kld": res["mean_kld"], "top1_agree_pct": res["top1_agree_pct"], "ppl": res["ppl"],
+            "ppl_base": res["ppl_base"], "rms_dp": res["rms_dp"], "mean_dp": res["mean_dp"],
             "variants": variants, "split_row": split_row,
         }
         if args.rows is not None or args.dtype != "f32" or args.split_calls != SPLIT_CALLS:

@@ -59,7 +59,7 @@
 extern "C" {
 #endif
 
-#define KLD_ABI_VERSION 1
+#define KLD_ABI_VERSION 2
 
 typedef enum {
   KLD_OK = 0,
@@ -85,11 +85,13 @@ typedef enum { KLD_F32 = 0, KLD_BF16 = 1, KLD_F16 = 2 } kld_dtype_t;
 #define KLD_ROW_INF_KL    (1u << 2)
 #define KLD_ROW_BAD_TOKEN (1u << 3)
 #define KLD_ROW_INF_NLL   (1u << 4)
+#define KLD_ROW_INF_NLL_BASE (1u << 5)  /* b[tok] = -inf: nll_base = +inf */
 
-/* One 32-byte record per row, written by the row pass. */
+/* One 40-byte record per row, written by the row pass. */
 typedef struct {
   double kld;            /* KL(P_base || P_quant) in nats (NaN if excluded) */
   double nll;            /* -log P_quant(tok) (NaN if no/bad token)        */
+  double nll_base;       /* -log P_base(tok), same conditions               */
   int32_t argmax_base;   /* lowest index of the row maximum, -1 if excluded */
   int32_t argmax_quant;
   uint32_t flags;        /* KLD_ROW_* bits                                  */
@@ -115,6 +117,15 @@ typedef struct {
   int64_t n_flagged;     /* rows with any flag                                */
   uint32_t flags_or;     /* OR of all row flags                               */
   uint32_t device_error; /* nonzero if a bounded device wait gave up          */
+  /* Over the same rows as mean_nll (NaN without token ids). The perplexity
+   * ratio and the probability the quantized model gives the token against
+   * the base ("Mistral-Small-4-119B-2603 GSQ-RCO IQ3_S GGUF", "Quality";
+   * "Qwen3.6 27B Quantization Benchmark", table column RMS dp (%)). */
+  double mean_nll_base;  /* mean of -log P_base(tok)                         */
+  double ppl_base;       /* exp(mean_nll_base)                                */
+  double ln_ppl_ratio;   /* mean_nll - mean_nll_base = ln(PPL(Q)/PPL(base))   */
+  double mean_dp;        /* mean of dp = P_quant(tok) - P_base(tok)           */
+  double rms_dp;         /* sqrt(mean of dp^2)                                */
 } kld_result_t;
 
 typedef struct kld_stats_s* kld_stats_t;
@@ -130,7 +141,7 @@ const char* kld_last_cuda_error(void);
 
 /*
  * Create a handle on `device` for runs of up to `max_rows` rows.
- * Allocates a device workspace of max_rows records (32 bytes each) plus a few
+ * Allocates a device workspace of max_rows records (40 bytes each) plus a few
  * KB, and a pinned host copy of the result. Returns KLD_ERR_NO_DEVICE if the
  * device is not a compute-capability 10.0 (B200-class) GPU.
  */
@@ -259,7 +270,7 @@ kld_status_t kld_plan(int64_t N, int64_t V, kld_dtype_t dtype, int sm_count,
  * start-up, or a loop that cannot afford the device synchronisation
  * cudaMalloc/cudaFree may cause. It takes no handle and allocates nothing:
  * per-row records and the error word live in one fixed array compiled into
- * the library (KLD_STATIC_MAX_ROWS records, about 2 MiB), which every GPU
+ * the library (KLD_STATIC_MAX_ROWS records, about 2.5 MiB), which every GPU
  * that loads the library keeps until the process exits.
  *
  * Runs on the calling thread's current device and enqueues the row pass and

@@ -17,12 +17,12 @@ import torch
 
 from . import _lib
 from ._lib import (KLD_BF16, KLD_F16, KLD_F32, ROW_BAD_TOKEN, ROW_EMPTY,  # noqa: F401
-                   ROW_INF_KL, ROW_INF_NLL, ROW_NONFINITE, KLDError)
+                   ROW_INF_KL, ROW_INF_NLL, ROW_INF_NLL_BASE, ROW_NONFINITE, KLDError)
 
 __all__ = ["KLDStats", "kld_stats", "run_static", "result_from_bytes", "plan", "dtype_code",
            "ROW_RECORD_BYTES"]
 
-ROW_RECORD_BYTES = 32
+ROW_RECORD_BYTES = 40
 
 _DTYPES = {torch.float32: KLD_F32, torch.bfloat16: KLD_BF16, torch.float16: KLD_F16}
 
@@ -66,12 +66,12 @@ def _check_pair(base: torch.Tensor, quant: torch.Tensor, token_ids, on_device: b
 
 
 def rows_view(records: torch.Tensor) -> dict:
-    """Field views of a [N, 32] uint8 tensor of row records."""
+    """Field views of a [N, 40] uint8 tensor of row records (kld_row_t)."""
     r = records.view(torch.uint8).reshape(-1, ROW_RECORD_BYTES)
-    f64 = r[:, :16].contiguous().view(torch.float64)
-    i32 = r[:, 16:28].contiguous().view(torch.int32)
-    return {"kld": f64[:, 0], "nll": f64[:, 1], "amax_b": i32[:, 0], "amax_q": i32[:, 1],
-            "flags": i32[:, 2]}
+    f64 = r[:, :24].contiguous().view(torch.float64)
+    i32 = r[:, 24:36].contiguous().view(torch.int32)
+    return {"kld": f64[:, 0], "nll": f64[:, 1], "nll_base": f64[:, 2], "amax_b": i32[:, 0],
+            "amax_q": i32[:, 1], "flags": i32[:, 2]}
 
 
 class KLDStats:
@@ -128,11 +128,11 @@ class KLDStats:
         _lib.check(st, "kld_stats_run_host")
 
     def run_rows(self, base, quant, token_ids=None, out: torch.Tensor | None = None, stream=None):
-        """Row pass only; records go to ``out`` ([N, 32] uint8 on the device)
+        """Row pass only; records go to ``out`` ([N, 40] uint8 on the device)
         or to the handle's workspace."""
         _check_pair(base, quant, token_ids, True)
         if out is not None and (out.dtype != torch.uint8 or out.numel() < base.shape[0] * ROW_RECORD_BYTES):
-            raise ValueError("out must be a uint8 tensor of N*32 bytes")
+            raise ValueError("out must be a uint8 tensor of N*40 bytes")
         st = self._lib.kld_stats_run_rows(self._h, _ptr(base), _ptr(quant), _ptr(token_ids),
                                           base.shape[0], base.shape[1], dtype_code(base), _ptr(out),
                                           ctypes.c_void_p(_stream_ptr(stream, base.device)))
@@ -159,7 +159,7 @@ class KLDStats:
         return out
 
     def rows(self) -> torch.Tensor:
-        """Copy of the last run's per-row records as a [N, 32] uint8 CUDA
+        """Copy of the last run's per-row records as a [N, 40] uint8 CUDA
         tensor (see :func:`rows_view`), ordered after the run on the current
         stream."""
         p = ctypes.c_void_p()

@@ -32,12 +32,14 @@ ROW_EMPTY = 1 << 1
 ROW_INF_KL = 1 << 2
 ROW_BAD_TOKEN = 1 << 3
 ROW_INF_NLL = 1 << 4
+ROW_INF_NLL_BASE = 1 << 5
 
 
 class Row(ctypes.Structure):
     _fields_ = [
         ("kld", ctypes.c_double),
         ("nll", ctypes.c_double),
+        ("nll_base", ctypes.c_double),
         ("argmax_base", ctypes.c_int32),
         ("argmax_quant", ctypes.c_int32),
         ("flags", ctypes.c_uint32),
@@ -64,6 +66,11 @@ class Result(ctypes.Structure):
         ("n_flagged", ctypes.c_int64),
         ("flags_or", ctypes.c_uint32),
         ("device_error", ctypes.c_uint32),
+        ("mean_nll_base", ctypes.c_double),
+        ("ppl_base", ctypes.c_double),
+        ("ln_ppl_ratio", ctypes.c_double),
+        ("mean_dp", ctypes.c_double),
+        ("rms_dp", ctypes.c_double),
     ]
 
 
@@ -80,7 +87,7 @@ class Plan(ctypes.Structure):
     ]
 
 
-assert ctypes.sizeof(Row) == 32
+assert ctypes.sizeof(Row) == 40
 _P = ctypes.c_void_p
 _I64 = ctypes.c_int64
 _I32 = ctypes.c_int

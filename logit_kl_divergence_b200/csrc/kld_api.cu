@@ -1,6 +1,6 @@
 // kld_api.cu -- host side of the C ABI declared in include/kld_stats.h.
 //
-// Owns the per-handle device workspace (one 32-byte record per row, an
+// Owns the per-handle device workspace (one 40-byte record per row, an
 // error word, the split-row scratch), the mapped pinned host result that the
 // reduction kernel writes directly, and the staging buffers of the
 // host-memory path; validates arguments before anything is enqueued and maps

@@ -7,7 +7,11 @@
 //   mean KLD   = sum of the valid rows' KL / n_valid,
 //   agreement  = valid rows whose two argmaxes are equal, and its percentage,
 //   mean NLL   = sum over valid rows with an in-range token / their count,
-//   PPL        = exp(mean NLL),
+//   PPL        = exp(mean NLL), and the same for the base model's NLL,
+//   ln ratio   = mean NLL - mean base NLL = ln(PPL(Q) / PPL(base)),
+//   dp         = exp(-NLL) - exp(-base NLL) = P_quant(tok) - P_base(tok) per
+//                row; its mean and sqrt(mean dp^2) ("Mistral-Small-4-119B-2603
+//                GSQ-RCO IQ3_S GGUF", "Quality"; the Qwen3.6 table's RMS dp),
 //   percentile = x_(k) + (pos - k) * (x_(k+1) - x_(k)),  pos = p*(n-1),
 //                k = floor(pos), over the sorted valid KL values; max = x_(n-1).
 //
@@ -53,7 +57,7 @@ __device__ double interpolate(double pos, double lo, double hi) {
 }
 
 struct ReduceShared {
-  double dsum[32][2];
+  double dsum[32][5];
   long long isum[32][4];
   unsigned int flags_or[32];
   // selection state
@@ -81,7 +85,7 @@ __global__ void __launch_bounds__(kReduceThreads, 1)
   asm volatile("griddepcontrol.wait;" ::: "memory");
 
   // ---------------------------------------------------------------- sums
-  double s_kl = 0.0, s_nll = 0.0;
+  double s_kl = 0.0, s_nll = 0.0, s_nllb = 0.0, s_dp = 0.0, s_dp2 = 0.0;
   long long n_valid = 0, agree = 0, n_nll = 0, n_flag = 0;
   unsigned int f_or = 0;
   for (int64_t i = tid; i < N; i += nt) {
@@ -94,6 +98,10 @@ __global__ void __launch_bounds__(kReduceThreads, 1)
     if (rec.argmax_base == rec.argmax_quant) ++agree;
     if (has_nll && !(rec.flags & KLD_ROW_BAD_TOKEN)) {
       s_nll += rec.nll;
+      s_nllb += rec.nll_base;
+      const double dp = exp(-rec.nll) - exp(-rec.nll_base);
+      s_dp += dp;
+      s_dp2 += dp * dp;
       ++n_nll;
     }
   }
@@ -101,6 +109,9 @@ __global__ void __launch_bounds__(kReduceThreads, 1)
   for (int o = 16; o > 0; o >>= 1) {
     s_kl += __shfl_down_sync(0xffffffffu, s_kl, o);
     s_nll += __shfl_down_sync(0xffffffffu, s_nll, o);
+    s_nllb += __shfl_down_sync(0xffffffffu, s_nllb, o);
+    s_dp += __shfl_down_sync(0xffffffffu, s_dp, o);
+    s_dp2 += __shfl_down_sync(0xffffffffu, s_dp2, o);
     n_valid += __shfl_down_sync(0xffffffffu, n_valid, o);
     agree += __shfl_down_sync(0xffffffffu, agree, o);
     n_nll += __shfl_down_sync(0xffffffffu, n_nll, o);
@@ -110,6 +121,9 @@ __global__ void __launch_bounds__(kReduceThreads, 1)
   if (lane == 0) {
     sh.dsum[warp][0] = s_kl;
     sh.dsum[warp][1] = s_nll;
+    sh.dsum[warp][2] = s_nllb;
+    sh.dsum[warp][3] = s_dp;
+    sh.dsum[warp][4] = s_dp2;
     sh.isum[warp][0] = n_valid;
     sh.isum[warp][1] = agree;
     sh.isum[warp][2] = n_nll;
@@ -121,6 +135,9 @@ __global__ void __launch_bounds__(kReduceThreads, 1)
     const bool has = lane < (nt >> 5);
     s_kl = has ? sh.dsum[lane][0] : 0.0;
     s_nll = has ? sh.dsum[lane][1] : 0.0;
+    s_nllb = has ? sh.dsum[lane][2] : 0.0;
+    s_dp = has ? sh.dsum[lane][3] : 0.0;
+    s_dp2 = has ? sh.dsum[lane][4] : 0.0;
     n_valid = has ? sh.isum[lane][0] : 0;
     agree = has ? sh.isum[lane][1] : 0;
     n_nll = has ? sh.isum[lane][2] : 0;
@@ -130,6 +147,9 @@ __global__ void __launch_bounds__(kReduceThreads, 1)
     for (int o = 16; o > 0; o >>= 1) {
       s_kl += __shfl_down_sync(0xffffffffu, s_kl, o);
       s_nll += __shfl_down_sync(0xffffffffu, s_nll, o);
+      s_nllb += __shfl_down_sync(0xffffffffu, s_nllb, o);
+      s_dp += __shfl_down_sync(0xffffffffu, s_dp, o);
+      s_dp2 += __shfl_down_sync(0xffffffffu, s_dp2, o);
       n_valid += __shfl_down_sync(0xffffffffu, n_valid, o);
       agree += __shfl_down_sync(0xffffffffu, agree, o);
       n_nll += __shfl_down_sync(0xffffffffu, n_nll, o);
@@ -139,6 +159,9 @@ __global__ void __launch_bounds__(kReduceThreads, 1)
     if (lane == 0) {
       sh.dsum[0][0] = s_kl;
       sh.dsum[0][1] = s_nll;
+      sh.dsum[0][2] = s_nllb;
+      sh.dsum[0][3] = s_dp;
+      sh.dsum[0][4] = s_dp2;
       sh.isum[0][0] = n_valid;
       sh.isum[0][1] = agree;
       sh.isum[0][2] = n_nll;
@@ -326,10 +349,18 @@ __global__ void __launch_bounds__(kReduceThreads, 1)
       r.top1_agree_pct = nan;
     }
     if (has_nll && sh.isum[0][2] > 0) {
-      r.mean_nll = sh.dsum[0][1] / static_cast<double>(sh.isum[0][2]);
+      const double nn = static_cast<double>(sh.isum[0][2]);
+      r.mean_nll = sh.dsum[0][1] / nn;
       r.ppl = exp(r.mean_nll);
+      r.mean_nll_base = sh.dsum[0][2] / nn;
+      r.ppl_base = exp(r.mean_nll_base);
+      r.ln_ppl_ratio = r.mean_nll - r.mean_nll_base;
+      r.mean_dp = sh.dsum[0][3] / nn;
+      r.rms_dp = sqrt(sh.dsum[0][4] / nn);
     } else {
       r.mean_nll = r.ppl = nan;
+      r.mean_nll_base = r.ppl_base = r.ln_ppl_ratio = nan;
+      r.mean_dp = r.rms_dp = nan;
     }
     *out = r;
   }

@@ -51,7 +51,7 @@
 //   - warp 17 (epilogue): per row, the unaligned head/tail (< 16 bytes each)
 //     and the token gather, the exact lowest-index argmax (re-reading only
 //     the chunks of lanes whose maximum equals the row maximum), the fp64
-//     combine of the 17 partials and the 32-byte record.
+//     combine of the 17 partials and the 40-byte record.
 //   All waits are mbarrier waits bounded by wall time; a wait that gives up
 //   sets an error bit that the reduction reports, and the CTA leaves only
 //   after its bulk copies have landed.
@@ -801,13 +801,15 @@ __device__ MPart warp_merge(const MPart& p) {
 }
 
 // The record of a whole row from its merged partial.
-__device__ kld_row_t finalize_row(const MPart& m, bool has_tok, bool tok_ok, float q_tok) {
+__device__ kld_row_t finalize_row(const MPart& m, bool has_tok, bool tok_ok, float q_tok,
+                                  float b_tok) {
   kld_row_t rec;
   uint32_t flags = 0;
   if (has_tok && !tok_ok) flags |= KLD_ROW_BAD_TOKEN;
   const double nan = __longlong_as_double(0x7ff8000000000000ll);
   rec.kld = nan;
   rec.nll = nan;
+  rec.nll_base = nan;
   rec.argmax_base = -1;
   rec.argmax_quant = -1;
   const bool nonfinite = (m.flags & (kPartNonfinite | kPartFailed)) || isnan(m.Sb) || isnan(m.B) ||
@@ -832,6 +834,14 @@ __device__ kld_row_t finalize_row(const MPart& m, bool has_tok, bool tok_ok, flo
         rec.nll = log(m.B + m.Sb) +
                   kLn2 * (static_cast<double>(m.Cb) -
                           (static_cast<double>(m.K) + static_cast<double>(q_tok)) * kLog2eD);
+      }
+      if (b_tok == -INFINITY) {
+        rec.nll_base = INFINITY;
+        flags |= KLD_ROW_INF_NLL_BASE;
+      } else {
+        // S is the sum of all base weights in frame Cb.
+        rec.nll_base = log(m.Sb) + kLn2 * (static_cast<double>(m.Cb) -
+                                           static_cast<double>(b_tok) * kLog2eD);
       }
     }
     rec.argmax_base = m.amax_b;
@@ -1192,18 +1202,21 @@ __global__ void __launch_bounds__(kRowThreads, 1)
       // Next-token gather (only the CTA that finalises the row needs it).
       int32_t tk = 0;
       bool tok_ok = false;
-      float q_tok = 0.f;
+      float q_tok = 0.f, b_tok = 0.f;
       auto gather_token = [&]() {
         if (tok != nullptr) {
           tk = __ldg(tok + r);
           tok_ok = tk >= 0 && static_cast<int64_t>(tk) < V;
-          if (tok_ok) q_tok = Elem<DT>::load(rq, tk);
+          if (tok_ok) {
+            q_tok = Elem<DT>::load(rq, tk);
+            b_tok = Elem<DT>::load(rb, tk);
+          }
         }
       };
 
       if (P == 1) {
         gather_token();
-        const kld_row_t rec = finalize_row(m, tok != nullptr, tok_ok, q_tok);
+        const kld_row_t rec = finalize_row(m, tok != nullptr, tok_ok, q_tok, b_tok);
         if (lane == 0) rows[r] = rec;
         continue;
       }
@@ -1274,7 +1287,7 @@ __global__ void __launch_bounds__(kRowThreads, 1)
       const int C = P / static_cast<int>(G);  // clusters per row
       if (C == 1) {
         gather_token();
-        const kld_row_t rec = finalize_row(cm, tok != nullptr, tok_ok, q_tok);
+        const kld_row_t rec = finalize_row(cm, tok != nullptr, tok_ok, q_tok, b_tok);
         if (lane == 0) rows[r] = rec;
         continue;
       }
@@ -1306,7 +1319,7 @@ __global__ void __launch_bounds__(kRowThreads, 1)
       }
       const MPart fm = warp_merge(q);
       gather_token();
-      const kld_row_t rec = finalize_row(fm, tok != nullptr, tok_ok, q_tok);
+      const kld_row_t rec = finalize_row(fm, tok != nullptr, tok_ok, q_tok, b_tok);
       if (lane == 0) {
         rows[r] = rec;
         tickets[r] = 0u;  // ready for the next launch

@@ -11,7 +11,7 @@
 // the inputs and a device buffer for the result.
 //
 // The array is part of this library's device image: every GPU that loads the
-// library holds it (KLD_STATIC_MAX_ROWS records, 2 MiB plus 256 bytes) until
+// library holds it (KLD_STATIC_MAX_ROWS records, 2.5 MiB plus 256 bytes) until
 // the process exits. Host code never dereferences it: the array's name on the
 // host is only a stand-in, so the first call on each device (with that device
 // current) looks up its device address with cudaGetSymbolAddress and keeps it.

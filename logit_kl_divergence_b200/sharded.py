@@ -2,7 +2,7 @@
 
 Rows are independent, so N rows split across ranks with no exchange in the
 row pass. The one real exchange is for the order statistics: every rank
-all-gathers the 32-byte per-row records in rank order (NCCL over NVLink on
+all-gathers the 40-byte per-row records in rank order (NCCL over NVLink on
 GPUs; any torch.distributed backend carries the gather) and reduces the full
 set, so the percentiles stay exact and every rank holds the same result.
 
@@ -14,7 +14,7 @@ from __future__ import annotations
 import torch
 import torch.distributed as dist
 
-ROW_RECORD_BYTES = 32
+ROW_RECORD_BYTES = 40  # sizeof(kld_row_t)
 
 
 def shard_bounds(n_rows: int, world: int, rank: int) -> tuple[int, int]:
@@ -28,13 +28,13 @@ def shard_bounds(n_rows: int, world: int, rank: int) -> tuple[int, int]:
 
 
 def gather_records(records: torch.Tensor, group=None, counts: list[int] | None = None) -> torch.Tensor:
-    """All-gather every rank's [n_r, 32] uint8 records, concatenated in rank
+    """All-gather every rank's [n_r, 40] uint8 records, concatenated in rank
     order (ranks may hold different row counts). Collective: every rank of
     `group` calls it with its own records, in the same order of calls.
     `counts`: every rank's row count when the caller knows them (skips one
     small all-gather)."""
     if records.dtype != torch.uint8 or records.dim() != 2 or records.shape[1] != ROW_RECORD_BYTES:
-        raise ValueError("records must be a [n, 32] uint8 tensor")
+        raise ValueError("records must be a [n, 40] uint8 tensor")
     world = dist.get_world_size(group)
     if counts is None:
         n = torch.tensor([records.shape[0]], dtype=torch.int64, device=records.device)

@@ -2,10 +2,13 @@
 and compare with the fp64 oracle at the stated tolerances.
 
 Tolerances: argmax indices, flags and agreement counts bit-exact; per-row KL
-and NLL |gpu - ref| <= 1e-6 + 1e-4 * |ref|; mean KLD, percentiles, mean NLL
-and PPL within 1e-5 relative, with an absolute floor where the reference is
-~0 (1e-9 nats for KL statistics, 1e-7 nats for mean NLL, i.e. 1e-7 relative
-for PPL): fp32 inputs do not resolve a log-probability better than that.
+and NLL (quant and base) |gpu - ref| <= 1e-6 + 1e-4 * |ref|; mean KLD,
+percentiles, mean NLL and PPL (quant and base), the PPL ratio and the mean
+and RMS of dp within 1e-5 relative, with an absolute floor where the
+reference is ~0 (1e-9 nats for KL statistics, 1e-7 nats for mean NLL, i.e.
+1e-7 relative for PPL, 1e-9 for dp statistics): fp32 inputs do not resolve a
+log-probability better than that. ln(PPL ratio) within 1e-5 absolute is the
+ratio within 1e-5 relative.
 """
 from __future__ import annotations
 
@@ -23,7 +26,8 @@ EXCLUDED = oracle.ROW_NONFINITE | oracle.ROW_EMPTY
 ROW_ATOL, ROW_RTOL = 1e-6, 1e-4
 STAT_RTOL = 1e-5
 STAT_ATOL = {"mean_kld": 1e-9, "median_kld": 1e-9, "p90_kld": 1e-9, "p99_kld": 1e-9,
-             "max_kld": 1e-9, "mean_nll": 1e-7, "top1_agree_pct": 0.0}
+             "max_kld": 1e-9, "mean_nll": 1e-7, "mean_nll_base": 1e-7, "top1_agree_pct": 0.0,
+             "mean_dp": 1e-9, "rms_dp": 1e-9}
 CORES = max(1, os.cpu_count() or 1)
 
 
@@ -35,7 +39,7 @@ def gpu_run(base, quant, tok=None, use_rows_api=False, split=None):
         st.set_split(split)
     try:
         if use_rows_api:
-            out = torch.empty((base.shape[0], 32), dtype=torch.uint8, device=base.device)
+            out = torch.empty((base.shape[0], 40), dtype=torch.uint8, device=base.device)
             st.run_rows(base, quant, tok, out=out)
             st.reduce(out, base.shape[0], tok is not None)
             res = st.result()
@@ -73,6 +77,7 @@ def assert_rows_match(g: dict, o: dict, idx=None):
         f"argmax_quant differs at rows {idx[np.nonzero(g['amax_q'] != o['amax_q'])[0][:8]]}")
     _close_rows(g["kld"], o["kld"], "kld", idx)
     _close_rows(g["nll"], o["nll"], "nll", idx)
+    _close_rows(g["nll_base"], o["nll_base"], "nll_base", idx)
 
 
 def stat_close(a, b, key):
@@ -80,8 +85,11 @@ def stat_close(a, b, key):
         return math.isnan(a) and math.isnan(b)
     if math.isinf(a) or math.isinf(b):
         return a == b
-    if key == "ppl":
+    if key in ("ppl", "ppl_base"):
         return abs(a - b) <= (STAT_RTOL + 1e-7) * abs(b)
+    if key == "ln_ppl_ratio":
+        # the ratio PPL(Q)/PPL(base) within STAT_RTOL relative
+        return abs(a - b) <= STAT_RTOL
     return abs(a - b) <= STAT_ATOL[key] + STAT_RTOL * abs(b)
 
 
@@ -89,7 +97,7 @@ def assert_stats_match(gres: dict, ores: dict):
     for k in ("n_rows", "n_valid", "top1_agree", "n_nll", "n_flagged", "flags_or", "has_nll"):
         assert int(gres[k]) == int(ores[k]), (k, gres[k], ores[k])
     for k in ("mean_kld", "median_kld", "p90_kld", "p99_kld", "max_kld", "top1_agree_pct",
-              "mean_nll", "ppl"):
+              "mean_nll", "ppl", "mean_nll_base", "ppl_base", "ln_ppl_ratio", "mean_dp", "rms_dp"):
         assert stat_close(gres[k], ores[k], k), (k, gres[k], ores[k])
     assert gres["device_error"] == 0
 
@@ -108,7 +116,7 @@ def assert_select_exact(g_rows: dict, gres: dict, has_nll: bool):
 def oracle_rows_chunked(w, nthreads=CORES, chunk_rows=1024):
     """Oracle per-row values of a device workload, computed on host chunks."""
     n = w.base.shape[0]
-    out = {k: [] for k in ("kld", "nll", "amax_b", "amax_q", "flags")}
+    out = {k: [] for k in ("kld", "nll", "nll_base", "amax_b", "amax_q", "flags")}
     for r0 in range(0, n, chunk_rows):
         r1 = min(n, r0 + chunk_rows)
         b = w.base[r0:r1].cpu()

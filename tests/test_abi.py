@@ -50,9 +50,11 @@ def test_struct_layouts_match_header():
 #include "kld_stats.h"
 int main(void) {
   printf("%zu %zu %zu\n", sizeof(kld_row_t), sizeof(kld_result_t), sizeof(kld_plan_t));
-  printf("%zu %zu %zu %zu\n", offsetof(kld_result_t, top1_agree), offsetof(kld_result_t, has_nll),
-         offsetof(kld_result_t, ppl), offsetof(kld_result_t, device_error));
-  printf("%zu %zu\n", offsetof(kld_row_t, argmax_base), offsetof(kld_row_t, flags));
+  printf("%zu %zu %zu %zu %zu %zu\n", offsetof(kld_result_t, top1_agree), offsetof(kld_result_t, has_nll),
+         offsetof(kld_result_t, ppl), offsetof(kld_result_t, device_error),
+         offsetof(kld_result_t, mean_nll_base), offsetof(kld_result_t, rms_dp));
+  printf("%zu %zu %zu\n", offsetof(kld_row_t, argmax_base), offsetof(kld_row_t, flags),
+         offsetof(kld_row_t, nll_base));
   return 0;
 }
 '''
@@ -66,13 +68,14 @@ int main(void) {
     assert sizes == [ctypes.sizeof(_lib.Row), ctypes.sizeof(_lib.Result), ctypes.sizeof(_lib.Plan)]
     offs = [int(x) for x in lines[1].split()]
     assert offs == [_lib.Result.top1_agree.offset, _lib.Result.has_nll.offset,
-                    _lib.Result.ppl.offset, _lib.Result.device_error.offset]
+                    _lib.Result.ppl.offset, _lib.Result.device_error.offset,
+                    _lib.Result.mean_nll_base.offset, _lib.Result.rms_dp.offset]
     roffs = [int(x) for x in lines[2].split()]
-    assert roffs == [_lib.Row.argmax_base.offset, _lib.Row.flags.offset]
+    assert roffs == [_lib.Row.argmax_base.offset, _lib.Row.flags.offset, _lib.Row.nll_base.offset]
 
 
 def test_abi_version_and_status_strings(lib):
-    assert lib.kld_abi_version() == 1
+    assert lib.kld_abi_version() == 2
     for s in range(0, 10):
         assert lib.kld_status_string(s)
     assert lib.kld_status_string(12345) == b"unknown status"

@@ -16,8 +16,9 @@ from logit_kl_divergence_b200 import KLDStats
 pytestmark = pytest.mark.gpu
 DEV = torch.device("cuda", 0)
 
-REC = np.dtype([("kld", "<f8"), ("nll", "<f8"), ("amax_b", "<i4"), ("amax_q", "<i4"),
-                ("flags", "<u4"), ("reserved", "<u4")])
+REC = np.dtype([("kld", "<f8"), ("nll", "<f8"), ("nll_base", "<f8"), ("amax_b", "<i4"),
+                ("amax_q", "<i4"), ("flags", "<u4"), ("reserved", "<u4")])
+assert REC.itemsize == 40
 
 
 def make_records(kld, rng, flags=None, nll=True):
@@ -25,6 +26,7 @@ def make_records(kld, rng, flags=None, nll=True):
     r = np.zeros(n, REC)
     r["kld"] = kld
     r["nll"] = rng.gamma(2.0, 1.0, n) if nll else np.nan
+    r["nll_base"] = rng.gamma(2.0, 1.0, n) if nll else np.nan
     r["amax_b"] = rng.integers(0, 5, n)
     r["amax_q"] = rng.integers(0, 5, n)
     if flags is not None:
@@ -47,19 +49,24 @@ def run_reduce(rec, has_nll=True):
 
 def check(rec, has_nll=True):
     g = run_reduce(rec, has_nll)
-    d = {"kld": rec["kld"], "nll": rec["nll"], "amax_b": rec["amax_b"],
+    d = {"kld": rec["kld"], "nll": rec["nll"], "nll_base": rec["nll_base"], "amax_b": rec["amax_b"],
          "amax_q": rec["amax_q"], "flags": rec["flags"]}
     o = oracle.reduce(d, has_nll)
     for k in ("median_kld", "p90_kld", "p99_kld", "max_kld"):
         assert g[k] == o[k] or (math.isnan(g[k]) and math.isnan(o[k])), (k, g[k], o[k])
     for k in ("n_rows", "n_valid", "top1_agree", "n_nll", "n_flagged", "flags_or"):
         assert int(g[k]) == int(o[k]), k
-    for k in ("mean_kld", "mean_nll", "ppl", "top1_agree_pct"):
+    for k in ("mean_kld", "mean_nll", "ppl", "top1_agree_pct", "mean_nll_base", "ppl_base",
+              "mean_dp"):
         a, b = g[k], o[k]
         if math.isnan(b) or math.isinf(b):
             assert (math.isnan(a) and math.isnan(b)) or a == b, (k, a, b)
         else:
             assert abs(a - b) <= 1e-12 * abs(b) + 1e-300, (k, a, b)
+    # differences of nearly equal sums: absolute bars at fp64 rounding level
+    for k, tol in (("ln_ppl_ratio", 1e-12), ("rms_dp", 1e-12)):
+        a, b = g[k], o[k]
+        assert (math.isnan(a) and math.isnan(b)) or a == b or abs(a - b) <= tol, (k, a, b)
     return g
 
 

@@ -35,7 +35,7 @@ def nccl_group():
 
 def test_sharded_run_equals_single_handle_run(nccl_group):
     w = synth.make_recipe("ctx", n=300, v=32001, dtype=synth.BF16, seed=31, device=DEV)
-    rec = torch.arange(5 * 32, dtype=torch.uint8, device=DEV).view(5, 32)
+    rec = torch.arange(5 * 40, dtype=torch.uint8, device=DEV).view(5, 40)
     assert torch.equal(gather_records(rec), rec)
     assert torch.equal(gather_records(rec, counts=[5]), rec)
     sk = ShardedKLDStats(max_rows_per_rank=300, device=DEV)

@@ -1,5 +1,5 @@
 """Row sharding across processes (the multi-GPU path's host logic), run as
-gloo ranks on the CPU: shard bounds, the rank-ordered all-gather of 32-byte
+gloo ranks on the CPU: shard bounds, the rank-ordered all-gather of 40-byte
 records (equal and unequal row counts), and the orchestration of
 ShardedKLDStats with the per-rank row pass and reduction supplied by the
 oracle, so the statistics of the gathered shards must equal the oracle's
@@ -18,16 +18,16 @@ import oracle
 from logit_kl_divergence_b200 import rows_view, synth
 from logit_kl_divergence_b200.sharded import ShardedKLDStats, gather_records, shard_bounds
 
-RECORD = np.dtype([("kld", "<f8"), ("nll", "<f8"), ("amax_b", "<i4"), ("amax_q", "<i4"),
-                   ("flags", "<u4"), ("reserved", "<u4")])
-assert RECORD.itemsize == 32
+RECORD = np.dtype([("kld", "<f8"), ("nll", "<f8"), ("nll_base", "<f8"), ("amax_b", "<i4"),
+                   ("amax_q", "<i4"), ("flags", "<u4"), ("reserved", "<u4")])
+assert RECORD.itemsize == 40
 
 
 def _pack(r: dict) -> np.ndarray:
     a = np.zeros(r["kld"].shape[0], dtype=RECORD)
-    for k in ("kld", "nll", "amax_b", "amax_q", "flags"):
+    for k in ("kld", "nll", "nll_base", "amax_b", "amax_q", "flags"):
         a[k] = r[k]
-    return a.view(np.uint8).reshape(-1, 32)
+    return a.view(np.uint8).reshape(-1, 40)
 
 
 class OracleStats:
@@ -77,9 +77,9 @@ def _worker(rank, world, port, n_rows, with_tokens, errq):
         tok = w.token_ids if with_tokens else None
         lo, hi = shard_bounds(n_rows, world, rank)
         # rank-ordered gather of raw records
-        mine = torch.full((hi - lo, 32), rank, dtype=torch.uint8)
+        mine = torch.full((hi - lo, 40), rank, dtype=torch.uint8)
         got = gather_records(mine)
-        expect = torch.cat([torch.full((b - a, 32), r, dtype=torch.uint8)
+        expect = torch.cat([torch.full((b - a, 40), r, dtype=torch.uint8)
                             for r, (a, b) in enumerate(shard_bounds(n_rows, world, q) for q in range(world))])
         assert torch.equal(got, expect)
         # the whole orchestration, oracle-backed
