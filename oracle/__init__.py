@@ -110,6 +110,11 @@ def _load():
                 ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
                 ctypes.c_int64, ctypes.c_int, ctypes.POINTER(_Result),
             ]
+            lib.oracle_grad.restype = ctypes.c_int
+            lib.oracle_grad.argtypes = [
+                ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64,
+                ctypes.c_int, ctypes.c_double, ctypes.c_void_p,
+            ]
             lib.oracle_percentile_sorted.restype = ctypes.c_double
             lib.oracle_percentile_sorted.argtypes = [
                 ctypes.c_void_p, ctypes.c_int64, ctypes.c_double,
@@ -200,6 +205,21 @@ def run(base, quant, token_ids=None, dtype: int = F32, nthreads: int = 1):
     """Per-row arrays and summary statistics for one [N, V] pair."""
     r = rows(base, quant, token_ids, dtype, nthreads)
     return r, reduce(r, token_ids is not None)
+
+
+def grad(base, quant, dtype: int = F32, scale: float = 1.0) -> np.ndarray:
+    """[N, V] float64 gradient of KL(P_base || P_quant) with respect to the
+    quant logits: scale * (softmax(q) - softmax(b)); zero on excluded rows."""
+    lib = _load()
+    b = _as_logits(base, dtype)
+    q = _as_logits(quant, dtype)
+    if b.shape != q.shape:
+        raise ValueError("base and quant shapes differ")
+    N, V = b.shape
+    out = np.empty((N, V), np.float64)
+    if lib.oracle_grad(b.ctypes.data, q.ctypes.data, N, V, dtype, float(scale), out.ctypes.data) != 0:
+        raise ValueError("oracle_grad rejected its arguments")
+    return out
 
 
 def percentile_sorted(x, p: float) -> float:

@@ -227,6 +227,42 @@ extern "C" int oracle_rows(const void* base, const void* quant,
   return 0;
 }
 
+extern "C" int oracle_grad(const void* base, const void* quant, int64_t N,
+                           int64_t V, int dtype, double scale, double* grad) {
+  if (!base || !quant || !grad || N < 0 || V < 1 || V > 0x7fffffffLL) return -1;
+  if (dtype != ORACLE_F32 && dtype != ORACLE_BF16 && dtype != ORACLE_F16)
+    return -1;
+  std::vector<double> b((size_t)V), q((size_t)V);
+  for (int64_t r = 0; r < N; ++r) {
+    load_row(base, dtype, r, V, b.data());
+    load_row(quant, dtype, r, V, q.data());
+    double* g = grad + r * V;
+    /* Excluded rows (NaN/+inf anywhere, or a row of -inf) add nothing to
+     * the mean over valid rows, so their gradient is zero. */
+    bool excluded = false;
+    double m_b = -kInf, m_q = -kInf;
+    for (int64_t j = 0; j < V; ++j) {
+      if (std::isnan(b[j]) || std::isnan(q[j]) || b[j] == kInf || q[j] == kInf)
+        excluded = true;
+      if (b[j] > m_b) m_b = b[j];
+      if (q[j] > m_q) m_q = q[j];
+    }
+    if (excluded || m_b == -kInf || m_q == -kInf) {
+      for (int64_t j = 0; j < V; ++j) g[j] = 0.0;
+      continue;
+    }
+    /* log-sum-exp of both rows, plain left-to-right sums */
+    double zb = 0.0, zq = 0.0;
+    for (int64_t j = 0; j < V; ++j) zb += std::exp(b[j] - m_b);
+    for (int64_t j = 0; j < V; ++j) zq += std::exp(q[j] - m_q);
+    const double lse_b = m_b + std::log(zb);
+    const double lse_q = m_q + std::log(zq);
+    for (int64_t j = 0; j < V; ++j)
+      g[j] = scale * (std::exp(q[j] - lse_q) - std::exp(b[j] - lse_b));
+  }
+  return 0;
+}
+
 extern "C" double oracle_percentile_sorted(const double* x, int64_t n,
                                            double p) {
   if (n <= 0) return kNaN;

@@ -91,6 +91,15 @@ int oracle_reduce(const double* kld, const double* nll, const double* nll_base,
                   const uint32_t* flags, int64_t N, int has_nll,
                   oracle_result_t* out);
 
+/* Gradient of KL(P_base || P_quant) with respect to the quant logits, per
+ * row i and entry j: grad[i][j] = scale * (P_quant_j - P_base_j), i.e.
+ * softmax(q_i) - softmax(b_i) (the objective minimised in
+ * "Mistral-Small-4-119B-2603 GSQ-RCO IQ3_S GGUF", "How it was made", step 7).
+ * Rows that are NONFINITE or EMPTY (excluded from the statistics) get zeros.
+ * Returns 0, or -1 on bad args. */
+int oracle_grad(const void* base, const void* quant, int64_t N, int64_t V,
+                int dtype, double scale, double* grad);
+
 /* Type-7 percentile of an ascending array x[0..n): pos = p*(n-1). */
 double oracle_percentile_sorted(const double* x, int64_t n, double p);
 

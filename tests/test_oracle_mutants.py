@@ -44,6 +44,10 @@ MUTANTS = {
                         "const double dp = std::exp(-nll_base[i]) - std::exp(-nll[i]);"),
     "rms_dp_without_root": ("out->rms_dp = std::sqrt(sum_dp2 / (double)n_nll);",
                             "out->rms_dp = sum_dp2 / (double)n_nll;"),
+    "grad_sign_flipped": ("g[j] = scale * (std::exp(q[j] - lse_q) - std::exp(b[j] - lse_b));",
+                          "g[j] = scale * (std::exp(b[j] - lse_b) - std::exp(q[j] - lse_q));"),
+    "grad_quant_normaliser_from_base": ("g[j] = scale * (std::exp(q[j] - lse_q) - std::exp(b[j] - lse_b));",
+                                        "g[j] = scale * (std::exp(q[j] - lse_b) - std::exp(b[j] - lse_b));"),
     "ppl_ratio_inverted": ("out->ln_ppl_ratio = out->mean_nll - out->mean_nll_base;",
                            "out->ln_ppl_ratio = out->mean_nll_base - out->mean_nll;"),
 }

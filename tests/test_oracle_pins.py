@@ -471,3 +471,68 @@ def test_threaded_rows_are_bit_identical():
     for k in r1:
         assert np.array_equal(r1[k], r4[k])
     assert s1 == s4
+
+
+# ---------------------------------------------------------------- KL gradient
+
+def _brute_kl64(b_row, q_row):
+    """KL in fp64 straight from sum p log(p/r), no max subtraction."""
+    eb = [math.exp(x) for x in b_row]
+    eq = [math.exp(x) for x in q_row]
+    sb, sq = math.fsum(eb), math.fsum(eq)
+    return math.fsum((x / sb) * math.log((x / sb) / (y / sq)) for x, y in zip(eb, eq) if x > 0)
+
+
+def test_grad_matches_central_differences_of_the_kl():
+    V = 6
+    b = RNG.normal(0, 1, size=(4, V)).astype(np.float32)
+    q = RNG.normal(0, 1, size=(4, V)).astype(np.float32)
+    g = oracle.grad(b, q)
+    h = 1e-5
+    for i in range(4):
+        bi = [float(x) for x in b[i]]
+        for j in range(V):
+            up = [float(x) for x in q[i]]
+            dn = list(up)
+            up[j] += h
+            dn[j] -= h
+            fd = (_brute_kl64(bi, up) - _brute_kl64(bi, dn)) / (2 * h)
+            assert abs(g[i, j] - fd) < 1e-8, (i, j, g[i, j], fd)
+
+
+def test_grad_rows_sum_to_zero_and_scale_linearly():
+    b = RNG.normal(0, 2, size=(5, 2000)).astype(np.float32)
+    q = (b + RNG.normal(0, 0.3, size=(5, 2000))).astype(np.float32)
+    g1 = oracle.grad(b, q)
+    assert np.all(np.abs(g1.sum(axis=1)) < 1e-14)
+    g3 = oracle.grad(b, q, scale=-0.25)
+    np.testing.assert_allclose(g3, -0.25 * g1, rtol=1e-15, atol=0)
+
+
+def test_grad_closed_forms():
+    V = 40
+    # identical rows: exactly zero
+    b = RNG.normal(0, 1, size=(2, V)).astype(np.float32)
+    assert np.all(oracle.grad(b, b.copy()) == 0.0)
+    # one-hot base (entry 7) against a uniform quant: 1/V - [j == 7]
+    b1 = np.full((1, V), NEG_INF, np.float32)
+    b1[0, 7] = 0.0
+    q1 = np.zeros((1, V), np.float32)
+    want = np.full(V, 1.0 / V)
+    want[7] -= 1.0
+    np.testing.assert_allclose(oracle.grad(b1, q1)[0], want, rtol=0, atol=1e-16)
+
+
+def test_grad_of_excluded_rows_is_zero_and_masks_are_zero():
+    V = 10
+    b = RNG.normal(0, 1, size=(3, V)).astype(np.float32)
+    q = RNG.normal(0, 1, size=(3, V)).astype(np.float32)
+    b[0, 3] = np.nan
+    q[1, :] = NEG_INF
+    b[2, 4] = NEG_INF      # P_base = 0 there
+    q[2, 5] = NEG_INF      # P_quant = 0 there
+    g = oracle.grad(b, q)
+    assert np.all(g[0] == 0.0) and np.all(g[1] == 0.0)
+    e = np.exp(q[2].astype(np.float64) - q[2].max())
+    r = e / e.sum()
+    assert g[2, 5] < 0 and abs(g[2, 4] - r[4]) < 1e-16
