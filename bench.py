@@ -307,6 +307,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-variants", action="store_true")
     ap.add_argument("--no-split-row", action="store_true")
+    ap.add_argument("--no-grad", action="store_true")
     ap.add_argument("--split-calls", type=int, default=SPLIT_CALLS,
                     help="profiling only: fewer calls per size in the split-row section")
     ap.add_argument("--rows", type=int, default=None,
@@ -448,6 +449,38 @@ def main():
         torch.cuda.empty_cache()
         w = synth.make(name, device=dev, seed=synth.WORKLOADS[name][4])
 
+    # Gradient of the KL w.r.t. the quant logits (row pass + reduction +
+    # gradient pass writing fp32 [N, V]) on the same context.
+    grad = None
+    if world == 1 and not args.no_grad:
+        gout = torch.empty_like(w.base)
+        st.set_timing(True)
+        for _ in range(3):
+            st.run_grad(w.base, w.quant, w.token_ids, out=gout, scale=1.0 / N)
+            st.result()
+        torch.cuda.synchronize(dev)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        gms = []
+        gsteps = max(3, min(args.steps, 10))
+        a.record(stream)
+        for _ in range(gsteps):
+            st.run_grad(w.base, w.quant, w.token_ids, out=gout, scale=1.0 / N)
+            st.result()
+            gms.append(st.grad_timing())
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        step_ms = a.elapsed_time(b) / gsteps
+        kms = sum(gms) / len(gms)
+        gbytes = 3 * N * V * eb  # reads b and q, writes the fp32 gradient
+        grad = {"workload": name, "grad_dtype": "f32", "steps": gsteps, "ms_per_step": step_ms,
+                "value": N / (step_ms / 1000.0), "unit": "rows/s",
+                "grad_pass_ms": kms, "grad_pass_gbs": gbytes / (kms / 1000.0) / 1e9,
+                "grad_pass_frac": gbytes / (kms / 1000.0) / 1e9 / peak,
+                "algorithmic_bytes_per_grad_launch": gbytes,
+                "step_gbs": (gbytes + in_bytes) / (step_ms / 1000.0) / 1e9}
+        del gout
+        torch.cuda.empty_cache()
+
     # End to end through the public host-memory entry point: pinned host
     # buffers in, the result struct out, copies inside the timed region.
     e2e = None
@@ -495,7 +528,7 @@ def main():
             "gbs": in_bytes * world / (ms_per_step / 1000.0) / 1e9,
             "mean_kld": res["mean_kld"], "top1_agree_pct": res["top1_agree_pct"], "ppl": res["ppl"],
             "ppl_base": res["ppl_base"], "rms_dp": res["rms_dp"], "mean_dp": res["mean_dp"],
-            "variants": variants, "split_row": split_row,
+            "variants": variants, "split_row": split_row, "grad": grad,
         }
         if args.rows is not None or args.dtype != "f32" or args.split_calls != SPLIT_CALLS:
             line["config"]["override"] = {"rows": N, "dtype": args.dtype,

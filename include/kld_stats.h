@@ -224,6 +224,34 @@ kld_status_t kld_stats_run_host(kld_stats_t h, const void* base_host,
 kld_status_t kld_stats_set_split(kld_stats_t h, int cluster_ctas);
 
 /*
+ * The statistic plus its gradient with respect to the quant logits, the
+ * objective of end-to-end tuning ("Mistral-Small-4-119B-2603 GSQ-RCO IQ3_S
+ * GGUF", "How it was made", step 7: minimise KL(BF16 || quantized)):
+ *   grad[i][j] = scale * (softmax(q_i)_j - softmax(b_i)_j)
+ * (e.g. scale = 1/N for the gradient of the mean over N rows), zero on rows
+ * the statistics exclude (NONFINITE / EMPTY). Inputs as for kld_stats_run;
+ * grad: caller-owned DEVICE memory for N*V values of grad_dtype (KLD_F32,
+ * KLD_BF16 or KLD_F16; row-major [N, V], aligned to its element size; 16-byte
+ * aligned with V % 8 == 0 takes the vectorised path). Enqueues the row pass
+ * (which also keeps per-row normalisers in the handle), the reduction (the
+ * same result as kld_stats_run) and a second streaming pass that reads b and q
+ * again and writes grad. Asynchronous on `stream`; kld_stats_result() waits
+ * for the statistics, the stream for grad. Errors as kld_stats_run, plus
+ * KLD_ERR_DTYPE for an unknown grad_dtype and KLD_ERR_INVALID_ARG for a NULL
+ * or misaligned grad or a NaN scale.
+ */
+kld_status_t kld_stats_run_grad(kld_stats_t h, const void* base, const void* quant,
+                                const int32_t* token_ids, int64_t N, int64_t V,
+                                kld_dtype_t dtype, void* grad, kld_dtype_t grad_dtype,
+                                double scale, void* stream);
+
+/*
+ * Duration in milliseconds of the last kld_stats_run_grad's gradient pass
+ * (timing enabled by kld_stats_set_timing; waits for that run).
+ */
+kld_status_t kld_stats_grad_timing(kld_stats_t h, float* grad_ms);
+
+/*
  * Kernel timing of the next runs: when enabled, kld_stats_run records CUDA
  * events around its row pass and its reduction; kld_stats_timing() returns
  * the last run's durations in milliseconds (waits for that run).

@@ -116,6 +116,32 @@ class KLDStats:
                                      ctypes.c_void_p(_stream_ptr(stream, base.device)))
         _lib.check(st, "kld_stats_run")
 
+    def run_grad(self, base: torch.Tensor, quant: torch.Tensor, token_ids: torch.Tensor | None = None,
+                 out: torch.Tensor | None = None, scale: float = 1.0, grad_dtype=None,
+                 stream=None) -> torch.Tensor:
+        """The statistic (read it with :meth:`result`) plus the gradient of
+        KL(P_base || P_quant) with respect to the quant logits,
+        ``scale * (softmax(quant) - softmax(base))`` per row (zero on excluded
+        rows), written to ``out`` (allocated as ``grad_dtype``, default the
+        logits' dtype, when None). Asynchronous on the stream."""
+        _check_pair(base, quant, token_ids, True)
+        if out is None:
+            out = torch.empty(base.shape, dtype=grad_dtype or base.dtype, device=base.device)
+        if out.shape != base.shape or not out.is_contiguous() or out.device != base.device:
+            raise ValueError("out must be a contiguous [N, V] tensor on the logits' device")
+        st = self._lib.kld_stats_run_grad(self._h, _ptr(base), _ptr(quant), _ptr(token_ids),
+                                          base.shape[0], base.shape[1], dtype_code(base), _ptr(out),
+                                          dtype_code(out), float(scale),
+                                          ctypes.c_void_p(_stream_ptr(stream, base.device)))
+        _lib.check(st, "kld_stats_run_grad")
+        return out
+
+    def grad_timing(self) -> float:
+        """Milliseconds of the last run_grad's gradient pass (timing enabled)."""
+        ms = ctypes.c_float()
+        _lib.check(self._lib.kld_stats_grad_timing(self._h, ctypes.byref(ms)), "kld_stats_grad_timing")
+        return ms.value
+
     def run_host(self, base: torch.Tensor, quant: torch.Tensor, token_ids: torch.Tensor | None = None,
                  stream=None) -> None:
         """Same as :meth:`run` for host (preferably pinned) CPU tensors."""

@@ -108,6 +108,8 @@ SIGNATURES = {
     "kld_stats_run_host": (_ST, [_P, _P, _P, _P, _I64, _I64, _I32, _P]),
     "kld_stats_set_timing": (_ST, [_P, _I32]),
     "kld_stats_set_split": (_ST, [_P, _I32]),
+    "kld_stats_run_grad": (_ST, [_P, _P, _P, _P, _I64, _I64, _I32, _P, _I32, ctypes.c_double, _P]),
+    "kld_stats_grad_timing": (_ST, [_P, ctypes.POINTER(ctypes.c_float)]),
     "kld_stats_timing": (_ST, [_P, ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ctypes.c_float)]),
     "kld_plan": (_ST, [_I64, _I64, _I32, _I32, ctypes.POINTER(Plan)]),
     "kld_stats_run_static": (_ST, [_P, _P, _P, _I64, _I64, _I32, _P, _P]),

@@ -64,6 +64,8 @@ struct kld_stats_s {
   int64_t max_rows = 0;
   kld_row_t* rows = nullptr;
   void* split_mem = nullptr;  // split-row scratch: partials, then tickets
+  float4* norms = nullptr;    // per-row softmax normalisers for the gradient pass
+  bool grad_timing_valid = false;
   kld::SplitScratch split = {nullptr, nullptr, 0, kld::kDefaultClusterCtas};
   uint32_t* derr = nullptr;
   kld_result_t* hres = nullptr;      // pinned, mapped host memory
@@ -73,7 +75,7 @@ struct kld_stats_s {
   int64_t last_rows = 0;
   bool timing = false;
   bool timing_valid = false;
-  cudaEvent_t tev[3] = {nullptr, nullptr, nullptr};
+  cudaEvent_t tev[4] = {nullptr, nullptr, nullptr, nullptr};
   // host path
   cudaStream_t copy_stream = nullptr;
   cudaEvent_t copied[2] = {nullptr, nullptr};
@@ -101,8 +103,10 @@ kld_status_t check_inputs(const void* base, const void* quant, const int32_t* to
 }
 
 cudaError_t launch_rows(kld_stats_s* h, const void* base, const void* quant, const int32_t* tok,
-                        int64_t N, int64_t V, kld_dtype_t dtype, kld_row_t* rows, cudaStream_t s) {
-  return kld::launch_rows(base, quant, tok, N, V, dtype, rows, h->derr, h->sm_count, &h->split, s);
+                        int64_t N, int64_t V, kld_dtype_t dtype, kld_row_t* rows, cudaStream_t s,
+                        float4* norms = nullptr) {
+  return kld::launch_rows(base, quant, tok, N, V, dtype, rows, h->derr, h->sm_count, &h->split,
+                          norms, s);
 }
 
 kld_status_t enqueue_reduce(kld_stats_t h, const kld_row_t* rows, int64_t N, int has_nll,
@@ -190,6 +194,8 @@ kld_status_t kld_stats_create(kld_stats_t* out, int64_t max_rows, int device) {
     cudaError_t err;
     if ((err = cudaMalloc(&h->rows, sizeof(kld_row_t) * static_cast<size_t>(max_rows))) !=
         cudaSuccess) { st = cuda_fail(err, "cudaMalloc(rows)"); break; }
+    if ((err = cudaMalloc(&h->norms, sizeof(float4) * static_cast<size_t>(max_rows))) !=
+        cudaSuccess) { st = cuda_fail(err, "cudaMalloc(norms)"); break; }
     if ((err = cudaMalloc(&h->derr, sizeof(uint32_t))) != cudaSuccess) {
       st = cuda_fail(err, "cudaMalloc(error word)"); break; }
     if ((err = cudaMemset(h->derr, 0, sizeof(uint32_t))) != cudaSuccess) {
@@ -216,7 +222,7 @@ kld_status_t kld_stats_create(kld_stats_t* out, int64_t max_rows, int device) {
         cudaSuccess) { st = cuda_fail(err, "cudaHostGetDevicePointer"); break; }
     if ((err = cudaEventCreateWithFlags(&h->done, cudaEventDisableTiming)) != cudaSuccess) {
       st = cuda_fail(err, "cudaEventCreate"); break; }
-    for (int i = 0; i < 3 && st == KLD_OK; ++i)
+    for (int i = 0; i < 4 && st == KLD_OK; ++i)
       if ((err = cudaEventCreate(&h->tev[i])) != cudaSuccess) st = cuda_fail(err, "cudaEventCreate");
   } while (0);
   if (st != KLD_OK) {
@@ -239,13 +245,14 @@ void kld_stats_destroy(kld_stats_t h) {
     if (h->freed[i]) cudaEventDestroy(h->freed[i]);
   }
   if (h->copy_stream) cudaStreamDestroy(h->copy_stream);
-  for (int i = 0; i < 3; ++i)
+  for (int i = 0; i < 4; ++i)
     if (h->tev[i]) cudaEventDestroy(h->tev[i]);
   if (h->done) cudaEventDestroy(h->done);
   if (h->hres) cudaFreeHost(h->hres);
   if (h->derr) cudaFree(h->derr);
   if (h->rows) cudaFree(h->rows);
   if (h->split_mem) cudaFree(h->split_mem);
+  if (h->norms) cudaFree(h->norms);
   delete h;
 }
 
@@ -263,6 +270,7 @@ kld_status_t kld_stats_run_rows(kld_stats_t h, const void* base, const void* qua
   KLD_CUDA(launch_rows(h, base, quant, token_ids, N, V, dtype, rows_out ? rows_out : h->rows, s));
   if (!rows_out) h->last_rows = N;
   h->timing_valid = false;
+  h->grad_timing_valid = false;
   return KLD_OK;
 }
 
@@ -275,6 +283,7 @@ kld_status_t kld_stats_reduce(kld_stats_t h, const kld_row_t* rows_dev, int64_t 
   DeviceGuard guard(h->device);
   if (!guard.ok()) return cuda_fail(cudaGetLastError(), "cudaSetDevice");
   h->timing_valid = false;
+  h->grad_timing_valid = false;
   return enqueue_reduce(h, rows_dev ? rows_dev : h->rows, N, has_nll ? 1 : 0,
                         static_cast<cudaStream_t>(stream));
 }
@@ -290,11 +299,49 @@ kld_status_t kld_stats_run(kld_stats_t h, const void* base, const void* quant,
   if (!guard.ok()) return cuda_fail(cudaGetLastError(), "cudaSetDevice");
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   h->timing_valid = h->timing;
+  h->grad_timing_valid = false;
   if (h->timing) KLD_CUDA(cudaEventRecord(h->tev[0], s));
   KLD_CUDA(launch_rows(h, base, quant, token_ids, N, V, dtype, h->rows, s));
   if (h->timing) KLD_CUDA(cudaEventRecord(h->tev[1], s));
   h->last_rows = N;
   return enqueue_reduce(h, h->rows, N, token_ids != nullptr, s);
+}
+
+kld_status_t kld_stats_run_grad(kld_stats_t h, const void* base, const void* quant,
+                                const int32_t* token_ids, int64_t N, int64_t V,
+                                kld_dtype_t dtype, void* grad, kld_dtype_t grad_dtype,
+                                double scale, void* stream) {
+  if (!h) return KLD_ERR_INVALID_ARG;
+  kld_status_t st = check_inputs(base, quant, token_ids, N, V, dtype, true);
+  if (st != KLD_OK) return st;
+  if (!valid_dtype(grad_dtype)) return KLD_ERR_DTYPE;
+  if (!grad || (reinterpret_cast<uintptr_t>(grad) % kld::elem_bytes(grad_dtype))) return KLD_ERR_INVALID_ARG;
+  if (N > h->max_rows || !(scale == scale)) return KLD_ERR_INVALID_ARG;
+  DeviceGuard guard(h->device);
+  if (!guard.ok()) return cuda_fail(cudaGetLastError(), "cudaSetDevice");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  h->timing_valid = h->timing;
+  h->grad_timing_valid = h->timing;
+  if (h->timing) KLD_CUDA(cudaEventRecord(h->tev[0], s));
+  KLD_CUDA(launch_rows(h, base, quant, token_ids, N, V, dtype, h->rows, s, h->norms));
+  if (h->timing) KLD_CUDA(cudaEventRecord(h->tev[1], s));
+  h->last_rows = N;
+  st = enqueue_reduce(h, h->rows, N, token_ids != nullptr, s);
+  if (st != KLD_OK) return st;
+  KLD_CUDA(kld::launch_grad(base, quant, h->norms, N, V, dtype, grad, grad_dtype,
+                            static_cast<float>(scale), h->sm_count, s));
+  if (h->timing) KLD_CUDA(cudaEventRecord(h->tev[3], s));
+  return KLD_OK;
+}
+
+kld_status_t kld_stats_grad_timing(kld_stats_t h, float* grad_ms) {
+  if (!h || !grad_ms) return KLD_ERR_INVALID_ARG;
+  if (!h->grad_timing_valid || !h->has_result) return KLD_ERR_NOT_READY;
+  DeviceGuard guard(h->device);
+  if (!guard.ok()) return cuda_fail(cudaGetLastError(), "cudaSetDevice");
+  KLD_CUDA(cudaEventSynchronize(h->tev[3]));
+  KLD_CUDA(cudaEventElapsedTime(grad_ms, h->tev[2], h->tev[3]));
+  return KLD_OK;
 }
 
 kld_status_t kld_stats_result(kld_stats_t h, kld_result_t* out) {
@@ -331,6 +378,7 @@ kld_status_t kld_stats_set_timing(kld_stats_t h, int enable) {
   if (!h) return KLD_ERR_INVALID_ARG;
   h->timing = enable != 0;
   h->timing_valid = false;
+  h->grad_timing_valid = false;
   return KLD_OK;
 }
 
@@ -385,6 +433,7 @@ kld_status_t kld_stats_run_host(kld_stats_t h, const void* base_host, const void
   for (int i = 0; i < 2; ++i) KLD_CUDA(cudaEventRecord(h->freed[i], s));
 
   h->timing_valid = false;
+  h->grad_timing_valid = false;
   const char* hb = static_cast<const char*>(base_host);
   const char* hq = static_cast<const char*>(quant_host);
   const int64_t nchunks = (N + chunk - 1) / chunk;

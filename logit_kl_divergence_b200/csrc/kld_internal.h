@@ -56,10 +56,13 @@ inline int elem_bytes(kld_dtype_t dt) { return dt == KLD_F32 ? 4 : 2; }
 // the launch error.
 // Row pass. With split == nullptr every CTA handles whole rows; otherwise
 // few-row launches spread each row over clusters of CTAs (see RowPlan).
+// norms (nullable): per-row normalisers {Fb, mb, Fq, mq} for the gradient
+// pass (see launch_grad).
 cudaError_t launch_rows(const void* base, const void* quant,
                         const int32_t* token_ids, int64_t N, int64_t V,
                         kld_dtype_t dtype, kld_row_t* rows, uint32_t* derr,
-                        int sm_count, const SplitScratch* split, cudaStream_t stream);
+                        int sm_count, const SplitScratch* split, float4* norms,
+                        cudaStream_t stream);
 
 // Launch shape of the row pass: parts_per_row = 1 (whole rows, persistent
 // grid) or > 1 (split rows: grid = N * parts_per_row, clusters of
@@ -74,6 +77,13 @@ struct RowPlan {
 // takes as many clusters (<= 32) as still fit in that wave.
 RowPlan plan_rows(int64_t N, int sm_count, const int fit[4], int max_cluster_ctas);
 cudaError_t prepare_rows_kernels();  // per-device attribute setup
+
+// Gradient pass: grad[i][j] = scale * (softmax(q_i)_j - softmax(b_i)_j)
+// from the per-row normalisers of the row pass (zero on excluded rows);
+// grad in grad_dtype, [N, V] row-major.
+cudaError_t launch_grad(const void* base, const void* quant, const float4* norms, int64_t N,
+                        int64_t V, kld_dtype_t dtype, void* grad, kld_dtype_t grad_dtype,
+                        float scale, int sm_count, cudaStream_t stream);
 
 cudaError_t launch_reduce(const kld_row_t* rows, int64_t N, int has_nll,
                           uint32_t* derr, kld_result_t* out,

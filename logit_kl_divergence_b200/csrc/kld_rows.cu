@@ -852,6 +852,25 @@ __device__ kld_row_t finalize_row(const MPart& m, bool has_tok, bool tok_ok, flo
   return rec;
 }
 
+// Per-row normalisers for the gradient pass, from the merged partial:
+// softmax(lambda*b)_j = 2^(b_j*L - Fb) * mb and softmax(lambda*q)_j =
+// 2^(q_j*L - Fq) * mq, with integer frames Fb = floor(log2 of the base sum),
+// Fq likewise, and mb, mq in (0.5, 1] (so the exponents stay small near the
+// row maximum and every value keeps fp32 accuracy). NaN frames mark rows
+// excluded from the statistics (their gradient is zero).
+__device__ float4 row_norms(const MPart& m, const kld_row_t& rec) {
+  if (rec.flags & (KLD_ROW_NONFINITE | KLD_ROW_EMPTY)) {
+    const float nan = __int_as_float(0x7fc00000);
+    return make_float4(nan, 0.f, nan, 0.f);
+  }
+  const double cb = log2(m.Sb) + static_cast<double>(m.Cb);
+  const double cq = log2(m.B + m.Sb) + static_cast<double>(m.Cb) -
+                    static_cast<double>(m.K) * kLog2eD;
+  const double fb = floor(cb), fq = floor(cq);
+  return make_float4(static_cast<float>(fb), static_cast<float>(exp2(fb - cb)),
+                     static_cast<float>(fq), static_cast<float>(exp2(fq - cq)));
+}
+
 __device__ __forceinline__ uint32_t cluster_ctarank() {
   uint32_t r;
   asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
@@ -873,7 +892,7 @@ __global__ void __launch_bounds__(kRowThreads, 1)
     kld_rows_kernel(const void* __restrict__ base, const void* __restrict__ quant,
                     const int32_t* __restrict__ tok, int64_t N, int64_t V,
                     kld_row_t* __restrict__ rows, uint32_t* __restrict__ derr, int P,
-                    MPart* __restrict__ gparts, unsigned* __restrict__ tickets) {
+                    MPart* __restrict__ gparts, unsigned* __restrict__ tickets, float4* __restrict__ norms) {
   constexpr int EB = Elem<DT>::kBytes;
   constexpr int E = Elem<DT>::kPerVec;
   constexpr int kStageElems = kStageBytes / EB;
@@ -1217,7 +1236,10 @@ __global__ void __launch_bounds__(kRowThreads, 1)
       if (P == 1) {
         gather_token();
         const kld_row_t rec = finalize_row(m, tok != nullptr, tok_ok, q_tok, b_tok);
-        if (lane == 0) rows[r] = rec;
+        if (lane == 0) {
+          rows[r] = rec;
+          if (norms != nullptr) norms[r] = row_norms(m, rec);
+        }
         continue;
       }
 
@@ -1288,7 +1310,10 @@ __global__ void __launch_bounds__(kRowThreads, 1)
       if (C == 1) {
         gather_token();
         const kld_row_t rec = finalize_row(cm, tok != nullptr, tok_ok, q_tok, b_tok);
-        if (lane == 0) rows[r] = rec;
+        if (lane == 0) {
+          rows[r] = rec;
+          if (norms != nullptr) norms[r] = row_norms(cm, rec);
+        }
         continue;
       }
       const int cid = it.k / static_cast<int>(G);
@@ -1322,6 +1347,7 @@ __global__ void __launch_bounds__(kRowThreads, 1)
       const kld_row_t rec = finalize_row(fm, tok != nullptr, tok_ok, q_tok, b_tok);
       if (lane == 0) {
         rows[r] = rec;
+        if (norms != nullptr) norms[r] = row_norms(fm, rec);
         tickets[r] = 0u;  // ready for the next launch
       }
     }
@@ -1359,7 +1385,7 @@ int max_active_clusters(int cluster_ctas) {
 template <int DT>
 cudaError_t launch_typed(const void* base, const void* quant, const int32_t* tok, int64_t N,
                          int64_t V, kld_row_t* rows, uint32_t* derr, const RowPlan& pl,
-                         const SplitScratch* split, cudaStream_t stream) {
+                         const SplitScratch* split, float4* norms, cudaStream_t stream) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(pl.grid));
   cfg.blockDim = dim3(kRowThreads);
@@ -1375,7 +1401,7 @@ cudaError_t launch_typed(const void* base, const void* quant, const int32_t* tok
   MPart* gp = split ? static_cast<MPart*>(split->parts) : nullptr;
   unsigned* tk = split ? split->tickets : nullptr;
   return cudaLaunchKernelEx(&cfg, kld_rows_kernel<DT>, base, quant, tok, N, V, rows, derr,
-                            pl.parts_per_row, gp, tk);
+                            pl.parts_per_row, gp, tk, norms);
 }
 
 }  // namespace
@@ -1438,7 +1464,8 @@ int active_clusters(kld_dtype_t dtype, int lg) {
 
 cudaError_t launch_rows(const void* base, const void* quant, const int32_t* token_ids, int64_t N,
                         int64_t V, kld_dtype_t dtype, kld_row_t* rows, uint32_t* derr,
-                        int sm_count, const SplitScratch* split, cudaStream_t stream) {
+                        int sm_count, const SplitScratch* split, float4* norms,
+                        cudaStream_t stream) {
   RowPlan pl = plan_rows(N, sm_count, nullptr, 0);
   if (split != nullptr && N * 2 <= sm_count && split->max_cluster_ctas >= 1) {
     int fit[4] = {0, 0, 0, 0};
@@ -1450,11 +1477,14 @@ cudaError_t launch_rows(const void* base, const void* quant, const int32_t* toke
   }
   switch (dtype) {
     case KLD_F32:
-      return launch_typed<KLD_F32>(base, quant, token_ids, N, V, rows, derr, pl, split, stream);
+      return launch_typed<KLD_F32>(base, quant, token_ids, N, V, rows, derr, pl, split, norms,
+                                 stream);
     case KLD_BF16:
-      return launch_typed<KLD_BF16>(base, quant, token_ids, N, V, rows, derr, pl, split, stream);
+      return launch_typed<KLD_BF16>(base, quant, token_ids, N, V, rows, derr, pl, split, norms,
+                                 stream);
     case KLD_F16:
-      return launch_typed<KLD_F16>(base, quant, token_ids, N, V, rows, derr, pl, split, stream);
+      return launch_typed<KLD_F16>(base, quant, token_ids, N, V, rows, derr, pl, split, norms,
+                                 stream);
   }
   return cudaErrorInvalidValue;
 }

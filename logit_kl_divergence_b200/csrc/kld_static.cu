@@ -113,7 +113,8 @@ extern "C" kld_status_t kld_stats_run_static(const void* base, const void* quant
   cudaError_t e = cudaMemsetAsync(derr, 0, sizeof(uint32_t), s);
   if (e != cudaSuccess) return fail_cuda(e);
   // Whole-row mode only: split rows would need scratch beyond the fixed array.
-  e = kld::launch_rows(base, quant, token_ids, N, V, dtype, rows, derr, dev.sm_count, nullptr, s);
+  e = kld::launch_rows(base, quant, token_ids, N, V, dtype, rows, derr, dev.sm_count, nullptr,
+                       nullptr, s);
   if (e != cudaSuccess) return fail_cuda(e);
   e = kld::launch_reduce(rows, N, token_ids != nullptr, derr, result_dev, s);
   if (e != cudaSuccess) return fail_cuda(e);
