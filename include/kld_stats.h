@@ -246,6 +246,31 @@ kld_status_t kld_stats_run_grad(kld_stats_t h, const void* base, const void* qua
                                 double scale, void* stream);
 
 /*
+ * Vocabulary-sharded rows (a tensor-parallel lm_head leaves each GPU with a
+ * column slice of the logits). kld_stats_run_partials takes this GPU's slice:
+ * [N, V] row-major logits holding columns [col_offset, col_offset + V) of a
+ * vocabulary of V_total entries (same pointer rules as kld_stats_run), and
+ * writes one 64-byte partial per row to parts_out (caller-owned DEVICE
+ * memory of N * KLD_PARTIAL_BYTES bytes, 16-byte aligned): the slice's
+ * maxima with their lowest global indices, its softmax sums in an exact
+ * frame, flags, and the token's two logits when token_ids[r] falls in the
+ * slice. Gather every slice's partials (any transport; [G][N] in slice
+ * order, G <= 32, the slices covering [0, V_total) without overlap) and
+ * call kld_stats_merge_partials: it merges each row's G partials into the
+ * handle's records (token ids checked against V_total) and enqueues the
+ * reduction; kld_stats_result() then returns the statistics of the full
+ * rows. Both are asynchronous on `stream`. Errors: KLD_ERR_INVALID_ARG for
+ * bad sizes, offsets or alignment, else as kld_stats_run.
+ */
+#define KLD_PARTIAL_BYTES 64
+kld_status_t kld_stats_run_partials(kld_stats_t h, const void* base, const void* quant,
+                                    const int32_t* token_ids, int64_t N, int64_t V,
+                                    int64_t col_offset, int64_t V_total, kld_dtype_t dtype,
+                                    void* parts_out, void* stream);
+kld_status_t kld_stats_merge_partials(kld_stats_t h, const void* parts, int G, int64_t N,
+                                      const int32_t* token_ids, int64_t V_total, void* stream);
+
+/*
  * Duration in milliseconds of the last kld_stats_run_grad's gradient pass
  * (timing enabled by kld_stats_set_timing; waits for that run).
  */

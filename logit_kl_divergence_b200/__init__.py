@@ -23,6 +23,7 @@ __all__ = ["KLDStats", "kld_stats", "run_static", "result_from_bytes", "plan", "
            "ROW_RECORD_BYTES"]
 
 ROW_RECORD_BYTES = 40
+PARTIAL_BYTES = 64
 
 _DTYPES = {torch.float32: KLD_F32, torch.bfloat16: KLD_BF16, torch.float16: KLD_F16}
 
@@ -141,6 +142,45 @@ class KLDStats:
         ms = ctypes.c_float()
         _lib.check(self._lib.kld_stats_grad_timing(self._h, ctypes.byref(ms)), "kld_stats_grad_timing")
         return ms.value
+
+    def run_partials(self, base: torch.Tensor, quant: torch.Tensor, token_ids: torch.Tensor | None,
+                     col_offset: int, v_total: int, out: torch.Tensor | None = None,
+                     stream=None) -> torch.Tensor:
+        """This GPU's vocabulary slice (columns [col_offset, col_offset + V) of
+        a V_total-wide vocabulary): one 64-byte partial per row, returned as
+        (or written to) an [N, 64] uint8 CUDA tensor."""
+        _check_pair(base, quant, token_ids, True)
+        n = base.shape[0]
+        if out is None:
+            out = torch.empty((n, PARTIAL_BYTES), dtype=torch.uint8, device=base.device)
+        if out.dtype != torch.uint8 or out.numel() < n * PARTIAL_BYTES or not out.is_contiguous():
+            raise ValueError("out must be a contiguous uint8 tensor of N*64 bytes")
+        st = self._lib.kld_stats_run_partials(self._h, _ptr(base), _ptr(quant), _ptr(token_ids), n,
+                                              base.shape[1], int(col_offset), int(v_total),
+                                              dtype_code(base), _ptr(out),
+                                              ctypes.c_void_p(_stream_ptr(stream, base.device)))
+        _lib.check(st, "kld_stats_run_partials")
+        return out
+
+    def merge_partials(self, parts: torch.Tensor, token_ids: torch.Tensor | None, v_total: int,
+                       stream=None) -> None:
+        """Merge [G, N, 64] (or [G*N, 64]) slice partials, in slice order,
+        into this handle's records and reduce them (read with :meth:`result`)."""
+        if parts.dtype != torch.uint8 or not parts.is_cuda or not parts.is_contiguous():
+            raise ValueError("parts must be a contiguous uint8 CUDA tensor")
+        p = parts.reshape(-1, PARTIAL_BYTES)
+        if token_ids is not None:
+            n = token_ids.shape[0]
+        elif parts.dim() == 3:
+            n = parts.shape[1]
+        else:
+            raise ValueError("give [G, N, 64] parts or the token ids")
+        if p.shape[0] % n:
+            raise ValueError("parts must hold G * N partials")
+        st = self._lib.kld_stats_merge_partials(self._h, _ptr(p), p.shape[0] // n, n, _ptr(token_ids),
+                                                int(v_total),
+                                                ctypes.c_void_p(_stream_ptr(stream, parts.device)))
+        _lib.check(st, "kld_stats_merge_partials")
 
     def run_host(self, base: torch.Tensor, quant: torch.Tensor, token_ids: torch.Tensor | None = None,
                  stream=None) -> None:

@@ -334,6 +334,41 @@ kld_status_t kld_stats_run_grad(kld_stats_t h, const void* base, const void* qua
   return KLD_OK;
 }
 
+kld_status_t kld_stats_run_partials(kld_stats_t h, const void* base, const void* quant,
+                                    const int32_t* token_ids, int64_t N, int64_t V,
+                                    int64_t col_offset, int64_t V_total, kld_dtype_t dtype,
+                                    void* parts_out, void* stream) {
+  if (!h) return KLD_ERR_INVALID_ARG;
+  kld_status_t st = check_inputs(base, quant, token_ids, N, V, dtype, true);
+  if (st != KLD_OK) return st;
+  if (!parts_out || (reinterpret_cast<uintptr_t>(parts_out) & 15u)) return KLD_ERR_INVALID_ARG;
+  if (col_offset < 0 || V_total > INT32_MAX || col_offset + V > V_total) return KLD_ERR_INVALID_ARG;
+  DeviceGuard guard(h->device);
+  if (!guard.ok()) return cuda_fail(cudaGetLastError(), "cudaSetDevice");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  h->timing_valid = false;
+  h->grad_timing_valid = false;
+  KLD_CUDA(kld::launch_rows(base, quant, token_ids, N, V, dtype, h->rows, h->derr, h->sm_count,
+                            &h->split, nullptr, s, parts_out, col_offset));
+  return KLD_OK;
+}
+
+kld_status_t kld_stats_merge_partials(kld_stats_t h, const void* parts, int G, int64_t N,
+                                      const int32_t* token_ids, int64_t V_total, void* stream) {
+  if (!h || !parts || G < 1 || G > 32 || N < 1 || N > h->max_rows) return KLD_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(parts) & 15u) || V_total < 1 || V_total > INT32_MAX)
+    return KLD_ERR_INVALID_ARG;
+  if (token_ids && (reinterpret_cast<uintptr_t>(token_ids) & 3u)) return KLD_ERR_INVALID_ARG;
+  DeviceGuard guard(h->device);
+  if (!guard.ok()) return cuda_fail(cudaGetLastError(), "cudaSetDevice");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  h->timing_valid = false;
+  h->grad_timing_valid = false;
+  KLD_CUDA(kld::launch_merge(parts, G, N, token_ids, V_total, h->rows, s));
+  h->last_rows = N;
+  return enqueue_reduce(h, h->rows, N, token_ids != nullptr, s);
+}
+
 kld_status_t kld_stats_grad_timing(kld_stats_t h, float* grad_ms) {
   if (!h || !grad_ms) return KLD_ERR_INVALID_ARG;
   if (!h->grad_timing_valid || !h->has_result) return KLD_ERR_NOT_READY;

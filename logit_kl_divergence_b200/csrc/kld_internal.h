@@ -58,11 +58,22 @@ inline int elem_bytes(kld_dtype_t dt) { return dt == KLD_F32 ? 4 : 2; }
 // few-row launches spread each row over clusters of CTAs (see RowPlan).
 // norms (nullable): per-row normalisers {Fb, mb, Fq, mq} for the gradient
 // pass (see launch_grad).
+// part_out (nullable): vocabulary-slice mode, the row is columns
+// [col_offset, col_offset + V) of a wider vocabulary and each row's merged
+// 64-byte partial goes to part_out[r] instead of a record (see
+// launch_merge).
 cudaError_t launch_rows(const void* base, const void* quant,
                         const int32_t* token_ids, int64_t N, int64_t V,
                         kld_dtype_t dtype, kld_row_t* rows, uint32_t* derr,
                         int sm_count, const SplitScratch* split, float4* norms,
-                        cudaStream_t stream);
+                        cudaStream_t stream, void* part_out = nullptr,
+                        int64_t col_offset = 0);
+
+// Records from the G vocabulary-slice partials of each row (parts: [G][N]
+// 64-byte partials, rank/slice order), tokens checked against V_total.
+constexpr int kPartialBytes = 64;
+cudaError_t launch_merge(const void* parts, int G, int64_t N, const int32_t* token_ids,
+                         int64_t V_total, kld_row_t* rows, cudaStream_t stream);
 
 // Launch shape of the row pass: parts_per_row = 1 (whole rows, persistent
 // grid) or > 1 (split rows: grid = N * parts_per_row, clusters of

@@ -401,7 +401,8 @@ struct __align__(16) MPart {
 };
 constexpr unsigned kPartNonfinite = 1u, kPartInfKl = 2u;
 constexpr unsigned kPartFailed = 4u;  // a bounded wait gave up on this part
-static_assert(sizeof(MPart) == kSplitPartBytes, "MPart layout");
+constexpr unsigned kPartHasTok = 8u;  // vocabulary slice holding the token: pad2 = (q, b) at it
+static_assert(sizeof(MPart) == kSplitPartBytes && sizeof(MPart) == kPartialBytes, "MPart layout");
 
 struct Ctrl {
   unsigned long long full[kStages];
@@ -728,7 +729,7 @@ __device__ __forceinline__ void part_words(const MPart& m, unsigned long long (&
   w[4] = static_cast<unsigned long long>(__double_as_longlong(m.B));
   w[5] = pack2(static_cast<unsigned>(m.amax_b), static_cast<unsigned>(m.amax_q));
   w[6] = pack2(m.flags, 0u);
-  w[7] = 0ull;
+  w[7] = m.pad2;  // a vocabulary slice's token logits (kPartHasTok)
 }
 __device__ __forceinline__ MPart part_from_words(const unsigned long long (&w)[8]) {
   MPart m;
@@ -743,7 +744,7 @@ __device__ __forceinline__ MPart part_from_words(const unsigned long long (&w)[8
   m.amax_q = static_cast<int>(static_cast<unsigned>(w[5] >> 32));
   m.flags = static_cast<unsigned>(w[6]);
   m.pad = 0u;
-  m.pad2 = 0ull;
+  m.pad2 = w[7];
   return m;
 }
 
@@ -892,7 +893,8 @@ __global__ void __launch_bounds__(kRowThreads, 1)
     kld_rows_kernel(const void* __restrict__ base, const void* __restrict__ quant,
                     const int32_t* __restrict__ tok, int64_t N, int64_t V,
                     kld_row_t* __restrict__ rows, uint32_t* __restrict__ derr, int P,
-                    MPart* __restrict__ gparts, unsigned* __restrict__ tickets, float4* __restrict__ norms) {
+                    MPart* __restrict__ gparts, unsigned* __restrict__ tickets, float4* __restrict__ norms,
+                    MPart* __restrict__ part_out, int64_t col0) {
   constexpr int EB = Elem<DT>::kBytes;
   constexpr int E = Elem<DT>::kPerVec;
   constexpr int kStageElems = kStageBytes / EB;
@@ -1233,6 +1235,30 @@ __global__ void __launch_bounds__(kRowThreads, 1)
         }
       };
 
+      if (P == 1 && part_out != nullptr) {
+        // Vocabulary slice [col0, col0 + V) of a wider row: publish the
+        // merged partial with global argmax indices, and the token's logits
+        // when the token falls in this slice; the rows' slices meet in
+        // kld_merge_kernel.
+        MPart o = m;
+        if (o.amax_b != INT_MAX) o.amax_b += static_cast<int>(col0);
+        if (o.amax_q != INT_MAX) o.amax_q += static_cast<int>(col0);
+        if (tok != nullptr) {
+          const int64_t local = static_cast<int64_t>(__ldg(tok + r)) - col0;
+          if (local >= 0 && local < V) {
+            o.flags |= kPartHasTok;
+            o.pad2 = pack2(Elem<DT>::load(rq, local), Elem<DT>::load(rb, local));
+          }
+        }
+        if (lane == 0) {
+          unsigned long long wds[8];
+          part_words(o, wds);
+          ulonglong2* dst = reinterpret_cast<ulonglong2*>(part_out + r);
+#pragma unroll
+          for (int w = 0; w < 4; ++w) dst[w] = make_ulonglong2(wds[2 * w], wds[2 * w + 1]);
+        }
+        continue;
+      }
       if (P == 1) {
         gather_token();
         const kld_row_t rec = finalize_row(m, tok != nullptr, tok_ok, q_tok, b_tok);
@@ -1361,6 +1387,47 @@ __global__ void __launch_bounds__(kRowThreads, 1)
   }
 }
 
+// Vocabulary-sharded rows: one warp per row merges the row's G slice
+// partials (lane g holds slice g; G <= 32) exactly as the split-row path
+// merges its parts, takes the token logits from the slice that holds the
+// token, and writes the record.
+constexpr int kMergeWarps = 8;
+__global__ void __launch_bounds__(kMergeWarps * 32)
+    kld_merge_kernel(const MPart* __restrict__ parts, int G, int64_t N,
+                     const int32_t* __restrict__ tok, int64_t v_total,
+                     kld_row_t* __restrict__ rows) {
+  const int lane = threadIdx.x & 31;
+  for (int64_t r = blockIdx.x * static_cast<int64_t>(kMergeWarps) + (threadIdx.x >> 5); r < N;
+       r += static_cast<int64_t>(gridDim.x) * kMergeWarps) {
+    MPart q = empty_part();
+    if (lane < G) {
+      const ulonglong2* src = reinterpret_cast<const ulonglong2*>(parts + static_cast<int64_t>(lane) * N + r);
+      unsigned long long wds[8];
+#pragma unroll
+      for (int w = 0; w < 4; ++w) {
+        const ulonglong2 v = __ldg(src + w);
+        wds[2 * w] = v.x;
+        wds[2 * w + 1] = v.y;
+      }
+      q = part_from_words(wds);
+    }
+    const unsigned holder = __ballot_sync(0xffffffffu, (q.flags & kPartHasTok) != 0u);
+    const unsigned long long tw = __shfl_sync(0xffffffffu, q.pad2, holder ? __ffs(holder) - 1 : 0);
+    q.flags &= ~kPartHasTok;
+    const MPart m = warp_merge(q);
+    bool tok_ok = false;
+    float q_tok = 0.f, b_tok = 0.f;
+    if (tok != nullptr) {
+      const int32_t tk = __ldg(tok + r);
+      tok_ok = tk >= 0 && static_cast<int64_t>(tk) < v_total && holder != 0u;
+      q_tok = __uint_as_float(static_cast<unsigned>(tw));
+      b_tok = __uint_as_float(static_cast<unsigned>(tw >> 32));
+    }
+    const kld_row_t rec = finalize_row(m, tok != nullptr, tok_ok, q_tok, b_tok);
+    if (lane == 0) rows[r] = rec;
+  }
+}
+
 template <int DT>
 int max_active_clusters(int cluster_ctas) {
   cudaLaunchConfig_t cfg = {};
@@ -1385,7 +1452,8 @@ int max_active_clusters(int cluster_ctas) {
 template <int DT>
 cudaError_t launch_typed(const void* base, const void* quant, const int32_t* tok, int64_t N,
                          int64_t V, kld_row_t* rows, uint32_t* derr, const RowPlan& pl,
-                         const SplitScratch* split, float4* norms, cudaStream_t stream) {
+                         const SplitScratch* split, float4* norms, MPart* part_out, int64_t col0,
+                         cudaStream_t stream) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(pl.grid));
   cfg.blockDim = dim3(kRowThreads);
@@ -1401,7 +1469,7 @@ cudaError_t launch_typed(const void* base, const void* quant, const int32_t* tok
   MPart* gp = split ? static_cast<MPart*>(split->parts) : nullptr;
   unsigned* tk = split ? split->tickets : nullptr;
   return cudaLaunchKernelEx(&cfg, kld_rows_kernel<DT>, base, quant, tok, N, V, rows, derr,
-                            pl.parts_per_row, gp, tk, norms);
+                            pl.parts_per_row, gp, tk, norms, part_out, col0);
 }
 
 }  // namespace
@@ -1462,12 +1530,23 @@ int active_clusters(kld_dtype_t dtype, int lg) {
   return n;
 }
 
+cudaError_t launch_merge(const void* parts, int G, int64_t N, const int32_t* token_ids,
+                         int64_t V_total, kld_row_t* rows, cudaStream_t stream) {
+  if (G < 1 || G > 32 || N < 1) return cudaErrorInvalidValue;
+  int64_t blocks = (N + kMergeWarps - 1) / kMergeWarps;
+  if (blocks > 65535) blocks = 65535;
+  kld_merge_kernel<<<static_cast<unsigned>(blocks), kMergeWarps * 32, 0, stream>>>(
+      static_cast<const MPart*>(parts), G, N, token_ids, V_total, rows);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_rows(const void* base, const void* quant, const int32_t* token_ids, int64_t N,
                         int64_t V, kld_dtype_t dtype, kld_row_t* rows, uint32_t* derr,
                         int sm_count, const SplitScratch* split, float4* norms,
-                        cudaStream_t stream) {
+                        cudaStream_t stream, void* part_out, int64_t col_offset) {
   RowPlan pl = plan_rows(N, sm_count, nullptr, 0);
-  if (split != nullptr && N * 2 <= sm_count && split->max_cluster_ctas >= 1) {
+  // Vocabulary-slice partials come from whole-row launches only.
+  if (split != nullptr && part_out == nullptr && N * 2 <= sm_count && split->max_cluster_ctas >= 1) {
     int fit[4] = {0, 0, 0, 0};
     for (int lg = 0; lg < 4 && (1 << lg) <= split->max_cluster_ctas; ++lg)
       fit[lg] = active_clusters(dtype, lg);
@@ -1478,13 +1557,13 @@ cudaError_t launch_rows(const void* base, const void* quant, const int32_t* toke
   switch (dtype) {
     case KLD_F32:
       return launch_typed<KLD_F32>(base, quant, token_ids, N, V, rows, derr, pl, split, norms,
-                                 stream);
+                                 static_cast<MPart*>(part_out), col_offset, stream);
     case KLD_BF16:
       return launch_typed<KLD_BF16>(base, quant, token_ids, N, V, rows, derr, pl, split, norms,
-                                 stream);
+                                 static_cast<MPart*>(part_out), col_offset, stream);
     case KLD_F16:
       return launch_typed<KLD_F16>(base, quant, token_ids, N, V, rows, derr, pl, split, norms,
-                                 stream);
+                                 static_cast<MPart*>(part_out), col_offset, stream);
   }
   return cudaErrorInvalidValue;
 }

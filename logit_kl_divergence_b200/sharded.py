@@ -28,13 +28,14 @@ def shard_bounds(n_rows: int, world: int, rank: int) -> tuple[int, int]:
 
 
 def gather_records(records: torch.Tensor, group=None, counts: list[int] | None = None) -> torch.Tensor:
-    """All-gather every rank's [n_r, 40] uint8 records, concatenated in rank
-    order (ranks may hold different row counts). Collective: every rank of
-    `group` calls it with its own records, in the same order of calls.
-    `counts`: every rank's row count when the caller knows them (skips one
-    small all-gather)."""
-    if records.dtype != torch.uint8 or records.dim() != 2 or records.shape[1] != ROW_RECORD_BYTES:
-        raise ValueError("records must be a [n, 40] uint8 tensor")
+    """All-gather every rank's [n_r, w] uint8 rows (40-byte records, 64-byte
+    vocabulary-slice partials), concatenated in rank order (ranks may hold
+    different row counts). Collective: every rank of `group` calls it with
+    its own rows, in the same order of calls. `counts`: every rank's row
+    count when the caller knows them (skips one small all-gather)."""
+    if records.dtype != torch.uint8 or records.dim() != 2:
+        raise ValueError("records must be a [n, w] uint8 tensor")
+    width = records.shape[1]
     world = dist.get_world_size(group)
     if counts is None:
         n = torch.tensor([records.shape[0]], dtype=torch.int64, device=records.device)
@@ -46,13 +47,13 @@ def gather_records(records: torch.Tensor, group=None, counts: list[int] | None =
     m = max(counts)
     padded = records
     if records.shape[0] != m:
-        padded = records.new_zeros((m, ROW_RECORD_BYTES))
+        padded = records.new_zeros((m, width))
         padded[:records.shape[0]] = records
     padded = padded.contiguous()
     if dist.get_backend(group) == "nccl":
-        out = records.new_empty((m * world, ROW_RECORD_BYTES))
+        out = records.new_empty((m * world, width))
         dist.all_gather_into_tensor(out, padded, group=group)
-        parts = list(out.view(world, m, ROW_RECORD_BYTES))
+        parts = list(out.view(world, m, width))
     else:
         parts = [torch.empty_like(padded) for _ in range(world)]
         dist.all_gather(parts, padded, group=group)
@@ -97,3 +98,32 @@ class ShardedKLDStats:
         close = getattr(self.stats, "close", None)
         if close is not None:
             close()
+
+
+class VocabShardedKLDStats:
+    """The statistic over vocabulary-sharded logits (tensor-parallel lm_head):
+    every rank of `group` holds all N rows but only its column slice
+    [col_offset, col_offset + V_r) of a V_total-wide vocabulary, ranks in
+    column order. Each rank computes one 64-byte partial per row for its
+    slice, the partials are all-gathered (N*64 bytes per rank), and every
+    rank merges the G partials of each row and reduces: the same statistics
+    on every rank as for the full rows on one GPU. At most 32 ranks."""
+
+    def __init__(self, n_rows: int, device=None, group=None):
+        from . import KLDStats
+
+        self.stats = KLDStats(max_rows=n_rows, device=device)
+        self.group = group
+
+    def run(self, base: torch.Tensor, quant: torch.Tensor, token_ids: torch.Tensor | None,
+            col_offset: int, v_total: int) -> dict:
+        """Collective. `token_ids` are the full-vocabulary ids (the same on
+        every rank, or None on every rank)."""
+        parts = self.stats.run_partials(base, quant, token_ids, col_offset, v_total)
+        world = dist.get_world_size(self.group)
+        gathered = gather_records(parts, self.group, counts=[base.shape[0]] * world)
+        self.stats.merge_partials(gathered.view(world, base.shape[0], -1), token_ids, v_total)
+        return self.stats.result()
+
+    def close(self):
+        self.stats.close()

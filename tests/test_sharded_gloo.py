@@ -82,6 +82,11 @@ def _worker(rank, world, port, n_rows, with_tokens, errq):
         expect = torch.cat([torch.full((b - a, 40), r, dtype=torch.uint8)
                             for r, (a, b) in enumerate(shard_bounds(n_rows, world, q) for q in range(world))])
         assert torch.equal(got, expect)
+        # 64-byte vocabulary-slice partials: every rank holds all rows, so
+        # the gather is [world][n] in rank order
+        slc = torch.full((n_rows, 64), 100 + rank, dtype=torch.uint8)
+        allp = gather_records(slc, counts=[n_rows] * world).view(world, n_rows, 64)
+        assert all(torch.all(allp[r] == 100 + r) for r in range(world))
         # the whole orchestration, oracle-backed
         sk = ShardedKLDStats(max_rows_per_rank=hi - lo + 1, stats=OracleStats(oracle.F32))
         res = sk.run(w.base[lo:hi].contiguous(), w.quant[lo:hi].contiguous(),
