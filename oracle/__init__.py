@@ -115,6 +115,12 @@ def _load():
                 ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64,
                 ctypes.c_int, ctypes.c_double, ctypes.c_void_p,
             ]
+            lib.oracle_topk.restype = ctypes.c_int
+            lib.oracle_topk.argtypes = [
+                ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64,
+                ctypes.c_int, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p,
+                ctypes.c_void_p, ctypes.c_void_p,
+            ]
             lib.oracle_percentile_sorted.restype = ctypes.c_double
             lib.oracle_percentile_sorted.argtypes = [
                 ctypes.c_void_p, ctypes.c_int64, ctypes.c_double,
@@ -219,6 +225,24 @@ def grad(base, quant, dtype: int = F32, scale: float = 1.0) -> np.ndarray:
     out = np.empty((N, V), np.float64)
     if lib.oracle_grad(b.ctypes.data, q.ctypes.data, N, V, dtype, float(scale), out.ctypes.data) != 0:
         raise ValueError("oracle_grad rejected its arguments")
+    return out
+
+
+def topk(base, quant, k: int = 128, dtype: int = F32) -> dict:
+    """Top-k compression of each base row and the KL of the quant row against
+    it: idx [N, k] int32, logp [N, k] and rest [N] (log P_base), kl_topk [N]."""
+    lib = _load()
+    b = _as_logits(base, dtype)
+    q = _as_logits(quant, dtype)
+    if b.shape != q.shape:
+        raise ValueError("base and quant shapes differ")
+    N, V = b.shape
+    out = {"idx": np.empty((N, k), np.int32), "logp": np.empty((N, k), np.float64),
+           "rest": np.empty(N, np.float64), "kl_topk": np.empty(N, np.float64)}
+    rc = lib.oracle_topk(b.ctypes.data, q.ctypes.data, N, V, dtype, int(k), out["idx"].ctypes.data,
+                         out["logp"].ctypes.data, out["rest"].ctypes.data, out["kl_topk"].ctypes.data)
+    if rc != 0:
+        raise ValueError("oracle_topk rejected its arguments")
     return out
 
 

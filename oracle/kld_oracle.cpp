@@ -263,6 +263,89 @@ extern "C" int oracle_grad(const void* base, const void* quant, int64_t N,
   return 0;
 }
 
+extern "C" int oracle_topk(const void* base, const void* quant, int64_t N,
+                           int64_t V, int dtype, int k, int32_t* idx,
+                           double* logp, double* rest, double* kl_topk) {
+  if (!base || !quant || !idx || !logp || !rest || !kl_topk) return -1;
+  if (N < 0 || V < 1 || V > 0x7fffffffLL || k < 1) return -1;
+  if (dtype != ORACLE_F32 && dtype != ORACLE_BF16 && dtype != ORACLE_F16)
+    return -1;
+  std::vector<double> b((size_t)V), q((size_t)V);
+  std::vector<int64_t> order((size_t)V);
+  std::vector<char> in_top((size_t)V);
+  for (int64_t r = 0; r < N; ++r) {
+    load_row(base, dtype, r, V, b.data());
+    load_row(quant, dtype, r, V, q.data());
+    int32_t* id = idx + r * k;
+    double* lp = logp + r * k;
+    /* Excluded rows, as for the statistics. */
+    bool excluded = false;
+    double m_b = -kInf, m_q = -kInf;
+    for (int64_t j = 0; j < V; ++j) {
+      if (std::isnan(b[j]) || std::isnan(q[j]) || b[j] == kInf || q[j] == kInf)
+        excluded = true;
+      if (b[j] > m_b) m_b = b[j];
+      if (q[j] > m_q) m_q = q[j];
+    }
+    if (excluded || m_b == -kInf || m_q == -kInf) {
+      for (int i = 0; i < k; ++i) {
+        id[i] = -1;
+        lp[i] = kNaN;
+      }
+      rest[r] = kNaN;
+      kl_topk[r] = kNaN;
+      continue;
+    }
+    /* The k largest base logits, ties to the lowest index: a stable sort of
+     * the indices by descending logit. */
+    for (int64_t j = 0; j < V; ++j) order[(size_t)j] = j;
+    std::stable_sort(order.begin(), order.end(),
+                     [&](int64_t x, int64_t y) { return b[x] > b[y]; });
+    const int64_t kt = std::min<int64_t>(k, V);
+    std::fill(in_top.begin(), in_top.end(), 0);
+    for (int64_t i = 0; i < kt; ++i) in_top[(size_t)order[(size_t)i]] = 1;
+    /* Both distributions over the full row. */
+    double zb = 0.0, zq = 0.0;
+    for (int64_t j = 0; j < V; ++j) zb += std::exp(b[j] - m_b);
+    for (int64_t j = 0; j < V; ++j) zq += std::exp(q[j] - m_q);
+    const double lse_b = m_b + std::log(zb);
+    const double lse_q = m_q + std::log(zq);
+    double kl = 0.0, p_rest = 0.0, r_rest = 0.0;
+    bool inf_kl = false;
+    for (int64_t i = 0; i < k; ++i) {
+      if (i >= kt) {
+        id[i] = -1;
+        lp[i] = -kInf;
+        continue;
+      }
+      const int64_t j = order[(size_t)i];
+      id[i] = (int32_t)j;
+      lp[i] = b[j] - lse_b;
+      if (b[j] == -kInf) continue; /* p_j = 0 adds nothing */
+      if (q[j] == -kInf) {
+        inf_kl = true;
+        continue;
+      }
+      const double logp_j = b[j] - lse_b, logr_j = q[j] - lse_q;
+      kl += std::exp(logp_j) * (logp_j - logr_j);
+    }
+    for (int64_t j = 0; j < V; ++j) {
+      if (in_top[(size_t)j]) continue;
+      p_rest += std::exp(b[j] - lse_b);
+      r_rest += std::exp(q[j] - lse_q);
+    }
+    if (p_rest > 0.0) {
+      if (r_rest > 0.0)
+        kl += p_rest * (std::log(p_rest) - std::log(r_rest));
+      else
+        inf_kl = true;
+    }
+    rest[r] = p_rest > 0.0 ? std::log(p_rest) : -kInf;
+    kl_topk[r] = inf_kl ? kInf : kl;
+  }
+  return 0;
+}
+
 extern "C" double oracle_percentile_sorted(const double* x, int64_t n,
                                            double p) {
   if (n <= 0) return kNaN;

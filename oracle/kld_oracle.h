@@ -100,6 +100,22 @@ int oracle_reduce(const double* kld, const double* nll, const double* nll_base,
 int oracle_grad(const void* base, const void* quant, int64_t N, int64_t V,
                 int dtype, double scale, double* grad);
 
+/* Top-k compression of the base row and the KL against it ("Mistral-Small-
+ * 4-119B-2603 GSQ-RCO IQ3_S GGUF", "How it was made", step 7: tuning
+ * "against the top-128 distributions (and the rest of the mass)"). Per row:
+ * T = the k entries with the largest base logits (ties: lowest index
+ * first), listed in that order in idx[r*k ..] with log P_base in
+ * logp[r*k ..] (entries past V: index -1, logp -inf); rest[r] =
+ * log(sum of P_base outside T) (-inf when T holds everything), and
+ *   kl_topk[r] = sum_{j in T} p_j log(p_j / r_j) + p_rest log(p_rest / r_rest),
+ * with p = softmax(b), r = softmax(q), p_rest = sum_{j not in T} p_j,
+ * r_rest likewise (a term with p = 0 is 0; p > 0 with r = 0 is +inf).
+ * Excluded rows (NONFINITE / EMPTY): idx -1, logp and rest NaN, kl NaN.
+ * Returns 0, or -1 on bad args. */
+int oracle_topk(const void* base, const void* quant, int64_t N, int64_t V,
+                int dtype, int k, int32_t* idx, double* logp, double* rest,
+                double* kl_topk);
+
 /* Type-7 percentile of an ascending array x[0..n): pos = p*(n-1). */
 double oracle_percentile_sorted(const double* x, int64_t n, double p);
 

@@ -48,6 +48,12 @@ MUTANTS = {
                           "g[j] = scale * (std::exp(b[j] - lse_b) - std::exp(q[j] - lse_q));"),
     "grad_quant_normaliser_from_base": ("g[j] = scale * (std::exp(q[j] - lse_q) - std::exp(b[j] - lse_b));",
                                         "g[j] = scale * (std::exp(q[j] - lse_b) - std::exp(b[j] - lse_b));"),
+    "topk_selected_by_quant": ("[&](int64_t x, int64_t y) { return b[x] > b[y]; });",
+                               "[&](int64_t x, int64_t y) { return q[x] > q[y]; });"),
+    "topk_rest_term_dropped": ("kl += p_rest * (std::log(p_rest) - std::log(r_rest));",
+                               "kl += 0.0 * (std::log(p_rest) - std::log(r_rest));"),
+    "topk_rest_from_quant_side": ("      p_rest += std::exp(b[j] - lse_b);",
+                                  "      p_rest += std::exp(q[j] - lse_q);"),
     "ppl_ratio_inverted": ("out->ln_ppl_ratio = out->mean_nll - out->mean_nll_base;",
                            "out->ln_ppl_ratio = out->mean_nll_base - out->mean_nll;"),
 }

@@ -536,3 +536,82 @@ def test_grad_of_excluded_rows_is_zero_and_masks_are_zero():
     e = np.exp(q[2].astype(np.float64) - q[2].max())
     r = e / e.sum()
     assert g[2, 5] < 0 and abs(g[2, 4] - r[4]) < 1e-16
+
+
+# ---------------------------------------------------- top-k compression + KL
+
+def _softmax_np(x):
+    x = x.astype(np.float64)
+    m = x.max(axis=1, keepdims=True)
+    e = np.exp(x - m)
+    return e / e.sum(axis=1, keepdims=True)
+
+
+def test_topk_with_k_at_least_V_is_the_full_kl():
+    b = RNG.normal(0, 2, size=(6, 50)).astype(np.float32)
+    q = (b + RNG.normal(0, 0.5, size=(6, 50))).astype(np.float32)
+    t = oracle.topk(b, q, k=64)
+    r, _ = _run(b, q)
+    np.testing.assert_allclose(t["kl_topk"], r["kld"], rtol=1e-11, atol=1e-15)
+    assert np.all(np.isneginf(t["rest"]))
+    assert np.all(t["idx"][:, 50:] == -1) and np.all(np.isneginf(t["logp"][:, 50:]))
+    np.testing.assert_array_equal(t["idx"][:, :50], np.argsort(-b, axis=1, kind="stable"))
+
+
+def test_topk_one_is_the_binary_kl_of_the_top_entry():
+    b = RNG.normal(0, 1.5, size=(10, 300)).astype(np.float32)
+    q = (b + RNG.normal(0, 0.4, size=(10, 300))).astype(np.float32)
+    t = oracle.topk(b, q, k=1)
+    p, r = _softmax_np(b), _softmax_np(q)
+    for i in range(10):
+        j = int(np.argmax(b[i]))
+        assert t["idx"][i, 0] == j
+        p1, r1 = p[i, j], r[i, j]
+        want = p1 * math.log(p1 / r1) + (1 - p1) * math.log((1 - p1) / (1 - r1))
+        assert abs(t["kl_topk"][i] - want) < 1e-12
+        assert abs(t["rest"][i] - math.log1p(-p1)) < 1e-12
+
+
+def test_topk_kl_grows_with_k_up_to_the_full_kl():
+    # merging categories never increases KL (data processing), and the top-k
+    # partitions refine each other as k grows
+    b = RNG.normal(0, 2.5, size=(8, 2000)).astype(np.float32)
+    q = (b + RNG.normal(0, 0.3, size=(8, 2000))).astype(np.float32)
+    full, _ = _run(b, q)
+    prev = np.zeros(8)
+    for k in (1, 2, 8, 32, 128, 512, 2000):
+        cur = oracle.topk(b, q, k=k)["kl_topk"]
+        assert np.all(cur >= prev - 1e-15) and np.all(cur <= full["kld"] + 1e-12)
+        prev = cur
+    np.testing.assert_allclose(prev, full["kld"], rtol=1e-11)
+
+
+def test_topk_indices_logp_and_rest_by_numpy_and_ties():
+    b = RNG.normal(0, 1, size=(5, 1000)).astype(np.float32)
+    b[0, [900, 3, 500]] = 9.0          # a three-way tie at the top
+    q = (b + RNG.normal(0, 0.2, size=(5, 1000))).astype(np.float32)
+    t = oracle.topk(b, q, k=128)
+    order = np.argsort(-b, axis=1, kind="stable")[:, :128]
+    np.testing.assert_array_equal(t["idx"], order)
+    assert list(t["idx"][0, :3]) == [3, 500, 900]
+    p = _softmax_np(b)
+    np.testing.assert_allclose(t["logp"], np.log(np.take_along_axis(p, order, axis=1)), rtol=1e-12)
+    mask = np.ones_like(p, bool)
+    np.put_along_axis(mask, order, False, axis=1)
+    np.testing.assert_allclose(t["rest"], np.log(np.where(mask, p, 0).sum(axis=1)), rtol=1e-12)
+
+
+def test_topk_identical_rows_masks_and_excluded_rows():
+    b = RNG.normal(0, 1, size=(4, 200)).astype(np.float32)
+    t = oracle.topk(b, b.copy(), k=16)
+    assert np.all(t["kl_topk"] == 0.0)
+    b2 = b.copy()
+    q2 = b.copy() + np.float32(0.25)
+    b2[0, 10:] = NEG_INF                 # only 10 finite base entries: k = 16 reaches p = 0
+    b2[1, 5] = np.nan                    # excluded row
+    q2[2, int(np.argmax(b2[2]))] = NEG_INF  # the quant gives the top entry nothing
+    t2 = oracle.topk(b2, q2, k=16)
+    assert np.isneginf(t2["rest"][0]) and np.all(np.isneginf(t2["logp"][0, 10:]))
+    assert np.all(t2["idx"][1] == -1) and math.isnan(t2["kl_topk"][1]) and math.isnan(t2["rest"][1])
+    assert t2["kl_topk"][2] == math.inf
+    assert abs(t2["kl_topk"][3]) < 1e-15   # a constant shift changes no probability
