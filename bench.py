@@ -308,6 +308,7 @@ def main():
     ap.add_argument("--no-variants", action="store_true")
     ap.add_argument("--no-split-row", action="store_true")
     ap.add_argument("--no-grad", action="store_true")
+    ap.add_argument("--no-topk", action="store_true")
     ap.add_argument("--split-calls", type=int, default=SPLIT_CALLS,
                     help="profiling only: fewer calls per size in the split-row section")
     ap.add_argument("--rows", type=int, default=None,
@@ -481,6 +482,29 @@ def main():
         del gout
         torch.cuda.empty_cache()
 
+    # Top-128 compression of the base rows + KL against it (row pass +
+    # reduction + top-k pass) on the same context.
+    topk = None
+    if world == 1 and not args.no_topk:
+        for _ in range(2):
+            st.run_topk(w.base, w.quant, w.token_ids, k=128)
+            st.result()
+        torch.cuda.synchronize(dev)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        tsteps = max(2, min(args.steps, 5))
+        a.record(stream)
+        for _ in range(tsteps):
+            out = st.run_topk(w.base, w.quant, w.token_ids, k=128)
+            st.result()
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        tms = a.elapsed_time(b) / tsteps
+        topk = {"workload": name, "k": 128, "steps": tsteps, "ms_per_step": tms,
+                "value": N / (tms / 1000.0), "unit": "rows/s",
+                "topk_pass_ms_estimate": tms - ms_per_step,
+                "mean_kl_topk": float(out["kl_topk"].mean().item())}
+        del out
+
     # End to end through the public host-memory entry point: pinned host
     # buffers in, the result struct out, copies inside the timed region.
     e2e = None
@@ -528,7 +552,7 @@ def main():
             "gbs": in_bytes * world / (ms_per_step / 1000.0) / 1e9,
             "mean_kld": res["mean_kld"], "top1_agree_pct": res["top1_agree_pct"], "ppl": res["ppl"],
             "ppl_base": res["ppl_base"], "rms_dp": res["rms_dp"], "mean_dp": res["mean_dp"],
-            "variants": variants, "split_row": split_row, "grad": grad,
+            "variants": variants, "split_row": split_row, "grad": grad, "topk": topk,
         }
         if args.rows is not None or args.dtype != "f32" or args.split_calls != SPLIT_CALLS:
             line["config"]["override"] = {"rows": N, "dtype": args.dtype,

@@ -271,6 +271,28 @@ kld_status_t kld_stats_merge_partials(kld_stats_t h, const void* parts, int G, i
                                       const int32_t* token_ids, int64_t V_total, void* stream);
 
 /*
+ * The statistic plus a top-k compression of each base row and the KL of the
+ * quant row against it ("Mistral-Small-4-119B-2603 GSQ-RCO IQ3_S GGUF",
+ * "How it was made", step 7: tuning "against the top-128 distributions (and
+ * the rest of the mass)"). Per row r, T = the k largest base logits (ties to
+ * the lowest index; 1 <= k <= 1024):
+ *   idx_out[r*k + i]  index of the i-th entry of T (int32; -1 past V)
+ *   logp_out[r*k + i] its log P_base (float; -inf past V)
+ *   rest_out[r]       log of P_base outside T (float; -inf if none)
+ *   kl_out[r]         sum_{T} p log(p/r) + p_rest log(p_rest/r_rest) (double)
+ * with p = softmax(base), r = softmax(quant). Rows the statistics exclude get
+ * idx -1 and NaN. idx_out, logp_out and rest_out may be NULL; all are
+ * caller-owned DEVICE memory, naturally aligned. Enqueues the row pass, the
+ * reduction (read with kld_stats_result) and a top-k pass that reads each
+ * base row 2-4 times (from L2 after the first) and the quant row once.
+ */
+#define KLD_MAX_TOPK 1024
+kld_status_t kld_stats_run_topk(kld_stats_t h, const void* base, const void* quant,
+                                const int32_t* token_ids, int64_t N, int64_t V,
+                                kld_dtype_t dtype, int k, int32_t* idx_out, float* logp_out,
+                                float* rest_out, double* kl_out, void* stream);
+
+/*
  * Duration in milliseconds of the last kld_stats_run_grad's gradient pass
  * (timing enabled by kld_stats_set_timing; waits for that run).
  */

@@ -137,6 +137,26 @@ class KLDStats:
         _lib.check(st, "kld_stats_run_grad")
         return out
 
+    def run_topk(self, base: torch.Tensor, quant: torch.Tensor, token_ids: torch.Tensor | None = None,
+                 k: int = 128, stream=None) -> dict:
+        """The statistic (read it with :meth:`result`) plus the top-k
+        compression of each base row and the KL of the quant row against it:
+        ``idx`` [N, k] int32, ``logp`` [N, k] float32 (log P_base), ``rest``
+        [N] float32 (log of the mass outside the top k) and ``kl_topk`` [N]
+        float64, CUDA tensors filled asynchronously on the stream."""
+        _check_pair(base, quant, token_ids, True)
+        n = base.shape[0]
+        out = {"idx": torch.empty((n, k), dtype=torch.int32, device=base.device),
+               "logp": torch.empty((n, k), dtype=torch.float32, device=base.device),
+               "rest": torch.empty(n, dtype=torch.float32, device=base.device),
+               "kl_topk": torch.empty(n, dtype=torch.float64, device=base.device)}
+        st = self._lib.kld_stats_run_topk(self._h, _ptr(base), _ptr(quant), _ptr(token_ids), n,
+                                          base.shape[1], dtype_code(base), int(k), _ptr(out["idx"]),
+                                          _ptr(out["logp"]), _ptr(out["rest"]), _ptr(out["kl_topk"]),
+                                          ctypes.c_void_p(_stream_ptr(stream, base.device)))
+        _lib.check(st, "kld_stats_run_topk")
+        return out
+
     def grad_timing(self) -> float:
         """Milliseconds of the last run_grad's gradient pass (timing enabled)."""
         ms = ctypes.c_float()

@@ -27,6 +27,7 @@ KLD_STATIC_MAX_ROWS = 65536
 
 KLD_F32, KLD_BF16, KLD_F16 = 0, 1, 2
 KLD_PARTIAL_BYTES = 64
+KLD_MAX_TOPK = 1024
 
 ROW_NONFINITE = 1 << 0
 ROW_EMPTY = 1 << 1
@@ -111,6 +112,7 @@ SIGNATURES = {
     "kld_stats_set_split": (_ST, [_P, _I32]),
     "kld_stats_run_grad": (_ST, [_P, _P, _P, _P, _I64, _I64, _I32, _P, _I32, ctypes.c_double, _P]),
     "kld_stats_grad_timing": (_ST, [_P, ctypes.POINTER(ctypes.c_float)]),
+    "kld_stats_run_topk": (_ST, [_P, _P, _P, _P, _I64, _I64, _I32, _I32, _P, _P, _P, _P, _P]),
     "kld_stats_run_partials": (_ST, [_P, _P, _P, _P, _I64, _I64, _I64, _I64, _I32, _P, _P]),
     "kld_stats_merge_partials": (_ST, [_P, _P, _I32, _I64, _P, _I64, _P]),
     "kld_stats_timing": (_ST, [_P, ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ctypes.c_float)]),

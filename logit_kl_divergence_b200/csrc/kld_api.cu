@@ -64,7 +64,7 @@ struct kld_stats_s {
   int64_t max_rows = 0;
   kld_row_t* rows = nullptr;
   void* split_mem = nullptr;  // split-row scratch: partials, then tickets
-  float4* norms = nullptr;    // per-row softmax normalisers for the gradient pass
+  kld::RowAux* aux = nullptr;  // per-row normalisers for the gradient and top-k passes
   bool grad_timing_valid = false;
   kld::SplitScratch split = {nullptr, nullptr, 0, kld::kDefaultClusterCtas};
   uint32_t* derr = nullptr;
@@ -104,9 +104,9 @@ kld_status_t check_inputs(const void* base, const void* quant, const int32_t* to
 
 cudaError_t launch_rows(kld_stats_s* h, const void* base, const void* quant, const int32_t* tok,
                         int64_t N, int64_t V, kld_dtype_t dtype, kld_row_t* rows, cudaStream_t s,
-                        float4* norms = nullptr) {
+                        kld::RowAux* aux = nullptr) {
   return kld::launch_rows(base, quant, tok, N, V, dtype, rows, h->derr, h->sm_count, &h->split,
-                          norms, s);
+                          aux, s);
 }
 
 kld_status_t enqueue_reduce(kld_stats_t h, const kld_row_t* rows, int64_t N, int has_nll,
@@ -194,8 +194,8 @@ kld_status_t kld_stats_create(kld_stats_t* out, int64_t max_rows, int device) {
     cudaError_t err;
     if ((err = cudaMalloc(&h->rows, sizeof(kld_row_t) * static_cast<size_t>(max_rows))) !=
         cudaSuccess) { st = cuda_fail(err, "cudaMalloc(rows)"); break; }
-    if ((err = cudaMalloc(&h->norms, sizeof(float4) * static_cast<size_t>(max_rows))) !=
-        cudaSuccess) { st = cuda_fail(err, "cudaMalloc(norms)"); break; }
+    if ((err = cudaMalloc(&h->aux, sizeof(kld::RowAux) * static_cast<size_t>(max_rows))) !=
+        cudaSuccess) { st = cuda_fail(err, "cudaMalloc(row normalisers)"); break; }
     if ((err = cudaMalloc(&h->derr, sizeof(uint32_t))) != cudaSuccess) {
       st = cuda_fail(err, "cudaMalloc(error word)"); break; }
     if ((err = cudaMemset(h->derr, 0, sizeof(uint32_t))) != cudaSuccess) {
@@ -252,7 +252,7 @@ void kld_stats_destroy(kld_stats_t h) {
   if (h->derr) cudaFree(h->derr);
   if (h->rows) cudaFree(h->rows);
   if (h->split_mem) cudaFree(h->split_mem);
-  if (h->norms) cudaFree(h->norms);
+  if (h->aux) cudaFree(h->aux);
   delete h;
 }
 
@@ -323,12 +323,12 @@ kld_status_t kld_stats_run_grad(kld_stats_t h, const void* base, const void* qua
   h->timing_valid = h->timing;
   h->grad_timing_valid = h->timing;
   if (h->timing) KLD_CUDA(cudaEventRecord(h->tev[0], s));
-  KLD_CUDA(launch_rows(h, base, quant, token_ids, N, V, dtype, h->rows, s, h->norms));
+  KLD_CUDA(launch_rows(h, base, quant, token_ids, N, V, dtype, h->rows, s, h->aux));
   if (h->timing) KLD_CUDA(cudaEventRecord(h->tev[1], s));
   h->last_rows = N;
   st = enqueue_reduce(h, h->rows, N, token_ids != nullptr, s);
   if (st != KLD_OK) return st;
-  KLD_CUDA(kld::launch_grad(base, quant, h->norms, N, V, dtype, grad, grad_dtype,
+  KLD_CUDA(kld::launch_grad(base, quant, h->aux, N, V, dtype, grad, grad_dtype,
                             static_cast<float>(scale), h->sm_count, s));
   if (h->timing) KLD_CUDA(cudaEventRecord(h->tev[3], s));
   return KLD_OK;
@@ -367,6 +367,31 @@ kld_status_t kld_stats_merge_partials(kld_stats_t h, const void* parts, int G, i
   KLD_CUDA(kld::launch_merge(parts, G, N, token_ids, V_total, h->rows, s));
   h->last_rows = N;
   return enqueue_reduce(h, h->rows, N, token_ids != nullptr, s);
+}
+
+kld_status_t kld_stats_run_topk(kld_stats_t h, const void* base, const void* quant,
+                                const int32_t* token_ids, int64_t N, int64_t V,
+                                kld_dtype_t dtype, int k, int32_t* idx_out, float* logp_out,
+                                float* rest_out, double* kl_out, void* stream) {
+  if (!h) return KLD_ERR_INVALID_ARG;
+  kld_status_t st = check_inputs(base, quant, token_ids, N, V, dtype, true);
+  if (st != KLD_OK) return st;
+  if (N > h->max_rows || k < 1 || k > kld::kMaxTopk || !kl_out) return KLD_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(kl_out) & 7u) || (reinterpret_cast<uintptr_t>(idx_out) & 3u) ||
+      (reinterpret_cast<uintptr_t>(logp_out) & 3u) || (reinterpret_cast<uintptr_t>(rest_out) & 3u))
+    return KLD_ERR_INVALID_ARG;
+  DeviceGuard guard(h->device);
+  if (!guard.ok()) return cuda_fail(cudaGetLastError(), "cudaSetDevice");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  h->timing_valid = false;
+  h->grad_timing_valid = false;
+  KLD_CUDA(launch_rows(h, base, quant, token_ids, N, V, dtype, h->rows, s, h->aux));
+  h->last_rows = N;
+  st = enqueue_reduce(h, h->rows, N, token_ids != nullptr, s);
+  if (st != KLD_OK) return st;
+  KLD_CUDA(kld::launch_topk(base, quant, h->aux, N, V, dtype, k, idx_out, logp_out, rest_out,
+                            kl_out, h->sm_count, s));
+  return KLD_OK;
 }
 
 kld_status_t kld_stats_grad_timing(kld_stats_t h, float* grad_ms) {

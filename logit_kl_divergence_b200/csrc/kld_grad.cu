@@ -7,7 +7,7 @@
 //
 // zero on rows that the statistics exclude (NaN / +inf, all -inf). The row
 // pass has already produced each row's normalisers (kld_rows.cu,
-// row_norms): softmax(b)_j = 2^(b_j*L - Fb) * mb with an integer frame Fb
+// row_aux): softmax(b)_j = 2^(b_j*L - Fb) * mb with an integer frame Fb
 // and mb in (0.5, 1], the same for q. This second pass streams b and q once
 // more and writes the gradient: a pure HBM-bound elementwise kernel (reads
 // 2*s, writes s_out bytes per element), 16-byte vector loads and stores,
@@ -137,7 +137,7 @@ __device__ __forceinline__ float grad_of(float b, float q, const float4& nb, flo
 template <int DT, int OT>
 __global__ void __launch_bounds__(kGradThreads)
     kld_grad_vec_kernel(const void* __restrict__ base, const void* __restrict__ quant,
-                        const float4* __restrict__ norms, int64_t N, int64_t V,
+                        const RowAux* __restrict__ aux, int64_t N, int64_t V,
                         void* __restrict__ grad, float scale) {
   const int64_t upr = V / kUnit;  // units per row
   const int64_t total = N * upr;
@@ -148,7 +148,7 @@ __global__ void __launch_bounds__(kGradThreads)
        u += static_cast<int64_t>(gridDim.x) * blockDim.x) {
     const int64_t r = u / upr;
     const int64_t e = u * kUnit;  // flattened element index (= r * V + column)
-    const float4 nb = __ldg(norms + r);
+    const float4 nb = __ldg(reinterpret_cast<const float4*>(aux + r));
     float g[kUnit];
     if (isnan(nb.x)) {
 #pragma unroll
@@ -168,7 +168,7 @@ __global__ void __launch_bounds__(kGradThreads)
 template <int DT, int OT>
 __global__ void __launch_bounds__(kGradThreads)
     kld_grad_scalar_kernel(const void* __restrict__ base, const void* __restrict__ quant,
-                           const float4* __restrict__ norms, int64_t N, int64_t V,
+                           const RowAux* __restrict__ aux, int64_t N, int64_t V,
                            void* __restrict__ grad, float scale) {
   const int64_t total = N * V;
   const char* B = static_cast<const char*>(base);
@@ -176,7 +176,7 @@ __global__ void __launch_bounds__(kGradThreads)
   char* G = static_cast<char*>(grad);
   for (int64_t e = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; e < total;
        e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const float4 nb = __ldg(norms + e / V);
+    const float4 nb = __ldg(reinterpret_cast<const float4*>(aux + e / V));
     float g = 0.f;
     if (!isnan(nb.x))
       g = grad_of(In<DT>::load1(B + e * In<DT>::kBytes), In<DT>::load1(Q + e * In<DT>::kBytes),
@@ -186,7 +186,7 @@ __global__ void __launch_bounds__(kGradThreads)
 }
 
 template <int DT, int OT>
-cudaError_t launch_typed(const void* base, const void* quant, const float4* norms, int64_t N,
+cudaError_t launch_typed(const void* base, const void* quant, const RowAux* aux, int64_t N,
                          int64_t V, void* grad, float scale, int sm_count, cudaStream_t s) {
   const uintptr_t a = reinterpret_cast<uintptr_t>(base) | reinterpret_cast<uintptr_t>(quant) |
                       reinterpret_cast<uintptr_t>(grad);
@@ -194,39 +194,39 @@ cudaError_t launch_typed(const void* base, const void* quant, const float4* norm
   // Enough resident threads to keep HBM busy: 8 CTAs of 256 per SM.
   const int grid = sm_count * 8;
   if (vec) {
-    kld_grad_vec_kernel<DT, OT><<<grid, kGradThreads, 0, s>>>(base, quant, norms, N, V, grad,
+    kld_grad_vec_kernel<DT, OT><<<grid, kGradThreads, 0, s>>>(base, quant, aux, N, V, grad,
                                                               scale);
   } else {
-    kld_grad_scalar_kernel<DT, OT><<<grid, kGradThreads, 0, s>>>(base, quant, norms, N, V, grad,
+    kld_grad_scalar_kernel<DT, OT><<<grid, kGradThreads, 0, s>>>(base, quant, aux, N, V, grad,
                                                                  scale);
   }
   return cudaGetLastError();
 }
 
 template <int DT>
-cudaError_t launch_out(const void* base, const void* quant, const float4* norms, int64_t N,
+cudaError_t launch_out(const void* base, const void* quant, const RowAux* aux, int64_t N,
                        int64_t V, void* grad, kld_dtype_t ot, float scale, int sm_count,
                        cudaStream_t s) {
   switch (ot) {
-    case KLD_F32: return launch_typed<DT, KLD_F32>(base, quant, norms, N, V, grad, scale, sm_count, s);
-    case KLD_BF16: return launch_typed<DT, KLD_BF16>(base, quant, norms, N, V, grad, scale, sm_count, s);
-    case KLD_F16: return launch_typed<DT, KLD_F16>(base, quant, norms, N, V, grad, scale, sm_count, s);
+    case KLD_F32: return launch_typed<DT, KLD_F32>(base, quant, aux, N, V, grad, scale, sm_count, s);
+    case KLD_BF16: return launch_typed<DT, KLD_BF16>(base, quant, aux, N, V, grad, scale, sm_count, s);
+    case KLD_F16: return launch_typed<DT, KLD_F16>(base, quant, aux, N, V, grad, scale, sm_count, s);
   }
   return cudaErrorInvalidValue;
 }
 
 }  // namespace
 
-cudaError_t launch_grad(const void* base, const void* quant, const float4* norms, int64_t N,
+cudaError_t launch_grad(const void* base, const void* quant, const RowAux* aux, int64_t N,
                         int64_t V, kld_dtype_t dtype, void* grad, kld_dtype_t grad_dtype,
                         float scale, int sm_count, cudaStream_t stream) {
   switch (dtype) {
     case KLD_F32:
-      return launch_out<KLD_F32>(base, quant, norms, N, V, grad, grad_dtype, scale, sm_count, stream);
+      return launch_out<KLD_F32>(base, quant, aux, N, V, grad, grad_dtype, scale, sm_count, stream);
     case KLD_BF16:
-      return launch_out<KLD_BF16>(base, quant, norms, N, V, grad, grad_dtype, scale, sm_count, stream);
+      return launch_out<KLD_BF16>(base, quant, aux, N, V, grad, grad_dtype, scale, sm_count, stream);
     case KLD_F16:
-      return launch_out<KLD_F16>(base, quant, norms, N, V, grad, grad_dtype, scale, sm_count, stream);
+      return launch_out<KLD_F16>(base, quant, aux, N, V, grad, grad_dtype, scale, sm_count, stream);
   }
   return cudaErrorInvalidValue;
 }

@@ -52,12 +52,24 @@ constexpr int kReduceThreads = 1024;
 
 inline int elem_bytes(kld_dtype_t dt) { return dt == KLD_F32 ? 4 : 2; }
 
+// Per-row normalisers the row pass leaves for the gradient and top-k passes
+// (48 bytes; the first 16 are read as a float4 by the gradient pass).
+struct RowAux {
+  float Fb, mb, Fq, mq;  // softmax(b)_j = 2^(b_j L - Fb) mb, softmax(q)_j likewise;
+                         // Fb NaN on rows excluded from the statistics
+  double lse_b;          // ln sum_j exp(lambda b_j)
+  double lr;             // log1p(B/S) = lse_q - lse_b + lambda K
+  float K;               // centre of the log-ratio x = q - b + K
+  uint32_t flags;        // the row's KLD_ROW_* flags
+  uint64_t pad;
+};
+static_assert(sizeof(RowAux) == 48, "RowAux layout");
+
 // Launchers (defined in the .cu files). They enqueue on `stream` and return
 // the launch error.
 // Row pass. With split == nullptr every CTA handles whole rows; otherwise
 // few-row launches spread each row over clusters of CTAs (see RowPlan).
-// norms (nullable): per-row normalisers {Fb, mb, Fq, mq} for the gradient
-// pass (see launch_grad).
+// aux (nullable): per-row normalisers for the gradient and top-k passes.
 // part_out (nullable): vocabulary-slice mode, the row is columns
 // [col_offset, col_offset + V) of a wider vocabulary and each row's merged
 // 64-byte partial goes to part_out[r] instead of a record (see
@@ -65,7 +77,7 @@ inline int elem_bytes(kld_dtype_t dt) { return dt == KLD_F32 ? 4 : 2; }
 cudaError_t launch_rows(const void* base, const void* quant,
                         const int32_t* token_ids, int64_t N, int64_t V,
                         kld_dtype_t dtype, kld_row_t* rows, uint32_t* derr,
-                        int sm_count, const SplitScratch* split, float4* norms,
+                        int sm_count, const SplitScratch* split, RowAux* aux,
                         cudaStream_t stream, void* part_out = nullptr,
                         int64_t col_offset = 0);
 
@@ -92,9 +104,16 @@ cudaError_t prepare_rows_kernels();  // per-device attribute setup
 // Gradient pass: grad[i][j] = scale * (softmax(q_i)_j - softmax(b_i)_j)
 // from the per-row normalisers of the row pass (zero on excluded rows);
 // grad in grad_dtype, [N, V] row-major.
-cudaError_t launch_grad(const void* base, const void* quant, const float4* norms, int64_t N,
+cudaError_t launch_grad(const void* base, const void* quant, const RowAux* aux, int64_t N,
                         int64_t V, kld_dtype_t dtype, void* grad, kld_dtype_t grad_dtype,
                         float scale, int sm_count, cudaStream_t stream);
+
+// Top-k compression of the base rows and KL of the quant rows against it
+// (k <= kMaxTopk), from the row pass's RowAux; idx, logp, rest nullable.
+constexpr int kMaxTopk = 1024;
+cudaError_t launch_topk(const void* base, const void* quant, const RowAux* aux, int64_t N,
+                        int64_t V, kld_dtype_t dtype, int k, int32_t* idx, float* logp,
+                        float* rest, double* kl, int sm_count, cudaStream_t stream);
 
 cudaError_t launch_reduce(const kld_row_t* rows, int64_t N, int has_nll,
                           uint32_t* derr, kld_result_t* out,

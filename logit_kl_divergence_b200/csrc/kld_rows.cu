@@ -853,23 +853,36 @@ __device__ kld_row_t finalize_row(const MPart& m, bool has_tok, bool tok_ok, flo
   return rec;
 }
 
-// Per-row normalisers for the gradient pass, from the merged partial:
-// softmax(lambda*b)_j = 2^(b_j*L - Fb) * mb and softmax(lambda*q)_j =
-// 2^(q_j*L - Fq) * mq, with integer frames Fb = floor(log2 of the base sum),
-// Fq likewise, and mb, mq in (0.5, 1] (so the exponents stay small near the
-// row maximum and every value keeps fp32 accuracy). NaN frames mark rows
-// excluded from the statistics (their gradient is zero).
-__device__ float4 row_norms(const MPart& m, const kld_row_t& rec) {
+// Per-row normalisers for the gradient and top-k passes, from the merged
+// partial: softmax(lambda*b)_j = 2^(b_j*L - Fb) * mb and softmax(lambda*q)_j
+// = 2^(q_j*L - Fq) * mq, with integer frames Fb = floor(log2 of the base
+// sum), Fq likewise, and mb, mq in (0.5, 1] (so the exponents stay small
+// near the row maximum and every value keeps fp32 accuracy); the base
+// log-normaliser and log1p(B/S) in fp64 for the top-k KL. A NaN Fb marks a
+// row excluded from the statistics.
+__device__ RowAux row_aux(const MPart& m, const kld_row_t& rec) {
+  RowAux a;
+  a.flags = rec.flags;
+  a.pad = 0ull;
+  a.K = m.K;
   if (rec.flags & (KLD_ROW_NONFINITE | KLD_ROW_EMPTY)) {
     const float nan = __int_as_float(0x7fc00000);
-    return make_float4(nan, 0.f, nan, 0.f);
+    a.Fb = a.Fq = nan;
+    a.mb = a.mq = 0.f;
+    a.lse_b = a.lr = __longlong_as_double(0x7ff8000000000000ll);
+    return a;
   }
   const double cb = log2(m.Sb) + static_cast<double>(m.Cb);
   const double cq = log2(m.B + m.Sb) + static_cast<double>(m.Cb) -
                     static_cast<double>(m.K) * kLog2eD;
   const double fb = floor(cb), fq = floor(cq);
-  return make_float4(static_cast<float>(fb), static_cast<float>(exp2(fb - cb)),
-                     static_cast<float>(fq), static_cast<float>(exp2(fq - cq)));
+  a.Fb = static_cast<float>(fb);
+  a.mb = static_cast<float>(exp2(fb - cb));
+  a.Fq = static_cast<float>(fq);
+  a.mq = static_cast<float>(exp2(fq - cq));
+  a.lse_b = cb * kLn2;
+  a.lr = log1p(m.B / m.Sb);
+  return a;
 }
 
 __device__ __forceinline__ uint32_t cluster_ctarank() {
@@ -893,7 +906,7 @@ __global__ void __launch_bounds__(kRowThreads, 1)
     kld_rows_kernel(const void* __restrict__ base, const void* __restrict__ quant,
                     const int32_t* __restrict__ tok, int64_t N, int64_t V,
                     kld_row_t* __restrict__ rows, uint32_t* __restrict__ derr, int P,
-                    MPart* __restrict__ gparts, unsigned* __restrict__ tickets, float4* __restrict__ norms,
+                    MPart* __restrict__ gparts, unsigned* __restrict__ tickets, RowAux* __restrict__ aux,
                     MPart* __restrict__ part_out, int64_t col0) {
   constexpr int EB = Elem<DT>::kBytes;
   constexpr int E = Elem<DT>::kPerVec;
@@ -1264,7 +1277,7 @@ __global__ void __launch_bounds__(kRowThreads, 1)
         const kld_row_t rec = finalize_row(m, tok != nullptr, tok_ok, q_tok, b_tok);
         if (lane == 0) {
           rows[r] = rec;
-          if (norms != nullptr) norms[r] = row_norms(m, rec);
+          if (aux != nullptr) aux[r] = row_aux(m, rec);
         }
         continue;
       }
@@ -1338,7 +1351,7 @@ __global__ void __launch_bounds__(kRowThreads, 1)
         const kld_row_t rec = finalize_row(cm, tok != nullptr, tok_ok, q_tok, b_tok);
         if (lane == 0) {
           rows[r] = rec;
-          if (norms != nullptr) norms[r] = row_norms(cm, rec);
+          if (aux != nullptr) aux[r] = row_aux(cm, rec);
         }
         continue;
       }
@@ -1373,7 +1386,7 @@ __global__ void __launch_bounds__(kRowThreads, 1)
       const kld_row_t rec = finalize_row(fm, tok != nullptr, tok_ok, q_tok, b_tok);
       if (lane == 0) {
         rows[r] = rec;
-        if (norms != nullptr) norms[r] = row_norms(fm, rec);
+        if (aux != nullptr) aux[r] = row_aux(fm, rec);
         tickets[r] = 0u;  // ready for the next launch
       }
     }
@@ -1452,7 +1465,7 @@ int max_active_clusters(int cluster_ctas) {
 template <int DT>
 cudaError_t launch_typed(const void* base, const void* quant, const int32_t* tok, int64_t N,
                          int64_t V, kld_row_t* rows, uint32_t* derr, const RowPlan& pl,
-                         const SplitScratch* split, float4* norms, MPart* part_out, int64_t col0,
+                         const SplitScratch* split, RowAux* aux, MPart* part_out, int64_t col0,
                          cudaStream_t stream) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(pl.grid));
@@ -1469,7 +1482,7 @@ cudaError_t launch_typed(const void* base, const void* quant, const int32_t* tok
   MPart* gp = split ? static_cast<MPart*>(split->parts) : nullptr;
   unsigned* tk = split ? split->tickets : nullptr;
   return cudaLaunchKernelEx(&cfg, kld_rows_kernel<DT>, base, quant, tok, N, V, rows, derr,
-                            pl.parts_per_row, gp, tk, norms, part_out, col0);
+                            pl.parts_per_row, gp, tk, aux, part_out, col0);
 }
 
 }  // namespace
@@ -1542,7 +1555,7 @@ cudaError_t launch_merge(const void* parts, int G, int64_t N, const int32_t* tok
 
 cudaError_t launch_rows(const void* base, const void* quant, const int32_t* token_ids, int64_t N,
                         int64_t V, kld_dtype_t dtype, kld_row_t* rows, uint32_t* derr,
-                        int sm_count, const SplitScratch* split, float4* norms,
+                        int sm_count, const SplitScratch* split, RowAux* aux,
                         cudaStream_t stream, void* part_out, int64_t col_offset) {
   RowPlan pl = plan_rows(N, sm_count, nullptr, 0);
   // Vocabulary-slice partials come from whole-row launches only.
@@ -1556,13 +1569,13 @@ cudaError_t launch_rows(const void* base, const void* quant, const int32_t* toke
   }
   switch (dtype) {
     case KLD_F32:
-      return launch_typed<KLD_F32>(base, quant, token_ids, N, V, rows, derr, pl, split, norms,
+      return launch_typed<KLD_F32>(base, quant, token_ids, N, V, rows, derr, pl, split, aux,
                                  static_cast<MPart*>(part_out), col_offset, stream);
     case KLD_BF16:
-      return launch_typed<KLD_BF16>(base, quant, token_ids, N, V, rows, derr, pl, split, norms,
+      return launch_typed<KLD_BF16>(base, quant, token_ids, N, V, rows, derr, pl, split, aux,
                                  static_cast<MPart*>(part_out), col_offset, stream);
     case KLD_F16:
-      return launch_typed<KLD_F16>(base, quant, token_ids, N, V, rows, derr, pl, split, norms,
+      return launch_typed<KLD_F16>(base, quant, token_ids, N, V, rows, derr, pl, split, aux,
                                  static_cast<MPart*>(part_out), col_offset, stream);
   }
   return cudaErrorInvalidValue;

@@ -1,0 +1,354 @@
+// kld_topk.cu -- top-k compression of the base row and the KL of the quant
+// row against it ("Mistral-Small-4-119B-2603 GSQ-RCO IQ3_S GGUF", "How it
+// was made", step 7: tuning "against the top-128 distributions (and the rest
+// of the mass)").
+//
+// Per row, T = the k largest base logits (ties to the lowest index), listed
+// in that order with log P_base, plus log of the rest mass, and
+//   KL_topk = sum_{j in T} p_j log(p_j / r_j) + p_rest log(p_rest / r_rest).
+// Runs after the row pass, which leaves each row's normalisers (RowAux:
+// lse_b, log1p(B/S), the centre K and fp32 frames) so that, for j in T,
+//   log p_j = lambda*b_j - lse_b,  log(p_j / r_j) = log1p(B/S) - lambda*x_j,
+// x_j = (q_j - b_j) + K rounded to fp32 as the row pass rounds it, the rest
+// in fp64.
+//
+// One CTA per row (persistent over rows): the k-th largest key of the base
+// row is found by an MSB radix select over order-preserving 32-bit keys
+// (11/11/10-bit levels, a shared histogram per level, stopping as soon as the
+// candidates fit in shared memory); if a tie group at the threshold is larger
+// than that, the lowest indices in it are found by a radix select over the
+// index. The candidates (at most kCap) are sorted in shared memory by (key
+// desc, index asc). A last pass over the row sums the rest mass of both rows.
+// The row is read 2-4 times, from L2 after the first.
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include <climits>
+
+#include "kld_internal.h"
+
+namespace kld {
+namespace {
+
+constexpr int kTopkThreads = 512;
+constexpr int kTopkWarps = kTopkThreads / 32;
+constexpr int kHistBins = 2048;
+constexpr int kCap = 4096;  // candidates sorted in shared memory
+constexpr float kL = 1.4426950408889634f;  // log2(e) rounded to fp32, as the row pass
+constexpr double kLn2 = 0.6931471805599453;
+
+template <int DT>
+__device__ __forceinline__ float load_el(const char* row, int64_t j);
+template <>
+__device__ __forceinline__ float load_el<KLD_F32>(const char* row, int64_t j) {
+  return __ldg(reinterpret_cast<const float*>(row) + j);
+}
+template <>
+__device__ __forceinline__ float load_el<KLD_BF16>(const char* row, int64_t j) {
+  return __uint_as_float(static_cast<uint32_t>(__ldg(reinterpret_cast<const unsigned short*>(row) + j)) << 16);
+}
+template <>
+__device__ __forceinline__ float load_el<KLD_F16>(const char* row, int64_t j) {
+  return __half2float(__ushort_as_half(__ldg(reinterpret_cast<const unsigned short*>(row) + j)));
+}
+
+// Order-preserving key of a float (larger float, larger key).
+__device__ __forceinline__ uint32_t okey(float x) {
+  const uint32_t u = __float_as_uint(x);
+  return (u >> 31) ? ~u : (u | 0x80000000u);
+}
+
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+struct TopkShared {
+  unsigned hist[kHistBins];
+  unsigned long long cand[kCap];
+  double red[kTopkWarps][4];
+  int ncand;
+  unsigned sel[3];  // bin, count above it, count in it
+};
+
+// Block-wide: the bin holding the `need`-th element counting from the top
+// (descending = true) or the bottom of hist[0..bins). Returns (bin, count
+// before it in that direction, count in it) through sh.sel.
+__device__ void find_bin(TopkShared& sh, int bins, unsigned need, bool descending) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (warp == 0) {
+    const int per = bins / 32;  // bins per lane, contiguous in scan order
+    unsigned part = 0;
+    for (int i = 0; i < per; ++i) {
+      const int b = descending ? bins - 1 - (lane * per + i) : lane * per + i;
+      part += sh.hist[b];
+    }
+    unsigned incl = part;  // inclusive prefix over lanes
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const unsigned v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    const unsigned excl = incl - part;
+    const unsigned hit = __ballot_sync(0xffffffffu, excl < need && incl >= need);
+    const int owner = hit ? __ffs(hit) - 1 : 31;
+    if (lane == owner) {
+      unsigned cum = excl;
+      int bin = descending ? bins - 1 - lane * per : lane * per;
+      for (int i = 0; i < per; ++i) {
+        const int b = descending ? bins - 1 - (lane * per + i) : lane * per + i;
+        bin = b;
+        if (cum + sh.hist[b] >= need) break;
+        cum += sh.hist[b];
+      }
+      sh.sel[0] = static_cast<unsigned>(bin);
+      sh.sel[1] = cum;
+      sh.sel[2] = sh.hist[bin];
+    }
+  }
+  __syncthreads();
+}
+
+__device__ double block_sum(TopkShared& sh, double v, int slot) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_down_sync(0xffffffffu, v, o);
+  if (lane == 0) sh.red[warp][slot] = v;
+  __syncthreads();
+  double t = 0.0;
+  for (int w = 0; w < kTopkWarps; ++w) t += sh.red[w][slot];  // fixed order
+  __syncthreads();
+  return t;
+}
+
+template <int DT>
+__global__ void __launch_bounds__(kTopkThreads)
+    kld_topk_kernel(const void* __restrict__ base, const void* __restrict__ quant,
+                    const RowAux* __restrict__ aux, int64_t N, int64_t V, int k,
+                    int32_t* __restrict__ idx_out, float* __restrict__ logp_out,
+                    float* __restrict__ rest_out, double* __restrict__ kl_out) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  TopkShared& sh = *reinterpret_cast<TopkShared*>(smem_raw);
+  constexpr int EB = DT == KLD_F32 ? 4 : 2;
+  const double lambda = static_cast<double>(kL) * kLn2;
+  const float nanf = __int_as_float(0x7fc00000);
+  const int tid = threadIdx.x;
+  const int kt = static_cast<int>(V < k ? V : k);
+
+  for (int64_t r = blockIdx.x; r < N; r += gridDim.x) {
+    const char* rb = static_cast<const char*>(base) + r * V * EB;
+    const char* rq = static_cast<const char*>(quant) + r * V * EB;
+    const RowAux a = aux[r];
+    if (isnan(a.Fb)) {  // excluded row
+      for (int i = tid; i < k; i += kTopkThreads) {
+        if (idx_out) idx_out[r * k + i] = -1;
+        if (logp_out) logp_out[r * k + i] = nanf;
+      }
+      if (tid == 0) {
+        if (rest_out) rest_out[r] = nanf;
+        kl_out[r] = __longlong_as_double(0x7ff8000000000000ll);
+      }
+      continue;
+    }
+
+    // ---- threshold key: MSB radix select for the kt-th largest key
+    uint32_t prefix = 0u, mask = 0u;
+    unsigned need = static_cast<unsigned>(kt);
+    unsigned ncount = static_cast<unsigned>(V);  // elements matching the prefix
+    const int shifts[3] = {21, 10, 0}, widths[3] = {11, 11, 10};
+    int levels = 0;
+    for (; levels < 3; ++levels) {
+      if ((static_cast<unsigned>(kt) - need) + ncount <= static_cast<unsigned>(kCap)) break;
+      const int sh_ = shifts[levels], bins = 1 << widths[levels];
+      for (int i = tid; i < kHistBins; i += kTopkThreads) sh.hist[i] = 0u;
+      __syncthreads();
+      // warp-aggregated shared atomics: the bins of a row are few and crowded
+      for (int64_t j0 = 0; j0 < V; j0 += kTopkThreads) {
+        const int64_t j = j0 + tid;
+        int bin = -1;
+        if (j < V) {
+          const uint32_t key = okey(load_el<DT>(rb, j));
+          if ((key & mask) == prefix) bin = static_cast<int>((key >> sh_) & (bins - 1));
+        }
+        const unsigned peers = __match_any_sync(0xffffffffu, bin);
+        if (bin >= 0 && (tid & 31) == __ffs(peers) - 1) atomicAdd(&sh.hist[bin], __popc(peers));
+      }
+      __syncthreads();
+      find_bin(sh, bins, need, true);
+      const unsigned bin = sh.sel[0], above = sh.sel[1], inbin = sh.sel[2];
+      __syncthreads();
+      need -= above;
+      prefix |= bin << sh_;
+      mask |= static_cast<uint32_t>(bins - 1) << sh_;
+      ncount = inbin;
+    }
+
+    // ---- collect the candidates
+    if (tid == 0) sh.ncand = 0;
+    __syncthreads();
+    if ((static_cast<unsigned>(kt) - need) + ncount <= static_cast<unsigned>(kCap)) {
+      // every element above the prefix, and every element in it
+      for (int64_t j = tid; j < V; j += kTopkThreads) {
+        const uint32_t key = okey(load_el<DT>(rb, j));
+        if ((key & mask) >= prefix) {
+          const int pos = atomicAdd(&sh.ncand, 1);
+          sh.cand[pos] = (static_cast<unsigned long long>(key) << 32) | (0xffffffffu - static_cast<uint32_t>(j));
+        }
+      }
+    } else {
+      // all 32 key bits fixed and a tie group too large to sort: the `need`
+      // lowest indices among keys equal to the threshold (radix select on the
+      // index from the bottom), then every key above it
+      const uint32_t tau = prefix;
+      uint32_t jp = 0u, jm = 0u;
+      unsigned jneed = need;
+      const int jshifts[3] = {20, 10, 0}, jwidths[3] = {11, 10, 10};
+      for (int lv = 0; lv < 3; ++lv) {
+        const int sh_ = jshifts[lv], bins = 1 << jwidths[lv];
+        for (int i = tid; i < kHistBins; i += kTopkThreads) sh.hist[i] = 0u;
+        __syncthreads();
+        for (int64_t j0 = 0; j0 < V; j0 += kTopkThreads) {
+          const int64_t j = j0 + tid;
+          int bin = -1;
+          if (j < V) {
+            const uint32_t uj = static_cast<uint32_t>(j);
+            if ((uj & jm) == jp && okey(load_el<DT>(rb, j)) == tau)
+              bin = static_cast<int>((uj >> sh_) & (bins - 1));
+          }
+          const unsigned peers = __match_any_sync(0xffffffffu, bin);
+          if (bin >= 0 && (tid & 31) == __ffs(peers) - 1) atomicAdd(&sh.hist[bin], __popc(peers));
+        }
+        __syncthreads();
+        find_bin(sh, bins, jneed, false);
+        const unsigned bin = sh.sel[0], below = sh.sel[1];
+        __syncthreads();
+        jneed -= below;
+        jp |= bin << sh_;
+        jm |= static_cast<uint32_t>(bins - 1) << sh_;
+      }
+      const uint32_t jlast = jp;  // the need-th lowest index with key == tau
+      for (int64_t j = tid; j < V; j += kTopkThreads) {
+        const uint32_t key = okey(load_el<DT>(rb, j));
+        if (key > tau || (key == tau && static_cast<uint32_t>(j) <= jlast)) {
+          const int pos = atomicAdd(&sh.ncand, 1);
+          sh.cand[pos] = (static_cast<unsigned long long>(key) << 32) | (0xffffffffu - static_cast<uint32_t>(j));
+        }
+      }
+    }
+    __syncthreads();
+
+    // ---- sort the candidates descending (bitonic), zeros pad to a power of 2
+    const int n = sh.ncand;
+    int p2 = 1;
+    while (p2 < n) p2 <<= 1;
+    for (int i = n + tid; i < p2; i += kTopkThreads) sh.cand[i] = 0ull;
+    __syncthreads();
+    for (int kk = 2; kk <= p2; kk <<= 1) {
+      for (int jj = kk >> 1; jj > 0; jj >>= 1) {
+        for (int i = tid; i < p2; i += kTopkThreads) {
+          const int ixj = i ^ jj;
+          if (ixj > i) {
+            const unsigned long long x = sh.cand[i], y = sh.cand[ixj];
+            const bool desc = (i & kk) == 0;
+            if (desc ? (x < y) : (x > y)) {
+              sh.cand[i] = y;
+              sh.cand[ixj] = x;
+            }
+          }
+        }
+        __syncthreads();
+      }
+    }
+
+    // ---- T: log P_base and the KL terms
+    double kl_t = 0.0, inf_t = 0.0;
+    for (int i = tid; i < k; i += kTopkThreads) {
+      if (i < kt) {
+        const uint32_t j = 0xffffffffu - static_cast<uint32_t>(sh.cand[i]);
+        const float bj = load_el<DT>(rb, j), qj = load_el<DT>(rq, j);
+        const double lp = lambda * static_cast<double>(bj) - a.lse_b;
+        if (idx_out) idx_out[r * k + i] = static_cast<int32_t>(j);
+        if (logp_out) logp_out[r * k + i] = static_cast<float>(lp);
+        if (bj != -INFINITY) {
+          if (qj == -INFINITY) {
+            inf_t = 1.0;
+          } else {
+            // x rounded exactly as the row pass rounds it, so that it agrees
+            // with the log1p(B/S) that pass summed from the same values (an
+            // exact x would leave their mean rounding error, ~1e-6 for a
+            // quant row offset from the base by 1000, in the result)
+            const float x = __fadd_rn(__fsub_rn(qj, bj), a.K);
+            const double lratio = a.lr - lambda * static_cast<double>(x);  // log p_j - log r_j
+            kl_t += exp(lp) * lratio;
+          }
+        }
+      } else {
+        if (idx_out) idx_out[r * k + i] = -1;
+        if (logp_out) logp_out[r * k + i] = -INFINITY;
+      }
+    }
+    // membership of T: key above the last selected, or equal with an index
+    // no larger than its
+    const unsigned long long last = sh.cand[kt - 1];
+    const uint32_t tau_f = static_cast<uint32_t>(last >> 32);
+    const uint32_t j_f = 0xffffffffu - static_cast<uint32_t>(last);
+    double prest = 0.0, rrest = 0.0;
+    for (int64_t j = tid; j < V; j += kTopkThreads) {
+      const float bj = load_el<DT>(rb, j);
+      const uint32_t key = okey(bj);
+      if (key > tau_f || (key == tau_f && static_cast<uint32_t>(j) <= j_f)) continue;
+      const float qj = load_el<DT>(rq, j);
+      prest += static_cast<double>(__fmul_rn(ex2(fmaf(bj, kL, -a.Fb)), a.mb));
+      rrest += static_cast<double>(__fmul_rn(ex2(fmaf(qj, kL, -a.Fq)), a.mq));
+    }
+    __syncthreads();  // everyone is done with cand before the next row reuses it
+    kl_t = block_sum(sh, kl_t, 0);
+    inf_t = block_sum(sh, inf_t, 1);
+    prest = block_sum(sh, prest, 2);
+    rrest = block_sum(sh, rrest, 3);
+    if (tid == 0) {
+      double kl = kl_t;
+      bool inf = inf_t > 0.0;
+      if (prest > 0.0) {
+        if (rrest > 0.0)
+          kl += prest * (log(prest) - log(rrest));
+        else
+          inf = true;
+      }
+      if (rest_out) rest_out[r] = prest > 0.0 ? static_cast<float>(log(prest)) : -INFINITY;
+      kl_out[r] = inf ? INFINITY : kl;
+    }
+  }
+}
+
+template <int DT>
+cudaError_t launch_typed(const void* base, const void* quant, const RowAux* aux, int64_t N,
+                         int64_t V, int k, int32_t* idx, float* logp, float* rest, double* kl,
+                         int sm_count, cudaStream_t s) {
+  const size_t smem = sizeof(TopkShared);
+  cudaError_t e = cudaFuncSetAttribute(kld_topk_kernel<DT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  int64_t grid = static_cast<int64_t>(sm_count) * 4;
+  if (grid > N) grid = N;
+  kld_topk_kernel<DT><<<static_cast<unsigned>(grid), kTopkThreads, smem, s>>>(base, quant, aux, N, V, k,
+                                                                            idx, logp, rest, kl);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_topk(const void* base, const void* quant, const RowAux* aux, int64_t N,
+                        int64_t V, kld_dtype_t dtype, int k, int32_t* idx, float* logp,
+                        float* rest, double* kl, int sm_count, cudaStream_t stream) {
+  if (k < 1 || k > kMaxTopk) return cudaErrorInvalidValue;
+  switch (dtype) {
+    case KLD_F32: return launch_typed<KLD_F32>(base, quant, aux, N, V, k, idx, logp, rest, kl, sm_count, stream);
+    case KLD_BF16: return launch_typed<KLD_BF16>(base, quant, aux, N, V, k, idx, logp, rest, kl, sm_count, stream);
+    case KLD_F16: return launch_typed<KLD_F16>(base, quant, aux, N, V, k, idx, logp, rest, kl, sm_count, stream);
+  }
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace kld
