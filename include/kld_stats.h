@@ -95,7 +95,7 @@ typedef struct {
   int32_t argmax_base;   /* lowest index of the row maximum, -1 if excluded */
   int32_t argmax_quant;
   uint32_t flags;        /* KLD_ROW_* bits                                  */
-  uint32_t reserved;
+  float dp;              /* P_quant(tok) - P_base(tok) (NaN if no/bad token) */
 } kld_row_t;
 
 /* Summary statistics (caller-owned plain struct). */

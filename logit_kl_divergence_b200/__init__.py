@@ -71,8 +71,9 @@ def rows_view(records: torch.Tensor) -> dict:
     r = records.view(torch.uint8).reshape(-1, ROW_RECORD_BYTES)
     f64 = r[:, :24].contiguous().view(torch.float64)
     i32 = r[:, 24:36].contiguous().view(torch.int32)
+    f32 = r[:, 36:40].contiguous().view(torch.float32)
     return {"kld": f64[:, 0], "nll": f64[:, 1], "nll_base": f64[:, 2], "amax_b": i32[:, 0],
-            "amax_q": i32[:, 1], "flags": i32[:, 2]}
+            "amax_q": i32[:, 1], "flags": i32[:, 2], "dp": f32[:, 0]}
 
 
 class KLDStats:

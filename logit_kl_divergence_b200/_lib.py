@@ -45,7 +45,7 @@ class Row(ctypes.Structure):
         ("argmax_base", ctypes.c_int32),
         ("argmax_quant", ctypes.c_int32),
         ("flags", ctypes.c_uint32),
-        ("reserved", ctypes.c_uint32),
+        ("dp", ctypes.c_float),
     ]
 
 

@@ -10,7 +10,8 @@
 //   PPL        = exp(mean NLL), and the same for the base model's NLL,
 //   ln ratio   = mean NLL - mean base NLL = ln(PPL(Q) / PPL(base)),
 //   dp         = exp(-NLL) - exp(-base NLL) = P_quant(tok) - P_base(tok) per
-//                row; its mean and sqrt(mean dp^2) ("Mistral-Small-4-119B-2603
+//                row (in the record, from the row pass); its mean and
+//                sqrt(mean dp^2) ("Mistral-Small-4-119B-2603
 //                GSQ-RCO IQ3_S GGUF", "Quality"; the Qwen3.6 table's RMS dp),
 //   percentile = x_(k) + (pos - k) * (x_(k+1) - x_(k)),  pos = p*(n-1),
 //                k = floor(pos), over the sorted valid KL values; max = x_(n-1).
@@ -34,6 +35,7 @@ namespace kld {
 namespace {
 
 constexpr int kTargets = 7;
+constexpr int kAhead = 4;  // records each thread loads before using them
 constexpr int kGatherCap = 4096;
 constexpr uint32_t kExcluded = KLD_ROW_NONFINITE | KLD_ROW_EMPTY;
 
@@ -88,21 +90,32 @@ __global__ void __launch_bounds__(kReduceThreads, 1)
   double s_kl = 0.0, s_nll = 0.0, s_nllb = 0.0, s_dp = 0.0, s_dp2 = 0.0;
   long long n_valid = 0, agree = 0, n_nll = 0, n_flag = 0;
   unsigned int f_or = 0;
-  for (int64_t i = tid; i < N; i += nt) {
-    const kld_row_t rec = rows[i];
-    f_or |= rec.flags;
-    if (rec.flags) ++n_flag;
-    if (rec.flags & kExcluded) continue;
-    ++n_valid;
-    s_kl += rec.kld;
-    if (rec.argmax_base == rec.argmax_quant) ++agree;
-    if (has_nll && !(rec.flags & KLD_ROW_BAD_TOKEN)) {
-      s_nll += rec.nll;
-      s_nllb += rec.nll_base;
-      const double dp = exp(-rec.nll) - exp(-rec.nll_base);
-      s_dp += dp;
-      s_dp2 += dp * dp;
-      ++n_nll;
+  // Records t, t + T, ... in order; kAhead loads in flight per thread.
+  for (int64_t i0 = tid; i0 < N; i0 += static_cast<int64_t>(kAhead) * nt) {
+    kld_row_t rec[kAhead];
+#pragma unroll
+    for (int u = 0; u < kAhead; ++u) {
+      const int64_t i = i0 + static_cast<int64_t>(u) * nt;
+      if (i < N) rec[u] = rows[i];
+    }
+#pragma unroll
+    for (int u = 0; u < kAhead; ++u) {
+      if (i0 + static_cast<int64_t>(u) * nt >= N) break;
+      const kld_row_t& rc = rec[u];
+      f_or |= rc.flags;
+      if (rc.flags) ++n_flag;
+      if (rc.flags & kExcluded) continue;
+      ++n_valid;
+      s_kl += rc.kld;
+      if (rc.argmax_base == rc.argmax_quant) ++agree;
+      if (has_nll && !(rc.flags & KLD_ROW_BAD_TOKEN)) {
+        s_nll += rc.nll;
+        s_nllb += rc.nll_base;
+        const double dp = static_cast<double>(rc.dp);  // computed per row by the row pass
+        s_dp += dp;
+        s_dp2 += dp * dp;
+        ++n_nll;
+      }
     }
   }
 #pragma unroll
@@ -207,13 +220,24 @@ __global__ void __launch_bounds__(kReduceThreads, 1)
       for (int i = tid; i < ng * 256; i += nt) (&sh.hist[0][0])[i] = 0u;
       __syncthreads();
       const uint64_t himask = decided == 0 ? 0ull : (~0ull << (64 - decided));
-      for (int64_t base_i = 0; base_i < N; base_i += nt) {
-        const int64_t i = base_i + tid;
-        int slot = -1;
-        if (i < N) {
-          const kld_row_t rec = rows[i];
-          if (!(rec.flags & kExcluded)) {
-            const uint64_t key = order_key(rec.kld);
+      // four records per thread in flight, then the warp-aggregated counts
+      for (int64_t base_i = 0; base_i < N; base_i += static_cast<int64_t>(kAhead) * nt) {
+        double kv[kAhead];
+        uint32_t fv[kAhead];
+#pragma unroll
+        for (int u = 0; u < kAhead; ++u) {
+          const int64_t i = base_i + static_cast<int64_t>(u) * nt + tid;
+          fv[u] = kExcluded;
+          if (i < N) {
+            fv[u] = rows[i].flags;
+            kv[u] = rows[i].kld;
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < kAhead; ++u) {
+          int slot = -1;
+          if (!(fv[u] & kExcluded)) {
+            const uint64_t key = order_key(kv[u]);
             for (int g = 0; g < ng; ++g) {
               if (((key ^ sh.gprefix[g]) & himask) == 0ull) {
                 slot = g * 256 + static_cast<int>((key >> shift) & 0xffu);
@@ -221,26 +245,42 @@ __global__ void __launch_bounds__(kReduceThreads, 1)
               }
             }
           }
+          const unsigned peers = __match_any_sync(0xffffffffu, slot);
+          if (slot >= 0 && lane == __ffs(peers) - 1)
+            atomicAdd(&(&sh.hist[0][0])[slot], static_cast<unsigned>(__popc(peers)));
         }
-        const unsigned peers = __match_any_sync(0xffffffffu, slot);
-        if (slot >= 0 && lane == __ffs(peers) - 1)
-          atomicAdd(&(&sh.hist[0][0])[slot], static_cast<unsigned>(__popc(peers)));
       }
       __syncthreads();
-      if (tid < kTargets) {
-        const int g = sh.tgroup[tid];
-        unsigned long long r = sh.rank[tid];
-        unsigned long long before = 0;
-        int bin = 0;
-        for (; bin < 256; ++bin) {
-          const unsigned long long c = sh.hist[g][bin];
-          if (r < before + c) break;
-          before += c;
+      for (int t = warp; t < kTargets; t += nt >> 5) {
+        // One warp per target: 8 bins per lane, a warp prefix scan, then the
+        // lane holding the rank finds its bin.
+        const int g = sh.tgroup[t];
+        const unsigned long long r = sh.rank[t];
+        unsigned long long part = 0;
+#pragma unroll
+        for (int b = 0; b < 8; ++b) part += sh.hist[g][lane * 8 + b];
+        unsigned long long incl = part;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const unsigned long long v = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += v;
         }
-        if (bin > 255) bin = 255;  // unreachable for consistent counts
-        sh.prefix[tid] = sh.gprefix[g] | (static_cast<unsigned long long>(bin) << shift);
-        sh.rank[tid] = r - before;
-        sh.gcount[tid] = sh.hist[g][bin];  // temporarily per target
+        const unsigned long long excl = incl - part;
+        const unsigned hit = __ballot_sync(0xffffffffu, r >= excl && r < incl);
+        const int owner = hit ? __ffs(hit) - 1 : 31;  // 31: unreachable for consistent counts
+        if (lane == owner) {
+          unsigned long long before = excl;
+          int bin = lane * 8;
+          for (int b = 0; b < 8; ++b) {
+            bin = lane * 8 + b;
+            const unsigned long long c = sh.hist[g][bin];
+            if (r < before + c) break;
+            before += c;
+          }
+          sh.prefix[t] = sh.gprefix[g] | (static_cast<unsigned long long>(bin) << shift);
+          sh.rank[t] = r - before;
+          sh.gcount[t] = sh.hist[g][bin];  // temporarily per target
+        }
       }
       __syncthreads();
       if (tid == 0) {
@@ -271,16 +311,23 @@ __global__ void __launch_bounds__(kReduceThreads, 1)
       __syncthreads();
       const uint64_t himask = decided == 0 ? 0ull : (~0ull << (64 - decided));
       const int ng = sh.ngroups;
-      for (int64_t i = tid; i < N; i += nt) {
-        const kld_row_t rec = rows[i];
-        if (rec.flags & kExcluded) continue;
-        const uint64_t key = order_key(rec.kld);
-        for (int g = 0; g < ng; ++g) {
-          if (((key ^ sh.gprefix[g]) & himask) == 0ull) {
-            const int pos = atomicAdd(&sh.ncand, 1);
-            if (pos < kGatherCap) sh.cand[pos] = key;
-            break;
-          }
+      for (int64_t base_i = 0; base_i < N; base_i += nt) {
+        const int64_t i = base_i + tid;
+        bool take = false;
+        uint64_t key = 0;
+        if (i < N && !(rows[i].flags & kExcluded)) {
+          key = order_key(rows[i].kld);
+          for (int g = 0; g < ng; ++g)
+            if (((key ^ sh.gprefix[g]) & himask) == 0ull) take = true;
+        }
+        // one shared atomic per warp
+        const unsigned m = __ballot_sync(0xffffffffu, take);
+        int basepos = 0;
+        if (lane == 0 && m) basepos = atomicAdd(&sh.ncand, __popc(m));
+        basepos = __shfl_sync(0xffffffffu, basepos, 0);
+        if (take) {
+          const int pos = basepos + __popc(m & ((1u << lane) - 1u));
+          if (pos < kGatherCap) sh.cand[pos] = key;
         }
       }
       __syncthreads();

@@ -849,7 +849,8 @@ __device__ kld_row_t finalize_row(const MPart& m, bool has_tok, bool tok_ok, flo
     rec.argmax_quant = m.amax_q;
   }
   rec.flags = flags;
-  rec.reserved = 0u;
+  // P(tok) = exp(-NLL) for each model (exp(-inf) = 0), differenced in fp64
+  rec.dp = static_cast<float>(exp(-rec.nll) - exp(-rec.nll_base));
   return rec;
 }
 

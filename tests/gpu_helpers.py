@@ -66,6 +66,13 @@ def _close_rows(g, o, what, idx):
         raise AssertionError(f"{what} mismatch at rows {idx[bad]}: gpu={g[bad]} ref={o[bad]}")
 
 
+def _close_dp(g, o, tol, idx):
+    ok = (np.isnan(g) & np.isnan(o)) | (np.abs(g - o) <= tol + 6e-8 * np.abs(o))
+    if not ok.all():
+        bad = np.nonzero(~ok)[0][:8]
+        raise AssertionError(f"dp mismatch at rows {idx[bad]}: gpu={g[bad]} ref={o[bad]}")
+
+
 def assert_rows_match(g: dict, o: dict, idx=None):
     n = len(o["kld"])
     idx = np.arange(n) if idx is None else np.asarray(idx)
@@ -78,6 +85,15 @@ def assert_rows_match(g: dict, o: dict, idx=None):
     _close_rows(g["kld"], o["kld"], "kld", idx)
     _close_rows(g["nll"], o["nll"], "nll", idx)
     _close_rows(g["nll_base"], o["nll_base"], "nll_base", idx)
+    # dp = P_quant(tok) - P_base(tok), fp32 in the record: each NLL within its
+    # bar (ROW_ATOL + ROW_RTOL * NLL) moves its probability by that much
+    # relative, plus fp32 rounding
+    with np.errstate(invalid="ignore", over="ignore"):
+        nq, nb = np.asarray(o["nll"], np.float64), np.asarray(o["nll_base"], np.float64)
+        pq, pb = np.exp(-nq), np.exp(-nb)
+        tol = (pq * (ROW_ATOL + ROW_RTOL * np.nan_to_num(nq, posinf=0.0))
+               + pb * (ROW_ATOL + ROW_RTOL * np.nan_to_num(nb, posinf=0.0)) + 1e-12)
+    _close_dp(np.asarray(g["dp"], np.float64), pq - pb, tol, idx)
 
 
 def stat_close(a, b, key):

@@ -19,7 +19,7 @@ from logit_kl_divergence_b200 import rows_view, synth
 from logit_kl_divergence_b200.sharded import ShardedKLDStats, gather_records, shard_bounds
 
 RECORD = np.dtype([("kld", "<f8"), ("nll", "<f8"), ("nll_base", "<f8"), ("amax_b", "<i4"),
-                   ("amax_q", "<i4"), ("flags", "<u4"), ("reserved", "<u4")])
+                   ("amax_q", "<i4"), ("flags", "<u4"), ("dp", "<f4")])
 assert RECORD.itemsize == 40
 
 
@@ -27,6 +27,7 @@ def _pack(r: dict) -> np.ndarray:
     a = np.zeros(r["kld"].shape[0], dtype=RECORD)
     for k in ("kld", "nll", "nll_base", "amax_b", "amax_q", "flags"):
         a[k] = r[k]
+    a["dp"] = np.exp(-r["nll"]) - np.exp(-r["nll_base"])
     return a.view(np.uint8).reshape(-1, 40)
 
 
