@@ -293,6 +293,19 @@ kld_status_t kld_stats_run_topk(kld_stats_t h, const void* base, const void* qua
                                 float* rest_out, double* kl_out, void* stream);
 
 /*
+ * Self-test of failure detection (no counterpart on the source pages; a
+ * diagnostic of this library). Every device wait of the kernels is bounded:
+ * this runs one small kernel on `device` whose warp waits on an mbarrier
+ * that nothing ever completes, with a limit of limit_ns nanoseconds (1e3 ..
+ * 1e10) -- or, with use_abort, until a second warp raises the kernel's abort
+ * flag after ~1 ms -- and reports what the kernels report: KLD_ERR_TIMEOUT
+ * when the wait gave up (the expected outcome), with the time waited in
+ * *waited_ns. The context stays usable afterwards. Synchronous.
+ */
+kld_status_t kld_selftest_bounded_wait(int device, uint64_t limit_ns, int use_abort,
+                                       uint64_t* waited_ns);
+
+/*
  * Duration in milliseconds of the last kld_stats_run_grad's gradient pass
  * (timing enabled by kld_stats_set_timing; waits for that run).
  */

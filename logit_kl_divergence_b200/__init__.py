@@ -20,7 +20,7 @@ from ._lib import (KLD_BF16, KLD_F16, KLD_F32, ROW_BAD_TOKEN, ROW_EMPTY,  # noqa
                    ROW_INF_KL, ROW_INF_NLL, ROW_INF_NLL_BASE, ROW_NONFINITE, KLDError)
 
 __all__ = ["KLDStats", "kld_stats", "run_static", "result_from_bytes", "plan", "dtype_code",
-           "ROW_RECORD_BYTES"]
+           "ROW_RECORD_BYTES", "selftest_bounded_wait"]
 
 ROW_RECORD_BYTES = 40
 PARTIAL_BYTES = 64
@@ -302,6 +302,19 @@ def plan(n_rows: int, vocab: int, dtype: int, sm_count: int) -> dict:
     p = _lib.Plan()
     _lib.check(lib.kld_plan(int(n_rows), int(vocab), int(dtype), int(sm_count), ctypes.byref(p)), "kld_plan")
     return {name: getattr(p, name) for name, _ in _lib.Plan._fields_}
+
+
+def selftest_bounded_wait(device: int = 0, limit_ns: int = 2_000_000, use_abort: bool = False) -> tuple[int, int]:
+    """Run the library's bounded-wait self-test on ``device``: a kernel waits
+    on a barrier nothing completes and must give up after ``limit_ns`` (or on
+    its abort flag). Returns ``(status, waited_ns)``; the expected status is
+    ``KLD_ERR_TIMEOUT``. Any other failure raises."""
+    lib = _lib.load()
+    waited = ctypes.c_uint64(0)
+    st = lib.kld_selftest_bounded_wait(int(device), int(limit_ns), int(bool(use_abort)), ctypes.byref(waited))
+    if st not in (_lib.KLD_OK, _lib.KLD_ERR_TIMEOUT):
+        _lib.check(st, "kld_selftest_bounded_wait")
+    return st, waited.value
 
 
 class _DeviceBytes:

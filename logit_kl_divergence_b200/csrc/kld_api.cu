@@ -394,6 +394,30 @@ kld_status_t kld_stats_run_topk(kld_stats_t h, const void* base, const void* qua
   return KLD_OK;
 }
 
+kld_status_t kld_selftest_bounded_wait(int device, uint64_t limit_ns, int use_abort,
+                                       uint64_t* waited_ns) {
+  if (device < 0 || limit_ns < 1000 || limit_ns > 10000000000ull) return KLD_ERR_INVALID_ARG;
+  DeviceGuard guard(device);
+  if (!guard.ok()) return cuda_fail(cudaGetLastError(), "cudaSetDevice");
+  void* mem = nullptr;
+  KLD_CUDA(cudaMalloc(&mem, 16));
+  uint32_t* derr = static_cast<uint32_t*>(mem);
+  unsigned long long* waited = reinterpret_cast<unsigned long long*>(static_cast<char*>(mem) + 8);
+  kld_status_t st = KLD_OK;
+  uint32_t err_word = 0;
+  unsigned long long w = 0;
+  cudaError_t e = cudaMemset(mem, 0, 16);
+  if (e == cudaSuccess) e = kld::launch_wait_selftest(limit_ns, use_abort, derr, waited, nullptr);
+  if (e == cudaSuccess) e = cudaDeviceSynchronize();
+  if (e == cudaSuccess) e = cudaMemcpy(&err_word, derr, 4, cudaMemcpyDeviceToHost);
+  if (e == cudaSuccess) e = cudaMemcpy(&w, waited, 8, cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) st = cuda_fail(e, "bounded-wait self-test");
+  cudaFree(mem);
+  if (st != KLD_OK) return st;
+  if (waited_ns) *waited_ns = w;
+  return err_word ? KLD_ERR_TIMEOUT : KLD_OK;
+}
+
 kld_status_t kld_stats_grad_timing(kld_stats_t h, float* grad_ms) {
   if (!h || !grad_ms) return KLD_ERR_INVALID_ARG;
   if (!h->grad_timing_valid || !h->has_result) return KLD_ERR_NOT_READY;

@@ -115,6 +115,10 @@ cudaError_t launch_topk(const void* base, const void* quant, const RowAux* aux, 
                         int64_t V, kld_dtype_t dtype, int k, int32_t* idx, float* logp,
                         float* rest, double* kl, int sm_count, cudaStream_t stream);
 
+// Bounded-wait self-test (see kld_selftest_bounded_wait).
+cudaError_t launch_wait_selftest(uint64_t limit_ns, int use_abort, uint32_t* derr,
+                                 unsigned long long* waited_ns, cudaStream_t stream);
+
 cudaError_t launch_reduce(const kld_row_t* rows, int64_t N, int has_nll,
                           uint32_t* derr, kld_result_t* out,
                           cudaStream_t stream);

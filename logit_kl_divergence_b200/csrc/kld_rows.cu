@@ -136,13 +136,14 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 }
 // Wait for the phase of `parity` to complete; gives up after kWaitLimitNs or
 // as soon as another thread of the CTA has raised *abort.
-__device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, volatile int* abort) {
+__device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, volatile int* abort,
+                                            uint64_t limit_ns = kWaitLimitNs) {
   const uint64_t t0 = globaltimer();
   for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((i & 63u) == 0u) {
       if (*abort) return false;
-      if (globaltimer() - t0 > kWaitLimitNs) return false;
+      if (globaltimer() - t0 > limit_ns) return false;
     }
   }
 }
@@ -1442,6 +1443,36 @@ __global__ void __launch_bounds__(kMergeWarps * 32)
   }
 }
 
+// Self-test of the bounded waits: warp 0 waits on an mbarrier that nothing
+// ever arrives at; it must give up after limit_ns (or, with use_abort, as
+// soon as warp 1 raises the abort flag after ~1 ms) and record the timeout
+// in the error word, leaving the context usable.
+__global__ void kld_wait_selftest_kernel(uint64_t limit_ns, int use_abort, uint32_t* derr,
+                                         unsigned long long* waited_ns) {
+  __shared__ __align__(8) unsigned long long bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bar), 1);
+    abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();
+  const int warp = threadIdx.x >> 5;
+  if (warp == 0) {
+    const uint64_t t0 = globaltimer();
+    const bool ok = mbar_wait_slow(smem_u32(&bar), 0u, &abort_flag, limit_ns);
+    if (threadIdx.x == 0) {
+      *waited_ns = globaltimer() - t0;
+      if (!ok) atomicOr(derr, kErrWaitTimeout);
+    }
+  } else if (use_abort && threadIdx.x == 32) {
+    const uint64_t t0 = globaltimer();
+    while (globaltimer() - t0 < 1000000ull) {
+    }
+    *reinterpret_cast<volatile int*>(&abort_flag) = 1;
+  }
+}
+
 template <int DT>
 int max_active_clusters(int cluster_ctas) {
   cudaLaunchConfig_t cfg = {};
@@ -1580,6 +1611,12 @@ cudaError_t launch_rows(const void* base, const void* quant, const int32_t* toke
                                  static_cast<MPart*>(part_out), col_offset, stream);
   }
   return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_wait_selftest(uint64_t limit_ns, int use_abort, uint32_t* derr,
+                                 unsigned long long* waited_ns, cudaStream_t stream) {
+  kld_wait_selftest_kernel<<<1, 64, 0, stream>>>(limit_ns, use_abort, derr, waited_ns);
+  return cudaGetLastError();
 }
 
 }  // namespace kld
