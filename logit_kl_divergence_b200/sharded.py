@@ -8,6 +8,14 @@ set, so the percentiles stay exact and every rank holds the same result.
 
     >>> sk = ShardedKLDStats(max_rows_per_rank=8192, device=dev)   # after init_process_group
     >>> res = sk.run(base_shard, quant_shard, token_shard)          # same dict on every rank
+
+Failure detection is on the host. A rank whose own pass fails (the library
+returned an error status, a bad argument) still takes the step's one small
+collective, the all-gather of row counts, with a count of -1; every rank
+then raises :class:`ShardFailure` naming the failed ranks, and the group
+stays usable for the next step. A rank that dies or never arrives ends its
+peers' next collective with an error after the process group's timeout
+(give the group a short one).
 """
 from __future__ import annotations
 
@@ -27,6 +35,33 @@ def shard_bounds(n_rows: int, world: int, rank: int) -> tuple[int, int]:
     return start, start + base + (1 if rank < extra else 0)
 
 
+class ShardFailure(RuntimeError):
+    """Raised on every rank when the pass failed on one or more ranks;
+    `ranks` lists them, `cause` is this rank's own exception (or None)."""
+
+    def __init__(self, ranks: list[int], cause: BaseException | None):
+        super().__init__(f"sharded pass failed on rank(s) {ranks}"
+                         + (f": {type(cause).__name__}: {cause}" if cause is not None else ""))
+        self.ranks = ranks
+        self.cause = cause
+
+
+def gather_counts(n: int, device, group=None) -> list[int]:
+    """All-gather one int64 per rank (a row count, or -1 for a failed pass)."""
+    t = torch.tensor([n], dtype=torch.int64, device=device)
+    sizes = [torch.zeros_like(t) for _ in range(dist.get_world_size(group))]
+    dist.all_gather(sizes, t, group=group)
+    return [int(c.item()) for c in sizes]
+
+
+def _checked_counts(n: int, err: BaseException | None, device, group) -> list[int]:
+    counts = gather_counts(-1 if err is not None else n, device, group)
+    failed = [r for r, c in enumerate(counts) if c < 0]
+    if failed:
+        raise ShardFailure(failed, err) from err
+    return counts
+
+
 def gather_records(records: torch.Tensor, group=None, counts: list[int] | None = None) -> torch.Tensor:
     """All-gather every rank's [n_r, w] uint8 rows (40-byte records, 64-byte
     vocabulary-slice partials), concatenated in rank order (ranks may hold
@@ -38,10 +73,7 @@ def gather_records(records: torch.Tensor, group=None, counts: list[int] | None =
     width = records.shape[1]
     world = dist.get_world_size(group)
     if counts is None:
-        n = torch.tensor([records.shape[0]], dtype=torch.int64, device=records.device)
-        sizes = [torch.zeros_like(n) for _ in range(world)]
-        dist.all_gather(sizes, n, group=group)
-        counts = [int(c.item()) for c in sizes]
+        counts = gather_counts(records.shape[0], records.device, group)
     elif len(counts) != world or counts[dist.get_rank(group)] != records.shape[0]:
         raise ValueError("counts must list every rank's row count")
     m = max(counts)
@@ -89,8 +121,13 @@ class ShardedKLDStats:
             self._records = torch.empty((self.max_rows_per_rank, ROW_RECORD_BYTES), dtype=torch.uint8,
                                         device=base.device)
         records = self._records[:n]
-        self.stats.run_rows(base, quant, token_ids, out=records)
-        gathered = gather_records(records, self.group)
+        err = None
+        try:
+            self.stats.run_rows(base, quant, token_ids, out=records)
+        except Exception as e:  # reported to every rank below
+            err = e
+        counts = _checked_counts(n, err, base.device, self.group)
+        gathered = gather_records(records, self.group, counts=counts)
         self.stats.reduce(gathered, gathered.shape[0], token_ids is not None)
         return self.stats.result()
 
@@ -109,21 +146,33 @@ class VocabShardedKLDStats:
     rank merges the G partials of each row and reduces: the same statistics
     on every rank as for the full rows on one GPU. At most 32 ranks."""
 
-    def __init__(self, n_rows: int, device=None, group=None):
-        from . import KLDStats
+    def __init__(self, n_rows: int, device=None, group=None, stats=None):
+        if stats is None:
+            from . import KLDStats
 
-        self.stats = KLDStats(max_rows=n_rows, device=device)
+            stats = KLDStats(max_rows=n_rows, device=device)
+        self.stats = stats
         self.group = group
 
     def run(self, base: torch.Tensor, quant: torch.Tensor, token_ids: torch.Tensor | None,
             col_offset: int, v_total: int) -> dict:
         """Collective. `token_ids` are the full-vocabulary ids (the same on
         every rank, or None on every rank)."""
-        parts = self.stats.run_partials(base, quant, token_ids, col_offset, v_total)
-        world = dist.get_world_size(self.group)
-        gathered = gather_records(parts, self.group, counts=[base.shape[0]] * world)
-        self.stats.merge_partials(gathered.view(world, base.shape[0], -1), token_ids, v_total)
+        n = base.shape[0]
+        err = parts = None
+        try:
+            parts = self.stats.run_partials(base, quant, token_ids, col_offset, v_total)
+        except Exception as e:  # reported to every rank below
+            err = e
+        counts = _checked_counts(n, err, base.device, self.group)
+        if any(c != n for c in counts):
+            raise ValueError(f"every rank must hold the same rows, got counts {counts}")
+        world = len(counts)
+        gathered = gather_records(parts, self.group, counts=counts)
+        self.stats.merge_partials(gathered.view(world, n, -1), token_ids, v_total)
         return self.stats.result()
 
     def close(self):
-        self.stats.close()
+        close = getattr(self.stats, "close", None)
+        if close is not None:
+            close()

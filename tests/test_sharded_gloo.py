@@ -125,3 +125,112 @@ def test_shard_bounds_cover_all_rows_in_order():
 @pytest.mark.parametrize("world,n_rows,with_tokens", [(2, 64, True), (2, 37, False), (3, 37, True)])
 def test_sharded_statistics_equal_single_process_oracle(world, n_rows, with_tokens):
     _spawn(world, n_rows, with_tokens)
+
+
+# ---- failure detection on the host: a failing or vanished rank ----------
+
+class FailingStats(OracleStats):
+    """OracleStats whose row pass fails with a library-style error on the
+    listed steps (the fake of an error status from the failing call)."""
+
+    def __init__(self, dtype, fail_steps):
+        super().__init__(dtype)
+        self.fail_steps = set(fail_steps)
+        self.step = 0
+
+    def run_rows(self, base, quant, token_ids=None, out=None):
+        step, self.step = self.step, self.step + 1
+        if step in self.fail_steps:
+            raise RuntimeError("kld_stats_run: KLD_ERR_CUDA (fake)")
+        return super().run_rows(base, quant, token_ids, out)
+
+
+class SliceStats:
+    """Stand-in for the vocabulary-slice handle: each rank's partials are
+    bytes that name the rank and row; the merge records what it was given."""
+
+    def __init__(self, rank, fail_steps):
+        self.rank, self.fail_steps, self.step, self.merged = rank, set(fail_steps), 0, None
+
+    def run_partials(self, base, quant, token_ids, col_offset, v_total):
+        step, self.step = self.step, self.step + 1
+        if step in self.fail_steps:
+            raise RuntimeError("kld_stats_run_partials: KLD_ERR_OOM (fake)")
+        n = base.shape[0]
+        p = torch.zeros((n, 64), dtype=torch.uint8)
+        p[:, 0] = self.rank
+        p[:, 1] = torch.arange(n, dtype=torch.uint8)
+        return p
+
+    def merge_partials(self, parts, token_ids, v_total):
+        self.merged = parts.clone()
+
+    def result(self):
+        return {"merged": self.merged}
+
+
+def _fail_worker(rank, world, port, mode, errq):
+    import datetime
+    import time
+
+    from logit_kl_divergence_b200.sharded import ShardFailure, VocabShardedKLDStats
+    try:
+        dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank,
+                                world_size=world, timeout=datetime.timedelta(seconds=5))
+        w = synth.make_recipe("ctx", n=24, v=1999, dtype=synth.F32, seed=11)
+        lo, hi = shard_bounds(24, world, rank)
+        b, q, t = w.base[lo:hi].contiguous(), w.quant[lo:hi].contiguous(), w.token_ids[lo:hi].contiguous()
+        if mode == "status":
+            # step 0 fails on the last rank only: every rank must raise the
+            # same ShardFailure; step 1 then runs normally on the same group
+            fails = [0] if rank == world - 1 else []
+            sk = ShardedKLDStats(max_rows_per_rank=hi - lo, stats=FailingStats(oracle.F32, fails))
+            with pytest.raises(ShardFailure) as ei:
+                sk.run(b, q, t)
+            assert ei.value.ranks == [world - 1]
+            assert (ei.value.cause is not None) == (rank == world - 1)
+            res = sk.run(b, q, t)
+            _, full = oracle.run(w.base, w.quant, w.token_ids, oracle.F32)
+            _same(res, full)
+        elif mode == "vocab":
+            fails = [0] if rank == 0 else []
+            vs = VocabShardedKLDStats(5, stats=SliceStats(rank, fails))
+            x = torch.zeros((5, 10))
+            with pytest.raises(ShardFailure) as ei:
+                vs.run(x, x, None, 10 * rank, 10 * world)
+            assert ei.value.ranks == [0]
+            got = vs.run(x, x, None, 10 * rank, 10 * world)["merged"]
+            assert got.shape == (world, 5, 64)
+            for r in range(world):
+                assert torch.all(got[r, :, 0] == r) and torch.equal(got[r, :, 1], torch.arange(5, dtype=torch.uint8))
+        elif mode == "exit":
+            # the last rank leaves between steps without telling anyone; the
+            # others' next collective must end with an error, not hang
+            if rank == world - 1:
+                dist.barrier()
+                os._exit(0)
+            sk = ShardedKLDStats(max_rows_per_rank=hi - lo, stats=OracleStats(oracle.F32))
+            dist.barrier()
+            t0 = time.monotonic()
+            try:
+                sk.run(b, q, t)
+            except Exception:
+                dt = time.monotonic() - t0
+                assert dt < 60, dt
+            else:
+                raise AssertionError("run completed without the vanished rank")
+            os._exit(0)  # the group cannot be torn down cleanly without its peer
+        dist.barrier()
+        dist.destroy_process_group()
+    except BaseException as e:  # reported to the parent
+        errq.put(f"rank {rank}: {type(e).__name__}: {e}")
+        raise
+
+
+@pytest.mark.parametrize("world,mode", [(2, "status"), (3, "status"), (2, "vocab"), (3, "vocab"), (2, "exit")])
+def test_rank_failure_is_seen_by_every_rank(world, mode):
+    ctx = mp.get_context("spawn")
+    errq = ctx.SimpleQueue()
+    mp.start_processes(_fail_worker, args=(world, _free_port(), mode, errq), nprocs=world, join=True,
+                       start_method="spawn")
+    assert errq.empty(), errq.get()
