@@ -279,6 +279,28 @@ __device__ __forceinline__ float max3_nan(float a, float b, float c) {
   asm("max.NaN.f32 %0, %1, %2, %3;" : "=f"(y) : "f"(a), "f"(b), "f"(c));
   return y;
 }
+// Maxima of N values as a tree of 3-input maxima (depth ~log3 N instead of
+// a chain of N/2); plain (NaN-ignoring) and NaN-propagating.
+template <int N, bool kNan>
+__device__ __forceinline__ float tree_max(const float* v) {
+  if constexpr (N == 1) {
+    return v[0];
+  } else if constexpr (N == 2) {
+    return kNan ? max3_nan(v[0], v[1], v[1]) : fmaxf(v[0], v[1]);
+  } else {
+    constexpr int M = N / 3 + (N % 3 != 0 ? 1 : 0);
+    float w[M];
+#pragma unroll
+    for (int i = 0; i < N / 3; ++i)
+      w[i] = kNan ? max3_nan(v[3 * i], v[3 * i + 1], v[3 * i + 2])
+                  : max3(v[3 * i], v[3 * i + 1], v[3 * i + 2]);
+    if constexpr (N % 3 == 1) w[M - 1] = v[N - 1];
+    if constexpr (N % 3 == 2)
+      w[M - 1] = kNan ? max3_nan(v[N - 2], v[N - 1], v[N - 1]) : fmaxf(v[N - 2], v[N - 1]);
+    return tree_max<M, kNan>(w);
+  }
+}
+
 __device__ __forceinline__ double warp_sum(double x) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
@@ -453,22 +475,40 @@ __device__ __forceinline__ void poly_accumulate(const float* b, const f2* X, con
   a.C += static_cast<double>(sc0 + sc1);
 }
 
+// Log-ratios x = (q - b) + K of one step, in packed pairs (x = 0 for absent
+// elements), and the largest |x| of the lane (NaN if any x is NaN).
+template <int PE>
+__device__ __forceinline__ float log_ratios(const float* b, const float* q, unsigned valid,
+                                            float K, f2* X) {
+  constexpr int NP = (PE + 1) / 2;
+  float ax0 = 0.f, ax1 = 0.f;
+  const f2 K2 = splat(K);
+#pragma unroll
+  for (int j = 0; j < NP; ++j) {
+    const int i0 = 2 * j, i1 = (2 * j + 1 < PE) ? 2 * j + 1 : 2 * j;
+    X[j] = add2(sub2(pk(q[i0], q[i1]), pk(b[i0], b[i1])), K2);
+    float x0, x1;
+    upk(X[j], x0, x1);
+    if (((valid >> i0) & 1u) == 0u) x0 = 0.f;
+    if (((valid >> i1) & 1u) == 0u || i1 == i0) x1 = 0.f;
+    X[j] = pk(x0, x1);
+    if (j & 1)
+      ax1 = max3_nan(ax1, fabsf(x0), fabsf(x1));
+    else
+      ax0 = max3_nan(ax0, fabsf(x0), fabsf(x1));
+  }
+  return max3_nan(ax0, ax1, 0.f);
+}
+
 // One step of PE element pairs per lane (a 16-element consumer chunk, or the
 // head/tail elements one per lane). Elements whose bit in `valid` is clear
 // are absent (b = q = -inf, x = 0: they contribute nothing).
 template <int PE>
 __device__ __forceinline__ void chunk_step(const float* b, const float* q, unsigned valid,
                                            Ref& r, Acc& a, Best& best, int chunk_id) {
-  float mb = b[0], mq = q[0];
-#pragma unroll
-  for (int i = 1; i + 1 < PE; i += 2) {
-    mb = max3(mb, b[i], b[i + 1]);
-    mq = max3(mq, q[i], q[i + 1]);
-  }
-  if (PE % 2 == 0) {
-    mb = fmaxf(mb, b[PE - 1]);
-    mq = fmaxf(mq, q[PE - 1]);
-  }
+  constexpr int NP = (PE + 1) / 2;
+  const float mb = tree_max<PE, false>(b), mq = tree_max<PE, false>(q);
+  f2 X[NP];  // log-ratios, formed once the centre K of this step is settled
   // The warp maximum is needed only when some lane's maximum passes the
   // threshold (a few chunks per row): a vote first, then the shuffle tree.
   if (__any_sync(0xffffffffu, mb > r.T)) {
@@ -526,29 +566,10 @@ __device__ __forceinline__ void chunk_step(const float* b, const float* q, unsig
     r.Mb = wmb;
     r.T = wmb + kRaiseMargin;
   }
+  const float axl = log_ratios<PE>(b, q, valid, r.K, X);
 
-  // Log-ratios x = (q - b) + K, in packed pairs.
-  constexpr int NP = (PE + 1) / 2;
-  f2 X[NP];
-  float ax0 = 0.f, ax1 = 0.f;  // max |x| of the lane (two chains), NaN if any x is NaN
-  const f2 K2 = splat(r.K);
-#pragma unroll
-  for (int j = 0; j < NP; ++j) {
-    const int i0 = 2 * j, i1 = (2 * j + 1 < PE) ? 2 * j + 1 : 2 * j;
-    X[j] = add2(sub2(pk(q[i0], q[i1]), pk(b[i0], b[i1])), K2);
-    float x0, x1;
-    upk(X[j], x0, x1);
-    if (((valid >> i0) & 1u) == 0u) x0 = 0.f;
-    if (((valid >> i1) & 1u) == 0u || i1 == i0) x1 = 0.f;
-    X[j] = pk(x0, x1);
-    if (j & 1)
-      ax1 = max3_nan(ax1, fabsf(x0), fabsf(x1));
-    else
-      ax0 = max3_nan(ax0, fabsf(x0), fabsf(x1));
-  }
   // The cheapest polynomial tier whose range holds every |x| of the warp's
   // step (a NaN fails every test and takes the direct path).
-  const float axl = max3_nan(ax0, ax1, 0.f);
   if (__all_sync(0xffffffffu, axl <= kTauA)) {
     poly_accumulate<PE, 0>(b, X, r, a);
   } else if (__all_sync(0xffffffffu, axl <= kTauB)) {
@@ -1032,8 +1053,10 @@ __global__ void __launch_bounds__(kRowThreads, 1)
         const uint4* tq = reinterpret_cast<const uint4*>(stage_q + s * kStageBytes);
         const int rem = n - t * kStageElems;
         if (rem >= kStageElems) {
-          // Full tile: this warp's chunks, no masking.
-#pragma unroll
+          // Full tile: this warp's chunks, no masking. Not unrolled: one
+          // copy of the chunk code keeps the hot loop small for the
+          // instruction cache (measured faster than two copies).
+#pragma unroll 1
           for (int k = 0; k < kChunksPerWarp; ++k) {
             const int c = warp + k * kConsumerWarps;
             process_chunk<DT, false>(tb + c * (kChunkElems / E), tq + c * (kChunkElems / E), lane,
