@@ -20,13 +20,18 @@
 // 128 and 1024 when N is smaller, so small inputs pay for few threads):
 //   1. thread t sums records t, t+T, ... in order; the T partials are
 //      combined by a fixed shuffle tree, so the fp64 sums are deterministic
-//      for a given N.
-//   2. the up to seven ranks the percentiles need are selected exactly with
-//      an MSB-first radix select on order-preserving 64-bit keys of the
-//      doubles (8 bits per pass, one shared histogram per distinct prefix,
-//      warp-aggregated shared atomics). As soon as the ranks' candidate sets
-//      together hold at most kGatherCap keys, those keys are gathered into
-//      shared memory and sorted (bitonic), which finishes the selection.
+//      for a given N. The same pass appends the order-preserving 64-bit keys
+//      of the valid rows' KL to shared memory (N <= kKeyCap; larger inputs
+//      re-read the records for every level instead).
+//   2. the up to seven ranks the percentiles need are selected exactly by an
+//      MSB-first radix select with 11-bit digits: per level, one shared
+//      histogram per distinct group of targets (keys that share the digits
+//      decided so far), a warp per group scans its 2048 bins and finds the
+//      digit and residual rank of each of its targets. A group of at most
+//      32 keys is gathered and sorted in one warp instead, which ends its
+//      targets; a group still large after all 64 bits holds equal keys.
+
+#include <atomic>
 #include <climits>
 
 #include "kld_internal.h"
@@ -35,8 +40,11 @@ namespace kld {
 namespace {
 
 constexpr int kTargets = 7;
-constexpr int kAhead = 4;  // records each thread loads before using them
-constexpr int kGatherCap = 4096;
+constexpr int kAhead = 4;       // records each thread loads before using them
+constexpr int kDigitBits = 11;  // radix digit of the selection
+constexpr int kBins = 1 << kDigitBits;
+constexpr int kSmall = 32;      // a group this small is finished by one warp
+constexpr int kKeyCap = 19968;  // keys kept in shared memory (N up to this)
 constexpr uint32_t kExcluded = KLD_ROW_NONFINITE | KLD_ROW_EMPTY;
 
 __device__ __forceinline__ uint64_t order_key(double x) {
@@ -62,60 +70,89 @@ struct ReduceShared {
   double dsum[32][5];
   long long isum[32][4];
   unsigned int flags_or[32];
-  // selection state
-  unsigned long long prefix[kTargets];
-  unsigned long long rank[kTargets];
+  // selection state: groups of targets whose keys share the decided digits
   unsigned long long gprefix[kTargets];
-  unsigned long long gcount[kTargets];
-  int tgroup[kTargets];
+  unsigned long long tnext[kTargets];  // a target's prefix after this level
+  unsigned long long trank[kTargets];  // its rank among its group's keys
+  unsigned long long tval[kTargets];   // its key, once found
+  unsigned int gcount[kTargets];
+  unsigned int gfill[kTargets];
+  unsigned int tcount[kTargets];  // size of a target's group after this level
+  int tgroup[kTargets];           // -1 once found
   int ngroups;
-  int done;
-  int ncand;
-  unsigned int hist[kTargets][256];
-  unsigned long long cand[kGatherCap];
+  unsigned int hist[kTargets][kBins];
+  unsigned long long gbuf[kTargets][kSmall];
 };
+constexpr size_t kReduceSmemMax = sizeof(ReduceShared) + sizeof(unsigned long long) * kKeyCap;
+static_assert(kReduceSmemMax <= 227 * 1024, "reduction shared memory");
+
+// Ascending bitonic sort of one 64-bit key per lane.
+__device__ __forceinline__ unsigned long long warp_sort(unsigned long long key, int lane) {
+#pragma unroll
+  for (int k = 2; k <= 32; k <<= 1) {
+#pragma unroll
+    for (int j = k >> 1; j > 0; j >>= 1) {
+      const unsigned long long other = __shfl_xor_sync(0xffffffffu, key, j);
+      const bool up = (lane & k) == 0;
+      const bool lower = (lane & j) == 0;
+      key = (lower == up) ? (key < other ? key : other) : (key > other ? key : other);
+    }
+  }
+  return key;
+}
 
 __global__ void __launch_bounds__(kReduceThreads, 1)
     kld_reduce_kernel(const kld_row_t* __restrict__ rows, int64_t N, int has_nll,
                       uint32_t* __restrict__ derr, kld_result_t* __restrict__ out) {
-  __shared__ ReduceShared sh;
+  extern __shared__ __align__(16) unsigned char reduce_smem[];
+  ReduceShared& sh = *reinterpret_cast<ReduceShared*>(reduce_smem);
+  unsigned long long* keys = reinterpret_cast<unsigned long long*>(reduce_smem + sizeof(ReduceShared));
+  const bool in_smem = N <= kKeyCap;
   const int tid = threadIdx.x;
   const int lane = tid & 31, warp = tid >> 5;
   const int nt = static_cast<int>(blockDim.x);
+  const int nw = nt >> 5;
   // Launched as a programmatic dependent of the row pass: its launch may
   // overlap the row pass, the records are read only after it completed.
   asm volatile("griddepcontrol.wait;" ::: "memory");
 
-  // ---------------------------------------------------------------- sums
+  // ------------------------------------------------------- sums and keys
   double s_kl = 0.0, s_nll = 0.0, s_nllb = 0.0, s_dp = 0.0, s_dp2 = 0.0;
   long long n_valid = 0, agree = 0, n_nll = 0, n_flag = 0;
   unsigned int f_or = 0;
   // Records t, t + T, ... in order; kAhead loads in flight per thread.
-  for (int64_t i0 = tid; i0 < N; i0 += static_cast<int64_t>(kAhead) * nt) {
+  for (int64_t base = 0; base < N; base += static_cast<int64_t>(kAhead) * nt) {
     kld_row_t rec[kAhead];
 #pragma unroll
     for (int u = 0; u < kAhead; ++u) {
-      const int64_t i = i0 + static_cast<int64_t>(u) * nt;
+      const int64_t i = base + static_cast<int64_t>(u) * nt + tid;
       if (i < N) rec[u] = rows[i];
     }
 #pragma unroll
     for (int u = 0; u < kAhead; ++u) {
-      if (i0 + static_cast<int64_t>(u) * nt >= N) break;
+      const bool in = base + static_cast<int64_t>(u) * nt + tid < N;
       const kld_row_t& rc = rec[u];
-      f_or |= rc.flags;
-      if (rc.flags) ++n_flag;
-      if (rc.flags & kExcluded) continue;
-      ++n_valid;
-      s_kl += rc.kld;
-      if (rc.argmax_base == rc.argmax_quant) ++agree;
-      if (has_nll && !(rc.flags & KLD_ROW_BAD_TOKEN)) {
-        s_nll += rc.nll;
-        s_nllb += rc.nll_base;
-        const double dp = static_cast<double>(rc.dp);  // computed per row by the row pass
-        s_dp += dp;
-        s_dp2 += dp * dp;
-        ++n_nll;
+      const bool valid = in && !(rc.flags & kExcluded);
+      if (in) {
+        f_or |= rc.flags;
+        if (rc.flags) ++n_flag;
       }
+      if (valid) {
+        ++n_valid;
+        s_kl += rc.kld;
+        if (rc.argmax_base == rc.argmax_quant) ++agree;
+        if (has_nll && !(rc.flags & KLD_ROW_BAD_TOKEN)) {
+          s_nll += rc.nll;
+          s_nllb += rc.nll_base;
+          const double dp = static_cast<double>(rc.dp);  // computed per row by the row pass
+          s_dp += dp;
+          s_dp2 += dp * dp;
+          ++n_nll;
+        }
+      }
+      // Key of every record in place; excluded rows get key 0, below every
+      // key of a non-NaN value, and the ranks are offset by their number.
+      if (in_smem && in) keys[base + static_cast<int64_t>(u) * nt + tid] = valid ? order_key(rc.kld) : 0ull;
     }
   }
 #pragma unroll
@@ -197,68 +234,128 @@ __global__ void __launch_bounds__(kReduceThreads, 1)
       } else {
         k = nv - 1;
       }
-      sh.prefix[tid] = 0ull;
-      sh.rank[tid] = static_cast<unsigned long long>(k);
+      sh.trank[tid] = static_cast<unsigned long long>(k);
+      sh.tgroup[tid] = 0;
+      sh.tval[tid] = 0ull;
     }
+    // Excluded rows have key 0, below every other key: they come first and
+    // offset the ranks.
+    __syncthreads();
+    if (in_smem && N <= 32) {
+      // Few rows: one warp sorts all keys.
+      if (warp == 0) {
+        const unsigned long long key = warp_sort(lane < N ? keys[lane] : ~0ull, lane);
+        for (int t = 0; t < kTargets; ++t) {
+          const unsigned long long v =
+              __shfl_sync(0xffffffffu, key, static_cast<int>(sh.trank[t] + (N - nv)));
+          if (lane == 0) {
+            sh.tval[t] = v;
+            sh.tgroup[t] = -1;
+          }
+        }
+      }
+      __syncthreads();
+    }
+    if (tid < kTargets) sh.trank[tid] += static_cast<unsigned long long>(N - nv);
     if (tid == 0) {
-      sh.done = 0;
       sh.ngroups = 1;
       sh.gprefix[0] = 0ull;
-      sh.gcount[0] = static_cast<unsigned long long>(nv);
-      for (int t = 0; t < kTargets; ++t) sh.tgroup[t] = 0;
+      sh.gcount[0] = static_cast<unsigned int>(N);
     }
     __syncthreads();
 
-    int decided = 0;  // number of high key bits fixed so far
-    for (int shift = 56; shift >= 0; shift -= 8) {
-      // Few candidates left: gather them and finish by sorting.
-      unsigned long long total = 0;
-      for (int g = 0; g < sh.ngroups; ++g) total += sh.gcount[g];
-      if (total <= static_cast<unsigned long long>(kGatherCap)) break;
-
+    for (int decided = 0;; ) {
+      bool open = false;
+      for (int t = 0; t < kTargets; ++t) open |= sh.tgroup[t] >= 0;
+      if (!open) break;
       const int ng = sh.ngroups;
-      for (int i = tid; i < ng * 256; i += nt) (&sh.hist[0][0])[i] = 0u;
+      if (decided >= 64) {
+        // every key of a remaining group equals its prefix
+        if (tid < kTargets && sh.tgroup[tid] >= 0) {
+          sh.tval[tid] = sh.gprefix[sh.tgroup[tid]];
+          sh.tgroup[tid] = -1;
+        }
+        __syncthreads();
+        break;
+      }
+      const int bits = 64 - decided < kDigitBits ? 64 - decided : kDigitBits;
+      const int shift = 64 - decided - bits;
+      const unsigned long long himask = decided == 0 ? 0ull : (~0ull << (64 - decided));
+      for (int i = tid; i < ng * kBins; i += nt)
+        if (sh.gcount[i / kBins] > static_cast<unsigned>(kSmall)) (&sh.hist[0][0])[i] = 0u;
+      if (tid < ng) sh.gfill[tid] = 0u;
       __syncthreads();
-      const uint64_t himask = decided == 0 ? 0ull : (~0ull << (64 - decided));
-      // four records per thread in flight, then the warp-aggregated counts
-      for (int64_t base_i = 0; base_i < N; base_i += static_cast<int64_t>(kAhead) * nt) {
-        double kv[kAhead];
-        uint32_t fv[kAhead];
+
+      // One pass over the keys: gather the keys of small groups, count the
+      // next digit of the keys of large ones (warp-aggregated atomics).
+      for (int64_t base = 0; base < N; base += static_cast<int64_t>(kAhead) * nt) {
+        unsigned long long kv[kAhead];
+        bool ok[kAhead];
 #pragma unroll
         for (int u = 0; u < kAhead; ++u) {
-          const int64_t i = base_i + static_cast<int64_t>(u) * nt + tid;
-          fv[u] = kExcluded;
-          if (i < N) {
-            fv[u] = rows[i].flags;
-            kv[u] = rows[i].kld;
+          const int64_t i = base + static_cast<int64_t>(u) * nt + tid;
+          ok[u] = i < N;
+          kv[u] = 0ull;
+          if (ok[u]) {
+            if (in_smem) {
+              kv[u] = keys[i];
+            } else if (!(rows[i].flags & kExcluded)) {
+              kv[u] = order_key(rows[i].kld);
+            }
           }
         }
 #pragma unroll
         for (int u = 0; u < kAhead; ++u) {
-          int slot = -1;
-          if (!(fv[u] & kExcluded)) {
-            const uint64_t key = order_key(kv[u]);
-            for (int g = 0; g < ng; ++g) {
-              if (((key ^ sh.gprefix[g]) & himask) == 0ull) {
-                slot = g * 256 + static_cast<int>((key >> shift) & 0xffu);
+          int g = -1;
+          if (ok[u]) {
+            for (int h = 0; h < ng; ++h) {
+              if (((kv[u] ^ sh.gprefix[h]) & himask) == 0ull) {
+                g = h;
                 break;
               }
             }
           }
-          const unsigned peers = __match_any_sync(0xffffffffu, slot);
-          if (slot >= 0 && lane == __ffs(peers) - 1)
-            atomicAdd(&(&sh.hist[0][0])[slot], static_cast<unsigned>(__popc(peers)));
+          const bool small = g >= 0 && sh.gcount[g] <= static_cast<unsigned>(kSmall);
+          if (small) {
+            const unsigned p = atomicAdd(&sh.gfill[g], 1u);
+            if (p < static_cast<unsigned>(kSmall)) sh.gbuf[g][p] = kv[u];
+          }
+          const int slot = (g >= 0 && !small)
+                               ? g * kBins + static_cast<int>((kv[u] >> shift) & (kBins - 1))
+                               : -1;
+          if (decided == 0) {
+            // first digit: few distinct bins, one atomic per bin and warp
+            const unsigned peers = __match_any_sync(0xffffffffu, slot);
+            if (slot >= 0 && lane == __ffs(peers) - 1)
+              atomicAdd(&(&sh.hist[0][0])[slot], static_cast<unsigned>(__popc(peers)));
+          } else if (slot >= 0) {
+            atomicAdd(&(&sh.hist[0][0])[slot], 1u);  // later digits spread out
+          }
         }
       }
       __syncthreads();
-      for (int t = warp; t < kTargets; t += nt >> 5) {
-        // One warp per target: 8 bins per lane, a warp prefix scan, then the
-        // lane holding the rank finds its bin.
+
+      // A warp per open target: finish a small group by sorting its keys, or
+      // find the target's digit in its group's histogram. Lane L sums bins
+      // [64L, 64L + 64) (rotated start: conflict-free), a warp scan finds the
+      // lane whose range holds the rank, and the warp scans those 64 bins.
+      for (int t = warp; t < kTargets; t += nw) {
         const int g = sh.tgroup[t];
-        const unsigned long long r = sh.rank[t];
+        if (g < 0) continue;
+        const unsigned cnt = sh.gcount[g];
+        const unsigned long long r = sh.trank[t];
+        if (cnt <= static_cast<unsigned>(kSmall)) {
+          const unsigned long long key =
+              warp_sort(lane < static_cast<int>(cnt) ? sh.gbuf[g][lane] : ~0ull, lane);
+          const unsigned long long v = __shfl_sync(0xffffffffu, key, static_cast<int>(r));
+          if (lane == 0) sh.tval[t] = v;
+          continue;
+        }
+        constexpr int kPer = kBins / 32;
+        const unsigned* hg = sh.hist[g];
         unsigned long long part = 0;
-#pragma unroll
-        for (int b = 0; b < 8; ++b) part += sh.hist[g][lane * 8 + b];
+#pragma unroll 8
+        for (int b = 0; b < kPer; ++b) part += hg[lane * kPer + ((b + lane) & (kPer - 1))];
         unsigned long long incl = part;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
@@ -268,101 +365,53 @@ __global__ void __launch_bounds__(kReduceThreads, 1)
         const unsigned long long excl = incl - part;
         const unsigned hit = __ballot_sync(0xffffffffu, r >= excl && r < incl);
         const int owner = hit ? __ffs(hit) - 1 : 31;  // 31: unreachable for consistent counts
-        if (lane == owner) {
-          unsigned long long before = excl;
-          int bin = lane * 8;
-          for (int b = 0; b < 8; ++b) {
-            bin = lane * 8 + b;
-            const unsigned long long c = sh.hist[g][bin];
-            if (r < before + c) break;
-            before += c;
+        const unsigned long long before = __shfl_sync(0xffffffffu, excl, owner);
+        const unsigned c0 = hg[owner * kPer + lane], c1 = hg[owner * kPer + 32 + lane];
+        unsigned long long s0 = c0, s1 = c1;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const unsigned long long v0 = __shfl_up_sync(0xffffffffu, s0, o);
+          const unsigned long long v1 = __shfl_up_sync(0xffffffffu, s1, o);
+          if (lane >= o) {
+            s0 += v0;
+            s1 += v1;
           }
-          sh.prefix[t] = sh.gprefix[g] | (static_cast<unsigned long long>(bin) << shift);
-          sh.rank[t] = r - before;
-          sh.gcount[t] = sh.hist[g][bin];  // temporarily per target
+        }
+        s1 += __shfl_sync(0xffffffffu, s0, 31);
+        const unsigned long long rr = r - before;  // rank within the owner's 64 bins
+        const unsigned m0 = __ballot_sync(0xffffffffu, s0 > rr);
+        const unsigned m1 = __ballot_sync(0xffffffffu, s1 > rr);
+        const int j = m0 ? __ffs(m0) - 1 : 32 + (m1 ? __ffs(m1) - 1 : 31);
+        const unsigned long long incl_j = __shfl_sync(0xffffffffu, j < 32 ? s0 : s1, j & 31);
+        const unsigned cnt_j = __shfl_sync(0xffffffffu, j < 32 ? c0 : c1, j & 31);
+        if (lane == 0) {
+          const int bin = owner * kPer + j;
+          sh.tnext[t] = sh.gprefix[g] | (static_cast<unsigned long long>(bin) << shift);
+          sh.trank[t] = rr - (incl_j - cnt_j);
+          sh.tcount[t] = cnt_j;
         }
       }
       __syncthreads();
-      if (tid == 0) {
-        // Distinct prefixes become the next pass's groups.
-        unsigned long long cnt[kTargets];
-        for (int t = 0; t < kTargets; ++t) cnt[t] = sh.gcount[t];
-        int n = 0;
-        for (int t = 0; t < kTargets; ++t) {
-          int g = -1;
-          for (int j = 0; j < n; ++j)
-            if (sh.gprefix[j] == sh.prefix[t]) g = j;
-          if (g < 0) {
-            g = n++;
-            sh.gprefix[g] = sh.prefix[t];
-            sh.gcount[g] = cnt[t];
-          }
-          sh.tgroup[t] = g;
+      if (warp == 0) {
+        // Targets of small groups are done; the others regroup by their new
+        // prefix (lane t = target t; groups numbered in lane order).
+        const int g0 = lane < kTargets ? sh.tgroup[lane] : -1;
+        const bool act = g0 >= 0 && sh.gcount[g0] > static_cast<unsigned>(kSmall);
+        const unsigned long long p = act ? sh.tnext[lane] : ~0ull;
+        const unsigned cnt = act ? sh.tcount[lane] : 0u;
+        const unsigned peers = __match_any_sync(0xffffffffu, p);
+        const int leader = __ffs(peers) - 1;
+        const unsigned leaders = __ballot_sync(0xffffffffu, act && lane == leader);
+        const int gid = __popc(leaders & ((1u << leader) - 1u));
+        __syncwarp();
+        if (act && lane == leader) {
+          sh.gprefix[gid] = p;
+          sh.gcount[gid] = cnt;
         }
-        sh.ngroups = n;
+        if (lane < kTargets) sh.tgroup[lane] = act ? gid : -1;
+        if (lane == 0) sh.ngroups = __popc(leaders);
       }
-      decided += 8;
-      __syncthreads();
-    }
-
-    if (decided < 64) {
-      // Gather every key whose decided bits match a group, sort, and index.
-      if (tid == 0) sh.ncand = 0;
-      __syncthreads();
-      const uint64_t himask = decided == 0 ? 0ull : (~0ull << (64 - decided));
-      const int ng = sh.ngroups;
-      for (int64_t base_i = 0; base_i < N; base_i += nt) {
-        const int64_t i = base_i + tid;
-        bool take = false;
-        uint64_t key = 0;
-        if (i < N && !(rows[i].flags & kExcluded)) {
-          key = order_key(rows[i].kld);
-          for (int g = 0; g < ng; ++g)
-            if (((key ^ sh.gprefix[g]) & himask) == 0ull) take = true;
-        }
-        // one shared atomic per warp
-        const unsigned m = __ballot_sync(0xffffffffu, take);
-        int basepos = 0;
-        if (lane == 0 && m) basepos = atomicAdd(&sh.ncand, __popc(m));
-        basepos = __shfl_sync(0xffffffffu, basepos, 0);
-        if (take) {
-          const int pos = basepos + __popc(m & ((1u << lane) - 1u));
-          if (pos < kGatherCap) sh.cand[pos] = key;
-        }
-      }
-      __syncthreads();
-      int n = sh.ncand;
-      if (n > kGatherCap) n = kGatherCap;  // unreachable: counts bound it
-      int p2 = 1;
-      while (p2 < n) p2 <<= 1;
-      for (int i = n + tid; i < p2; i += nt) sh.cand[i] = ~0ull;
-      __syncthreads();
-      for (int k = 2; k <= p2; k <<= 1) {
-        for (int j = k >> 1; j > 0; j >>= 1) {
-          for (int i = tid; i < p2; i += nt) {
-            const int ixj = i ^ j;
-            if (ixj > i) {
-              const unsigned long long a = sh.cand[i], b = sh.cand[ixj];
-              const bool up = (i & k) == 0;
-              if ((a > b) == up) {
-                sh.cand[i] = b;
-                sh.cand[ixj] = a;
-              }
-            }
-          }
-          __syncthreads();
-        }
-      }
-      if (tid < kTargets) {
-        // Groups are disjoint key ranges: a target's group starts after all
-        // candidates of groups with smaller prefixes.
-        const int g = sh.tgroup[tid];
-        unsigned long long off = 0;
-        for (int h = 0; h < ng; ++h)
-          if (sh.gprefix[h] < sh.gprefix[g]) off += sh.gcount[h];
-        const unsigned long long idx = off + sh.rank[tid];
-        sh.prefix[tid] = idx < static_cast<unsigned long long>(n) ? sh.cand[idx] : ~0ull;
-      }
+      decided += bits;
       __syncthreads();
     }
   }
@@ -386,10 +435,10 @@ __global__ void __launch_bounds__(kReduceThreads, 1)
     if (nv > 0) {
       const double dn = static_cast<double>(nv - 1);
       r.mean_kld = sh.dsum[0][0] / static_cast<double>(nv);
-      r.median_kld = interpolate(0.5 * dn, key_value(sh.prefix[0]), key_value(sh.prefix[1]));
-      r.p90_kld = interpolate(0.9 * dn, key_value(sh.prefix[2]), key_value(sh.prefix[3]));
-      r.p99_kld = interpolate(0.99 * dn, key_value(sh.prefix[4]), key_value(sh.prefix[5]));
-      r.max_kld = key_value(sh.prefix[6]);
+      r.median_kld = interpolate(0.5 * dn, key_value(sh.tval[0]), key_value(sh.tval[1]));
+      r.p90_kld = interpolate(0.9 * dn, key_value(sh.tval[2]), key_value(sh.tval[3]));
+      r.p99_kld = interpolate(0.99 * dn, key_value(sh.tval[4]), key_value(sh.tval[5]));
+      r.max_kld = key_value(sh.tval[6]);
       r.top1_agree_pct = 100.0 * static_cast<double>(sh.isum[0][1]) / static_cast<double>(nv);
     } else {
       r.mean_kld = r.median_kld = r.p90_kld = r.p99_kld = r.max_kld = nan;
@@ -417,14 +466,30 @@ __global__ void __launch_bounds__(kReduceThreads, 1)
 
 cudaError_t launch_reduce(const kld_row_t* rows, int64_t N, int has_nll, uint32_t* derr,
                           kld_result_t* out, cudaStream_t stream) {
+  if (N < 0 || N > static_cast<int64_t>(UINT32_MAX)) return cudaErrorInvalidValue;  // 32-bit counts
   int threads = kReduceThreads;
   if (N < kReduceThreads) {
     threads = static_cast<int>((N + 31) / 32 * 32);
     if (threads < 128) threads = 128;
   }
+  // Shared memory beyond the static 48 KB: allowed once per device.
+  static std::atomic<unsigned long long> smem_set{0ull};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const unsigned long long bit = 1ull << (dev & 63);
+  if (!(smem_set.load(std::memory_order_acquire) & bit)) {
+    e = cudaFuncSetAttribute(kld_reduce_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(kReduceSmemMax));
+    if (e != cudaSuccess) return e;
+    smem_set.fetch_or(bit, std::memory_order_acq_rel);
+  }
+  const size_t smem = sizeof(ReduceShared) +
+                      (N <= kKeyCap ? static_cast<size_t>(N) * sizeof(unsigned long long) : 0);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(1);
   cfg.blockDim = dim3(static_cast<unsigned>(threads));
+  cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
   cudaLaunchAttribute attr;
   attr.id = cudaLaunchAttributeProgrammaticStreamSerialization;
