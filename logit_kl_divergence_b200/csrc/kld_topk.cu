@@ -12,14 +12,20 @@
 // x_j = (q_j - b_j) + K rounded to fp32 as the row pass rounds it, the rest
 // in fp64.
 //
-// One CTA per row (persistent over rows): the k-th largest key of the base
-// row is found by an MSB radix select over order-preserving 32-bit keys
-// (11/11/10-bit levels, a shared histogram per level, stopping as soon as the
-// candidates fit in shared memory); if a tie group at the threshold is larger
-// than that, the lowest indices in it are found by a radix select over the
-// index. The candidates (at most kCap) are sorted in shared memory by (key
-// desc, index asc). A last pass over the row sums the rest mass of both rows.
-// The row is read 2-4 times, from L2 after the first.
+// One CTA per row (persistent over rows, two per SM). Fast path: 4096
+// evenly spaced samples of the base row give a threshold key t0 (the bin of
+// the m-th largest sample, m ~ 1.5 k * 4096 / V + 8, refined by a second
+// digit when the bin is wide), and one fused pass over both rows appends
+// every element with key >= t0 to a shared candidate list and sums the rest
+// masses of all other elements: each logit is read once. If fewer than k or
+// more than kCap elements pass the threshold (ties or extreme rows), an exact
+// path takes the row instead: an MSB radix select over order-preserving
+// 32-bit keys (11/11/10-bit levels, stopping as soon as the candidates fit
+// in shared memory; for a tie group at the threshold larger than that, the
+// lowest indices in it by a radix select over the index), the candidates,
+// and a last pass for the rest masses (the row is read 2-4 times). Either
+// way the candidates are sorted in shared memory by (key desc, index asc)
+// and the first k are T; candidates beyond T join the rest.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -32,8 +38,10 @@ namespace {
 
 constexpr int kTopkThreads = 512;
 constexpr int kTopkWarps = kTopkThreads / 32;
+constexpr int kTopkCtasPerSm = 2;
 constexpr int kHistBins = 2048;
 constexpr int kCap = 4096;  // candidates sorted in shared memory
+constexpr int kSample = 4096;  // samples of a row for the threshold
 constexpr float kL = 1.4426950408889634f;  // log2(e) rounded to fp32, as the row pass
 constexpr double kLn2 = 0.6931471805599453;
 
@@ -122,8 +130,211 @@ __device__ double block_sum(TopkShared& sh, double v, int slot) {
   return t;
 }
 
+// Inverse of okey.
+__device__ __forceinline__ float key_float(uint32_t k) {
+  return __uint_as_float((k >> 31) ? (k & 0x7fffffffu) : ~k);
+}
+
+// Fast-path threshold: a key t0 with, by the samples, comfortably more than
+// kt but fewer than kCap elements of the row at or above it (block-wide).
 template <int DT>
-__global__ void __launch_bounds__(kTopkThreads)
+__device__ uint32_t sample_threshold(TopkShared& sh, const char* rb, int64_t V, int kt) {
+  const int tid = threadIdx.x;
+  uint32_t* skey = reinterpret_cast<uint32_t*>(sh.cand);  // kSample keys
+  double mm = 1.5 * static_cast<double>(kt) * kSample / static_cast<double>(V) + 8.0;
+  const unsigned m = mm > kSample ? static_cast<unsigned>(kSample) : static_cast<unsigned>(mm);
+  for (int i = tid; i < kSample; i += kTopkThreads)
+    skey[i] = okey(load_el<DT>(rb, static_cast<int64_t>(i) * V / kSample));
+  for (int i = tid; i < kHistBins; i += kTopkThreads) sh.hist[i] = 0u;
+  __syncthreads();
+  for (int i = tid; i < kSample; i += kTopkThreads) atomicAdd(&sh.hist[skey[i] >> 21], 1u);
+  __syncthreads();
+  find_bin(sh, kHistBins, m, true);
+  const uint32_t bin = sh.sel[0], above = sh.sel[1], inbin = sh.sel[2];
+  uint32_t t0 = bin << 21;
+  const double per = static_cast<double>(V) / kSample;  // row elements per sample
+  if (static_cast<double>(above + inbin) * per > 0.5 * kCap && inbin > 1) {
+    // wide bin: the next 11 bits of the samples in it
+    __syncthreads();
+    for (int i = tid; i < kHistBins; i += kTopkThreads) sh.hist[i] = 0u;
+    __syncthreads();
+    for (int i = tid; i < kSample; i += kTopkThreads)
+      if ((skey[i] >> 21) == bin) atomicAdd(&sh.hist[(skey[i] >> 10) & (kHistBins - 1)], 1u);
+    __syncthreads();
+    find_bin(sh, kHistBins, m - above, true);
+    t0 |= sh.sel[0] << 10;
+  }
+  __syncthreads();  // the sample keys share memory with the candidates
+  return t0;
+}
+
+// Rest-mass terms of one element (fp32, as the row pass rounds them).
+__device__ __forceinline__ float rest_b(float bj, const RowAux& a) {
+  return __fmul_rn(ex2(fmaf(bj, kL, -a.Fb)), a.mb);
+}
+__device__ __forceinline__ float rest_q(float qj, const RowAux& a) {
+  return __fmul_rn(ex2(fmaf(qj, kL, -a.Fq)), a.mq);
+}
+
+// Fused pass: elements with key >= t0 become candidates (the count goes on
+// past kCap, which sends the row to the exact path); all others add to the
+// rest masses (fp32 over one vector, fp64 across vectors).
+template <int DT>
+__device__ void gather_pass(TopkShared& sh, const char* rb, const char* rq, int64_t V,
+                            uint32_t t0, const RowAux& a, double& prest, double& rrest) {
+  const int tid = threadIdx.x;
+  auto take = [&](float bj, int64_t j, float& sp, float& sr, float qj) {
+    const uint32_t key = okey(bj);
+    if (key >= t0) {
+      const int pos = atomicAdd(&sh.ncand, 1);
+      if (pos < kCap)
+        sh.cand[pos] = (static_cast<unsigned long long>(key) << 32) | (0xffffffffu - static_cast<uint32_t>(j));
+    } else {
+      sp += rest_b(bj, a);
+      sr += rest_q(qj, a);
+    }
+  };
+  constexpr int EB = DT == KLD_F32 ? 4 : 2;
+  constexpr int E = 16 / EB;  // elements per 16-byte vector
+  const bool vec = ((reinterpret_cast<uintptr_t>(rb) | reinterpret_cast<uintptr_t>(rq)) & 15u) == 0 &&
+                   (V % E) == 0;
+  if (vec) {
+    const uint4* vb = reinterpret_cast<const uint4*>(rb);
+    const uint4* vq = reinterpret_cast<const uint4*>(rq);
+    const int64_t nv = V / E;
+    for (int64_t v0 = tid; v0 < nv; v0 += 2 * kTopkThreads) {
+      uint4 xb[2], xq[2];
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const int64_t v = v0 + u * kTopkThreads;
+        if (v < nv) {
+          xb[u] = __ldg(vb + v);
+          xq[u] = __ldg(vq + v);
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const int64_t v = v0 + u * kTopkThreads;
+        if (v >= nv) continue;
+        float fb[E], fq[E];
+        const uint32_t wb[4] = {xb[u].x, xb[u].y, xb[u].z, xb[u].w};
+        const uint32_t wq[4] = {xq[u].x, xq[u].y, xq[u].z, xq[u].w};
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+          if (DT == KLD_F32) {
+            fb[w] = __uint_as_float(wb[w]);
+            fq[w] = __uint_as_float(wq[w]);
+          } else if (DT == KLD_BF16) {
+            fb[2 * w] = __uint_as_float(wb[w] << 16);
+            fb[2 * w + 1] = __uint_as_float(wb[w] & 0xffff0000u);
+            fq[2 * w] = __uint_as_float(wq[w] << 16);
+            fq[2 * w + 1] = __uint_as_float(wq[w] & 0xffff0000u);
+          } else {
+            fb[2 * w] = __half2float(__ushort_as_half(static_cast<unsigned short>(wb[w] & 0xffffu)));
+            fb[2 * w + 1] = __half2float(__ushort_as_half(static_cast<unsigned short>(wb[w] >> 16)));
+            fq[2 * w] = __half2float(__ushort_as_half(static_cast<unsigned short>(wq[w] & 0xffffu)));
+            fq[2 * w + 1] = __half2float(__ushort_as_half(static_cast<unsigned short>(wq[w] >> 16)));
+          }
+        }
+        float sp = 0.f, sr = 0.f;
+#pragma unroll
+        for (int e = 0; e < E; ++e) take(fb[e], v * E + e, sp, sr, fq[e]);
+        prest += static_cast<double>(sp);
+        rrest += static_cast<double>(sr);
+      }
+    }
+  } else {
+    for (int64_t j = tid; j < V; j += kTopkThreads) {
+      float sp = 0.f, sr = 0.f;
+      take(load_el<DT>(rb, j), j, sp, sr, load_el<DT>(rq, j));
+      prest += static_cast<double>(sp);
+      rrest += static_cast<double>(sr);
+    }
+  }
+}
+
+// Bitonic sort of sh.cand[0..n) descending; zeros pad to a power of 2.
+__device__ void sort_cand(TopkShared& sh, int n) {
+  const int tid = threadIdx.x;
+  int p2 = 1;
+  while (p2 < n) p2 <<= 1;
+  for (int i = n + tid; i < p2; i += kTopkThreads) sh.cand[i] = 0ull;
+  __syncthreads();
+  for (int kk = 2; kk <= p2; kk <<= 1) {
+    for (int jj = kk >> 1; jj > 0; jj >>= 1) {
+      for (int i = tid; i < p2; i += kTopkThreads) {
+        const int ixj = i ^ jj;
+        if (ixj > i) {
+          const unsigned long long x = sh.cand[i], y = sh.cand[ixj];
+          const bool desc = (i & kk) == 0;
+          if (desc ? (x < y) : (x > y)) {
+            sh.cand[i] = y;
+            sh.cand[ixj] = x;
+          }
+        }
+      }
+      __syncthreads();
+    }
+  }
+}
+
+// T (the first kt sorted candidates): indices, log P_base and this thread's
+// share of sum_T p_j log(p_j / r_j); inf_t = 1 if the quant row gives an
+// element of T no mass.
+template <int DT>
+__device__ void t_terms(const TopkShared& sh, const char* rb, const char* rq, const RowAux& a,
+                        int64_t r, int k, int kt, double lambda, int32_t* idx_out,
+                        float* logp_out, double& kl_t, double& inf_t) {
+  for (int i = threadIdx.x; i < k; i += kTopkThreads) {
+    if (i < kt) {
+      const uint32_t j = 0xffffffffu - static_cast<uint32_t>(sh.cand[i]);
+      const float bj = load_el<DT>(rb, j), qj = load_el<DT>(rq, j);
+      const double lp = lambda * static_cast<double>(bj) - a.lse_b;
+      if (idx_out) idx_out[r * k + i] = static_cast<int32_t>(j);
+      if (logp_out) logp_out[r * k + i] = static_cast<float>(lp);
+      if (bj != -INFINITY) {
+        if (qj == -INFINITY) {
+          inf_t = 1.0;
+        } else {
+          // x rounded exactly as the row pass rounds it, so that it agrees
+          // with the log1p(B/S) that pass summed from the same values (an
+          // exact x would leave their mean rounding error, ~1e-6 for a
+          // quant row offset from the base by 1000, in the result)
+          const float x = __fadd_rn(__fsub_rn(qj, bj), a.K);
+          const double lratio = a.lr - lambda * static_cast<double>(x);  // log p_j - log r_j
+          kl_t += exp(lp) * lratio;
+        }
+      }
+    } else {
+      if (idx_out) idx_out[r * k + i] = -1;
+      if (logp_out) logp_out[r * k + i] = -INFINITY;
+    }
+  }
+}
+
+// Block sums and the row's outputs.
+__device__ void finish_row(TopkShared& sh, int64_t r, double kl_t, double inf_t, double prest,
+                           double rrest, float* rest_out, double* kl_out) {
+  kl_t = block_sum(sh, kl_t, 0);
+  inf_t = block_sum(sh, inf_t, 1);
+  prest = block_sum(sh, prest, 2);
+  rrest = block_sum(sh, rrest, 3);
+  if (threadIdx.x == 0) {
+    double kl = kl_t;
+    bool inf = inf_t > 0.0;
+    if (prest > 0.0) {
+      if (rrest > 0.0)
+        kl += prest * (log(prest) - log(rrest));
+      else
+        inf = true;
+    }
+    if (rest_out) rest_out[r] = prest > 0.0 ? static_cast<float>(log(prest)) : -INFINITY;
+    kl_out[r] = inf ? INFINITY : kl;
+  }
+}
+
+template <int DT>
+__global__ void __launch_bounds__(kTopkThreads, kTopkCtasPerSm)
     kld_topk_kernel(const void* __restrict__ base, const void* __restrict__ quant,
                     const RowAux* __restrict__ aux, int64_t N, int64_t V, int k,
                     int32_t* __restrict__ idx_out, float* __restrict__ logp_out,
@@ -152,7 +363,32 @@ __global__ void __launch_bounds__(kTopkThreads)
       continue;
     }
 
-    // ---- threshold key: MSB radix select for the kt-th largest key
+    // ---- fast path: sampled threshold, one fused pass over both rows
+    {
+      const uint32_t t0 = V > kCap ? sample_threshold<DT>(sh, rb, V, kt) : 0u;
+      if (tid == 0) sh.ncand = 0;
+      __syncthreads();
+      double prest = 0.0, rrest = 0.0;
+      gather_pass<DT>(sh, rb, rq, V, t0, a, prest, rrest);
+      __syncthreads();
+      const int n = sh.ncand;
+      if (n >= kt && n <= kCap) {
+        sort_cand(sh, n);
+        double kl_t = 0.0, inf_t = 0.0;
+        t_terms<DT>(sh, rb, rq, a, r, k, kt, lambda, idx_out, logp_out, kl_t, inf_t);
+        // candidates beyond T join the rest
+        for (int i = kt + tid; i < n; i += kTopkThreads) {
+          const uint32_t j = 0xffffffffu - static_cast<uint32_t>(sh.cand[i]);
+          prest += static_cast<double>(rest_b(key_float(static_cast<uint32_t>(sh.cand[i] >> 32)), a));
+          rrest += static_cast<double>(rest_q(load_el<DT>(rq, j), a));
+        }
+        __syncthreads();  // everyone is done with cand before the next row reuses it
+        finish_row(sh, r, kl_t, inf_t, prest, rrest, rest_out, kl_out);
+        continue;
+      }
+    }
+
+    // ---- exact path. Threshold key: MSB radix select for the kt-th largest key
     uint32_t prefix = 0u, mask = 0u;
     unsigned need = static_cast<unsigned>(kt);
     unsigned ncount = static_cast<unsigned>(V);  // elements matching the prefix
@@ -238,56 +474,9 @@ __global__ void __launch_bounds__(kTopkThreads)
     }
     __syncthreads();
 
-    // ---- sort the candidates descending (bitonic), zeros pad to a power of 2
-    const int n = sh.ncand;
-    int p2 = 1;
-    while (p2 < n) p2 <<= 1;
-    for (int i = n + tid; i < p2; i += kTopkThreads) sh.cand[i] = 0ull;
-    __syncthreads();
-    for (int kk = 2; kk <= p2; kk <<= 1) {
-      for (int jj = kk >> 1; jj > 0; jj >>= 1) {
-        for (int i = tid; i < p2; i += kTopkThreads) {
-          const int ixj = i ^ jj;
-          if (ixj > i) {
-            const unsigned long long x = sh.cand[i], y = sh.cand[ixj];
-            const bool desc = (i & kk) == 0;
-            if (desc ? (x < y) : (x > y)) {
-              sh.cand[i] = y;
-              sh.cand[ixj] = x;
-            }
-          }
-        }
-        __syncthreads();
-      }
-    }
-
-    // ---- T: log P_base and the KL terms
+    sort_cand(sh, sh.ncand);
     double kl_t = 0.0, inf_t = 0.0;
-    for (int i = tid; i < k; i += kTopkThreads) {
-      if (i < kt) {
-        const uint32_t j = 0xffffffffu - static_cast<uint32_t>(sh.cand[i]);
-        const float bj = load_el<DT>(rb, j), qj = load_el<DT>(rq, j);
-        const double lp = lambda * static_cast<double>(bj) - a.lse_b;
-        if (idx_out) idx_out[r * k + i] = static_cast<int32_t>(j);
-        if (logp_out) logp_out[r * k + i] = static_cast<float>(lp);
-        if (bj != -INFINITY) {
-          if (qj == -INFINITY) {
-            inf_t = 1.0;
-          } else {
-            // x rounded exactly as the row pass rounds it, so that it agrees
-            // with the log1p(B/S) that pass summed from the same values (an
-            // exact x would leave their mean rounding error, ~1e-6 for a
-            // quant row offset from the base by 1000, in the result)
-            const float x = __fadd_rn(__fsub_rn(qj, bj), a.K);
-            const double lratio = a.lr - lambda * static_cast<double>(x);  // log p_j - log r_j
-            kl_t += exp(lp) * lratio;
-          }
-        }
-      } else {
-        if (idx_out) idx_out[r * k + i] = -1;
-        if (logp_out) logp_out[r * k + i] = -INFINITY;
-      }
-    }
+    t_terms<DT>(sh, rb, rq, a, r, k, kt, lambda, idx_out, logp_out, kl_t, inf_t);
     // membership of T: key above the last selected, or equal with an index
     // no larger than its
     const unsigned long long last = sh.cand[kt - 1];
@@ -298,27 +487,11 @@ __global__ void __launch_bounds__(kTopkThreads)
       const float bj = load_el<DT>(rb, j);
       const uint32_t key = okey(bj);
       if (key > tau_f || (key == tau_f && static_cast<uint32_t>(j) <= j_f)) continue;
-      const float qj = load_el<DT>(rq, j);
-      prest += static_cast<double>(__fmul_rn(ex2(fmaf(bj, kL, -a.Fb)), a.mb));
-      rrest += static_cast<double>(__fmul_rn(ex2(fmaf(qj, kL, -a.Fq)), a.mq));
+      prest += static_cast<double>(rest_b(bj, a));
+      rrest += static_cast<double>(rest_q(load_el<DT>(rq, j), a));
     }
     __syncthreads();  // everyone is done with cand before the next row reuses it
-    kl_t = block_sum(sh, kl_t, 0);
-    inf_t = block_sum(sh, inf_t, 1);
-    prest = block_sum(sh, prest, 2);
-    rrest = block_sum(sh, rrest, 3);
-    if (tid == 0) {
-      double kl = kl_t;
-      bool inf = inf_t > 0.0;
-      if (prest > 0.0) {
-        if (rrest > 0.0)
-          kl += prest * (log(prest) - log(rrest));
-        else
-          inf = true;
-      }
-      if (rest_out) rest_out[r] = prest > 0.0 ? static_cast<float>(log(prest)) : -INFINITY;
-      kl_out[r] = inf ? INFINITY : kl;
-    }
+    finish_row(sh, r, kl_t, inf_t, prest, rrest, rest_out, kl_out);
   }
 }
 
@@ -330,7 +503,7 @@ cudaError_t launch_typed(const void* base, const void* quant, const RowAux* aux,
   cudaError_t e = cudaFuncSetAttribute(kld_topk_kernel<DT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  int64_t grid = static_cast<int64_t>(sm_count) * 4;
+  int64_t grid = static_cast<int64_t>(sm_count) * kTopkCtasPerSm;
   if (grid > N) grid = N;
   kld_topk_kernel<DT><<<static_cast<unsigned>(grid), kTopkThreads, smem, s>>>(base, quant, aux, N, V, k,
                                                                             idx, logp, rest, kl);
