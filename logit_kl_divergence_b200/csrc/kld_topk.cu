@@ -12,10 +12,11 @@
 // x_j = (q_j - b_j) + K rounded to fp32 as the row pass rounds it, the rest
 // in fp64.
 //
-// One CTA per row (persistent over rows, two per SM). Fast path: 4096
-// evenly spaced samples of the base row give a threshold key t0 (the bin of
-// the m-th largest sample, m ~ 1.5 k * 4096 / V + 8, refined by a second
-// digit when the bin is wide), and one fused pass over both rows appends
+// One CTA per row (persistent over rows, four per SM). Fast path: 4096
+// samples of the base row (512 evenly spaced runs of 8 adjacent elements,
+// one memory sector each) give a threshold key t0 (the m-th
+// largest sample, m ~ 1.5 k * 4096 / V + 8, to 21 bits by two 11-bit
+// histogram levels), and one fused pass over both rows appends
 // every element with key >= t0 to a shared candidate list and sums the rest
 // masses of all other elements: each logit is read once. If fewer than k or
 // more than kCap elements pass the threshold (ties or extreme rows), an exact
@@ -23,9 +24,10 @@
 // 32-bit keys (11/11/10-bit levels, stopping as soon as the candidates fit
 // in shared memory; for a tie group at the threshold larger than that, the
 // lowest indices in it by a radix select over the index), the candidates,
-// and a last pass for the rest masses (the row is read 2-4 times). Either
-// way the candidates are sorted in shared memory by (key desc, index asc)
-// and the first k are T; candidates beyond T join the rest.
+// and a last pass for the rest masses (the row is read 2-4 times). T is the
+// first k candidates by (key desc, index asc): ranked by counting when there
+// are at most kRankMax of them (the fast path's usual few hundred), else by
+// a bitonic sort in shared memory; candidates beyond T join the rest.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -36,12 +38,13 @@
 namespace kld {
 namespace {
 
-constexpr int kTopkThreads = 512;
+constexpr int kTopkThreads = 256;
 constexpr int kTopkWarps = kTopkThreads / 32;
-constexpr int kTopkCtasPerSm = 2;
+constexpr int kTopkCtasPerSm = 4;
 constexpr int kHistBins = 2048;
 constexpr int kCap = 4096;  // candidates sorted in shared memory
 constexpr int kSample = 4096;  // samples of a row for the threshold
+constexpr int kRankMax = 1536;  // at most this many candidates: rank by counting
 constexpr float kL = 1.4426950408889634f;  // log2(e) rounded to fp32, as the row pass
 constexpr double kLn2 = 0.6931471805599453;
 
@@ -74,7 +77,7 @@ __device__ __forceinline__ float ex2(float x) {
 
 struct TopkShared {
   unsigned hist[kHistBins];
-  unsigned long long cand[kCap];
+  unsigned long long cand[kCap + kMaxTopk];  // candidates, then T sorted by rank
   double red[kTopkWarps][4];
   int ncand;
   unsigned sel[3];  // bin, count above it, count in it
@@ -143,8 +146,11 @@ __device__ uint32_t sample_threshold(TopkShared& sh, const char* rb, int64_t V, 
   uint32_t* skey = reinterpret_cast<uint32_t*>(sh.cand);  // kSample keys
   double mm = 1.5 * static_cast<double>(kt) * kSample / static_cast<double>(V) + 8.0;
   const unsigned m = mm > kSample ? static_cast<unsigned>(kSample) : static_cast<unsigned>(mm);
-  for (int i = tid; i < kSample; i += kTopkThreads)
-    skey[i] = okey(load_el<DT>(rb, static_cast<int64_t>(i) * V / kSample));
+  // kSample / 8 evenly spaced runs of 8 adjacent elements (one sector each)
+  for (int i = tid; i < kSample; i += kTopkThreads) {
+    const int64_t start = (static_cast<int64_t>(i >> 3) * (V - 8) / (kSample / 8)) & ~static_cast<int64_t>(7);
+    skey[i] = okey(load_el<DT>(rb, start + (i & 7)));
+  }
   for (int i = tid; i < kHistBins; i += kTopkThreads) sh.hist[i] = 0u;
   __syncthreads();
   for (int i = tid; i < kSample; i += kTopkThreads) atomicAdd(&sh.hist[skey[i] >> 21], 1u);
@@ -152,9 +158,9 @@ __device__ uint32_t sample_threshold(TopkShared& sh, const char* rb, int64_t V, 
   find_bin(sh, kHistBins, m, true);
   const uint32_t bin = sh.sel[0], above = sh.sel[1], inbin = sh.sel[2];
   uint32_t t0 = bin << 21;
-  const double per = static_cast<double>(V) / kSample;  // row elements per sample
-  if (static_cast<double>(above + inbin) * per > 0.5 * kCap && inbin > 1) {
-    // wide bin: the next 11 bits of the samples in it
+  if (inbin > 1) {
+    // the next 11 bits of the samples in the bin (a bin of the first digit
+    // spans a quarter of a binade: too coarse near the top of a row)
     __syncthreads();
     for (int i = tid; i < kHistBins; i += kTopkThreads) sh.hist[i] = 0u;
     __syncthreads();
@@ -167,6 +173,7 @@ __device__ uint32_t sample_threshold(TopkShared& sh, const char* rb, int64_t V, 
   __syncthreads();  // the sample keys share memory with the candidates
   return t0;
 }
+
 
 // Rest-mass terms of one element (fp32, as the row pass rounds them).
 __device__ __forceinline__ float rest_b(float bj, const RowAux& a) {
@@ -253,6 +260,42 @@ __device__ void gather_pass(TopkShared& sh, const char* rb, const char* rq, int6
   }
 }
 
+// The first kt of the n (unique) candidates in descending order, by counting
+// for each candidate how many are larger: for the few hundred candidates of
+// the fast path this beats a bitonic network and its barriers. T goes to
+// sh.cand[kCap .. kCap + kt) (the sorted list the outputs read), candidates
+// beyond T add to the rest masses.
+template <int DT>
+__device__ void rank_select(TopkShared& sh, int n, int kt, const char* rq, const RowAux& a,
+                            double& prest, double& rrest) {
+  unsigned long long* out = sh.cand + kCap;
+  for (int e0 = threadIdx.x; e0 < n; e0 += 2 * kTopkThreads) {
+    const int e1 = e0 + kTopkThreads;
+    const unsigned long long x0 = sh.cand[e0];
+    const unsigned long long x1 = e1 < n ? sh.cand[e1] : ~0ull;
+    int r0 = 0, r1 = 0;
+    for (int i = 0; i < n; ++i) {
+      const unsigned long long y = sh.cand[i];  // same address in every lane: broadcast
+      r0 += y > x0;
+      r1 += y > x1;
+    }
+    const unsigned long long xs[2] = {x0, x1};
+    const int rs[2] = {r0, r1};
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      if (u == 1 && e1 >= n) break;
+      if (rs[u] < kt) {
+        out[rs[u]] = xs[u];
+      } else {
+        const uint32_t j = 0xffffffffu - static_cast<uint32_t>(xs[u]);
+        prest += static_cast<double>(rest_b(key_float(static_cast<uint32_t>(xs[u] >> 32)), a));
+        rrest += static_cast<double>(rest_q(load_el<DT>(rq, j), a));
+      }
+    }
+  }
+  __syncthreads();
+}
+
 // Bitonic sort of sh.cand[0..n) descending; zeros pad to a power of 2.
 __device__ void sort_cand(TopkShared& sh, int n) {
   const int tid = threadIdx.x;
@@ -282,12 +325,12 @@ __device__ void sort_cand(TopkShared& sh, int n) {
 // share of sum_T p_j log(p_j / r_j); inf_t = 1 if the quant row gives an
 // element of T no mass.
 template <int DT>
-__device__ void t_terms(const TopkShared& sh, const char* rb, const char* rq, const RowAux& a,
-                        int64_t r, int k, int kt, double lambda, int32_t* idx_out,
-                        float* logp_out, double& kl_t, double& inf_t) {
+__device__ void t_terms(const unsigned long long* sorted, const char* rb, const char* rq,
+                        const RowAux& a, int64_t r, int k, int kt, double lambda,
+                        int32_t* idx_out, float* logp_out, double& kl_t, double& inf_t) {
   for (int i = threadIdx.x; i < k; i += kTopkThreads) {
     if (i < kt) {
-      const uint32_t j = 0xffffffffu - static_cast<uint32_t>(sh.cand[i]);
+      const uint32_t j = 0xffffffffu - static_cast<uint32_t>(sorted[i]);
       const float bj = load_el<DT>(rb, j), qj = load_el<DT>(rq, j);
       const double lp = lambda * static_cast<double>(bj) - a.lse_b;
       if (idx_out) idx_out[r * k + i] = static_cast<int32_t>(j);
@@ -373,14 +416,19 @@ __global__ void __launch_bounds__(kTopkThreads, kTopkCtasPerSm)
       __syncthreads();
       const int n = sh.ncand;
       if (n >= kt && n <= kCap) {
-        sort_cand(sh, n);
         double kl_t = 0.0, inf_t = 0.0;
-        t_terms<DT>(sh, rb, rq, a, r, k, kt, lambda, idx_out, logp_out, kl_t, inf_t);
-        // candidates beyond T join the rest
-        for (int i = kt + tid; i < n; i += kTopkThreads) {
-          const uint32_t j = 0xffffffffu - static_cast<uint32_t>(sh.cand[i]);
-          prest += static_cast<double>(rest_b(key_float(static_cast<uint32_t>(sh.cand[i] >> 32)), a));
-          rrest += static_cast<double>(rest_q(load_el<DT>(rq, j), a));
+        if (n <= kRankMax) {
+          rank_select<DT>(sh, n, kt, rq, a, prest, rrest);
+          t_terms<DT>(sh.cand + kCap, rb, rq, a, r, k, kt, lambda, idx_out, logp_out, kl_t, inf_t);
+        } else {
+          sort_cand(sh, n);
+          t_terms<DT>(sh.cand, rb, rq, a, r, k, kt, lambda, idx_out, logp_out, kl_t, inf_t);
+          // candidates beyond T join the rest
+          for (int i = kt + tid; i < n; i += kTopkThreads) {
+            const uint32_t j = 0xffffffffu - static_cast<uint32_t>(sh.cand[i]);
+            prest += static_cast<double>(rest_b(key_float(static_cast<uint32_t>(sh.cand[i] >> 32)), a));
+            rrest += static_cast<double>(rest_q(load_el<DT>(rq, j), a));
+          }
         }
         __syncthreads();  // everyone is done with cand before the next row reuses it
         finish_row(sh, r, kl_t, inf_t, prest, rrest, rest_out, kl_out);
@@ -476,7 +524,7 @@ __global__ void __launch_bounds__(kTopkThreads, kTopkCtasPerSm)
 
     sort_cand(sh, sh.ncand);
     double kl_t = 0.0, inf_t = 0.0;
-    t_terms<DT>(sh, rb, rq, a, r, k, kt, lambda, idx_out, logp_out, kl_t, inf_t);
+    t_terms<DT>(sh.cand, rb, rq, a, r, k, kt, lambda, idx_out, logp_out, kl_t, inf_t);
     // membership of T: key above the last selected, or equal with an index
     // no larger than its
     const unsigned long long last = sh.cand[kt - 1];
