@@ -169,9 +169,34 @@ def cpu_baseline(name: str, budget_s: float = 12.0, max_rows: int = 4096):
     r = oracle.rows(w.base, w.quant, w.token_ids, odt[w.dtype], 1)
     oracle.reduce(r, True)
     dt = time.perf_counter() - t0
-    return {"value": rows / dt, "unit": "rows/s", "cores": 1, "kind": "oracle",
-            "sample": f"{rows} rows of {name} (same recipe, host-generated), "
-                      f"fp64 two-pass oracle, single thread, {dt:.1f} s"}
+    single = {"value": rows / dt, "unit": "rows/s", "cores": 1, "kind": "oracle",
+              "sample": f"{rows} rows of {name} (same recipe, host-generated), "
+                        f"fp64 two-pass oracle, single thread, {dt:.1f} s",
+              "cpu_model": _cpu_model()}
+    # The same per-row code on every host core (whole rows per thread, so the
+    # records are bit-identical to the single-threaded run).
+    cores = os.cpu_count() or 1
+    rows_mt = int(max(cores, min(64 * cores, 8.0 * cores / max(per_row, 1e-6))))
+    w = synth.make(name, n=rows_mt, seed=synth.WORKLOADS[name][4] + 2000)
+    t0 = time.perf_counter()
+    r = oracle.rows(w.base, w.quant, w.token_ids, odt[w.dtype], cores)
+    oracle.reduce(r, True)
+    dt = time.perf_counter() - t0
+    multi = {"value": rows_mt / dt, "unit": "rows/s", "cores": cores, "kind": "oracle",
+             "sample": f"{rows_mt} rows of {name}, the same oracle row-parallel on {cores} "
+                       f"threads, {dt:.1f} s"}
+    return single, multi
+
+
+def _cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
 
 
 def run_reference(args, rank: int):
@@ -534,20 +559,20 @@ def main():
         torch.cuda.empty_cache()
         split_row = split_row_latency(dev, stream, max(1, args.split_calls))
 
-    cpu = None
+    cpu = cpu_mt = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline(name)
+        cpu, cpu_mt = cpu_baseline(name)
 
     if rank == 0:
         line = {
             "metric": METRIC, "value": value, "unit": "rows/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-            "config": {"workload": name, "rows_per_gpu": N, "vocab": V, "logit_dtype": "f32",
+            "scaling": "weak", "vs_baseline": None, "dtype": args.dtype, "data": "synthetic",
+            "config": {"workload": name, "rows_per_gpu": N, "vocab": V, "logit_dtype": args.dtype,
                        "global_rows": total_rows,
                        "parallelism": f"rows sharded over {world} GPU(s), records all-gathered",
                        "l2": "inputs (9.96 GB per step per GPU) exceed the 126 MB L2; no flush"},
-            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+            "roofline": roofline, "cpu_baseline": cpu, "cpu_baseline_all_cores": cpu_mt, "e2e": e2e,
             "gpu_launches": 2 * args.steps, "clocks": clocks,
             "gbs": in_bytes * world / (ms_per_step / 1000.0) / 1e9,
             "mean_kld": res["mean_kld"], "top1_agree_pct": res["top1_agree_pct"], "ppl": res["ppl"],
