@@ -1158,6 +1158,19 @@ __global__ void __launch_bounds__(kRowThreads, 1)
         xe_b = Elem<DT>::load(rb, jj);
         xe_q = Elem<DT>::load(rq, jj);
       }
+      // Next-token gather, issued now so that its latency hides behind the
+      // consumers' work (the CTA that finalises the row needs it).
+      int32_t tk = 0;
+      bool tok_ok = false;
+      float q_tok = 0.f, b_tok = 0.f;
+      if (tok != nullptr && part_out == nullptr) {
+        tk = __ldg(tok + r);
+        tok_ok = tk >= 0 && static_cast<int64_t>(tk) < V;
+        if (tok_ok) {
+          q_tok = Elem<DT>::load(rq, tk);
+          b_tok = Elem<DT>::load(rb, tk);
+        }
+      }
       Ref eref{-INFINITY, -INFINITY, 0.f, 0.f, 0.f, -INFINITY};
       Acc eacc{0.0, 0.0, 0.0, 0.0, 0.0, 0.0};
       Best ebest{-INFINITY, -INFINITY, -1, -1};
@@ -1258,20 +1271,6 @@ __global__ void __launch_bounds__(kRowThreads, 1)
       if (lane == 0) mbar_arrive(smem_u32(&ctrl->slot_empty[slot]));
       }
 
-      // Next-token gather (only the CTA that finalises the row needs it).
-      int32_t tk = 0;
-      bool tok_ok = false;
-      float q_tok = 0.f, b_tok = 0.f;
-      auto gather_token = [&]() {
-        if (tok != nullptr) {
-          tk = __ldg(tok + r);
-          tok_ok = tk >= 0 && static_cast<int64_t>(tk) < V;
-          if (tok_ok) {
-            q_tok = Elem<DT>::load(rq, tk);
-            b_tok = Elem<DT>::load(rb, tk);
-          }
-        }
-      };
 
       if (P == 1 && part_out != nullptr) {
         // Vocabulary slice [col0, col0 + V) of a wider row: publish the
@@ -1298,8 +1297,7 @@ __global__ void __launch_bounds__(kRowThreads, 1)
         continue;
       }
       if (P == 1) {
-        gather_token();
-        const kld_row_t rec = finalize_row(m, tok != nullptr, tok_ok, q_tok, b_tok);
+          const kld_row_t rec = finalize_row(m, tok != nullptr, tok_ok, q_tok, b_tok);
         if (lane == 0) {
           rows[r] = rec;
           if (aux != nullptr) aux[r] = row_aux(m, rec);
@@ -1372,8 +1370,7 @@ __global__ void __launch_bounds__(kRowThreads, 1)
       }
       const int C = P / static_cast<int>(G);  // clusters per row
       if (C == 1) {
-        gather_token();
-        const kld_row_t rec = finalize_row(cm, tok != nullptr, tok_ok, q_tok, b_tok);
+          const kld_row_t rec = finalize_row(cm, tok != nullptr, tok_ok, q_tok, b_tok);
         if (lane == 0) {
           rows[r] = rec;
           if (aux != nullptr) aux[r] = row_aux(cm, rec);
@@ -1388,12 +1385,16 @@ __global__ void __launch_bounds__(kRowThreads, 1)
         ulonglong2* dst = reinterpret_cast<ulonglong2*>(&gparts[r * C + cid]);
 #pragma unroll
         for (int w = 0; w < 4; ++w) dst[w] = make_ulonglong2(wds[2 * w], wds[2 * w + 1]);
-        __threadfence();
-        ticket = atomicAdd(&tickets[r], 1u);
+        // release: the partial above is visible to whoever sees the count;
+        // acquire: the last arriver sees every other part's partial
+        asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;"
+                     : "=r"(ticket)
+                     : "l"(&tickets[r])
+                     : "memory");
       }
       ticket = __shfl_sync(0xffffffffu, ticket, 0);
       if (ticket != static_cast<unsigned>(C - 1)) continue;  // not the last cluster
-      __threadfence();
+      __syncwarp();  // lane 0's acquire orders the other lanes' loads below
       MPart q = empty_part();
       if (lane < C) {
         const ulonglong2* src = reinterpret_cast<const ulonglong2*>(&gparts[r * C + lane]);
@@ -1407,7 +1408,6 @@ __global__ void __launch_bounds__(kRowThreads, 1)
         q = part_from_words(wds);
       }
       const MPart fm = warp_merge(q);
-      gather_token();
       const kld_row_t rec = finalize_row(fm, tok != nullptr, tok_ok, q_tok, b_tok);
       if (lane == 0) {
         rows[r] = rec;
