@@ -824,8 +824,21 @@ __device__ MPart warp_merge(const MPart& p) {
 }
 
 // The record of a whole row from its merged partial.
+// Called by a full warp with warp-uniform arguments: the record's three
+// logarithms run at once on lanes 0-2 (all as log1p, so the warp does not
+// diverge) and its two exponentials on lanes 1-2.
 __device__ kld_row_t finalize_row(const MPart& m, bool has_tok, bool tok_ok, float q_tok,
                                   float b_tok) {
+  const int lane = threadIdx.x & 31;
+  // lane 0: log1p(B/S); lane 1: log(B + S); lane 2 and up: log(S). S >= 1
+  // (the frame's maximum weight is at least 1), and B + S >= 0.5 but for
+  // rows whose quant row misses the base maximum (taken apart below).
+  const double bs = m.B + m.Sb;
+  const double lg = log1p(lane == 0 ? m.B / m.Sb : (lane == 1 ? bs - 1.0 : m.Sb - 1.0));
+  const double log1p_bs = __shfl_sync(0xffffffffu, lg, 0);
+  double log_bs = __shfl_sync(0xffffffffu, lg, 1);
+  const double log_s = __shfl_sync(0xffffffffu, lg, 2);
+  if (!(bs >= 0.5)) log_bs = log(bs);
   kld_row_t rec;
   uint32_t flags = 0;
   if (has_tok && !tok_ok) flags |= KLD_ROW_BAD_TOKEN;
@@ -846,7 +859,7 @@ __device__ kld_row_t finalize_row(const MPart& m, bool has_tok, bool tok_ok, flo
       rec.kld = INFINITY;
       flags |= KLD_ROW_INF_KL;
     } else {
-      rec.kld = -kLambda * (m.A / m.Sb) + log1p(m.B / m.Sb);
+      rec.kld = -kLambda * (m.A / m.Sb) + log1p_bs;
     }
     if (tok_ok) {
       if (q_tok == -INFINITY) {
@@ -854,7 +867,7 @@ __device__ kld_row_t finalize_row(const MPart& m, bool has_tok, bool tok_ok, flo
         flags |= KLD_ROW_INF_NLL;
       } else {
         // B + S is the sum of all quant weights in frame Cb - K*L.
-        rec.nll = log(m.B + m.Sb) +
+        rec.nll = log_bs +
                   kLn2 * (static_cast<double>(m.Cb) -
                           (static_cast<double>(m.K) + static_cast<double>(q_tok)) * kLog2eD);
       }
@@ -863,7 +876,7 @@ __device__ kld_row_t finalize_row(const MPart& m, bool has_tok, bool tok_ok, flo
         flags |= KLD_ROW_INF_NLL_BASE;
       } else {
         // S is the sum of all base weights in frame Cb.
-        rec.nll_base = log(m.Sb) + kLn2 * (static_cast<double>(m.Cb) -
+        rec.nll_base = log_s + kLn2 * (static_cast<double>(m.Cb) -
                                            static_cast<double>(b_tok) * kLog2eD);
       }
     }
@@ -872,7 +885,8 @@ __device__ kld_row_t finalize_row(const MPart& m, bool has_tok, bool tok_ok, flo
   }
   rec.flags = flags;
   // P(tok) = exp(-NLL) for each model (exp(-inf) = 0), differenced in fp64
-  rec.dp = static_cast<float>(exp(-rec.nll) - exp(-rec.nll_base));
+  const double ex = exp(-(lane == 1 ? rec.nll : rec.nll_base));
+  rec.dp = static_cast<float>(__shfl_sync(0xffffffffu, ex, 1) - __shfl_sync(0xffffffffu, ex, 2));
   return rec;
 }
 
