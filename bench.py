@@ -80,9 +80,15 @@ def recorded_traffic(workload: str):
 
 
 class ClockSampler:
-    """SM clock and throttle reasons sampled during the timed region: NVML
-    polled from a thread every ~2 ms (the region lasts tens of ms), with
-    nvidia-smi as the fallback."""
+    """SM clock and throttle reasons during the timed region.
+
+    NVML is polled from a thread every ~2 ms with a host timestamp per sample
+    (nvidia-smi at 100 ms as the fallback). The sampler starts before the
+    warm-up steps, so that polling is already running when the timed region
+    opens; `mark_start` / `mark_end` bracket that region on the host clock and
+    `stop` reports the samples inside it. A region too short to hold three
+    samples also reports the warm-up samples (they run the same kernels) and
+    says so in "window"."""
 
     REASONS = {  # NVML clocks-event reason bits
         "hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
@@ -92,7 +98,9 @@ class ClockSampler:
     def __init__(self, gpu_index: int):
         import threading
 
-        self.samples, self.maxes, self.reasons = [], [], set()
+        self.samples = []  # (host time, sm MHz, max sm MHz, reason names)
+        self.t_start = self.t_end = None
+        self.t_open = time.perf_counter()
         self._stop = threading.Event()
         self._thread = None
         self._proc = None
@@ -117,20 +125,26 @@ class ClockSampler:
         nv, h = self._nv, self._h
         while not self._stop.is_set():
             try:
-                self.samples.append(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM))
-                self.maxes.append(nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM))
+                sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+                mx = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
                 bits = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
-                for name, bit in self.REASONS.items():
-                    if bits & bit:
-                        self.reasons.add(name)
+                names = {name for name, bit in self.REASONS.items() if bits & bit}
+                self.samples.append((time.perf_counter(), sm, mx, names))
             except Exception:
                 pass
             self._stop.wait(0.002)
+
+    def mark_start(self):
+        self.t_start = time.perf_counter()
+
+    def mark_end(self):
+        self.t_end = time.perf_counter()
 
     def stop(self):
         if self._thread is not None:
             self._stop.set()
             self._thread.join(timeout=5)
+            samples = self.samples
         elif self._proc is not None:
             self._proc.terminate()
             try:
@@ -138,17 +152,37 @@ class ClockSampler:
             except subprocess.TimeoutExpired:
                 self._proc.kill()
                 out, _ = self._proc.communicate()
-            for line in out.strip().splitlines():
+            # nvidia-smi lines carry no host time: spread them evenly over
+            # the sampler's lifetime.
+            lines = out.strip().splitlines()
+            t1 = time.perf_counter()
+            samples = []
+            for i, line in enumerate(lines):
                 parts = [x.strip() for x in line.split(",")]
                 try:
-                    self.samples.append(float(parts[0]))
-                    self.maxes.append(float(parts[1]))
+                    t = self.t_open + (t1 - self.t_open) * (i + 0.5) / max(1, len(lines))
+                    samples.append((t, float(parts[0]), float(parts[1]), set()))
                 except (ValueError, IndexError):
                     continue
-        if not self.samples:
+        else:
             return None
-        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": max(self.maxes),
-                "reasons": sorted(self.reasons), "samples": len(self.samples),
+        t0 = self.t_start if self.t_start is not None else self.t_open
+        t1 = self.t_end if self.t_end is not None else time.perf_counter()
+        inside = [s for s in samples if t0 <= s[0] <= t1]
+        window = "timed region"
+        if len(inside) < 3:
+            inside = [s for s in samples if s[0] <= t1]
+            window = "warm-up and timed region (the timed region alone held fewer than 3 samples)"
+        if not inside:
+            return None
+        reasons = set()
+        for s in inside:
+            reasons |= s[3]
+        return {"sm_mhz": statistics.median(s[1] for s in inside),
+                "sm_max_mhz": max(s[2] for s in inside),
+                "sm_min_mhz": min(s[1] for s in inside),
+                "reasons": sorted(reasons), "samples": len(inside), "window": window,
+                "timed_region_ms": round(1000.0 * (t1 - t0), 3),
                 "source": "nvml" if self._thread is not None else "nvidia-smi"}
 
 
@@ -394,6 +428,7 @@ def main():
             res = st.result()
         return res
 
+    sampler = ClockSampler(local)
     for _ in range(args.warmup):
         res = step(False)
 
@@ -402,11 +437,11 @@ def main():
     if world > 1:
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
 
-    sampler = ClockSampler(local)
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize(dev)
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler.mark_start()
     start.record(stream)
     for _ in range(args.steps):
         if world == 1:
@@ -421,6 +456,7 @@ def main():
             row_ms.append(e0.elapsed_time(e1))
     end.record(stream)
     torch.cuda.synchronize(dev)
+    sampler.mark_end()
     if world > 1:
         dist.barrier()
     clocks = sampler.stop()
