@@ -306,8 +306,9 @@ kld_status_t kld_selftest_bounded_wait(int device, uint64_t limit_ns, int use_ab
                                        uint64_t* waited_ns);
 
 /*
- * Duration in milliseconds of the last kld_stats_run_grad's gradient pass
- * (timing enabled by kld_stats_set_timing; waits for that run).
+ * Duration in milliseconds of the pass that follows the reduction in the
+ * last kld_stats_run_grad (the gradient pass) or kld_stats_run_topk (the
+ * top-k pass); timing enabled by kld_stats_set_timing; waits for that run.
  */
 kld_status_t kld_stats_grad_timing(kld_stats_t h, float* grad_ms);
 

@@ -159,7 +159,8 @@ class KLDStats:
         return out
 
     def grad_timing(self) -> float:
-        """Milliseconds of the last run_grad's gradient pass (timing enabled)."""
+        """Milliseconds of the last run_grad's gradient pass or run_topk's
+        top-k pass (timing enabled)."""
         ms = ctypes.c_float()
         _lib.check(self._lib.kld_stats_grad_timing(self._h, ctypes.byref(ms)), "kld_stats_grad_timing")
         return ms.value

@@ -383,14 +383,17 @@ kld_status_t kld_stats_run_topk(kld_stats_t h, const void* base, const void* qua
   DeviceGuard guard(h->device);
   if (!guard.ok()) return cuda_fail(cudaGetLastError(), "cudaSetDevice");
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  h->timing_valid = false;
-  h->grad_timing_valid = false;
+  h->timing_valid = h->timing;
+  h->grad_timing_valid = h->timing;
+  if (h->timing) KLD_CUDA(cudaEventRecord(h->tev[0], s));
   KLD_CUDA(launch_rows(h, base, quant, token_ids, N, V, dtype, h->rows, s, h->aux));
+  if (h->timing) KLD_CUDA(cudaEventRecord(h->tev[1], s));
   h->last_rows = N;
   st = enqueue_reduce(h, h->rows, N, token_ids != nullptr, s);
   if (st != KLD_OK) return st;
   KLD_CUDA(kld::launch_topk(base, quant, h->aux, N, V, dtype, k, idx_out, logp_out, rest_out,
                             kl_out, h->sm_count, s));
+  if (h->timing) KLD_CUDA(cudaEventRecord(h->tev[3], s));
   return KLD_OK;
 }
 

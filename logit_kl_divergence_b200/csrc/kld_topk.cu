@@ -26,8 +26,10 @@
 // lowest indices in it by a radix select over the index), the candidates,
 // and a last pass for the rest masses (the row is read 2-4 times). T is the
 // first k candidates by (key desc, index asc): ranked by counting when there
-// are at most kRankMax of them (the fast path's usual few hundred), else by
-// a bitonic sort in shared memory; candidates beyond T join the rest.
+// are at most kRankMax of them (the fast path's usual few hundred; with many
+// more than k, a histogram of the candidates' keys first leaves only those
+// in or above the bin of the k-th largest to be ranked), else by a bitonic
+// sort in shared memory; candidates beyond T join the rest.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -45,8 +47,12 @@ constexpr int kHistBins = 2048;
 constexpr int kCap = 4096;  // candidates sorted in shared memory
 constexpr int kSample = 4096;  // samples of a row for the threshold
 constexpr int kRankMax = 1536;  // at most this many candidates: rank by counting
+constexpr int kSetBase = 2048;  // where the boundary set of the ranking is kept in cand[]
+static_assert(kSetBase >= kRankMax && kSetBase + kRankMax <= kCap, "boundary set layout");
 constexpr float kL = 1.4426950408889634f;  // log2(e) rounded to fp32, as the row pass
 constexpr double kLn2 = 0.6931471805599453;
+constexpr int kGatherUnroll = 2;  // 16-byte vectors per operand per thread per step
+static_assert(kSample % kTopkThreads == 0, "sample loads per thread");
 
 template <int DT>
 __device__ __forceinline__ float load_el(const char* row, int64_t j);
@@ -79,39 +85,53 @@ struct TopkShared {
   unsigned hist[kHistBins];
   unsigned long long cand[kCap + kMaxTopk];  // candidates, then T sorted by rank
   double red[kTopkWarps][4];
+  unsigned wmax[kTopkWarps];
   int ncand;
+  int nset;
   unsigned sel[3];  // bin, count above it, count in it
 };
 
 // Block-wide: the bin holding the `need`-th element counting from the top
 // (descending = true) or the bottom of hist[0..bins). Returns (bin, count
-// before it in that direction, count in it) through sh.sel.
+// before it in that direction, count in it) through sh.sel. Warp 0 scans the
+// lanes' contiguous segments of bins/32 bins, then the owner segment again
+// with a few bins per lane, so no lane walks more than a couple of bins.
+__device__ __forceinline__ unsigned warp_incl_scan(unsigned v, int lane) {
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const unsigned t = __shfl_up_sync(0xffffffffu, v, o);
+    if (lane >= o) v += t;
+  }
+  return v;
+}
 __device__ void find_bin(TopkShared& sh, int bins, unsigned need, bool descending) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (warp == 0) {
+    auto bin_at = [&](int pos) { return descending ? bins - 1 - pos : pos; };  // pos: scan order
     const int per = bins / 32;  // bins per lane, contiguous in scan order
     unsigned part = 0;
-    for (int i = 0; i < per; ++i) {
-      const int b = descending ? bins - 1 - (lane * per + i) : lane * per + i;
-      part += sh.hist[b];
-    }
-    unsigned incl = part;  // inclusive prefix over lanes
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const unsigned v = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += v;
-    }
+    for (int i = 0; i < per; ++i) part += sh.hist[bin_at(lane * per + i)];
+    const unsigned incl = warp_incl_scan(part, lane);
     const unsigned excl = incl - part;
     const unsigned hit = __ballot_sync(0xffffffffu, excl < need && incl >= need);
     const int owner = hit ? __ffs(hit) - 1 : 31;
-    if (lane == owner) {
-      unsigned cum = excl;
-      int bin = descending ? bins - 1 - lane * per : lane * per;
-      for (int i = 0; i < per; ++i) {
-        const int b = descending ? bins - 1 - (lane * per + i) : lane * per + i;
-        bin = b;
-        if (cum + sh.hist[b] >= need) break;
-        cum += sh.hist[b];
+    const unsigned cum0 = __shfl_sync(0xffffffffu, excl, owner);
+    // the owner's segment, a few bins per lane
+    const int sub = (per + 31) / 32;
+    const int p0 = owner * per + min(lane * sub, per), p1 = owner * per + min((lane + 1) * sub, per);
+    unsigned part2 = 0;
+    for (int q = p0; q < p1; ++q) part2 += sh.hist[bin_at(q)];
+    const unsigned incl2 = warp_incl_scan(part2, lane) + cum0;
+    const unsigned excl2 = incl2 - part2;
+    const unsigned hit2 = __ballot_sync(0xffffffffu, p1 > p0 && excl2 < need && incl2 >= need);
+    const int own2 = hit2 ? __ffs(hit2) - 1 : 31;
+    if (lane == own2) {
+      unsigned cum = excl2;
+      int bin = bin_at(p0 < p1 ? p0 : p1 - 1);
+      for (int q = p0; q < p1; ++q) {
+        bin = bin_at(q);
+        if (cum + sh.hist[bin] >= need) break;
+        cum += sh.hist[bin];
       }
       sh.sel[0] = static_cast<unsigned>(bin);
       sh.sel[1] = cum;
@@ -121,16 +141,33 @@ __device__ void find_bin(TopkShared& sh, int bins, unsigned need, bool descendin
   __syncthreads();
 }
 
-__device__ double block_sum(TopkShared& sh, double v, int slot) {
+// Block sums of four values at once (one barrier pair); the totals come
+// back in the same variables, summed in a fixed order (lanes by the shuffle
+// tree, then warps in index order), so a row's result does not depend on
+// timing.
+__device__ void block_sum4(TopkShared& sh, double& v0, double& v1, double& v2, double& v3) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  double v[4] = {v0, v1, v2, v3};
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v += __shfl_down_sync(0xffffffffu, v, o);
-  if (lane == 0) sh.red[warp][slot] = v;
+  for (int s = 0; s < 4; ++s) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v[s] += __shfl_down_sync(0xffffffffu, v[s], o);
+  }
+  if (lane == 0) {
+#pragma unroll
+    for (int s = 0; s < 4; ++s) sh.red[warp][s] = v[s];
+  }
   __syncthreads();
-  double t = 0.0;
-  for (int w = 0; w < kTopkWarps; ++w) t += sh.red[w][slot];  // fixed order
+  double t[4] = {0.0, 0.0, 0.0, 0.0};
+  for (int w = 0; w < kTopkWarps; ++w) {
+#pragma unroll
+    for (int s = 0; s < 4; ++s) t[s] += sh.red[w][s];
+  }
   __syncthreads();
-  return t;
+  v0 = t[0];
+  v1 = t[1];
+  v2 = t[2];
+  v3 = t[3];
 }
 
 // Inverse of okey.
@@ -146,14 +183,23 @@ __device__ uint32_t sample_threshold(TopkShared& sh, const char* rb, int64_t V, 
   uint32_t* skey = reinterpret_cast<uint32_t*>(sh.cand);  // kSample keys
   double mm = 1.5 * static_cast<double>(kt) * kSample / static_cast<double>(V) + 8.0;
   const unsigned m = mm > kSample ? static_cast<unsigned>(kSample) : static_cast<unsigned>(mm);
-  // kSample / 8 evenly spaced runs of 8 adjacent elements (one sector each)
-  for (int i = tid; i < kSample; i += kTopkThreads) {
+  // kSample / 8 evenly spaced runs of 8 adjacent elements (one sector each);
+  // every thread issues all of its loads before using any, so the sampling
+  // costs one memory latency instead of one per load
+  constexpr int kPer = kSample / kTopkThreads;
+  float sv[kPer];
+#pragma unroll
+  for (int u = 0; u < kPer; ++u) {
+    const int i = tid + u * kTopkThreads;
     const int64_t start = (static_cast<int64_t>(i >> 3) * (V - 8) / (kSample / 8)) & ~static_cast<int64_t>(7);
-    skey[i] = okey(load_el<DT>(rb, start + (i & 7)));
+    sv[u] = load_el<DT>(rb, start + (i & 7));
   }
+#pragma unroll
+  for (int u = 0; u < kPer; ++u) skey[tid + u * kTopkThreads] = okey(sv[u]);
   for (int i = tid; i < kHistBins; i += kTopkThreads) sh.hist[i] = 0u;
   __syncthreads();
-  for (int i = tid; i < kSample; i += kTopkThreads) atomicAdd(&sh.hist[skey[i] >> 21], 1u);
+#pragma unroll
+  for (int u = 0; u < kPer; ++u) atomicAdd(&sh.hist[okey(sv[u]) >> 21], 1u);
   __syncthreads();
   find_bin(sh, kHistBins, m, true);
   const uint32_t bin = sh.sel[0], above = sh.sel[1], inbin = sh.sel[2];
@@ -209,10 +255,10 @@ __device__ void gather_pass(TopkShared& sh, const char* rb, const char* rq, int6
     const uint4* vb = reinterpret_cast<const uint4*>(rb);
     const uint4* vq = reinterpret_cast<const uint4*>(rq);
     const int64_t nv = V / E;
-    for (int64_t v0 = tid; v0 < nv; v0 += 2 * kTopkThreads) {
-      uint4 xb[2], xq[2];
+    for (int64_t v0 = tid; v0 < nv; v0 += kGatherUnroll * kTopkThreads) {
+      uint4 xb[kGatherUnroll], xq[kGatherUnroll];
 #pragma unroll
-      for (int u = 0; u < 2; ++u) {
+      for (int u = 0; u < kGatherUnroll; ++u) {
         const int64_t v = v0 + u * kTopkThreads;
         if (v < nv) {
           xb[u] = __ldg(vb + v);
@@ -220,7 +266,7 @@ __device__ void gather_pass(TopkShared& sh, const char* rb, const char* rq, int6
         }
       }
 #pragma unroll
-      for (int u = 0; u < 2; ++u) {
+      for (int u = 0; u < kGatherUnroll; ++u) {
         const int64_t v = v0 + u * kTopkThreads;
         if (v >= nv) continue;
         float fb[E], fq[E];
@@ -262,20 +308,79 @@ __device__ void gather_pass(TopkShared& sh, const char* rb, const char* rq, int6
 
 // The first kt of the n (unique) candidates in descending order, by counting
 // for each candidate how many are larger: for the few hundred candidates of
-// the fast path this beats a bitonic network and its barriers. T goes to
-// sh.cand[kCap .. kCap + kt) (the sorted list the outputs read), candidates
-// beyond T add to the rest masses.
+// the fast path this beats a bitonic network and its barriers. When there
+// are many more candidates than kt, a histogram of their keys above t0 first
+// finds the bin that holds the kt-th largest: every candidate below that bin
+// is outside T, and only the ones in it or above (about kt) are ranked
+// against each other. T goes to sh.cand[kCap .. kCap + kt) (the sorted list
+// the outputs read), candidates beyond T add to the rest masses.
 template <int DT>
-__device__ void rank_select(TopkShared& sh, int n, int kt, const char* rq, const RowAux& a,
-                            double& prest, double& rrest) {
+__device__ void rank_select(TopkShared& sh, int n, int kt, uint32_t t0, const char* rq,
+                            const RowAux& a, double& prest, double& rrest) {
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   unsigned long long* out = sh.cand + kCap;
-  for (int e0 = threadIdx.x; e0 < n; e0 += 2 * kTopkThreads) {
+  auto to_rest = [&](unsigned long long x) {
+    const uint32_t j = 0xffffffffu - static_cast<uint32_t>(x);
+    prest += static_cast<double>(rest_b(key_float(static_cast<uint32_t>(x >> 32)), a));
+    rrest += static_cast<double>(rest_q(load_el<DT>(rq, j), a));
+  };
+  const unsigned long long* set = sh.cand;
+  int ns = n;
+  if (n > 2 * kt + 64) {
+    // digit = (key - t0) >> s over 2048 bins, s from the largest key
+    unsigned mx = 0u;
+    for (int e = tid; e < n; e += kTopkThreads)
+      mx = max(mx, static_cast<uint32_t>(sh.cand[e] >> 32) - t0);
+    mx = __reduce_max_sync(0xffffffffu, mx);
+    if (lane == 0) sh.wmax[warp] = mx;
+    for (int i = tid; i < kHistBins; i += kTopkThreads) sh.hist[i] = 0u;
+    if (tid == 0) sh.nset = 0;
+    __syncthreads();
+    mx = 0u;
+#pragma unroll
+    for (int w = 0; w < kTopkWarps; ++w) mx = max(mx, sh.wmax[w]);
+    const int bits = 32 - __clz(mx);  // mx < 2^bits
+    const int s = bits > 11 ? bits - 11 : 0;
+    for (int e = tid; e < n; e += kTopkThreads)
+      atomicAdd(&sh.hist[(static_cast<uint32_t>(sh.cand[e] >> 32) - t0) >> s], 1u);
+    __syncthreads();
+    find_bin(sh, kHistBins, static_cast<unsigned>(kt), true);
+    const uint32_t B = sh.sel[0];
+    unsigned long long* setw = sh.cand + kSetBase;
+    // two candidates per thread and step, so that the quant logits of those
+    // that join the rest are fetched together (one memory latency)
+    for (int e0 = tid; e0 < n; e0 += 2 * kTopkThreads) {
+      const int e1 = e0 + kTopkThreads;
+      const unsigned long long x0 = sh.cand[e0], x1 = e1 < n ? sh.cand[e1] : 0ull;
+      const bool in0 = ((static_cast<uint32_t>(x0 >> 32) - t0) >> s) >= B;
+      const bool in1 = e1 < n && ((static_cast<uint32_t>(x1 >> 32) - t0) >> s) >= B;
+      const bool out1 = e1 < n && !in1;
+      const float q0 = in0 ? 0.f : load_el<DT>(rq, 0xffffffffu - static_cast<uint32_t>(x0));
+      const float q1 = out1 ? load_el<DT>(rq, 0xffffffffu - static_cast<uint32_t>(x1)) : 0.f;
+      if (in0) {
+        setw[atomicAdd(&sh.nset, 1)] = x0;
+      } else {
+        prest += static_cast<double>(rest_b(key_float(static_cast<uint32_t>(x0 >> 32)), a));
+        rrest += static_cast<double>(rest_q(q0, a));
+      }
+      if (in1) {
+        setw[atomicAdd(&sh.nset, 1)] = x1;
+      } else if (out1) {
+        prest += static_cast<double>(rest_b(key_float(static_cast<uint32_t>(x1 >> 32)), a));
+        rrest += static_cast<double>(rest_q(q1, a));
+      }
+    }
+    __syncthreads();
+    set = setw;
+    ns = sh.nset;
+  }
+  for (int e0 = tid; e0 < ns; e0 += 2 * kTopkThreads) {
     const int e1 = e0 + kTopkThreads;
-    const unsigned long long x0 = sh.cand[e0];
-    const unsigned long long x1 = e1 < n ? sh.cand[e1] : ~0ull;
+    const unsigned long long x0 = set[e0];
+    const unsigned long long x1 = e1 < ns ? set[e1] : ~0ull;
     int r0 = 0, r1 = 0;
-    for (int i = 0; i < n; ++i) {
-      const unsigned long long y = sh.cand[i];  // same address in every lane: broadcast
+    for (int i = 0; i < ns; ++i) {
+      const unsigned long long y = set[i];  // same address in every lane: broadcast
       r0 += y > x0;
       r1 += y > x1;
     }
@@ -283,14 +388,11 @@ __device__ void rank_select(TopkShared& sh, int n, int kt, const char* rq, const
     const int rs[2] = {r0, r1};
 #pragma unroll
     for (int u = 0; u < 2; ++u) {
-      if (u == 1 && e1 >= n) break;
-      if (rs[u] < kt) {
+      if (u == 1 && e1 >= ns) break;
+      if (rs[u] < kt)
         out[rs[u]] = xs[u];
-      } else {
-        const uint32_t j = 0xffffffffu - static_cast<uint32_t>(xs[u]);
-        prest += static_cast<double>(rest_b(key_float(static_cast<uint32_t>(xs[u] >> 32)), a));
-        rrest += static_cast<double>(rest_q(load_el<DT>(rq, j), a));
-      }
+      else
+        to_rest(xs[u]);
     }
   }
   __syncthreads();
@@ -358,10 +460,7 @@ __device__ void t_terms(const unsigned long long* sorted, const char* rb, const 
 // Block sums and the row's outputs.
 __device__ void finish_row(TopkShared& sh, int64_t r, double kl_t, double inf_t, double prest,
                            double rrest, float* rest_out, double* kl_out) {
-  kl_t = block_sum(sh, kl_t, 0);
-  inf_t = block_sum(sh, inf_t, 1);
-  prest = block_sum(sh, prest, 2);
-  rrest = block_sum(sh, rrest, 3);
+  block_sum4(sh, kl_t, inf_t, prest, rrest);
   if (threadIdx.x == 0) {
     double kl = kl_t;
     bool inf = inf_t > 0.0;
@@ -418,7 +517,7 @@ __global__ void __launch_bounds__(kTopkThreads, kTopkCtasPerSm)
       if (n >= kt && n <= kCap) {
         double kl_t = 0.0, inf_t = 0.0;
         if (n <= kRankMax) {
-          rank_select<DT>(sh, n, kt, rq, a, prest, rrest);
+          rank_select<DT>(sh, n, kt, t0, rq, a, prest, rrest);
           t_terms<DT>(sh.cand + kCap, rb, rq, a, r, k, kt, lambda, idx_out, logp_out, kl_t, inf_t);
         } else {
           sort_cand(sh, n);

@@ -49,7 +49,8 @@ def _check(b, q, tok, dt, k, split=None):
 
 @pytest.mark.parametrize("dt", [synth.F32, synth.BF16, synth.F16])
 @pytest.mark.parametrize("n,v,k", [(100, 151936, 128), (40, 32000, 1), (40, 32000, 1024),
-                                   (7, 4099, 128), (3, 5, 128), (9, 4096, 4096 // 4)])
+                                   (7, 4099, 128), (3, 5, 128), (9, 4096, 4096 // 4),
+                                   (5, 1000, 128), (4, 1536, 1), (6, 2000, 700)])
 def test_topk_matches_oracle(n, v, k, dt):
     w = synth.make_recipe("ctx", n=n, v=v, dtype=dt, seed=n + v + k)
     _check(w.base, w.quant, w.token_ids, dt, k)
@@ -79,6 +80,27 @@ def test_topk_huge_tie_group_and_masks():
     assert list(g["idx"][0, :5]) == [0, 1, 2, 3, 4]
     assert list(g["idx"][1, :3]) == [1000, 1001, 1002]
     assert g["kl_topk"][3] == math.inf and np.all(g["idx"][4] == -1)
+
+
+@pytest.mark.parametrize("dt", [synth.F32, synth.BF16])
+def test_topk_tie_group_inside_the_boundary_bin(dt):
+    # a few hundred equal logits at the top of a wide row: the candidates
+    # hold the whole tie group and more, the bin holding the k-th largest is
+    # the tie group itself, and T is its lowest k indices
+    n, v = 8, 151936
+    w = synth.make_recipe("ctx", n=n, v=v, dtype=synth.F32, seed=31)
+    b, q = w.base.clone(), w.quant.clone()
+    gen = torch.Generator().manual_seed(4)
+    for i in range(n):
+        cnt = [130, 300, 600, 129][i % 4]
+        idx = torch.randperm(v, generator=gen)[:cnt]
+        b[i, idx] = float(b[i].max()) + 1.0
+    if dt == synth.BF16:
+        b, q = b.to(torch.bfloat16), q.to(torch.bfloat16)
+    g, _ = _check(b.contiguous(), q.contiguous(), w.token_ids, dt, 128)
+    for i in range(n):
+        top = np.sort(np.flatnonzero(b[i].float().numpy() == float(b[i].float().max())))[:128]
+        np.testing.assert_array_equal(g["idx"][i, :128], top)
 
 
 @pytest.mark.parametrize("split", [1, -1])
