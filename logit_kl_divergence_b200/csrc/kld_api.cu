@@ -301,10 +301,18 @@ kld_status_t kld_stats_run(kld_stats_t h, const void* base, const void* quant,
   h->timing_valid = h->timing;
   h->grad_timing_valid = false;
   if (h->timing) KLD_CUDA(cudaEventRecord(h->tev[0], s));
-  KLD_CUDA(launch_rows(h, base, quant, token_ids, N, V, dtype, h->rows, s));
+  // A split-row launch of few rows reduces its own records into the result
+  // buffer; otherwise the reduction kernel follows.
+  bool reduced = false;
+  KLD_CUDA(kld::launch_rows(base, quant, token_ids, N, V, dtype, h->rows, h->derr, h->sm_count,
+                            &h->split, nullptr, s, nullptr, 0, h->hres_dev, &reduced));
   if (h->timing) KLD_CUDA(cudaEventRecord(h->tev[1], s));
   h->last_rows = N;
-  return enqueue_reduce(h, h->rows, N, token_ids != nullptr, s);
+  if (!reduced) return enqueue_reduce(h, h->rows, N, token_ids != nullptr, s);
+  if (h->timing) KLD_CUDA(cudaEventRecord(h->tev[2], s));
+  KLD_CUDA(cudaEventRecord(h->done, s));
+  h->has_result = true;
+  return KLD_OK;
 }
 
 kld_status_t kld_stats_run_grad(kld_stats_t h, const void* base, const void* quant,

@@ -30,8 +30,10 @@ constexpr int kMaxClusterCtas = 8;
 
 // Per-launch global scratch of split-row mode: one merged partial per
 // cluster (kSplitPartBytes) and one arrival ticket per row; `parts` holds
-// `capacity` partials and `tickets` at least as many counters as rows. Tickets start at zero and are reset by
-// the last arriver.
+// `capacity` partials and `tickets` `capacity` counters (a launch of N rows
+// uses tickets[0, N), and tickets[N] counts finished rows when the launch
+// reduces its own records). Tickets start at zero and are reset by the last
+// arriver.
 constexpr int kSplitPartBytes = 64;
 struct SplitScratch {
   void* parts;
@@ -74,12 +76,17 @@ static_assert(sizeof(RowAux) == 48, "RowAux layout");
 // [col_offset, col_offset + V) of a wider vocabulary and each row's merged
 // 64-byte partial goes to part_out[r] instead of a record (see
 // launch_merge).
+// result_out (nullable): a split-row launch of at most kFusedReduceRows rows
+// then also reduces its records into *result_out (the launch's last
+// finaliser does it; no reduction kernel needed) and sets *reduced.
+constexpr int kFusedReduceRows = 32;
 cudaError_t launch_rows(const void* base, const void* quant,
                         const int32_t* token_ids, int64_t N, int64_t V,
                         kld_dtype_t dtype, kld_row_t* rows, uint32_t* derr,
                         int sm_count, const SplitScratch* split, RowAux* aux,
                         cudaStream_t stream, void* part_out = nullptr,
-                        int64_t col_offset = 0);
+                        int64_t col_offset = 0, kld_result_t* result_out = nullptr,
+                        bool* reduced = nullptr);
 
 // Records from the G vocabulary-slice partials of each row (parts: [G][N]
 // 64-byte partials, rank/slice order), tokens checked against V_total.

@@ -34,37 +34,23 @@
 #include <atomic>
 #include <climits>
 
+#include "kld_finish.cuh"
 #include "kld_internal.h"
 
 namespace kld {
 namespace {
 
-constexpr int kTargets = 7;
+using fin::interpolate;
+using fin::key_value;
+using fin::kExcluded;
+using fin::kTargets;
+using fin::order_key;
+using fin::warp_sort;
 constexpr int kAhead = 4;       // records each thread loads before using them
 constexpr int kDigitBits = 11;  // radix digit of the selection
 constexpr int kBins = 1 << kDigitBits;
 constexpr int kSmall = 32;      // a group this small is finished by one warp
 constexpr int kKeyCap = 19968;  // keys kept in shared memory (N up to this)
-constexpr uint32_t kExcluded = KLD_ROW_NONFINITE | KLD_ROW_EMPTY;
-
-__device__ __forceinline__ uint64_t order_key(double x) {
-  const uint64_t b = static_cast<uint64_t>(__double_as_longlong(x));
-  return (b >> 63) ? ~b : (b | 0x8000000000000000ull);
-}
-__device__ __forceinline__ double key_value(uint64_t k) {
-  const uint64_t b = (k >> 63) ? (k & 0x7fffffffffffffffull) : ~k;
-  return __longlong_as_double(static_cast<long long>(b));
-}
-
-// Type-7 interpolation between the two selected order statistics, with
-// explicitly rounded operations (no FMA contraction), so it rounds exactly as
-// the plain expression lo + frac * (hi - lo) evaluated step by step.
-__device__ double interpolate(double pos, double lo, double hi) {
-  const double k = floor(pos);
-  const double frac = __dsub_rn(pos, k);
-  if (frac == 0.0 || lo == hi) return lo;
-  return __dadd_rn(lo, __dmul_rn(frac, __dsub_rn(hi, lo)));
-}
 
 struct ReduceShared {
   double dsum[32][5];
@@ -85,21 +71,6 @@ struct ReduceShared {
 };
 constexpr size_t kReduceSmemMax = sizeof(ReduceShared) + sizeof(unsigned long long) * kKeyCap;
 static_assert(kReduceSmemMax <= 227 * 1024, "reduction shared memory");
-
-// Ascending bitonic sort of one 64-bit key per lane.
-__device__ __forceinline__ unsigned long long warp_sort(unsigned long long key, int lane) {
-#pragma unroll
-  for (int k = 2; k <= 32; k <<= 1) {
-#pragma unroll
-    for (int j = k >> 1; j > 0; j >>= 1) {
-      const unsigned long long other = __shfl_xor_sync(0xffffffffu, key, j);
-      const bool up = (lane & k) == 0;
-      const bool lower = (lane & j) == 0;
-      key = (lower == up) ? (key < other ? key : other) : (key > other ? key : other);
-    }
-  }
-  return key;
-}
 
 __global__ void __launch_bounds__(kReduceThreads, 1)
     kld_reduce_kernel(const kld_row_t* __restrict__ rows, int64_t N, int has_nll,
@@ -417,48 +388,23 @@ __global__ void __launch_bounds__(kReduceThreads, 1)
   }
 
   if (tid == 0) {
-    kld_result_t r;
-    const double nan = __longlong_as_double(0x7ff8000000000000ll);
-    r.n_rows = N;
-    r.n_valid = nv;
-    r.top1_agree = sh.isum[0][1];
-    r.has_nll = has_nll ? 1 : 0;
-    r.reserved0 = 0;
-    r.n_nll = sh.isum[0][2];
-    r.n_flagged = sh.isum[0][3];
-    r.flags_or = sh.flags_or[0];
-    r.device_error = 0u;
+    fin::Sums s;
+    s.kl = sh.dsum[0][0];
+    s.nll = sh.dsum[0][1];
+    s.nll_base = sh.dsum[0][2];
+    s.dp = sh.dsum[0][3];
+    s.dp2 = sh.dsum[0][4];
+    s.n_valid = nv;
+    s.agree = sh.isum[0][1];
+    s.n_nll = sh.isum[0][2];
+    s.n_flag = sh.isum[0][3];
+    s.flags_or = sh.flags_or[0];
+    uint32_t de = 0u;
     if (derr) {  // report and clear the row pass's error word
-      r.device_error = *derr;
+      de = *derr;
       *derr = 0u;
     }
-    if (nv > 0) {
-      const double dn = static_cast<double>(nv - 1);
-      r.mean_kld = sh.dsum[0][0] / static_cast<double>(nv);
-      r.median_kld = interpolate(0.5 * dn, key_value(sh.tval[0]), key_value(sh.tval[1]));
-      r.p90_kld = interpolate(0.9 * dn, key_value(sh.tval[2]), key_value(sh.tval[3]));
-      r.p99_kld = interpolate(0.99 * dn, key_value(sh.tval[4]), key_value(sh.tval[5]));
-      r.max_kld = key_value(sh.tval[6]);
-      r.top1_agree_pct = 100.0 * static_cast<double>(sh.isum[0][1]) / static_cast<double>(nv);
-    } else {
-      r.mean_kld = r.median_kld = r.p90_kld = r.p99_kld = r.max_kld = nan;
-      r.top1_agree_pct = nan;
-    }
-    if (has_nll && sh.isum[0][2] > 0) {
-      const double nn = static_cast<double>(sh.isum[0][2]);
-      r.mean_nll = sh.dsum[0][1] / nn;
-      r.ppl = exp(r.mean_nll);
-      r.mean_nll_base = sh.dsum[0][2] / nn;
-      r.ppl_base = exp(r.mean_nll_base);
-      r.ln_ppl_ratio = r.mean_nll - r.mean_nll_base;
-      r.mean_dp = sh.dsum[0][3] / nn;
-      r.rms_dp = sqrt(sh.dsum[0][4] / nn);
-    } else {
-      r.mean_nll = r.ppl = nan;
-      r.mean_nll_base = r.ppl_base = r.ln_ppl_ratio = nan;
-      r.mean_dp = r.rms_dp = nan;
-    }
-    *out = r;
+    *out = fin::make_result(N, s, sh.tval, has_nll, de);
   }
 }
 

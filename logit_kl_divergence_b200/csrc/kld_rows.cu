@@ -61,6 +61,7 @@
 #include <atomic>
 #include <climits>
 
+#include "kld_finish.cuh"
 #include "kld_internal.h"
 
 namespace kld {
@@ -681,12 +682,29 @@ __device__ __forceinline__ int64_t chunk_elem_offset(int chunk_id, int lane, int
          static_cast<int64_t>((i / E) * 32 + lane) * E + (i % E);
 }
 
+// Element i of a tile staged in shared memory.
+template <int DT>
+__device__ __forceinline__ float load_staged(const unsigned char* stage, int i) {
+  if constexpr (DT == KLD_F32) {
+    return reinterpret_cast<const float*>(stage)[i];
+  } else if constexpr (DT == KLD_BF16) {
+    return __uint_as_float(static_cast<uint32_t>(reinterpret_cast<const unsigned short*>(stage)[i]) << 16);
+  } else {
+    return __half2float(__ushort_as_half(reinterpret_cast<const unsigned short*>(stage)[i]));
+  }
+}
+
 // Lowest index holding `m` among the candidate lanes (mask) of one warp's
 // published partial (chunk ids counted from body element s0); lanes 0..15 of
-// the calling warp each test one element.
+// the calling warp each test one element. staged (nullable): the item's
+// tiles are still in the shared-memory ring (tile t in stage t; a split part
+// of at most kStages tiles), so the elements are read there instead of from
+// global memory; n = the item's element count.
 template <int DT>
 __device__ int rescan_candidates(const void* row, const RowGeom& g, int64_t s0, unsigned mask,
-                                 const int* locs, float m, int lane) {
+                                 const int* locs, float m, int lane,
+                                 const unsigned char* staged = nullptr, int64_t n = 0) {
+  constexpr int kStageElems = kStageBytes / Elem<DT>::kBytes;
   int best = INT_MAX;
   while (mask) {
     const int cl = __ffs(mask) - 1;
@@ -694,9 +712,15 @@ __device__ int rescan_candidates(const void* row, const RowGeom& g, int64_t s0, 
     const int loc = locs[cl];
     int idx = INT_MAX;
     if (lane < kLaneElems && loc >= 0) {
-      const int64_t off = s0 + chunk_elem_offset<DT>(loc, cl, lane);
-      if (off < g.body_len && Elem<DT>::load(row, g.head + off) == m)
-        idx = static_cast<int>(g.head + off);
+      const int64_t io = chunk_elem_offset<DT>(loc, cl, lane);  // within the item
+      const int64_t off = s0 + io;
+      if (off < g.body_len) {
+        const float x = staged != nullptr && io < n
+                            ? load_staged<DT>(staged + (io / kStageElems) * kStageBytes,
+                                              static_cast<int>(io % kStageElems))
+                            : Elem<DT>::load(row, g.head + off);
+        if (x == m) idx = static_cast<int>(g.head + off);
+      }
     }
     idx = __reduce_min_sync(0xffffffffu, idx);
     if (idx < best) best = idx;
@@ -938,13 +962,31 @@ __device__ __forceinline__ uint32_t map_to_rank(uint32_t local, uint32_t rank) {
   return r;
 }
 
+// Few split rows (red_out set): every row's finaliser counts its record on
+// the launch's counter; the warp that counts the last record reduces all N
+// records on the spot, so the statistic needs no second kernel. The counter
+// goes back to zero for the next launch.
+__device__ __forceinline__ void count_row(unsigned* counter, const kld_row_t* rows, int64_t N,
+                                          int has_nll, uint32_t* derr, kld_result_t* out,
+                                          int lane) {
+  unsigned t = 0u;
+  if (lane == 0)  // release: this warp's record; acquire: every other record
+    asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;" : "=r"(t) : "l"(counter) : "memory");
+  t = __shfl_sync(0xffffffffu, t, 0);
+  if (t != static_cast<unsigned>(N - 1)) return;
+  __syncwarp();  // lane 0's acquire orders the other lanes' loads
+  if (lane == 0) *counter = 0u;
+  fin::reduce_few_rows(rows, static_cast<int>(N), has_nll, derr, out, lane);
+}
+
 template <int DT>
 __global__ void __launch_bounds__(kRowThreads, 1)
     kld_rows_kernel(const void* __restrict__ base, const void* __restrict__ quant,
                     const int32_t* __restrict__ tok, int64_t N, int64_t V,
                     kld_row_t* __restrict__ rows, uint32_t* __restrict__ derr, int P,
                     MPart* __restrict__ gparts, unsigned* __restrict__ tickets, RowAux* __restrict__ aux,
-                    MPart* __restrict__ part_out, int64_t col0) {
+                    MPart* __restrict__ part_out, int64_t col0,
+                    kld_result_t* __restrict__ red_out) {
   constexpr int EB = Elem<DT>::kBytes;
   constexpr int E = Elem<DT>::kPerVec;
   constexpr int kStageElems = kStageBytes / EB;
@@ -1264,18 +1306,24 @@ __global__ void __launch_bounds__(kRowThreads, 1)
         amq = __reduce_min_sync(0xffffffffu, amq);
         unsigned wb = __ballot_sync(0xffffffffu, fin_b && lane < kConsumerWarps && mp.Mb == m.Mb);
         unsigned wq = __ballot_sync(0xffffffffu, fin_q && lane < kConsumerWarps && mp.Mq == m.Mq);
+        // A split part of at most kStages tiles (the CTA's only item) is
+        // still whole in the ring: rescan it there.
+        const int64_t n_item = it.s1 - it.s0;
+        const bool in_ring = P > 1 && n_item <= static_cast<int64_t>(kStages) * (kStageBytes / EB);
         while (wb) {
           const int w = __ffs(wb) - 1;
           wb &= wb - 1u;
           const unsigned cm = __shfl_sync(0xffffffffu, cand_b, w);
-          const int i = rescan_candidates<DT>(rb, g, it.s0, cm, sl.loc_b[w], m.Mb, lane);
+          const int i = rescan_candidates<DT>(rb, g, it.s0, cm, sl.loc_b[w], m.Mb, lane,
+                                              in_ring ? stage_b : nullptr, n_item);
           if (i < amb) amb = i;
         }
         while (wq) {
           const int w = __ffs(wq) - 1;
           wq &= wq - 1u;
           const unsigned cm = __shfl_sync(0xffffffffu, cand_q, w);
-          const int i = rescan_candidates<DT>(rq, g, it.s0, cm, sl.loc_q[w], m.Mq, lane);
+          const int i = rescan_candidates<DT>(rq, g, it.s0, cm, sl.loc_q[w], m.Mq, lane,
+                                              in_ring ? stage_q : nullptr, n_item);
           if (i < amq) amq = i;
         }
         m.amax_b = amb;
@@ -1389,6 +1437,7 @@ __global__ void __launch_bounds__(kRowThreads, 1)
           rows[r] = rec;
           if (aux != nullptr) aux[r] = row_aux(cm, rec);
         }
+        if (red_out != nullptr) count_row(tickets + N, rows, N, tok != nullptr, derr, red_out, lane);
         continue;
       }
       const int cid = it.k / static_cast<int>(G);
@@ -1428,6 +1477,7 @@ __global__ void __launch_bounds__(kRowThreads, 1)
         if (aux != nullptr) aux[r] = row_aux(fm, rec);
         tickets[r] = 0u;  // ready for the next launch
       }
+      if (red_out != nullptr) count_row(tickets + N, rows, N, tok != nullptr, derr, red_out, lane);
     }
   }
 
@@ -1535,7 +1585,7 @@ template <int DT>
 cudaError_t launch_typed(const void* base, const void* quant, const int32_t* tok, int64_t N,
                          int64_t V, kld_row_t* rows, uint32_t* derr, const RowPlan& pl,
                          const SplitScratch* split, RowAux* aux, MPart* part_out, int64_t col0,
-                         cudaStream_t stream) {
+                         kld_result_t* red_out, cudaStream_t stream) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(pl.grid));
   cfg.blockDim = dim3(kRowThreads);
@@ -1551,7 +1601,7 @@ cudaError_t launch_typed(const void* base, const void* quant, const int32_t* tok
   MPart* gp = split ? static_cast<MPart*>(split->parts) : nullptr;
   unsigned* tk = split ? split->tickets : nullptr;
   return cudaLaunchKernelEx(&cfg, kld_rows_kernel<DT>, base, quant, tok, N, V, rows, derr,
-                            pl.parts_per_row, gp, tk, aux, part_out, col0);
+                            pl.parts_per_row, gp, tk, aux, part_out, col0, red_out);
 }
 
 }  // namespace
@@ -1625,7 +1675,9 @@ cudaError_t launch_merge(const void* parts, int G, int64_t N, const int32_t* tok
 cudaError_t launch_rows(const void* base, const void* quant, const int32_t* token_ids, int64_t N,
                         int64_t V, kld_dtype_t dtype, kld_row_t* rows, uint32_t* derr,
                         int sm_count, const SplitScratch* split, RowAux* aux,
-                        cudaStream_t stream, void* part_out, int64_t col_offset) {
+                        cudaStream_t stream, void* part_out, int64_t col_offset,
+                        kld_result_t* result_out, bool* reduced) {
+  if (reduced) *reduced = false;
   RowPlan pl = plan_rows(N, sm_count, nullptr, 0);
   // Vocabulary-slice partials come from whole-row launches only.
   if (split != nullptr && part_out == nullptr && N * 2 <= sm_count && split->max_cluster_ctas >= 1) {
@@ -1636,18 +1688,28 @@ cudaError_t launch_rows(const void* base, const void* quant, const int32_t* toke
     if (static_cast<int64_t>(pl.grid) / pl.cluster_ctas > split->capacity || N > split->capacity)
       pl = plan_rows(N, sm_count, nullptr, 0);
   }
+  // Few split rows: the row pass reduces its own records (the launch counter
+  // is the ticket after the last row's).
+  const bool fuse = result_out != nullptr && pl.parts_per_row > 1 && N <= kFusedReduceRows &&
+                    split != nullptr && N + 1 <= split->capacity;
+  kld_result_t* red = fuse ? result_out : nullptr;
+  cudaError_t e = cudaErrorInvalidValue;
   switch (dtype) {
     case KLD_F32:
-      return launch_typed<KLD_F32>(base, quant, token_ids, N, V, rows, derr, pl, split, aux,
-                                 static_cast<MPart*>(part_out), col_offset, stream);
+      e = launch_typed<KLD_F32>(base, quant, token_ids, N, V, rows, derr, pl, split, aux,
+                                static_cast<MPart*>(part_out), col_offset, red, stream);
+      break;
     case KLD_BF16:
-      return launch_typed<KLD_BF16>(base, quant, token_ids, N, V, rows, derr, pl, split, aux,
-                                 static_cast<MPart*>(part_out), col_offset, stream);
+      e = launch_typed<KLD_BF16>(base, quant, token_ids, N, V, rows, derr, pl, split, aux,
+                                 static_cast<MPart*>(part_out), col_offset, red, stream);
+      break;
     case KLD_F16:
-      return launch_typed<KLD_F16>(base, quant, token_ids, N, V, rows, derr, pl, split, aux,
-                                 static_cast<MPart*>(part_out), col_offset, stream);
+      e = launch_typed<KLD_F16>(base, quant, token_ids, N, V, rows, derr, pl, split, aux,
+                                static_cast<MPart*>(part_out), col_offset, red, stream);
+      break;
   }
-  return cudaErrorInvalidValue;
+  if (e == cudaSuccess && reduced) *reduced = fuse;
+  return e;
 }
 
 cudaError_t launch_wait_selftest(uint64_t limit_ns, int use_abort, uint32_t* derr,

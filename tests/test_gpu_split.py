@@ -12,6 +12,7 @@ come back to zero after every launch.
 """
 import ctypes
 import math
+import struct
 
 import numpy as np
 import pytest
@@ -124,6 +125,48 @@ def test_split_rows_repeat_launches_on_one_handle():
             gres = st.result()
             _, ores = oracle.run(w.base, w.quant, w.token_ids, ODT[dt])
             assert_stats_match(dict(gres), ores)
+    finally:
+        st.close()
+
+
+def _same_bits(a, b):
+    if isinstance(a, float) or isinstance(b, float):
+        if math.isnan(a) and math.isnan(b):
+            return True
+        return struct.pack("<d", a) == struct.pack("<d", b)
+    return a == b
+
+
+@pytest.mark.parametrize("split", [1, 2, 8])
+@pytest.mark.parametrize("n", [1, 2, 5, 16, 31, 32, 33])
+def test_few_split_rows_reduce_in_the_row_pass_like_the_reduction_kernel(n, split):
+    # A split launch of at most 32 rows reduces its own records (the warp
+    # that finalises the last row does it): its result must equal the
+    # reduction kernel's on the same records bit for bit, with excluded
+    # rows, a bad token and no tokens at all, over repeated launches on one
+    # handle (the launch counter must come back to zero). 33 rows take the
+    # reduction kernel both ways.
+    v = 70001
+    w = synth.make_recipe("ctx", n=n, v=v, dtype=synth.F32, seed=100 + n)
+    b, q, t = w.base.clone(), w.quant.clone(), w.token_ids.clone()
+    if n >= 5:
+        b[1, 17] = math.nan   # excluded row
+        t[3] = v + 5          # token outside the vocabulary
+    bd, qd, td = b.to(DEV), q.to(DEV), t.to(DEV)
+    st = KLDStats(max_rows=n, device=DEV)
+    try:
+        st.set_split(split)
+        for tok in (td, None, td):
+            st.run(bd, qd, tok)
+            fused = st.result()
+            st.run_rows(bd, qd, tok)
+            st.reduce(None, n, tok is not None)
+            ref = st.result()
+            assert fused.keys() == ref.keys()
+            for k in fused:
+                assert _same_bits(fused[k], ref[k]), (k, fused[k], ref[k])
+            _, ores = oracle.run(b, q, None if tok is None else t, oracle.F32)
+            assert_stats_match(fused, ores)
     finally:
         st.close()
 
