@@ -110,6 +110,9 @@ class ClockSampler:
             pynvml.nvmlInit()
             self._nv = pynvml
             self._h = pynvml.nvmlDeviceGetHandleByIndex(gpu_index)
+            # queried once: this call takes milliseconds, the per-sample
+            # clock and reason queries about a microsecond
+            self._max = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
             self._thread = threading.Thread(target=self._poll, daemon=True)
             self._thread.start()
         except Exception:
@@ -126,7 +129,7 @@ class ClockSampler:
         while not self._stop.is_set():
             try:
                 sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
-                mx = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+                mx = self._max
                 bits = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
                 names = {name for name, bit in self.REASONS.items() if bits & bit}
                 self.samples.append((time.perf_counter(), sm, mx, names))
