@@ -416,14 +416,16 @@ def main():
     if world > 1:
         records = torch.empty((N, ROW_RECORD_BYTES), dtype=torch.uint8, device=dev)
 
-    row_ms = []
+    row_ms, red_ms = [], []
 
     def step(timed: bool):
         if world == 1:
             st.run(w.base, w.quant, w.token_ids)
             res = st.result()
             if timed:
-                row_ms.append(st.timing()[0])
+                rp_ms, rd_ms = st.timing()
+                row_ms.append(rp_ms)
+                red_ms.append(rd_ms)
         else:
             st.run_rows(w.base, w.quant, w.token_ids, out=records)
             gathered = gather_records(records, counts=[N] * world)
@@ -481,6 +483,7 @@ def main():
                 "peak_source": f"{peak_kind} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)",
                 "frac_of_8TBs_nominal": achieved / 8000.0,
                 "kernel": "kld_rows_kernel<f32>", "row_pass_ms": avg_row_ms,
+                "reduce_ms": (sum(red_ms) / len(red_ms)) if red_ms else None,
                 "algorithmic_bytes_per_launch": in_bytes}
 
     # bf16 variant of the same context (the target names both dtypes).

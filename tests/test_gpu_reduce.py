@@ -106,6 +106,20 @@ def test_tiny_negatives_zeros_and_infinities():
     check(make_records(v, rng))
 
 
+@pytest.mark.parametrize("n", [8192, 30000])
+def test_outliers_at_both_ends_of_a_narrow_cluster(n):
+    # the selection starts from the range of the keys present: a range made
+    # huge by outliers (the largest finite double, +inf, the smallest
+    # subnormal, tiny negatives) around a cluster narrower than one first digit
+    rng = np.random.default_rng(n)
+    v = 0.02 + 1e-9 * rng.random(n)
+    v[rng.integers(0, n, 3)] = 1.7976931348623157e308
+    v[rng.integers(0, n, 2)] = np.inf
+    v[rng.integers(0, n, 3)] = 5e-324
+    v[rng.integers(0, n, 3)] = -1e-300
+    check(make_records(v, rng))
+
+
 def test_excluded_rows_and_bad_tokens():
     rng = np.random.default_rng(5)
     n = 20000
