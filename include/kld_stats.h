@@ -152,9 +152,13 @@ void kld_stats_destroy(kld_stats_t h);
 
 /*
  * The whole statistic for rows [0, N): the fused row pass, then the
- * fixed-order reduction and exact percentile selection, then an async copy
- * of the result to pinned host memory. token_ids (device, int32[N]) may be
- * NULL: no NLL/PPL. 1 <= N <= max_rows, 1 <= V <= 2^31-1. Asynchronous.
+ * fixed-order reduction and exact percentile selection, which writes the
+ * result straight into the handle's pinned host buffer (read it with
+ * kld_stats_result). When the row pass splits few rows (N <= 32) over
+ * many CTAs, the CTA that finishes the last row performs the reduction
+ * itself, in the same arithmetic order, and no reduction kernel follows.
+ * token_ids (device, int32[N]) may be NULL: no NLL/PPL.
+ * 1 <= N <= max_rows, 1 <= V <= 2^31-1. Asynchronous.
  */
 kld_status_t kld_stats_run(kld_stats_t h, const void* base, const void* quant,
                            const int32_t* token_ids, int64_t N, int64_t V,
@@ -315,7 +319,10 @@ kld_status_t kld_stats_grad_timing(kld_stats_t h, float* grad_ms);
 /*
  * Kernel timing of the next runs: when enabled, kld_stats_run records CUDA
  * events around its row pass and its reduction; kld_stats_timing() returns
- * the last run's durations in milliseconds (waits for that run).
+ * the last run's durations in milliseconds (waits for that run). For a run
+ * whose row pass reduced its own records (few split rows, see
+ * kld_stats_run) the row-pass time includes the reduction and reduce_ms is
+ * about zero.
  */
 kld_status_t kld_stats_set_timing(kld_stats_t h, int enable);
 kld_status_t kld_stats_timing(kld_stats_t h, float* row_pass_ms,
