@@ -169,6 +169,9 @@ __device__ __forceinline__ Sums zero_sums() {
 // SMs); the device error word is read and cleared; the result goes to *out.
 __device__ __forceinline__ void reduce_few_rows(const kld_row_t* rows, int N, int has_nll,
                                                 uint32_t* derr, kld_result_t* out, int lane) {
+  // The error word is taken first: its round trip overlaps the record loads
+  // (every row's record is written, so no part of the pass can still set it).
+  const uint32_t de = (lane == 0 && derr) ? atomicExch(derr, 0u) : 0u;
   Sums s = zero_sums();
   unsigned long long key = ~0ull;  // lanes past N sort last
   if (lane < N) {
@@ -207,10 +210,7 @@ __device__ __forceinline__ void reduce_few_rows(const kld_row_t* rows, int N, in
     const int src = nv > 0 ? static_cast<int>(target_rank(q, nv) + (N - nv)) : 0;
     tval[q] = __shfl_sync(0xffffffffu, key, src);
   }
-  if (lane == 0) {
-    const uint32_t de = derr ? atomicExch(derr, 0u) : 0u;
-    *out = make_result(N, t, tval, has_nll, de);
-  }
+  if (lane == 0) *out = make_result(N, t, tval, has_nll, de);
 }
 
 }  // namespace fin
