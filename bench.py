@@ -377,6 +377,9 @@ def main():
                     help="profiling only: fewer rows of the same recipe (not a bench line)")
     ap.add_argument("--dtype", choices=["f32", "bf16"], default="f32",
                     help="profiling only: logit dtype of the workload")
+    ap.add_argument("--sharded", action="store_true",
+                    help="take the row-sharded path (NCCL group, record all-gather) even on "
+                         "one GPU: the multi-GPU step with a group of one rank")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
 
@@ -396,9 +399,18 @@ def main():
 
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    if world > 1:
+    sharded = world > 1 or args.sharded
+    if sharded:
         import datetime
 
+        if "MASTER_ADDR" not in os.environ:  # one rank, launched without torchrun
+            import socket
+
+            with socket.socket() as sk:
+                sk.bind(("127.0.0.1", 0))
+                port = sk.getsockname()[1]
+            os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK="0",
+                              WORLD_SIZE="1", LOCAL_RANK=str(local))
         dist.init_process_group("nccl", device_id=dev, timeout=datetime.timedelta(seconds=120))
 
     name = WORKLOAD
@@ -411,15 +423,15 @@ def main():
     stream = torch.cuda.current_stream(dev)
 
     st = KLDStats(max_rows=N * world, device=dev)
-    st.set_timing(world == 1)
+    st.set_timing(not sharded)
     records = None
-    if world > 1:
+    if sharded:
         records = torch.empty((N, ROW_RECORD_BYTES), dtype=torch.uint8, device=dev)
 
     row_ms, red_ms = [], []
 
     def step(timed: bool):
-        if world == 1:
+        if not sharded:
             st.run(w.base, w.quant, w.token_ids)
             res = st.result()
             if timed:
@@ -439,17 +451,17 @@ def main():
 
     # Row-kernel time on its own stream for multi-GPU too (events bracket the
     # row pass only; used for the roofline).
-    if world > 1:
+    if sharded:
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
 
-    if world > 1:
+    if sharded:
         dist.barrier()
     torch.cuda.synchronize(dev)
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     sampler.mark_start()
     start.record(stream)
     for _ in range(args.steps):
-        if world == 1:
+        if not sharded:
             res = step(True)
         else:
             e0.record(stream)
@@ -462,11 +474,11 @@ def main():
     end.record(stream)
     torch.cuda.synchronize(dev)
     sampler.mark_end()
-    if world > 1:
+    if sharded:
         dist.barrier()
     clocks = sampler.stop()
     ms = start.elapsed_time(end)
-    if world > 1:
+    if sharded:
         t = torch.tensor([ms], dtype=torch.float64, device=dev)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         ms = float(t.item())
@@ -488,7 +500,7 @@ def main():
 
     # bf16 variant of the same context (the target names both dtypes).
     variants = {}
-    if world == 1 and not args.no_variants:
+    if not sharded and not args.no_variants:
         del w
         torch.cuda.empty_cache()
         wb = synth.make(VARIANT, device=dev)
@@ -520,7 +532,7 @@ def main():
     # Gradient of the KL w.r.t. the quant logits (row pass + reduction +
     # gradient pass writing fp32 [N, V]) on the same context.
     grad = None
-    if world == 1 and not args.no_grad:
+    if not sharded and not args.no_grad:
         gout = torch.empty_like(w.base)
         st.set_timing(True)
         for _ in range(3):
@@ -552,7 +564,7 @@ def main():
     # Top-128 compression of the base rows + KL against it (row pass +
     # reduction + top-k pass) on the same context.
     topk = None
-    if world == 1 and not args.no_topk:
+    if not sharded and not args.no_topk:
         for _ in range(2):
             st.run_topk(w.base, w.quant, w.token_ids, k=128)
             st.result()
@@ -564,8 +576,7 @@ def main():
         for _ in range(tsteps):
             out = st.run_topk(w.base, w.quant, w.token_ids, k=128)
             st.result()
-            if world == 1:
-                kms.append(st.grad_timing())
+            kms.append(st.grad_timing())
         b.record(stream)
         torch.cuda.synchronize(dev)
         tms = a.elapsed_time(b) / tsteps
@@ -581,7 +592,7 @@ def main():
     # End to end through the public host-memory entry point: pinned host
     # buffers in, the result struct out, copies inside the timed region.
     e2e = None
-    if world == 1 and args.e2e_steps > 0:
+    if not sharded and args.e2e_steps > 0:
         hb = w.base.cpu().pin_memory()
         hq = w.quant.cpu().pin_memory()
         ht = w.token_ids.cpu().pin_memory()
@@ -602,7 +613,7 @@ def main():
         del hb, hq, ht
 
     split_row = None
-    if world == 1 and not args.no_split_row and args.rows is None:
+    if not sharded and not args.no_split_row and args.rows is None:
         del w
         torch.cuda.empty_cache()
         split_row = split_row_latency(dev, stream, max(1, args.split_calls))
@@ -618,7 +629,8 @@ def main():
             "scaling": "weak", "vs_baseline": None, "dtype": args.dtype, "data": "synthetic",
             "config": {"workload": name, "rows_per_gpu": N, "vocab": V, "logit_dtype": args.dtype,
                        "global_rows": total_rows,
-                       "parallelism": f"rows sharded over {world} GPU(s), records all-gathered",
+                       "parallelism": (f"rows sharded over {world} GPU(s) (NCCL group), records all-gathered"
+                                       if sharded else "one GPU, whole statistic per step (kld_stats_run)"),
                        "l2": "inputs (9.96 GB per step per GPU) exceed the 126 MB L2; no flush"},
             "roofline": roofline, "cpu_baseline": cpu, "cpu_baseline_all_cores": cpu_mt, "e2e": e2e,
             "gpu_launches": 2 * args.steps, "clocks": clocks,
@@ -634,7 +646,7 @@ def main():
         print(json.dumps(line), flush=True)
 
     st.close()
-    if world > 1:
+    if sharded:
         dist.destroy_process_group()
 
 
