@@ -204,3 +204,27 @@ def test_set_split_rejects_unknown_shapes():
             st.set_split(ok)
     finally:
         st.close()
+
+
+def test_few_split_rows_time_no_separate_reduction():
+    # the row pass of a few-row split launch includes the reduction: the
+    # reduction's events sit back to back; whole-row launches still run the
+    # reduction kernel after the row pass
+    w = synth.make_recipe("ctx", n=4, v=V_FULL, dtype=synth.F32, seed=41)
+    b, q, t = w.base.to(DEV), w.quant.to(DEV), w.token_ids.to(DEV)
+    st = KLDStats(max_rows=4, device=DEV)
+    try:
+        st.set_timing(True)
+        st.run(b, q, t)
+        fused = st.result()
+        row_ms, red_ms = st.timing()
+        assert row_ms > 0.0 and 0.0 <= red_ms < 0.01, (row_ms, red_ms)
+        st.set_split(-1)
+        st.run(b, q, t)
+        whole = st.result()
+        row2_ms, red2_ms = st.timing()
+        assert row2_ms > 0.0 and red2_ms > 0.0
+        assert fused["top1_agree"] == whole["top1_agree"]
+        assert math.isclose(fused["mean_kld"], whole["mean_kld"], rel_tol=1e-5, abs_tol=1e-9)
+    finally:
+        st.close()

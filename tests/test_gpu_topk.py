@@ -119,3 +119,18 @@ def test_topk_never_exceeds_the_full_kl():
     from logit_kl_divergence_b200 import rows_view
     full = rows_view(kld)["kld"].cpu().numpy()
     assert np.all(out["kl_topk"].cpu().numpy() <= full + 1e-6 + 1e-4 * full)
+
+
+def test_topk_pass_is_timed():
+    # with timing on, the top-k pass is bracketed by its own events
+    w = synth.make_recipe("ctx", n=64, v=32000, dtype=synth.F32, seed=12)
+    st = KLDStats(max_rows=64, device=DEV)
+    try:
+        st.set_timing(True)
+        st.run_topk(w.base.to(DEV), w.quant.to(DEV), w.token_ids.to(DEV), k=128)
+        st.result()
+        row_ms, red_ms = st.timing()
+        topk_ms = st.grad_timing()
+        assert 0.0 < row_ms < 100.0 and 0.0 < red_ms < 100.0 and 0.0 < topk_ms < 100.0
+    finally:
+        st.close()
