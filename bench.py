@@ -498,35 +498,49 @@ def main():
                 "reduce_ms": (sum(red_ms) / len(red_ms)) if red_ms else None,
                 "algorithmic_bytes_per_launch": in_bytes}
 
-    # bf16 variant of the same context (the target names both dtypes).
-    variants = {}
-    if not sharded and not args.no_variants:
-        del w
-        torch.cuda.empty_cache()
-        wb = synth.make(VARIANT, device=dev)
+    # Other workloads of the same statistic, each through its own handle: the
+    # bf16 variant of the same context (the target names both dtypes), four
+    # 8192-token contexts in bf16, and the edge-case rows (near-one-hot, exact
+    # ties, -inf padding, constant shifts). Row pass timed by the library's
+    # events, step = kld_stats_run + kld_stats_result.
+    def time_variant(wname):
+        wv = synth.make(wname, device=dev)
+        sv = KLDStats(max_rows=wv.n, device=dev)
+        sv.set_timing(True)
         for _ in range(3):
-            st.run(wb.base, wb.quant, wb.token_ids)
-            st.result()
+            sv.run(wv.base, wv.quant, wv.token_ids)
+            sv.result()
         torch.cuda.synchronize(dev)
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         rms = []
         a.record(stream)
         for _ in range(args.steps):
-            st.run(wb.base, wb.quant, wb.token_ids)
-            st.result()
-            rms.append(st.timing()[0])
+            sv.run(wv.base, wv.quant, wv.token_ids)
+            rv = sv.result()
+            rms.append(sv.timing()[0])
         b.record(stream)
         torch.cuda.synchronize(dev)
-        vb_bytes = 2 * wb.base.numel() * wb.bytes_per_elem
+        vbytes = 2 * wv.base.numel() * wv.bytes_per_elem
         vms = a.elapsed_time(b) / args.steps
         rrow = sum(rms) / len(rms)
-        variants[VARIANT] = {"value": wb.n / (vms / 1000.0), "unit": "rows/s", "ms_per_step": vms,
-                             "row_pass_ms": rrow, "achieved_gbs": vb_bytes / (rrow / 1000.0) / 1e9,
-                             "frac": vb_bytes / (rrow / 1000.0) / 1e9 / peak,
-                             "traffic": recorded_traffic(VARIANT),
-                             "algorithmic_bytes_per_launch": vb_bytes}
-        del wb
+        out = {"rows": wv.n, "vocab": wv.base.shape[1], "logit_dtype": "f32" if wv.bytes_per_elem == 4 else "bf16",
+               "value": wv.n / (vms / 1000.0), "unit": "rows/s", "ms_per_step": vms,
+               "row_pass_ms": rrow, "achieved_gbs": vbytes / (rrow / 1000.0) / 1e9,
+               "frac": vbytes / (rrow / 1000.0) / 1e9 / peak,
+               "traffic": recorded_traffic(wname), "algorithmic_bytes_per_launch": vbytes,
+               "stats": {k: rv[k] for k in ("mean_kld", "median_kld", "p90_kld", "p99_kld", "max_kld",
+                                            "top1_agree_pct", "ppl", "n_flagged")}}
+        sv.close()
+        del wv
         torch.cuda.empty_cache()
+        return out
+
+    variants = {}
+    if not sharded and not args.no_variants:
+        del w
+        torch.cuda.empty_cache()
+        for vname in (VARIANT, "ctx4x8192_v151936_bf16", "edge_16384x131072_f32"):
+            variants[vname] = time_variant(vname)
         w = synth.make(name, device=dev, seed=synth.WORKLOADS[name][4])
 
     # Gradient of the KL w.r.t. the quant logits (row pass + reduction +
