@@ -486,6 +486,23 @@ def main():
     total_rows = N * world
     value = total_rows / (ms_per_step / 1000.0)
 
+    # Read-only roofline of the row pass on this device, for context beside the
+    # copy-bandwidth peak: the library's probe streams the same two inputs
+    # into shared memory with the row pass's bulk copies and computes nothing.
+    read_probe_gbs = None
+    if not sharded:
+        for _ in range(3):
+            st.read_probe(w.base, w.quant)
+        torch.cuda.synchronize(dev)
+        pa, pb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        preps = 10
+        pa.record(stream)
+        for _ in range(preps):
+            st.read_probe(w.base, w.quant)
+        pb.record(stream)
+        torch.cuda.synchronize(dev)
+        read_probe_gbs = in_bytes / (pa.elapsed_time(pb) / preps / 1000.0) / 1e9
+
     peak, peak_kind = measured_peak()
     avg_row_ms = sum(row_ms) / len(row_ms)
     achieved = in_bytes / (avg_row_ms / 1000.0) / 1e9
@@ -494,6 +511,8 @@ def main():
                 "frac": achieved / peak, "traffic": traffic,
                 "peak_source": f"{peak_kind} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)",
                 "frac_of_8TBs_nominal": achieved / 8000.0,
+                "read_probe_gbs": read_probe_gbs,
+                "frac_of_read_probe": (achieved / read_probe_gbs) if read_probe_gbs else None,
                 "kernel": "kld_rows_kernel<f32>", "row_pass_ms": avg_row_ms,
                 "reduce_ms": (sum(red_ms) / len(red_ms)) if red_ms else None,
                 "algorithmic_bytes_per_launch": in_bytes}

@@ -317,6 +317,21 @@ kld_status_t kld_selftest_bounded_wait(int device, uint64_t limit_ns, int use_ab
 kld_status_t kld_stats_grad_timing(kld_stats_t h, float* grad_ms);
 
 /*
+ * Read-bandwidth probe, a measuring aid with no counterpart in the
+ * statistic: streams `bytes` of each of the device buffers a and b from HBM
+ * into shared memory with the row pass's bulk copies (32 KB tiles, one CTA
+ * per SM, nothing computed), so that the time the caller measures around it
+ * (CUDA events on `stream`) gives the read-only bandwidth the row pass can
+ * reach on this device. a and b: 16-byte aligned; bytes: a positive
+ * multiple of 16; otherwise KLD_ERR_INVALID_ARG and nothing is enqueued.
+ * Asynchronous on `stream`. A bounded wait that gives up sets the handle's
+ * device error word, which the next kld_stats_result reports
+ * (KLD_ERR_TIMEOUT).
+ */
+kld_status_t kld_stats_read_probe(kld_stats_t h, const void* a, const void* b, int64_t bytes,
+                                  void* stream);
+
+/*
  * Kernel timing of the next runs: when enabled, kld_stats_run records CUDA
  * events around its row pass and its reduction; kld_stats_timing() returns
  * the last run's durations in milliseconds (waits for that run). For a run

@@ -165,6 +165,19 @@ class KLDStats:
         _lib.check(self._lib.kld_stats_grad_timing(self._h, ctypes.byref(ms)), "kld_stats_grad_timing")
         return ms.value
 
+    def read_probe(self, a: torch.Tensor, b: torch.Tensor, stream=None) -> None:
+        """Read-bandwidth probe: stream both (contiguous, same-size) device
+        tensors from HBM into shared memory as the row pass does, computing
+        nothing; time it with CUDA events on the stream."""
+        if not (a.is_cuda and b.is_cuda and a.is_contiguous() and b.is_contiguous()):
+            raise ValueError("a and b must be contiguous CUDA tensors")
+        nbytes = a.numel() * a.element_size()
+        if b.numel() * b.element_size() != nbytes:
+            raise ValueError("a and b must have the same size in bytes")
+        st = self._lib.kld_stats_read_probe(self._h, _ptr(a), _ptr(b), nbytes,
+                                            ctypes.c_void_p(_stream_ptr(stream, a.device)))
+        _lib.check(st, "kld_stats_read_probe")
+
     def run_partials(self, base: torch.Tensor, quant: torch.Tensor, token_ids: torch.Tensor | None,
                      col_offset: int, v_total: int, out: torch.Tensor | None = None,
                      stream=None) -> torch.Tensor:

@@ -58,6 +58,12 @@ constexpr size_t kStageTargetBytes = 128ull << 20;  // per operand per buffer
 
 }  // namespace
 
+namespace kld {
+// Read-bandwidth probe (kld_probe.cu; see kld_stats_read_probe).
+cudaError_t launch_read_probe(const void* a, const void* b, int64_t bytes, uint32_t* derr,
+                              int sm_count, cudaStream_t stream);
+}  // namespace kld
+
 struct kld_stats_s {
   int device = 0;
   int sm_count = 0;
@@ -427,6 +433,18 @@ kld_status_t kld_selftest_bounded_wait(int device, uint64_t limit_ns, int use_ab
   if (st != KLD_OK) return st;
   if (waited_ns) *waited_ns = w;
   return err_word ? KLD_ERR_TIMEOUT : KLD_OK;
+}
+
+kld_status_t kld_stats_read_probe(kld_stats_t h, const void* a, const void* b, int64_t bytes,
+                                  void* stream) {
+  if (!h || !a || !b || bytes <= 0 || (bytes & 15)) return KLD_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(a) | reinterpret_cast<uintptr_t>(b)) & 15u)
+    return KLD_ERR_INVALID_ARG;
+  DeviceGuard guard(h->device);
+  if (!guard.ok()) return cuda_fail(cudaGetLastError(), "cudaSetDevice");
+  KLD_CUDA(kld::launch_read_probe(a, b, bytes, h->derr, h->sm_count,
+                                  static_cast<cudaStream_t>(stream)));
+  return KLD_OK;
 }
 
 kld_status_t kld_stats_grad_timing(kld_stats_t h, float* grad_ms) {

@@ -92,6 +92,7 @@ def test_arguments_rejected_before_any_gpu_work(lib):
     assert lib.kld_stats_reduce(None, None, 1, 0, None) == _lib.KLD_ERR_INVALID_ARG
     assert lib.kld_stats_run_host(None, p, p, None, 1, 1, 0, None) == _lib.KLD_ERR_INVALID_ARG
     assert lib.kld_stats_set_timing(None, 1) == _lib.KLD_ERR_INVALID_ARG
+    assert lib.kld_stats_read_probe(None, p, p, 1 << 20, None) == _lib.KLD_ERR_INVALID_ARG
     w = ctypes.c_uint64()
     assert lib.kld_selftest_bounded_wait(-1, 10**6, 0, ctypes.byref(w)) == _lib.KLD_ERR_INVALID_ARG
     assert lib.kld_selftest_bounded_wait(0, 999, 0, ctypes.byref(w)) == _lib.KLD_ERR_INVALID_ARG
