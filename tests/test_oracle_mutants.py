@@ -56,6 +56,21 @@ MUTANTS = {
                                   "      p_rest += std::exp(q[j] - lse_q);"),
     "ppl_ratio_inverted": ("out->ln_ppl_ratio = out->mean_nll - out->mean_nll_base;",
                            "out->ln_ppl_ratio = out->mean_nll_base - out->mean_nll;"),
+    "kl_in_bits": ("kl += std::exp(logp) * (logp - logr);",
+                   "kl += std::exp(logp) * (logp - logr) / std::log(2.0);"),
+    "lse_without_the_maximum": ("const double lse_b = m_b + std::log(s_b);",
+                                "const double lse_b = std::log(s_b);"),
+    "mean_kld_over_all_rows": ("out->mean_kld = sum_kl / (double)n;",
+                               "out->mean_kld = sum_kl / (double)N;"),
+    "agreement_pct_over_all_rows": ("out->top1_agree_pct = 100.0 * (double)agree / (double)n;",
+                                    "out->top1_agree_pct = 100.0 * (double)agree / (double)N;"),
+    "ppl_in_base_two": ("out->ppl = std::exp(out->mean_nll);",
+                        "out->ppl = std::exp2(out->mean_nll);"),
+    "percentile_takes_the_upper_neighbour": ("return lo + frac * (hi - lo);", "return hi;"),
+    "topk_ties_to_highest_index": ("for (int64_t j = 0; j < V; ++j) order[(size_t)j] = j;",
+                                   "for (int64_t j = 0; j < V; ++j) order[(size_t)j] = V - 1 - j;"),
+    "grad_scale_dropped": ("g[j] = scale * (std::exp(q[j] - lse_q) - std::exp(b[j] - lse_b));",
+                           "g[j] = (std::exp(q[j] - lse_q) - std::exp(b[j] - lse_b));"),
 }
 
 

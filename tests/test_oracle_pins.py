@@ -419,6 +419,31 @@ def test_nonfinite_and_empty_rows_are_flagged_and_excluded():
     assert abs(res["mean_kld"] - (r["kld"][0] + r["kld"][5]) / 2) < 1e-15
 
 
+def test_statistics_are_over_the_valid_rows_only():
+    # excluded rows (NaN, all -inf) count in n_rows but in none of the
+    # means, percentages or order statistics: each is the same statistic of
+    # the valid rows alone
+    V = 64
+    b = RNG.normal(0, 2, size=(10, V)).astype(np.float32)
+    q = (b + RNG.normal(0, 0.7, size=b.shape)).astype(np.float32)
+    b[2, 7] = np.nan
+    q[6, :] = -np.inf
+    r, res = _run(b, q)
+    keep = [i for i in range(10) if i not in (2, 6)]
+    valid = np.array([r["kld"][i] for i in keep])
+    assert res["n_rows"] == 10 and res["n_valid"] == 8
+    assert abs(res["mean_kld"] - math.fsum(valid) / 8) <= 1e-14 * res["mean_kld"]
+    agree = sum(int(r["amax_b"][i] == r["amax_q"][i]) for i in keep)
+    assert res["top1_agree"] == agree
+    assert abs(res["top1_agree_pct"] - 100.0 * agree / 8) <= 1e-12
+    assert res["median_kld"] == np.percentile(np.sort(valid), 50, method="linear")
+    assert res["max_kld"] == valid.max()
+    # the valid rows alone give the same statistics
+    _, alone = _run(b[keep], q[keep])
+    for k in ("mean_kld", "median_kld", "p90_kld", "p99_kld", "max_kld", "top1_agree_pct"):
+        assert abs(res[k] - alone[k]) <= 1e-14 * abs(alone[k]) + 1e-300, k
+
+
 def test_masked_vocab_entries_contribute_nothing():
     # -inf in both rows on the same entries == dropping those entries
     V = 300
