@@ -58,7 +58,7 @@ def measured_peak():
 
 def kernel_source_hash() -> str:
     h = hashlib.sha256()
-    for name in ("kld_rows.cu", "kld_internal.h"):
+    for name in ("kld_rows.cu", "kld_internal.h", "kld_finish.cuh"):  # what the row kernel compiles from
         with open(os.path.join(ROOT, "logit_kl_divergence_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]

@@ -13,6 +13,7 @@
 #include <string>
 
 #include "kld_internal.h"
+#include "kld_probe.h"
 
 namespace {
 
@@ -57,12 +58,6 @@ class DeviceGuard {
 constexpr size_t kStageTargetBytes = 128ull << 20;  // per operand per buffer
 
 }  // namespace
-
-namespace kld {
-// Read-bandwidth probe (kld_probe.cu; see kld_stats_read_probe).
-cudaError_t launch_read_probe(const void* a, const void* b, int64_t bytes, uint32_t* derr,
-                              int sm_count, cudaStream_t stream);
-}  // namespace kld
 
 struct kld_stats_s {
   int device = 0;

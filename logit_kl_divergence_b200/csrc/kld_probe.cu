@@ -16,6 +16,7 @@
 #include <cstdint>
 
 #include "kld_internal.h"
+#include "kld_probe.h"
 
 namespace kld {
 namespace {
