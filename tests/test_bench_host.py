@@ -46,6 +46,7 @@ def test_traffic_is_reported_only_for_the_kernel_source_it_was_taken_on(tmp_path
     csrc.mkdir(parents=True)
     (csrc / "kld_rows.cu").write_text("// kernel v1\n")
     (csrc / "kld_internal.h").write_text("// header\n")
+    (csrc / "kld_finish.cuh").write_text("// finishing steps\n")
     (root / "profiles").mkdir()
     monkeypatch.setattr(bench, "ROOT", str(root))
     h = bench.kernel_source_hash()
