@@ -69,6 +69,11 @@ MUTANTS = {
     "percentile_takes_the_upper_neighbour": ("return lo + frac * (hi - lo);", "return hi;"),
     "topk_ties_to_highest_index": ("for (int64_t j = 0; j < V; ++j) order[(size_t)j] = j;",
                                    "for (int64_t j = 0; j < V; ++j) order[(size_t)j] = V - 1 - j;"),
+    "plus_inf_treated_as_finite": (
+        "if (std::isnan(b[j]) || std::isnan(q[j]) || b[j] == kInf || q[j] == kInf) {",
+        "if (std::isnan(b[j]) || std::isnan(q[j])) {"),
+    "empty_quant_row_not_excluded": ("if (m_b == -kInf || m_q == -kInf) {", "if (m_b == -kInf) {"),
+    "masked_token_not_flagged": ("        f |= ORACLE_ROW_INF_NLL;\n", ""),
     "grad_scale_dropped": ("g[j] = scale * (std::exp(q[j] - lse_q) - std::exp(b[j] - lse_b));",
                            "g[j] = (std::exp(q[j] - lse_q) - std::exp(b[j] - lse_b));"),
 }
