@@ -122,10 +122,11 @@ class ShardedKLDStats:
                                         device=base.device)
         records = self._records[:n]
         err = None
-        try:
-            self.stats.run_rows(base, quant, token_ids, out=records)
-        except Exception as e:  # reported to every rank below
-            err = e
+        if n > 0:  # an uneven split can leave a rank without rows; it still gathers and reduces
+            try:
+                self.stats.run_rows(base, quant, token_ids, out=records)
+            except Exception as e:  # reported to every rank below
+                err = e
         counts = _checked_counts(n, err, base.device, self.group)
         gathered = gather_records(records, self.group, counts=counts)
         self.stats.reduce(gathered, gathered.shape[0], token_ids is not None)

@@ -40,6 +40,8 @@ class OracleStats:
         self.res = None
 
     def run_rows(self, base, quant, token_ids=None, out=None):
+        if base.shape[0] < 1:  # as the library: a row pass needs at least one row
+            raise ValueError("kld_stats_run_rows: N must be >= 1")
         r = oracle.rows(base, quant, token_ids, self.dtype)
         out.copy_(torch.from_numpy(_pack(r)))
         return out
@@ -122,7 +124,8 @@ def test_shard_bounds_cover_all_rows_in_order():
         shard_bounds(4, 2, 2)
 
 
-@pytest.mark.parametrize("world,n_rows,with_tokens", [(2, 64, True), (2, 37, False), (3, 37, True)])
+@pytest.mark.parametrize("world,n_rows,with_tokens", [(2, 64, True), (2, 37, False), (3, 37, True),
+                                                     (3, 2, True)])  # the last rank holds no rows
 def test_sharded_statistics_equal_single_process_oracle(world, n_rows, with_tokens):
     _spawn(world, n_rows, with_tokens)
 
