@@ -59,7 +59,7 @@
 extern "C" {
 #endif
 
-#define KLD_ABI_VERSION 2
+#define KLD_ABI_VERSION 3
 
 typedef enum {
   KLD_OK = 0,
@@ -141,7 +141,9 @@ const char* kld_last_cuda_error(void);
 
 /*
  * Create a handle on `device` for runs of up to `max_rows` rows.
- * Allocates a device workspace of max_rows records (40 bytes each) plus a few
+ * Allocates a device workspace of max_rows records (40 bytes each), the
+ * per-field arrays of kld_stats_rows (24 bytes per row), the per-row
+ * normalisers of the gradient and top-k passes (48 bytes per row) plus a few
  * KB, and a pinned host copy of the result. Returns KLD_ERR_NO_DEVICE if the
  * device is not a compute-capability 10.0 (B200-class) GPU.
  */
@@ -172,11 +174,32 @@ kld_status_t kld_stats_run(kld_stats_t h, const void* base, const void* quant,
 kld_status_t kld_stats_result(kld_stats_t h, kld_result_t* out);
 
 /*
- * Device pointer to the per-row records of the last kld_stats_run (N of
- * them, stream-ordered after that run). Valid until the next run or destroy.
+ * Per-row results of the last run that wrote the handle's workspace
+ * (kld_stats_run, kld_stats_run_rows with rows_out NULL, kld_stats_run_host,
+ * kld_stats_run_grad, kld_stats_run_topk, kld_stats_merge_partials) as four
+ * contiguous DEVICE arrays of N values each, row i at index i:
+ *   *kld    KL(P_base || P_quant) in nats, NaN on excluded rows;
+ *   *nll    -log P_quant(tok), NaN without tokens or with a bad token;
+ *   *amax_b lowest index of the base row's maximum, -1 on excluded rows;
+ *   *amax_q the same for the quant row.
+ * Any of the four output pointers may be NULL (that array is not returned).
+ * The arrays are owned by the handle. The call enqueues a small kernel, on
+ * the stream of that run, that copies the fields out of the run's records
+ * (kld_stats_records); the arrays are valid in that stream's order after it
+ * and until the next run or kld_stats_destroy. KLD_ERR_NOT_READY before any
+ * such run.
  */
-kld_status_t kld_stats_rows(kld_stats_t h, const kld_row_t** rows_dev,
-                            int64_t* n_rows);
+kld_status_t kld_stats_rows(kld_stats_t h, const double** kld, const double** nll,
+                            const int32_t** amax_b, const int32_t** amax_q);
+
+/*
+ * The same rows as 40-byte records (kld_row_t, with the flags, the base
+ * model's NLL and dp as well): device pointer to the workspace's N records
+ * and their count, stream-ordered after the run that wrote them. Valid until
+ * the next run or destroy. No kernel is enqueued.
+ */
+kld_status_t kld_stats_records(kld_stats_t h, const kld_row_t** rows_dev,
+                               int64_t* n_rows);
 
 /*
  * The row pass alone: per-row records for rows [0, N) written to rows_out
@@ -287,14 +310,55 @@ kld_status_t kld_stats_merge_partials(kld_stats_t h, const void* parts, int G, i
  * with p = softmax(base), r = softmax(quant). Rows the statistics exclude get
  * idx -1 and NaN. idx_out, logp_out and rest_out may be NULL; all are
  * caller-owned DEVICE memory, naturally aligned. Enqueues the row pass, the
- * reduction (read with kld_stats_result) and a top-k pass that reads each
- * base row 2-4 times (from L2 after the first) and the quant row once.
+ * reduction (read with kld_stats_result) and a top-k pass. The top-k pass
+ * derives a threshold from a sample of each base row, then reads both rows
+ * once, collecting the elements above the threshold and summing the rest
+ * masses of all others in the same sweep. Rows whose threshold holds fewer
+ * than k or too many elements (large tie groups, masked rows) fall back to
+ * an exact radix selection that reads the base row 2-4 times.
  */
 #define KLD_MAX_TOPK 1024
 kld_status_t kld_stats_run_topk(kld_stats_t h, const void* base, const void* quant,
                                 const int32_t* token_ids, int64_t N, int64_t V,
                                 kld_dtype_t dtype, int k, int32_t* idx_out, float* logp_out,
                                 float* rest_out, double* kl_out, void* stream);
+
+/*
+ * Allocation-free kld_stats_run (no counterpart on the source pages: it is a
+ * deployment convenience of this library).
+ *
+ * For callers that cannot allocate device memory when they need the
+ * statistic -- e.g. a server that reserves almost all HBM for its own pool at
+ * start-up, or a loop that cannot afford the device synchronisation
+ * cudaMalloc/cudaFree may cause. It takes no handle and allocates nothing:
+ * per-row records and the error word live in one fixed array compiled into
+ * the library (KLD_STATIC_MAX_ROWS records, about 2.5 MiB), which every GPU
+ * that loads the library keeps until the process exits.
+ *
+ * Runs on the calling thread's current device and enqueues the row pass and
+ * the reduction on `stream`; inputs as for kld_stats_run (device pointers).
+ * result_dev: caller-owned DEVICE memory for one kld_result_t (8-byte
+ * aligned), written asynchronously; its flags_or / device_error fields carry
+ * what kld_stats_result() would report as status. 1 <= N <=
+ * KLD_STATIC_MAX_ROWS, else KLD_ERR_CAPACITY (nothing enqueued).
+ *
+ * The first call on a device (with it current) looks up the array's device
+ * address and sets kernel attributes; make that first call before any stream
+ * capture. All calls share the one array and each overwrites the previous
+ * call's records, so calls whose GPU work overlaps (other streams or threads)
+ * race: order them.
+ */
+#define KLD_STATIC_MAX_ROWS 65536
+kld_status_t kld_stats_run_static(const void* base, const void* quant,
+                                  const int32_t* token_ids, int64_t N,
+                                  int64_t V, kld_dtype_t dtype,
+                                  kld_result_t* result_dev, void* stream);
+
+/* ======================================================================
+ * Diagnostics. None of these computes anything the pages define: they
+ * expose timing, launch shape and self-checks of this library, for
+ * benchmarks and tests. A caller of the statistic needs none of them.
+ * ====================================================================== */
 
 /*
  * Self-test of failure detection (no counterpart on the source pages; a
@@ -310,11 +374,13 @@ kld_status_t kld_selftest_bounded_wait(int device, uint64_t limit_ns, int use_ab
                                        uint64_t* waited_ns);
 
 /*
- * Duration in milliseconds of the pass that follows the reduction in the
- * last kld_stats_run_grad (the gradient pass) or kld_stats_run_topk (the
- * top-k pass); timing enabled by kld_stats_set_timing; waits for that run.
+ * Duration in milliseconds of the second streaming pass of the last
+ * kld_stats_run_grad (the gradient pass) or kld_stats_run_topk (the top-k
+ * pass), the pass that follows the reduction; timing enabled by
+ * kld_stats_set_timing; waits for that run. KLD_ERR_NOT_READY when the last
+ * run had no such pass or was not timed.
  */
-kld_status_t kld_stats_grad_timing(kld_stats_t h, float* grad_ms);
+kld_status_t kld_stats_second_pass_timing(kld_stats_t h, float* pass_ms);
 
 /*
  * Read-bandwidth probe, a measuring aid with no counterpart in the
@@ -371,37 +437,6 @@ typedef struct {
 
 kld_status_t kld_plan(int64_t N, int64_t V, kld_dtype_t dtype, int sm_count,
                       kld_plan_t* out);
-
-/*
- * Allocation-free kld_stats_run (no counterpart on the source pages: it is a
- * deployment convenience of this library).
- *
- * For callers that cannot allocate device memory when they need the
- * statistic -- e.g. a server that reserves almost all HBM for its own pool at
- * start-up, or a loop that cannot afford the device synchronisation
- * cudaMalloc/cudaFree may cause. It takes no handle and allocates nothing:
- * per-row records and the error word live in one fixed array compiled into
- * the library (KLD_STATIC_MAX_ROWS records, about 2.5 MiB), which every GPU
- * that loads the library keeps until the process exits.
- *
- * Runs on the calling thread's current device and enqueues the row pass and
- * the reduction on `stream`; inputs as for kld_stats_run (device pointers).
- * result_dev: caller-owned DEVICE memory for one kld_result_t (8-byte
- * aligned), written asynchronously; its flags_or / device_error fields carry
- * what kld_stats_result() would report as status. 1 <= N <=
- * KLD_STATIC_MAX_ROWS, else KLD_ERR_CAPACITY (nothing enqueued).
- *
- * The first call on a device (with it current) looks up the array's device
- * address and sets kernel attributes; make that first call before any stream
- * capture. All calls share the one array and each overwrites the previous
- * call's records, so calls whose GPU work overlaps (other streams or threads)
- * race: order them.
- */
-#define KLD_STATIC_MAX_ROWS 65536
-kld_status_t kld_stats_run_static(const void* base, const void* quant,
-                                  const int32_t* token_ids, int64_t N,
-                                  int64_t V, kld_dtype_t dtype,
-                                  kld_result_t* result_dev, void* stream);
 
 #ifdef __cplusplus
 }

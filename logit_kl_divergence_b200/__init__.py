@@ -158,11 +158,12 @@ class KLDStats:
         _lib.check(st, "kld_stats_run_topk")
         return out
 
-    def grad_timing(self) -> float:
-        """Milliseconds of the last run_grad's gradient pass or run_topk's
-        top-k pass (timing enabled)."""
+    def second_pass_timing(self) -> float:
+        """Milliseconds of the second streaming pass of the last run_grad
+        (the gradient pass) or run_topk (the top-k pass); timing enabled."""
         ms = ctypes.c_float()
-        _lib.check(self._lib.kld_stats_grad_timing(self._h, ctypes.byref(ms)), "kld_stats_grad_timing")
+        _lib.check(self._lib.kld_stats_second_pass_timing(self._h, ctypes.byref(ms)),
+                   "kld_stats_second_pass_timing")
         return ms.value
 
     def read_probe(self, a: torch.Tensor, b: torch.Tensor, stream=None) -> None:
@@ -259,18 +260,41 @@ class KLDStats:
         out["status"] = st
         return out
 
-    def rows(self) -> torch.Tensor:
+    def records(self) -> torch.Tensor:
         """Copy of the last run's per-row records as a [N, 40] uint8 CUDA
         tensor (see :func:`rows_view`), ordered after the run on the current
-        stream."""
+        stream (kld_stats_records)."""
         p = ctypes.c_void_p()
         n = ctypes.c_int64()
-        _lib.check(self._lib.kld_stats_rows(self._h, ctypes.byref(p), ctypes.byref(n)), "kld_stats_rows")
+        _lib.check(self._lib.kld_stats_records(self._h, ctypes.byref(p), ctypes.byref(n)),
+                   "kld_stats_records")
         nbytes = n.value * ROW_RECORD_BYTES
         if nbytes == 0:
             return torch.empty((0, ROW_RECORD_BYTES), dtype=torch.uint8, device=self.device)
         view = torch.as_tensor(_DeviceBytes(p.value, nbytes), device=self.device)
         return view.view(n.value, ROW_RECORD_BYTES).clone()
+
+    def rows(self, stream=None) -> dict:
+        """Per-row results of the last run as four CUDA tensors of N values
+        (kld_stats_rows): ``kld`` and ``nll`` float64, ``amax_b`` and
+        ``amax_q`` int32. Copies of the handle's arrays, taken after the
+        library's per-field kernel on the run's stream."""
+        ptrs = [ctypes.c_void_p() for _ in range(4)]
+        _lib.check(self._lib.kld_stats_rows(self._h, *(ctypes.byref(p) for p in ptrs)),
+                   "kld_stats_rows")
+        n = ctypes.c_int64()
+        dummy = ctypes.c_void_p()
+        _lib.check(self._lib.kld_stats_records(self._h, ctypes.byref(dummy), ctypes.byref(n)),
+                   "kld_stats_records")
+        # the per-field kernel runs on the run's stream; order the copies after it
+        torch.cuda.synchronize(self.device)
+        out = {}
+        for name, p, (dt, size) in zip(("kld", "nll", "amax_b", "amax_q"), ptrs,
+                                       ((torch.float64, 8), (torch.float64, 8),
+                                        (torch.int32, 4), (torch.int32, 4))):
+            view = torch.as_tensor(_DeviceBytes(p.value, n.value * size), device=self.device)
+            out[name] = view.view(dt).clone()
+        return out
 
     def set_split(self, cluster_ctas: int) -> None:
         """Few-row launch shape: -1 never split rows, 0 default, 1 plain

@@ -104,14 +104,16 @@ SIGNATURES = {
     "kld_stats_destroy": (None, [_P]),
     "kld_stats_run": (_ST, [_P, _P, _P, _P, _I64, _I64, _I32, _P]),
     "kld_stats_result": (_ST, [_P, ctypes.POINTER(Result)]),
-    "kld_stats_rows": (_ST, [_P, ctypes.POINTER(_P), ctypes.POINTER(_I64)]),
+    "kld_stats_rows": (_ST, [_P, ctypes.POINTER(_P), ctypes.POINTER(_P), ctypes.POINTER(_P),
+                             ctypes.POINTER(_P)]),
+    "kld_stats_records": (_ST, [_P, ctypes.POINTER(_P), ctypes.POINTER(_I64)]),
     "kld_stats_run_rows": (_ST, [_P, _P, _P, _P, _I64, _I64, _I32, _P, _P]),
     "kld_stats_reduce": (_ST, [_P, _P, _I64, _I32, _P]),
     "kld_stats_run_host": (_ST, [_P, _P, _P, _P, _I64, _I64, _I32, _P]),
     "kld_stats_set_timing": (_ST, [_P, _I32]),
     "kld_stats_set_split": (_ST, [_P, _I32]),
     "kld_stats_run_grad": (_ST, [_P, _P, _P, _P, _I64, _I64, _I32, _P, _I32, ctypes.c_double, _P]),
-    "kld_stats_grad_timing": (_ST, [_P, ctypes.POINTER(ctypes.c_float)]),
+    "kld_stats_second_pass_timing": (_ST, [_P, ctypes.POINTER(ctypes.c_float)]),
     "kld_stats_read_probe": (_ST, [_P, _P, _P, _I64, _P]),
     "kld_selftest_bounded_wait": (_ST, [_I32, ctypes.c_uint64, _I32, ctypes.POINTER(ctypes.c_uint64)]),
     "kld_stats_run_topk": (_ST, [_P, _P, _P, _P, _I64, _I64, _I32, _I32, _P, _P, _P, _P, _P]),

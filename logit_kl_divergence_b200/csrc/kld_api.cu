@@ -64,6 +64,13 @@ struct kld_stats_s {
   int sm_count = 0;
   int64_t max_rows = 0;
   kld_row_t* rows = nullptr;
+  // kld_stats_rows: per-field arrays filled from the records on request
+  double* soa_kld = nullptr;  // one allocation: kld, nll (double), then amax_b, amax_q
+  double* soa_nll = nullptr;
+  int32_t* soa_amax_b = nullptr;
+  int32_t* soa_amax_q = nullptr;
+  cudaStream_t last_stream = nullptr;  // stream of the last run that wrote `rows`
+  bool rows_written = false;
   void* split_mem = nullptr;  // split-row scratch: partials, then tickets
   kld::RowAux* aux = nullptr;  // per-row normalisers for the gradient and top-k passes
   bool grad_timing_valid = false;
@@ -197,6 +204,11 @@ kld_status_t kld_stats_create(kld_stats_t* out, int64_t max_rows, int device) {
         cudaSuccess) { st = cuda_fail(err, "cudaMalloc(rows)"); break; }
     if ((err = cudaMalloc(&h->aux, sizeof(kld::RowAux) * static_cast<size_t>(max_rows))) !=
         cudaSuccess) { st = cuda_fail(err, "cudaMalloc(row normalisers)"); break; }
+    if ((err = cudaMalloc(&h->soa_kld, 24 * static_cast<size_t>(max_rows))) != cudaSuccess) {
+      st = cuda_fail(err, "cudaMalloc(per-field rows)"); break; }
+    h->soa_nll = h->soa_kld + max_rows;
+    h->soa_amax_b = reinterpret_cast<int32_t*>(h->soa_nll + max_rows);
+    h->soa_amax_q = h->soa_amax_b + max_rows;
     if ((err = cudaMalloc(&h->derr, sizeof(uint32_t))) != cudaSuccess) {
       st = cuda_fail(err, "cudaMalloc(error word)"); break; }
     if ((err = cudaMemset(h->derr, 0, sizeof(uint32_t))) != cudaSuccess) {
@@ -252,6 +264,7 @@ void kld_stats_destroy(kld_stats_t h) {
   if (h->hres) cudaFreeHost(h->hres);
   if (h->derr) cudaFree(h->derr);
   if (h->rows) cudaFree(h->rows);
+  if (h->soa_kld) cudaFree(h->soa_kld);
   if (h->split_mem) cudaFree(h->split_mem);
   if (h->aux) cudaFree(h->aux);
   delete h;
@@ -269,7 +282,11 @@ kld_status_t kld_stats_run_rows(kld_stats_t h, const void* base, const void* qua
   if (!guard.ok()) return cuda_fail(cudaGetLastError(), "cudaSetDevice");
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   KLD_CUDA(launch_rows(h, base, quant, token_ids, N, V, dtype, rows_out ? rows_out : h->rows, s));
-  if (!rows_out) h->last_rows = N;
+  if (!rows_out) {
+    h->last_rows = N;
+    h->last_stream = s;
+    h->rows_written = true;
+  }
   h->timing_valid = false;
   h->grad_timing_valid = false;
   return KLD_OK;
@@ -309,6 +326,8 @@ kld_status_t kld_stats_run(kld_stats_t h, const void* base, const void* quant,
                             &h->split, nullptr, s, nullptr, 0, h->hres_dev, &reduced));
   if (h->timing) KLD_CUDA(cudaEventRecord(h->tev[1], s));
   h->last_rows = N;
+  h->last_stream = s;
+  h->rows_written = true;
   if (!reduced) return enqueue_reduce(h, h->rows, N, token_ids != nullptr, s);
   if (h->timing) KLD_CUDA(cudaEventRecord(h->tev[2], s));
   KLD_CUDA(cudaEventRecord(h->done, s));
@@ -335,6 +354,8 @@ kld_status_t kld_stats_run_grad(kld_stats_t h, const void* base, const void* qua
   KLD_CUDA(launch_rows(h, base, quant, token_ids, N, V, dtype, h->rows, s, h->aux));
   if (h->timing) KLD_CUDA(cudaEventRecord(h->tev[1], s));
   h->last_rows = N;
+  h->last_stream = s;
+  h->rows_written = true;
   st = enqueue_reduce(h, h->rows, N, token_ids != nullptr, s);
   if (st != KLD_OK) return st;
   KLD_CUDA(kld::launch_grad(base, quant, h->aux, N, V, dtype, grad, grad_dtype,
@@ -375,6 +396,8 @@ kld_status_t kld_stats_merge_partials(kld_stats_t h, const void* parts, int G, i
   h->grad_timing_valid = false;
   KLD_CUDA(kld::launch_merge(parts, G, N, token_ids, V_total, h->rows, s));
   h->last_rows = N;
+  h->last_stream = s;
+  h->rows_written = true;
   return enqueue_reduce(h, h->rows, N, token_ids != nullptr, s);
 }
 
@@ -398,6 +421,8 @@ kld_status_t kld_stats_run_topk(kld_stats_t h, const void* base, const void* qua
   KLD_CUDA(launch_rows(h, base, quant, token_ids, N, V, dtype, h->rows, s, h->aux));
   if (h->timing) KLD_CUDA(cudaEventRecord(h->tev[1], s));
   h->last_rows = N;
+  h->last_stream = s;
+  h->rows_written = true;
   st = enqueue_reduce(h, h->rows, N, token_ids != nullptr, s);
   if (st != KLD_OK) return st;
   KLD_CUDA(kld::launch_topk(base, quant, h->aux, N, V, dtype, k, idx_out, logp_out, rest_out,
@@ -442,13 +467,13 @@ kld_status_t kld_stats_read_probe(kld_stats_t h, const void* a, const void* b, i
   return KLD_OK;
 }
 
-kld_status_t kld_stats_grad_timing(kld_stats_t h, float* grad_ms) {
-  if (!h || !grad_ms) return KLD_ERR_INVALID_ARG;
+kld_status_t kld_stats_second_pass_timing(kld_stats_t h, float* pass_ms) {
+  if (!h || !pass_ms) return KLD_ERR_INVALID_ARG;
   if (!h->grad_timing_valid || !h->has_result) return KLD_ERR_NOT_READY;
   DeviceGuard guard(h->device);
   if (!guard.ok()) return cuda_fail(cudaGetLastError(), "cudaSetDevice");
   KLD_CUDA(cudaEventSynchronize(h->tev[3]));
-  KLD_CUDA(cudaEventElapsedTime(grad_ms, h->tev[2], h->tev[3]));
+  KLD_CUDA(cudaEventElapsedTime(pass_ms, h->tev[2], h->tev[3]));
   return KLD_OK;
 }
 
@@ -465,10 +490,25 @@ kld_status_t kld_stats_result(kld_stats_t h, kld_result_t* out) {
   return KLD_OK;
 }
 
-kld_status_t kld_stats_rows(kld_stats_t h, const kld_row_t** rows_dev, int64_t* n_rows) {
+kld_status_t kld_stats_records(kld_stats_t h, const kld_row_t** rows_dev, int64_t* n_rows) {
   if (!h || !rows_dev || !n_rows) return KLD_ERR_INVALID_ARG;
   *rows_dev = h->rows;
   *n_rows = h->last_rows;
+  return KLD_OK;
+}
+
+kld_status_t kld_stats_rows(kld_stats_t h, const double** kld, const double** nll,
+                            const int32_t** amax_b, const int32_t** amax_q) {
+  if (!h) return KLD_ERR_INVALID_ARG;
+  if (!h->rows_written) return KLD_ERR_NOT_READY;
+  DeviceGuard guard(h->device);
+  if (!guard.ok()) return cuda_fail(cudaGetLastError(), "cudaSetDevice");
+  KLD_CUDA(kld::launch_split_records(h->rows, h->last_rows, h->soa_kld, h->soa_nll,
+                                     h->soa_amax_b, h->soa_amax_q, h->last_stream));
+  if (kld) *kld = h->soa_kld;
+  if (nll) *nll = h->soa_nll;
+  if (amax_b) *amax_b = h->soa_amax_b;
+  if (amax_q) *amax_q = h->soa_amax_q;
   return KLD_OK;
 }
 
@@ -568,6 +608,8 @@ kld_status_t kld_stats_run_host(kld_stats_t h, const void* base_host, const void
     KLD_CUDA(cudaEventRecord(h->freed[b], s));
   }
   h->last_rows = N;
+  h->last_stream = s;
+  h->rows_written = true;
   return enqueue_reduce(h, h->rows, N, token_ids_host != nullptr, s);
 }
 

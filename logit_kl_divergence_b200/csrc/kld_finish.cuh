@@ -169,8 +169,13 @@ __device__ __forceinline__ Sums zero_sums() {
 // SMs); the device error word is read and cleared; the result goes to *out.
 __device__ __forceinline__ void reduce_few_rows(const kld_row_t* rows, int N, int has_nll,
                                                 uint32_t* derr, kld_result_t* out, int lane) {
-  // The error word is taken first: its round trip overlaps the record loads
-  // (every row's record is written, so no part of the pass can still set it).
+  // The error word is taken first: its round trip overlaps the record loads.
+  // Every row's record is written, so every consumer and epilogue wait of
+  // the pass has ended. The one wait that can still end later is a
+  // producer's bounded drain of its own last bulk copies, after its CTA's
+  // part is done; those copies were consumed before the record could be
+  // written, so the drain finds them complete. Were one still to time out,
+  // its bit would be reported by the next run of the same handle, not this.
   const uint32_t de = (lane == 0 && derr) ? atomicExch(derr, 0u) : 0u;
   Sums s = zero_sums();
   unsigned long long key = ~0ull;  // lanes past N sort last

@@ -130,4 +130,9 @@ cudaError_t launch_reduce(const kld_row_t* rows, int64_t N, int has_nll,
                           uint32_t* derr, kld_result_t* out,
                           cudaStream_t stream);
 
+// Per-field copies of N records (kld_stats_rows): kld[i], nll[i], amax_b[i],
+// amax_q[i] from rows[i].
+cudaError_t launch_split_records(const kld_row_t* rows, int64_t N, double* kld, double* nll,
+                                 int32_t* amax_b, int32_t* amax_q, cudaStream_t stream);
+
 }  // namespace kld

@@ -408,7 +408,32 @@ __global__ void __launch_bounds__(kReduceThreads, 1)
   }
 }
 
+// Per-field arrays from the records, one thread per row.
+__global__ void kld_split_records_kernel(const kld_row_t* __restrict__ rows, int64_t N,
+                                         double* __restrict__ kld, double* __restrict__ nll,
+                                         int32_t* __restrict__ amax_b, int32_t* __restrict__ amax_q) {
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < N;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const kld_row_t r = rows[i];
+    kld[i] = r.kld;
+    nll[i] = r.nll;
+    amax_b[i] = r.argmax_base;
+    amax_q[i] = r.argmax_quant;
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_split_records(const kld_row_t* rows, int64_t N, double* kld, double* nll,
+                                 int32_t* amax_b, int32_t* amax_q, cudaStream_t stream) {
+  if (N < 1) return cudaSuccess;
+  constexpr int kThreads = 256;
+  int64_t blocks = (N + kThreads - 1) / kThreads;
+  if (blocks > 4096) blocks = 4096;
+  kld_split_records_kernel<<<static_cast<unsigned>(blocks), kThreads, 0, stream>>>(
+      rows, N, kld, nll, amax_b, amax_q);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_reduce(const kld_row_t* rows, int64_t N, int has_nll, uint32_t* derr,
                           kld_result_t* out, cudaStream_t stream) {

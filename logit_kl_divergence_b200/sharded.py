@@ -113,7 +113,8 @@ class ShardedKLDStats:
     def run(self, base: torch.Tensor, quant: torch.Tensor, token_ids: torch.Tensor | None = None) -> dict:
         """Collective. Every rank passes its own [n_r, V] rows (same V, dtype
         and token-id presence on every rank); returns the statistics of all
-        ranks' rows."""
+        ranks' rows. The ranks together must hold at least one row: with
+        none, every rank raises ValueError after the same collective steps."""
         n = base.shape[0]
         if n > self.max_rows_per_rank:
             raise ValueError("more rows than max_rows_per_rank")
@@ -128,6 +129,8 @@ class ShardedKLDStats:
             except Exception as e:  # reported to every rank below
                 err = e
         counts = _checked_counts(n, err, base.device, self.group)
+        if sum(counts) == 0:  # every rank sees the same counts: all raise together
+            raise ValueError("sharded statistic over zero rows: every rank passed an empty shard")
         gathered = gather_records(records, self.group, counts=counts)
         self.stats.reduce(gathered, gathered.shape[0], token_ids is not None)
         return self.stats.result()

@@ -47,7 +47,7 @@ def gpu_run(base, quant, tok=None, use_rows_api=False, split=None):
         else:
             st.run(base, quant, tok)
             res = st.result()
-            rec = rows_view(st.rows())
+            rec = rows_view(st.records())
         rows = {k: v.cpu().numpy() for k, v in rec.items()}
         rows["flags"] = rows["flags"].astype(np.uint32)
         return rows, res

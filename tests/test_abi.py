@@ -75,7 +75,7 @@ int main(void) {
 
 
 def test_abi_version_and_status_strings(lib):
-    assert lib.kld_abi_version() == 2
+    assert lib.kld_abi_version() == 3
     for s in range(0, 10):
         assert lib.kld_status_string(s)
     assert lib.kld_status_string(12345) == b"unknown status"
@@ -93,11 +93,44 @@ def test_arguments_rejected_before_any_gpu_work(lib):
     assert lib.kld_stats_run_host(None, p, p, None, 1, 1, 0, None) == _lib.KLD_ERR_INVALID_ARG
     assert lib.kld_stats_set_timing(None, 1) == _lib.KLD_ERR_INVALID_ARG
     assert lib.kld_stats_read_probe(None, p, p, 1 << 20, None) == _lib.KLD_ERR_INVALID_ARG
+    d, n = ctypes.c_void_p(), ctypes.c_int64()
+    assert lib.kld_stats_rows(None, ctypes.byref(d), None, None, None) == _lib.KLD_ERR_INVALID_ARG
+    assert lib.kld_stats_records(None, ctypes.byref(d), ctypes.byref(n)) == _lib.KLD_ERR_INVALID_ARG
+    ms = ctypes.c_float()
+    assert lib.kld_stats_second_pass_timing(None, ctypes.byref(ms)) == _lib.KLD_ERR_INVALID_ARG
     w = ctypes.c_uint64()
     assert lib.kld_selftest_bounded_wait(-1, 10**6, 0, ctypes.byref(w)) == _lib.KLD_ERR_INVALID_ARG
     assert lib.kld_selftest_bounded_wait(0, 999, 0, ctypes.byref(w)) == _lib.KLD_ERR_INVALID_ARG
     assert lib.kld_selftest_bounded_wait(0, 10**10 + 1, 0, ctypes.byref(w)) == _lib.KLD_ERR_INVALID_ARG
     lib.kld_stats_destroy(None)  # no-op
+
+
+def test_header_declarations_link_and_reject_a_null_handle():
+    # A C caller compiled against include/kld_stats.h, linked to the library:
+    # the per-field row accessor of the boundary takes exactly the declared
+    # arguments (four output arrays), and its checks run before any CUDA call.
+    src = r'''
+#include <stdio.h>
+#include "kld_stats.h"
+int main(void) {
+  const double* kld = 0; const double* nll = 0;
+  const int32_t* amax_b = 0; const int32_t* amax_q = 0;
+  const kld_row_t* rec = 0; int64_t n = 0; float ms = 0.f;
+  printf("%d %d %d %d\n", (int)kld_stats_rows(0, &kld, &nll, &amax_b, &amax_q),
+         (int)kld_stats_records(0, &rec, &n), (int)kld_stats_second_pass_timing(0, &ms),
+         kld_abi_version());
+  return 0;
+}
+'''
+    with tempfile.TemporaryDirectory() as d:
+        c = os.path.join(d, "t.c")
+        exe = os.path.join(d, "t")
+        open(c, "w").write(src)
+        libdir = os.path.dirname(build.LIB)
+        subprocess.run(["gcc", "-I", os.path.join(ROOT, "include"), c, "-o", exe, build.LIB,
+                        f"-Wl,-rpath,{libdir}"], check=True)
+        out = subprocess.run([exe], capture_output=True, text=True, check=True).stdout.split()
+    assert [int(x) for x in out] == [_lib.KLD_ERR_INVALID_ARG] * 3 + [3]
 
 
 def test_create_without_gpu_reports_no_device(lib):

@@ -207,3 +207,52 @@ def test_handle_reuse_across_sizes_and_dtypes():
         _, ores = oracle.run(w.base, w.quant, w.token_ids, ODT[dt])
         assert_stats_match({**gres}, ores)
     st.close()
+
+
+def test_per_field_row_arrays_match_records_and_oracle():
+    # kld_stats_rows: four device arrays (KL, NLL, both argmaxes) taken from
+    # the records of the last run, including excluded rows (NaN / -1) and a
+    # run that reused the handle with fewer rows.
+    import ctypes
+
+    from logit_kl_divergence_b200 import _lib, rows_view
+
+    st = KLDStats(max_rows=300, device=DEV)
+    for n, seed in ((300, 8), (37, 9)):
+        w = synth.make_recipe("edge", n=n, v=4099, dtype=synth.F32, seed=seed)
+        st.run(w.base.to(DEV), w.quant.to(DEV), w.token_ids.to(DEV))
+        st.result()
+        soa = {k: v.cpu().numpy() for k, v in st.rows().items()}
+        rec = {k: v.cpu().numpy() for k, v in rows_view(st.records()).items()}
+        # the same call through the C ABI with some outputs not requested
+        lib = _lib.load()
+        p = ctypes.c_void_p()
+        assert lib.kld_stats_rows(st._h, None, None, ctypes.byref(p), None) == _lib.KLD_OK
+        assert p.value
+        for k in ("kld", "nll"):
+            assert soa[k].shape == (n,)
+            np.testing.assert_array_equal(soa[k], rec[k])  # NaN positions included
+        np.testing.assert_array_equal(soa["amax_b"], rec["amax_b"])
+        np.testing.assert_array_equal(soa["amax_q"], rec["amax_q"])
+        o_rows, _ = oracle.run(w.base, w.quant, w.token_ids, ODT[synth.F32])
+        np.testing.assert_array_equal(soa["amax_b"], o_rows["amax_b"])
+        np.testing.assert_array_equal(soa["amax_q"], o_rows["amax_q"])
+        ok = np.isnan(o_rows["kld"]) & np.isnan(soa["kld"])
+        ok |= np.abs(soa["kld"] - o_rows["kld"]) <= 1e-6 + 1e-4 * np.abs(o_rows["kld"])
+        ok |= np.isinf(o_rows["kld"]) & (soa["kld"] == o_rows["kld"])
+        assert ok.all()
+    st.close()
+
+
+def test_per_field_rows_before_any_run_is_not_ready():
+    import ctypes
+
+    from logit_kl_divergence_b200 import _lib
+
+    st = KLDStats(max_rows=4, device=DEV)
+    try:
+        d = ctypes.c_void_p()
+        lib = _lib.load()
+        assert lib.kld_stats_rows(st._h, ctypes.byref(d), None, None, None) == _lib.KLD_ERR_NOT_READY
+    finally:
+        st.close()

@@ -42,7 +42,7 @@ def _sharded(b, q, tok, bounds):
         st.run_partials(bd[:, c0:c1].contiguous(), qd[:, c0:c1].contiguous(), td, c0, v, out=parts[g])
     st.merge_partials(parts, td, v)
     res = st.result()
-    rec = {k: t.cpu().numpy() for k, t in rows_view(st.rows()).items()}
+    rec = {k: t.cpu().numpy() for k, t in rows_view(st.records()).items()}
     rec["flags"] = rec["flags"].astype(np.uint32)
     st.close()
     return rec, res

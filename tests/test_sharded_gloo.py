@@ -206,6 +206,16 @@ def _fail_worker(rank, world, port, mode, errq):
             assert got.shape == (world, 5, 64)
             for r in range(world):
                 assert torch.all(got[r, :, 0] == r) and torch.equal(got[r, :, 1], torch.arange(5, dtype=torch.uint8))
+        elif mode == "zero":
+            # every rank passes an empty shard: all raise the same clear
+            # error after the same collective steps, and the group stays
+            # usable for a normal step
+            sk = ShardedKLDStats(max_rows_per_rank=hi - lo, stats=OracleStats(oracle.F32))
+            with pytest.raises(ValueError, match="zero rows"):
+                sk.run(b[:0], q[:0], t[:0])
+            res = sk.run(b, q, t)
+            _, full = oracle.run(w.base, w.quant, w.token_ids, oracle.F32)
+            _same(res, full)
         elif mode == "exit":
             # the last rank leaves between steps without telling anyone; the
             # others' next collective must end with an error, not hang
@@ -230,7 +240,8 @@ def _fail_worker(rank, world, port, mode, errq):
         raise
 
 
-@pytest.mark.parametrize("world,mode", [(2, "status"), (3, "status"), (2, "vocab"), (3, "vocab"), (2, "exit")])
+@pytest.mark.parametrize("world,mode", [(2, "status"), (3, "status"), (2, "vocab"), (3, "vocab"),
+                                        (2, "zero"), (2, "exit")])
 def test_rank_failure_is_seen_by_every_rank(world, mode):
     ctx = mp.get_context("spawn")
     errq = ctx.SimpleQueue()
