@@ -9,9 +9,10 @@ to the host. The batch is one 8192-token context at a vocabulary of 151936
 (fp32 logits, 2 x 4.98 GB per GPU), generated on the device by the seeded
 generator; it is far larger than L2, so no L2 flush is needed between steps.
 
-With N GPUs (torchrun, one rank per GPU) every rank scores its own context
-(weak scaling); the per-row records are all-gathered over NCCL and every
-rank reduces the full set, since exact percentiles need all rows.
+With N GPUs, one process per GPU (launched with torchrun, or by this script
+itself when --gpus N > 1 is given without it), every rank scores its own
+context (weak scaling); the per-row records are all-gathered over NCCL and
+every rank reduces the full set, since exact percentiles need all rows.
 
 Prints one JSON line (rank 0).
 """
@@ -359,6 +360,223 @@ def split_row_latency(dev, stream, min_calls: int = SPLIT_CALLS):
     return out
 
 
+def free_port() -> int:
+    import socket
+
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        return sk.getsockname()[1]
+
+
+def torchrun_argv(n: int, port: int, script: str, argv: list[str]) -> list[str]:
+    """One process per GPU on this node, rendezvous on the loopback address."""
+    return [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={n}",
+            "--master-addr", "127.0.0.1", "--master-port", str(port), script, *argv]
+
+
+def relaunch(n: int, argv: list[str]) -> int:
+    """`python bench.py --gpus N` without torchrun: start the N ranks here.
+    Returns the launcher's exit code (2 when fewer than N GPUs are visible)."""
+    import torch
+
+    visible = torch.cuda.device_count()
+    if visible < n:
+        print(f"bench.py: {n} GPUs requested (--gpus {n}) but {visible} visible; "
+              f"nothing was run", file=sys.stderr)
+        return 2
+    return subprocess.run(torchrun_argv(n, free_port(), os.path.abspath(__file__), argv)).returncode
+
+
+class DeviceClock:
+    """Device time: CUDA events recorded on the launching stream."""
+
+    def __init__(self, dev):
+        import torch
+
+        self.torch = torch
+        self.dev = dev
+        self.stream = torch.cuda.current_stream(dev)
+
+    def mark(self):
+        e = self.torch.cuda.Event(enable_timing=True)
+        e.record(self.stream)
+        return e
+
+    def sync(self):
+        self.torch.cuda.synchronize(self.dev)
+
+    def ms(self, a, b) -> float:
+        return a.elapsed_time(b)
+
+
+class HostClock:
+    """Host wall time, for ranks that run on CPU cores (the multi-rank logic
+    checked with gloo and a stand-in handle); never a GPU measurement."""
+
+    def mark(self):
+        return time.perf_counter()
+
+    def sync(self):
+        pass
+
+    def ms(self, a, b) -> float:
+        return 1000.0 * (b - a)
+
+
+def _over_ranks(x: float, device, op) -> float:
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=op)
+    return float(t.item())
+
+
+def sharded_line(args, rank: int, world: int, dev, sk, shard, clock, peak: float, peak_kind: str,
+                 sampler=None, cpu_fn=None, workload: str = WORKLOAD):
+    """The multi-GPU step, timed: every rank runs the row pass on its own
+    shard, the records are all-gathered and every rank reduces all of them
+    (``sk``: a ShardedKLDStats, the public multi-GPU API), then reads the
+    result. Returns rank 0's JSON line (None on the other ranks).
+
+    value: rows of all ranks / the max over ranks of the device time of the
+    timed steps. e2e: the same step through ShardedKLDStats.run_host from
+    (pinned) host copies of each shard, max over ranks. roofline: the row
+    pass of each rank timed by the library's events; achieved = sum over
+    ranks of that rank's algorithmic bytes / its mean row-pass time, against
+    world x the per-GPU peak."""
+    import torch
+    import torch.distributed as dist
+
+    base, quant, tok = shard
+    N, V = base.shape
+    eb = base.element_size()
+    in_bytes = 2 * N * V * eb
+    sk.stats.set_timing(True)
+    res = None
+    counts = [N] * world  # equal shards: one host wait per step (the result)
+    for _ in range(args.warmup):
+        res = sk.run(base, quant, tok, counts=counts)
+    dist.barrier()
+    clock.sync()
+    if sampler is not None:
+        sampler.mark_start()
+    start = clock.mark()
+    row_ms = []
+    for _ in range(args.steps):
+        res = sk.run(base, quant, tok, counts=counts)
+        row_ms.append(sk.stats.timing()[0])
+    end = clock.mark()
+    clock.sync()
+    if sampler is not None:
+        sampler.mark_end()
+    dist.barrier()
+    clocks = sampler.stop() if sampler is not None else None
+    ms = _over_ranks(clock.ms(start, end), dev, dist.ReduceOp.MAX)
+    ms_per_step = ms / args.steps
+    total_rows = N * world
+    value = total_rows / (ms_per_step / 1000.0)
+    avg_row_ms = sum(row_ms) / len(row_ms)
+    achieved_rank = in_bytes / (avg_row_ms / 1000.0) / 1e9
+    achieved = _over_ranks(achieved_rank, dev, dist.ReduceOp.SUM)
+    slowest_row_ms = _over_ranks(avg_row_ms, dev, dist.ReduceOp.MAX)
+    traffic = recorded_traffic(workload)
+    roofline = {"bound": "hbm", "achieved": achieved, "peak": peak * world, "unit": "GB/s",
+                "frac": achieved / (peak * world), "traffic": traffic,
+                "peak_source": f"{world} x {peak_kind} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)",
+                "frac_of_8TBs_nominal": achieved / (8000.0 * world),
+                "kernel": f"kld_rows_kernel<{'f32' if eb == 4 else 'bf16'}>",
+                "row_pass_ms": avg_row_ms, "row_pass_ms_max_over_ranks": slowest_row_ms,
+                "algorithmic_bytes_per_launch": in_bytes,
+                "note": "achieved summed over ranks; traffic and bytes per launch are per rank"}
+
+    # End to end: each rank's shard in host memory (pinned where a GPU is
+    # present), copied by the library in chunks overlapped with its row pass.
+    pin = torch.cuda.is_available() and base.is_cuda
+    hb, hq = base.cpu(), quant.cpu()
+    ht = None if tok is None else tok.cpu()
+    if pin:
+        hb, hq = hb.pin_memory(), hq.pin_memory()
+        ht = None if ht is None else ht.pin_memory()
+    e2e = None
+    if args.e2e_steps > 0:
+        sk.run_host(hb, hq, ht, device=dev, counts=counts)
+        dist.barrier()
+        clock.sync()
+        a = clock.mark()
+        for _ in range(args.e2e_steps):
+            sk.run_host(hb, hq, ht, device=dev, counts=counts)
+        b = clock.mark()
+        clock.sync()
+        ems = _over_ranks(clock.ms(a, b), dev, dist.ReduceOp.MAX) / args.e2e_steps
+        e2e = {"value": total_rows / (ems / 1000.0), "unit": "rows/s",
+               "h2d_bytes_per_step": (in_bytes + (4 * N if tok is not None else 0)) * world,
+               "d2h_bytes_per_step": RESULT_BYTES * world, "ms_per_step": ems,
+               "path": "ShardedKLDStats.run_host (kld_stats_run_rows_host per rank, record "
+                       "all-gather, kld_stats_reduce; host buffers pinned); bytes summed over ranks"}
+    del hb, hq, ht
+
+    cpu = cpu_mt = None
+    if rank == 0 and cpu_fn is not None and not args.no_cpu_baseline:
+        cpu, cpu_mt = cpu_fn(workload)
+    dist.barrier()  # the other ranks wait for rank 0's host-core baseline
+    if rank != 0:
+        return None
+    return {
+        "metric": METRIC, "value": value, "unit": "rows/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32" if eb == 4 else "bf16",
+        "data": "synthetic",
+        "config": {"workload": workload, "rows_per_gpu": N, "vocab": V,
+                   "logit_dtype": "f32" if eb == 4 else "bf16", "global_rows": total_rows,
+                   "parallelism": f"rows sharded over {world} GPU(s): one 8192-token context per "
+                                  f"rank, records all-gathered (NCCL), every rank reduces all rows",
+                   "l2": f"inputs ({in_bytes / 1e9:.2f} GB per step per GPU) exceed the 126 MB L2; "
+                         f"no flush"},
+        "roofline": roofline, "cpu_baseline": cpu, "cpu_baseline_all_cores": cpu_mt, "e2e": e2e,
+        "gpu_launches": 2 * args.steps * world, "gpu_launches_note": "row pass + reduction per step per rank",
+        "clocks": clocks, "gbs": in_bytes * world / (ms_per_step / 1000.0) / 1e9,
+        "mean_kld": res["mean_kld"], "top1_agree_pct": res["top1_agree_pct"], "ppl": res["ppl"],
+        "ppl_base": res["ppl_base"], "rms_dp": res["rms_dp"], "mean_dp": res["mean_dp"],
+        "median_kld": res["median_kld"], "p99_kld": res["p99_kld"], "max_kld": res["max_kld"],
+    }
+
+
+def run_sharded_main(args, rank: int, world: int, local: int):
+    """The multi-GPU benchmark (NCCL group, one rank per GPU; --sharded runs
+    it on a group of one rank)."""
+    import datetime
+
+    import torch
+    import torch.distributed as dist
+
+    from logit_kl_divergence_b200 import synth
+    from logit_kl_divergence_b200.sharded import ShardedKLDStats
+
+    dev = torch.device("cuda", local)
+    if "MASTER_ADDR" not in os.environ:  # one rank, launched without torchrun
+        os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(free_port()), RANK="0",
+                          WORLD_SIZE="1", LOCAL_RANK=str(local))
+    dist.init_process_group("nccl", device_id=dev, timeout=datetime.timedelta(seconds=120))
+    dt = synth.F32 if args.dtype == "f32" else synth.BF16
+    w = synth.make(WORKLOAD, device=dev, seed=synth.WORKLOADS[WORKLOAD][4] + 7919 * rank, n=args.rows,
+                   dtype=dt)
+    sk = ShardedKLDStats(max_rows_per_rank=w.base.shape[0], device=dev)
+    peak, peak_kind = measured_peak()
+    sampler = ClockSampler(local)
+    try:
+        line = sharded_line(args, rank, world, dev, sk, (w.base, w.quant, w.token_ids), DeviceClock(dev),
+                            peak, peak_kind, sampler=sampler, cpu_fn=cpu_baseline)
+        if line is not None:
+            if args.rows is not None or args.dtype != "f32":
+                line["config"]["override"] = {"rows": w.base.shape[0], "dtype": args.dtype,
+                                              "note": "profiling run, not the benchmark workload"}
+            print(json.dumps(line), flush=True)
+    finally:
+        sk.close()
+        dist.destroy_process_group()
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -390,118 +608,74 @@ def main():
     if args.impl == "reference":
         run_reference(args, rank)
         return
+    if world == 1 and args.gpus > 1 and "LOCAL_RANK" not in os.environ:
+        sys.exit(relaunch(args.gpus, sys.argv[1:]))
 
     import torch
-    import torch.distributed as dist
 
     from logit_kl_divergence_b200 import KLDStats, synth
-    from logit_kl_divergence_b200.sharded import gather_records
 
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    sharded = world > 1 or args.sharded
-    if sharded:
-        import datetime
-
-        if "MASTER_ADDR" not in os.environ:  # one rank, launched without torchrun
-            import socket
-
-            with socket.socket() as sk:
-                sk.bind(("127.0.0.1", 0))
-                port = sk.getsockname()[1]
-            os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK="0",
-                              WORLD_SIZE="1", LOCAL_RANK=str(local))
-        dist.init_process_group("nccl", device_id=dev, timeout=datetime.timedelta(seconds=120))
+    if world > 1 or args.sharded:
+        run_sharded_main(args, rank, world, local)
+        return
 
     name = WORKLOAD
     dt = synth.F32 if args.dtype == "f32" else synth.BF16
-    w = synth.make(name, device=dev, seed=synth.WORKLOADS[name][4] + 7919 * rank, n=args.rows,
-                   dtype=dt)
+    w = synth.make(name, device=dev, seed=synth.WORKLOADS[name][4], n=args.rows, dtype=dt)
     N, V = w.base.shape
     eb = w.bytes_per_elem
     in_bytes = 2 * N * V * eb
     stream = torch.cuda.current_stream(dev)
 
-    st = KLDStats(max_rows=N * world, device=dev)
-    st.set_timing(not sharded)
-    records = None
-    if sharded:
-        records = torch.empty((N, ROW_RECORD_BYTES), dtype=torch.uint8, device=dev)
-
+    st = KLDStats(max_rows=N, device=dev)
+    st.set_timing(True)
     row_ms, red_ms = [], []
 
     def step(timed: bool):
-        if not sharded:
-            st.run(w.base, w.quant, w.token_ids)
-            res = st.result()
-            if timed:
-                rp_ms, rd_ms = st.timing()
-                row_ms.append(rp_ms)
-                red_ms.append(rd_ms)
-        else:
-            st.run_rows(w.base, w.quant, w.token_ids, out=records)
-            gathered = gather_records(records, counts=[N] * world)
-            st.reduce(gathered, N * world, True)
-            res = st.result()
+        st.run(w.base, w.quant, w.token_ids)
+        res = st.result()
+        if timed:
+            rp_ms, rd_ms = st.timing()
+            row_ms.append(rp_ms)
+            red_ms.append(rd_ms)
         return res
 
     sampler = ClockSampler(local)
     for _ in range(args.warmup):
         res = step(False)
 
-    # Row-kernel time on its own stream for multi-GPU too (events bracket the
-    # row pass only; used for the roofline).
-    if sharded:
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-
-    if sharded:
-        dist.barrier()
     torch.cuda.synchronize(dev)
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     sampler.mark_start()
     start.record(stream)
     for _ in range(args.steps):
-        if not sharded:
-            res = step(True)
-        else:
-            e0.record(stream)
-            st.run_rows(w.base, w.quant, w.token_ids, out=records)
-            e1.record(stream)
-            gathered = gather_records(records, counts=[N] * world)
-            st.reduce(gathered, N * world, True)
-            res = st.result()
-            row_ms.append(e0.elapsed_time(e1))
+        res = step(True)
     end.record(stream)
     torch.cuda.synchronize(dev)
     sampler.mark_end()
-    if sharded:
-        dist.barrier()
     clocks = sampler.stop()
     ms = start.elapsed_time(end)
-    if sharded:
-        t = torch.tensor([ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
     ms_per_step = ms / args.steps
-    total_rows = N * world
+    total_rows = N
     value = total_rows / (ms_per_step / 1000.0)
 
     # Read-only roofline of the row pass on this device, for context beside the
     # copy-bandwidth peak: the library's probe streams the same two inputs
     # into shared memory with the row pass's bulk copies and computes nothing.
     read_probe_gbs = None
-    if not sharded:
-        for _ in range(3):
-            st.read_probe(w.base, w.quant)
-        torch.cuda.synchronize(dev)
-        pa, pb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        preps = 10
-        pa.record(stream)
-        for _ in range(preps):
-            st.read_probe(w.base, w.quant)
-        pb.record(stream)
-        torch.cuda.synchronize(dev)
-        read_probe_gbs = in_bytes / (pa.elapsed_time(pb) / preps / 1000.0) / 1e9
+    for _ in range(3):
+        st.read_probe(w.base, w.quant)
+    torch.cuda.synchronize(dev)
+    pa, pb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    preps = 10
+    pa.record(stream)
+    for _ in range(preps):
+        st.read_probe(w.base, w.quant)
+    pb.record(stream)
+    torch.cuda.synchronize(dev)
+    read_probe_gbs = in_bytes / (pa.elapsed_time(pb) / preps / 1000.0) / 1e9
 
     peak, peak_kind = measured_peak()
     avg_row_ms = sum(row_ms) / len(row_ms)
@@ -513,7 +687,7 @@ def main():
                 "frac_of_8TBs_nominal": achieved / 8000.0,
                 "read_probe_gbs": read_probe_gbs,
                 "frac_of_read_probe": (achieved / read_probe_gbs) if read_probe_gbs else None,
-                "kernel": "kld_rows_kernel<f32>", "row_pass_ms": avg_row_ms,
+                "kernel": f"kld_rows_kernel<{args.dtype}>", "row_pass_ms": avg_row_ms,
                 "reduce_ms": (sum(red_ms) / len(red_ms)) if red_ms else None,
                 "algorithmic_bytes_per_launch": in_bytes}
 
@@ -555,7 +729,7 @@ def main():
         return out
 
     variants = {}
-    if not sharded and not args.no_variants:
+    if not args.no_variants:
         del w
         torch.cuda.empty_cache()
         for vname in (VARIANT, "ctx4x8192_v151936_bf16", "edge_16384x131072_f32"):
@@ -565,7 +739,7 @@ def main():
     # Gradient of the KL w.r.t. the quant logits (row pass + reduction +
     # gradient pass writing fp32 [N, V]) on the same context.
     grad = None
-    if not sharded and not args.no_grad:
+    if not args.no_grad:
         gout = torch.empty_like(w.base)
         st.set_timing(True)
         for _ in range(3):
@@ -597,7 +771,7 @@ def main():
     # Top-128 compression of the base rows + KL against it (row pass +
     # reduction + top-k pass) on the same context.
     topk = None
-    if not sharded and not args.no_topk:
+    if not args.no_topk:
         for _ in range(2):
             st.run_topk(w.base, w.quant, w.token_ids, k=128)
             st.result()
@@ -625,7 +799,7 @@ def main():
     # End to end through the public host-memory entry point: pinned host
     # buffers in, the result struct out, copies inside the timed region.
     e2e = None
-    if not sharded and args.e2e_steps > 0:
+    if args.e2e_steps > 0:
         hb = w.base.cpu().pin_memory()
         hq = w.quant.cpu().pin_memory()
         ht = w.token_ids.cpu().pin_memory()
@@ -646,41 +820,37 @@ def main():
         del hb, hq, ht
 
     split_row = None
-    if not sharded and not args.no_split_row and args.rows is None:
+    if not args.no_split_row and args.rows is None:
         del w
         torch.cuda.empty_cache()
         split_row = split_row_latency(dev, stream, max(1, args.split_calls))
 
     cpu = cpu_mt = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if not args.no_cpu_baseline:
         cpu, cpu_mt = cpu_baseline(name)
 
-    if rank == 0:
-        line = {
-            "metric": METRIC, "value": value, "unit": "rows/s", "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": args.dtype, "data": "synthetic",
-            "config": {"workload": name, "rows_per_gpu": N, "vocab": V, "logit_dtype": args.dtype,
-                       "global_rows": total_rows,
-                       "parallelism": (f"rows sharded over {world} GPU(s) (NCCL group), records all-gathered"
-                                       if sharded else "one GPU, whole statistic per step (kld_stats_run)"),
-                       "l2": "inputs (9.96 GB per step per GPU) exceed the 126 MB L2; no flush"},
-            "roofline": roofline, "cpu_baseline": cpu, "cpu_baseline_all_cores": cpu_mt, "e2e": e2e,
-            "gpu_launches": 2 * args.steps, "clocks": clocks,
-            "gbs": in_bytes * world / (ms_per_step / 1000.0) / 1e9,
-            "mean_kld": res["mean_kld"], "top1_agree_pct": res["top1_agree_pct"], "ppl": res["ppl"],
-            "ppl_base": res["ppl_base"], "rms_dp": res["rms_dp"], "mean_dp": res["mean_dp"],
-            "variants": variants, "split_row": split_row, "grad": grad, "topk": topk,
-        }
-        if args.rows is not None or args.dtype != "f32" or args.split_calls != SPLIT_CALLS:
-            line["config"]["override"] = {"rows": N, "dtype": args.dtype,
-                                          "split_calls": args.split_calls,
-                                          "note": "profiling run, not the benchmark workload"}
-        print(json.dumps(line), flush=True)
+    line = {
+        "metric": METRIC, "value": value, "unit": "rows/s", "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": args.dtype, "data": "synthetic",
+        "config": {"workload": name, "rows_per_gpu": N, "vocab": V, "logit_dtype": args.dtype,
+                   "global_rows": total_rows,
+                   "parallelism": "one GPU, whole statistic per step (kld_stats_run)",
+                   "l2": "inputs (9.96 GB per step per GPU) exceed the 126 MB L2; no flush"},
+        "roofline": roofline, "cpu_baseline": cpu, "cpu_baseline_all_cores": cpu_mt, "e2e": e2e,
+        "gpu_launches": 2 * args.steps, "clocks": clocks,
+        "gbs": in_bytes / (ms_per_step / 1000.0) / 1e9,
+        "mean_kld": res["mean_kld"], "top1_agree_pct": res["top1_agree_pct"], "ppl": res["ppl"],
+        "ppl_base": res["ppl_base"], "rms_dp": res["rms_dp"], "mean_dp": res["mean_dp"],
+        "variants": variants, "split_row": split_row, "grad": grad, "topk": topk,
+    }
+    if args.rows is not None or args.dtype != "f32" or args.split_calls != SPLIT_CALLS:
+        line["config"]["override"] = {"rows": N, "dtype": args.dtype,
+                                      "split_calls": args.split_calls,
+                                      "note": "profiling run, not the benchmark workload"}
+    print(json.dumps(line), flush=True)
 
     st.close()
-    if sharded:
-        dist.destroy_process_group()
 
 
 if __name__ == "__main__":

@@ -235,6 +235,21 @@ kld_status_t kld_stats_run_host(kld_stats_t h, const void* base_host,
                                 int64_t V, kld_dtype_t dtype, void* stream);
 
 /*
+ * The row pass alone for logits in HOST memory: the chunked, overlapped
+ * copies of kld_stats_run_host, then per-row records for rows [0, N) in
+ * rows_out (device, N records, caller-owned; NULL = the handle's
+ * workspace), without the reduction. This is what one rank of a
+ * row-sharded run executes when its shard of logits lives in host memory,
+ * before the records are gathered and reduced (kld_stats_reduce).
+ * Asynchronous on `stream`; errors as kld_stats_run_host.
+ */
+kld_status_t kld_stats_run_rows_host(kld_stats_t h, const void* base_host,
+                                     const void* quant_host,
+                                     const int32_t* token_ids_host, int64_t N,
+                                     int64_t V, kld_dtype_t dtype,
+                                     kld_row_t* rows_out, void* stream);
+
+/*
  * Launch shape of the row pass for few rows (N <= SMs / 2), where whole-row
  * launches would leave most SMs idle and each row is split into parts
  * instead (see kld_plan):
@@ -398,12 +413,16 @@ kld_status_t kld_stats_read_probe(kld_stats_t h, const void* a, const void* b, i
                                   void* stream);
 
 /*
- * Kernel timing of the next runs: when enabled, kld_stats_run records CUDA
- * events around its row pass and its reduction; kld_stats_timing() returns
- * the last run's durations in milliseconds (waits for that run). For a run
- * whose row pass reduced its own records (few split rows, see
- * kld_stats_run) the row-pass time includes the reduction and reduce_ms is
- * about zero.
+ * Kernel timing of the next runs: when enabled, kld_stats_run (and
+ * kld_stats_run_grad, kld_stats_run_topk) records CUDA events around its row
+ * pass and its reduction; kld_stats_timing() returns the last run's
+ * durations in milliseconds (waits for that run). A kld_stats_run_rows
+ * followed by kld_stats_reduce on the same stream is timed the same way:
+ * row_pass_ms covers the row pass, reduce_ms everything enqueued between
+ * the end of the row pass and the end of the reduction (in a row-sharded
+ * run, the record gather too). For a run whose row pass reduced its own
+ * records (few split rows, see kld_stats_run) the row-pass time includes
+ * the reduction and reduce_ms is about zero.
  */
 kld_status_t kld_stats_set_timing(kld_stats_t h, int enable);
 kld_status_t kld_stats_timing(kld_stats_t h, float* row_pass_ms,

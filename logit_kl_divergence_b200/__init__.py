@@ -229,6 +229,23 @@ class KLDStats:
                                           ctypes.c_void_p(_stream_ptr(stream, self.device)))
         _lib.check(st, "kld_stats_run_host")
 
+    def run_rows_host(self, base: torch.Tensor, quant: torch.Tensor, token_ids: torch.Tensor | None = None,
+                      out: torch.Tensor | None = None, stream=None):
+        """Row pass only, for host (preferably pinned) CPU tensors: chunked
+        copies overlapped with the row pass; records go to ``out`` ([N, 40]
+        uint8 on the device) or to the handle's workspace."""
+        _check_pair(base, quant, token_ids, False)
+        if base.is_cuda:
+            raise ValueError("run_rows_host takes CPU tensors")
+        if out is not None and (out.dtype != torch.uint8 or not out.is_cuda
+                                or out.numel() < base.shape[0] * ROW_RECORD_BYTES):
+            raise ValueError("out must be a CUDA uint8 tensor of N*40 bytes")
+        st = self._lib.kld_stats_run_rows_host(self._h, _ptr(base), _ptr(quant), _ptr(token_ids),
+                                               base.shape[0], base.shape[1], dtype_code(base), _ptr(out),
+                                               ctypes.c_void_p(_stream_ptr(stream, self.device)))
+        _lib.check(st, "kld_stats_run_rows_host")
+        return out
+
     def run_rows(self, base, quant, token_ids=None, out: torch.Tensor | None = None, stream=None):
         """Row pass only; records go to ``out`` ([N, 40] uint8 on the device)
         or to the handle's workspace."""

@@ -110,6 +110,7 @@ SIGNATURES = {
     "kld_stats_run_rows": (_ST, [_P, _P, _P, _P, _I64, _I64, _I32, _P, _P]),
     "kld_stats_reduce": (_ST, [_P, _P, _I64, _I32, _P]),
     "kld_stats_run_host": (_ST, [_P, _P, _P, _P, _I64, _I64, _I32, _P]),
+    "kld_stats_run_rows_host": (_ST, [_P, _P, _P, _P, _I64, _I64, _I32, _P, _P]),
     "kld_stats_set_timing": (_ST, [_P, _I32]),
     "kld_stats_set_split": (_ST, [_P, _I32]),
     "kld_stats_run_grad": (_ST, [_P, _P, _P, _P, _I64, _I64, _I32, _P, _I32, ctypes.c_double, _P]),

@@ -83,6 +83,7 @@ struct kld_stats_s {
   int64_t last_rows = 0;
   bool timing = false;
   bool timing_valid = false;
+  bool rows_pending = false;  // a timed kld_stats_run_rows awaits its reduction
   cudaEvent_t tev[4] = {nullptr, nullptr, nullptr, nullptr};
   // host path
   cudaStream_t copy_stream = nullptr;
@@ -281,14 +282,18 @@ kld_status_t kld_stats_run_rows(kld_stats_t h, const void* base, const void* qua
   DeviceGuard guard(h->device);
   if (!guard.ok()) return cuda_fail(cudaGetLastError(), "cudaSetDevice");
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  // Timed like kld_stats_run: the reduction that follows records the end.
+  h->timing_valid = h->timing;
+  h->rows_pending = h->timing;
+  h->grad_timing_valid = false;
+  if (h->timing) KLD_CUDA(cudaEventRecord(h->tev[0], s));
   KLD_CUDA(launch_rows(h, base, quant, token_ids, N, V, dtype, rows_out ? rows_out : h->rows, s));
+  if (h->timing) KLD_CUDA(cudaEventRecord(h->tev[1], s));
   if (!rows_out) {
     h->last_rows = N;
     h->last_stream = s;
     h->rows_written = true;
   }
-  h->timing_valid = false;
-  h->grad_timing_valid = false;
   return KLD_OK;
 }
 
@@ -300,7 +305,11 @@ kld_status_t kld_stats_reduce(kld_stats_t h, const kld_row_t* rows_dev, int64_t 
   if (rows_dev && (reinterpret_cast<uintptr_t>(rows_dev) & 7u)) return KLD_ERR_INVALID_ARG;
   DeviceGuard guard(h->device);
   if (!guard.ok()) return cuda_fail(cudaGetLastError(), "cudaSetDevice");
-  h->timing_valid = false;
+  // Timed only as the reduction that follows a timed kld_stats_run_rows
+  // (whose start and end events are recorded): then the end of this
+  // reduction completes the measurement.
+  h->timing_valid = h->timing_valid && h->rows_pending;
+  h->rows_pending = false;
   h->grad_timing_valid = false;
   return enqueue_reduce(h, rows_dev ? rows_dev : h->rows, N, has_nll ? 1 : 0,
                         static_cast<cudaStream_t>(stream));
@@ -317,6 +326,7 @@ kld_status_t kld_stats_run(kld_stats_t h, const void* base, const void* quant,
   if (!guard.ok()) return cuda_fail(cudaGetLastError(), "cudaSetDevice");
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   h->timing_valid = h->timing;
+  h->rows_pending = false;
   h->grad_timing_valid = false;
   if (h->timing) KLD_CUDA(cudaEventRecord(h->tev[0], s));
   // A split-row launch of few rows reduces its own records into the result
@@ -349,6 +359,7 @@ kld_status_t kld_stats_run_grad(kld_stats_t h, const void* base, const void* qua
   if (!guard.ok()) return cuda_fail(cudaGetLastError(), "cudaSetDevice");
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   h->timing_valid = h->timing;
+  h->rows_pending = false;
   h->grad_timing_valid = h->timing;
   if (h->timing) KLD_CUDA(cudaEventRecord(h->tev[0], s));
   KLD_CUDA(launch_rows(h, base, quant, token_ids, N, V, dtype, h->rows, s, h->aux));
@@ -377,6 +388,7 @@ kld_status_t kld_stats_run_partials(kld_stats_t h, const void* base, const void*
   if (!guard.ok()) return cuda_fail(cudaGetLastError(), "cudaSetDevice");
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   h->timing_valid = false;
+  h->rows_pending = false;
   h->grad_timing_valid = false;
   KLD_CUDA(kld::launch_rows(base, quant, token_ids, N, V, dtype, h->rows, h->derr, h->sm_count,
                             &h->split, nullptr, s, parts_out, col_offset));
@@ -393,6 +405,7 @@ kld_status_t kld_stats_merge_partials(kld_stats_t h, const void* parts, int G, i
   if (!guard.ok()) return cuda_fail(cudaGetLastError(), "cudaSetDevice");
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   h->timing_valid = false;
+  h->rows_pending = false;
   h->grad_timing_valid = false;
   KLD_CUDA(kld::launch_merge(parts, G, N, token_ids, V_total, h->rows, s));
   h->last_rows = N;
@@ -416,6 +429,7 @@ kld_status_t kld_stats_run_topk(kld_stats_t h, const void* base, const void* qua
   if (!guard.ok()) return cuda_fail(cudaGetLastError(), "cudaSetDevice");
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   h->timing_valid = h->timing;
+  h->rows_pending = false;
   h->grad_timing_valid = h->timing;
   if (h->timing) KLD_CUDA(cudaEventRecord(h->tev[0], s));
   KLD_CUDA(launch_rows(h, base, quant, token_ids, N, V, dtype, h->rows, s, h->aux));
@@ -526,6 +540,7 @@ kld_status_t kld_stats_set_timing(kld_stats_t h, int enable) {
   if (!h) return KLD_ERR_INVALID_ARG;
   h->timing = enable != 0;
   h->timing_valid = false;
+  h->rows_pending = false;
   h->grad_timing_valid = false;
   return KLD_OK;
 }
@@ -541,17 +556,16 @@ kld_status_t kld_stats_timing(kld_stats_t h, float* row_pass_ms, float* reduce_m
   return KLD_OK;
 }
 
-kld_status_t kld_stats_run_host(kld_stats_t h, const void* base_host, const void* quant_host,
-                                const int32_t* token_ids_host, int64_t N, int64_t V,
-                                kld_dtype_t dtype, void* stream) {
-  if (!h) return KLD_ERR_INVALID_ARG;
-  kld_status_t st = check_inputs(base_host, quant_host, token_ids_host, N, V, dtype, false);
-  if (st != KLD_OK) return st;
-  if (N > h->max_rows) return KLD_ERR_INVALID_ARG;
-  DeviceGuard guard(h->device);
-  if (!guard.ok()) return cuda_fail(cudaGetLastError(), "cudaSetDevice");
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
+}  // extern "C"
 
+namespace {
+
+// Host-memory row pass: rows [0, N) copied to the device in chunks on the
+// handle's copy stream (two staging buffers, so the copy of one chunk
+// overlaps the row pass of the previous one), records to rows_out[0, N).
+kld_status_t host_rows(kld_stats_t h, const void* base_host, const void* quant_host,
+                       const int32_t* token_ids_host, int64_t N, int64_t V, kld_dtype_t dtype,
+                       kld_row_t* rows_out, cudaStream_t s) {
   const size_t row_bytes = static_cast<size_t>(V) * static_cast<size_t>(kld::elem_bytes(dtype));
   int64_t chunk = static_cast<int64_t>(kStageTargetBytes / row_bytes);
   if (chunk < 1) chunk = 1;
@@ -581,6 +595,7 @@ kld_status_t kld_stats_run_host(kld_stats_t h, const void* base_host, const void
   for (int i = 0; i < 2; ++i) KLD_CUDA(cudaEventRecord(h->freed[i], s));
 
   h->timing_valid = false;
+  h->rows_pending = false;
   h->grad_timing_valid = false;
   const char* hb = static_cast<const char*>(base_host);
   const char* hq = static_cast<const char*>(quant_host);
@@ -604,13 +619,49 @@ kld_status_t kld_stats_run_host(kld_stats_t h, const void* base_host, const void
                                cudaMemcpyHostToDevice, h->copy_stream));
     KLD_CUDA(cudaEventRecord(h->copied[b], h->copy_stream));
     KLD_CUDA(cudaStreamWaitEvent(s, h->copied[b], 0));
-    KLD_CUDA(launch_rows(h, sb, sq, token_ids_host ? stok : nullptr, n, V, dtype, h->rows + r0, s));
+    KLD_CUDA(launch_rows(h, sb, sq, token_ids_host ? stok : nullptr, n, V, dtype, rows_out + r0,
+                         s));
     KLD_CUDA(cudaEventRecord(h->freed[b], s));
   }
-  h->last_rows = N;
-  h->last_stream = s;
-  h->rows_written = true;
+  if (rows_out == h->rows) {
+    h->last_rows = N;
+    h->last_stream = s;
+    h->rows_written = true;
+  }
+  return KLD_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+kld_status_t kld_stats_run_host(kld_stats_t h, const void* base_host, const void* quant_host,
+                                const int32_t* token_ids_host, int64_t N, int64_t V,
+                                kld_dtype_t dtype, void* stream) {
+  if (!h) return KLD_ERR_INVALID_ARG;
+  kld_status_t st = check_inputs(base_host, quant_host, token_ids_host, N, V, dtype, false);
+  if (st != KLD_OK) return st;
+  if (N > h->max_rows) return KLD_ERR_INVALID_ARG;
+  DeviceGuard guard(h->device);
+  if (!guard.ok()) return cuda_fail(cudaGetLastError(), "cudaSetDevice");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  st = host_rows(h, base_host, quant_host, token_ids_host, N, V, dtype, h->rows, s);
+  if (st != KLD_OK) return st;
   return enqueue_reduce(h, h->rows, N, token_ids_host != nullptr, s);
+}
+
+kld_status_t kld_stats_run_rows_host(kld_stats_t h, const void* base_host, const void* quant_host,
+                                     const int32_t* token_ids_host, int64_t N, int64_t V,
+                                     kld_dtype_t dtype, kld_row_t* rows_out, void* stream) {
+  if (!h) return KLD_ERR_INVALID_ARG;
+  kld_status_t st = check_inputs(base_host, quant_host, token_ids_host, N, V, dtype, false);
+  if (st != KLD_OK) return st;
+  if (!rows_out && N > h->max_rows) return KLD_ERR_INVALID_ARG;
+  if (rows_out && (reinterpret_cast<uintptr_t>(rows_out) & 7u)) return KLD_ERR_INVALID_ARG;
+  DeviceGuard guard(h->device);
+  if (!guard.ok()) return cuda_fail(cudaGetLastError(), "cudaSetDevice");
+  return host_rows(h, base_host, quant_host, token_ids_host, N, V, dtype,
+                   rows_out ? rows_out : h->rows, static_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"

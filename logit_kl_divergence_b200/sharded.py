@@ -110,30 +110,77 @@ class ShardedKLDStats:
         self.max_rows_per_rank = int(max_rows_per_rank)
         self._records = None
 
-    def run(self, base: torch.Tensor, quant: torch.Tensor, token_ids: torch.Tensor | None = None) -> dict:
+    def run(self, base: torch.Tensor, quant: torch.Tensor, token_ids: torch.Tensor | None = None,
+            counts: list[int] | None = None) -> dict:
         """Collective. Every rank passes its own [n_r, V] rows (same V, dtype
         and token-id presence on every rank); returns the statistics of all
         ranks' rows. The ranks together must hold at least one row: with
-        none, every rank raises ValueError after the same collective steps."""
+        none, every rank raises ValueError after the same collective steps.
+
+        counts: every rank's row count in rank order, when the caller knows
+        them (equal shards, say; the same list on every rank). The step then
+        waits on the host once, for the result, instead of also waiting for
+        the exchange of row counts before it can enqueue the gather: each
+        rank's status travels in a collective enqueued with the gather and is
+        read after the result, so a failed rank still makes every rank raise
+        ShardFailure (the statistics of that step are discarded)."""
+        return self._run(base, quant, token_ids, base.device, host=False, counts=counts)
+
+    def run_host(self, base: torch.Tensor, quant: torch.Tensor, token_ids: torch.Tensor | None = None,
+                 device=None, counts: list[int] | None = None) -> dict:
+        """As :meth:`run` for a shard held in host memory (pinned for full
+        copy bandwidth): the library copies it to `device` (the handle's
+        GPU by default) in chunks overlapped with the row pass."""
+        if device is None:
+            device = getattr(self.stats, "device", base.device)
+        return self._run(base, quant, token_ids, torch.device(device), host=True, counts=counts)
+
+    def _run(self, base, quant, token_ids, device, host: bool, counts=None) -> dict:
         n = base.shape[0]
         if n > self.max_rows_per_rank:
             raise ValueError("more rows than max_rows_per_rank")
-        if self._records is None or self._records.device != base.device:
+        world = dist.get_world_size(self.group)
+        if counts is not None:
+            counts = [int(c) for c in counts]
+            if len(counts) != world or counts[dist.get_rank(self.group)] != n or min(counts) < 0:
+                raise ValueError("counts must list every rank's row count, this rank's included")
+        if self._records is None or self._records.device != device:
             self._records = torch.empty((self.max_rows_per_rank, ROW_RECORD_BYTES), dtype=torch.uint8,
-                                        device=base.device)
+                                        device=device)
         records = self._records[:n]
         err = None
         if n > 0:  # an uneven split can leave a rank without rows; it still gathers and reduces
             try:
-                self.stats.run_rows(base, quant, token_ids, out=records)
+                if host:
+                    self.stats.run_rows_host(base, quant, token_ids, out=records)
+                else:
+                    self.stats.run_rows(base, quant, token_ids, out=records)
             except Exception as e:  # reported to every rank below
                 err = e
-        counts = _checked_counts(n, err, base.device, self.group)
+        if counts is None:
+            counts = _checked_counts(n, err, device, self.group)
+            statuses = None
+        else:
+            # the status exchange is enqueued, not waited for
+            mine = torch.tensor([-1 if err is not None else n], dtype=torch.int64, device=device)
+            statuses = [torch.zeros_like(mine) for _ in range(world)]
+            dist.all_gather(statuses, mine, group=self.group)
         if sum(counts) == 0:  # every rank sees the same counts: all raise together
             raise ValueError("sharded statistic over zero rows: every rank passed an empty shard")
         gathered = gather_records(records, self.group, counts=counts)
-        self.stats.reduce(gathered, gathered.shape[0], token_ids is not None)
-        return self.stats.result()
+        res = None
+        try:
+            self.stats.reduce(gathered, gathered.shape[0], token_ids is not None)
+            res = self.stats.result()
+        except Exception as e:
+            if statuses is None or err is None:
+                raise
+        if statuses is not None:
+            got = [int(t.item()) for t in statuses]
+            failed = [r for r, c in enumerate(got) if c < 0]
+            if failed:
+                raise ShardFailure(failed, err) from err
+        return res
 
     def close(self):
         close = getattr(self.stats, "close", None)

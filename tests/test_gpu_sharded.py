@@ -39,12 +39,21 @@ def test_sharded_run_equals_single_handle_run(nccl_group):
     assert torch.equal(gather_records(rec), rec)
     assert torch.equal(gather_records(rec, counts=[5]), rec)
     sk = ShardedKLDStats(max_rows_per_rank=300, device=DEV)
+    sk.stats.set_timing(True)
     a = sk.run(w.base, w.quant, w.token_ids)
+    # the row pass and the gather + reduction of a sharded step are timed
+    # through the handle (kld_stats_run_rows then kld_stats_reduce)
+    row_ms, red_ms = sk.stats.timing()
+    assert 0.0 < row_ms < 100.0 and 0.0 < red_ms < 100.0
+    # the same shard from pinned host memory (kld_stats_run_rows_host)
+    hb, hq, ht = (t.cpu().pin_memory() for t in (w.base, w.quant, w.token_ids))
+    c = sk.run_host(hb, hq, ht)
     sk.close()
     st = KLDStats(max_rows=300, device=DEV)
     st.run(w.base, w.quant, w.token_ids)
     b = st.result()
     st.close()
-    for k in b:
-        x, y = a[k], b[k]
-        assert x == y or (isinstance(x, float) and math.isnan(x) and math.isnan(y)), k
+    for res in (a, c):
+        for k in b:
+            x, y = res[k], b[k]
+            assert x == y or (isinstance(x, float) and math.isnan(x) and math.isnan(y)), k

@@ -195,6 +195,22 @@ def _fail_worker(rank, world, port, mode, errq):
             res = sk.run(b, q, t)
             _, full = oracle.run(w.base, w.quant, w.token_ids, oracle.F32)
             _same(res, full)
+        elif mode == "status_counts":
+            # the same with the row counts given by the caller: the status
+            # travels in a collective enqueued with the gather and is read
+            # after the result; every rank still raises, and the next step
+            # on the same group is normal
+            counts = [b - a for a, b in (shard_bounds(24, world, r) for r in range(world))]
+            fails = [1] if rank == 0 else []
+            sk = ShardedKLDStats(max_rows_per_rank=hi - lo, stats=FailingStats(oracle.F32, fails))
+            _, full = oracle.run(w.base, w.quant, w.token_ids, oracle.F32)
+            _same(sk.run(b, q, t, counts=counts), full)
+            with pytest.raises(ShardFailure) as ei:
+                sk.run(b, q, t, counts=counts)
+            assert ei.value.ranks == [0]
+            _same(sk.run(b, q, t, counts=counts), full)
+            with pytest.raises(ValueError, match="counts"):
+                sk.run(b, q, t, counts=counts[::-1] if len(set(counts)) > 1 else [c + 1 for c in counts])
         elif mode == "vocab":
             fails = [0] if rank == 0 else []
             vs = VocabShardedKLDStats(5, stats=SliceStats(rank, fails))
@@ -240,7 +256,8 @@ def _fail_worker(rank, world, port, mode, errq):
         raise
 
 
-@pytest.mark.parametrize("world,mode", [(2, "status"), (3, "status"), (2, "vocab"), (3, "vocab"),
+@pytest.mark.parametrize("world,mode", [(2, "status"), (3, "status"), (2, "status_counts"),
+                                        (3, "status_counts"), (2, "vocab"), (3, "vocab"),
                                         (2, "zero"), (2, "exit")])
 def test_rank_failure_is_seen_by_every_rank(world, mode):
     ctx = mp.get_context("spawn")
