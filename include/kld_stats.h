@@ -153,12 +153,10 @@ kld_status_t kld_stats_create(kld_stats_t* out, int64_t max_rows, int device);
 void kld_stats_destroy(kld_stats_t h);
 
 /*
- * The whole statistic for rows [0, N): the fused row pass, then the
- * fixed-order reduction and exact percentile selection, which writes the
- * result straight into the handle's pinned host buffer (read it with
- * kld_stats_result). When the row pass splits few rows (N <= 32) over
- * many CTAs, the CTA that finishes the last row performs the reduction
- * itself, in the same arithmetic order, and no reduction kernel follows.
+ * The whole statistic for rows [0, N) in one kernel: the fused row pass,
+ * whose last CTA to finish then performs the fixed-order reduction and the
+ * exact percentile selection and writes the result straight into the
+ * handle's pinned host buffer (read it with kld_stats_result).
  * token_ids (device, int32[N]) may be NULL: no NLL/PPL.
  * 1 <= N <= max_rows, 1 <= V <= 2^31-1. Asynchronous.
  */
@@ -250,15 +248,16 @@ kld_status_t kld_stats_run_rows_host(kld_stats_t h, const void* base_host,
                                      kld_row_t* rows_out, void* stream);
 
 /*
- * Launch shape of the row pass for few rows (N <= SMs / 2), where whole-row
- * launches would leave most SMs idle and each row is split into parts
- * instead (see kld_plan):
- *   -1: never split (one CTA per row at any N);
+ * How the row pass splits rows (see kld_plan):
+ *   -1: never split: whole rows round robin at any N (the last partial wave
+ *       may leave SMs idle);
  *    0: the library default (currently 1);
- *    1: split over independent CTAs, merged through global memory;
- *    2, 4, 8: split over thread-block clusters of up to that many CTAs,
- *       merged first through distributed shared memory, then across the
- *       row's clusters through global memory.
+ *    1: whole rows, with the rows of a last partial wave (all rows when
+ *       N < SMs) split over plain CTAs by balanced chunk ranges, merged
+ *       through global memory;
+ *    2, 4, 8: as 1, but few rows (N <= SMs / 2) are split over thread-block
+ *       clusters of up to that many CTAs, merged first through distributed
+ *       shared memory, then across the row's clusters through global memory.
  * Results agree within rounding whatever the shape. Measured on B200 with
  * V = 262144 fp32 rows, plain CTAs were as fast as or up to ~10% faster than
  * clusters, hence the default. Other values: KLD_ERR_INVALID_ARG.
@@ -430,18 +429,18 @@ kld_status_t kld_stats_timing(kld_stats_t h, float* row_pass_ms,
 
 /*
  * Launch plan of the row pass for (N, V, dtype) on a device with sm_count
- * SMs, for the default split setting (kld_stats_set_split): variant 0 =
- * whole rows (one persistent CTA per SM, each taking rows r, r + grid, ...);
- * variant 1 = split rows, used when N <= sm_count / 2 so that few rows still
- * occupy the GPU: each row's 512-element chunks are divided among
- * ctas_per_row CTAs, in groups (thread-block clusters when cluster_ctas > 1,
- * whose partial sums meet in the cluster leader's shared memory) that meet
- * through a small global scratch and a per-row arrival counter; all of a
- * launch's CTAs fit on the device at once. Also: threads per CTA, dynamic
- * shared memory bytes, stage bytes per operand, stages. Pure host logic;
- * enqueues nothing. With clusters the launch may use fewer CTAs per row when
- * the device holds fewer clusters at once than sm_count / cluster_ctas (the
- * count comes from cudaOccupancyMaxActiveClusters).
+ * SMs, for the default split setting (kld_stats_set_split). One persistent
+ * CTA per SM takes whole rows round robin (rows r, r + grid, ...) for
+ * whole_rounds rounds; the tail_rows rows that would leave most SMs idle in
+ * a last partial wave (all N rows when N < sm_count) are instead split over
+ * tail_ctas CTAs, each taking a balanced, contiguous range of the tail's
+ * 512-element chunks (at most two rows' worth); a row's parts meet through a
+ * small global scratch and a per-row arrival counter. variant: 0 = whole
+ * rows only, 1 = few rows split over thread-block clusters (only when asked
+ * for with kld_stats_set_split), 2 = whole rounds plus a split tail.
+ * ctas_per_row: the most CTAs any row is split over. Also: threads per CTA,
+ * dynamic shared memory bytes, stage bytes per operand, stages. Pure host
+ * logic; enqueues nothing.
  */
 typedef struct {
   int32_t variant;
@@ -452,6 +451,10 @@ typedef struct {
   int32_t stage_bytes;
   int32_t stages;
   int32_t cluster_ctas;
+  int32_t whole_rounds;
+  int32_t tail_rows;
+  int32_t tail_ctas;
+  int32_t reserved;
 } kld_plan_t;
 
 kld_status_t kld_plan(int64_t N, int64_t V, kld_dtype_t dtype, int sm_count,

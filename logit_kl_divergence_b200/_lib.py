@@ -86,6 +86,10 @@ class Plan(ctypes.Structure):
         ("stage_bytes", ctypes.c_int32),
         ("stages", ctypes.c_int32),
         ("cluster_ctas", ctypes.c_int32),
+        ("whole_rounds", ctypes.c_int32),
+        ("tail_rows", ctypes.c_int32),
+        ("tail_ctas", ctypes.c_int32),
+        ("reserved", ctypes.c_int32),
     ]
 
 

@@ -71,7 +71,7 @@ struct kld_stats_s {
   int32_t* soa_amax_q = nullptr;
   cudaStream_t last_stream = nullptr;  // stream of the last run that wrote `rows`
   bool rows_written = false;
-  void* split_mem = nullptr;  // split-row scratch: partials, then tickets
+  void* split_mem = nullptr;  // split-row scratch (kld::SplitScratch)
   kld::RowAux* aux = nullptr;  // per-row normalisers for the gradient and top-k passes
   bool grad_timing_valid = false;
   kld::SplitScratch split = {nullptr, nullptr, 0, kld::kDefaultClusterCtas};
@@ -129,6 +129,29 @@ kld_status_t enqueue_reduce(kld_stats_t h, const kld_row_t* rows, int64_t N, int
   return KLD_OK;
 }
 
+// The row pass, then the reduction (in the row pass itself for few split
+// rows), each timed when timing is on. aux: per-row normalisers for a second
+// pass (nullable).
+kld_status_t run_statistic(kld_stats_t h, const void* base, const void* quant, const int32_t* tok,
+                           int64_t N, int64_t V, kld_dtype_t dtype, cudaStream_t s,
+                           kld::RowAux* aux) {
+  h->timing_valid = h->timing;
+  h->rows_pending = false;
+  if (h->timing) KLD_CUDA(cudaEventRecord(h->tev[0], s));
+  bool reduced = false;
+  KLD_CUDA(kld::launch_rows(base, quant, tok, N, V, dtype, h->rows, h->derr, h->sm_count,
+                            &h->split, aux, s, nullptr, 0, h->hres_dev, &reduced));
+  if (h->timing) KLD_CUDA(cudaEventRecord(h->tev[1], s));
+  h->last_rows = N;
+  h->last_stream = s;
+  h->rows_written = true;
+  if (!reduced) return enqueue_reduce(h, h->rows, N, tok != nullptr, s);
+  if (h->timing) KLD_CUDA(cudaEventRecord(h->tev[2], s));
+  KLD_CUDA(cudaEventRecord(h->done, s));
+  h->has_result = true;
+  return KLD_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -159,11 +182,14 @@ kld_status_t kld_plan(int64_t N, int64_t V, kld_dtype_t dtype, int sm_count, kld
   if (!valid_dtype(dtype)) return KLD_ERR_DTYPE;
   if (N < 1 || V < 1 || V > INT32_MAX || sm_count < 1) return KLD_ERR_INVALID_ARG;
   std::memset(out, 0, sizeof(*out));
-  const kld::RowPlan pl = kld::plan_rows(N, sm_count, nullptr, kld::kDefaultClusterCtas);
-  out->variant = pl.parts_per_row > 1 ? 1 : 0;
+  const kld::RowPlan pl = kld::plan_rows(N, V, sm_count, nullptr, kld::kDefaultClusterCtas);
+  out->variant = pl.cluster_ctas > 1 ? 1 : (pl.tail_rows > 0 ? 2 : 0);
   out->grid = pl.grid;
   out->ctas_per_row = pl.parts_per_row;
   out->cluster_ctas = pl.cluster_ctas;
+  out->whole_rounds = pl.whole;
+  out->tail_rows = pl.tail_rows;
+  out->tail_ctas = pl.tail_ctas;
   out->threads = kld::kRowThreads;
   out->smem_bytes = kld::kRowSmemBytes;
   out->stage_bytes = kld::kStageBytes;
@@ -215,11 +241,12 @@ kld_status_t kld_stats_create(kld_stats_t* out, int64_t max_rows, int device) {
     if ((err = cudaMemset(h->derr, 0, sizeof(uint32_t))) != cudaSuccess) {
       st = cuda_fail(err, "cudaMemset"); break; }
     {
-      // Split rows: at most one partial per SM-sized cluster slot and one
-      // arrival counter per row (rows <= SMs / 2), counters zeroed once;
-      // each row's last arriver puts its counter back to zero.
-      const size_t pbytes = static_cast<size_t>(sms) * kld::kSplitPartBytes;
-      const size_t tbytes = static_cast<size_t>(sms) * sizeof(unsigned);
+      // Split-row scratch (see kld::SplitScratch): partial slots and a
+      // ticket for each of up to SMs split rows, plus the few-row launch
+      // counter, all zeroed once here (each launch leaves them zero).
+      auto up = [](size_t b) { return (b + 255) & ~static_cast<size_t>(255); };
+      const size_t pbytes = up(static_cast<size_t>(sms) * kld::kPartSlotsPerRow * kld::kSplitPartBytes);
+      const size_t tbytes = up(static_cast<size_t>(sms + 1) * sizeof(unsigned));
       if ((err = cudaMalloc(&h->split_mem, pbytes + tbytes)) != cudaSuccess) {
         st = cuda_fail(err, "cudaMalloc(split scratch)"); break; }
       if ((err = cudaMemset(h->split_mem, 0, pbytes + tbytes)) != cudaSuccess) {
@@ -324,25 +351,9 @@ kld_status_t kld_stats_run(kld_stats_t h, const void* base, const void* quant,
   if (N > h->max_rows) return KLD_ERR_INVALID_ARG;
   DeviceGuard guard(h->device);
   if (!guard.ok()) return cuda_fail(cudaGetLastError(), "cudaSetDevice");
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  h->timing_valid = h->timing;
-  h->rows_pending = false;
   h->grad_timing_valid = false;
-  if (h->timing) KLD_CUDA(cudaEventRecord(h->tev[0], s));
-  // A split-row launch of few rows reduces its own records into the result
-  // buffer; otherwise the reduction kernel follows.
-  bool reduced = false;
-  KLD_CUDA(kld::launch_rows(base, quant, token_ids, N, V, dtype, h->rows, h->derr, h->sm_count,
-                            &h->split, nullptr, s, nullptr, 0, h->hres_dev, &reduced));
-  if (h->timing) KLD_CUDA(cudaEventRecord(h->tev[1], s));
-  h->last_rows = N;
-  h->last_stream = s;
-  h->rows_written = true;
-  if (!reduced) return enqueue_reduce(h, h->rows, N, token_ids != nullptr, s);
-  if (h->timing) KLD_CUDA(cudaEventRecord(h->tev[2], s));
-  KLD_CUDA(cudaEventRecord(h->done, s));
-  h->has_result = true;
-  return KLD_OK;
+  return run_statistic(h, base, quant, token_ids, N, V, dtype, static_cast<cudaStream_t>(stream),
+                       nullptr);
 }
 
 kld_status_t kld_stats_run_grad(kld_stats_t h, const void* base, const void* quant,
@@ -358,16 +369,8 @@ kld_status_t kld_stats_run_grad(kld_stats_t h, const void* base, const void* qua
   DeviceGuard guard(h->device);
   if (!guard.ok()) return cuda_fail(cudaGetLastError(), "cudaSetDevice");
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  h->timing_valid = h->timing;
-  h->rows_pending = false;
   h->grad_timing_valid = h->timing;
-  if (h->timing) KLD_CUDA(cudaEventRecord(h->tev[0], s));
-  KLD_CUDA(launch_rows(h, base, quant, token_ids, N, V, dtype, h->rows, s, h->aux));
-  if (h->timing) KLD_CUDA(cudaEventRecord(h->tev[1], s));
-  h->last_rows = N;
-  h->last_stream = s;
-  h->rows_written = true;
-  st = enqueue_reduce(h, h->rows, N, token_ids != nullptr, s);
+  st = run_statistic(h, base, quant, token_ids, N, V, dtype, s, h->aux);
   if (st != KLD_OK) return st;
   KLD_CUDA(kld::launch_grad(base, quant, h->aux, N, V, dtype, grad, grad_dtype,
                             static_cast<float>(scale), h->sm_count, s));
@@ -428,16 +431,8 @@ kld_status_t kld_stats_run_topk(kld_stats_t h, const void* base, const void* qua
   DeviceGuard guard(h->device);
   if (!guard.ok()) return cuda_fail(cudaGetLastError(), "cudaSetDevice");
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  h->timing_valid = h->timing;
-  h->rows_pending = false;
   h->grad_timing_valid = h->timing;
-  if (h->timing) KLD_CUDA(cudaEventRecord(h->tev[0], s));
-  KLD_CUDA(launch_rows(h, base, quant, token_ids, N, V, dtype, h->rows, s, h->aux));
-  if (h->timing) KLD_CUDA(cudaEventRecord(h->tev[1], s));
-  h->last_rows = N;
-  h->last_stream = s;
-  h->rows_written = true;
-  st = enqueue_reduce(h, h->rows, N, token_ids != nullptr, s);
+  st = run_statistic(h, base, quant, token_ids, N, V, dtype, s, h->aux);
   if (st != KLD_OK) return st;
   KLD_CUDA(kld::launch_topk(base, quant, h->aux, N, V, dtype, k, idx_out, logp_out, rest_out,
                             kl_out, h->sm_count, s));

@@ -1,11 +1,11 @@
 // kld_finish.cuh -- the last steps of the statistic, shared by the reduction
 // kernel and the row kernel's few-row path: order-preserving keys of the
 // per-row KL values, the type-7 interpolation between two order statistics,
-// a one-warp sort, and the assembly of kld_result_t from the fixed-order
-// sums and the selected order statistics ("Qwen3.6 27B Quantization
-// Benchmark", "Raw benchmark data" table: Mean KLD, Same top p (%), Mean
-// PPL(Q); the percentiles are order statistics of the same per-row values).
-// Device code only; included by .cu files of this library.
+// a one-warp sort, fixed-order sums, the exact MSB radix selection of the
+// order statistics, and the assembly of kld_result_t ("Qwen3.6 27B
+// Quantization Benchmark", "Raw benchmark data" table: Mean KLD, Same top p
+// (%), Mean PPL(Q); the percentiles are order statistics of the same per-row
+// values). Device code only; included by .cu files of this library.
 #pragma once
 
 #include <stdint.h>
@@ -159,6 +159,204 @@ __device__ __forceinline__ Sums zero_sums() {
   s.n_valid = s.agree = s.n_nll = s.n_flag = 0;
   s.flags_or = 0u;
   return s;
+}
+
+
+// ------------------------------------------------------------- selection
+
+constexpr int kAhead = 4;       // keys each thread loads before using them
+constexpr int kDigitBits = 11;  // radix digit of the selection
+constexpr int kBins = 1 << kDigitBits;
+constexpr int kSmall = 32;      // a group this small is finished by one warp
+
+// Selection state in shared memory: groups of targets whose keys share the
+// digits decided so far.
+struct SelectShared {
+  unsigned long long gprefix[kTargets];
+  unsigned long long tnext[kTargets];  // a target's prefix after this level
+  unsigned long long trank[kTargets];  // its rank among its group's keys
+  unsigned long long tval[kTargets];   // its key, once found
+  unsigned int gcount[kTargets];
+  unsigned int gfill[kTargets];
+  unsigned int tcount[kTargets];  // size of a target's group after this level
+  int tgroup[kTargets];           // -1 once found
+  int ngroups;
+  unsigned int hist[kTargets][kBins];
+  unsigned long long gbuf[kTargets][kSmall];
+};
+
+// Exact order statistics by an MSB-first radix select with 11-bit digits,
+// run by all nt threads of the CTA from `decided` known leading bits on.
+// On entry (visible to all threads): ngroups groups with prefix gprefix[g]
+// (the decided bits) and key count gcount[g]; every open target t has
+// tgroup[t] >= 0 and its rank trank[t] among its group's keys; found targets
+// have tgroup[t] = -1. src.at(i), i < n_keys, gives the keys (keys outside
+// every group are ignored). Per level: one shared histogram per group, a warp
+// per target finds its digit and residual rank, and warp 0 regroups the
+// targets by their new prefix; a group of at most kSmall keys is gathered and
+// sorted by one warp, which ends its targets; a group still open after all 64
+// bits holds equal keys. On return tval[t] holds every target's key.
+// Where select_levels reads its keys: an array of keys (shared or global
+// memory, read through L2), or the KL values of records (key 0 for excluded
+// rows).
+struct KeySource {
+  const unsigned long long* keys;  // nullable
+  const kld_row_t* rows;           // used when keys is null
+  bool global;                     // keys in global memory written by this kernel
+  __device__ __forceinline__ unsigned long long at(int64_t i) const {
+    if (keys != nullptr) return global ? __ldcg(keys + i) : keys[i];
+    return (rows[i].flags & kExcluded) ? 0ull : order_key(rows[i].kld);
+  }
+};
+
+__device__ __forceinline__ void select_levels(SelectShared& sh, KeySource src, int64_t n_keys,
+                                              int decided, int nt) {
+  const int tid = threadIdx.x;
+  const int lane = tid & 31, warp = tid >> 5;
+  const int nw = nt >> 5;
+  for (;;) {
+    bool open = false;
+    for (int t = 0; t < kTargets; ++t) open |= sh.tgroup[t] >= 0;
+    if (!open) break;
+    const int ng = sh.ngroups;
+    if (decided >= 64) {
+      // every key of a remaining group equals its prefix
+      if (tid < kTargets && sh.tgroup[tid] >= 0) {
+        sh.tval[tid] = sh.gprefix[sh.tgroup[tid]];
+        sh.tgroup[tid] = -1;
+      }
+      __syncthreads();
+      break;
+    }
+    const int bits = 64 - decided < kDigitBits ? 64 - decided : kDigitBits;
+    const int shift = 64 - decided - bits;
+    const unsigned long long himask = decided == 0 ? 0ull : (~0ull << (64 - decided));
+    for (int i = tid; i < ng * kBins; i += nt)
+      if (sh.gcount[i / kBins] > static_cast<unsigned>(kSmall)) (&sh.hist[0][0])[i] = 0u;
+    if (tid < ng) sh.gfill[tid] = 0u;
+    __syncthreads();
+
+    // One pass over the keys: gather the keys of small groups, count the
+    // next digit of the keys of large ones.
+    for (int64_t base = 0; base < n_keys; base += static_cast<int64_t>(kAhead) * nt) {
+      unsigned long long kv[kAhead];
+      bool ok[kAhead];
+#pragma unroll
+      for (int u = 0; u < kAhead; ++u) {
+        const int64_t i = base + static_cast<int64_t>(u) * nt + tid;
+        ok[u] = i < n_keys;
+        kv[u] = ok[u] ? src.at(i) : 0ull;
+      }
+#pragma unroll
+      for (int u = 0; u < kAhead; ++u) {
+        int g = -1;
+        if (ok[u]) {
+          for (int h = 0; h < ng; ++h) {
+            if (((kv[u] ^ sh.gprefix[h]) & himask) == 0ull) {
+              g = h;
+              break;
+            }
+          }
+        }
+        const bool small = g >= 0 && sh.gcount[g] <= static_cast<unsigned>(kSmall);
+        if (small) {
+          const unsigned p = atomicAdd(&sh.gfill[g], 1u);
+          if (p < static_cast<unsigned>(kSmall)) sh.gbuf[g][p] = kv[u];
+        }
+        const int slot = (g >= 0 && !small)
+                             ? g * kBins + static_cast<int>((kv[u] >> shift) & (kBins - 1))
+                             : -1;
+        if (decided == 0) {
+          // first digit: few distinct bins, one atomic per bin and warp
+          const unsigned peers = __match_any_sync(0xffffffffu, slot);
+          if (slot >= 0 && lane == __ffs(peers) - 1)
+            atomicAdd(&(&sh.hist[0][0])[slot], static_cast<unsigned>(__popc(peers)));
+        } else if (slot >= 0) {
+          atomicAdd(&(&sh.hist[0][0])[slot], 1u);  // later digits spread out
+        }
+      }
+    }
+    __syncthreads();
+
+    // A warp per open target: finish a small group by sorting its keys, or
+    // find the target's digit in its group's histogram. Lane L sums bins
+    // [64L, 64L + 64) (rotated start: conflict-free), a warp scan finds the
+    // lane whose range holds the rank, and the warp scans those 64 bins.
+    for (int t = warp; t < kTargets; t += nw) {
+      const int g = sh.tgroup[t];
+      if (g < 0) continue;
+      const unsigned cnt = sh.gcount[g];
+      const unsigned long long r = sh.trank[t];
+      if (cnt <= static_cast<unsigned>(kSmall)) {
+        const unsigned long long key =
+            warp_sort(lane < static_cast<int>(cnt) ? sh.gbuf[g][lane] : ~0ull, lane);
+        const unsigned long long v = __shfl_sync(0xffffffffu, key, static_cast<int>(r & 31));
+        if (lane == 0) sh.tval[t] = v;
+        continue;
+      }
+      constexpr int kPer = kBins / 32;
+      const unsigned* hg = sh.hist[g];
+      unsigned long long part = 0;
+#pragma unroll 8
+      for (int b = 0; b < kPer; ++b) part += hg[lane * kPer + ((b + lane) & (kPer - 1))];
+      unsigned long long incl = part;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const unsigned long long v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += v;
+      }
+      const unsigned long long excl = incl - part;
+      const unsigned hit = __ballot_sync(0xffffffffu, r >= excl && r < incl);
+      const int owner = hit ? __ffs(hit) - 1 : 31;  // 31: unreachable for consistent counts
+      const unsigned long long before = __shfl_sync(0xffffffffu, excl, owner);
+      const unsigned c0 = hg[owner * kPer + lane], c1 = hg[owner * kPer + 32 + lane];
+      unsigned long long s0 = c0, s1 = c1;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const unsigned long long v0 = __shfl_up_sync(0xffffffffu, s0, o);
+        const unsigned long long v1 = __shfl_up_sync(0xffffffffu, s1, o);
+        if (lane >= o) {
+          s0 += v0;
+          s1 += v1;
+        }
+      }
+      s1 += __shfl_sync(0xffffffffu, s0, 31);
+      const unsigned long long rr = r - before;  // rank within the owner's 64 bins
+      const unsigned m0 = __ballot_sync(0xffffffffu, s0 > rr);
+      const unsigned m1 = __ballot_sync(0xffffffffu, s1 > rr);
+      const int j = m0 ? __ffs(m0) - 1 : 32 + (m1 ? __ffs(m1) - 1 : 31);
+      const unsigned long long incl_j = __shfl_sync(0xffffffffu, j < 32 ? s0 : s1, j & 31);
+      const unsigned cnt_j = __shfl_sync(0xffffffffu, j < 32 ? c0 : c1, j & 31);
+      if (lane == 0) {
+        const int bin = owner * kPer + j;
+        sh.tnext[t] = sh.gprefix[g] | (static_cast<unsigned long long>(bin) << shift);
+        sh.trank[t] = rr - (incl_j - cnt_j);
+        sh.tcount[t] = cnt_j;
+      }
+    }
+    __syncthreads();
+    if (warp == 0) {
+      // Targets of small groups are done; the others regroup by their new
+      // prefix (lane t = target t; groups numbered in lane order).
+      const int g0 = lane < kTargets ? sh.tgroup[lane] : -1;
+      const bool act = g0 >= 0 && sh.gcount[g0] > static_cast<unsigned>(kSmall);
+      const unsigned long long p = act ? sh.tnext[lane] : ~0ull;
+      const unsigned cnt = act ? sh.tcount[lane] : 0u;
+      const unsigned peers = __match_any_sync(0xffffffffu, p);
+      const int leader = __ffs(peers) - 1;
+      const unsigned leaders = __ballot_sync(0xffffffffu, act && lane == leader);
+      const int gid = __popc(leaders & ((1u << leader) - 1u));
+      __syncwarp();
+      if (act && lane == leader) {
+        sh.gprefix[gid] = p;
+        sh.gcount[gid] = cnt;
+      }
+      if (lane < kTargets) sh.tgroup[lane] = act ? gid : -1;
+      if (lane == 0) sh.ngroups = __popc(leaders);
+    }
+    decided += bits;
+    __syncthreads();
+  }
 }
 
 // The whole statistic of N <= 32 records by one warp, in the same

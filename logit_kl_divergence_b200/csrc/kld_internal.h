@@ -28,18 +28,19 @@ constexpr int kSlots = 4;
 // one row; their partials meet in the cluster leader's shared memory.
 constexpr int kMaxClusterCtas = 8;
 
-// Per-launch global scratch of split-row mode: one merged partial per
-// cluster (kSplitPartBytes) and one arrival ticket per row; `parts` holds
-// `capacity` partials and `tickets` `capacity` counters (a launch of N rows
-// uses tickets[0, N), and tickets[N] counts finished rows when the launch
-// reduces its own records). Tickets start at zero and are reset by the last
-// arriver.
+// Per-handle global scratch of split rows (parts of one row on several
+// CTAs): kPartSlotsPerRow 64-byte partials and one arrival ticket per split
+// row; a launch splits at most `capacity` rows (>= the SM count), and the
+// ticket after the last split row's counts a few-row launch's finished rows
+// (its in-pass reduction). Tickets start at zero and whoever finishes with
+// one puts it back.
 constexpr int kSplitPartBytes = 64;
+constexpr int kPartSlotsPerRow = 32;
 struct SplitScratch {
   void* parts;
   unsigned* tickets;
   int capacity;
-  int max_cluster_ctas;  // largest cluster the plan may use (1: plain CTAs)
+  int max_cluster_ctas;  // largest cluster the plan may use (1: plain CTAs; 0: never split)
 };
 // Cluster size split rows use unless the caller asks otherwise.
 constexpr int kDefaultClusterCtas = 1;
@@ -53,6 +54,13 @@ constexpr int kRowSmemBytes = kStages * 2 * kStageBytes + kRowCtrlBytes;
 constexpr int kReduceThreads = 1024;
 
 inline int elem_bytes(kld_dtype_t dt) { return dt == KLD_F32 ? 4 : 2; }
+
+// The row pass forms the log-ratio x = q - b + K of fp32 inputs in the order
+// that keeps it exact for rows offset by a large constant: when |K| >= this,
+// (q + K) - b or q - (b - K); below it, (q - b) + K (the order 16-bit
+// inputs always take, where q - b is exact). Passes that reuse the row
+// pass's sums form x the same way.
+constexpr float kShiftForm = 8.0f;
 
 // Per-row normalisers the row pass leaves for the gradient and top-k passes
 // (48 bytes; the first 16 are read as a float4 by the gradient pass).
@@ -70,15 +78,18 @@ static_assert(sizeof(RowAux) == 48, "RowAux layout");
 // Launchers (defined in the .cu files). They enqueue on `stream` and return
 // the launch error.
 // Row pass. With split == nullptr every CTA handles whole rows; otherwise
-// few-row launches spread each row over clusters of CTAs (see RowPlan).
+// the plan of plan_rows (whole-row rounds, then the last partial wave's rows
+// split over all CTAs; few rows over clusters when asked) using the split
+// scratch.
 // aux (nullable): per-row normalisers for the gradient and top-k passes.
 // part_out (nullable): vocabulary-slice mode, the row is columns
 // [col_offset, col_offset + V) of a wider vocabulary and each row's merged
 // 64-byte partial goes to part_out[r] instead of a record (see
-// launch_merge).
-// result_out (nullable): a split-row launch of at most kFusedReduceRows rows
-// then also reduces its records into *result_out (the launch's last
-// finaliser does it; no reduction kernel needed) and sets *reduced.
+// launch_merge); whole rows only.
+// result_out (nullable): a launch whose rows are all split (fewer rows than
+// SMs) and at most kFusedReduceRows of them also reduces its records into
+// *result_out (the launch's last finaliser does it; no reduction kernel
+// needed) and sets *reduced.
 constexpr int kFusedReduceRows = 32;
 cudaError_t launch_rows(const void* base, const void* quant,
                         const int32_t* token_ids, int64_t N, int64_t V,
@@ -94,18 +105,25 @@ constexpr int kPartialBytes = 64;
 cudaError_t launch_merge(const void* parts, int G, int64_t N, const int32_t* token_ids,
                          int64_t V_total, kld_row_t* rows, cudaStream_t stream);
 
-// Launch shape of the row pass: parts_per_row = 1 (whole rows, persistent
-// grid) or > 1 (split rows: grid = N * parts_per_row, clusters of
-// cluster_ctas CTAs, parts_per_row / cluster_ctas clusters per row).
+// Launch shape of the row pass.
+//   cluster_ctas > 1: few rows split over thread-block clusters: grid =
+//     N * parts_per_row CTAs, parts_per_row / cluster_ctas clusters per row.
+//   otherwise: `whole` rounds of whole rows (CTA b takes rows b + j * grid),
+//     then the tail_rows remaining rows split over tail_ctas CTAs by balanced
+//     ranges of their tail_chunks chunks (nchv per row); parts_per_row is
+//     the most CTAs any tail row is split over (1 without a tail).
 struct RowPlan {
   int grid, parts_per_row, cluster_ctas;
+  int whole, tail_rows, tail_ctas, nchv;
+  int64_t tail_chunks;
 };
 // fit[i]: clusters of 2^i CTAs the device holds at once (i = 0..3; <= 0:
-// unknown, estimated as sm_count >> i). Split rows only when N <= sm_count/2
-// and max_cluster_ctas >= 1: the cluster is the largest power of two <=
-// max_cluster_ctas that leaves one cluster per row in one wave, and each row
-// takes as many clusters (<= 32) as still fit in that wave.
-RowPlan plan_rows(int64_t N, int sm_count, const int fit[4], int max_cluster_ctas);
+// unknown, estimated as sm_count >> i). max_cluster_ctas: 0 = whole rows
+// only (grid = min(N, SMs), rows round robin); 1 = whole rounds plus a split
+// tail; 2, 4, 8: as 1, but N <= sm_count / 2 rows are split over clusters of
+// the largest power of two <= max_cluster_ctas that leaves one cluster per
+// row in one wave, each row taking as many clusters (<= 32) as still fit.
+RowPlan plan_rows(int64_t N, int64_t V, int sm_count, const int fit[4], int max_cluster_ctas);
 cudaError_t prepare_rows_kernels();  // per-device attribute setup
 
 // Gradient pass: grad[i][j] = scale * (softmax(q_i)_j - softmax(b_i)_j)

@@ -40,34 +40,18 @@
 namespace kld {
 namespace {
 
-using fin::interpolate;
-using fin::key_value;
 using fin::kExcluded;
 using fin::kTargets;
 using fin::order_key;
 using fin::warp_sort;
-constexpr int kAhead = 4;       // records each thread loads before using them
-constexpr int kDigitBits = 11;  // radix digit of the selection
-constexpr int kBins = 1 << kDigitBits;
-constexpr int kSmall = 32;      // a group this small is finished by one warp
+using fin::kAhead;
 constexpr int kKeyCap = 19968;  // keys kept in shared memory (N up to this)
 
 struct ReduceShared {
   double dsum[32][5];
   long long isum[32][4];
   unsigned int flags_or[32];
-  // selection state: groups of targets whose keys share the decided digits
-  unsigned long long gprefix[kTargets];
-  unsigned long long tnext[kTargets];  // a target's prefix after this level
-  unsigned long long trank[kTargets];  // its rank among its group's keys
-  unsigned long long tval[kTargets];   // its key, once found
-  unsigned int gcount[kTargets];
-  unsigned int gfill[kTargets];
-  unsigned int tcount[kTargets];  // size of a target's group after this level
-  int tgroup[kTargets];           // -1 once found
-  int ngroups;
-  unsigned int hist[kTargets][kBins];
-  unsigned long long gbuf[kTargets][kSmall];
+  fin::SelectShared sel;
 };
 constexpr size_t kReduceSmemMax = sizeof(ReduceShared) + sizeof(unsigned long long) * kKeyCap;
 static_assert(kReduceSmemMax <= 227 * 1024, "reduction shared memory");
@@ -82,7 +66,6 @@ __global__ void __launch_bounds__(kReduceThreads, 1)
   const int tid = threadIdx.x;
   const int lane = tid & 31, warp = tid >> 5;
   const int nt = static_cast<int>(blockDim.x);
-  const int nw = nt >> 5;
   // Launched as a programmatic dependent of the row pass: its launch may
   // overlap the row pass, the records are read only after it completed.
   asm volatile("griddepcontrol.wait;" ::: "memory");
@@ -194,20 +177,16 @@ __global__ void __launch_bounds__(kReduceThreads, 1)
   const long long nv = sh.isum[0][0];
 
   // ------------------------------------------------------------- selection
-  const double ps[3] = {0.5, 0.9, 0.99};
+  fin::SelectShared& sel = sh.sel;
+  if (tid < kTargets) {
+    sel.tval[tid] = 0ull;
+    sel.tgroup[tid] = -1;
+  }
+  __syncthreads();
   if (nv > 0) {
     if (tid < kTargets) {
-      long long k;
-      if (tid < 6) {
-        const double pos = ps[tid >> 1] * static_cast<double>(nv - 1);
-        k = static_cast<long long>(floor(pos)) + (tid & 1);
-        if (k > nv - 1) k = nv - 1;
-      } else {
-        k = nv - 1;
-      }
-      sh.trank[tid] = static_cast<unsigned long long>(k);
-      sh.tgroup[tid] = 0;
-      sh.tval[tid] = 0ull;
+      sel.trank[tid] = static_cast<unsigned long long>(fin::target_rank(tid, nv));
+      sel.tgroup[tid] = 0;
     }
     // Excluded rows have key 0, below every other key: they come first and
     // offset the ranks.
@@ -218,173 +197,25 @@ __global__ void __launch_bounds__(kReduceThreads, 1)
         const unsigned long long key = warp_sort(lane < N ? keys[lane] : ~0ull, lane);
         for (int t = 0; t < kTargets; ++t) {
           const unsigned long long v =
-              __shfl_sync(0xffffffffu, key, static_cast<int>(sh.trank[t] + (N - nv)));
+              __shfl_sync(0xffffffffu, key, static_cast<int>(sel.trank[t] + (N - nv)));
           if (lane == 0) {
-            sh.tval[t] = v;
-            sh.tgroup[t] = -1;
+            sel.tval[t] = v;
+            sel.tgroup[t] = -1;
           }
         }
       }
       __syncthreads();
     }
-    if (tid < kTargets) sh.trank[tid] += static_cast<unsigned long long>(N - nv);
+    if (tid < kTargets) sel.trank[tid] += static_cast<unsigned long long>(N - nv);
     if (tid == 0) {
-      sh.ngroups = 1;
-      sh.gprefix[0] = 0ull;
-      sh.gcount[0] = static_cast<unsigned int>(N);
+      sel.ngroups = 1;
+      sel.gprefix[0] = 0ull;
+      sel.gcount[0] = static_cast<unsigned int>(N);
     }
     __syncthreads();
-
-    for (int decided = 0;; ) {
-      bool open = false;
-      for (int t = 0; t < kTargets; ++t) open |= sh.tgroup[t] >= 0;
-      if (!open) break;
-      const int ng = sh.ngroups;
-      if (decided >= 64) {
-        // every key of a remaining group equals its prefix
-        if (tid < kTargets && sh.tgroup[tid] >= 0) {
-          sh.tval[tid] = sh.gprefix[sh.tgroup[tid]];
-          sh.tgroup[tid] = -1;
-        }
-        __syncthreads();
-        break;
-      }
-      const int bits = 64 - decided < kDigitBits ? 64 - decided : kDigitBits;
-      const int shift = 64 - decided - bits;
-      const unsigned long long himask = decided == 0 ? 0ull : (~0ull << (64 - decided));
-      for (int i = tid; i < ng * kBins; i += nt)
-        if (sh.gcount[i / kBins] > static_cast<unsigned>(kSmall)) (&sh.hist[0][0])[i] = 0u;
-      if (tid < ng) sh.gfill[tid] = 0u;
-      __syncthreads();
-
-      // One pass over the keys: gather the keys of small groups, count the
-      // next digit of the keys of large ones (warp-aggregated atomics).
-      for (int64_t base = 0; base < N; base += static_cast<int64_t>(kAhead) * nt) {
-        unsigned long long kv[kAhead];
-        bool ok[kAhead];
-#pragma unroll
-        for (int u = 0; u < kAhead; ++u) {
-          const int64_t i = base + static_cast<int64_t>(u) * nt + tid;
-          ok[u] = i < N;
-          kv[u] = 0ull;
-          if (ok[u]) {
-            if (in_smem) {
-              kv[u] = keys[i];
-            } else if (!(rows[i].flags & kExcluded)) {
-              kv[u] = order_key(rows[i].kld);
-            }
-          }
-        }
-#pragma unroll
-        for (int u = 0; u < kAhead; ++u) {
-          int g = -1;
-          if (ok[u]) {
-            for (int h = 0; h < ng; ++h) {
-              if (((kv[u] ^ sh.gprefix[h]) & himask) == 0ull) {
-                g = h;
-                break;
-              }
-            }
-          }
-          const bool small = g >= 0 && sh.gcount[g] <= static_cast<unsigned>(kSmall);
-          if (small) {
-            const unsigned p = atomicAdd(&sh.gfill[g], 1u);
-            if (p < static_cast<unsigned>(kSmall)) sh.gbuf[g][p] = kv[u];
-          }
-          const int slot = (g >= 0 && !small)
-                               ? g * kBins + static_cast<int>((kv[u] >> shift) & (kBins - 1))
-                               : -1;
-          if (decided == 0) {
-            // first digit: few distinct bins, one atomic per bin and warp
-            const unsigned peers = __match_any_sync(0xffffffffu, slot);
-            if (slot >= 0 && lane == __ffs(peers) - 1)
-              atomicAdd(&(&sh.hist[0][0])[slot], static_cast<unsigned>(__popc(peers)));
-          } else if (slot >= 0) {
-            atomicAdd(&(&sh.hist[0][0])[slot], 1u);  // later digits spread out
-          }
-        }
-      }
-      __syncthreads();
-
-      // A warp per open target: finish a small group by sorting its keys, or
-      // find the target's digit in its group's histogram. Lane L sums bins
-      // [64L, 64L + 64) (rotated start: conflict-free), a warp scan finds the
-      // lane whose range holds the rank, and the warp scans those 64 bins.
-      for (int t = warp; t < kTargets; t += nw) {
-        const int g = sh.tgroup[t];
-        if (g < 0) continue;
-        const unsigned cnt = sh.gcount[g];
-        const unsigned long long r = sh.trank[t];
-        if (cnt <= static_cast<unsigned>(kSmall)) {
-          const unsigned long long key =
-              warp_sort(lane < static_cast<int>(cnt) ? sh.gbuf[g][lane] : ~0ull, lane);
-          const unsigned long long v = __shfl_sync(0xffffffffu, key, static_cast<int>(r));
-          if (lane == 0) sh.tval[t] = v;
-          continue;
-        }
-        constexpr int kPer = kBins / 32;
-        const unsigned* hg = sh.hist[g];
-        unsigned long long part = 0;
-#pragma unroll 8
-        for (int b = 0; b < kPer; ++b) part += hg[lane * kPer + ((b + lane) & (kPer - 1))];
-        unsigned long long incl = part;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          const unsigned long long v = __shfl_up_sync(0xffffffffu, incl, o);
-          if (lane >= o) incl += v;
-        }
-        const unsigned long long excl = incl - part;
-        const unsigned hit = __ballot_sync(0xffffffffu, r >= excl && r < incl);
-        const int owner = hit ? __ffs(hit) - 1 : 31;  // 31: unreachable for consistent counts
-        const unsigned long long before = __shfl_sync(0xffffffffu, excl, owner);
-        const unsigned c0 = hg[owner * kPer + lane], c1 = hg[owner * kPer + 32 + lane];
-        unsigned long long s0 = c0, s1 = c1;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          const unsigned long long v0 = __shfl_up_sync(0xffffffffu, s0, o);
-          const unsigned long long v1 = __shfl_up_sync(0xffffffffu, s1, o);
-          if (lane >= o) {
-            s0 += v0;
-            s1 += v1;
-          }
-        }
-        s1 += __shfl_sync(0xffffffffu, s0, 31);
-        const unsigned long long rr = r - before;  // rank within the owner's 64 bins
-        const unsigned m0 = __ballot_sync(0xffffffffu, s0 > rr);
-        const unsigned m1 = __ballot_sync(0xffffffffu, s1 > rr);
-        const int j = m0 ? __ffs(m0) - 1 : 32 + (m1 ? __ffs(m1) - 1 : 31);
-        const unsigned long long incl_j = __shfl_sync(0xffffffffu, j < 32 ? s0 : s1, j & 31);
-        const unsigned cnt_j = __shfl_sync(0xffffffffu, j < 32 ? c0 : c1, j & 31);
-        if (lane == 0) {
-          const int bin = owner * kPer + j;
-          sh.tnext[t] = sh.gprefix[g] | (static_cast<unsigned long long>(bin) << shift);
-          sh.trank[t] = rr - (incl_j - cnt_j);
-          sh.tcount[t] = cnt_j;
-        }
-      }
-      __syncthreads();
-      if (warp == 0) {
-        // Targets of small groups are done; the others regroup by their new
-        // prefix (lane t = target t; groups numbered in lane order).
-        const int g0 = lane < kTargets ? sh.tgroup[lane] : -1;
-        const bool act = g0 >= 0 && sh.gcount[g0] > static_cast<unsigned>(kSmall);
-        const unsigned long long p = act ? sh.tnext[lane] : ~0ull;
-        const unsigned cnt = act ? sh.tcount[lane] : 0u;
-        const unsigned peers = __match_any_sync(0xffffffffu, p);
-        const int leader = __ffs(peers) - 1;
-        const unsigned leaders = __ballot_sync(0xffffffffu, act && lane == leader);
-        const int gid = __popc(leaders & ((1u << leader) - 1u));
-        __syncwarp();
-        if (act && lane == leader) {
-          sh.gprefix[gid] = p;
-          sh.gcount[gid] = cnt;
-        }
-        if (lane < kTargets) sh.tgroup[lane] = act ? gid : -1;
-        if (lane == 0) sh.ngroups = __popc(leaders);
-      }
-      decided += bits;
-      __syncthreads();
-    }
+    fin::select_levels(sel, in_smem ? fin::KeySource{keys, nullptr, false}
+                                    : fin::KeySource{nullptr, rows, false},
+                       N, 0, nt);
   }
 
   if (tid == 0) {
@@ -404,7 +235,7 @@ __global__ void __launch_bounds__(kReduceThreads, 1)
       de = *derr;
       *derr = 0u;
     }
-    *out = fin::make_result(N, s, sh.tval, has_nll, de);
+    *out = fin::make_result(N, s, sel.tval, has_nll, de);
   }
 }
 

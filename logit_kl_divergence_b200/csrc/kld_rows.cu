@@ -384,7 +384,19 @@ struct Ref {
   float Rb, Rq;  // integer frames floor(M*L) once M is finite, 0 before
   float K;       // log-ratio centre: (b - q) at the element that set Mb
   float T;       // Mb + kRaiseMargin: a chunk maximum above it moves the frame
+  int mode;      // order of the log-ratio's two roundings (see log_ratios)
 };
+
+// Order in which x = q - b + K is formed in fp32. For 16-bit inputs q - b is
+// exact, so (q - b) + K rounds once. For fp32 inputs q - b rounds to half an
+// ulp of |q - b|: rows whose logits are offset by a large constant (|K| >=
+// kShiftForm) would lose ~1e-5 there, so the operand as large as K is paired
+// with K first, which is then exact: (q + K) - b when |q| >= |b| at the
+// element that set K, q - (b - K) otherwise.
+__device__ __forceinline__ int ratio_form(float Mb, float K) {
+  if (!(fabsf(K) >= kShiftForm)) return 0;
+  return fabsf(Mb - K) >= fabsf(Mb) ? 1 : 2;
+}
 
 // Per-lane fp64 accumulators (see the file comment): S_b over all chunks;
 // Ap = sum e*x and C = sum e*phi over polynomial-path chunks; Ad = sum e*x,
@@ -476,18 +488,37 @@ __device__ __forceinline__ void poly_accumulate(const float* b, const f2* X, con
   a.C += static_cast<double>(sc0 + sc1);
 }
 
-// Log-ratios x = (q - b) + K of one step, in packed pairs (x = 0 for absent
-// elements), and the largest |x| of the lane (NaN if any x is NaN).
+// Log-ratios x = q - b + K of one step, in packed pairs (x = 0 for absent
+// elements), and the largest |x| of the lane (NaN if any x is NaN). `form`
+// (warp-uniform) picks the order of the roundings (ratio_form).
 template <int PE>
 __device__ __forceinline__ float log_ratios(const float* b, const float* q, unsigned valid,
-                                            float K, f2* X) {
+                                            float K, int form, f2* X) {
   constexpr int NP = (PE + 1) / 2;
   float ax0 = 0.f, ax1 = 0.f;
   const f2 K2 = splat(K);
+  if (form == 0) {
+#pragma unroll
+    for (int j = 0; j < NP; ++j) {
+      const int i0 = 2 * j, i1 = (2 * j + 1 < PE) ? 2 * j + 1 : 2 * j;
+      X[j] = add2(sub2(pk(q[i0], q[i1]), pk(b[i0], b[i1])), K2);
+    }
+  } else if (form == 1) {
+#pragma unroll
+    for (int j = 0; j < NP; ++j) {
+      const int i0 = 2 * j, i1 = (2 * j + 1 < PE) ? 2 * j + 1 : 2 * j;
+      X[j] = sub2(add2(pk(q[i0], q[i1]), K2), pk(b[i0], b[i1]));
+    }
+  } else {
+#pragma unroll
+    for (int j = 0; j < NP; ++j) {
+      const int i0 = 2 * j, i1 = (2 * j + 1 < PE) ? 2 * j + 1 : 2 * j;
+      X[j] = sub2(pk(q[i0], q[i1]), sub2(pk(b[i0], b[i1]), K2));
+    }
+  }
 #pragma unroll
   for (int j = 0; j < NP; ++j) {
     const int i0 = 2 * j, i1 = (2 * j + 1 < PE) ? 2 * j + 1 : 2 * j;
-    X[j] = add2(sub2(pk(q[i0], q[i1]), pk(b[i0], b[i1])), K2);
     float x0, x1;
     upk(X[j], x0, x1);
     if (((valid >> i0) & 1u) == 0u) x0 = 0.f;
@@ -504,7 +535,9 @@ __device__ __forceinline__ float log_ratios(const float* b, const float* q, unsi
 // One step of PE element pairs per lane (a 16-element consumer chunk, or the
 // head/tail elements one per lane). Elements whose bit in `valid` is clear
 // are absent (b = q = -inf, x = 0: they contribute nothing).
-template <int PE>
+// kWide: fp32 inputs (the log-ratio's rounding order follows the centre,
+// ratio_form); 16-bit inputs always form q - b first, which is exact.
+template <int PE, bool kWide>
 __device__ __forceinline__ void chunk_step(const float* b, const float* q, unsigned valid,
                                            Ref& r, Acc& a, Best& best, int chunk_id) {
   constexpr int NP = (PE + 1) / 2;
@@ -547,12 +580,14 @@ __device__ __forceinline__ void chunk_step(const float* b, const float* q, unsig
           a.Ap += d * Sp;
           a.Ad += d * a.Se;
           r.K = Kn;
+          if (kWide) r.mode = ratio_form(wmb, Kn);
         }
       } else {
         // First finite maximum: only direct-path terms of masked base
         // entries (e = 0) can have been accumulated.
         a.Ad += d * a.Se;
         r.K = Kn;
+        if (kWide) r.mode = ratio_form(wmb, Kn);
       }
     }
     if (r.Mb != -INFINITY) {
@@ -567,7 +602,7 @@ __device__ __forceinline__ void chunk_step(const float* b, const float* q, unsig
     r.Mb = wmb;
     r.T = wmb + kRaiseMargin;
   }
-  const float axl = log_ratios<PE>(b, q, valid, r.K, X);
+  const float axl = log_ratios<PE>(b, q, valid, r.K, kWide ? r.mode : 0, X);
 
   // The cheapest polynomial tier whose range holds every |x| of the warp's
   // step (a NaN fails every test and takes the direct path).
@@ -646,7 +681,7 @@ __device__ __forceinline__ void process_chunk(const uint4* cb, const uint4* cq, 
       }
     }
   }
-  chunk_step<kLaneElems>(xb, xq, valid, r, a, best, chunk_id);
+  chunk_step<kLaneElems, DT == KLD_F32>(xb, xq, valid, r, a, best, chunk_id);
 }
 
 __device__ __forceinline__ void fail(Ctrl* ctrl, uint32_t* derr) {
@@ -728,33 +763,102 @@ __device__ int rescan_candidates(const void* row, const RowGeom& g, int64_t s0, 
   return best;
 }
 
-// One work item: body elements [s0, s1) of row r; part k of parts_per_row.
-struct Item {
-  int64_t r, s0, s1;
-  int k;
+// Launch schedule (computed on the host, see plan_rows):
+//   P > 1: cluster split, one item per CTA: part blockIdx % P of row
+//          blockIdx / P (each row's chunks divided evenly over P CTAs);
+//   else:  W rounds of whole rows (CTA b takes rows b + j*gridDim, j < W,
+//          r < N), then the R remaining rows [W*gridDim, N) as a tail that
+//          the first Gt CTAs share by balanced ranges of the tail's
+//          Tc = R * nchv virtual chunks (nchv = chunks of a full row): CTA b
+//          takes [Tc*b/Gt, Tc*(b+1)/Gt), which touches at most two rows;
+//          a row is split among the at most 32 CTAs whose ranges touch it.
+//   A > 0: no whole rounds and the tail's ranges fall on row boundaries
+//          (Gt = R * A): CTA b is part b % A of row b / A, found in 32-bit
+//          arithmetic (the general case needs 64-bit divisions).
+struct Sched {
+  int P, W, R, Gt, nchv, A;
+  int64_t Tc;
 };
 
+// One work item: body elements [s0, s1) of row r; part k of the row's np
+// parts (np == 1: the item is the whole row). rt: the row's index among the
+// split rows (its ticket and partial slots). whole: a whole-row round.
+struct Item {
+  int64_t r, s0, s1, rt;
+  int k, np;
+  bool whole;
+};
+
+// CTA holding virtual chunk c of the tail (ranges [Tc*b/Gt, Tc*(b+1)/Gt)).
+__device__ __forceinline__ int64_t tail_cta(int64_t c, const Sched& sc) {
+  return ((c + 1) * sc.Gt - 1) / sc.Tc;
+}
+
 template <int DT>
-__device__ __forceinline__ bool item_at(int j, int P, const char* B, int64_t N, int64_t V,
+__device__ __forceinline__ bool item_at(int j, const Sched& sc, const char* B, int64_t N, int64_t V,
                                         Item& it, RowGeom& g) {
   constexpr int EB = Elem<DT>::kBytes;
-  if (P == 1) {
-    it.r = blockIdx.x + static_cast<int64_t>(j) * gridDim.x;
+  const int64_t b = blockIdx.x;
+  if (sc.P > 1) {
+    if (j > 0) return false;
+    it.r = b / sc.P;
+    it.rt = it.r;
+    it.k = static_cast<int>(b % sc.P);
+    it.np = sc.P;
+    it.whole = false;
+    g = row_geom<DT>(B + it.r * V * EB, V);
+    const int64_t c0 = g.nch * it.k / sc.P, c1 = g.nch * (it.k + 1) / sc.P;
+    it.s0 = c0 * kChunkElems;
+    it.s1 = c1 * kChunkElems < g.body_len ? c1 * kChunkElems : g.body_len;
+    if (it.s1 < it.s0) it.s1 = it.s0;
+    return true;
+  }
+  if (sc.A > 0) {
+    if (j > 0) return false;
+    const int bi = static_cast<int>(blockIdx.x);
+    it.r = bi / sc.A;
+    it.rt = it.r;
+    it.k = bi % sc.A;
+    it.np = sc.A;
+    it.whole = false;
+    g = row_geom<DT>(B + it.r * V * EB, V);
+    const int64_t lo = static_cast<int64_t>(static_cast<unsigned>(sc.nchv) * static_cast<unsigned>(it.k) /
+                                            static_cast<unsigned>(sc.A));
+    const int64_t hi = static_cast<int64_t>(static_cast<unsigned>(sc.nchv) * static_cast<unsigned>(it.k + 1) /
+                                            static_cast<unsigned>(sc.A));
+    it.s0 = lo * kChunkElems < g.body_len ? lo * kChunkElems : g.body_len;
+    it.s1 = hi * kChunkElems < g.body_len ? hi * kChunkElems : g.body_len;
+    return true;
+  }
+  if (j < sc.W) {
+    it.r = b + static_cast<int64_t>(j) * gridDim.x;
     if (it.r >= N) return false;
     g = row_geom<DT>(B + it.r * V * EB, V);
     it.s0 = 0;
     it.s1 = g.body_len;
+    it.rt = -1;
     it.k = 0;
+    it.np = 1;
+    it.whole = true;
     return true;
   }
-  if (j > 0) return false;
-  it.r = blockIdx.x / P;
-  it.k = static_cast<int>(blockIdx.x % P);
+  const int t = j - sc.W;
+  if (t > 1 || b >= sc.Gt) return false;
+  const int64_t c0 = sc.Tc * b / sc.Gt, c1 = sc.Tc * (b + 1) / sc.Gt;
+  const int64_t rt = c0 / sc.nchv + t;
+  if (rt > (c1 - 1) / sc.nchv) return false;
+  it.rt = rt;
+  it.r = static_cast<int64_t>(sc.W) * gridDim.x + rt;
   g = row_geom<DT>(B + it.r * V * EB, V);
-  const int64_t c0 = g.nch * it.k / P, c1 = g.nch * (it.k + 1) / P;
-  it.s0 = c0 * kChunkElems;
-  it.s1 = c1 * kChunkElems < g.body_len ? c1 * kChunkElems : g.body_len;
-  if (it.s1 < it.s0) it.s1 = it.s0;
+  const int64_t rc0 = rt * sc.nchv;
+  const int64_t lo = (c0 > rc0 ? c0 : rc0) - rc0;
+  const int64_t hi = (c1 < rc0 + sc.nchv ? c1 : rc0 + sc.nchv) - rc0;
+  it.s0 = lo * kChunkElems < g.body_len ? lo * kChunkElems : g.body_len;
+  it.s1 = hi * kChunkElems < g.body_len ? hi * kChunkElems : g.body_len;
+  const int64_t first = tail_cta(rc0, sc);
+  it.k = static_cast<int>(b - first);
+  it.np = static_cast<int>(tail_cta(rc0 + sc.nchv - 1, sc) - first + 1);
+  it.whole = false;
   return true;
 }
 
@@ -962,10 +1066,34 @@ __device__ __forceinline__ uint32_t map_to_rank(uint32_t local, uint32_t rank) {
   return r;
 }
 
-// Few split rows (red_out set): every row's finaliser counts its record on
-// the launch's counter; the warp that counts the last record reduces all N
-// records on the spot, so the statistic needs no second kernel. The counter
-// goes back to zero for the next launch.
+// Arguments of the row kernel (passed by value, __grid_constant__).
+struct RowParams {
+  const void* base;
+  const void* quant;
+  const int32_t* tok;
+  int64_t N, V;
+  kld_row_t* rows;
+  uint32_t* derr;
+  Sched sc;
+  MPart* gparts;       // split rows: partials, kPartSlots per split row
+  unsigned* tickets;   // split rows: one arrival counter per split row
+  RowAux* aux;         // nullable: per-row normalisers
+  MPart* part_out;     // nullable: vocabulary-slice partials instead of records
+  int64_t col0;
+  // Few split rows (nullable): the launch also reduces its records into
+  // *out, counting finished rows on *counter (see count_row).
+  kld_result_t* out;
+  unsigned* counter;
+};
+
+// Slots of partials per split row in the split scratch (one per part; a
+// row has at most 32 parts, merged by one warp).
+constexpr int kPartSlots = kPartSlotsPerRow;
+
+// Few split rows (RowParams.out set): every row's finaliser counts its
+// record on the launch's counter; the warp that counts the last record
+// reduces all N records on the spot, so the statistic needs no second
+// kernel. The counter goes back to zero for the next launch.
 __device__ __forceinline__ void count_row(unsigned* counter, const kld_row_t* rows, int64_t N,
                                           int has_nll, uint32_t* derr, kld_result_t* out,
                                           int lane) {
@@ -979,14 +1107,27 @@ __device__ __forceinline__ void count_row(unsigned* counter, const kld_row_t* ro
   fin::reduce_few_rows(rows, static_cast<int>(N), has_nll, derr, out, lane);
 }
 
+// A finished row, written by lane 0 of the warp that finalised it: the
+// record and the row's normalisers.
+__device__ __forceinline__ void write_row(const RowParams& p, int64_t r, const kld_row_t& rec,
+                                          const MPart& m) {
+  p.rows[r] = rec;
+  if (p.aux != nullptr) p.aux[r] = row_aux(m, rec);
+}
+
 template <int DT>
-__global__ void __launch_bounds__(kRowThreads, 1)
-    kld_rows_kernel(const void* __restrict__ base, const void* __restrict__ quant,
-                    const int32_t* __restrict__ tok, int64_t N, int64_t V,
-                    kld_row_t* __restrict__ rows, uint32_t* __restrict__ derr, int P,
-                    MPart* __restrict__ gparts, unsigned* __restrict__ tickets, RowAux* __restrict__ aux,
-                    MPart* __restrict__ part_out, int64_t col0,
-                    kld_result_t* __restrict__ red_out) {
+__global__ void __launch_bounds__(kRowThreads, 1) kld_rows_kernel(const __grid_constant__ RowParams prm) {
+  const void* __restrict__ base = prm.base;
+  const void* __restrict__ quant = prm.quant;
+  const int32_t* __restrict__ tok = prm.tok;
+  const int64_t N = prm.N, V = prm.V;
+  kld_row_t* __restrict__ rows = prm.rows;
+  uint32_t* __restrict__ derr = prm.derr;
+  const Sched& sc = prm.sc;  // read from parameter space where used
+  MPart* __restrict__ gparts = prm.gparts;
+  unsigned* __restrict__ tickets = prm.tickets;
+  MPart* __restrict__ part_out = prm.part_out;
+  const int64_t col0 = prm.col0;
   constexpr int EB = Elem<DT>::kBytes;
   constexpr int E = Elem<DT>::kPerVec;
   constexpr int kStageElems = kStageBytes / EB;
@@ -1000,7 +1141,7 @@ __global__ void __launch_bounds__(kRowThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const uint32_t G = P > 1 ? cluster_nctarank() : 1u;  // CTAs per cluster
+  const uint32_t G = sc.P > 1 ? cluster_nctarank() : 1u;  // CTAs per cluster
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -1038,7 +1179,7 @@ __global__ void __launch_bounds__(kRowThreads, 1)
       bool ok = true;
       Item it;
       RowGeom g;
-      for (int j = 0; ok && item_at<DT>(j, P, B, N, V, it, g); ++j) {
+      for (int j = 0; ok && item_at<DT>(j, sc, B, N, V, it, g); ++j) {
         const char* rb = B + it.r * V * EB;
         const char* rq = Q + it.r * V * EB;
         const int64_t n = it.s1 - it.s0;
@@ -1096,7 +1237,7 @@ __global__ void __launch_bounds__(kRowThreads, 1)
     // whole-row and split-row loops below each inline their own copy, so
     // the split bookkeeping costs the whole-row loop no registers.
     auto consume = [&](int n, int j) -> bool {
-      Ref ref{-INFINITY, -INFINITY, 0.f, 0.f, 0.f, -INFINITY};
+      Ref ref{-INFINITY, -INFINITY, 0.f, 0.f, 0.f, -INFINITY, 0};
       Acc acc{0.0, 0.0, 0.0, 0.0, 0.0, 0.0};
       Best best{-INFINITY, -INFINITY, -1, -1};
       const int ntiles = (n + kStageElems - 1) / kStageElems;
@@ -1182,24 +1323,27 @@ __global__ void __launch_bounds__(kRowThreads, 1)
       if (lane == 0) mbar_arrive(smem_u32(&ctrl->slot_full[slot]));
       return true;
     };
-    if (P == 1) {
-      for (int j = 0;; ++j) {
+    bool ok = true;
+    int j = 0;
+    if (sc.P <= 1) {
+      for (; j < sc.W; ++j) {  // whole rows
         const int64_t r = blockIdx.x + static_cast<int64_t>(j) * gridDim.x;
         if (r >= N) break;
         const RowGeom g = row_geom<DT>(B + r * V * EB, V);
-        if (!consume(static_cast<int>(g.body_len), j)) break;
+        if (!(ok = consume(static_cast<int>(g.body_len), j))) break;
       }
-    } else {
+    }
+    if (ok) {  // parts of split rows
       Item it;
       RowGeom g;
-      item_at<DT>(0, P, B, N, V, it, g);
-      consume(static_cast<int>(it.s1 - it.s0), 0);
+      for (j = sc.P > 1 ? 0 : sc.W; item_at<DT>(j, sc, B, N, V, it, g); ++j)
+        if (!consume(static_cast<int>(it.s1 - it.s0), j)) break;
     }
   } else {
     // ---------------------------------------------------------------- epilogue
     Item it;
     RowGeom g;
-    for (int j = 0; item_at<DT>(j, P, B, N, V, it, g); ++j) {
+    for (int j = 0; item_at<DT>(j, sc, B, N, V, it, g); ++j) {
       const int64_t r = it.r;
       const char* rb = B + r * V * EB;
       const char* rq = Q + r * V * EB;
@@ -1227,10 +1371,11 @@ __global__ void __launch_bounds__(kRowThreads, 1)
           b_tok = Elem<DT>::load(rb, tk);
         }
       }
-      Ref eref{-INFINITY, -INFINITY, 0.f, 0.f, 0.f, -INFINITY};
+      Ref eref{-INFINITY, -INFINITY, 0.f, 0.f, 0.f, -INFINITY, 0};
       Acc eacc{0.0, 0.0, 0.0, 0.0, 0.0, 0.0};
       Best ebest{-INFINITY, -INFINITY, -1, -1};
-      if (n_extra > 0) chunk_step<1>(&xe_b, &xe_q, lane < n_extra ? 1u : 0u, eref, eacc, ebest, 0);
+      if (n_extra > 0)
+        chunk_step<1, DT == KLD_F32>(&xe_b, &xe_q, lane < n_extra ? 1u : 0u, eref, eacc, ebest, 0);
       const float eMb = warp_max(xe_b), eMq = warp_max(xe_q);
       const double eSb = warp_sum(eacc.Sb), eAp = warp_sum(eacc.Ap), eC = warp_sum(eacc.C);
       const double eAd = warp_sum(eacc.Ad), eSe = warp_sum(eacc.Se), eSh = warp_sum(eacc.Sh);
@@ -1244,7 +1389,7 @@ __global__ void __launch_bounds__(kRowThreads, 1)
         // Whole rows: nothing is written for this or later rows. Split rows:
         // the part still travels, flagged, so the row's combine completes.
         fail(ctrl, derr);
-        if (P == 1) break;
+        if (it.np == 1) break;
         m.flags = kPartFailed;
       } else {
       const Slot& sl = ctrl->slot[slot];
@@ -1309,7 +1454,11 @@ __global__ void __launch_bounds__(kRowThreads, 1)
         // A split part of at most kStages tiles (the CTA's only item) is
         // still whole in the ring: rescan it there.
         const int64_t n_item = it.s1 - it.s0;
-        const bool in_ring = P > 1 && n_item <= static_cast<int64_t>(kStages) * (kStageBytes / EB);
+        Item nx;
+        RowGeom ng;
+        const bool in_ring = !it.whole && j == 0 &&
+                             n_item <= static_cast<int64_t>(kStages) * (kStageBytes / EB) &&
+                             !item_at<DT>(1, sc, B, N, V, nx, ng);
         while (wb) {
           const int w = __ffs(wb) - 1;
           wb &= wb - 1u;
@@ -1334,7 +1483,7 @@ __global__ void __launch_bounds__(kRowThreads, 1)
       }
 
 
-      if (P == 1 && part_out != nullptr) {
+      if (part_out != nullptr) {
         // Vocabulary slice [col0, col0 + V) of a wider row: publish the
         // merged partial with global argmax indices, and the token's logits
         // when the token falls in this slice; the rows' slices meet in
@@ -1358,109 +1507,111 @@ __global__ void __launch_bounds__(kRowThreads, 1)
         }
         continue;
       }
-      if (P == 1) {
-          const kld_row_t rec = finalize_row(m, tok != nullptr, tok_ok, q_tok, b_tok);
-        if (lane == 0) {
-          rows[r] = rec;
-          if (aux != nullptr) aux[r] = row_aux(m, rec);
-        }
+      if (it.np == 1) {  // the whole row is this item
+        const kld_row_t rec = finalize_row(m, tok != nullptr, tok_ok, q_tok, b_tok);
+        if (lane == 0) write_row(prm, r, rec, m);
+        if (prm.out != nullptr) count_row(prm.counter, rows, N, tok != nullptr, derr, prm.out, lane);
         continue;
       }
 
       // ---------------- split row: cluster combine through DSMEM, then across
-      // the row's clusters through global memory and a ticket.
-      const uint32_t rank = G > 1 ? cluster_ctarank() : 0u;
-      if (G > 1 && rank != 0) {
-        // Push this CTA's partial into the leader's shared memory (its
-        // barrier is initialised once the first cluster phase completes),
-        // then arrive on the leader's barrier (release at cluster scope).
-        asm volatile("barrier.cluster.wait.acquire;" ::: "memory");
-        cl_waited = true;
-        if (lane == 0) {
-          const uint32_t dst = map_to_rank(smem_u32(&ctrl->cl_part[rank]), 0u);
-          unsigned long long wds[8];
-          part_words(m, wds);
-#pragma unroll
-          for (int w = 0; w < 8; ++w)
-            asm volatile("st.shared::cluster.u64 [%0], %1;" ::"r"(dst + 8 * w), "l"(wds[w])
-                         : "memory");
-          const uint32_t bar = map_to_rank(smem_u32(&ctrl->cl_full), 0u);
-          asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar)
-                       : "memory");
-        }
-        continue;
-      }
+      // the row's clusters (or the CTAs sharing a tail row) through global
+      // memory and a ticket.
       MPart cm = m;
-      if (G > 1) {
-        // Wait (bounded) for the peers' partials; every lane acquires them.
-        const uint32_t bar = smem_u32(&ctrl->cl_full);
-        uint32_t okw = 0;
-        const uint64_t t0 = globaltimer();
-        for (uint32_t i = 0;; ++i) {
-          asm volatile(
-              "{\n\t.reg .pred p;\n\t"
-              "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], 0;\n\t"
-              "selp.u32 %0, 1, 0, p;\n\t}"
-              : "=r"(okw)
-              : "r"(bar)
-              : "memory");
-          if (okw) break;
-          if ((i & 63u) == 63u && globaltimer() - t0 > kWaitLimitNs) break;
-        }
-        MPart q = empty_part();
-        if (__all_sync(0xffffffffu, okw != 0)) {
-          if (lane == 0) q = m;
-          if (lane >= 1 && lane < static_cast<int>(G)) {
-            const ulonglong2* src = reinterpret_cast<const ulonglong2*>(&ctrl->cl_part[lane]);
-            unsigned long long wds[8];
-#pragma unroll
-            for (int w = 0; w < 4; ++w) {
-              const ulonglong2 v = src[w];
-              wds[2 * w] = v.x;
-              wds[2 * w + 1] = v.y;
-            }
-            q = part_from_words(wds);
-          }
-        } else {
-          fail(ctrl, derr);
+      int nparts = it.np, part = it.k;
+      int64_t tix = it.rt;  // the row's ticket and partial slots
+      if (sc.P > 1) {
+        const uint32_t rank = G > 1 ? cluster_ctarank() : 0u;
+        if (G > 1 && rank != 0) {
+          // Push this CTA's partial into the leader's shared memory (its
+          // barrier is initialised once the first cluster phase completes),
+          // then arrive on the leader's barrier (release at cluster scope).
+          asm volatile("barrier.cluster.wait.acquire;" ::: "memory");
+          cl_waited = true;
           if (lane == 0) {
-            q = m;
-            q.flags |= kPartFailed;
+            const uint32_t dst = map_to_rank(smem_u32(&ctrl->cl_part[rank]), 0u);
+            unsigned long long wds[8];
+            part_words(m, wds);
+#pragma unroll
+            for (int w = 0; w < 8; ++w)
+              asm volatile("st.shared::cluster.u64 [%0], %1;" ::"r"(dst + 8 * w), "l"(wds[w])
+                           : "memory");
+            const uint32_t bar = map_to_rank(smem_u32(&ctrl->cl_full), 0u);
+            asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar)
+                         : "memory");
           }
+          continue;
         }
-        cm = warp_merge(q);
-      }
-      const int C = P / static_cast<int>(G);  // clusters per row
-      if (C == 1) {
+        if (G > 1) {
+          // Wait (bounded) for the peers' partials; every lane acquires them.
+          const uint32_t bar = smem_u32(&ctrl->cl_full);
+          uint32_t okw = 0;
+          const uint64_t t0 = globaltimer();
+          for (uint32_t i = 0;; ++i) {
+            asm volatile(
+                "{\n\t.reg .pred p;\n\t"
+                "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], 0;\n\t"
+                "selp.u32 %0, 1, 0, p;\n\t}"
+                : "=r"(okw)
+                : "r"(bar)
+                : "memory");
+            if (okw) break;
+            if ((i & 63u) == 63u && globaltimer() - t0 > kWaitLimitNs) break;
+          }
+          MPart q = empty_part();
+          if (__all_sync(0xffffffffu, okw != 0)) {
+            if (lane == 0) q = m;
+            if (lane >= 1 && lane < static_cast<int>(G)) {
+              const ulonglong2* src = reinterpret_cast<const ulonglong2*>(&ctrl->cl_part[lane]);
+              unsigned long long wds[8];
+#pragma unroll
+              for (int w = 0; w < 4; ++w) {
+                const ulonglong2 v = src[w];
+                wds[2 * w] = v.x;
+                wds[2 * w + 1] = v.y;
+              }
+              q = part_from_words(wds);
+            }
+          } else {
+            fail(ctrl, derr);
+            if (lane == 0) {
+              q = m;
+              q.flags |= kPartFailed;
+            }
+          }
+          cm = warp_merge(q);
+        }
+        nparts = sc.P / static_cast<int>(G);  // clusters per row
+        part = it.k / static_cast<int>(G);
+        tix = r;
+        if (nparts == 1) {
           const kld_row_t rec = finalize_row(cm, tok != nullptr, tok_ok, q_tok, b_tok);
-        if (lane == 0) {
-          rows[r] = rec;
-          if (aux != nullptr) aux[r] = row_aux(cm, rec);
+          if (lane == 0) write_row(prm, r, rec, cm);
+          if (prm.out != nullptr) count_row(prm.counter, rows, N, tok != nullptr, derr, prm.out, lane);
+          continue;
         }
-        if (red_out != nullptr) count_row(tickets + N, rows, N, tok != nullptr, derr, red_out, lane);
-        continue;
       }
-      const int cid = it.k / static_cast<int>(G);
+      MPart* slots = gparts + tix * kPartSlots;
       unsigned ticket = 0u;
       if (lane == 0) {
         unsigned long long wds[8];
         part_words(cm, wds);
-        ulonglong2* dst = reinterpret_cast<ulonglong2*>(&gparts[r * C + cid]);
+        ulonglong2* dst = reinterpret_cast<ulonglong2*>(&slots[part]);
 #pragma unroll
         for (int w = 0; w < 4; ++w) dst[w] = make_ulonglong2(wds[2 * w], wds[2 * w + 1]);
         // release: the partial above is visible to whoever sees the count;
         // acquire: the last arriver sees every other part's partial
         asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;"
                      : "=r"(ticket)
-                     : "l"(&tickets[r])
+                     : "l"(&tickets[tix])
                      : "memory");
       }
       ticket = __shfl_sync(0xffffffffu, ticket, 0);
-      if (ticket != static_cast<unsigned>(C - 1)) continue;  // not the last cluster
+      if (ticket != static_cast<unsigned>(nparts - 1)) continue;  // not the last part
       __syncwarp();  // lane 0's acquire orders the other lanes' loads below
       MPart q = empty_part();
-      if (lane < C) {
-        const ulonglong2* src = reinterpret_cast<const ulonglong2*>(&gparts[r * C + lane]);
+      if (lane < nparts) {
+        const ulonglong2* src = reinterpret_cast<const ulonglong2*>(&slots[lane]);
         unsigned long long wds[8];
 #pragma unroll
         for (int w = 0; w < 4; ++w) {
@@ -1473,11 +1624,10 @@ __global__ void __launch_bounds__(kRowThreads, 1)
       const MPart fm = warp_merge(q);
       const kld_row_t rec = finalize_row(fm, tok != nullptr, tok_ok, q_tok, b_tok);
       if (lane == 0) {
-        rows[r] = rec;
-        if (aux != nullptr) aux[r] = row_aux(fm, rec);
-        tickets[r] = 0u;  // ready for the next launch
+        write_row(prm, r, rec, fm);
+        tickets[tix] = 0u;  // ready for the next launch
       }
-      if (red_out != nullptr) count_row(tickets + N, rows, N, tok != nullptr, derr, red_out, lane);
+      if (prm.out != nullptr) count_row(prm.counter, rows, N, tok != nullptr, derr, prm.out, lane);
     }
   }
 
@@ -1487,6 +1637,7 @@ __global__ void __launch_bounds__(kRowThreads, 1)
     if (!cl_waited) asm volatile("barrier.cluster.wait.acquire;" ::: "memory");
     asm volatile("barrier.cluster.arrive.release;\n\tbarrier.cluster.wait.acquire;" ::: "memory");
   }
+
 }
 
 // Vocabulary-sharded rows: one warp per row merges the row's G slice
@@ -1582,10 +1733,7 @@ int max_active_clusters(int cluster_ctas) {
 }
 
 template <int DT>
-cudaError_t launch_typed(const void* base, const void* quant, const int32_t* tok, int64_t N,
-                         int64_t V, kld_row_t* rows, uint32_t* derr, const RowPlan& pl,
-                         const SplitScratch* split, RowAux* aux, MPart* part_out, int64_t col0,
-                         kld_result_t* red_out, cudaStream_t stream) {
+cudaError_t launch_typed(const RowParams& prm, const RowPlan& pl, cudaStream_t stream) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(pl.grid));
   cfg.blockDim = dim3(kRowThreads);
@@ -1598,10 +1746,7 @@ cudaError_t launch_typed(const void* base, const void* quant, const int32_t* tok
   attr.val.clusterDim.z = 1;
   cfg.attrs = &attr;
   cfg.numAttrs = pl.cluster_ctas > 1 ? 1 : 0;
-  MPart* gp = split ? static_cast<MPart*>(split->parts) : nullptr;
-  unsigned* tk = split ? split->tickets : nullptr;
-  return cudaLaunchKernelEx(&cfg, kld_rows_kernel<DT>, base, quant, tok, N, V, rows, derr,
-                            pl.parts_per_row, gp, tk, aux, part_out, col0, red_out);
+  return cudaLaunchKernelEx(&cfg, kld_rows_kernel<DT>, prm);
 }
 
 }  // namespace
@@ -1618,26 +1763,83 @@ cudaError_t prepare_rows_kernels() {
                               cudaFuncAttributeMaxDynamicSharedMemorySize, kRowSmemBytes);
 }
 
-RowPlan plan_rows(int64_t N, int sm_count, const int fit[4], int max_cluster_ctas) {
+RowPlan plan_rows(int64_t N, int64_t V, int sm_count, const int fit[4], int max_cluster_ctas) {
   RowPlan pl;
   pl.parts_per_row = 1;
   pl.cluster_ctas = 1;
-  pl.grid = static_cast<int>(N < sm_count ? N : sm_count);
-  if (pl.grid < 1) pl.grid = 1;
-  if (max_cluster_ctas < 1 || N * 2 > sm_count) return pl;
-  int lg = 0;
-  while (lg < 3 && (2 << lg) <= max_cluster_ctas) ++lg;
-  for (; lg >= 0; --lg) {
-    const int G = 1 << lg;
-    const int f = fit != nullptr && fit[lg] > 0 ? fit[lg] : sm_count / G;
-    if (f < N) continue;  // not one cluster per row in one wave
-    int C = static_cast<int>(f / N);
-    if (C > 32) C = 32;  // a row's clusters are merged by one warp
-    if (G * C < 2) continue;
-    pl.cluster_ctas = G;
-    pl.parts_per_row = G * C;
-    pl.grid = static_cast<int>(N) * pl.parts_per_row;
+  pl.tail_rows = 0;
+  pl.tail_ctas = 0;
+  pl.tail_chunks = 0;
+  const int64_t nchv = (V + kChunkElems - 1) / kChunkElems;
+  pl.nchv = static_cast<int>(nchv);
+  const int64_t G = sm_count > 0 ? sm_count : 1;
+  if (max_cluster_ctas < 1) {  // whole rows, round robin
+    pl.grid = static_cast<int>(N < G ? N : G);
+    if (pl.grid < 1) pl.grid = 1;
+    pl.whole = static_cast<int>((N + pl.grid - 1) / pl.grid);
     return pl;
+  }
+  if (max_cluster_ctas >= 2 && N * 2 <= G) {
+    int lg = 0;
+    while (lg < 3 && (2 << lg) <= max_cluster_ctas) ++lg;
+    for (; lg >= 1; --lg) {
+      const int C0 = 1 << lg;
+      const int f = fit != nullptr && fit[lg] > 0 ? fit[lg] : static_cast<int>(G / C0);
+      if (f < N) continue;  // not one cluster per row in one wave
+      int C = static_cast<int>(f / N);
+      if (C > kPartSlots) C = kPartSlots;  // a row's clusters are merged by one warp
+      pl.cluster_ctas = C0;
+      pl.parts_per_row = C0 * C;
+      pl.grid = static_cast<int>(N) * pl.parts_per_row;
+      pl.whole = 0;
+      return pl;
+    }
+  }
+  // Whole-row rounds, then a last partial wave of R <= G/2 rows split over
+  // the CTAs by balanced chunk ranges: a CTA's range then covers at most
+  // two rows, and a range of at least ceil(nchv / 30) chunks keeps every
+  // row within 31 CTAs. Below one wave, rows are split into P row-aligned
+  // parts (one part per CTA, as many as the SMs hold, at most 32 per row).
+  // A larger last wave, or N between G/2 and G, takes whole rows: splitting
+  // it would give most CTAs two partial rows to finish, which measured
+  // slower than letting the wave's CTAs stream whole rows.
+  const int64_t W = N / G, R = N % G;
+  pl.whole = static_cast<int>(W);
+  pl.grid = static_cast<int>(G);
+  int64_t Gt = 0;
+  if (W == 0) {
+    int64_t P = G / N;
+    if (P > kPartSlots) P = kPartSlots;
+    if (P > nchv) P = nchv;
+    if (N * 2 > G || P < 2) {  // whole rows, one per CTA
+      pl.grid = static_cast<int>(N);
+      pl.whole = 1;
+      return pl;
+    }
+    Gt = N * P;  // ranges of the balanced split fall on row boundaries
+  } else if (R > 0) {
+    if (R * 2 > G) {  // whole rows, one more round
+      pl.whole = static_cast<int>(W + 1);
+      return pl;
+    }
+    const int64_t q = (nchv + 29) / 30;
+    Gt = (R * nchv) / q;
+    if (Gt > G) Gt = G;
+    if (Gt < R) Gt = R;
+  }
+  if (R > 0) {
+    const int64_t Tc = R * nchv;
+    pl.tail_rows = static_cast<int>(R);
+    pl.tail_ctas = static_cast<int>(Gt);
+    pl.tail_chunks = Tc;
+    if (W == 0) pl.grid = static_cast<int>(Gt);
+    int most = 1;
+    for (int64_t rt = 0; rt < R; ++rt) {
+      const int64_t first = ((rt * nchv + 1) * Gt - 1) / Tc;
+      const int64_t last = (((rt + 1) * nchv) * Gt - 1) / Tc;
+      if (last - first + 1 > most) most = static_cast<int>(last - first + 1);
+    }
+    pl.parts_per_row = most;
   }
   return pl;
 }
@@ -1678,35 +1880,58 @@ cudaError_t launch_rows(const void* base, const void* quant, const int32_t* toke
                         cudaStream_t stream, void* part_out, int64_t col_offset,
                         kld_result_t* result_out, bool* reduced) {
   if (reduced) *reduced = false;
-  RowPlan pl = plan_rows(N, sm_count, nullptr, 0);
-  // Vocabulary-slice partials come from whole-row launches only.
-  if (split != nullptr && part_out == nullptr && N * 2 <= sm_count && split->max_cluster_ctas >= 1) {
+  // Vocabulary-slice partials and launches without split scratch take
+  // whole rows only.
+  const bool can_split = split != nullptr && part_out == nullptr && split->max_cluster_ctas >= 1;
+  RowPlan pl = plan_rows(N, V, sm_count, nullptr, can_split ? 1 : 0);
+  if (can_split) {
     int fit[4] = {0, 0, 0, 0};
-    for (int lg = 0; lg < 4 && (1 << lg) <= split->max_cluster_ctas; ++lg)
-      fit[lg] = active_clusters(dtype, lg);
-    pl = plan_rows(N, sm_count, fit, split->max_cluster_ctas);
-    if (static_cast<int64_t>(pl.grid) / pl.cluster_ctas > split->capacity || N > split->capacity)
-      pl = plan_rows(N, sm_count, nullptr, 0);
+    if (split->max_cluster_ctas >= 2 && N * 2 <= sm_count)
+      for (int lg = 1; lg < 4 && (1 << lg) <= split->max_cluster_ctas; ++lg)
+        fit[lg] = active_clusters(dtype, lg);
+    pl = plan_rows(N, V, sm_count, fit, split->max_cluster_ctas);
+    const int64_t split_rows = pl.cluster_ctas > 1 ? N : pl.tail_rows;
+    if (split_rows > split->capacity || pl.grid > split->capacity)
+      pl = plan_rows(N, V, sm_count, nullptr, 0);
   }
-  // Few split rows: the row pass reduces its own records (the launch counter
-  // is the ticket after the last row's).
-  const bool fuse = result_out != nullptr && pl.parts_per_row > 1 && N <= kFusedReduceRows &&
-                    split != nullptr && N + 1 <= split->capacity;
-  kld_result_t* red = fuse ? result_out : nullptr;
+  RowParams prm = {};
+  prm.base = base;
+  prm.quant = quant;
+  prm.tok = token_ids;
+  prm.N = N;
+  prm.V = V;
+  prm.rows = rows;
+  prm.derr = derr;
+  prm.sc.P = pl.cluster_ctas > 1 ? pl.parts_per_row : 0;
+  prm.sc.W = pl.whole;
+  prm.sc.R = pl.tail_rows;
+  prm.sc.Gt = pl.tail_ctas;
+  prm.sc.nchv = pl.nchv;
+  prm.sc.Tc = pl.tail_chunks;
+  // row-aligned parts (no whole rounds): nchv * A stays within 32 bits
+  prm.sc.A = (pl.cluster_ctas == 1 && pl.whole == 0 && pl.tail_rows > 0 &&
+              pl.tail_ctas == pl.tail_rows * pl.parts_per_row &&
+              static_cast<int64_t>(pl.nchv) * pl.parts_per_row < (int64_t{1} << 32))
+                 ? pl.parts_per_row
+                 : 0;
+  prm.gparts = split ? static_cast<MPart*>(split->parts) : nullptr;
+  prm.tickets = split ? split->tickets : nullptr;
+  prm.aux = aux;
+  prm.part_out = static_cast<MPart*>(part_out);
+  prm.col0 = col_offset;
+  // Few split rows (no whole-row round): the row pass reduces its own
+  // records (the launch counter is the ticket after the last split row's).
+  const bool fuse = result_out != nullptr && can_split && pl.whole == 0 &&
+                    N <= kFusedReduceRows && N + 1 <= split->capacity;
+  if (fuse) {
+    prm.out = result_out;
+    prm.counter = split->tickets + N;
+  }
   cudaError_t e = cudaErrorInvalidValue;
   switch (dtype) {
-    case KLD_F32:
-      e = launch_typed<KLD_F32>(base, quant, token_ids, N, V, rows, derr, pl, split, aux,
-                                static_cast<MPart*>(part_out), col_offset, red, stream);
-      break;
-    case KLD_BF16:
-      e = launch_typed<KLD_BF16>(base, quant, token_ids, N, V, rows, derr, pl, split, aux,
-                                 static_cast<MPart*>(part_out), col_offset, red, stream);
-      break;
-    case KLD_F16:
-      e = launch_typed<KLD_F16>(base, quant, token_ids, N, V, rows, derr, pl, split, aux,
-                                static_cast<MPart*>(part_out), col_offset, red, stream);
-      break;
+    case KLD_F32: e = launch_typed<KLD_F32>(prm, pl, stream); break;
+    case KLD_BF16: e = launch_typed<KLD_BF16>(prm, pl, stream); break;
+    case KLD_F16: e = launch_typed<KLD_F16>(prm, pl, stream); break;
   }
   if (e == cudaSuccess && reduced) *reduced = fuse;
   return e;

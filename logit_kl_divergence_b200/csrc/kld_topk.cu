@@ -9,8 +9,8 @@
 // Runs after the row pass, which leaves each row's normalisers (RowAux:
 // lse_b, log1p(B/S), the centre K and fp32 frames) so that, for j in T,
 //   log p_j = lambda*b_j - lse_b,  log(p_j / r_j) = log1p(B/S) - lambda*x_j,
-// x_j = (q_j - b_j) + K rounded to fp32 as the row pass rounds it, the rest
-// in fp64.
+// x_j = q_j - b_j + K formed as the row pass forms it (kShiftForm), the
+// rest in fp64.
 //
 // One CTA per row (persistent over rows, four per SM). Fast path: 4096
 // samples of the base row (512 evenly spaced runs of 8 adjacent elements,
@@ -441,12 +441,17 @@ __device__ void t_terms(const unsigned long long* sorted, const char* rb, const 
         if (qj == -INFINITY) {
           inf_t = 1.0;
         } else {
-          // x rounded exactly as the row pass rounds it, so that it agrees
-          // with the log1p(B/S) that pass summed from the same values (an
-          // exact x would leave their mean rounding error, ~1e-6 for a
-          // quant row offset from the base by 1000, in the result)
-          const float x = __fadd_rn(__fsub_rn(qj, bj), a.K);
-          const double lratio = a.lr - lambda * static_cast<double>(x);  // log p_j - log r_j
+          // x formed as the row pass forms it, so that it agrees with the
+          // log1p(B/S) that pass summed: rounded as (q - b) + K for small
+          // centres (an exact x would leave the sums' mean rounding error
+          // in the result), exact for fp32 rows offset by a large constant
+          // (where the row pass's order keeps x exact)
+          double x;
+          if (DT == KLD_F32 && fabsf(a.K) >= kShiftForm)
+            x = (static_cast<double>(qj) - static_cast<double>(bj)) + static_cast<double>(a.K);
+          else
+            x = static_cast<double>(__fadd_rn(__fsub_rn(qj, bj), a.K));
+          const double lratio = a.lr - lambda * x;  // log p_j - log r_j
           kl_t += exp(lp) * lratio;
         }
       }

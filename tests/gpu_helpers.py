@@ -6,8 +6,11 @@ and NLL (quant and base) |gpu - ref| <= 1e-6 + 1e-4 * |ref|; mean KLD,
 percentiles, mean NLL and PPL (quant and base), the PPL ratio and the mean
 and RMS of dp within 1e-5 relative, with an absolute floor where the
 reference is ~0 (1e-9 nats for KL statistics, 1e-7 nats for mean NLL, i.e.
-1e-7 relative for PPL, 1e-9 for dp statistics): fp32 inputs do not resolve a
-log-probability better than that. ln(PPL ratio) within 1e-5 absolute is the
+1e-7 relative for PPL): fp32 inputs do not resolve a log-probability better
+than that. The dp statistics take a floor of 5e-8: a row's dp carries the
+absolute rounding of its two NLLs (fp32 exponentials in the row pass, ~1e-8
+where the NLL is ~0, as in single-token vocabularies), far inside the dp bar
+the per-row NLL bars allow (~1e-6). ln(PPL ratio) within 1e-5 absolute is the
 ratio within 1e-5 relative.
 """
 from __future__ import annotations
@@ -27,7 +30,7 @@ ROW_ATOL, ROW_RTOL = 1e-6, 1e-4
 STAT_RTOL = 1e-5
 STAT_ATOL = {"mean_kld": 1e-9, "median_kld": 1e-9, "p90_kld": 1e-9, "p99_kld": 1e-9,
              "max_kld": 1e-9, "mean_nll": 1e-7, "mean_nll_base": 1e-7, "top1_agree_pct": 0.0,
-             "mean_dp": 1e-9, "rms_dp": 1e-9}
+             "mean_dp": 5e-8, "rms_dp": 5e-8}
 CORES = max(1, os.cpu_count() or 1)
 
 

@@ -144,28 +144,80 @@ def test_create_without_gpu_reports_no_device(lib):
     assert lib.kld_last_cuda_error()
 
 
+def _tail_ranges(n, v, sms, p):
+    """Items of every CTA under plan p, recomputed from the plan's fields:
+    whole rows round robin, then balanced ranges of the tail's chunks."""
+    nchv = -(-v // 512)
+    items = {b: [] for b in range(p["grid"])}
+    for b in range(p["grid"]):
+        for j in range(p["whole_rounds"]):
+            r = b + j * p["grid"]
+            if r < n:
+                items[b].append((r, 0, nchv))
+    R, Gt = p["tail_rows"], p["tail_ctas"]
+    if R:
+        Tc = R * nchv
+        for b in range(Gt):
+            c0, c1 = Tc * b // Gt, Tc * (b + 1) // Gt
+            for rt in range(c0 // nchv, (c1 - 1) // nchv + 1):
+                lo, hi = max(c0, rt * nchv) - rt * nchv, min(c1, (rt + 1) * nchv) - rt * nchv
+                items[b].append((p["whole_rounds"] * p["grid"] + rt, lo, hi))
+    return items
+
+
 def test_plan_host_logic():
     p = plan(8192, 151936, _lib.KLD_F32, 148)
-    assert p["grid"] == 148 and p["threads"] % 32 == 0
-    assert p["smem_bytes"] <= 227 * 1024
-    # few rows: split into as many parts (<= 32 per row) as fit in one wave
-    p = plan(1, 151936, _lib.KLD_F32, 148)
-    assert (p["variant"], p["cluster_ctas"], p["ctas_per_row"], p["grid"]) == (1, 1, 32, 32)
-    p = plan(5, 1000, _lib.KLD_BF16, 148)
-    assert (p["variant"], p["cluster_ctas"], p["ctas_per_row"], p["grid"]) == (1, 1, 29, 145)
-    p = plan(74, 1000, _lib.KLD_F16, 148)
-    assert (p["cluster_ctas"], p["ctas_per_row"], p["grid"]) == (1, 2, 148)
-    p = plan(75, 1000, _lib.KLD_F32, 148)
-    assert (p["variant"], p["cluster_ctas"], p["ctas_per_row"], p["grid"]) == (0, 1, 1, 75)
+    # 55 whole rounds; the 52 rows of the last partial wave split over all SMs
+    assert (p["variant"], p["grid"], p["whole_rounds"], p["tail_rows"], p["tail_ctas"]) == (2, 148, 55, 52, 148)
+    assert p["threads"] % 32 == 0 and p["smem_bytes"] <= 227 * 1024
+    p = plan(8192 * 3 + 0, 151936, _lib.KLD_BF16, 148)
+    assert p["tail_rows"] == (8192 * 3) % 148
+    p = plan(148 * 4, 151936, _lib.KLD_F32, 148)
+    assert (p["variant"], p["whole_rounds"], p["tail_rows"]) == (0, 4, 0)
+    # one row more than a wave: that row over as many CTAs as keep >= 10 chunks each
+    p = plan(149, 151936, _lib.KLD_F32, 148)
+    assert (p["variant"], p["whole_rounds"], p["tail_rows"], p["tail_ctas"]) == (2, 1, 1, 29)
+    # few rows: every row split into row-aligned parts, one per CTA
+    p = plan(1, 262144, _lib.KLD_F32, 148)
+    assert (p["variant"], p["whole_rounds"], p["tail_rows"], p["grid"], p["ctas_per_row"]) == (2, 0, 1, 32, 32)
+    p = plan(16, 262144, _lib.KLD_F32, 148)
+    assert (p["grid"], p["ctas_per_row"]) == (144, 9)
+    # between half a wave and a wave, and a large last wave: whole rows
+    assert plan(100, 151936, _lib.KLD_F32, 148)["variant"] == 0
+    p = plan(1000, 151936, _lib.KLD_F32, 148)
+    assert (p["variant"], p["whole_rounds"], p["grid"]) == (0, 7, 148)
     for sms in (1, 8, 132, 148):
-        for n in range(1, 300):
-            p = plan(n, 4096, _lib.KLD_F32, sms)
-            g, per = p["cluster_ctas"], p["ctas_per_row"]
-            assert g in (1, 2, 4, 8) and per % g == 0 and per // g <= 32
-            if p["variant"] == 0:
-                assert per == 1 and g == 1 and p["grid"] == min(n, sms)
-            else:
-                assert 2 * n <= sms and p["grid"] == n * per <= sms and per >= 2
+        for n in list(range(1, 320)) + [1000, 8192, 8193, 32768]:
+            for v in (1, 7, 512, 513, 4096, 70001, 151936):
+                p = plan(n, v, _lib.KLD_F32, sms)
+                assert p["cluster_ctas"] == 1 and p["variant"] in (0, 2) and p["grid"] <= sms
+                if p["tail_rows"]:
+                    # a split last wave of at most sms/2 rows (all rows below one
+                    # wave, then in row-aligned parts), whole rounds before it
+                    assert p["variant"] == 2 and 2 * p["tail_rows"] <= sms
+                    assert p["whole_rounds"] == n // sms and p["tail_rows"] == n % sms
+                    assert p["tail_rows"] <= p["tail_ctas"] <= p["grid"]
+                    if p["whole_rounds"] == 0:
+                        assert p["tail_ctas"] % n == 0 and p["ctas_per_row"] == p["tail_ctas"] // n
+                else:
+                    # whole rows round robin over grid CTAs
+                    assert p["variant"] == 0 and p["whole_rounds"] * p["grid"] >= n
+                    assert (p["whole_rounds"] - 1) * p["grid"] < n
+                if n > 300 and v > 4096:
+                    continue  # the item check below is exhaustive for the small cases
+                items = _tail_ranges(n, v, sms, p)
+                nchv = -(-v // 512)
+                seen = {}
+                for b, its in items.items():
+                    assert len(its) <= p["whole_rounds"] + 2
+                    for r, lo, hi in its:
+                        seen.setdefault(r, []).append((lo, hi, b))
+                assert sorted(seen) == list(range(n))  # every row, once per part
+                for r, parts in seen.items():
+                    parts.sort()
+                    assert parts[0][0] == 0 and parts[-1][1] == nchv
+                    assert all(parts[i][1] == parts[i + 1][0] for i in range(len(parts) - 1))
+                    assert len(parts) <= 32 and len(parts) <= max(1, p["ctas_per_row"])
     lib = _lib.load()
     out = _lib.Plan()
     assert lib.kld_plan(0, 10, 0, 148, ctypes.byref(out)) == _lib.KLD_ERR_INVALID_ARG

@@ -1,11 +1,12 @@
-"""Split-row launches (few rows: each row's chunks spread over thread-block
-clusters of CTAs whose partial sums merge in shared memory, then across
-clusters through global memory) against the fp64 CPU oracle.
+"""Split-row launches (few rows: each row's chunks spread over several CTAs
+whose partial sums merge through global memory, or over thread-block
+clusters whose partials merge in shared memory first) against the fp64 CPU
+oracle.
 
-Rows <= SMs / 2 take this path. By default a row is split over plain CTAs
-(kld_stats_set_split(1)); the cluster shapes (2, 4, 8 CTAs, combined through
-distributed shared memory) and whole-row launches (-1) are selected
-explicitly here. The cases put maxima, ties, NaN, masks and the target token
+Rows fewer than the SMs are all split. By default a row is split over plain
+CTAs by balanced chunk ranges (kld_stats_set_split(1)); the cluster shapes
+(2, 4, 8 CTAs, combined through distributed shared memory) and whole-row
+launches (-1) are selected explicitly here. The cases put maxima, ties, NaN, masks and the target token
 in parts other than the first, leave parts with no chunk at small
 vocabularies, and reuse one handle so that the per-row arrival counters must
 come back to zero after every launch.
@@ -52,7 +53,7 @@ def test_split_rows_full_vocabulary(n, dtype):
     p = st.plan(n, V_FULL, _lib.KLD_F32 if dtype == synth.F32 else _lib.KLD_BF16)
     st.close()
     if 2 * n <= _sm_count():
-        assert p["variant"] == 1 and p["ctas_per_row"] >= 2
+        assert p["variant"] == 2 and p["whole_rounds"] == 0 and p["ctas_per_row"] >= 2
     w = synth.make_recipe("ctx", n=n, v=V_FULL, dtype=dtype, seed=100 + n)
     _parity(w.base, w.quant, w.token_ids, ODT[dtype])
 
