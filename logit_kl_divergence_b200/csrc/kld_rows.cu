@@ -489,36 +489,25 @@ __device__ __forceinline__ void poly_accumulate(const float* b, const f2* X, con
 }
 
 // Log-ratios x = q - b + K of one step, in packed pairs (x = 0 for absent
-// elements), and the largest |x| of the lane (NaN if any x is NaN). `form`
-// (warp-uniform) picks the order of the roundings (ratio_form).
-template <int PE>
+// elements), and the largest |x| of the lane (NaN if any x is NaN). kForm
+// picks the order of the roundings (ratio_form): 0 (q - b) + K, 1
+// (q + K) - b, 2 q - (b - K).
+template <int PE, int kForm>
 __device__ __forceinline__ float log_ratios(const float* b, const float* q, unsigned valid,
-                                            float K, int form, f2* X) {
+                                            float K, f2* X) {
   constexpr int NP = (PE + 1) / 2;
   float ax0 = 0.f, ax1 = 0.f;
   const f2 K2 = splat(K);
-  if (form == 0) {
-#pragma unroll
-    for (int j = 0; j < NP; ++j) {
-      const int i0 = 2 * j, i1 = (2 * j + 1 < PE) ? 2 * j + 1 : 2 * j;
-      X[j] = add2(sub2(pk(q[i0], q[i1]), pk(b[i0], b[i1])), K2);
-    }
-  } else if (form == 1) {
-#pragma unroll
-    for (int j = 0; j < NP; ++j) {
-      const int i0 = 2 * j, i1 = (2 * j + 1 < PE) ? 2 * j + 1 : 2 * j;
-      X[j] = sub2(add2(pk(q[i0], q[i1]), K2), pk(b[i0], b[i1]));
-    }
-  } else {
-#pragma unroll
-    for (int j = 0; j < NP; ++j) {
-      const int i0 = 2 * j, i1 = (2 * j + 1 < PE) ? 2 * j + 1 : 2 * j;
-      X[j] = sub2(pk(q[i0], q[i1]), sub2(pk(b[i0], b[i1]), K2));
-    }
-  }
 #pragma unroll
   for (int j = 0; j < NP; ++j) {
     const int i0 = 2 * j, i1 = (2 * j + 1 < PE) ? 2 * j + 1 : 2 * j;
+    const f2 Q = pk(q[i0], q[i1]), B = pk(b[i0], b[i1]);
+    if (kForm == 1)
+      X[j] = sub2(add2(Q, K2), B);
+    else if (kForm == 2)
+      X[j] = sub2(Q, sub2(B, K2));
+    else
+      X[j] = add2(sub2(Q, B), K2);
     float x0, x1;
     upk(X[j], x0, x1);
     if (((valid >> i0) & 1u) == 0u) x0 = 0.f;
@@ -602,7 +591,13 @@ __device__ __forceinline__ void chunk_step(const float* b, const float* q, unsig
     r.Mb = wmb;
     r.T = wmb + kRaiseMargin;
   }
-  const float axl = log_ratios<PE>(b, q, valid, r.K, kWide ? r.mode : 0, X);
+  float axl;
+  if (!kWide || r.mode == 0)
+    axl = log_ratios<PE, 0>(b, q, valid, r.K, X);
+  else if (r.mode == 1)
+    axl = log_ratios<PE, 1>(b, q, valid, r.K, X);
+  else
+    axl = log_ratios<PE, 2>(b, q, valid, r.K, X);
 
   // The cheapest polynomial tier whose range holds every |x| of the warp's
   // step (a NaN fails every test and takes the direct path).
