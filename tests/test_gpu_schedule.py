@@ -1,8 +1,9 @@
 """The row pass's schedule against the fp64 oracle.
 
-Whole rows go round robin over one CTA per SM; the rows of a last partial
-wave (all rows, below one wave) are split over the CTAs by balanced chunk
-ranges and merged per row; the reduction follows (fixed-order sums, the
+Whole rows go round robin over one CTA per SM; a last partial wave of at
+most SMs/2 rows is split over the CTAs by balanced chunk ranges, fewer rows
+than SMs/2 in all into row-aligned parts, and the parts are merged per row;
+the reduction follows (fixed-order sums, the
 seven order statistics by an exact radix select). The cases sweep row counts
 around multiples of the SM count,
 cover the mid-range counts of scoring 512-token chunks one chunk per row at
