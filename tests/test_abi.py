@@ -167,11 +167,15 @@ def _tail_ranges(n, v, sms, p):
 
 def test_plan_host_logic():
     p = plan(8192, 151936, _lib.KLD_F32, 148)
-    # 55 whole rounds; the 52 rows of the last partial wave split over all SMs
-    assert (p["variant"], p["grid"], p["whole_rounds"], p["tail_rows"], p["tail_ctas"]) == (2, 148, 55, 52, 148)
+    # many whole rounds: the last partial wave takes whole rows too
+    assert (p["variant"], p["grid"], p["whole_rounds"], p["tail_rows"]) == (0, 148, 56, 0)
     assert p["threads"] % 32 == 0 and p["smem_bytes"] <= 227 * 1024
-    p = plan(8192 * 3 + 0, 151936, _lib.KLD_BF16, 148)
-    assert p["tail_rows"] == (8192 * 3) % 148
+    # two whole rounds, then 4 rows split over the SMs
+    p = plan(300, 151936, _lib.KLD_BF16, 148)
+    assert (p["variant"], p["whole_rounds"], p["tail_rows"]) == (2, 2, 4)
+    # three whole rounds: whole rows
+    p = plan(3 * 148 + 5, 151936, _lib.KLD_F32, 148)
+    assert (p["variant"], p["whole_rounds"], p["tail_rows"]) == (0, 4, 0)
     p = plan(148 * 4, 151936, _lib.KLD_F32, 148)
     assert (p["variant"], p["whole_rounds"], p["tail_rows"]) == (0, 4, 0)
     # one row more than a wave: that row over as many CTAs as keep >= 10 chunks each
@@ -192,10 +196,10 @@ def test_plan_host_logic():
                 p = plan(n, v, _lib.KLD_F32, sms)
                 assert p["cluster_ctas"] == 1 and p["variant"] in (0, 2) and p["grid"] <= sms
                 if p["tail_rows"]:
-                    # a split last wave of at most sms/2 rows (all rows below one
-                    # wave, then in row-aligned parts), whole rounds before it
+                    # a split last wave of at most sms/2 rows after at most two
+                    # whole rounds (all rows below one wave: row-aligned parts)
                     assert p["variant"] == 2 and 2 * p["tail_rows"] <= sms
-                    assert p["whole_rounds"] == n // sms and p["tail_rows"] == n % sms
+                    assert p["whole_rounds"] == n // sms <= 2 and p["tail_rows"] == n % sms
                     assert p["tail_rows"] <= p["tail_ctas"] <= p["grid"]
                     if p["whole_rounds"] == 0:
                         assert p["tail_ctas"] % n == 0 and p["ctas_per_row"] == p["tail_ctas"] // n
