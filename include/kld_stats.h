@@ -59,7 +59,7 @@
 extern "C" {
 #endif
 
-#define KLD_ABI_VERSION 3
+#define KLD_ABI_VERSION 4
 
 typedef enum {
   KLD_OK = 0,
@@ -143,8 +143,10 @@ const char* kld_last_cuda_error(void);
  * Create a handle on `device` for runs of up to `max_rows` rows.
  * Allocates a device workspace of max_rows records (40 bytes each), the
  * per-field arrays of kld_stats_rows (24 bytes per row), the per-row
- * normalisers of the gradient and top-k passes (48 bytes per row) plus a few
- * KB, and a pinned host copy of the result. Returns KLD_ERR_NO_DEVICE if the
+ * normalisers of the gradient and top-k passes (64 bytes per row) plus a few
+ * KB, and a pinned host copy of the result. The first kld_stats_run_topk on
+ * rows of more than 4096 elements adds the top-k scan's workspace (about
+ * 200 KB per row of max_rows). Returns KLD_ERR_NO_DEVICE if the
  * device is not a compute-capability 10.0 (B200-class) GPU.
  */
 kld_status_t kld_stats_create(kld_stats_t* out, int64_t max_rows, int device);
@@ -153,10 +155,12 @@ kld_status_t kld_stats_create(kld_stats_t* out, int64_t max_rows, int device);
 void kld_stats_destroy(kld_stats_t h);
 
 /*
- * The whole statistic for rows [0, N) in one kernel: the fused row pass,
- * whose last CTA to finish then performs the fixed-order reduction and the
- * exact percentile selection and writes the result straight into the
- * handle's pinned host buffer (read it with kld_stats_result).
+ * The whole statistic for rows [0, N): the fused row pass, then the
+ * fixed-order reduction and the exact percentile selection, which writes the
+ * result straight into the handle's pinned host buffer (read it with
+ * kld_stats_result). A launch whose rows are all split over several CTAs
+ * (at most 32 rows, fewer than half the SMs) reduces its own records at the
+ * end of the row pass and needs no second kernel.
  * token_ids (device, int32[N]) may be NULL: no NLL/PPL.
  * 1 <= N <= max_rows, 1 <= V <= 2^31-1. Asynchronous.
  */
@@ -323,13 +327,18 @@ kld_status_t kld_stats_merge_partials(kld_stats_t h, const void* parts, int G, i
  *   kl_out[r]         sum_{T} p log(p/r) + p_rest log(p_rest/r_rest) (double)
  * with p = softmax(base), r = softmax(quant). Rows the statistics exclude get
  * idx -1 and NaN. idx_out, logp_out and rest_out may be NULL; all are
- * caller-owned DEVICE memory, naturally aligned. Enqueues the row pass, the
- * reduction (read with kld_stats_result) and a top-k pass. The top-k pass
- * derives a threshold from a sample of each base row, then reads both rows
- * once, collecting the elements above the threshold and summing the rest
- * masses of all others in the same sweep. Rows whose threshold holds fewer
- * than k or too many elements (large tie groups, masked rows) fall back to
- * an exact radix selection that reads the base row 2-4 times.
+ * caller-owned DEVICE memory, naturally aligned. For V > 4096 it enqueues
+ * a threshold kernel (a base threshold per row from 4096 samples, with
+ * comfortably more than k elements at or above it), the row pass in its
+ * top-k scan form (it also copies out the 16-element lanes that hold an
+ * element at or above the threshold, about 5 % of the row, and sums the
+ * rest masses of all other lanes), the reduction (read with
+ * kld_stats_result) and the top-k pass, which selects T in the copies: each
+ * logit is read from memory once. For V <=
+ * 4096 the top-k pass reads both rows once after the row pass instead.
+ * Rows whose threshold holds fewer than k or too many elements (large tie
+ * groups, masked rows) fall back to an exact radix selection that reads
+ * the base row 2-4 times.
  */
 #define KLD_MAX_TOPK 1024
 kld_status_t kld_stats_run_topk(kld_stats_t h, const void* base, const void* quant,
@@ -388,13 +397,24 @@ kld_status_t kld_selftest_bounded_wait(int device, uint64_t limit_ns, int use_ab
                                        uint64_t* waited_ns);
 
 /*
- * Duration in milliseconds of the second streaming pass of the last
+ * Duration in milliseconds of the second pass of the last
  * kld_stats_run_grad (the gradient pass) or kld_stats_run_topk (the top-k
- * pass), the pass that follows the reduction; timing enabled by
- * kld_stats_set_timing; waits for that run. KLD_ERR_NOT_READY when the last
- * run had no such pass or was not timed.
+ * pass that follows the reduction, plus the threshold kernel before the row
+ * pass when there is one); timing enabled by kld_stats_set_timing; waits for
+ * that run. KLD_ERR_NOT_READY when the last run had no such pass or was not
+ * timed.
  */
 kld_status_t kld_stats_second_pass_timing(kld_stats_t h, float* pass_ms);
+
+/*
+ * Rows of the last kld_stats_run_topk that took the exact path (a radix
+ * selection that reads the base row 2-4 times) instead of the threshold's
+ * fast path: large tie groups at the threshold, masked rows, or a scanned
+ * row whose flagged chunks overflowed the scan's lists (rows of more than
+ * 512 * 16 * 64 elements only). Waits for that run. KLD_ERR_NOT_READY if
+ * the handle has run no top-k yet.
+ */
+kld_status_t kld_stats_topk_exact_rows(kld_stats_t h, int64_t* rows);
 
 /*
  * Read-bandwidth probe, a measuring aid with no counterpart in the

@@ -158,9 +158,18 @@ class KLDStats:
         _lib.check(st, "kld_stats_run_topk")
         return out
 
+    def topk_exact_rows(self) -> int:
+        """Rows of the last run_topk that took the exact path instead of the
+        threshold's fast path (waits for that run)."""
+        n = ctypes.c_int64()
+        _lib.check(self._lib.kld_stats_topk_exact_rows(self._h, ctypes.byref(n)),
+                   "kld_stats_topk_exact_rows")
+        return n.value
+
     def second_pass_timing(self) -> float:
-        """Milliseconds of the second streaming pass of the last run_grad
-        (the gradient pass) or run_topk (the top-k pass); timing enabled."""
+        """Milliseconds of the second pass of the last run_grad (the gradient
+        pass) or run_topk (the top-k pass, with its threshold kernel when the
+        row pass scanned); timing enabled."""
         ms = ctypes.c_float()
         _lib.check(self._lib.kld_stats_second_pass_timing(self._h, ctypes.byref(ms)),
                    "kld_stats_second_pass_timing")

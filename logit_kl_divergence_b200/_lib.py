@@ -119,6 +119,7 @@ SIGNATURES = {
     "kld_stats_set_split": (_ST, [_P, _I32]),
     "kld_stats_run_grad": (_ST, [_P, _P, _P, _P, _I64, _I64, _I32, _P, _I32, ctypes.c_double, _P]),
     "kld_stats_second_pass_timing": (_ST, [_P, ctypes.POINTER(ctypes.c_float)]),
+    "kld_stats_topk_exact_rows": (_ST, [_P, ctypes.POINTER(ctypes.c_int64)]),
     "kld_stats_read_probe": (_ST, [_P, _P, _P, _I64, _P]),
     "kld_selftest_bounded_wait": (_ST, [_I32, ctypes.c_uint64, _I32, ctypes.POINTER(ctypes.c_uint64)]),
     "kld_stats_run_topk": (_ST, [_P, _P, _P, _P, _I64, _I64, _I32, _I32, _P, _P, _P, _P, _P]),

@@ -75,7 +75,10 @@ struct kld_stats_s {
   kld::RowAux* aux = nullptr;  // per-row normalisers for the gradient and top-k passes
   bool grad_timing_valid = false;
   kld::SplitScratch split = {nullptr, nullptr, 0, kld::kDefaultClusterCtas};
-  uint32_t* derr = nullptr;
+  uint32_t* derr = nullptr;  // the device error word, then the top-k exact-path row count
+  unsigned long long* topk_exact = nullptr;
+  cudaEvent_t topk_done = nullptr;  // after the last top-k pass
+  bool has_topk = false;
   kld_result_t* hres = nullptr;      // pinned, mapped host memory
   kld_result_t* hres_dev = nullptr;  // its device-side pointer
   cudaEvent_t done = nullptr;
@@ -84,7 +87,12 @@ struct kld_stats_s {
   bool timing = false;
   bool timing_valid = false;
   bool rows_pending = false;  // a timed kld_stats_run_rows awaits its reduction
-  cudaEvent_t tev[4] = {nullptr, nullptr, nullptr, nullptr};
+  // row pass start / end, reduction end, second pass end, top-k threshold start
+  cudaEvent_t tev[5] = {nullptr, nullptr, nullptr, nullptr, nullptr};
+  bool threshold_timed = false;  // the last timed second pass had a threshold kernel
+  // top-k scan workspace (kld::TopkScan), allocated by the first scanned run_topk
+  void* topk_mem = nullptr;
+  kld::TopkScan topk_scan = {nullptr, nullptr, nullptr};
   // host path
   cudaStream_t copy_stream = nullptr;
   cudaEvent_t copied[2] = {nullptr, nullptr};
@@ -134,13 +142,13 @@ kld_status_t enqueue_reduce(kld_stats_t h, const kld_row_t* rows, int64_t N, int
 // pass (nullable).
 kld_status_t run_statistic(kld_stats_t h, const void* base, const void* quant, const int32_t* tok,
                            int64_t N, int64_t V, kld_dtype_t dtype, cudaStream_t s,
-                           kld::RowAux* aux) {
+                           kld::RowAux* aux, const kld::TopkScan* topk = nullptr) {
   h->timing_valid = h->timing;
   h->rows_pending = false;
   if (h->timing) KLD_CUDA(cudaEventRecord(h->tev[0], s));
   bool reduced = false;
   KLD_CUDA(kld::launch_rows(base, quant, tok, N, V, dtype, h->rows, h->derr, h->sm_count,
-                            &h->split, aux, s, nullptr, 0, h->hres_dev, &reduced));
+                            &h->split, aux, s, nullptr, 0, h->hres_dev, &reduced, topk));
   if (h->timing) KLD_CUDA(cudaEventRecord(h->tev[1], s));
   h->last_rows = N;
   h->last_stream = s;
@@ -236,10 +244,13 @@ kld_status_t kld_stats_create(kld_stats_t* out, int64_t max_rows, int device) {
     h->soa_nll = h->soa_kld + max_rows;
     h->soa_amax_b = reinterpret_cast<int32_t*>(h->soa_nll + max_rows);
     h->soa_amax_q = h->soa_amax_b + max_rows;
-    if ((err = cudaMalloc(&h->derr, sizeof(uint32_t))) != cudaSuccess) {
+    if ((err = cudaMalloc(&h->derr, 16)) != cudaSuccess) {
       st = cuda_fail(err, "cudaMalloc(error word)"); break; }
-    if ((err = cudaMemset(h->derr, 0, sizeof(uint32_t))) != cudaSuccess) {
+    if ((err = cudaMemset(h->derr, 0, 16)) != cudaSuccess) {
       st = cuda_fail(err, "cudaMemset"); break; }
+    h->topk_exact = reinterpret_cast<unsigned long long*>(reinterpret_cast<char*>(h->derr) + 8);
+    if ((err = cudaEventCreateWithFlags(&h->topk_done, cudaEventDisableTiming)) != cudaSuccess) {
+      st = cuda_fail(err, "cudaEventCreate"); break; }
     {
       // Split-row scratch (see kld::SplitScratch): partial slots and a
       // ticket for each of up to SMs split rows, plus the few-row launch
@@ -263,7 +274,7 @@ kld_status_t kld_stats_create(kld_stats_t* out, int64_t max_rows, int device) {
         cudaSuccess) { st = cuda_fail(err, "cudaHostGetDevicePointer"); break; }
     if ((err = cudaEventCreateWithFlags(&h->done, cudaEventDisableTiming)) != cudaSuccess) {
       st = cuda_fail(err, "cudaEventCreate"); break; }
-    for (int i = 0; i < 4 && st == KLD_OK; ++i)
+    for (int i = 0; i < 5 && st == KLD_OK; ++i)
       if ((err = cudaEventCreate(&h->tev[i])) != cudaSuccess) st = cuda_fail(err, "cudaEventCreate");
   } while (0);
   if (st != KLD_OK) {
@@ -286,15 +297,20 @@ void kld_stats_destroy(kld_stats_t h) {
     if (h->freed[i]) cudaEventDestroy(h->freed[i]);
   }
   if (h->copy_stream) cudaStreamDestroy(h->copy_stream);
-  for (int i = 0; i < 4; ++i)
+  for (int i = 0; i < 5; ++i)
     if (h->tev[i]) cudaEventDestroy(h->tev[i]);
   if (h->done) cudaEventDestroy(h->done);
+  if (h->topk_done) {
+    if (h->has_topk) cudaEventSynchronize(h->topk_done);
+    cudaEventDestroy(h->topk_done);
+  }
   if (h->hres) cudaFreeHost(h->hres);
   if (h->derr) cudaFree(h->derr);
   if (h->rows) cudaFree(h->rows);
   if (h->soa_kld) cudaFree(h->soa_kld);
   if (h->split_mem) cudaFree(h->split_mem);
   if (h->aux) cudaFree(h->aux);
+  if (h->topk_mem) cudaFree(h->topk_mem);
   delete h;
 }
 
@@ -313,6 +329,7 @@ kld_status_t kld_stats_run_rows(kld_stats_t h, const void* base, const void* qua
   h->timing_valid = h->timing;
   h->rows_pending = h->timing;
   h->grad_timing_valid = false;
+  h->threshold_timed = false;
   if (h->timing) KLD_CUDA(cudaEventRecord(h->tev[0], s));
   KLD_CUDA(launch_rows(h, base, quant, token_ids, N, V, dtype, rows_out ? rows_out : h->rows, s));
   if (h->timing) KLD_CUDA(cudaEventRecord(h->tev[1], s));
@@ -338,6 +355,7 @@ kld_status_t kld_stats_reduce(kld_stats_t h, const kld_row_t* rows_dev, int64_t 
   h->timing_valid = h->timing_valid && h->rows_pending;
   h->rows_pending = false;
   h->grad_timing_valid = false;
+  h->threshold_timed = false;
   return enqueue_reduce(h, rows_dev ? rows_dev : h->rows, N, has_nll ? 1 : 0,
                         static_cast<cudaStream_t>(stream));
 }
@@ -352,6 +370,7 @@ kld_status_t kld_stats_run(kld_stats_t h, const void* base, const void* quant,
   DeviceGuard guard(h->device);
   if (!guard.ok()) return cuda_fail(cudaGetLastError(), "cudaSetDevice");
   h->grad_timing_valid = false;
+  h->threshold_timed = false;
   return run_statistic(h, base, quant, token_ids, N, V, dtype, static_cast<cudaStream_t>(stream),
                        nullptr);
 }
@@ -370,6 +389,7 @@ kld_status_t kld_stats_run_grad(kld_stats_t h, const void* base, const void* qua
   if (!guard.ok()) return cuda_fail(cudaGetLastError(), "cudaSetDevice");
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   h->grad_timing_valid = h->timing;
+  h->threshold_timed = false;
   st = run_statistic(h, base, quant, token_ids, N, V, dtype, s, h->aux);
   if (st != KLD_OK) return st;
   KLD_CUDA(kld::launch_grad(base, quant, h->aux, N, V, dtype, grad, grad_dtype,
@@ -393,6 +413,7 @@ kld_status_t kld_stats_run_partials(kld_stats_t h, const void* base, const void*
   h->timing_valid = false;
   h->rows_pending = false;
   h->grad_timing_valid = false;
+  h->threshold_timed = false;
   KLD_CUDA(kld::launch_rows(base, quant, token_ids, N, V, dtype, h->rows, h->derr, h->sm_count,
                             &h->split, nullptr, s, parts_out, col_offset));
   return KLD_OK;
@@ -410,6 +431,7 @@ kld_status_t kld_stats_merge_partials(kld_stats_t h, const void* parts, int G, i
   h->timing_valid = false;
   h->rows_pending = false;
   h->grad_timing_valid = false;
+  h->threshold_timed = false;
   KLD_CUDA(kld::launch_merge(parts, G, N, token_ids, V_total, h->rows, s));
   h->last_rows = N;
   h->last_stream = s;
@@ -431,12 +453,42 @@ kld_status_t kld_stats_run_topk(kld_stats_t h, const void* base, const void* qua
   DeviceGuard guard(h->device);
   if (!guard.ok()) return cuda_fail(cudaGetLastError(), "cudaSetDevice");
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  // Rows longer than the top-k pass's candidate capacity: a threshold per
+  // row first, so that the row pass can list the lanes holding candidates.
+  const bool scan = V > kld::kTopkCap;
+  if (scan && !h->topk_mem) {
+    // Synchronises the device once (the first scanned call of the handle).
+    auto up = [](size_t b) { return (b + 255) & ~static_cast<size_t>(255); };
+    const size_t rows = static_cast<size_t>(h->max_rows);
+    const size_t tf_b = up(rows * sizeof(float));
+    const size_t rg_b = up(rows * kld::kConsumerWarps * kld::kRegionVecs * sizeof(uint4));
+    const size_t ct_b = up(rows * kld::kConsumerWarps * sizeof(int));
+    const cudaError_t err = cudaMalloc(&h->topk_mem, tf_b + rg_b + ct_b);
+    if (err != cudaSuccess) {
+      h->topk_mem = nullptr;
+      return cuda_fail(err, "cudaMalloc(top-k scan)");
+    }
+    char* m = static_cast<char*>(h->topk_mem);
+    h->topk_scan.tf = reinterpret_cast<const float*>(m);
+    h->topk_scan.regions = reinterpret_cast<uint4*>(m + tf_b);
+    h->topk_scan.counts = reinterpret_cast<int*>(m + tf_b + rg_b);
+  }
   h->grad_timing_valid = h->timing;
-  st = run_statistic(h, base, quant, token_ids, N, V, dtype, s, h->aux);
+  h->threshold_timed = h->timing && scan;
+  if (scan) {
+    if (h->timing) KLD_CUDA(cudaEventRecord(h->tev[4], s));
+    KLD_CUDA(kld::launch_topk_threshold(base, N, V, dtype, k, const_cast<float*>(h->topk_scan.tf),
+                                        h->sm_count, s));
+  }
+  st = run_statistic(h, base, quant, token_ids, N, V, dtype, s, h->aux,
+                     scan ? &h->topk_scan : nullptr);
   if (st != KLD_OK) return st;
+  KLD_CUDA(cudaMemsetAsync(h->topk_exact, 0, sizeof(unsigned long long), s));
   KLD_CUDA(kld::launch_topk(base, quant, h->aux, N, V, dtype, k, idx_out, logp_out, rest_out,
-                            kl_out, h->sm_count, s));
+                            kl_out, h->sm_count, s, scan ? &h->topk_scan : nullptr, h->topk_exact));
   if (h->timing) KLD_CUDA(cudaEventRecord(h->tev[3], s));
+  KLD_CUDA(cudaEventRecord(h->topk_done, s));
+  h->has_topk = true;
   return KLD_OK;
 }
 
@@ -483,6 +535,23 @@ kld_status_t kld_stats_second_pass_timing(kld_stats_t h, float* pass_ms) {
   if (!guard.ok()) return cuda_fail(cudaGetLastError(), "cudaSetDevice");
   KLD_CUDA(cudaEventSynchronize(h->tev[3]));
   KLD_CUDA(cudaEventElapsedTime(pass_ms, h->tev[2], h->tev[3]));
+  if (h->threshold_timed) {
+    float t = 0.f;
+    KLD_CUDA(cudaEventElapsedTime(&t, h->tev[4], h->tev[0]));
+    *pass_ms += t;
+  }
+  return KLD_OK;
+}
+
+kld_status_t kld_stats_topk_exact_rows(kld_stats_t h, int64_t* rows) {
+  if (!h || !rows) return KLD_ERR_INVALID_ARG;
+  if (!h->has_topk) return KLD_ERR_NOT_READY;
+  DeviceGuard guard(h->device);
+  if (!guard.ok()) return cuda_fail(cudaGetLastError(), "cudaSetDevice");
+  KLD_CUDA(cudaEventSynchronize(h->topk_done));
+  unsigned long long n = 0;
+  KLD_CUDA(cudaMemcpy(&n, h->topk_exact, sizeof(n), cudaMemcpyDeviceToHost));
+  *rows = static_cast<int64_t>(n);
   return KLD_OK;
 }
 
@@ -537,6 +606,7 @@ kld_status_t kld_stats_set_timing(kld_stats_t h, int enable) {
   h->timing_valid = false;
   h->rows_pending = false;
   h->grad_timing_valid = false;
+  h->threshold_timed = false;
   return KLD_OK;
 }
 
@@ -592,6 +662,7 @@ kld_status_t host_rows(kld_stats_t h, const void* base_host, const void* quant_h
   h->timing_valid = false;
   h->rows_pending = false;
   h->grad_timing_valid = false;
+  h->threshold_timed = false;
   const char* hb = static_cast<const char*>(base_host);
   const char* hq = static_cast<const char*>(quant_host);
   const int64_t nchunks = (N + chunk - 1) / chunk;

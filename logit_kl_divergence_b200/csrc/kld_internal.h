@@ -63,7 +63,7 @@ inline int elem_bytes(kld_dtype_t dt) { return dt == KLD_F32 ? 4 : 2; }
 constexpr float kShiftForm = 8.0f;
 
 // Per-row normalisers the row pass leaves for the gradient and top-k passes
-// (48 bytes; the first 16 are read as a float4 by the gradient pass).
+// (64 bytes; the first 16 are read as a float4 by the gradient pass).
 struct RowAux {
   float Fb, mb, Fq, mq;  // softmax(b)_j = 2^(b_j L - Fb) mb, softmax(q)_j likewise;
                          // Fb NaN on rows excluded from the statistics
@@ -72,8 +72,56 @@ struct RowAux {
   float K;               // centre of the log-ratio x = q - b + K
   uint32_t flags;        // the row's KLD_ROW_* flags
   uint64_t pad;
+  // Top-k scan launches only (TopkScan), else 0: softmax(b) and softmax(q)
+  // summed over the elements of the lanes the scan left unflagged.
+  double rest_b, rest_q;
 };
-static_assert(sizeof(RowAux) == 48, "RowAux layout");
+static_assert(sizeof(RowAux) == 64, "RowAux layout");
+
+// Where a row's elements lie for the row pass: `head` elements before the
+// row's first 16-byte boundary, a 16-byte-aligned body of `body` elements
+// streamed in chunks of kChunkElems, then `tail` elements (the head and
+// tail are read apart, < 16 bytes each). Inside the body, element i < 16 of
+// lane l in chunk c is at c * kChunkElems + ((i / E) * 32 + l) * E + i % E,
+// E = 16 / (element bytes): each lane reads 16-byte vectors, a warp 512
+// contiguous bytes per vector step.
+struct RowSpan {
+  int64_t head, body, tail;
+};
+__host__ __device__ __forceinline__ RowSpan row_span(const void* row, int64_t V, int eb) {
+  RowSpan g;
+  const uint32_t mis = static_cast<uint32_t>(reinterpret_cast<uintptr_t>(row) & 15u);
+  g.head = static_cast<int64_t>(((16u - mis) & 15u) / static_cast<uint32_t>(eb));
+  if (g.head > V) g.head = V;
+  const int64_t e = 16 / eb;
+  g.body = ((V - g.head) / e) * e;
+  g.tail = V - g.head - g.body;
+  return g;
+}
+
+// Top-k scan of the row pass (launch_rows with `topk` set; whole rows
+// only), for a threshold tf[r] on the base logits of row r. In every chunk a
+// consumer warp streams, each lane whose 16 elements hold a base logit >=
+// tf[r] copies them, both rows' 16-byte vectors as they sit in shared
+// memory, to its warp's region of kCopyCap lane records, and notes the
+// chunk and lane in ids; every lane of a chunk that takes the direct path
+// of the log-ratio sums does the same. The other lanes add their elements'
+// softmax weights to rest sums, which go to RowAux.rest_b / rest_q (as
+// shares of softmax(b) and softmax(q)). counts[r][w]: the lanes warp w
+// copied (it runs on past kCopyCap; the top-k pass then takes that row by
+// its exact path). So the top-k pass reads the copies and the row's head
+// and tail, never the rows again.
+constexpr int kCopyCap = 96;
+constexpr int kCopyVecs = 8;  // 16-byte vectors of a lane record: both rows' 16 elements (fp32)
+// One warp's region of one row: kCopyCap records, then their kCopyCap ids
+// (chunk index in the body * 32 + lane), in 16-byte vectors.
+constexpr int kRegionVecs = kCopyCap * kCopyVecs + kCopyCap / 4;
+static_assert(kCopyCap % 4 == 0, "ids pack four to a vector");
+struct TopkScan {
+  const float* tf;  // [N]
+  uint4* regions;   // [N][kConsumerWarps][kRegionVecs]: records (b vectors, then q vectors), ids
+  int* counts;      // [N][kConsumerWarps]
+};
 
 // Launchers (defined in the .cu files). They enqueue on `stream` and return
 // the launch error.
@@ -97,7 +145,16 @@ cudaError_t launch_rows(const void* base, const void* quant,
                         int sm_count, const SplitScratch* split, RowAux* aux,
                         cudaStream_t stream, void* part_out = nullptr,
                         int64_t col_offset = 0, kld_result_t* result_out = nullptr,
-                        bool* reduced = nullptr);
+                        bool* reduced = nullptr, const TopkScan* topk = nullptr);
+
+// The row pass with the top-k scan (TopkScan; whole rows, aux required):
+// what launch_rows does when given `topk`. prepare_rows_scan_kernels: its
+// per-device attribute setup (called by prepare_rows_kernels).
+cudaError_t launch_rows_scan(const void* base, const void* quant, const int32_t* token_ids,
+                             int64_t N, int64_t V, kld_dtype_t dtype, kld_row_t* rows,
+                             uint32_t* derr, int sm_count, RowAux* aux, const TopkScan& topk,
+                             cudaStream_t stream);
+cudaError_t prepare_rows_scan_kernels();
 
 // Records from the G vocabulary-slice partials of each row (parts: [G][N]
 // 64-byte partials, rank/slice order), tokens checked against V_total.
@@ -135,10 +192,23 @@ cudaError_t launch_grad(const void* base, const void* quant, const RowAux* aux, 
 
 // Top-k compression of the base rows and KL of the quant rows against it
 // (k <= kMaxTopk), from the row pass's RowAux; idx, logp, rest nullable.
+// scan (nullable): the row pass ran the top-k scan with these thresholds
+// (from launch_topk_threshold), so only the flagged lanes are read back.
+// exact_rows (nullable): counts the rows that took the exact path.
+// Rows of at most kTopkCap elements take no threshold (every element is a
+// candidate) and no scan.
 constexpr int kMaxTopk = 1024;
+constexpr int kTopkCap = 4096;
 cudaError_t launch_topk(const void* base, const void* quant, const RowAux* aux, int64_t N,
                         int64_t V, kld_dtype_t dtype, int k, int32_t* idx, float* logp,
-                        float* rest, double* kl, int sm_count, cudaStream_t stream);
+                        float* rest, double* kl, int sm_count, cudaStream_t stream,
+                        const TopkScan* scan = nullptr,
+                        unsigned long long* exact_rows = nullptr);
+// Per-row base thresholds for the top-k scan: tf[r] from 4096 samples of
+// row r, with comfortably more than k but (by the samples) at most
+// kTopkCap elements at or above it.
+cudaError_t launch_topk_threshold(const void* base, int64_t N, int64_t V, kld_dtype_t dtype,
+                                  int k, float* tf, int sm_count, cudaStream_t stream);
 
 // Bounded-wait self-test (see kld_selftest_bounded_wait).
 cudaError_t launch_wait_selftest(uint64_t limit_ns, int use_abort, uint32_t* derr,

@@ -12,13 +12,18 @@
 // x_j = q_j - b_j + K formed as the row pass forms it (kShiftForm), the
 // rest in fp64.
 //
-// One CTA per row (persistent over rows, four per SM). Fast path: 4096
+// One CTA per row (persistent over rows, three per SM). Fast path: 4096
 // samples of the base row (512 evenly spaced runs of 8 adjacent elements,
 // one memory sector each) give a threshold key t0 (the m-th
 // largest sample, m ~ 1.5 k * 4096 / V + 8, to 21 bits by two 11-bit
-// histogram levels), and one fused pass over both rows appends
-// every element with key >= t0 to a shared candidate list and sums the rest
-// masses of all other elements: each logit is read once. If fewer than k or
+// histogram levels), and every element with key >= t0 goes to a shared
+// candidate list, every other one to the rest masses. For rows of more than
+// kCap elements the thresholds come first (kld_topk_threshold_kernel), and
+// the row pass, in its top-k scan form, copies out the 16-element lanes
+// that hold such an element and sums the rest masses of all others
+// (TopkScan): this pass then reads only the copies (copied_pass), and each
+// logit is read from memory once in all. Without a scan, one fused pass
+// over both rows here (gather_pass) does the same. If fewer than k or
 // more than kCap elements pass the threshold (ties or extreme rows), an exact
 // path takes the row instead: an MSB radix select over order-preserving
 // 32-bit keys (11/11/10-bit levels, stopping as soon as the candidates fit
@@ -26,9 +31,9 @@
 // lowest indices in it by a radix select over the index), the candidates,
 // and a last pass for the rest masses (the row is read 2-4 times). T is the
 // first k candidates by (key desc, index asc): ranked by counting when there
-// are at most kRankMax of them (the fast path's usual few hundred; with many
-// more than k, a histogram of the candidates' keys first leaves only those
-// in or above the bin of the k-th largest to be ranked), else by a bitonic
+// are at most kRankMax of them (the fast path's usual few hundred; with more
+// than kRankDirect, a histogram of the candidates' keys first leaves only
+// those in or above the bin of the k-th largest to be ranked), else by a bitonic
 // sort in shared memory; candidates beyond T join the rest.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -42,11 +47,12 @@ namespace {
 
 constexpr int kTopkThreads = 256;
 constexpr int kTopkWarps = kTopkThreads / 32;
-constexpr int kTopkCtasPerSm = 4;
+constexpr int kTopkCtasPerSm = 3;  // 85 registers a thread: the copies' loads stay in flight
 constexpr int kHistBins = 2048;
-constexpr int kCap = 4096;  // candidates sorted in shared memory
+constexpr int kCap = kTopkCap;  // candidates sorted in shared memory
 constexpr int kSample = 4096;  // samples of a row for the threshold
 constexpr int kRankMax = 1536;  // at most this many candidates: rank by counting
+constexpr int kRankDirect = 768;  // up to this many: rank all against all (else a histogram first)
 constexpr int kSetBase = 2048;  // where the boundary set of the ranking is kept in cand[]
 static_assert(kSetBase >= kRankMax && kSetBase + kRankMax <= kCap, "boundary set layout");
 constexpr float kL = 1.4426950408889634f;  // log2(e) rounded to fp32, as the row pass
@@ -89,6 +95,7 @@ struct TopkShared {
   int ncand;
   int nset;
   unsigned sel[3];  // bin, count above it, count in it
+  int fcnt[kConsumerWarps];  // scanned rows: lanes copied by each consumer warp of the row pass
 };
 
 // Block-wide: the bin holding the `need`-th element counting from the top
@@ -306,10 +313,101 @@ __device__ void gather_pass(TopkShared& sh, const char* rb, const char* rq, int6
   }
 }
 
+// Rows the row pass scanned (TopkScan): the same split into candidates and
+// rest as gather_pass, over the lane records the row pass copied and the
+// row's head and tail; the rest masses of all other elements come with the
+// row (RowAux.rest_b, rest_q). Every thread takes whole lane records; a
+// warp's records are contiguous, so the loads coalesce. False (for the
+// whole block, before anything is taken) if a consumer warp copied more
+// lanes than its region holds: the row then reads both rows once
+// (gather_pass) with the same threshold.
+template <int DT>
+__device__ bool copied_pass(TopkShared& sh, const char* rb, const char* rq, int64_t V,
+                            uint32_t t0, const RowAux& a, const uint4* regions, const int* cnt,
+                            double& prest, double& rrest) {
+  const int tid = threadIdx.x;
+  constexpr int EB = DT == KLD_F32 ? 4 : 2;
+  constexpr int E = 16 / EB;        // elements per 16-byte vector
+  constexpr int VPC = 16 / E;       // vectors per lane and row
+  if (tid < kConsumerWarps) sh.fcnt[tid] = cnt[tid];
+  __syncthreads();
+  bool over = false;
+#pragma unroll
+  for (int w = 0; w < kConsumerWarps; ++w) over |= sh.fcnt[w] > kCopyCap;
+  if (over) return false;
+  auto take = [&](float bj, int64_t j, float qj, float& sp, float& sr) {
+    const uint32_t key = okey(bj);
+    if (key >= t0) {
+      const int pos = atomicAdd(&sh.ncand, 1);
+      if (pos < kCap)
+        sh.cand[pos] = (static_cast<unsigned long long>(key) << 32) | (0xffffffffu - static_cast<uint32_t>(j));
+    } else {
+      sp += rest_b(bj, a);
+      sr += rest_q(qj, a);
+    }
+  };
+  const RowSpan g = row_span(rb, V, EB);
+  // head and tail (< 16 bytes each)
+  const int n_extra = static_cast<int>(g.head + g.tail);
+  if (tid < n_extra) {
+    const int64_t j = tid < g.head ? tid : g.head + g.body + (tid - g.head);
+    float sp = 0.f, sr = 0.f;
+    take(load_el<DT>(rb, j), j, load_el<DT>(rq, j), sp, sr);
+    prest += static_cast<double>(sp);
+    rrest += static_cast<double>(sr);
+  }
+  for (int i = tid; i < kConsumerWarps * kCopyCap; i += kTopkThreads) {
+    const int w = i / kCopyCap, e = i % kCopyCap;
+    if (e >= sh.fcnt[w]) continue;
+    const uint4* reg = regions + w * kRegionVecs;
+    const uint32_t id = reinterpret_cast<const uint32_t*>(reg + kCopyCap * kCopyVecs)[e];
+    const uint4* rec = reg + e * kCopyVecs;
+    uint4 xb[VPC], xq[VPC];
+#pragma unroll
+    for (int k = 0; k < VPC; ++k) {
+      xb[k] = rec[k];
+      xq[k] = rec[VPC + k];
+    }
+    const int64_t chunk = id >> 5;
+    const int ln = static_cast<int>(id & 31u);
+    float sp = 0.f, sr = 0.f;
+#pragma unroll
+    for (int k = 0; k < VPC; ++k) {
+      const int64_t off = chunk * kChunkElems + static_cast<int64_t>(k * 32 + ln) * E;
+      if (off >= g.body) break;
+      float fb[E], fq[E];
+      const uint32_t wb[4] = {xb[k].x, xb[k].y, xb[k].z, xb[k].w};
+      const uint32_t wq[4] = {xq[k].x, xq[k].y, xq[k].z, xq[k].w};
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        if (DT == KLD_F32) {
+          fb[u] = __uint_as_float(wb[u]);
+          fq[u] = __uint_as_float(wq[u]);
+        } else if (DT == KLD_BF16) {
+          fb[2 * u] = __uint_as_float(wb[u] << 16);
+          fb[2 * u + 1] = __uint_as_float(wb[u] & 0xffff0000u);
+          fq[2 * u] = __uint_as_float(wq[u] << 16);
+          fq[2 * u + 1] = __uint_as_float(wq[u] & 0xffff0000u);
+        } else {
+          fb[2 * u] = __half2float(__ushort_as_half(static_cast<unsigned short>(wb[u] & 0xffffu)));
+          fb[2 * u + 1] = __half2float(__ushort_as_half(static_cast<unsigned short>(wb[u] >> 16)));
+          fq[2 * u] = __half2float(__ushort_as_half(static_cast<unsigned short>(wq[u] & 0xffffu)));
+          fq[2 * u + 1] = __half2float(__ushort_as_half(static_cast<unsigned short>(wq[u] >> 16)));
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < E; ++u) take(fb[u], g.head + off + u, fq[u], sp, sr);
+    }
+    prest += static_cast<double>(sp);
+    rrest += static_cast<double>(sr);
+  }
+  return true;
+}
+
 // The first kt of the n (unique) candidates in descending order, by counting
 // for each candidate how many are larger: for the few hundred candidates of
 // the fast path this beats a bitonic network and its barriers. When there
-// are many more candidates than kt, a histogram of their keys above t0 first
+// are more than kRankDirect candidates, a histogram of their keys above t0 first
 // finds the bin that holds the kt-th largest: every candidate below that bin
 // is outside T, and only the ones in it or above (about kt) are ranked
 // against each other. T goes to sh.cand[kCap .. kCap + kt) (the sorted list
@@ -326,7 +424,7 @@ __device__ void rank_select(TopkShared& sh, int n, int kt, uint32_t t0, const ch
   };
   const unsigned long long* set = sh.cand;
   int ns = n;
-  if (n > 2 * kt + 64) {
+  if (n > kRankDirect) {
     // digit = (key - t0) >> s over 2048 bins, s from the largest key
     unsigned mx = 0u;
     for (int e = tid; e < n; e += kTopkThreads)
@@ -485,7 +583,9 @@ __global__ void __launch_bounds__(kTopkThreads, kTopkCtasPerSm)
     kld_topk_kernel(const void* __restrict__ base, const void* __restrict__ quant,
                     const RowAux* __restrict__ aux, int64_t N, int64_t V, int k,
                     int32_t* __restrict__ idx_out, float* __restrict__ logp_out,
-                    float* __restrict__ rest_out, double* __restrict__ kl_out) {
+                    float* __restrict__ rest_out, double* __restrict__ kl_out,
+                    const float* __restrict__ scan_tf, const uint4* __restrict__ scan_regions,
+                    const int* __restrict__ scan_counts, unsigned long long* __restrict__ exact_rows) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   TopkShared& sh = *reinterpret_cast<TopkShared*>(smem_raw);
   constexpr int EB = DT == KLD_F32 ? 4 : 2;
@@ -510,13 +610,31 @@ __global__ void __launch_bounds__(kTopkThreads, kTopkCtasPerSm)
       continue;
     }
 
-    // ---- fast path: sampled threshold, one fused pass over both rows
+    // ---- fast path: a threshold, then every element at or above it is a
+    // candidate and every other one adds to the rest masses. Rows the row
+    // pass scanned read the lanes it copied (all their candidates) and the
+    // head and tail; the others sample their threshold here and read both
+    // rows once.
     {
-      const uint32_t t0 = V > kCap ? sample_threshold<DT>(sh, rb, V, kt) : 0u;
+      const bool scanned = scan_tf != nullptr;
+      const uint32_t t0 = scanned ? okey(scan_tf[r])
+                                  : (V > kCap ? sample_threshold<DT>(sh, rb, V, kt) : 0u);
       if (tid == 0) sh.ncand = 0;
       __syncthreads();
       double prest = 0.0, rrest = 0.0;
-      gather_pass<DT>(sh, rb, rq, V, t0, a, prest, rrest);
+      if (scanned) {
+        if (copied_pass<DT>(sh, rb, rq, V, t0, a, scan_regions + r * kConsumerWarps * kRegionVecs,
+                            scan_counts + r * kConsumerWarps, prest, rrest)) {
+          if (tid == 0) {  // the unflagged lanes' shares, added once
+            prest += a.rest_b;
+            rrest += a.rest_q;
+          }
+        } else {  // a region overflowed: both rows once, with the same threshold
+          gather_pass<DT>(sh, rb, rq, V, t0, a, prest, rrest);
+        }
+      } else {
+        gather_pass<DT>(sh, rb, rq, V, t0, a, prest, rrest);
+      }
       __syncthreads();
       const int n = sh.ncand;
       if (n >= kt && n <= kCap) {
@@ -541,6 +659,7 @@ __global__ void __launch_bounds__(kTopkThreads, kTopkCtasPerSm)
     }
 
     // ---- exact path. Threshold key: MSB radix select for the kt-th largest key
+    if (tid == 0 && exact_rows != nullptr) atomicAdd(exact_rows, 1ull);
     uint32_t prefix = 0u, mask = 0u;
     unsigned need = static_cast<unsigned>(kt);
     unsigned ncount = static_cast<unsigned>(V);  // elements matching the prefix
@@ -647,18 +766,50 @@ __global__ void __launch_bounds__(kTopkThreads, kTopkCtasPerSm)
   }
 }
 
+// Thresholds of the top-k scan: the fast path's sampled threshold of each
+// row, as the float whose order key it is.
+template <int DT>
+__global__ void __launch_bounds__(kTopkThreads, kTopkCtasPerSm)
+    kld_topk_threshold_kernel(const void* __restrict__ base, int64_t N, int64_t V, int kt,
+                              float* __restrict__ tf) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  TopkShared& sh = *reinterpret_cast<TopkShared*>(smem_raw);
+  constexpr int EB = DT == KLD_F32 ? 4 : 2;
+  for (int64_t r = blockIdx.x; r < N; r += gridDim.x) {
+    const uint32_t t0 = sample_threshold<DT>(sh, static_cast<const char*>(base) + r * V * EB, V, kt);
+    if (threadIdx.x == 0) tf[r] = key_float(t0);
+  }
+}
+
+int64_t topk_grid(int sm_count, int64_t N) {
+  const int64_t grid = static_cast<int64_t>(sm_count) * kTopkCtasPerSm;
+  return grid > N ? N : grid;
+}
+
 template <int DT>
 cudaError_t launch_typed(const void* base, const void* quant, const RowAux* aux, int64_t N,
                          int64_t V, int k, int32_t* idx, float* logp, float* rest, double* kl,
-                         int sm_count, cudaStream_t s) {
+                         int sm_count, cudaStream_t s, const TopkScan* scan,
+                         unsigned long long* exact_rows) {
   const size_t smem = sizeof(TopkShared);
   cudaError_t e = cudaFuncSetAttribute(kld_topk_kernel<DT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  int64_t grid = static_cast<int64_t>(sm_count) * kTopkCtasPerSm;
-  if (grid > N) grid = N;
-  kld_topk_kernel<DT><<<static_cast<unsigned>(grid), kTopkThreads, smem, s>>>(base, quant, aux, N, V, k,
-                                                                            idx, logp, rest, kl);
+  kld_topk_kernel<DT><<<static_cast<unsigned>(topk_grid(sm_count, N)), kTopkThreads, smem, s>>>(
+      base, quant, aux, N, V, k, idx, logp, rest, kl, scan ? scan->tf : nullptr,
+      scan ? scan->regions : nullptr, scan ? scan->counts : nullptr, exact_rows);
+  return cudaGetLastError();
+}
+
+template <int DT>
+cudaError_t launch_threshold_typed(const void* base, int64_t N, int64_t V, int kt, float* tf,
+                                   int sm_count, cudaStream_t s) {
+  const size_t smem = sizeof(TopkShared);
+  cudaError_t e = cudaFuncSetAttribute(kld_topk_threshold_kernel<DT>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  kld_topk_threshold_kernel<DT><<<static_cast<unsigned>(topk_grid(sm_count, N)), kTopkThreads, smem, s>>>(
+      base, N, V, kt, tf);
   return cudaGetLastError();
 }
 
@@ -666,12 +817,30 @@ cudaError_t launch_typed(const void* base, const void* quant, const RowAux* aux,
 
 cudaError_t launch_topk(const void* base, const void* quant, const RowAux* aux, int64_t N,
                         int64_t V, kld_dtype_t dtype, int k, int32_t* idx, float* logp,
-                        float* rest, double* kl, int sm_count, cudaStream_t stream) {
+                        float* rest, double* kl, int sm_count, cudaStream_t stream,
+                        const TopkScan* scan, unsigned long long* exact_rows) {
   if (k < 1 || k > kMaxTopk) return cudaErrorInvalidValue;
+  if (scan != nullptr && (V <= kCap || !scan->tf || !scan->regions || !scan->counts))
+    return cudaErrorInvalidValue;
   switch (dtype) {
-    case KLD_F32: return launch_typed<KLD_F32>(base, quant, aux, N, V, k, idx, logp, rest, kl, sm_count, stream);
-    case KLD_BF16: return launch_typed<KLD_BF16>(base, quant, aux, N, V, k, idx, logp, rest, kl, sm_count, stream);
-    case KLD_F16: return launch_typed<KLD_F16>(base, quant, aux, N, V, k, idx, logp, rest, kl, sm_count, stream);
+    case KLD_F32:
+      return launch_typed<KLD_F32>(base, quant, aux, N, V, k, idx, logp, rest, kl, sm_count, stream, scan, exact_rows);
+    case KLD_BF16:
+      return launch_typed<KLD_BF16>(base, quant, aux, N, V, k, idx, logp, rest, kl, sm_count, stream, scan, exact_rows);
+    case KLD_F16:
+      return launch_typed<KLD_F16>(base, quant, aux, N, V, k, idx, logp, rest, kl, sm_count, stream, scan, exact_rows);
+  }
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_topk_threshold(const void* base, int64_t N, int64_t V, kld_dtype_t dtype,
+                                  int k, float* tf, int sm_count, cudaStream_t stream) {
+  if (k < 1 || k > kMaxTopk || V <= kCap || N < 1 || !tf) return cudaErrorInvalidValue;
+  const int kt = static_cast<int>(V < k ? V : k);
+  switch (dtype) {
+    case KLD_F32: return launch_threshold_typed<KLD_F32>(base, N, V, kt, tf, sm_count, stream);
+    case KLD_BF16: return launch_threshold_typed<KLD_BF16>(base, N, V, kt, tf, sm_count, stream);
+    case KLD_F16: return launch_threshold_typed<KLD_F16>(base, N, V, kt, tf, sm_count, stream);
   }
   return cudaErrorInvalidValue;
 }

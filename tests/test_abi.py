@@ -75,7 +75,7 @@ int main(void) {
 
 
 def test_abi_version_and_status_strings(lib):
-    assert lib.kld_abi_version() == 3
+    assert lib.kld_abi_version() == 4
     for s in range(0, 10):
         assert lib.kld_status_string(s)
     assert lib.kld_status_string(12345) == b"unknown status"
@@ -130,7 +130,7 @@ int main(void) {
         subprocess.run(["gcc", "-I", os.path.join(ROOT, "include"), c, "-o", exe, build.LIB,
                         f"-Wl,-rpath,{libdir}"], check=True)
         out = subprocess.run([exe], capture_output=True, text=True, check=True).stdout.split()
-    assert [int(x) for x in out] == [_lib.KLD_ERR_INVALID_ARG] * 3 + [3]
+    assert [int(x) for x in out] == [_lib.KLD_ERR_INVALID_ARG] * 3 + [4]
 
 
 def test_create_without_gpu_reports_no_device(lib):

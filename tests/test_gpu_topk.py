@@ -132,3 +132,76 @@ def test_topk_pass_is_timed():
         assert 0.0 < row_ms < 100.0 and 0.0 < red_ms < 100.0 and 0.0 < topk_ms < 100.0
     finally:
         st.close()
+
+
+def _sampled(v):
+    # positions the threshold's samples read: 512 evenly spaced runs of 8
+    cover = np.zeros(v, bool)
+    for i in range(512):
+        s = (i * (v - 8) // 512) & ~7
+        cover[s:s + 8] = True
+    return cover
+
+
+@pytest.mark.parametrize("dt", [synth.F32, synth.BF16])
+def test_topk_scan_takes_the_fast_path(dt):
+    # rows longer than the candidate capacity: thresholds first, the row
+    # pass copies the lanes holding candidates, the top-k pass reads only
+    # those; no row of the benchmark's recipe needs the exact path
+    w = synth.make_recipe("ctx", n=48, v=151936, dtype=dt, seed=41)
+    st = KLDStats(max_rows=48, device=DEV)
+    try:
+        out = st.run_topk(w.base.to(DEV), w.quant.to(DEV), w.token_ids.to(DEV), k=128)
+        st.result()
+        assert st.topk_exact_rows() == 0
+        g = {key: t.cpu().numpy() for key, t in out.items()}
+    finally:
+        st.close()
+    o = oracle.topk(w.base, w.quant, 128, ODT[dt])
+    np.testing.assert_array_equal(g["idx"], o["idx"])
+    _close(g["rest"], o["rest"], 2e-6, 1e-6, "rest")
+    _close(g["kl_topk"], o["kl_topk"], 1e-6, 1e-4, "kl_topk")
+
+
+@pytest.mark.parametrize("dt", [synth.F32, synth.BF16])
+def test_topk_scan_overflow_direct_chunks_and_misaligned_rows(dt):
+    # row 0: 3000 high logits where the samples do not look, so far more
+    # than the copy regions hold pass the threshold (the row is read again
+    # with the same threshold); row 1: the quant row far from the base row
+    # everywhere (every chunk takes the direct path and is copied whole);
+    # row 2: three chunks with quant spikes (a few direct-path chunks);
+    # rows 3-5 ordinary; V odd, so rows start at every misalignment
+    n, v = 6, 151937
+    w = synth.make_recipe("ctx", n=n, v=v, dtype=synth.F32, seed=43)
+    b, q = w.base.clone(), w.quant.clone()
+    gen = torch.Generator().manual_seed(5)
+    free = np.flatnonzero(~_sampled(v))
+    pos = torch.from_numpy(free[torch.randperm(len(free), generator=gen)[:3000].numpy()])
+    b[0, pos] = float(b[0].max()) + 2.0
+    q[1] = b[1] + 5.0 * torch.randn(v, generator=gen)
+    for c in (3, 100, 250):
+        q[2, c * 512 + 17] = float(q[2].max()) + 30.0
+    if dt == synth.BF16:
+        b, q = b.to(torch.bfloat16), q.to(torch.bfloat16)
+    st = KLDStats(max_rows=n, device=DEV)
+    try:
+        out = st.run_topk(b.contiguous().to(DEV), q.contiguous().to(DEV), w.token_ids.to(DEV), k=128)
+        st.result()
+        assert st.topk_exact_rows() == 0
+        g = {key: t.cpu().numpy() for key, t in out.items()}
+    finally:
+        st.close()
+    o = oracle.topk(b.contiguous(), q.contiguous(), 128, ODT[dt])
+    np.testing.assert_array_equal(g["idx"], o["idx"])
+    _close(g["logp"], o["logp"], 2e-6, 1e-6, "logp")
+    _close(g["rest"], o["rest"], 2e-6, 1e-6, "rest")
+    _close(g["kl_topk"], o["kl_topk"], 1e-6, 1e-4, "kl_topk")
+
+
+def test_topk_exact_rows_before_any_topk():
+    st = KLDStats(max_rows=4, device=DEV)
+    try:
+        with pytest.raises(Exception):
+            st.topk_exact_rows()
+    finally:
+        st.close()
