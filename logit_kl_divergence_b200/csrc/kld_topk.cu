@@ -111,7 +111,8 @@ __device__ __forceinline__ unsigned warp_incl_scan(unsigned v, int lane) {
   }
   return v;
 }
-__device__ void find_bin(TopkShared& sh, int bins, unsigned need, bool descending) {
+template <class Sh>
+__device__ void find_bin(Sh& sh, int bins, unsigned need, bool descending) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (warp == 0) {
     auto bin_at = [&](int pos) { return descending ? bins - 1 - pos : pos; };  // pos: scan order
@@ -184,8 +185,8 @@ __device__ __forceinline__ float key_float(uint32_t k) {
 
 // Fast-path threshold: a key t0 with, by the samples, comfortably more than
 // kt but fewer than kCap elements of the row at or above it (block-wide).
-template <int DT>
-__device__ uint32_t sample_threshold(TopkShared& sh, const char* rb, int64_t V, int kt) {
+template <int DT, class Sh>
+__device__ uint32_t sample_threshold(Sh& sh, const char* rb, int64_t V, int kt) {
   const int tid = threadIdx.x;
   uint32_t* skey = reinterpret_cast<uint32_t*>(sh.cand);  // kSample keys
   double mm = 1.5 * static_cast<double>(kt) * kSample / static_cast<double>(V) + 8.0;
@@ -767,13 +768,21 @@ __global__ void __launch_bounds__(kTopkThreads, kTopkCtasPerSm)
 }
 
 // Thresholds of the top-k scan: the fast path's sampled threshold of each
-// row, as the float whose order key it is.
+// row, as the float whose order key it is. Only the histogram and the
+// sample keys in shared memory, so that more rows are in flight per SM
+// (each row is a chain of dependent steps).
+struct ThresholdShared {
+  unsigned hist[kHistBins];
+  unsigned long long cand[kSample / 2];  // the kSample sample keys
+  unsigned sel[3];
+};
+constexpr int kThresholdCtasPerSm = 4;
 template <int DT>
-__global__ void __launch_bounds__(kTopkThreads, kTopkCtasPerSm)
+__global__ void __launch_bounds__(kTopkThreads, kThresholdCtasPerSm)
     kld_topk_threshold_kernel(const void* __restrict__ base, int64_t N, int64_t V, int kt,
                               float* __restrict__ tf) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
-  TopkShared& sh = *reinterpret_cast<TopkShared*>(smem_raw);
+  ThresholdShared& sh = *reinterpret_cast<ThresholdShared*>(smem_raw);
   constexpr int EB = DT == KLD_F32 ? 4 : 2;
   for (int64_t r = blockIdx.x; r < N; r += gridDim.x) {
     const uint32_t t0 = sample_threshold<DT>(sh, static_cast<const char*>(base) + r * V * EB, V, kt);
@@ -804,11 +813,13 @@ cudaError_t launch_typed(const void* base, const void* quant, const RowAux* aux,
 template <int DT>
 cudaError_t launch_threshold_typed(const void* base, int64_t N, int64_t V, int kt, float* tf,
                                    int sm_count, cudaStream_t s) {
-  const size_t smem = sizeof(TopkShared);
+  const size_t smem = sizeof(ThresholdShared);
   cudaError_t e = cudaFuncSetAttribute(kld_topk_threshold_kernel<DT>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  kld_topk_threshold_kernel<DT><<<static_cast<unsigned>(topk_grid(sm_count, N)), kTopkThreads, smem, s>>>(
+  int64_t grid = static_cast<int64_t>(sm_count) * kThresholdCtasPerSm;
+  if (grid > N) grid = N;
+  kld_topk_threshold_kernel<DT><<<static_cast<unsigned>(grid), kTopkThreads, smem, s>>>(
       base, N, V, kt, tf);
   return cudaGetLastError();
 }
