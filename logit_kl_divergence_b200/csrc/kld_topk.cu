@@ -31,9 +31,9 @@
 // lowest indices in it by a radix select over the index), the candidates,
 // and a last pass for the rest masses (the row is read 2-4 times). T is the
 // first k candidates by (key desc, index asc): ranked by counting when there
-// are at most kRankMax of them (the fast path's usual few hundred; with more
-// than kRankDirect, a histogram of the candidates' keys first leaves only
-// those in or above the bin of the k-th largest to be ranked), else by a bitonic
+// are at most kRankMax of them (the fast path's usual few hundred; with many
+// more than k, a histogram of the candidates' keys first leaves only those
+// in or above the bin of the k-th largest to be ranked), else by a bitonic
 // sort in shared memory; candidates beyond T join the rest.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -52,7 +52,6 @@ constexpr int kHistBins = 2048;
 constexpr int kCap = kTopkCap;  // candidates sorted in shared memory
 constexpr int kSample = 4096;  // samples of a row for the threshold
 constexpr int kRankMax = 1536;  // at most this many candidates: rank by counting
-constexpr int kRankDirect = 768;  // up to this many: rank all against all (else a histogram first)
 constexpr int kSetBase = 2048;  // where the boundary set of the ranking is kept in cand[]
 static_assert(kSetBase >= kRankMax && kSetBase + kRankMax <= kCap, "boundary set layout");
 constexpr float kL = 1.4426950408889634f;  // log2(e) rounded to fp32, as the row pass
@@ -408,7 +407,7 @@ __device__ bool copied_pass(TopkShared& sh, const char* rb, const char* rq, int6
 // The first kt of the n (unique) candidates in descending order, by counting
 // for each candidate how many are larger: for the few hundred candidates of
 // the fast path this beats a bitonic network and its barriers. When there
-// are more than kRankDirect candidates, a histogram of their keys above t0 first
+// are many more candidates than kt, a histogram of their keys above t0 first
 // finds the bin that holds the kt-th largest: every candidate below that bin
 // is outside T, and only the ones in it or above (about kt) are ranked
 // against each other. T goes to sh.cand[kCap .. kCap + kt) (the sorted list
@@ -425,7 +424,7 @@ __device__ void rank_select(TopkShared& sh, int n, int kt, uint32_t t0, const ch
   };
   const unsigned long long* set = sh.cand;
   int ns = n;
-  if (n > kRankDirect) {
+  if (n > 2 * kt + 64) {
     // digit = (key - t0) >> s over 2048 bins, s from the largest key
     unsigned mx = 0u;
     for (int e = tid; e < n; e += kTopkThreads)
