@@ -5,7 +5,8 @@
 // reduction kernel writes directly, and the staging buffers of the
 // host-memory path; validates arguments before anything is enqueued and maps
 // CUDA failures to status codes. Every step of the statistic runs in the
-// kernels of kld_rows.cu and kld_reduce.cu.
+// kernels of kld_rows_kernel.cuh (launched from kld_rows.cu and kld_rows_scan.cu),
+// kld_reduce.cu, kld_grad.cu and kld_topk.cu.
 #include <cuda_runtime.h>
 
 #include <cstdint>

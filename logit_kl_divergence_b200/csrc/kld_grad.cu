@@ -6,7 +6,7 @@
 //   grad[i][j] = scale * (softmax(q_i)_j - softmax(b_i)_j),
 //
 // zero on rows that the statistics exclude (NaN / +inf, all -inf). The row
-// pass has already produced each row's normalisers (kld_rows.cu,
+// pass has already produced each row's normalisers (kld_rows_kernel.cuh,
 // row_aux): softmax(b)_j = 2^(b_j*L - Fb) * mb with an integer frame Fb
 // and mb in (0.5, 1], the same for q. This second pass streams b and q once
 // more and writes the gradient: a pure HBM-bound elementwise kernel (reads

@@ -12,7 +12,7 @@ evaluation on a dense grid (1.7e-6, 1.6e-6, 9.0e-7).
 
     python logit_kl_divergence_b200/csrc/phi_poly_fit.py
 
-Not run at build time; the printed coefficients are written into kld_rows.cu.
+Not run at build time; the printed coefficients are written into kld_rows_kernel.cuh.
 """
 import numpy as np
 from mpmath import mp

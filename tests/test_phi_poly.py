@@ -4,7 +4,7 @@ error bound as the kernel evaluates it.
 
 The kernel computes phi(lambda*x) = x^2 * Q(x) in fp32 Horner form with
 Q_k = P_k * lambda^(k+2) rounded to fp32 (lambda = fl32(log2 e) * ln 2), the
-P_k being the coefficients written into kld_rows.cu from the printout of
+P_k being the coefficients written into kld_rows_kernel.cuh from the printout of
 csrc/phi_poly_fit.py. A transcription slip in any coefficient (a high-order
 one only matters where |x| is large, which the benchmark data rarely reach)
 fails the first test against the re-run fit, or the second against the
@@ -18,7 +18,7 @@ import pytest
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 CSRC = os.path.join(ROOT, "logit_kl_divergence_b200", "csrc")
-SRC = open(os.path.join(CSRC, "kld_rows.cu")).read()
+SRC = open(os.path.join(CSRC, "kld_rows_kernel.cuh")).read()
 
 
 def _fit_module():
