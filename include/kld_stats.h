@@ -338,7 +338,9 @@ kld_status_t kld_stats_merge_partials(kld_stats_t h, const void* parts, int G, i
  * 4096 the top-k pass reads both rows once after the row pass instead.
  * Rows whose threshold holds fewer than k or too many elements (large tie
  * groups, masked rows) fall back to an exact radix selection that reads
- * the base row 2-4 times.
+ * the base row 2-4 times. The first call with V > 4096 allocates the scan's
+ * workspace (cudaMalloc, synchronising the device): make one such call
+ * before capturing this call into a CUDA graph.
  */
 #define KLD_MAX_TOPK 1024
 kld_status_t kld_stats_run_topk(kld_stats_t h, const void* base, const void* quant,

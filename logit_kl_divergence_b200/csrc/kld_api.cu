@@ -470,7 +470,7 @@ kld_status_t kld_stats_run_topk(kld_stats_t h, const void* base, const void* qua
       return cuda_fail(err, "cudaMalloc(top-k scan)");
     }
     char* m = static_cast<char*>(h->topk_mem);
-    h->topk_scan.tf = reinterpret_cast<const float*>(m);
+    h->topk_scan.tf = reinterpret_cast<float*>(m);
     h->topk_scan.regions = reinterpret_cast<uint4*>(m + tf_b);
     h->topk_scan.counts = reinterpret_cast<int*>(m + tf_b + rg_b);
   }
@@ -478,7 +478,7 @@ kld_status_t kld_stats_run_topk(kld_stats_t h, const void* base, const void* qua
   h->threshold_timed = h->timing && scan;
   if (scan) {
     if (h->timing) KLD_CUDA(cudaEventRecord(h->tev[4], s));
-    KLD_CUDA(kld::launch_topk_threshold(base, N, V, dtype, k, const_cast<float*>(h->topk_scan.tf),
+    KLD_CUDA(kld::launch_topk_threshold(base, N, V, dtype, k, h->topk_scan.tf,
                                         h->sm_count, s));
   }
   st = run_statistic(h, base, quant, token_ids, N, V, dtype, s, h->aux,

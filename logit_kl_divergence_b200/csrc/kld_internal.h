@@ -118,7 +118,7 @@ constexpr int kCopyVecs = 8;  // 16-byte vectors of a lane record: both rows' 16
 constexpr int kRegionVecs = kCopyCap * kCopyVecs + kCopyCap / 4;
 static_assert(kCopyCap % 4 == 0, "ids pack four to a vector");
 struct TopkScan {
-  const float* tf;  // [N]
+  float* tf;        // [N], written by launch_topk_threshold
   uint4* regions;   // [N][kConsumerWarps][kRegionVecs]: records (b vectors, then q vectors), ids
   int* counts;      // [N][kConsumerWarps]
 };
