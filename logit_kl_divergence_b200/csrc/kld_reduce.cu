@@ -23,8 +23,9 @@
 //      for a given N. The same pass appends the order-preserving 64-bit keys
 //      of the valid rows' KL to shared memory (N <= kKeyCap; larger inputs
 //      re-read the records for every level instead).
-//   2. the up to seven ranks the percentiles need are selected exactly by an
-//      MSB-first radix select with 11-bit digits: per level, one shared
+//   2. the up to seven ranks the percentiles need are selected exactly: for
+//      at most kCountMax keys by counting each key's rank (ties ordered by
+//      index); otherwise by an MSB-first radix select with 11-bit digits: per level, one shared
 //      histogram per distinct group of targets (keys that share the digits
 //      decided so far), a warp per group scans its 2048 bins and finds the
 //      digit and residual rank of each of its targets. A group of at most
@@ -46,6 +47,7 @@ using fin::order_key;
 using fin::warp_sort;
 using fin::kAhead;
 constexpr int kKeyCap = 19968;  // keys kept in shared memory (N up to this)
+constexpr int kCountMax = 512;  // up to this many keys: ranks by counting instead of radix levels
 
 struct ReduceShared {
   double dsum[32][5];
@@ -207,15 +209,37 @@ __global__ void __launch_bounds__(kReduceThreads, 1)
       __syncthreads();
     }
     if (tid < kTargets) sel.trank[tid] += static_cast<unsigned long long>(N - nv);
-    if (tid == 0) {
-      sel.ngroups = 1;
-      sel.gprefix[0] = 0ull;
-      sel.gcount[0] = static_cast<unsigned int>(N);
+    if (in_smem && N > 32 && N <= kCountMax) {
+      // A few hundred keys: each key's rank by counting the keys before it
+      // (equal keys ordered by index, so the ranks are 0..N-1, each once),
+      // and the keys at the target ranks read off directly. At this size
+      // that is cheaper than the radix levels, whose fixed costs (clearing
+      // and scanning 2048-bin histograms, a barrier per step) dominate.
+      __syncthreads();
+      for (int i = tid; i < N; i += nt) {
+        const unsigned long long k = keys[i];
+        unsigned rank = 0u;
+#pragma unroll 4
+        for (int j = 0; j < N; ++j) {
+          const unsigned long long y = keys[j];  // same address in every lane: broadcast
+          rank += (y < k || (y == k && j < i)) ? 1u : 0u;
+        }
+#pragma unroll
+        for (int t = 0; t < kTargets; ++t)
+          if (sel.trank[t] == rank) sel.tval[t] = k;
+      }
+      __syncthreads();
+    } else {
+      if (tid == 0) {
+        sel.ngroups = 1;
+        sel.gprefix[0] = 0ull;
+        sel.gcount[0] = static_cast<unsigned int>(N);
+      }
+      __syncthreads();
+      fin::select_levels(sel, in_smem ? fin::KeySource{keys, nullptr, false}
+                                      : fin::KeySource{nullptr, rows, false},
+                         N, 0, nt);
     }
-    __syncthreads();
-    fin::select_levels(sel, in_smem ? fin::KeySource{keys, nullptr, false}
-                                    : fin::KeySource{nullptr, rows, false},
-                       N, 0, nt);
   }
 
   if (tid == 0) {
