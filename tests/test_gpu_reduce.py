@@ -89,7 +89,23 @@ def test_heavy_duplicates(n):
     check(make_records(vals, rng))
 
 
-@pytest.mark.parametrize("n", [1, 4097, 50000])
+@pytest.mark.parametrize("n", [33, 64, 200, 511, 512, 513])
+def test_counted_ranks_around_their_size_limit(n):
+    # 33..512 keys take the counting path (equal keys ordered by index),
+    # 513 the radix levels: a tie group, signed zeros, infinities and
+    # excluded rows on both sides of the limit
+    rng = np.random.default_rng(n + 1)
+    v = rng.gamma(0.6, 0.08, n)
+    v[rng.integers(0, n, n // 4)] = 0.05
+    v[rng.integers(0, n, 3)] = -0.0
+    v[rng.integers(0, n, 3)] = 0.0
+    v[rng.integers(0, n, 2)] = np.inf
+    flags = np.zeros(n, np.uint32)
+    flags[rng.integers(0, n, n // 10)] |= oracle.ROW_EMPTY
+    check(make_records(v, rng, flags))
+
+
+@pytest.mark.parametrize("n", [1, 300, 4097, 50000])
 def test_all_equal(n):
     rng = np.random.default_rng(3)
     check(make_records(np.full(n, 0.0123), rng))
