@@ -521,33 +521,66 @@ __device__ __forceinline__ void poly_accumulate(const float* b, const f2* X, con
   }
 }
 
+// 16-bit quant rows stay packed in the hot loop (two elements per 32-bit
+// word: element 2w in the low half, 2w + 1 in the high half): their maximum
+// is taken on packed pairs and q - b by a mixed-precision subtract of the
+// 16-bit operand from the fp32 base, so the quant row is never widened
+// (measured for bf16: row pass 0.943 -> 0.906 ms at 8192 x 151936). Results
+// are bit-identical: q - b of two bf16 or two f16 values is exact in fp32,
+// and the maximum of 16-bit values is one of them.
+template <int DT>
+struct Packed;
+template <>
+struct Packed<KLD_BF16> {
+  static constexpr uint32_t kNegInfPair = 0xff80ff80u;
+  __device__ __forceinline__ static float lo(uint32_t w) { return __uint_as_float(w << 16); }
+  __device__ __forceinline__ static float hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+  __device__ __forceinline__ static uint32_t max2(uint32_t a, uint32_t c) {
+    uint32_t d;
+    asm("max.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(c));
+    return d;
+  }
+  __device__ __forceinline__ static void sub(uint32_t w, float b0, float b1, float& x0, float& x1) {
+    asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %2;\n\tsub.f32.bf16 %0, lo, %3;\n\t"
+        "sub.f32.bf16 %1, hi, %4;\n\t}"
+        : "=f"(x0), "=f"(x1) : "r"(w), "f"(b0), "f"(b1));
+  }
+};
+template <>
+struct Packed<KLD_F16> {
+  static constexpr uint32_t kNegInfPair = 0xfc00fc00u;
+  __device__ __forceinline__ static float lo(uint32_t w) {
+    return __half2float(__ushort_as_half(static_cast<unsigned short>(w & 0xffffu)));
+  }
+  __device__ __forceinline__ static float hi(uint32_t w) {
+    return __half2float(__ushort_as_half(static_cast<unsigned short>(w >> 16)));
+  }
+  __device__ __forceinline__ static uint32_t max2(uint32_t a, uint32_t c) {
+    uint32_t d;
+    asm("max.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(c));
+    return d;
+  }
+  __device__ __forceinline__ static void sub(uint32_t w, float b0, float b1, float& x0, float& x1) {
+    asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %2;\n\tsub.f32.f16 %0, lo, %3;\n\t"
+        "sub.f32.f16 %1, hi, %4;\n\t}"
+        : "=f"(x0), "=f"(x1) : "r"(w), "f"(b0), "f"(b1));
+  }
+};
+// Quant element i of a step: from the packed words (kPk = the row's 16-bit
+// type) or the widened array (kPk = 0).
+template <int kPk>
+__device__ __forceinline__ float q_el(const float* q, const uint32_t* qw, int i) {
+  if constexpr (kPk != 0)
+    return (i & 1) ? Packed<kPk>::hi(qw[i >> 1]) : Packed<kPk>::lo(qw[i >> 1]);
+  else
+    return q[i];
+}
+
 // Log-ratios x = q - b + K of one step, in packed pairs (x = 0 for absent
 // elements), and the largest |x| of the lane (NaN if any x is NaN). kForm
 // picks the order of the roundings (ratio_form): 0 (q - b) + K, 1
 // (q + K) - b, 2 q - (b - K).
-// bf16 quant rows stay packed in the hot loop (two elements per 32-bit word:
-// element 2w in the low half, 2w + 1 in the high half): their maximum is
-// taken on packed pairs and q - b by a mixed-precision subtract of the bf16
-// operand from the fp32 base, so the quant row is never widened (measured:
-// bf16 row pass 0.943 -> 0.906 ms at 8192 x 151936, results bit-identical,
-// since q - b of two bf16 values is exact in fp32 either way).
-__device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
-__device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
-__device__ __forceinline__ float bf_el(const uint32_t* qw, int i) {
-  return (i & 1) ? bf_hi(qw[i >> 1]) : bf_lo(qw[i >> 1]);
-}
-__device__ __forceinline__ uint32_t bf2_max(uint32_t a, uint32_t c) {
-  uint32_t d;
-  asm("max.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(c));
-  return d;
-}
-// q - b for the two bf16 of w against two fp32 b (exact: both are bf16 values).
-__device__ __forceinline__ void bf2_sub(uint32_t w, float b0, float b1, float& x0, float& x1) {
-  asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %2;\n\tsub.f32.bf16 %0, lo, %3;\n\tsub.f32.bf16 %1, hi, %4;\n\t}"
-      : "=f"(x0), "=f"(x1) : "r"(w), "f"(b0), "f"(b1));
-}
-
-template <int PE, int kForm, bool kPk = false>
+template <int PE, int kForm, int kPk = 0>
 __device__ __forceinline__ float log_ratios(const float* b, const float* q, unsigned valid,
                                             float K, f2* X, const uint32_t* qw = nullptr) {
   constexpr int NP = (PE + 1) / 2;
@@ -556,9 +589,9 @@ __device__ __forceinline__ float log_ratios(const float* b, const float* q, unsi
 #pragma unroll
   for (int j = 0; j < NP; ++j) {
     const int i0 = 2 * j, i1 = (2 * j + 1 < PE) ? 2 * j + 1 : 2 * j;
-    if constexpr (kPk) {
+    if constexpr (kPk != 0) {
       float d0, d1;
-      bf2_sub(qw[j], b[i0], b[i1], d0, d1);
+      Packed<kPk>::sub(qw[j], b[i0], b[i1], d0, d1);
       X[j] = add2(pk(d0, d1), K2);
     } else {
       const f2 Q = pk(q[i0], q[i1]), B = pk(b[i0], b[i1]);
@@ -591,18 +624,18 @@ __device__ __forceinline__ float log_ratios(const float* b, const float* q, unsi
 // logit >= the row's threshold, and for every lane of a direct-path step:
 // those lanes are copied (see process_chunk); the other lanes add their
 // weights to the rest sums in poly_accumulate.
-template <int PE, bool kWide, bool kScan = false, bool kPk = false>
+template <int PE, bool kWide, bool kScan = false, int kPk = 0>
 __device__ __forceinline__ bool chunk_step(const float* b, const float* q, unsigned valid,
                                            Ref& r, Acc& a, Best& best, int chunk_id,
                                            const uint32_t* qw = nullptr) {
   constexpr int NP = (PE + 1) / 2;
   const float mb = tree_max<PE, false>(b);
   float mq;
-  if constexpr (kPk) {
+  if constexpr (kPk != 0) {
     uint32_t m2 = qw[0];
 #pragma unroll
-    for (int w = 1; w < NP; ++w) m2 = bf2_max(m2, qw[w]);
-    mq = fmaxf(bf_lo(m2), bf_hi(m2));
+    for (int w = 1; w < NP; ++w) m2 = Packed<kPk>::max2(m2, qw[w]);
+    mq = fmaxf(Packed<kPk>::lo(m2), Packed<kPk>::hi(m2));
   } else {
     mq = tree_max<PE, false>(q);
   }
@@ -618,7 +651,7 @@ __device__ __forceinline__ bool chunk_step(const float* b, const float* q, unsig
 #pragma unroll
     for (int i = 0; i < PE; ++i) {
       if (!has && b[i] == wmb) {
-        dl = b[i] - (kPk ? bf_el(qw, i) : q[i]);
+        dl = b[i] - q_el<kPk>(q, qw, i);
         has = true;
       }
     }
@@ -720,7 +753,7 @@ __device__ __forceinline__ bool chunk_step(const float* b, const float* q, unsig
           const float e = ex2(fmaf(b[i], kLog2e, nRb));
           sb += e;
           sa = fmaf(e, fminf(xs[h], kBig), sa);
-          sh += ex2(fmaf(kPk ? bf_el(qw, i) : q[i], kLog2e, nRq));
+          sh += ex2(fmaf(q_el<kPk>(q, qw, i), kLog2e, nRq));
         }
       }
     }
@@ -747,7 +780,7 @@ __device__ __forceinline__ void process_chunk(const uint4* cb, const uint4* cq, 
                                               int chunk_id) {
   constexpr int E = Elem<DT>::kPerVec;
   constexpr int VPC = kLaneElems / E;
-  constexpr bool kPk = DT == KLD_BF16;
+  constexpr int kPk = DT == KLD_F32 ? 0 : DT;  // 16-bit quant rows stay packed
   float xb[kLaneElems], xq[kPk ? 1 : kLaneElems];
   uint32_t qw[kLaneElems / 2];
   unsigned valid = (1u << kLaneElems) - 1u;
@@ -757,7 +790,7 @@ __device__ __forceinline__ void process_chunk(const uint4* cb, const uint4* cq, 
     const uint4 vb = cb[vi];
     const uint4 vq = cq[vi];
     Elem<DT>::unpack(vb, &xb[k * E]);
-    if constexpr (kPk) {
+    if constexpr (kPk != 0) {
       qw[4 * k] = vq.x;
       qw[4 * k + 1] = vq.y;
       qw[4 * k + 2] = vq.z;
@@ -770,11 +803,11 @@ __device__ __forceinline__ void process_chunk(const uint4* cb, const uint4* cq, 
 #pragma unroll
       for (int i = 0; i < E; ++i) {
         xb[k * E + i] = -INFINITY;
-        if constexpr (!kPk) xq[k * E + i] = -INFINITY;
+        if constexpr (kPk == 0) xq[k * E + i] = -INFINITY;
       }
-      if constexpr (kPk) {
+      if constexpr (kPk != 0) {
 #pragma unroll
-        for (int u = 0; u < 4; ++u) qw[4 * k + u] = 0xff80ff80u;  // bf16 -inf pairs
+        for (int u = 0; u < 4; ++u) qw[4 * k + u] = Packed<kPk>::kNegInfPair;
       }
     }
   }
