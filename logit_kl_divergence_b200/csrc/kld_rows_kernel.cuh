@@ -408,17 +408,21 @@ struct Acc {
 };
 
 // Top-k scan state (TopkScan), in shared memory after the control block of
-// scan launches, so that it costs the consumers' hot loop no registers: per
-// consumer warp the region of its current row, the row's threshold and the
-// lanes copied so far; per lane its rest sums of base weights (rest[0]) and
-// quant weights (rest[1]) in the lane's frame and centre.
+// scan launches, so that it costs the consumers' hot loop few registers: per
+// consumer warp the region of its current row; per lane its rest sums of
+// base weights (rest[0]) and quant weights (rest[1]) in the lane's frame and
+// centre (kept in registers, they made the scan kernel spill in its hot loop).
 struct ScanArea {
   uint4* region[kConsumerWarps];
-  int ncopy[kConsumerWarps];
-  float tf[kConsumerWarps];
   double rest[2][kConsumerWarps][32];
 };
 constexpr int kScanSmemBytes = static_cast<int>((sizeof(ScanArea) + 127) / 128 * 128);
+// The warp-uniform part of the scan state that every chunk touches, kept in
+// registers: the row's threshold and the lanes copied so far.
+struct ScanRegs {
+  int ncopy;
+  float tf;
+};
 static_assert(kRowSmemBytes + kScanSmemBytes <= 227 * 1024, "row kernel shared memory");
 __device__ __forceinline__ ScanArea& scan_area() {
   extern __shared__ __align__(128) unsigned char smem[];
@@ -627,7 +631,7 @@ __device__ __forceinline__ float log_ratios(const float* b, const float* q, unsi
 template <int PE, bool kWide, bool kScan = false, int kPk = 0>
 __device__ __forceinline__ bool chunk_step(const float* b, const float* q, unsigned valid,
                                            Ref& r, Acc& a, Best& best, int chunk_id,
-                                           const uint32_t* qw = nullptr) {
+                                           const uint32_t* qw = nullptr, float scan_tf = 0.f) {
   constexpr int NP = (PE + 1) / 2;
   const float mb = tree_max<PE, false>(b);
   float mq;
@@ -720,7 +724,7 @@ __device__ __forceinline__ bool chunk_step(const float* b, const float* q, unsig
   if constexpr (kScan) {
     // the vote first, in every lane (a short-circuit would leave lanes out)
     const bool direct = !__all_sync(0xffffffffu, axl <= kTau);  // the direct path follows
-    flag = direct || mb >= scan_area().tf[threadIdx.x >> 5];
+    flag = direct || mb >= scan_tf;
   }
   if (__all_sync(0xffffffffu, axl <= kTauA)) {
     poly_accumulate<PE, 0, kScan>(b, X, r, a, !flag);
@@ -777,7 +781,7 @@ __device__ __forceinline__ bool chunk_step(const float* b, const float* q, unsig
 template <int DT, bool kMasked, bool kScan>
 __device__ __forceinline__ void process_chunk(const uint4* cb, const uint4* cq, int lane,
                                               int valid_vecs, Ref& r, Acc& a, Best& best,
-                                              int chunk_id) {
+                                              int chunk_id, ScanRegs* sr) {
   constexpr int E = Elem<DT>::kPerVec;
   constexpr int VPC = kLaneElems / E;
   constexpr int kPk = DT == KLD_F32 ? 0 : DT;  // 16-bit quant rows stay packed
@@ -811,8 +815,8 @@ __device__ __forceinline__ void process_chunk(const uint4* cb, const uint4* cq, 
       }
     }
   }
-  const bool cp = chunk_step<kLaneElems, DT == KLD_F32, kScan, kPk>(xb, xq, valid, r, a, best,
-                                                                   chunk_id, qw);
+  const bool cp = chunk_step<kLaneElems, DT == KLD_F32, kScan, kPk>(
+      xb, xq, valid, r, a, best, chunk_id, qw, kScan ? sr->tf : 0.f);
   if constexpr (kScan) {
     // copy the marked lanes' vectors from the stage into their records
     // (past the body's end of a last chunk they hold stale data; the top-k
@@ -821,7 +825,7 @@ __device__ __forceinline__ void process_chunk(const uint4* cb, const uint4* cq, 
     if (fm != 0u) {
       ScanArea& s = scan_area();
       const int w = threadIdx.x >> 5;
-      const int n0 = s.ncopy[w];
+      const int n0 = sr->ncopy;
       if (cp) {
         const int pos = n0 + __popc(fm & ((1u << lane) - 1u));
         if (pos < kCopyCap) {
@@ -835,9 +839,7 @@ __device__ __forceinline__ void process_chunk(const uint4* cb, const uint4* cq, 
               static_cast<uint32_t>(chunk_id) * 32u + static_cast<uint32_t>(lane);
         }
       }
-      __syncwarp();
-      if (lane == 0) s.ncopy[w] = n0 + __popc(fm);
-      __syncwarp();
+      sr->ncopy = n0 + __popc(fm);
     }
   }
 }
@@ -1406,13 +1408,11 @@ __global__ void __launch_bounds__(kRowThreads, 1) kld_rows_kernel(const __grid_c
       Ref ref{-INFINITY, -INFINITY, 0.f, 0.f, 0.f, -INFINITY, 0};
       Acc acc{0.0, 0.0, 0.0, 0.0, 0.0, 0.0};
       Best best{-INFINITY, -INFINITY, -1, -1};
+      ScanRegs sr{0, 0.f};
       if constexpr (kScan) {
         ScanArea& s = scan_area();
-        if (lane == 0) {
-          s.region[warp] = prm.scan.regions + (r * kConsumerWarps + warp) * kRegionVecs;
-          s.ncopy[warp] = 0;
-          s.tf[warp] = __ldg(prm.scan.tf + r);
-        }
+        sr.tf = __ldg(prm.scan.tf + r);
+        if (lane == 0) s.region[warp] = prm.scan.regions + (r * kConsumerWarps + warp) * kRegionVecs;
         s.rest[0][warp][lane] = 0.0;
         s.rest[1][warp][lane] = 0.0;
         __syncwarp();
@@ -1434,7 +1434,7 @@ __global__ void __launch_bounds__(kRowThreads, 1) kld_rows_kernel(const __grid_c
           for (int k = 0; k < kChunksPerWarp; ++k) {
             const int c = warp + k * kConsumerWarps;
             process_chunk<DT, false, kScan>(tb + c * (kChunkElems / E), tq + c * (kChunkElems / E),
-                                            lane, 0, ref, acc, best, t * kChunksPerTile + c);
+                                            lane, 0, ref, acc, best, t * kChunksPerTile + c, &sr);
           }
         } else {
           const int len = rem;
@@ -1445,7 +1445,7 @@ __global__ void __launch_bounds__(kRowThreads, 1) kld_rows_kernel(const __grid_c
             if (cstart >= len) break;
             process_chunk<DT, true, kScan>(tb + cstart / E, tq + cstart / E, lane,
                                            (len - cstart) / E, ref, acc, best,
-                                           t * kChunksPerTile + c);
+                                           t * kChunksPerTile + c, &sr);
           }
         }
         __syncwarp();
@@ -1473,7 +1473,7 @@ __global__ void __launch_bounds__(kRowThreads, 1) kld_rows_kernel(const __grid_c
         const ScanArea& s = scan_area();
         Sr = warp_sum(s.rest[0][warp][lane]);
         Qr = warp_sum(s.rest[1][warp][lane]);
-        if (lane == 0) prm.scan.counts[r * kConsumerWarps + warp] = s.ncopy[warp];
+        if (lane == 0) prm.scan.counts[r * kConsumerWarps + warp] = sr.ncopy;
       }
       const float wb = warp_max(best.b);  // the warp's exact maxima of b and q
       const float wq = warp_max(best.q);
