@@ -20,6 +20,7 @@ from __future__ import annotations
 
 import argparse
 import hashlib
+import re
 import json
 import math
 import os
@@ -57,11 +58,19 @@ def measured_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
+def _code_only(text: str) -> str:
+    """C/CUDA source without its comments and blank lines, so that an edit
+    of the comments alone does not change the hash of the code."""
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    lines = (re.sub(r"//.*$", "", ln).rstrip() for ln in text.splitlines())
+    return "\n".join(ln for ln in lines if ln)
+
+
 def kernel_source_hash() -> str:
     h = hashlib.sha256()
     for name in ("kld_rows_kernel.cuh", "kld_rows.cu", "kld_internal.h", "kld_finish.cuh"):  # the row kernel and its launch
-        with open(os.path.join(ROOT, "logit_kl_divergence_b200", "csrc", name), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(ROOT, "logit_kl_divergence_b200", "csrc", name), encoding="utf-8") as f:
+            h.update(_code_only(f.read()).encode())
     return h.hexdigest()[:16]
 
 

@@ -34,9 +34,9 @@
 // within 3e-8 relative of the exact one.
 //
 // Structure (whole rows: one CTA per SM, persistent over rows
-// r = blockIdx.x + k*grid; split rows, for few rows: CTA k of a row's P
-// parts takes a contiguous run of its 512-element chunks, and the parts
-// merge in shared memory of a cluster and / or through global memory):
+// r = blockIdx.x + k*grid; split rows, for the last partial wave or a few
+// rows: a CTA takes a contiguous run of a row's 512-element chunks, and the
+// parts merge through global memory or in shared memory of a cluster):
 //   - warp 16 (producer): one lane streams the 16-byte-aligned body of each
 //     row pair in 32 KB tiles per operand into a 3-stage shared-memory ring
 //     with cp.async.bulk (no multicast) completing on mbarriers, running
@@ -56,6 +56,10 @@
 //   All waits are mbarrier waits bounded by wall time; a wait that gives up
 //   sets an error bit that the reduction reports, and the CTA leaves only
 //   after its bulk copies have landed.
+// 16-bit quant rows stay packed in the consumers (see Packed). The top-k
+// scan form (kld_rows_kernel<DT, true>, see TopkScan; instantiated in
+// kld_rows_scan.cu) also copies out the lanes holding candidates and sums
+// the rest masses of the others.
 #pragma once
 
 #include <cuda_bf16.h>

@@ -44,10 +44,10 @@ def test_traffic_is_reported_only_for_the_kernel_source_it_was_taken_on(tmp_path
     root = tmp_path
     csrc = root / "logit_kl_divergence_b200" / "csrc"
     csrc.mkdir(parents=True)
-    (csrc / "kld_rows_kernel.cuh").write_text("// kernel v1\n")
-    (csrc / "kld_rows.cu").write_text("// launches\n")
-    (csrc / "kld_internal.h").write_text("// header\n")
-    (csrc / "kld_finish.cuh").write_text("// finishing steps\n")
+    (csrc / "kld_rows_kernel.cuh").write_text("int kernel = 1;  // kernel v1\n")
+    (csrc / "kld_rows.cu").write_text("int launches = 1;\n")
+    (csrc / "kld_internal.h").write_text("int header = 1;\n")
+    (csrc / "kld_finish.cuh").write_text("int finishing = 1;\n")
     (root / "profiles").mkdir()
     monkeypatch.setattr(bench, "ROOT", str(root))
     h = bench.kernel_source_hash()
@@ -55,10 +55,13 @@ def test_traffic_is_reported_only_for_the_kernel_source_it_was_taken_on(tmp_path
     (root / "profiles" / "traffic.json").write_text(json.dumps(rec))
     assert bench.recorded_traffic("w") == 123.0
     assert bench.recorded_traffic("other") is None
-    (csrc / "kld_rows_kernel.cuh").write_text("// kernel v2\n")   # the kernel changed since
+    # an edit of the comments alone keeps the record
+    (csrc / "kld_rows_kernel.cuh").write_text("/* kernel */\nint kernel = 1;  // kernel v1, reworded\n\n")
+    assert bench.kernel_source_hash() == h and bench.recorded_traffic("w") == 123.0
+    (csrc / "kld_rows_kernel.cuh").write_text("int kernel = 2;  // kernel v2\n")   # the code changed since
     assert bench.kernel_source_hash() != h
     assert bench.recorded_traffic("w") is None
     h2 = bench.kernel_source_hash()
-    (csrc / "kld_rows.cu").write_text("// launches v2\n")   # and so did its launch
+    (csrc / "kld_rows.cu").write_text("int launches = 2;\n")   # and so did its launch
     assert bench.kernel_source_hash() != h2
 
